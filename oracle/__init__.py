@@ -1,0 +1,303 @@
+"""fp64 CPU oracle for the mLSTM / retention recurrence -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline legs of
+``bench.py`` may import this package.  The CUDA library and its Python binding
+never import it, and it imports nothing from them: the two sides share only
+the seeded input generators, which hold none of the method's arithmetic.
+
+Contents
+--------
+``sequential``       C, fp64, one token at a time (``mlstm_oracle.c``).  The
+                     primary oracle; also the timed CPU baseline.
+``parallel_form``    numpy, fp64, the quadratic "parallel" evaluation with the
+                     decay matrix D (Edifice.Attention.RetNet, "Key Innovation",
+                     generalised to the mLSTM's stabilised gates).  Tiny inputs.
+``chunkwise``        numpy, fp64, the chunked evaluation (intra-chunk quadratic
+                     part plus an inter-chunk carried state), used to check the
+                     chunk algebra independently of any GPU code.
+``unstabilised``     numpy, fp64, the recurrence with raw exponential gates and
+                     the floor 1 of the mLSTM read-out, no stabiliser at all.
+``state_bytes``      size of a model's recurrent state (xLSTM 7B "Modelled costs").
+
+Pins (tests/test_oracle_*.py) tie every function to something other than
+itself: closed forms, brute-force double loops, special cases and invariants.
+The per-block normaliser (num_blocks > 1) and the optional output gate o_t are
+fixed by this project's reading of the pages, not by them: parity unpinned
+for those two readings (their self-consistency is still tested).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mlstm_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile mlstm_oracle.c with gcc into oracle/liboracle.so (in-tree)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-std=c11", "-pthread",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        _lib.oracle_mlstm_sequential.argtypes = [I] * 7 + [P] * 13 + [I]
+        _lib.oracle_mlstm_sequential.restype = I
+    return _lib
+
+
+def _f64(x):
+    return None if x is None else np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(x):
+    return None if x is None else x.ctypes.data_as(ctypes.c_void_p)
+
+
+def sequential(q, k, v, igate=None, fgate=None, ogate=None, C0=None, n0=None, m0=None,
+               num_blocks: int = 1, retention: bool = False, threads: int | None = None):
+    """Sequential fp64 recurrence (mlstm_oracle.c).
+
+    q, k: [B,NH,S,DHQK]; v: [B,NH,S,DHV]; igate, fgate: [B,NH,S] pre-activations;
+    ogate: [B,NH,S,DHV] already-activated output gate or None (= 1);
+    C0: [B,NH,nb,DHV/nb,DHQK/nb]; n0: [B,NH,nb,DHQK/nb]; m0: [B,NH]; None = zeros.
+    Returns (h, C, n, m); n and m are None in retention mode.
+    """
+    lib = _load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, NH, S, DHQK = q.shape
+    DHV = v.shape[-1]
+    nb = int(num_blocks)
+    if DHQK % nb or DHV % nb:
+        raise ValueError("num_blocks must divide DHQK and DHV")
+    dk, dv = DHQK // nb, DHV // nb
+    ig, fg = _f64(igate), _f64(fgate)
+    og = _f64(ogate)
+    C0, n0, m0 = _f64(C0), _f64(n0), _f64(m0)
+    h = np.zeros((B, NH, S, DHV))
+    C = np.zeros((B, NH, nb, dv, dk))
+    n = None if retention else np.zeros((B, NH, nb, dk))
+    m = None if retention else np.zeros((B, NH))
+    if threads is None:
+        threads = len(os.sched_getaffinity(0))
+    rc = lib.oracle_mlstm_sequential(B, NH, S, DHQK, DHV, nb, int(bool(retention)),
+                                     _ptr(q), _ptr(k), _ptr(v), _ptr(ig), _ptr(fg), _ptr(og),
+                                     _ptr(C0), _ptr(n0), _ptr(m0),
+                                     _ptr(h), _ptr(C), _ptr(n), _ptr(m), int(threads))
+    if rc != 0:
+        raise ValueError("oracle_mlstm_sequential rejected the shapes")
+    return h, C, n, m
+
+
+def log_sigmoid(x):
+    """log(1 / (1 + exp(-x))) in the overflow-free form min(x, 0) - log1p(exp(-|x|))."""
+    x = np.asarray(x, dtype=np.float64)
+    return np.minimum(x, 0.0) - np.log1p(np.exp(-np.abs(x)))
+
+
+def retention_gamma(NH: int):
+    """Per-head decay gamma_h = 1 - 2^(-5-h), h = 0 .. NH-1 (RetNet "Multi-Scale Retention")."""
+    return 1.0 - np.exp2(-5.0 - np.arange(NH, dtype=np.float64))
+
+
+def _split_blocks(x, nb):
+    """[..., D] -> [..., nb, D/nb] (block j takes the j-th contiguous slice)."""
+    return x.reshape(x.shape[:-1] + (nb, x.shape[-1] // nb))
+
+
+def parallel_form(q, k, v, igate=None, fgate=None, ogate=None, C0=None, n0=None, m0=None,
+                  num_blocks: int = 1, retention: bool = False):
+    """Quadratic (all pairs) evaluation, fp64.  For tiny S only.
+
+    Retention (RetNet "Key Innovation"): Y = (Q K^T * D) V with
+    D[t, s] = gamma^(t-s) for s <= t, plus the initial state decayed by gamma^(t+1).
+    mLSTM: log D[t, s] = b_t - b_s + itilde_s (s <= t) with b the inclusive cumulative
+    sum of log f; the initial state enters with weight b_t + m0; the stabiliser is the
+    row maximum of those log weights, which is the recurrence's m_t.
+    Returns (h, C, n, m) like ``sequential``.
+    """
+    q, k, v = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
+    B, NH, S, DHQK = q.shape
+    DHV = v.shape[-1]
+    nb = num_blocks
+    dk, dv = DHQK // nb, DHV // nb
+    qb = _split_blocks(q, nb).transpose(0, 1, 3, 2, 4)  # [B,NH,nb,S,dk]
+    kb = _split_blocks(k, nb).transpose(0, 1, 3, 2, 4)
+    vb = _split_blocks(v, nb).transpose(0, 1, 3, 2, 4)  # [B,NH,nb,S,dv]
+    C0 = np.zeros((B, NH, nb, dv, dk)) if C0 is None else np.asarray(C0, dtype=np.float64)
+    n0 = np.zeros((B, NH, nb, dk)) if n0 is None else np.asarray(n0, dtype=np.float64)
+    m0 = np.zeros((B, NH)) if m0 is None else np.asarray(m0, dtype=np.float64)
+    tril = np.tril(np.ones((S, S), dtype=bool))
+    t_idx = np.arange(S)
+    h = np.zeros((B, NH, nb, S, dv))
+    C = np.zeros((B, NH, nb, dv, dk))
+    n = np.zeros((B, NH, nb, dk))
+    m = np.zeros((B, NH))
+    gam = retention_gamma(NH)
+    for b in range(B):
+        for hd in range(NH):
+            if retention:
+                g = gam[hd]
+                expo = (t_idx[:, None] - t_idx[None, :]).astype(np.float64)
+                D = np.where(tril, g ** np.where(tril, expo, 0.0), 0.0)
+                w_init = g ** (t_idx + 1.0)
+                for j in range(nb):
+                    Q, K, V = qb[b, hd, j], kb[b, hd, j], vb[b, hd, j]
+                    h[b, hd, j] = (Q @ K.T * D) @ V + w_init[:, None] * (Q @ C0[b, hd, j].T)
+                    wS = g ** (S - 1 - t_idx)
+                    C[b, hd, j] = (V * wS[:, None]).T @ K + g ** S * C0[b, hd, j]
+                continue
+            lf = log_sigmoid(fgate[b, hd])
+            li = np.asarray(igate[b, hd], dtype=np.float64)
+            bcum = np.cumsum(lf)
+            logD = np.where(tril, bcum[:, None] - bcum[None, :] + li[None, :], -np.inf)
+            log_init = bcum + m0[b, hd]
+            mt = np.maximum(log_init, logD.max(axis=1))
+            D = np.exp(logD - mt[:, None])
+            w_init = np.exp(log_init - mt)
+            # final state at t = S-1
+            mS = mt[-1] if S > 0 else m0[b, hd]
+            wS = np.exp(bcum[-1] - bcum + li - mS) if S > 0 else np.zeros(0)
+            aS = np.exp(bcum[-1] + m0[b, hd] - mS) if S > 0 else 1.0
+            for j in range(nb):
+                Q, K, V = qb[b, hd, j], kb[b, hd, j], vb[b, hd, j]
+                P = (Q @ K.T) * D
+                num = P @ V + w_init[:, None] * (Q @ C0[b, hd, j].T)
+                den = P.sum(axis=1) + w_init * (Q @ n0[b, hd, j])
+                hh = num / np.maximum(np.abs(den), np.exp(-mt))[:, None]
+                if ogate is not None:
+                    hh = hh * _split_blocks(np.asarray(ogate[b, hd], dtype=np.float64), nb)[:, j, :]
+                h[b, hd, j] = hh
+                C[b, hd, j] = (V * wS[:, None]).T @ K + aS * C0[b, hd, j]
+                n[b, hd, j] = (K * wS[:, None]).sum(axis=0) + aS * n0[b, hd, j]
+            m[b, hd] = mS
+    h = h.transpose(0, 1, 3, 2, 4).reshape(B, NH, S, DHV)
+    if retention:
+        return h, C, None, None
+    return h, C, n, m
+
+
+def chunkwise(q, k, v, igate=None, fgate=None, ogate=None, C0=None, n0=None, m0=None,
+              num_blocks: int = 1, retention: bool = False, chunk: int = 16):
+    """Chunked evaluation, fp64: quadratic inside each chunk, a carried state between.
+
+    Per chunk with local cumulative log-forget b (inclusive) and total g:
+      m_t   = max(b_t + m_c, max_{s<=t} (b_t - b_s + itilde_s))   (max-plus form of the
+              stabiliser recurrence)
+      h_t   = [sum_s e^{b_t-b_s+i_s-m_t} (q_t.k_s) v_s + e^{b_t+m_c-m_t} C_c q_t] / den_t
+      C_c+1 = e^{g+m_c-m_c+1} C_c + sum_s e^{g-b_s+i_s-m_c+1} v_s k_s^T
+    Retention uses gamma powers and no normaliser.  S need not divide by chunk.
+    Returns (h, C, n, m) like ``sequential``.
+    """
+    q, k, v = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
+    B, NH, S, DHQK = q.shape
+    DHV = v.shape[-1]
+    nb = num_blocks
+    dk, dv = DHQK // nb, DHV // nb
+    qb = _split_blocks(q, nb)
+    kb = _split_blocks(k, nb)
+    vb = _split_blocks(v, nb)
+    ob = None if ogate is None else _split_blocks(np.asarray(ogate, dtype=np.float64), nb)
+    C = np.zeros((B, NH, nb, dv, dk)) if C0 is None else np.array(C0, dtype=np.float64)
+    n = np.zeros((B, NH, nb, dk)) if n0 is None else np.array(n0, dtype=np.float64)
+    m = np.zeros((B, NH)) if m0 is None else np.array(m0, dtype=np.float64)
+    h = np.zeros((B, NH, S, nb, dv))
+    gam = retention_gamma(NH)
+    for b in range(B):
+        for hd in range(NH):
+            for c0 in range(0, S, chunk):
+                L = min(chunk, S - c0)
+                sl = slice(c0, c0 + L)
+                tril = np.tril(np.ones((L, L), dtype=bool))
+                if retention:
+                    lf = np.full(L, np.log(gam[hd]))
+                    li = np.zeros(L)
+                else:
+                    lf = log_sigmoid(fgate[b, hd, sl])
+                    li = np.asarray(igate[b, hd, sl], dtype=np.float64)
+                bl = np.cumsum(lf)
+                g = bl[-1]
+                logD = np.where(tril, bl[:, None] - bl[None, :] + li[None, :], -np.inf)
+                mc = 0.0 if retention else m[b, hd]
+                if retention:
+                    mt = np.zeros(L)
+                else:
+                    mt = np.maximum(bl + mc, logD.max(axis=1))
+                D = np.exp(logD - mt[:, None])
+                s_inter = np.exp(bl + mc - mt)
+                m_next = 0.0 if retention else mt[-1]
+                a = np.exp(g + mc - m_next)
+                w = np.exp(g - bl + li - m_next)
+                for j in range(nb):
+                    Q, K, V = qb[b, hd, sl, j], kb[b, hd, sl, j], vb[b, hd, sl, j]
+                    P = (Q @ K.T) * D
+                    num = P @ V + s_inter[:, None] * (Q @ C[b, hd, j].T)
+                    if retention:
+                        hh = num
+                    else:
+                        den = P.sum(axis=1) + s_inter * (Q @ n[b, hd, j])
+                        hh = num / np.maximum(np.abs(den), np.exp(-mt))[:, None]
+                        if ob is not None:
+                            hh = hh * ob[b, hd, sl, j]
+                        n[b, hd, j] = a * n[b, hd, j] + (K * w[:, None]).sum(axis=0)
+                    h[b, hd, sl, j] = hh
+                    C[b, hd, j] = a * C[b, hd, j] + (V * w[:, None]).T @ K
+                if not retention:
+                    m[b, hd] = m_next
+    h = h.reshape(B, NH, S, DHV)
+    if retention:
+        return h, C, None, None
+    return h, C, n, m
+
+
+def unstabilised(q, k, v, igate, fgate, ogate=None, C0=None, n0=None, num_blocks: int = 1):
+    """The mLSTM recurrence with raw gates i = exp(itilde), f = sigmoid(ftilde), fp64.
+
+    C_t = f C + i v k^T, n_t = f n + i k, h_t = o * C_t q_t / max(|n_t . q_t|, 1); no
+    stabiliser.  Valid only while exp(itilde) and the products stay in range.
+    Returns (h, C_true, n_true) with the state in raw (unstabilised) units.
+    """
+    q, k, v = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
+    B, NH, S, DHQK = q.shape
+    DHV = v.shape[-1]
+    nb = num_blocks
+    dk, dv = DHQK // nb, DHV // nb
+    qb, kb, vb = _split_blocks(q, nb), _split_blocks(k, nb), _split_blocks(v, nb)
+    C = np.zeros((B, NH, nb, dv, dk)) if C0 is None else np.array(C0, dtype=np.float64)
+    n = np.zeros((B, NH, nb, dk)) if n0 is None else np.array(n0, dtype=np.float64)
+    h = np.zeros((B, NH, S, nb, dv))
+    f = 1.0 / (1.0 + np.exp(-np.asarray(fgate, dtype=np.float64)))
+    i = np.exp(np.asarray(igate, dtype=np.float64))
+    for t in range(S):
+        ft = f[:, :, t, None, None, None]
+        it = i[:, :, t, None, None, None]
+        C = ft * C + it * vb[:, :, t, :, :, None] * kb[:, :, t, :, None, :]
+        n = f[:, :, t, None, None] * n + i[:, :, t, None, None] * kb[:, :, t]
+        num = np.einsum("bhjvk,bhjk->bhjv", C, qb[:, :, t])
+        den = np.maximum(np.abs(np.einsum("bhjk,bhjk->bhj", n, qb[:, :, t])), 1.0)
+        ht = num / den[..., None]
+        if ogate is not None:
+            ht = ht * _split_blocks(np.asarray(ogate[:, :, t], dtype=np.float64), nb)
+        h[:, :, t] = ht
+    return h.reshape(B, NH, S, DHV), C, n
+
+
+def state_bytes(layers: int, heads: int, dqk: int, dv: int, bytes_per_value: int) -> int:
+    """Bytes of recurrent state per sequence: per head a dv x dqk matrix, a dqk
+    normaliser and one stabiliser scalar (xLSTM 7B "Modelled costs": the state
+    does not grow with context)."""
+    return layers * heads * (dqk * dv + dqk + 1) * bytes_per_value
