@@ -1,0 +1,469 @@
+"""Benchmark of the mLSTM hot path on B200: chunkwise prefill + decode step.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One JSON line on rank 0.  Headline (value): chunkwise-prefill tokens/s of the
+large-head workload (B1 NH8 S8192 DHQK256 DHV512 chunk64, bf16 in / fp32 state),
+with its dominant kernel's TFLOP/s against the measured bf16 tensor peak.  The
+decode workload (B128 NH8 256x512, fp32 state updated in place) is measured in
+the same run and reported under "decode" with its state GB/s against the
+measured HBM bandwidth.  The path does not shard: with N GPUs every rank runs
+its own replica (weak scaling) and value sums the tokens of all ranks over the
+slowest rank's time.  --impl reference times the fp64 CPU oracle on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "mLSTM chunkwise-fwd tokens/s (% bf16 TC peak); decode-step state GB/s (% HBM)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ work accounting
+def chunkwise_flops(B, NH, S, dk, dv, L, nb=1, retention=False):
+    """Algorithmic flops of a chunkwise prefill: causal intra-chunk pairs (L+1)(dk+dv) per
+    token, inter-chunk read-out 2 dk dv and update 2 dk dv per token, normaliser 4 dk
+    (not in retention); per (head, block), dk and dv of one block."""
+    per_tok = (L + 1) * (dk + dv) + 4 * dk * dv + (0 if retention else 4 * dk)
+    return B * NH * nb * S * per_tok
+
+
+def chunkwise_min_bytes(B, NH, S, DHQK, DHV, esize, nb=1, retention=False):
+    """Each input read once, h written once, final state written once."""
+    tok = B * NH * S
+    b = tok * (2 * DHQK + 2 * DHV) * esize  # q, k, v in; h out
+    if not retention:
+        b += tok * 2 * 4  # gates
+    b += B * NH * (DHV * DHQK // nb + (0 if retention else DHQK + 1)) * 4
+    return b
+
+
+def decode_step_bytes(B, NH, DHQK, DHV, esize, nb=1):
+    """Bytes one decode step must move: C and n read + written (fp32), m read + written,
+    q, k, v read, h written, two gates read."""
+    state = B * NH * (DHV * DHQK // nb + DHQK) * 4 * 2 + B * NH * 4 * 2
+    io = B * NH * (2 * DHQK + 2 * DHV) * esize + B * NH * 2 * 4
+    return state + io
+
+
+def decode_step_flops(B, NH, DHQK, DHV, nb=1):
+    """Update (f'C + i' v k^T: 3 flops/element) plus read-out (2 per element) plus n."""
+    return B * NH * (5 * DHV * DHQK // nb + 6 * DHQK)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ distributed helpers
+def dist_setup(gpus: int):
+    """Returns (rank, world, local_rank); initialises NCCL when launched under torchrun."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def dist_max(x: float, world: int) -> float:
+    """Maximum of a float over ranks (the slowest rank's time)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the GPU is busy."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+        self.thread = None
+        self.active = False
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append((self.active, parts))
+
+    def mark(self, active: bool):
+        self.active = active
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self):
+        rows = [p for a, p in self.rows if a] or [p for _, p in self.rows]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_chunkwise_sample(w, tokens: int):
+    """The fp64 oracle over the first `tokens` positions of every (batch, head) of the
+    workload; returns (seconds, tokens_processed, threads)."""
+    import oracle
+    from linear_recurrent_token_b200 import inputs
+    inp = inputs.forward_inputs(w, S=tokens)
+    threads = len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    oracle.sequential(inp["q"], inp["k"], inp["v"], inp["igate"], inp["fgate"], num_blocks=w.num_blocks,
+                      retention=w.retention, threads=threads)
+    return time.perf_counter() - t0, w.B * tokens, min(threads, w.B * w.NH * w.num_blocks)
+
+
+def cpu_baseline(w, budget_s: float = 12.0, steps: int = 1):
+    """Oracle tokens/s on a bounded sample: the sampled prefix is sized so that `steps`
+    repetitions take about budget_s seconds in total (capped at the whole sequence)."""
+    tokens = min(w.S, 128)
+    secs, _, _ = oracle_chunkwise_sample(w, tokens)
+    per_step = budget_s / max(1, steps)
+    if secs < per_step and tokens < w.S:
+        tokens = int(min(w.S, max(tokens, tokens * per_step / max(secs, 1e-3))))
+    total_s, total_tok, threads, times = 0.0, 0, 1, []
+    for _ in range(max(1, steps)):
+        secs, done, threads = oracle_chunkwise_sample(w, tokens)
+        total_s += secs
+        total_tok += done
+        times.append(secs)
+    sample = (f"first {tokens} of {w.S} positions of all {w.B * w.NH} (batch, head) sequences of "
+              f"{w.describe()}, fp64 sequential recurrence, {len(times)} repetition(s)")
+    return {"value": total_tok / total_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": sample, "ms_per_step": 1e3 * total_s / len(times)}
+
+
+# ------------------------------------------------------------------ GPU legs
+def run_chunkwise(w, steps, warmup, flush_bytes, clocks):
+    import torch
+
+    from linear_recurrent_token_b200 import inputs, mlstm
+    td = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    inp = inputs.forward_inputs(w)
+    dev = lambda x, dt: torch.from_numpy(np.ascontiguousarray(x)).to("cuda", dt)
+    q, k, v = dev(inp["q"], td), dev(inp["k"], td), dev(inp["v"], td)
+    ig, fg = dev(inp["igate"], torch.float32), dev(inp["fgate"], torch.float32)
+    h = torch.empty((w.B, w.NH, w.S, w.DHV), dtype=td, device="cuda")
+    C = torch.empty((w.B, w.NH, w.num_blocks, w.dv, w.dk), dtype=torch.float32, device="cuda")
+    n = torch.empty((w.B, w.NH, w.num_blocks, w.dk), dtype=torch.float32, device="cuda")
+    m = torch.empty((w.B, w.NH), dtype=torch.float32, device="cuda")
+    p = mlstm.fwd_params(w.B, w.NH, w.S, w.DHQK, w.DHV, w.chunk, w.num_blocks, td, w.retention)
+    plan = mlstm.plan(p)
+    ws = torch.empty(max(1, plan["workspace_bytes"]), dtype=torch.uint8, device="cuda")
+    flush = torch.empty(flush_bytes // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    gi = (None, None) if w.retention else (ig, fg)
+
+    def one(ev=None):
+        mlstm.fwd_chunkwise(q, k, v, *gi, chunk=w.chunk, num_blocks=w.num_blocks, retention=w.retention,
+                            h=h, C_out=C, n_out=None if w.retention else n, m_out=None if w.retention else m,
+                            workspace=ws, stream=stream, events=ev)
+
+    for _ in range(warmup):
+        flush.fill_(1.0)
+        one()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    clocks.mark(True)
+    t_wall = time.perf_counter()
+    for e in ev:
+        flush.fill_(float(len(ev)))
+        e[0].record(stream)
+        one((e[2], e[3]))
+        e[1].record(stream)
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall
+    clocks.mark(False)
+    step_ms = [a.elapsed_time(b) for a, b, _, _ in ev]
+    main_ms = [c.elapsed_time(d) for _, _, c, d in ev]
+    return dict(step_ms=step_ms, main_ms=main_ms, wall_s=t_wall, plan=plan,
+                tensors=(q, k, v, ig, fg, h, C, n, m, ws))
+
+
+def run_chunkwise_e2e(w, steps, tensors):
+    """Same prefill through the public API with HOST buffers: pinned host inputs copied in,
+    the call, h and the final state copied back, all inside the timed region."""
+    import torch
+
+    from linear_recurrent_token_b200 import mlstm
+    q, k, v, ig, fg, h, C, n, m, ws = tensors
+    pin = lambda t: t.cpu().pin_memory()
+    hq, hk, hv, hig, hfg = pin(q), pin(k), pin(v), pin(ig), pin(fg)
+    oh, oC, on_, om = (torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (h, C, n, m))
+    stream = torch.cuda.current_stream()
+    gi = (None, None) if w.retention else (ig, fg)
+
+    def one():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        if not w.retention:
+            ig.copy_(hig, non_blocking=True)
+            fg.copy_(hfg, non_blocking=True)
+        mlstm.fwd_chunkwise(q, k, v, *gi, chunk=w.chunk, num_blocks=w.num_blocks, retention=w.retention,
+                            h=h, C_out=C, n_out=None if w.retention else n, m_out=None if w.retention else m,
+                            workspace=ws, stream=stream)
+        oh.copy_(h, non_blocking=True)
+        oC.copy_(C, non_blocking=True)
+        if not w.retention:
+            on_.copy_(n, non_blocking=True)
+            om.copy_(m, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    h2d = sum(t.numel() * t.element_size() for t in ((hq, hk, hv) + (() if w.retention else (hig, hfg))))
+    d2h = sum(t.numel() * t.element_size() for t in ((oh, oC) + (() if w.retention else (on_, om))))
+    return ms, h2d, d2h
+
+
+def run_decode(w, steps, warmup, clocks):
+    import torch
+
+    from linear_recurrent_token_b200 import inputs, mlstm
+    td = torch.bfloat16
+    T = min(w.steps, steps + warmup)
+    C0, n0, m0 = inputs.decode_initial_state(w)
+    C = torch.from_numpy(C0).cuda()
+    n = torch.from_numpy(n0).cuda()
+    m = torch.from_numpy(m0).cuda()
+    per = [inputs.decode_step_inputs(w, t) for t in range(T)]
+    stack = lambda key, dt: torch.from_numpy(np.stack([p[key] for p in per])).to("cuda", dt)
+    q, k, v = stack("q", td), stack("k", td), stack("v", td)
+    ig, fg = stack("igate", torch.float32), stack("fgate", torch.float32)
+    h = torch.empty((T, w.B, w.NH, w.DHV), dtype=td, device="cuda")
+    stream = torch.cuda.current_stream()
+    for t in range(warmup):
+        mlstm.step(q[t % T], k[t % T], v[t % T], ig[t % T], fg[t % T], C, n, m, h=h[t % T], stream=stream)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    clocks.mark(True)
+    for i, (a, b) in enumerate(ev):
+        t = (warmup + i) % T
+        a.record(stream)
+        mlstm.step(q[t], k[t], v[t], ig[t], fg[t], C, n, m, h=h[t], stream=stream)
+        b.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark(False)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+
+    # end to end: per step, pinned host q/k/v/gates in, the step, h out
+    hq, hk, hv = (x[:1].cpu().pin_memory() for x in (q, k, v))
+    hig, hfg = (x[:1].cpu().pin_memory() for x in (ig, fg))
+    oh = torch.empty(h[0].shape, dtype=td).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        q[0].copy_(hq[0], non_blocking=True)
+        k[0].copy_(hk[0], non_blocking=True)
+        v[0].copy_(hv[0], non_blocking=True)
+        ig[0].copy_(hig[0], non_blocking=True)
+        fg[0].copy_(hfg[0], non_blocking=True)
+        mlstm.step(q[0], k[0], v[0], ig[0], fg[0], C, n, m, h=h[0], stream=stream)
+        oh.copy_(h[0], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / steps
+    h2d = sum(x[0].numel() * x.element_size() for x in (hq, hk, hv, hig, hfg))
+    d2h = oh.numel() * oh.element_size()
+    return dict(step_ms=step_ms, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h)
+
+
+# ------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=3, help="chunkwise workload index (default 3)")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    from linear_recurrent_token_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]
+    wd = inputs.WORKLOADS[4]
+    if args.impl == "reference":
+        rank, world, local = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), 0
+    else:
+        rank, world, local = dist_setup(args.gpus)
+    config = {"workload": w.describe(), "decode_workload": wd.describe(), "global_batch": w.B * world,
+              "seq_len": w.S, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+              "l2": "flushed between chunkwise steps (256 MiB write); decode state (512 MiB) exceeds L2"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        cb = cpu_baseline(w, budget_s=min(120.0, 6.0 * args.steps), steps=args.steps)
+        line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": cb["ms_per_step"],
+                "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+                "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import torch
+    assert torch.cuda.is_available(), "bench.py --impl ours needs a CUDA device"
+    torch.cuda.set_device(local)
+    from linear_recurrent_token_b200 import mlstm
+    mlstm.lib()
+    peaks, peak_src = load_peaks()
+    clocks = ClockSampler(local)
+    clocks.start()
+    try:
+        dist_barrier(world)
+        torch.cuda.synchronize()
+        cw = run_chunkwise(w, args.steps, args.warmup, 256 << 20, clocks)
+        dist_barrier(world)
+        torch.cuda.synchronize()
+        step_ms = statistics.mean(cw["step_ms"])
+        main_ms = statistics.mean(cw["main_ms"])
+        slow_ms = dist_max(step_ms, world)
+        tokens = w.B * w.S * world
+        value = tokens / (slow_ms * 1e-3)
+        flops = chunkwise_flops(w.B, w.NH, w.S, w.dk, w.dv, w.chunk, w.num_blocks, w.retention)
+        mbytes = chunkwise_min_bytes(w.B, w.NH, w.S, w.DHQK, w.DHV, 2 if w.dtype == "bf16" else 4,
+                                     w.num_blocks, w.retention)
+        achieved_tf = flops / (main_ms * 1e-3) / 1e12
+        e2e_ms, h2d, d2h = run_chunkwise_e2e(w, max(3, args.steps // 4), cw["tensors"])
+        e2e_ms = dist_max(e2e_ms, world)
+        del cw["tensors"]
+        torch.cuda.empty_cache()
+        dec = None
+        if not args.no_decode:
+            dist_barrier(world)
+            dec = run_decode(wd, args.steps * 5, args.warmup, clocks)
+            dist_barrier(world)
+    finally:
+        clocks.stop()
+    launches = cw["plan"]["kernels"] * args.steps
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": slow_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": config,
+        "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved_tf / peaks["bf16_tflops"], "traffic": None,
+                     "kernel": "chunkwise walk" + (" (tcgen05)" if cw["plan"]["tensor_core"] else " (SIMT)"),
+                     "kernel_ms": main_ms, "flops_per_launch": flops, "peak_source": f"{peak_src} bf16 burst",
+                     "hbm_frac": mbytes / (main_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "min_bytes_per_launch": mbytes},
+        "e2e": {"value": w.B * w.S * world / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "plan": cw["plan"],
+        "clocks": clocks.summary(),
+    }
+    if dec is not None:
+        dms = statistics.mean(dec["step_ms"])
+        dms_max = dist_max(dms, world)
+        dbytes = decode_step_bytes(wd.B, wd.NH, wd.DHQK, wd.DHV, 2, wd.num_blocks)
+        gbs = dbytes * world / (dms_max * 1e-3) / 1e9
+        per_rank_gbs = dbytes / (dms * 1e-3) / 1e9
+        line["decode"] = {
+            "value": gbs, "unit": "GB/s", "ms_per_step": dms_max, "steps": len(dec["step_ms"]),
+            "tokens_per_s": wd.B * world / (dms_max * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": per_rank_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": per_rank_gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "step_kernel<256>",
+                         "bytes_per_launch": dbytes, "peak_source": f"{peak_src} copy bandwidth"},
+            "e2e": {"value": wd.B * world / (dec["e2e_ms"] * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": dec["h2d"], "d2h_bytes_per_step": dec["d2h"]},
+        }
+        line["gpu_launches"] += len(dec["step_ms"])
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(w)
+        line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,188 @@
+/*
+ * mlstm.h -- C ABI of the B200 mLSTM / retention recurrence library (libmlstm.so).
+ *
+ * The recurrence (DeepChrInteract-v2 "mLSTM Model", "Core idea"; gates stabilised
+ * in log space as stated there):
+ *
+ *     m_t = max(log f_t + m_{t-1}, log i_t)        log f_t = logsigmoid(ftilde_t),
+ *                                                  log i_t = itilde_t
+ *     C_t = f'_t C_{t-1} + i'_t v_t k_t^T          f'_t = exp(log f_t + m_{t-1} - m_t)
+ *     n_t = f'_t n_{t-1} + i'_t k_t                i'_t = exp(itilde_t - m_t)
+ *     h_t = o_t * (C_t q_t) / max(|n_t . q_t|, exp(-m_t))
+ *
+ * C and n are kept in stabilised units (the raw state times exp(-m_t)); the floor
+ * exp(-m_t) is the floor 1 of the raw form, so h does not depend on the stabiliser.
+ *
+ * Retention flag (Edifice.Attention.RetNet, "Key Innovation", recurrent form, and
+ * "Multi-Scale Retention"): i = 1, f = gamma_h = 1 - 2^(-5-h) for head h (0-based),
+ * no normaliser, no stabiliser, no output gate:  C_t = gamma_h C_{t-1} + v_t k_t^T,
+ * h_t = C_t q_t.
+ *
+ * Block-diagonal memory (Edifice.Recurrent.XLSTMv2, "Key Improvements" #1):
+ * num_blocks = nb splits each head's q, k (DHQK) and v, o, h (DHV) into nb
+ * contiguous slices; block j owns C_j [DHV/nb x DHQK/nb] and n_j [DHQK/nb] and
+ * shares the head's gates and m.
+ *
+ * Two evaluation orders of the same recurrence (RetNet "Triple Paradigm"):
+ *   mlstm_fwd_chunkwise  chunkwise-parallel prefill over a whole sequence,
+ *   mlstm_step           one recurrent decode step, state updated in place.
+ *
+ * Conventions for every entry point
+ *   - Every data pointer is DEVICE memory owned by the caller.  The library never
+ *     allocates, frees or keeps a pointer past the call.  Scratch memory of the
+ *     prefill is a caller-supplied workspace sized by
+ *     mlstm_fwd_chunkwise_workspace_size().
+ *   - All tensors are dense, row-major (last index fastest), 16-byte aligned.
+ *   - q, k, v, o, h use the dtype of the params (fp32 or bf16); gates are always
+ *     fp32; the state (C, n, m) is always fp32.
+ *   - Work is enqueued on `stream`; the call returns without synchronising.
+ *   - Arguments are validated on the host before anything is enqueued; on any
+ *     error nothing is enqueued and no output is touched.  Errors raised by the
+ *     CUDA runtime at launch are returned as MLSTM_ERR_CUDA.
+ *   - Calls that share no output buffer may run concurrently on different
+ *     streams.  The library holds no global mutable state.
+ */
+#ifndef MLSTM_H_
+#define MLSTM_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same underlying types as cudaStream_t / cudaEvent_t of the CUDA runtime. */
+typedef struct CUstream_st* mlstm_stream_t;
+typedef struct CUevent_st* mlstm_event_t;
+
+typedef enum {
+  MLSTM_OK = 0,
+  MLSTM_ERR_NULL = 1,       /* a required pointer is NULL                          */
+  MLSTM_ERR_SHAPE = 2,      /* a size is negative, inconsistent or unsupported     */
+  MLSTM_ERR_DTYPE = 3,      /* dtype is not MLSTM_F32 or MLSTM_BF16                */
+  MLSTM_ERR_ALIGN = 4,      /* a pointer is not 16-byte aligned                    */
+  MLSTM_ERR_WORKSPACE = 5,  /* workspace NULL or smaller than the size query       */
+  MLSTM_ERR_CUDA = 6,       /* the CUDA runtime reported an error at launch        */
+  MLSTM_ERR_ALIAS = 7       /* an output overlaps an input it must not overlap     */
+} mlstm_status_t;
+
+typedef enum { MLSTM_F32 = 0, MLSTM_BF16 = 1 } mlstm_dtype_t;
+
+/* Sizes of one chunkwise prefill.  B, NH >= 0; S >= 0; DHQK, DHV >= 1 and
+ * divisible by num_blocks (>= 1); chunk >= 1 (the intra-chunk tile length; the
+ * result does not depend on it beyond rounding; S need not be a multiple of it).
+ * retention: 0 = mLSTM, 1 = retention. */
+typedef struct {
+  int B, NH, S, DHQK, DHV;
+  int chunk;
+  int num_blocks;
+  mlstm_dtype_t dtype;
+  int retention;
+} mlstm_fwd_params_t;
+
+/* Sizes of one decode step (one token per sequence). */
+typedef struct {
+  int B, NH, DHQK, DHV;
+  int num_blocks;
+  mlstm_dtype_t dtype;
+  int retention;
+} mlstm_step_params_t;
+
+/* How a prefill will be executed (for tests, benchmarks and logs). */
+typedef struct {
+  int tensor_core;      /* 1: tcgen05/TMEM kernels; 0: SIMT fp32 kernels            */
+  int segments;         /* sequence segments run in parallel per head (>= 1)        */
+  int dv_tile;          /* value rows of the state owned by one CTA                 */
+  int ctas_main;        /* CTAs of the dominant (intra-chunk + state walk) kernel   */
+  int kernels;          /* kernel launches one call enqueues                         */
+  size_t workspace_bytes;
+} mlstm_fwd_plan_t;
+
+/* Workspace bytes mlstm_fwd_chunkwise needs for these sizes (0 if none); returns
+ * 0 as well for invalid sizes, which mlstm_fwd_chunkwise then rejects. */
+size_t mlstm_fwd_chunkwise_workspace_size(const mlstm_fwd_params_t* p);
+
+/* Fills *plan for these sizes.  MLSTM_ERR_NULL / MLSTM_ERR_SHAPE / MLSTM_ERR_DTYPE
+ * as for mlstm_fwd_chunkwise. */
+mlstm_status_t mlstm_fwd_chunkwise_plan(const mlstm_fwd_params_t* p, mlstm_fwd_plan_t* plan);
+
+/*
+ * Chunkwise-parallel prefill of a whole sequence (RetNet "Triple Paradigm",
+ * chunkwise mode: O(S) work, state carried between chunks).
+ *
+ *   q, k    [B,NH,S,DHQK]  dtype          required (if S > 0)
+ *   v       [B,NH,S,DHV]   dtype          required (if S > 0)
+ *   igate   [B,NH,S]       fp32           input-gate pre-activation itilde; required
+ *                                          unless retention (then ignored, may be NULL)
+ *   fgate   [B,NH,S]       fp32           forget-gate pre-activation ftilde; same rule
+ *   ogate   [B,NH,S,DHV]   dtype          already-activated output gate o_t; NULL = 1;
+ *                                          ignored in retention mode
+ *   C0      [B,NH,nb,DHV/nb,DHQK/nb] fp32 initial state (value row, key column),
+ *   n0      [B,NH,nb,DHQK/nb]        fp32 stabilised units; NULL = zeros.  n0 and m0
+ *   m0      [B,NH]                   fp32 are ignored in retention mode.
+ *   h       [B,NH,S,DHV]   dtype          output; required (if S > 0)
+ *   C_out, n_out, m_out               fp32 final state in the sequential recurrence's
+ *                                          representation (same m_S); NULL = not written.
+ *                                          May alias C0 / n0 / m0 exactly (in place);
+ *                                          any other overlap with an input is an error.
+ *   workspace, workspace_bytes        device scratch of at least
+ *                                          mlstm_fwd_chunkwise_workspace_size(p) bytes,
+ *                                          16-byte aligned; contents need not be
+ *                                          initialised and are garbage afterwards.
+ *                                          Two calls in flight must not share it.
+ *   stream                            CUDA stream (NULL = legacy default stream)
+ */
+mlstm_status_t mlstm_fwd_chunkwise(const mlstm_fwd_params_t* p,
+                                   const void* q, const void* k, const void* v,
+                                   const float* igate, const float* fgate, const void* ogate,
+                                   const float* C0, const float* n0, const float* m0,
+                                   void* h, float* C_out, float* n_out, float* m_out,
+                                   void* workspace, size_t workspace_bytes,
+                                   mlstm_stream_t stream);
+
+/* mlstm_fwd_chunkwise, plus: if main_begin / main_end are non-NULL, they are recorded
+ * on `stream` immediately before and after the dominant kernel (intra-chunk
+ * contraction + state walk), so its duration can be timed with cudaEventElapsedTime. */
+mlstm_status_t mlstm_fwd_chunkwise_timed(const mlstm_fwd_params_t* p,
+                                         const void* q, const void* k, const void* v,
+                                         const float* igate, const float* fgate, const void* ogate,
+                                         const float* C0, const float* n0, const float* m0,
+                                         void* h, float* C_out, float* n_out, float* m_out,
+                                         void* workspace, size_t workspace_bytes,
+                                         mlstm_stream_t stream,
+                                         mlstm_event_t main_begin, mlstm_event_t main_end);
+
+/*
+ * One recurrent decode step for every sequence of the batch, state updated in
+ * place (RetNet recurrent_retention_step: O(1) per token; burn-gdn2 Gdn2Mode
+ * FusedRecurrent: state [B,H,K,V] carried across tokens and updated in place).
+ *
+ *   q, k    [B,NH,DHQK]  dtype      required
+ *   v       [B,NH,DHV]   dtype      required
+ *   igate, fgate [B,NH]  fp32       pre-activations; required unless retention
+ *   ogate   [B,NH,DHV]   dtype      activated output gate; NULL = 1; ignored in retention
+ *   C       [B,NH,nb,DHV/nb,DHQK/nb] fp32  in/out, required
+ *   n       [B,NH,nb,DHQK/nb]        fp32  in/out, required unless retention
+ *   m       [B,NH]                   fp32  in/out, required unless retention
+ *   h       [B,NH,DHV]   dtype      output, required; must not overlap the state
+ *   stream
+ * Supported block key widths DHQK/nb: 4, 8, 16, 32, 64, 128, 256, 512 (else
+ * MLSTM_ERR_SHAPE).
+ */
+mlstm_status_t mlstm_step(const mlstm_step_params_t* p,
+                          const void* q, const void* k, const void* v,
+                          const float* igate, const float* fgate, const void* ogate,
+                          float* C, float* n, float* m, void* h,
+                          mlstm_stream_t stream);
+
+/* Static, never-NULL description of a status code. */
+const char* mlstm_status_string(mlstm_status_t s);
+
+/* ABI version: (major << 16) | minor. */
+int mlstm_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLSTM_H_ */

@@ -1,0 +1,306 @@
+// C ABI of libmlstm (declared in include/mlstm.h): host-side validation, workspace
+// layout and kernel dispatch.  No entry point allocates, frees or synchronises.
+#include <stdint.h>
+#include <string.h>
+
+#include "kernels.h"
+#include "mlstm.h"
+
+namespace {
+
+using namespace mlstm;
+
+struct FwdShape {
+  int B, NH, S, DHQK, DHV, chunk, nb, dk, dv, retention, dtype;
+  size_t esize;
+  long long BH;
+};
+
+mlstm_status_t check_fwd(const mlstm_fwd_params_t* p, FwdShape* s) {
+  if (!p) return MLSTM_ERR_NULL;
+  if (p->dtype != MLSTM_F32 && p->dtype != MLSTM_BF16) return MLSTM_ERR_DTYPE;
+  if (p->B < 0 || p->NH < 0 || p->S < 0 || p->DHQK < 1 || p->DHV < 1 || p->chunk < 1 || p->num_blocks < 1)
+    return MLSTM_ERR_SHAPE;
+  if (p->DHQK % p->num_blocks || p->DHV % p->num_blocks) return MLSTM_ERR_SHAPE;
+  s->B = p->B;
+  s->NH = p->NH;
+  s->S = p->S;
+  s->DHQK = p->DHQK;
+  s->DHV = p->DHV;
+  s->chunk = p->chunk;
+  s->nb = p->num_blocks;
+  s->dk = p->DHQK / p->num_blocks;
+  s->dv = p->DHV / p->num_blocks;
+  s->retention = p->retention ? 1 : 0;
+  s->dtype = p->dtype == MLSTM_BF16 ? 1 : 0;
+  s->esize = p->dtype == MLSTM_BF16 ? 2 : 4;
+  s->BH = (long long)p->B * p->NH;
+  // grid limits of the kernels
+  if (s->BH * s->nb > 65535LL || s->BH > (1LL << 31) / 1024) return MLSTM_ERR_SHAPE;
+  if ((long long)s->S * s->BH > (1LL << 40)) return MLSTM_ERR_SHAPE;
+  if (s->S > 0 && s->BH > 0 && simt_walk_pick_tile(s->chunk, s->dk, s->dv) == 0) return MLSTM_ERR_SHAPE;
+  return MLSTM_OK;
+}
+
+size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct WsLayout {
+  size_t m_tok, m_init, n_init, total;
+};
+
+WsLayout fwd_layout(const FwdShape& s) {
+  WsLayout w = {0, 0, 0, 0};
+  if (s.retention || s.BH == 0) return w;
+  size_t off = 0;
+  w.m_tok = off;
+  off = align_up(off + sizeof(float) * (size_t)s.BH * s.S);
+  w.m_init = off;
+  off = align_up(off + sizeof(float) * (size_t)s.BH);
+  w.n_init = off;
+  off = align_up(off + sizeof(float) * (size_t)s.BH * s.nb * s.dk);
+  w.total = off;
+  return w;
+}
+
+bool misaligned(const void* p) { return ((uintptr_t)p & 15) != 0; }
+
+struct Range {
+  const void* p;
+  size_t n;
+};
+bool overlaps(Range a, Range b) {
+  if (!a.p || !b.p || a.n == 0 || b.n == 0) return false;
+  const uintptr_t a0 = (uintptr_t)a.p, b0 = (uintptr_t)b.p;
+  return a0 < b0 + b.n && b0 < a0 + a.n;
+}
+
+mlstm_status_t fwd_impl(const mlstm_fwd_params_t* p, const void* q, const void* k, const void* v,
+                        const float* igate, const float* fgate, const void* ogate, const float* C0,
+                        const float* n0, const float* m0, void* h, float* C_out, float* n_out, float* m_out,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream, cudaEvent_t ev0,
+                        cudaEvent_t ev1) {
+  FwdShape s;
+  mlstm_status_t st = check_fwd(p, &s);
+  if (st != MLSTM_OK) return st;
+  const bool ret = s.retention != 0;
+  if (ret) {
+    igate = fgate = nullptr;
+    ogate = nullptr;
+    n0 = m0 = nullptr;
+    n_out = m_out = nullptr;
+  }
+  const size_t tok = (size_t)s.BH * s.S;
+  const size_t bq = tok * s.DHQK * s.esize, bv = tok * s.DHV * s.esize, bg = tok * sizeof(float);
+  const size_t bC = (size_t)s.BH * s.nb * s.dv * s.dk * sizeof(float);
+  const size_t bn = (size_t)s.BH * s.nb * s.dk * sizeof(float), bm = (size_t)s.BH * sizeof(float);
+  if (tok > 0) {
+    if (!q || !k || !v || !h) return MLSTM_ERR_NULL;
+    if (!ret && (!igate || !fgate)) return MLSTM_ERR_NULL;
+  }
+  const void* all[] = {q, k, v, igate, fgate, ogate, C0, n0, m0, h, C_out, n_out, m_out, workspace};
+  for (const void* ptr : all)
+    if (ptr && misaligned(ptr)) return MLSTM_ERR_ALIGN;
+  const WsLayout ws = fwd_layout(s);
+  if (ws.total > 0 && (!workspace || workspace_bytes < ws.total)) return MLSTM_ERR_WORKSPACE;
+
+  // aliasing: outputs may not overlap inputs, except the exact in-place state aliases
+  const Range in_q{q, bq}, in_k{k, bq}, in_v{v, bv}, in_ig{igate, bg}, in_fg{fgate, bg}, in_o{ogate, bv};
+  const Range in_C{C0, bC}, in_n{n0, bn}, in_m{m0, bm};
+  const Range out_h{h, bv}, out_C{C_out, bC}, out_n{n_out, bn}, out_m{m_out, bm};
+  const Range wsr{workspace, ws.total};
+  const Range inputs[] = {in_q, in_k, in_v, in_ig, in_fg, in_o};
+  const Range outs[] = {out_h, out_C, out_n, out_m, wsr};
+  for (const Range& o : outs) {
+    for (const Range& i : inputs)
+      if (overlaps(o, i)) return MLSTM_ERR_ALIAS;
+  }
+  for (int a = 0; a < 5; ++a)
+    for (int b = a + 1; b < 5; ++b)
+      if (overlaps(outs[a], outs[b])) return MLSTM_ERR_ALIAS;
+  const Range states_in[] = {in_C, in_n, in_m};
+  const Range states_out[] = {out_C, out_n, out_m};
+  for (const Range& si : states_in) {
+    if (overlaps(out_h, si) || overlaps(wsr, si)) return MLSTM_ERR_ALIAS;
+    for (int j = 0; j < 3; ++j) {
+      const Range& so = states_out[j];
+      const bool exact = so.p == si.p && so.n == si.n && (&si - states_in) == j;
+      if (overlaps(so, si) && !exact) return MLSTM_ERR_ALIAS;
+    }
+  }
+  if (s.BH == 0) return MLSTM_OK;
+
+  cudaError_t e = cudaSuccess;
+  if (s.S == 0) {  // nothing to read: the final state is the initial state
+    if (C_out && C_out != C0)
+      e = C0 ? cudaMemcpyAsync(C_out, C0, bC, cudaMemcpyDeviceToDevice, stream) : cudaMemsetAsync(C_out, 0, bC, stream);
+    if (e == cudaSuccess && n_out && n_out != n0)
+      e = n0 ? cudaMemcpyAsync(n_out, n0, bn, cudaMemcpyDeviceToDevice, stream) : cudaMemsetAsync(n_out, 0, bn, stream);
+    if (e == cudaSuccess && m_out && m_out != m0)
+      e = m0 ? cudaMemcpyAsync(m_out, m0, bm, cudaMemcpyDeviceToDevice, stream) : cudaMemsetAsync(m_out, 0, bm, stream);
+    return e == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA;
+  }
+
+  char* wsb = static_cast<char*>(workspace);
+  WalkArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = s.B;
+  a.NH = s.NH;
+  a.S = s.S;
+  a.DHQK = s.DHQK;
+  a.DHV = s.DHV;
+  a.chunk = s.chunk;
+  a.nb = s.nb;
+  a.retention = s.retention;
+  a.dk = s.dk;
+  a.dv = s.dv;
+  a.dtype = s.dtype;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.og = ogate;
+  a.ig = igate;
+  a.fg = fgate;
+  a.C0 = C0;
+  a.h = h;
+  a.C_out = C_out;
+  a.n_out = n_out;
+  a.m_out = m_out;
+  if (!ret) {
+    a.m_tok = reinterpret_cast<const float*>(wsb + ws.m_tok);
+    a.m_init = reinterpret_cast<const float*>(wsb + ws.m_init);
+    a.n_init = reinterpret_cast<const float*>(wsb + ws.n_init);
+    e = launch_gate_prep((int)s.BH, s.S, s.nb * s.dk, igate, fgate, m0, n0, reinterpret_cast<float*>(wsb + ws.m_tok),
+                         reinterpret_cast<float*>(wsb + ws.m_init), reinterpret_cast<float*>(wsb + ws.n_init),
+                         stream);
+    if (e != cudaSuccess) return MLSTM_ERR_CUDA;
+  }
+  a.dv_tile = simt_walk_pick_tile(s.chunk, s.dk, s.dv);
+  if (ev0 && cudaEventRecord(ev0, stream) != cudaSuccess) return MLSTM_ERR_CUDA;
+  e = launch_simt_walk(a, stream);
+  if (e != cudaSuccess) return MLSTM_ERR_CUDA;
+  if (ev1 && cudaEventRecord(ev1, stream) != cudaSuccess) return MLSTM_ERR_CUDA;
+  return MLSTM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mlstm_abi_version(void) { return (1 << 16) | 0; }
+
+const char* mlstm_status_string(mlstm_status_t s) {
+  switch (s) {
+    case MLSTM_OK: return "ok";
+    case MLSTM_ERR_NULL: return "a required pointer is NULL";
+    case MLSTM_ERR_SHAPE: return "a size is negative, inconsistent or unsupported";
+    case MLSTM_ERR_DTYPE: return "unsupported dtype";
+    case MLSTM_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case MLSTM_ERR_WORKSPACE: return "workspace missing or too small";
+    case MLSTM_ERR_CUDA: return "CUDA runtime error at launch";
+    case MLSTM_ERR_ALIAS: return "an output overlaps an input";
+  }
+  return "unknown status";
+}
+
+size_t mlstm_fwd_chunkwise_workspace_size(const mlstm_fwd_params_t* p) {
+  FwdShape s;
+  if (check_fwd(p, &s) != MLSTM_OK) return 0;
+  return fwd_layout(s).total;
+}
+
+mlstm_status_t mlstm_fwd_chunkwise_plan(const mlstm_fwd_params_t* p, mlstm_fwd_plan_t* plan) {
+  if (!plan) return MLSTM_ERR_NULL;
+  FwdShape s;
+  mlstm_status_t st = check_fwd(p, &s);
+  if (st != MLSTM_OK) return st;
+  memset(plan, 0, sizeof(*plan));
+  plan->tensor_core = 0;
+  plan->segments = 1;
+  plan->dv_tile = simt_walk_pick_tile(s.chunk, s.dk, s.dv);
+  plan->ctas_main = plan->dv_tile > 0 ? (int)(((s.dv + plan->dv_tile - 1) / plan->dv_tile) * s.BH * s.nb) : 0;
+  plan->kernels = (s.BH == 0 || s.S == 0) ? 0 : (s.retention ? 1 : 2);
+  plan->workspace_bytes = fwd_layout(s).total;
+  return MLSTM_OK;
+}
+
+mlstm_status_t mlstm_fwd_chunkwise(const mlstm_fwd_params_t* p, const void* q, const void* k, const void* v,
+                                   const float* igate, const float* fgate, const void* ogate, const float* C0,
+                                   const float* n0, const float* m0, void* h, float* C_out, float* n_out,
+                                   float* m_out, void* workspace, size_t workspace_bytes, mlstm_stream_t stream) {
+  return fwd_impl(p, q, k, v, igate, fgate, ogate, C0, n0, m0, h, C_out, n_out, m_out, workspace, workspace_bytes,
+                  (cudaStream_t)stream, nullptr, nullptr);
+}
+
+mlstm_status_t mlstm_fwd_chunkwise_timed(const mlstm_fwd_params_t* p, const void* q, const void* k, const void* v,
+                                         const float* igate, const float* fgate, const void* ogate, const float* C0,
+                                         const float* n0, const float* m0, void* h, float* C_out, float* n_out,
+                                         float* m_out, void* workspace, size_t workspace_bytes,
+                                         mlstm_stream_t stream, mlstm_event_t main_begin, mlstm_event_t main_end) {
+  return fwd_impl(p, q, k, v, igate, fgate, ogate, C0, n0, m0, h, C_out, n_out, m_out, workspace, workspace_bytes,
+                  (cudaStream_t)stream, (cudaEvent_t)main_begin, (cudaEvent_t)main_end);
+}
+
+mlstm_status_t mlstm_step(const mlstm_step_params_t* p, const void* q, const void* k, const void* v,
+                          const float* igate, const float* fgate, const void* ogate, float* C, float* n, float* m,
+                          void* h, mlstm_stream_t stream) {
+  if (!p) return MLSTM_ERR_NULL;
+  if (p->dtype != MLSTM_F32 && p->dtype != MLSTM_BF16) return MLSTM_ERR_DTYPE;
+  if (p->B < 0 || p->NH < 0 || p->DHQK < 1 || p->DHV < 1 || p->num_blocks < 1) return MLSTM_ERR_SHAPE;
+  if (p->DHQK % p->num_blocks || p->DHV % p->num_blocks || p->num_blocks > 8) return MLSTM_ERR_SHAPE;
+  const int dk = p->DHQK / p->num_blocks, dv = p->DHV / p->num_blocks;
+  if (!step_supported_dk(dk)) return MLSTM_ERR_SHAPE;
+  const long long BHll = (long long)p->B * p->NH;
+  if (BHll * 8 > (1LL << 31) - 1) return MLSTM_ERR_SHAPE;
+  const size_t BH = (size_t)BHll;
+  const bool ret = p->retention != 0;
+  if (ret) {
+    igate = fgate = nullptr;
+    ogate = nullptr;
+    n = m = nullptr;
+  }
+  if (BH > 0) {
+    if (!q || !k || !v || !C || !h) return MLSTM_ERR_NULL;
+    if (!ret && (!igate || !fgate || !n || !m)) return MLSTM_ERR_NULL;
+  }
+  const void* all[] = {q, k, v, igate, fgate, ogate, C, n, m, h};
+  for (const void* ptr : all)
+    if (ptr && misaligned(ptr)) return MLSTM_ERR_ALIGN;
+  const size_t es = p->dtype == MLSTM_BF16 ? 2 : 4;
+  const Range rq{q, BH * p->DHQK * es}, rk{k, BH * p->DHQK * es}, rv{v, BH * p->DHV * es};
+  const Range rig{igate, BH * 4}, rfg{fgate, BH * 4}, ro{ogate, BH * p->DHV * es};
+  const Range rC{C, (size_t)BH * p->num_blocks * dv * dk * 4}, rn{n, (size_t)BH * p->num_blocks * dk * 4};
+  const Range rm{m, BH * 4}, rh{h, BH * p->DHV * es};
+  const Range ins[] = {rq, rk, rv, rig, rfg, ro};
+  const Range outs[] = {rC, rn, rm, rh};
+  for (int a = 0; a < 4; ++a) {
+    for (const Range& i : ins)
+      if (overlaps(outs[a], i)) return MLSTM_ERR_ALIAS;
+    for (int b = a + 1; b < 4; ++b)
+      if (overlaps(outs[a], outs[b])) return MLSTM_ERR_ALIAS;
+  }
+  if (BH == 0) return MLSTM_OK;
+  StepArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = p->B;
+  a.NH = p->NH;
+  a.DHQK = p->DHQK;
+  a.DHV = p->DHV;
+  a.nb = p->num_blocks;
+  a.retention = ret ? 1 : 0;
+  a.dtype = p->dtype == MLSTM_BF16 ? 1 : 0;
+  a.dk = dk;
+  a.dv = dv;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.og = ogate;
+  a.ig = igate;
+  a.fg = fgate;
+  a.C = C;
+  a.n = n;
+  a.m = m;
+  a.h = h;
+  return launch_step(a, (cudaStream_t)stream) == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,178 @@
+"""Python binding of libmlstm (include/mlstm.h): argument marshalling only.
+
+Every step of the recurrence runs in the library's CUDA kernels.  PyTorch only
+provides device memory (outputs and workspace are allocated here with
+torch.empty when the caller does not pass them) and the current CUDA stream.
+There is no CPU fallback: if the compiled library is missing or no CUDA device
+is present, these functions raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmlstm.so")
+
+MLSTM_F32, MLSTM_BF16 = 0, 1
+_DTYPES = {torch.float32: MLSTM_F32, torch.bfloat16: MLSTM_BF16}
+
+
+class FwdParams(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("NH", ctypes.c_int), ("S", ctypes.c_int), ("DHQK", ctypes.c_int),
+                ("DHV", ctypes.c_int), ("chunk", ctypes.c_int), ("num_blocks", ctypes.c_int),
+                ("dtype", ctypes.c_int), ("retention", ctypes.c_int)]
+
+
+class StepParams(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("NH", ctypes.c_int), ("DHQK", ctypes.c_int), ("DHV", ctypes.c_int),
+                ("num_blocks", ctypes.c_int), ("dtype", ctypes.c_int), ("retention", ctypes.c_int)]
+
+
+class FwdPlan(ctypes.Structure):
+    _fields_ = [("tensor_core", ctypes.c_int), ("segments", ctypes.c_int), ("dv_tile", ctypes.c_int),
+                ("ctas_main", ctypes.c_int), ("kernels", ctypes.c_int), ("workspace_bytes", ctypes.c_size_t)]
+
+
+class MlstmError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: status {status} ({status_string(status)})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libmlstm.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m linear_recurrent_token_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.mlstm_fwd_chunkwise_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
+        L.mlstm_fwd_chunkwise_workspace_size.restype = Z
+        L.mlstm_fwd_chunkwise_plan.argtypes = [ctypes.POINTER(FwdParams), ctypes.POINTER(FwdPlan)]
+        L.mlstm_fwd_chunkwise_plan.restype = I
+        L.mlstm_fwd_chunkwise.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 14 + [Z, P]
+        L.mlstm_fwd_chunkwise.restype = I
+        L.mlstm_fwd_chunkwise_timed.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 14 + [Z, P, P, P]
+        L.mlstm_fwd_chunkwise_timed.restype = I
+        L.mlstm_step.argtypes = [ctypes.POINTER(StepParams)] + [P] * 10 + [P]
+        L.mlstm_step.restype = I
+        L.mlstm_status_string.argtypes = [I]
+        L.mlstm_status_string.restype = ctypes.c_char_p
+        L.mlstm_abi_version.argtypes = []
+        L.mlstm_abi_version.restype = I
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().mlstm_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    try:
+        return _DTYPES[t.dtype]
+    except KeyError:
+        raise TypeError(f"q/k/v must be float32 or bfloat16, got {t.dtype}") from None
+
+
+def fwd_params(B, NH, S, DHQK, DHV, chunk=64, num_blocks=1, dtype=torch.bfloat16, retention=False) -> FwdParams:
+    return FwdParams(int(B), int(NH), int(S), int(DHQK), int(DHV), int(chunk), int(num_blocks),
+                     _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype), int(bool(retention)))
+
+
+def workspace_size(params: FwdParams) -> int:
+    return int(lib().mlstm_fwd_chunkwise_workspace_size(ctypes.byref(params)))
+
+
+def plan(params: FwdParams) -> dict:
+    out = FwdPlan()
+    st = lib().mlstm_fwd_chunkwise_plan(ctypes.byref(params), ctypes.byref(out))
+    if st != 0:
+        raise MlstmError(st, "mlstm_fwd_chunkwise_plan")
+    return {name: getattr(out, name) for name, _ in FwdPlan._fields_}
+
+
+def fwd_chunkwise(q, k, v, igate=None, fgate=None, ogate=None, C0=None, n0=None, m0=None, *,
+                  chunk: int = 64, num_blocks: int = 1, retention: bool = False,
+                  h=None, C_out=None, n_out=None, m_out=None, workspace=None,
+                  return_state: bool = True, stream=None, events=None):
+    """Chunkwise-parallel prefill (mlstm_fwd_chunkwise).  CUDA tensors, contiguous.
+
+    q, k [B,NH,S,DHQK], v [B,NH,S,DHV] (fp32 or bf16); igate, fgate [B,NH,S] fp32;
+    ogate [B,NH,S,DHV] or None; C0 [B,NH,nb,DHV/nb,DHQK/nb], n0 [B,NH,nb,DHQK/nb],
+    m0 [B,NH] fp32 or None (zeros).  Returns (h, C, n, m); n, m are None in
+    retention mode and the state is None when return_state is False.
+    ``events`` = (begin, end) torch.cuda.Event pair recorded around the main kernel.
+    """
+    B, NH, S, DHQK = q.shape
+    DHV = v.shape[-1]
+    nb = int(num_blocks)
+    p = fwd_params(B, NH, S, DHQK, DHV, chunk, nb, q.dtype, retention)
+    dev = q.device
+    if h is None:
+        h = torch.empty((B, NH, S, DHV), dtype=q.dtype, device=dev)
+    if return_state and C_out is None:
+        C_out = torch.empty((B, NH, nb, DHV // nb, DHQK // nb), dtype=torch.float32, device=dev)
+    if return_state and not retention:
+        if n_out is None:
+            n_out = torch.empty((B, NH, nb, DHQK // nb), dtype=torch.float32, device=dev)
+        if m_out is None:
+            m_out = torch.empty((B, NH), dtype=torch.float32, device=dev)
+    ws_bytes = workspace_size(p)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    args = [ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(igate), _ptr(fgate), _ptr(ogate),
+            _ptr(C0), _ptr(n0), _ptr(m0), _ptr(h), _ptr(C_out), _ptr(n_out), _ptr(m_out),
+            _ptr(workspace), ctypes.c_size_t(ws_len), _stream_ptr(stream)]
+    if events is None:
+        st = lib().mlstm_fwd_chunkwise(*args)
+    else:
+        st = lib().mlstm_fwd_chunkwise_timed(*args, ctypes.c_void_p(events[0].cuda_event),
+                                             ctypes.c_void_p(events[1].cuda_event))
+    if st != 0:
+        raise MlstmError(st, "mlstm_fwd_chunkwise")
+    if retention:
+        return h, C_out, None, None
+    return h, C_out, n_out, m_out
+
+
+def step(q, k, v, igate, fgate, C, n, m, ogate=None, *, num_blocks: int = 1, retention: bool = False,
+         h=None, stream=None):
+    """One decode step (mlstm_step), updating C, n, m in place.  Returns h [B,NH,DHV].
+
+    q, k [B,NH,DHQK]; v [B,NH,DHV]; igate, fgate [B,NH] fp32; C [B,NH,nb,DHV/nb,DHQK/nb],
+    n [B,NH,nb,DHQK/nb], m [B,NH] fp32 (n, m, gates may be None in retention mode).
+    """
+    B, NH, DHQK = q.shape
+    DHV = v.shape[-1]
+    p = StepParams(int(B), int(NH), int(DHQK), int(DHV), int(num_blocks), _dtype_code(q), int(bool(retention)))
+    if h is None:
+        h = torch.empty((B, NH, DHV), dtype=q.dtype, device=q.device)
+    st = lib().mlstm_step(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(igate), _ptr(fgate), _ptr(ogate),
+                          _ptr(C), _ptr(n), _ptr(m), _ptr(h), _stream_ptr(stream))
+    if st != 0:
+        raise MlstmError(st, "mlstm_step")
+    return h

@@ -1,0 +1,133 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol and
+rejects invalid arguments on the host before anything is enqueued."""
+import ctypes
+import re
+
+import pytest
+import torch
+
+from linear_recurrent_token_b200 import build, mlstm
+from tests.conftest import ROOT
+
+HEADER = f"{ROOT}/include/mlstm.h"
+
+# Fake, 16-byte aligned, never dereferenced: every call below fails validation first.
+A, B_, C_, D_, E_, F_, G_, H_ = (0x100000 * (i + 1) for i in range(8))
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mlstm_[a-z_]+)\s*\(", text)))
+
+
+def test_library_builds_and_exports_every_declared_symbol():
+    build.build()
+    lib = mlstm.lib()
+    names = declared_functions()
+    assert "mlstm_fwd_chunkwise" in names and "mlstm_step" in names
+    for name in names:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version():
+    for code in range(8):
+        assert mlstm.status_string(code)
+    assert mlstm.status_string(99) == "unknown status"
+    assert mlstm.lib().mlstm_abi_version() >> 16 == 1
+
+
+def fwd(p, q=A, k=B_, v=C_, ig=D_, fg=E_, og=None, C0=None, n0=None, m0=None, h=F_, C=None, n=None, m=None,
+        ws=G_, ws_bytes=1 << 40):
+    P = ctypes.c_void_p
+    return mlstm.lib().mlstm_fwd_chunkwise(ctypes.byref(p), q, k, v, ig, fg, og, C0, n0, m0, h, C, n, m, ws,
+                                           ctypes.c_size_t(ws_bytes), P(0))
+
+
+def params(**kw):
+    base = dict(B=2, NH=2, S=64, DHQK=16, DHV=16, chunk=16, num_blocks=1, dtype=torch.float32, retention=False)
+    base.update(kw)
+    return mlstm.fwd_params(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=-1), 2), (dict(S=-1), 2), (dict(DHQK=0), 2), (dict(chunk=0), 2),
+    (dict(num_blocks=3), 2), (dict(num_blocks=0), 2), (dict(dtype=7), 3),
+])
+def test_fwd_rejects_bad_params(kw, status):
+    assert fwd(params(**kw)) == status
+
+
+def test_fwd_null_pointers():
+    p = params()
+    assert fwd(p, q=None) == 1
+    assert fwd(p, h=None) == 1
+    assert fwd(p, ig=None) == 1
+    assert fwd(p, fg=None) == 1
+
+
+def test_fwd_null_params():
+    P = ctypes.c_void_p
+    st = mlstm.lib().mlstm_fwd_chunkwise(None, A, B_, C_, D_, E_, None, None, None, None, F_, None, None,
+                                         None, G_, ctypes.c_size_t(1 << 30), P(0))
+    assert st == 1
+
+
+def test_fwd_misaligned_pointer():
+    assert fwd(params(), q=A + 8) == 4
+    assert fwd(params(), C=H_ + 4) == 4
+
+
+def test_fwd_workspace_checks():
+    p = params()
+    need = mlstm.workspace_size(p)
+    assert need > 0
+    assert fwd(p, ws=None) == 5
+    assert fwd(p, ws_bytes=need - 1) == 5
+
+
+def test_fwd_aliasing():
+    p = params()
+    # h on top of q
+    assert fwd(p, h=A) == 7
+    # final state partially overlapping the initial state (not an exact in-place alias)
+    assert fwd(p, C0=H_, C=H_ + 256) == 7
+    # workspace on top of v
+    assert fwd(p, ws=C_) == 7
+
+
+def test_workspace_size_and_plan():
+    for kw in (dict(), dict(retention=True), dict(S=0), dict(B=0)):
+        p = params(**kw)
+        plan = mlstm.plan(p)
+        assert plan["workspace_bytes"] == mlstm.workspace_size(p)
+    assert mlstm.workspace_size(params(retention=True)) == 0  # retention needs no gate workspace
+    assert mlstm.workspace_size(params(B=-1)) == 0
+    big = mlstm.fwd_params(1, 8, 8192, 256, 512, 64, 1, torch.bfloat16, False)
+    assert mlstm.workspace_size(big) >= 8 * 8192 * 4
+
+
+def step_call(p, q=A, k=B_, v=C_, ig=D_, fg=E_, og=None, C=F_, n=G_, m=H_, h=0x9000000):
+    return mlstm.lib().mlstm_step(ctypes.byref(p), q, k, v, ig, fg, og, C, n, m, h, ctypes.c_void_p(0))
+
+
+def sparams(**kw):
+    base = dict(B=2, NH=2, DHQK=16, DHV=16, num_blocks=1, dtype=0, retention=0)
+    base.update(kw)
+    return mlstm.StepParams(*[int(base[k]) for k in ("B", "NH", "DHQK", "DHV", "num_blocks", "dtype", "retention")])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(DHQK=24), 2),            # block key width 24 is not a supported power of two
+    (dict(num_blocks=3), 2), (dict(num_blocks=16, DHQK=64, DHV=64), 2), (dict(B=-2), 2), (dict(dtype=5), 3),
+])
+def test_step_rejects_bad_params(kw, status):
+    assert step_call(sparams(**kw)) == status
+
+
+def test_step_null_and_alias():
+    assert step_call(sparams(), C=None) == 1
+    assert step_call(sparams(), n=None) == 1
+    assert step_call(sparams(), h=F_) == 7        # h on top of C
+    assert step_call(sparams(), C=A) == 7         # state on top of q
+    assert step_call(sparams(), q=A + 4) == 4

@@ -1,0 +1,257 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Element-by-element on the same seeded inputs.  Bounds: max relative error per
+(batch, head[, block]) slice <= 1e-4 for fp32 inputs, <= 2e-2 for bf16 inputs
+(fp32 state in both); m within the same bound relative to max(1, |m|).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_recurrent_token_b200 import inputs, mlstm
+from tests.helpers import TOL, TORCH_DTYPE, dev, host, m_err, slice_relerr
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_fwd(inp, dtype, chunk, nb=1, retention=False, ogate=None, C0=None, n0=None, m0=None):
+    td = TORCH_DTYPE[dtype]
+    q, k, v = (dev(inp[x], td) for x in ("q", "k", "v"))
+    ig = None if retention else dev(inp["igate"])
+    fg = None if retention else dev(inp["fgate"])
+    h, C, n, m = mlstm.fwd_chunkwise(q, k, v, ig, fg, dev(ogate, td) if ogate is not None else None,
+                                     dev(C0), dev(n0), dev(m0), chunk=chunk, num_blocks=nb, retention=retention)
+    torch.cuda.synchronize()
+    return host(h), host(C), host(n), host(m)
+
+
+def oracle_fwd(inp, nb=1, retention=False, ogate=None, C0=None, n0=None, m0=None):
+    if retention:
+        return oracle.sequential(inp["q"], inp["k"], inp["v"], C0=C0, num_blocks=nb, retention=True)
+    return oracle.sequential(inp["q"], inp["k"], inp["v"], inp["igate"], inp["fgate"], ogate, C0, n0, m0,
+                             num_blocks=nb)
+
+
+def check(got, ref, dtype, retention=False, what=""):
+    tol = TOL[dtype]
+    h, C, n, m = got
+    hr, Cr, nr, mr = ref
+    errs = {"h": slice_relerr(h, hr, 2), "C": slice_relerr(C, Cr, 3)}
+    if not retention:
+        errs["n"] = slice_relerr(n, nr, 3)
+        errs["m"] = m_err(m, mr)
+    bad = {key: val for key, val in errs.items() if not val <= tol}
+    assert not bad, f"{what} errors above {tol}: {errs}"
+    return errs
+
+
+@pytest.mark.parametrize("idx", [0, 1, 2, 3])
+def test_workload_forward_parity(idx):
+    w = inputs.WORKLOADS[idx]
+    inp = inputs.forward_inputs(w)
+    got = gpu_fwd(inp, w.dtype, w.chunk, w.num_blocks, w.retention)
+    ref = oracle_fwd(inp, w.num_blocks, w.retention)
+    errs = check(got, ref, w.dtype, w.retention, w.describe())
+    print(w.describe(), errs)
+
+
+@pytest.mark.parametrize("S,chunk", [(70, 16), (1, 16), (5, 64), (16, 1), (33, 8), (128, 128)])
+def test_forward_ragged_and_small(S, chunk):
+    w = inputs.WORKLOADS[0]
+    inp = inputs.forward_inputs(w, seed=7, S=S)
+    check(gpu_fwd(inp, "f32", chunk), oracle_fwd(inp), "f32", what=f"S={S} chunk={chunk}")
+
+
+def test_forward_empty_sequence_returns_initial_state():
+    rng = np.random.default_rng(3)
+    C0 = rng.standard_normal((1, 2, 1, 16, 16)).astype(np.float32)
+    n0 = rng.standard_normal((1, 2, 1, 16)).astype(np.float32)
+    m0 = rng.standard_normal((1, 2)).astype(np.float32)
+    z = np.zeros((1, 2, 0, 16), np.float32)
+    inp = dict(q=z, k=z, v=z, igate=np.zeros((1, 2, 0), np.float32), fgate=np.zeros((1, 2, 0), np.float32))
+    h, C, n, m = gpu_fwd(inp, "f32", 16, C0=C0, n0=n0, m0=m0)
+    assert h.shape == (1, 2, 0, 16)
+    assert np.array_equal(C, C0) and np.array_equal(n, n0) and np.array_equal(m, m0)
+
+
+def test_forward_empty_batch():
+    z = np.zeros((0, 2, 8, 16), np.float32)
+    g = np.zeros((0, 2, 8), np.float32)
+    h, C, n, m = gpu_fwd(dict(q=z, k=z, v=z, igate=g, fgate=g), "f32", 4)
+    assert h.shape == (0, 2, 8, 16) and C.shape == (0, 2, 1, 16, 16)
+
+
+@pytest.mark.parametrize("dtype,nb", [("f32", 1), ("bf16", 1), ("f32", 2), ("bf16", 4)])
+def test_forward_initial_state_and_output_gate(dtype, nb):
+    rng = np.random.default_rng(11)
+    B, NH, S, DHQK, DHV = 2, 3, 100, 32, 64
+    w = inputs.Workload(0, "t", B, NH, S, DHQK, DHV, 16, nb, dtype, False, 1 / np.sqrt(DHQK))
+    inp = inputs.forward_inputs(w, seed=12)
+    dk, dv = DHQK // nb, DHV // nb
+    C0 = (rng.standard_normal((B, NH, nb, dv, dk)) * 0.3).astype(np.float32)
+    n0 = (rng.standard_normal((B, NH, nb, dk)) * 0.3).astype(np.float32)
+    m0 = rng.standard_normal((B, NH)).astype(np.float32)
+    og = inputs.round_to(1 / (1 + np.exp(-rng.standard_normal((B, NH, S, DHV)))), dtype)
+    got = gpu_fwd(inp, dtype, 16, nb, ogate=og, C0=C0, n0=n0, m0=m0)
+    ref = oracle_fwd(inp, nb, ogate=og, C0=C0, n0=n0, m0=m0)
+    check(got, ref, dtype, what=f"{dtype} nb={nb}")
+
+
+def test_forward_state_in_place():
+    w = inputs.WORKLOADS[0]
+    inp = inputs.forward_inputs(w, seed=21)
+    rng = np.random.default_rng(22)
+    C0 = (rng.standard_normal((1, 2, 1, 16, 16)) * 0.2).astype(np.float32)
+    n0 = (rng.standard_normal((1, 2, 1, 16)) * 0.2).astype(np.float32)
+    m0 = rng.standard_normal((1, 2)).astype(np.float32)
+    C, n, m = dev(C0), dev(n0), dev(m0)
+    q, k, v, ig, fg = (dev(inp[x]) for x in ("q", "k", "v", "igate", "fgate"))
+    h, C2, n2, m2 = mlstm.fwd_chunkwise(q, k, v, ig, fg, None, C, n, m, chunk=16, C_out=C, n_out=n, m_out=m)
+    torch.cuda.synchronize()
+    assert C2.data_ptr() == C.data_ptr()
+    ref = oracle_fwd(inp, C0=C0, n0=n0, m0=m0)
+    check((host(h), host(C), host(n), host(m)), ref, "f32", what="in place")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_retention_with_initial_state(dtype):
+    rng = np.random.default_rng(31)
+    w = inputs.Workload(2, "r", 2, 4, 90, 32, 48, 16, 1, dtype, True, 1 / np.sqrt(32))
+    inp = inputs.forward_inputs(w, seed=32)
+    C0 = (rng.standard_normal((2, 4, 1, 48, 32)) * 0.2).astype(np.float32)
+    got = gpu_fwd(inp, dtype, 16, retention=True, C0=C0)
+    ref = oracle_fwd(inp, retention=True, C0=C0)
+    check(got, ref, dtype, retention=True, what="retention C0")
+
+
+def test_split_prefill_resume_equals_one_prefill():
+    w = inputs.Workload(1, "s", 2, 2, 192, 64, 64, 64, 2, "bf16", False, 1 / 8)
+    inp = inputs.forward_inputs(w, seed=41)
+    td = torch.bfloat16
+    q, k, v = (dev(inp[x], td) for x in ("q", "k", "v"))
+    ig, fg = dev(inp["igate"]), dev(inp["fgate"])
+    h, C, n, m = mlstm.fwd_chunkwise(q, k, v, ig, fg, chunk=64, num_blocks=2)
+    cut = 100
+    sl = lambda t: t[:, :, :cut].contiguous()
+    sr = lambda t: t[:, :, cut:].contiguous()
+    h1, C1, n1, m1 = mlstm.fwd_chunkwise(sl(q), sl(k), sl(v), sl(ig), sl(fg), chunk=64, num_blocks=2)
+    h2, C2, n2, m2 = mlstm.fwd_chunkwise(sr(q), sr(k), sr(v), sr(ig), sr(fg), None, C1, n1, m1, chunk=64,
+                                         num_blocks=2)
+    torch.cuda.synchronize()
+    ref = oracle_fwd(inp, 2)
+    check((host(torch.cat([h1, h2], 2)), host(C2), host(n2), host(m2)), ref, "bf16", what="split")
+    check((host(h), host(C), host(n), host(m)), ref, "bf16", what="one pass")
+
+
+@pytest.mark.parametrize("dtype,nb,retention", [("f32", 1, False), ("bf16", 2, False), ("bf16", 1, True)])
+def test_prefill_then_decode_steps_equals_longer_prefill(dtype, nb, retention):
+    B, NH, S, K, DHQK, DHV = 2, 2, 80, 12, 64, 32
+    w = inputs.Workload(0, "x", B, NH, S + K, DHQK, DHV, 16, nb, dtype, retention, 1 / 8)
+    inp = inputs.forward_inputs(w, seed=51)
+    td = TORCH_DTYPE[dtype]
+    q, k, v = (dev(inp[x], td) for x in ("q", "k", "v"))
+    ig, fg = dev(inp["igate"]), dev(inp["fgate"])
+    pre = lambda t: t[:, :, :S].contiguous()
+    gi = (None, None) if retention else (pre(ig), pre(fg))
+    h, C, n, m = mlstm.fwd_chunkwise(pre(q), pre(k), pre(v), *gi, chunk=16, num_blocks=nb, retention=retention)
+    hs = [h]
+    for t in range(S, S + K):
+        g2 = (None, None) if retention else (ig[:, :, t].contiguous(), fg[:, :, t].contiguous())
+        ht = mlstm.step(q[:, :, t].contiguous(), k[:, :, t].contiguous(), v[:, :, t].contiguous(), *g2, C, n, m,
+                        num_blocks=nb, retention=retention)
+        hs.append(ht[:, :, None])
+    torch.cuda.synchronize()
+    ref = oracle_fwd(inp, nb, retention)
+    check((host(torch.cat(hs, 2)), host(C), host(n), host(m)), ref, dtype, retention, "prefill+steps")
+
+
+@pytest.mark.parametrize("dk", [4, 8, 16, 32, 64, 128, 256, 512])
+def test_decode_key_widths(dk):
+    B, NH, T, dv = 3, 2, 6, 40
+    w = inputs.Workload(4, "d", B, NH, T, dk, dv, 1, 1, "f32", False, 1 / np.sqrt(dk))
+    inp = inputs.forward_inputs(w, seed=60 + dk)
+    rng = np.random.default_rng(dk)
+    C0 = (rng.standard_normal((B, NH, 1, dv, dk)) * 0.1).astype(np.float32)
+    n0 = (rng.standard_normal((B, NH, 1, dk)) * 0.1).astype(np.float32)
+    m0 = rng.standard_normal((B, NH)).astype(np.float32)
+    C, n, m = dev(C0), dev(n0), dev(m0)
+    hs = []
+    for t in range(T):
+        step_in = [dev(np.ascontiguousarray(inp[x][:, :, t])) for x in ("q", "k", "v", "igate", "fgate")]
+        hs.append(mlstm.step(*step_in, C, n, m)[:, :, None])
+    torch.cuda.synchronize()
+    ref = oracle_fwd(inp, C0=C0, n0=n0, m0=m0)
+    check((host(torch.cat(hs, 2)), host(C), host(n), host(m)), ref, "f32", what=f"decode dk={dk}")
+
+
+@pytest.mark.parametrize("retention,og", [(True, False), (False, True)])
+def test_decode_retention_and_output_gate(retention, og):
+    B, NH, T, DHQK, DHV = 4, 8, 5, 64, 64
+    w = inputs.Workload(4, "d", B, NH, T, DHQK, DHV, 1, 1, "bf16", retention, 1 / 8)
+    inp = inputs.forward_inputs(w, seed=70)
+    rng = np.random.default_rng(71)
+    C0 = (rng.standard_normal((B, NH, 1, DHV, DHQK)) * 0.1).astype(np.float32)
+    n0 = (rng.standard_normal((B, NH, 1, DHQK)) * 0.1).astype(np.float32)
+    m0 = np.zeros((B, NH), np.float32)
+    ogv = inputs.round_to(rng.uniform(0, 1, (B, NH, T, DHV)), "bf16") if og else None
+    C, n, m = dev(C0), dev(n0), dev(m0)
+    hs = []
+    for t in range(T):
+        x = [dev(np.ascontiguousarray(inp[key][:, :, t]), torch.bfloat16) for key in ("q", "k", "v")]
+        g = (None, None) if retention else [dev(np.ascontiguousarray(inp[key][:, :, t])) for key in ("igate", "fgate")]
+        o = dev(np.ascontiguousarray(ogv[:, :, t]), torch.bfloat16) if og else None
+        hs.append(mlstm.step(*x, *g, C, None if retention else n, None if retention else m, o,
+                             retention=retention)[:, :, None])
+    torch.cuda.synchronize()
+    if retention:
+        ref = oracle.sequential(inp["q"], inp["k"], inp["v"], C0=C0, retention=True)
+        got = (host(torch.cat(hs, 2)), host(C), None, None)
+    else:
+        ref = oracle_fwd(inp, ogate=ogv, C0=C0, n0=n0, m0=m0)
+        got = (host(torch.cat(hs, 2)), host(C), host(n), host(m))
+    check(got, ref, "bf16", retention, "decode")
+
+
+def test_large_input_gates_stay_finite():
+    w = inputs.WORKLOADS[0]
+    inp = inputs.forward_inputs(w, seed=80)
+    inp["igate"] = inp["igate"] + 60.0  # exp(60) overflows fp32 without the stabiliser
+    got = gpu_fwd(inp, "f32", 16)
+    assert all(np.all(np.isfinite(x)) for x in got)
+    check(got, oracle_fwd(inp), "f32", what="large igate")
+
+
+@pytest.fixture(scope="module")
+def decode_workload():
+    w = inputs.WORKLOADS[4]
+    C0, n0, m0 = inputs.decode_initial_state(w)
+    seq = inputs.decode_sequence_inputs(w, w.steps)
+    return w, C0, n0, m0, seq
+
+
+def test_decode_workload_parity(decode_workload):
+    """Full decode workload: B128 NH8 256x512, 1024 in-place steps on the GPU; the oracle
+    recomputes 16 sampled (batch, head) slices over all 1024 steps."""
+    w, C0, n0, m0, seq = decode_workload
+    T = w.steps
+    td = torch.bfloat16
+    stacked = {key: dev(np.ascontiguousarray(np.moveaxis(seq[key], 2, 0)), td if key in "qkv" else torch.float32)
+               for key in ("q", "k", "v", "igate", "fgate")}
+    C, n, m = dev(C0), dev(n0), dev(m0)
+    h_all = torch.empty((T, w.B, w.NH, w.DHV), dtype=td, device="cuda")
+    for t in range(T):
+        mlstm.step(stacked["q"][t], stacked["k"][t], stacked["v"][t], stacked["igate"][t], stacked["fgate"][t],
+                   C, n, m, h=h_all[t])
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(99)
+    picks = [(int(b), int(hd)) for b, hd in zip(rng.choice(w.B, 16), rng.choice(w.NH, 16))]
+    bs = [b for b, _ in picks]
+    hs = [hd for _, hd in picks]
+    sub = lambda x: x[bs, hs][:, None]
+    ref = oracle.sequential(sub(seq["q"]), sub(seq["k"]), sub(seq["v"]), sub(seq["igate"]), sub(seq["fgate"]),
+                            None, C0[bs, hs][:, None], n0[bs, hs][:, None], m0[bs, hs][:, None])
+    h = host(h_all).transpose(1, 2, 0, 3)[bs, hs][:, None]
+    got = (h, host(C)[bs, hs][:, None], host(n)[bs, hs][:, None], host(m)[bs, hs][:, None])
+    errs = check(got, ref, "bf16", what="decode workload")
+    print("decode workload", errs)
