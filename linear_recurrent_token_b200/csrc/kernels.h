@@ -32,6 +32,24 @@ size_t simt_walk_smem_bytes(int chunk, int dk, int dv_tile);
 int simt_walk_pick_tile(int chunk, int dk, int dv);
 cudaError_t launch_simt_walk(const WalkArgs& a, cudaStream_t stream);
 
+// Tensor-core (tcgen05) chunkwise prefill: bf16, chunk 64, block key width 64/128/256,
+// block value width a multiple of 64.
+struct TcPlan {
+  int dvt;         // value rows per CTA (MMA M): 128 or 64
+  int n_tiles;     // value tiles per block
+  int G;           // sequence segments per (batch, head, block)
+  int seg_chunks;  // chunks per segment
+};
+bool tc_supported(int dtype, int chunk, int dk, int dv, int DHQK, int DHV);
+int tc_num_sms();
+TcPlan tc_plan(int B, int NH, int S, int nb, int dk, int dv, int num_sms);
+size_t tc_workspace_bytes(const TcPlan& pl, long long BH, int nb, int dk, int dv);
+// ws: workspace of at least tc_workspace_bytes bytes; its first 4 bytes become an error
+// word (0 = ok; nonzero = a bounded wait expired).  ev0/ev1 (may be NULL) are recorded
+// around the walk kernel.
+cudaError_t launch_tc(const WalkArgs& a, const TcPlan& pl, void* ws, cudaStream_t stream, cudaEvent_t ev0,
+                      cudaEvent_t ev1);
+
 // Decode step.
 struct StepArgs {
   int B, NH, DHQK, DHV, nb, retention, dtype;

@@ -14,6 +14,8 @@ struct FwdShape {
   int B, NH, S, DHQK, DHV, chunk, nb, dk, dv, retention, dtype;
   size_t esize;
   long long BH;
+  bool tc;     // tensor-core path
+  TcPlan tcp;  // its plan
 };
 
 mlstm_status_t check_fwd(const mlstm_fwd_params_t* p, FwdShape* s) {
@@ -38,7 +40,13 @@ mlstm_status_t check_fwd(const mlstm_fwd_params_t* p, FwdShape* s) {
   // grid limits of the kernels
   if (s->BH * s->nb > 65535LL || s->BH > (1LL << 31) / 1024) return MLSTM_ERR_SHAPE;
   if ((long long)s->S * s->BH > (1LL << 40)) return MLSTM_ERR_SHAPE;
-  if (s->S > 0 && s->BH > 0 && simt_walk_pick_tile(s->chunk, s->dk, s->dv) == 0) return MLSTM_ERR_SHAPE;
+  s->tc = tc_supported(s->dtype, s->chunk, s->dk, s->dv, s->DHQK, s->DHV);
+  if (s->tc) {
+    s->tcp = tc_plan(s->B, s->NH, s->S, s->nb, s->dk, s->dv, tc_num_sms());
+    if ((long long)s->tcp.G * s->tcp.n_tiles > 65535 || s->BH * s->nb > 65535) return MLSTM_ERR_SHAPE;
+  } else if (s->S > 0 && s->BH > 0 && simt_walk_pick_tile(s->chunk, s->dk, s->dv) == 0) {
+    return MLSTM_ERR_SHAPE;
+  }
   return MLSTM_OK;
 }
 
@@ -46,11 +54,30 @@ size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct WsLayout {
   size_t m_tok, m_init, n_init, total;
+  size_t tc, c_init;  // tensor-core path: its own area, snapshot of C0
 };
 
 WsLayout fwd_layout(const FwdShape& s) {
-  WsLayout w = {0, 0, 0, 0};
-  if (s.retention || s.BH == 0) return w;
+  WsLayout w = {0, 0, 0, 0, 0, 0};
+  if (s.BH == 0) return w;
+  if (s.tc) {
+    size_t off = 0;
+    w.tc = off;
+    off = align_up(off + tc_workspace_bytes(s.tcp, s.BH, s.nb, s.dk, s.dv));
+    if (!s.retention) {
+      w.n_init = off;
+      off = align_up(off + sizeof(float) * (size_t)s.BH * s.nb * s.dk);
+      w.m_init = off;
+      off = align_up(off + sizeof(float) * (size_t)s.BH);
+    }
+    if (s.tcp.G > 1) {
+      w.c_init = off;
+      off = align_up(off + sizeof(float) * (size_t)s.BH * s.nb * s.dv * s.dk);
+    }
+    w.total = off;
+    return w;
+  }
+  if (s.retention) return w;
   size_t off = 0;
   w.m_tok = off;
   off = align_up(off + sizeof(float) * (size_t)s.BH * s.S);
@@ -165,6 +192,25 @@ mlstm_status_t fwd_impl(const mlstm_fwd_params_t* p, const void* q, const void* 
   a.C_out = C_out;
   a.n_out = n_out;
   a.m_out = m_out;
+  if (s.tc) {
+    // snapshots: the walk writes n_out / m_out (and C_out across segments) while other
+    // CTAs may still read n0 / m0 / C0, which the caller may have aliased to them
+    if (!ret && n0) {
+      e = cudaMemcpyAsync(wsb + ws.n_init, n0, bn, cudaMemcpyDeviceToDevice, stream);
+      a.n_init = reinterpret_cast<const float*>(wsb + ws.n_init);
+    }
+    if (e == cudaSuccess && !ret && m0) {
+      e = cudaMemcpyAsync(wsb + ws.m_init, m0, bm, cudaMemcpyDeviceToDevice, stream);
+      a.m_init = reinterpret_cast<const float*>(wsb + ws.m_init);
+    }
+    if (e == cudaSuccess && C0 && C_out == C0 && s.tcp.G > 1) {
+      e = cudaMemcpyAsync(wsb + ws.c_init, C0, bC, cudaMemcpyDeviceToDevice, stream);
+      a.C0 = reinterpret_cast<const float*>(wsb + ws.c_init);
+    }
+    if (e != cudaSuccess) return MLSTM_ERR_CUDA;
+    e = launch_tc(a, s.tcp, wsb + ws.tc, stream, ev0, ev1);
+    return e == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA;
+  }
   if (!ret) {
     a.m_tok = reinterpret_cast<const float*>(wsb + ws.m_tok);
     a.m_init = reinterpret_cast<const float*>(wsb + ws.m_init);
@@ -214,6 +260,15 @@ mlstm_status_t mlstm_fwd_chunkwise_plan(const mlstm_fwd_params_t* p, mlstm_fwd_p
   mlstm_status_t st = check_fwd(p, &s);
   if (st != MLSTM_OK) return st;
   memset(plan, 0, sizeof(*plan));
+  if (s.tc) {
+    plan->tensor_core = 1;
+    plan->segments = s.tcp.G;
+    plan->dv_tile = s.tcp.dvt;
+    plan->ctas_main = (int)(s.tcp.n_tiles * s.tcp.G * s.BH * s.nb);
+    plan->kernels = (s.BH == 0 || s.S == 0) ? 0 : (s.tcp.G > 1 ? 2 : 1);
+    plan->workspace_bytes = fwd_layout(s).total;
+    return MLSTM_OK;
+  }
   plan->tensor_core = 0;
   plan->segments = 1;
   plan->dv_tile = simt_walk_pick_tile(s.chunk, s.dk, s.dv);

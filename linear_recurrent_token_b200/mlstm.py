@@ -150,6 +150,9 @@ def fwd_chunkwise(q, k, v, igate=None, fgate=None, ogate=None, C0=None, n0=None,
     if events is None:
         st = lib().mlstm_fwd_chunkwise(*args)
     else:
+        for e in events:  # torch creates the CUDA event lazily, on its first record
+            if e.cuda_event == 0:
+                e.record(stream)
         st = lib().mlstm_fwd_chunkwise_timed(*args, ctypes.c_void_p(events[0].cuda_event),
                                              ctypes.c_void_p(events[1].cuda_event))
     if st != 0:
