@@ -13,14 +13,16 @@
 //   phase C  (tc_walk_kernel)  per (segment, value tile): combine the initial state and
 //            the summaries of all earlier segments into the segment's start state
 //            (max-plus composition of (Gtot, M) gives the stabiliser), load it into TMEM
-//            as fp32, and walk the segment's chunks:
-//              S = Q K^T                       (tcgen05, M=64 N=64, K=DK)
-//              P = S o D',  D'[t,s] = exp(b_t - b_s + itilde_s - m_t)  (s <= t)
-//              H^T = C_bf16 Q^T  (read-out)    (tcgen05, M=DVT N=64 K=DK)
-//              H^T += ... V^T P^T (intra)      (tcgen05, M=DVT N=64 K=64, own accumulator)
-//              C <- a C + (V o w)^T K          (TMEM round trip for a, then tcgen05 M=DVT N=DK)
-//              h_t = o_t (e^{b_t+m_c-m_t} H_inter + H_intra) / max(|r_t + e^{..} n.q_t|, e^{-m_t})
-//            The last segment writes the final (C, n, m).
+//            as fp32, and walk the segment's chunks (Q, K, V double-buffered by TMA):
+//              S   = Q K^T                          tcgen05 M=64 N=64 K=DK
+//              P   = S o D',  D'[t,s] = exp(b_t - b_s + itilde_s - m_t), s <= t
+//              Cb  = bf16(C) written into TMEM; C <- a C   (TMEM round trip)
+//              H^T = Cb (e^{b_t+m_c-m_t} Q)^T       tcgen05, A from TMEM, M=DVT N=64
+//              H^T += V^T P^T                      tcgen05 M=DVT N=64 K=64 (same accumulator)
+//              C   += (V o w)^T K                  tcgen05 M=DVT N=DK K=64
+//              h_t = o_t H_t / max(|sum_s P[t,s] + e^{b_t+m_c-m_t} n.q_t|, e^{-m_t})
+//            with n <- a n + sum_s w_s k_s kept in fp32 shared memory.  The last segment
+//            writes the final (C, n, m).
 // Retention (RetNet "Key Innovation"): log f = log gamma_h, itilde = 0, m = 0, no
 // normaliser; the same kernels with those gate values.
 //
@@ -69,9 +71,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
-__device__ __forceinline__ float bf16_at(const uint8_t* tile, int row, int col) {
-  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tile + sw128_offset(row, col)));
-}
 
 // Gate values of token t (global index) for head `head`: (log f, itilde).
 __device__ __forceinline__ void gate_vals(const TcParams& p, size_t tok, int head, float& lf, float& li) {
@@ -87,6 +86,7 @@ __device__ __forceinline__ void gate_vals(const TcParams& p, size_t tok, int hea
 }  // namespace
 
 // ===================================================================== phase A
+// CTA = (value tile, segment < G-1, slice); 128 threads.  Two TMA stages of (K, V).
 template <int DK, int DVT>
 __global__ void __launch_bounds__(NT, 1)
     tc_segment_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV, TcParams p) {
@@ -96,7 +96,8 @@ __global__ void __launch_bounds__(NT, 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* Ks[2] = {sm, sm + KB};
   uint8_t* Vs[2] = {sm + 2 * KB, sm + 2 * KB + VB};
-  float* omega = reinterpret_cast<float*>(sm + 2 * KB + 2 * VB);  // [seg_chunks * L]
+  float* dnp = reinterpret_cast<float*>(sm + 2 * KB + 2 * VB);  // [NT * 8] partial sums of dn
+  float* omega = dnp + NT * 8;                                   // [seg_chunks * L]
   __shared__ uint64_t bar_load[2], bar_mma[2];
   __shared__ uint32_t tmem_base;
   __shared__ float red[NT / 32];
@@ -108,6 +109,10 @@ __global__ void __launch_bounds__(NT, 1)
   const int seg_len = p.seg_chunks * L;
   const int T0 = g * seg_len;  // phase A covers full segments only
   const int v0 = tile * DVT;
+  // this tile accumulates dn over key columns [dn0, min(DK, dn0 + dnw)), dnw a multiple of 8
+  const int dnw = ((DK + p.n_tiles - 1) / p.n_tiles + 7) / 8 * 8;
+  const int dn0 = tile * dnw;
+  const bool do_dn = !p.retention && dn0 < DK;
 
   if (tid == 0) {
     mbar_init(&bar_load[0], 1);
@@ -124,16 +129,19 @@ __global__ void __launch_bounds__(NT, 1)
   tc_fence_after();
   const uint32_t tm = tmem_base;
 
-  // first chunk in flight while the gates are prepared
   const int nck = p.seg_chunks;
   auto issue = [&](int c) {
     const int st = c & 1;
     mbar_arrive_expect_tx(&bar_load[st], KB + VB);
-    for (int j = 0; j < DK / 64; ++j) tma_load_3d(Ks[st] + j * 8192, &mapK, blk * p.dk + 64 * j, T0 + c * L, bh, &bar_load[st]);
+    for (int j = 0; j < DK / 64; ++j)
+      tma_load_3d(Ks[st] + j * 8192, &mapK, blk * p.dk + 64 * j, T0 + c * L, bh, &bar_load[st]);
     for (int j = 0; j < DVT / 64; ++j)
       tma_load_3d(Vs[st] + j * 8192, &mapV, blk * p.dv + v0 + 64 * j, T0 + c * L, bh, &bar_load[st]);
   };
-  if (tid == 0) issue(0);
+  if (tid == 0) {
+    issue(0);
+    if (nck > 1) issue(1);
+  }
 
   // ---- gates: G_s (inclusive cumulative log f), Gtot, M, omega_s
   const size_t tok0 = (size_t)bh * p.S + T0;
@@ -143,9 +151,9 @@ __global__ void __launch_bounds__(NT, 1)
   for (int t = r0; t < r1; ++t) {
     float lf, li;
     gate_vals(p, tok0 + t, head, lf, li);
+    omega[t] = lf;
     run += lf;
   }
-  // exclusive scan of run sums over the block
   float inc = run;
   for (int o = 1; o < 32; o <<= 1) {
     const float u = __shfl_up_sync(0xffffffffu, inc, o);
@@ -158,12 +166,11 @@ __global__ void __launch_bounds__(NT, 1)
     if (w < warp) wexcl += red[w];
     total += red[w];
   }
-  float Gs = wexcl + inc - run;  // exclusive prefix of this thread's run
+  float Gs = wexcl + inc - run;
   float lmax = -INFINITY;
   for (int t = r0; t < r1; ++t) {
-    float lf, li;
-    gate_vals(p, tok0 + t, head, lf, li);
-    Gs += lf;
+    Gs += omega[t];
+    const float li = p.retention ? 0.f : p.ig[tok0 + t];
     const float x = li - Gs;  // log weight minus Gtot
     omega[t] = x;
     lmax = fmaxf(lmax, total + x);
@@ -184,20 +191,18 @@ __global__ void __launch_bounds__(NT, 1)
 
   // ---- main loop: D[dv, dk] += (V o omega)^T K over the segment
   const uint32_t idesc = idesc_bf16(DVT, DK, 1, 1);
-  float dn_acc[2] = {0.f, 0.f};  // columns tid and tid + 128 of dn (value tile 0 only)
+  // dn partials: thread -> (column group of 8 inside this tile's columns, row group)
+  const int ncg = dnw / 8 < NT ? dnw / 8 : NT, nrg = NT / ncg, rows_per = (L + nrg - 1) / nrg;
+  const int cg = tid % ncg, rg = tid / ncg;
+  const int dcol = dn0 + 8 * cg;  // first of this thread's 8 columns
+  float dacc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) dacc[j] = 0.f;
   for (int c = 0; c < nck; ++c) {
     const int st = c & 1;
-    if (c + 1 < nck) {
-      if (c >= 1 && !abort_flag) {  // the MMAs of chunk c-1 read stage st^1
-        if (!mbar_wait(&bar_mma[st ^ 1], ((c - 1) >> 1) & 1, WAIT)) atomicOr(&abort_flag, 1);
-      }
-      __syncthreads();
-      if (tid == 0 && !abort_flag) issue(c + 1);
-    }
     if (!abort_flag && !mbar_wait(&bar_load[st], (c >> 1) & 1, WAIT)) atomicOr(&abort_flag, 1);
     __syncthreads();
     if (abort_flag) break;
-    // V rows scaled in place by omega (a row is 128 contiguous bytes whatever the swizzle)
     const float* om = omega + c * L;
     for (int i = tid; i < L * (DVT / 8); i += NT) {
       const int row = i / (DVT / 8), ch = i % (DVT / 8);
@@ -207,18 +212,22 @@ __global__ void __launch_bounds__(NT, 1)
       const float w = om[row];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        float2 f = __bfloat1622float2(b2[j]);
+        const float2 f = __bfloat1622float2(b2[j]);
         b2[j] = __floats2bfloat162_rn(f.x * w, f.y * w);
       }
       *reinterpret_cast<uint4*>(ptr) = u;
     }
-    if (tile == 0) {
-      for (int j = 0; j < 2; ++j) {
-        const int col = tid + 128 * j;
-        if (col < DK) {
-          float a = 0.f;
-          for (int s = 0; s < L; ++s) a += om[s] * bf16_at(Ks[st] + (col >> 6) * 8192, s, col & 63);
-          dn_acc[j] += a;
+    if (do_dn && rg < nrg && dcol < DK) {
+      const uint8_t* kt = Ks[st] + (dcol >> 6) * 8192;
+      for (int s = rg * rows_per; s < min(L, (rg + 1) * rows_per); ++s) {
+        const uint4 u = *reinterpret_cast<const uint4*>(kt + sw128_offset(s, dcol & 63));
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+        const float w = om[s];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __bfloat1622float2(b2[j]);
+          dacc[2 * j] += w * f.x;
+          dacc[2 * j + 1] += w * f.y;
         }
       }
     }
@@ -234,6 +243,12 @@ __global__ void __launch_bounds__(NT, 1)
       }
       mma_commit(&bar_mma[st]);
     }
+    // stage st is reloaded with chunk c+2 once this chunk's MMAs have read it
+    if (c + 2 < nck) {
+      if (!abort_flag && !mbar_wait(&bar_mma[st], (c >> 1) & 1, WAIT)) atomicOr(&abort_flag, 1);
+      __syncthreads();
+      if (tid == 0 && !abort_flag) issue(c + 2);
+    }
   }
   if (!abort_flag && !mbar_wait(&bar_mma[(nck - 1) & 1], ((nck - 1) >> 1) & 1, WAIT)) atomicOr(&abort_flag, 1);
   __syncthreads();
@@ -241,19 +256,25 @@ __global__ void __launch_bounds__(NT, 1)
   if (!abort_flag) {
     const int row = acc_row<DVT>(warp, lane);
     float* dst = row >= 0 ? p.dC + (((size_t)slice * (p.G - 1) + g) * p.dv + v0 + row) * p.dk : nullptr;
-    for (int c0 = 0; c0 < DK; c0 += 16) {
-      float r[16];
-      tmem_ld16(tm + ((uint32_t)(32 * warp) << 16) + c0, r);
+    for (int c0 = 0; c0 < DK; c0 += 32) {
+      float r[32];
+      tmem_ld32(tm + ((uint32_t)(32 * warp) << 16) + c0, r);
       tmem_wait_ld();
       if (dst)
-        for (int j = 0; j < 16; j += 4)
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
           *reinterpret_cast<float4*>(dst + c0 + j) = make_float4(r[j], r[j + 1], r[j + 2], r[j + 3]);
     }
-    if (tile == 0)
-      for (int j = 0; j < 2; ++j) {
-        const int col = tid + 128 * j;
-        if (col < DK) p.dn[((size_t)slice * (p.G - 1) + g) * p.dk + col] = dn_acc[j];
+    if (do_dn) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) dnp[tid * 8 + j] = dacc[j];
+      __syncthreads();
+      for (int col = tid; col < ncg * 8 && dn0 + col < DK; col += NT) {
+        float x = 0.f;
+        for (int r = 0; r < nrg; ++r) x += dnp[(r * ncg + col / 8) * 8 + (col & 7)];
+        p.dn[((size_t)slice * (p.G - 1) + g) * p.dk + dn0 + col] = x;
       }
+    }
   } else if (tid == 0) {
     atomicOr(p.err, 1u);
   }
@@ -263,51 +284,61 @@ __global__ void __launch_bounds__(NT, 1)
 }
 
 // ===================================================================== phase C
+constexpr int NTW = 256;  // walk kernel: 8 warps; warps w and w+4 share TMEM lane quarter w%4
+
 template <int DK, int DVT>
 struct WalkSmem {
-  static constexpr int QB = DK * 128, KB = DK * 128, VB = DVT * 128, PB = 64 * 128, CB = DVT * DK * 2;
-  static constexpr int OQ = 0, OK = OQ + QB, OV = OK + KB, OVW = OV + VB, OP = OVW + VB, OC = OP + PB;
-  static constexpr int OF = OC + CB;                   // floats start here
-  static constexpr int NF = DK + 8 * L + 16;           // n, per-token arrays, scalars
-  static constexpr int BYTES = OF + NF * 4 + 1024;     // + alignment slack
+  static constexpr int QB = DK * 128, KB = DK * 128, VB = DVT * 128, PB = 64 * 128;
+  static constexpr int STAGE = QB + KB + VB;
+  static constexpr int OS0 = 0, OS1 = STAGE, OVW = 2 * STAGE, OP = OVW + VB;
+  static constexpr int OF = OP + PB;                                  // floats start here
+  static constexpr int NF = DK + NTW * 8 + 10 * L + 16;               // n, n partials, per-token, scalars
+  static constexpr int BYTES = OF + NF * 4 + 1024;                    // + alignment slack
 };
 
 template <int DK, int DVT>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NTW, 1)
     tc_walk_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                    const __grid_constant__ CUtensorMap mapV, TcParams p) {
   using SM = WalkSmem<DK, DVT>;
-  constexpr uint32_t TM_C = 0, TM_S = DK, TM_I = DK + 64, TM_J = DK + 128;  // TMEM columns
-  constexpr uint32_t TM_COLS = (DK + 192 <= 256) ? 256 : 512;
+  // TMEM columns: C fp32 [DK], bf16 copy of C as MMA operand [DK/2], S [64], H [64]
+  constexpr uint32_t TM_C = 0, TM_CB = DK, TM_S = DK + DK / 2, TM_H = TM_S + 64;
+  constexpr uint32_t TM_COLS = (TM_H + 64 <= 256) ? 256 : 512;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *Qs = sm + SM::OQ, *Ks = sm + SM::OK, *Vs = sm + SM::OV, *Vw = sm + SM::OVW, *Ps = sm + SM::OP,
-          *Cb = sm + SM::OC;
+  uint8_t* stage_base[2] = {sm + SM::OS0, sm + SM::OS1};
+  uint8_t *Vw = sm + SM::OVW, *Ps = sm + SM::OP;
   float* nvec = reinterpret_cast<float*>(sm + SM::OF);
-  float* bl = nvec + DK;
+  float* npart = nvec + DK;  // [NTW * 8]
+  float* bl = npart + NTW * 8;
   float* li = bl + L;
   float* mt = li + L;
   float* sint = mt + L;
   float* wv = sint + L;
-  float* den = wv + L;
-  float* nq = den + L;
-  float* scal = nq + L;  // [0] decay a, [1] m_c, [2] m_next
-  __shared__ uint64_t bar_load, bar_s, bar_mma;
+  float* rden = wv + L;
+  float* nq = rden + L;
+  float* rs2 = nq + L;       // [2][L] row-sum halves
+  float* cs = rs2 + 2 * L;   // li - bl (per column s of P)
+  float* scal = cs + L;      // [0] decay a, [1] m_c, [2] m_next
+  __shared__ uint64_t bar_load[2], bar_s, bar_mma;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quarter = warp & 3, half = warp >> 2;
   const int tile = blockIdx.x, g = blockIdx.y, slice = blockIdx.z;
   const int blk = slice % p.nb, bh = slice / p.nb, head = bh % p.NH;
   const int v0 = tile * DVT;
   const int seg_len = p.seg_chunks * L;
   const int T0 = g * seg_len, T1 = min(p.S, T0 + seg_len);
+  const int nck = (T1 - T0 + L - 1) / L;
   const bool ret = p.retention != 0;
   const bool last_seg = g == p.G - 1;
-  const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+  const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
 
   if (tid == 0) {
-    mbar_init(&bar_load, 1);
+    mbar_init(&bar_load[0], 1);
+    mbar_init(&bar_load[1], 1);
     mbar_init(&bar_s, 1);
     mbar_init(&bar_mma, 1);
     abort_flag = 0;
@@ -321,54 +352,85 @@ __global__ void __launch_bounds__(NT, 1)
   tc_fence_after();
   const uint32_t tm = tmem_base;
 
-  auto issue = [&](int t0) {
-    mbar_arrive_expect_tx(&bar_load, SM::QB + SM::KB + SM::VB);
+  auto issue = [&](int c) {
+    const int st = c & 1;
+    uint8_t* base = stage_base[st];
+    const int t0 = T0 + c * L;
+    mbar_arrive_expect_tx(&bar_load[st], SM::STAGE);
     for (int j = 0; j < DK / 64; ++j) {
-      tma_load_3d(Qs + j * 8192, &mapQ, blk * p.dk + 64 * j, t0, bh, &bar_load);
-      tma_load_3d(Ks + j * 8192, &mapK, blk * p.dk + 64 * j, t0, bh, &bar_load);
+      tma_load_3d(base + j * 8192, &mapQ, blk * p.dk + 64 * j, t0, bh, &bar_load[st]);
+      tma_load_3d(base + SM::QB + j * 8192, &mapK, blk * p.dk + 64 * j, t0, bh, &bar_load[st]);
     }
-    for (int j = 0; j < DVT / 64; ++j) tma_load_3d(Vs + j * 8192, &mapV, blk * p.dv + v0 + 64 * j, t0, bh, &bar_load);
+    for (int j = 0; j < DVT / 64; ++j)
+      tma_load_3d(base + SM::QB + SM::KB + j * 8192, &mapV, blk * p.dv + v0 + 64 * j, t0, bh, &bar_load[st]);
   };
-  if (tid == 0) issue(T0);
+  if (tid == 0) issue(0);
 
-  // ---- start state of the segment: stabiliser by max-plus composition of the earlier
-  // segments' (Gtot, M); C and n as the matching weighted sum of C0 and the summaries.
+  // raw gates of the next chunk, held by warp 0 (two tokens per lane)
+  float rfa = 0.f, ria = 0.f, rfb = 0.f, rib = 0.f;
+  auto fetch_gates = [&](int c) {
+    const int t0 = T0 + c * L;
+    const int Lc = min(L, T1 - t0);
+    const size_t tok = (size_t)bh * p.S + t0;
+    const int ta = 2 * lane, tb = 2 * lane + 1;
+    if (!ret) {
+      rfa = ta < Lc ? p.fg[tok + ta] : 0.f;
+      ria = ta < Lc ? p.ig[tok + ta] : 0.f;
+      rfb = tb < Lc ? p.fg[tok + tb] : 0.f;
+      rib = tb < Lc ? p.ig[tok + tb] : 0.f;
+    }
+  };
+  if (warp == 0) fetch_gates(0);
+
+  // ---- start state of the segment (see the file header)
   float m_start = ret ? 0.f : (p.m0 ? p.m0[bh] : 0.f);
   const float m_init = m_start;
-  float gsum = 0.f;  // sum of Gtot over segments 0..g-1
+  float gsum = 0.f;
   for (int j = 0; j < g; ++j) {
     const float A = p.segA[(size_t)bh * (p.G - 1) + j], Bm = p.segB[(size_t)bh * (p.G - 1) + j];
     if (!ret) m_start = fmaxf(A + m_start, Bm);
     gsum += A;
   }
-  // weight of C0: exp(gsum + m_init - m_start); of summary j: exp(M_j + sum_{j<i<g} Gtot_i - m_start)
   {
-    const int row = acc_row<DVT>(warp, lane);
+    const int row = acc_row<DVT>(quarter, lane);
     const float wc0 = expf(gsum + m_init - m_start);
-    for (int c0 = 0; c0 < DK; c0 += 16) {
+    for (int c0 = half * (DK / 2); c0 < (half + 1) * (DK / 2); c0 += 16) {
       float r[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) r[j] = 0.f;
       if (row >= 0) {
         if (p.C0) {
-          const float* src = p.C0 + ((size_t)slice * p.dv + v0 + row) * p.dk + c0;
+          const float4* src = reinterpret_cast<const float4*>(p.C0 + ((size_t)slice * p.dv + v0 + row) * p.dk + c0);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) r[j] = wc0 * src[j];
+          for (int j = 0; j < 4; ++j) {
+            const float4 x = src[j];
+            r[4 * j] = wc0 * x.x;
+            r[4 * j + 1] = wc0 * x.y;
+            r[4 * j + 2] = wc0 * x.z;
+            r[4 * j + 3] = wc0 * x.w;
+          }
         }
         float after = gsum;
         for (int jg = 0; jg < g; ++jg) {
           after -= p.segA[(size_t)bh * (p.G - 1) + jg];
           const float wj = expf(p.segB[(size_t)bh * (p.G - 1) + jg] + after - m_start);
-          const float* src = p.dC + (((size_t)slice * (p.G - 1) + jg) * p.dv + v0 + row) * p.dk + c0;
+          const float4* src = reinterpret_cast<const float4*>(
+              p.dC + (((size_t)slice * (p.G - 1) + jg) * p.dv + v0 + row) * p.dk + c0);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) r[j] += wj * src[j];
+          for (int j = 0; j < 4; ++j) {
+            const float4 x = src[j];
+            r[4 * j] += wj * x.x;
+            r[4 * j + 1] += wj * x.y;
+            r[4 * j + 2] += wj * x.z;
+            r[4 * j + 3] += wj * x.w;
+          }
         }
       }
       tmem_st16(tm + lane_off + TM_C + c0, r);
     }
     tmem_wait_st();
     if (!ret)
-      for (int col = tid; col < DK; col += NT) {
+      for (int col = tid; col < DK; col += NTW) {
         float x = p.n0 ? wc0 * p.n0[(size_t)slice * p.dk + col] : 0.f;
         float after = gsum;
         for (int jg = 0; jg < g; ++jg) {
@@ -389,22 +451,35 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t id_pv = idesc_bf16(DVT, 64, 1, 0);
   const uint32_t id_up = idesc_bf16(DVT, DK, 1, 1);
   const float lg = ret ? retention_log_gamma(head) : 0.f;
+  constexpr float LOG2E = 1.4426950408889634f;
 
-  int it = 0;
-  for (int t0 = T0; t0 < T1; t0 += L, ++it) {
+  for (int it = 0; it < nck; ++it) {
+    const int st = it & 1;
+    const int t0 = T0 + it * L;
     const int Lc = min(L, T1 - t0);
     const size_t tok0 = (size_t)bh * p.S + t0;
+    uint8_t* Qs = stage_base[st];
+    uint8_t* Ks = Qs + SM::QB;
+    uint8_t* Vs = Ks + SM::KB;
+    // the other stage was released at the end of the previous chunk: prefetch chunk it+1
+    if (tid == 0 && it + 1 < nck && !abort_flag) issue(it + 1);
     // ---- per-token gate quantities (warp 0): b (cumulative log f), m_t, scales
     if (warp == 0) {
       const float mc = scal[1];
-      float lfa, lia, lfb, lib;
       const int ta = 2 * lane, tb = 2 * lane + 1;
-      if (ta < Lc) gate_vals(p, tok0 + ta, head, lfa, lia); else { lfa = 0.f; lia = -INFINITY; }
-      if (tb < Lc) gate_vals(p, tok0 + tb, head, lfb, lib); else { lfb = 0.f; lib = -INFINITY; }
-      float sum = lfa + lfb;
-      float isum = sum;
-      MaxPlus mp = mp_then(MaxPlus{lfa, lia}, MaxPlus{lfb, lib});
-      MaxPlus imp = mp;
+      float lfa, lia, lfb, lib;
+      if (ret) {
+        lfa = lfb = lg;
+        lia = lib = 0.f;
+      } else {
+        lfa = ta < Lc ? log_sigmoid(rfa) : 0.f;
+        lia = ta < Lc ? ria : -INFINITY;
+        lfb = tb < Lc ? log_sigmoid(rfb) : 0.f;
+        lib = tb < Lc ? rib : -INFINITY;
+      }
+      if (it + 1 < nck) fetch_gates(it + 1);
+      float isum = lfa + lfb;
+      MaxPlus imp = mp_then(MaxPlus{lfa, lia}, MaxPlus{lfb, lib});
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const float us = __shfl_up_sync(0xffffffffu, isum, o);
@@ -421,21 +496,14 @@ __global__ void __launch_bounds__(NT, 1)
         emp = MaxPlus{0.f, -INFINITY};
       }
       const float ba = esum + lfa, bb = esum + lfa + lfb;
-      float ma, mb;
-      if (ret) {
-        ma = mb = 0.f;
-      } else {
+      float ma = 0.f, mb = 0.f;
+      if (!ret) {
         const MaxPlus pa = mp_then(emp, MaxPlus{lfa, lia});
         ma = mp_apply(pa, mc);
         mb = mp_apply(mp_then(pa, MaxPlus{lfb, lib}), mc);
       }
-      if (ret) {
-        bl[ta] = (float)(ta + 1) * lg;
-        bl[tb] = (float)(tb + 1) * lg;
-      } else {
-        bl[ta] = ba;
-        bl[tb] = bb;
-      }
+      bl[ta] = ba;
+      bl[tb] = bb;
       li[ta] = ret ? 0.f : lia;
       li[tb] = ret ? 0.f : lib;
       mt[ta] = ma;
@@ -443,16 +511,18 @@ __global__ void __launch_bounds__(NT, 1)
       __syncwarp();
       const float gtot = bl[Lc - 1];
       const float mn = mt[Lc - 1];
-      sint[ta] = expf(bl[ta] + mc - ma);
-      sint[tb] = expf(bl[tb] + mc - mb);
-      wv[ta] = ta < Lc ? expf(gtot - bl[ta] + li[ta] - mn) : 0.f;
-      wv[tb] = tb < Lc ? expf(gtot - bl[tb] + li[tb] - mn) : 0.f;
+      sint[ta] = expf(ba + mc - ma);
+      sint[tb] = expf(bb + mc - mb);
+      wv[ta] = ta < Lc ? expf(gtot - ba + li[ta] - mn) : 0.f;
+      wv[tb] = tb < Lc ? expf(gtot - bb + li[tb] - mn) : 0.f;
+      cs[ta] = ta < Lc ? (li[ta] - ba) * LOG2E : -INFINITY;
+      cs[tb] = tb < Lc ? (li[tb] - bb) * LOG2E : -INFINITY;
       if (lane == 0) {
         scal[0] = expf(gtot + mc - mn);
         scal[2] = mn;
       }
     }
-    if (!abort_flag && !mbar_wait(&bar_load, it & 1, WAIT)) atomicOr(&abort_flag, 1);
+    if (!abort_flag && !mbar_wait(&bar_load[st], (it >> 1) & 1, WAIT)) atomicOr(&abort_flag, 1);
     __syncthreads();
     if (abort_flag) break;
     // ---- S = Q K^T
@@ -466,24 +536,29 @@ __global__ void __launch_bounds__(NT, 1)
       }
       mma_commit(&bar_s);
     }
-    // ---- n . q_t (two threads per token) and V o w
+    // ---- n . q_t (four threads per token) and V o w
     if (!ret) {
-      const int t = tid >> 1, half = tid & 1;
+      const int t = tid >> 2, part = tid & 3;
       float a = 0.f;
-      for (int col = half * (DK / 2); col < (half + 1) * (DK / 2); col += 8) {
-        const uint8_t* ptr = Qs + (col >> 6) * 8192 + sw128_offset(t, col & 63);
-        const uint4 u = *reinterpret_cast<const uint4*>(ptr);
+      for (int col = part * (DK / 4); col < (part + 1) * (DK / 4); col += 8) {
+        const uint4 u = *reinterpret_cast<const uint4*>(Qs + (col >> 6) * 8192 + sw128_offset(t, col & 63));
         const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float2 f = __bfloat1622float2(b2[j]);
-          a += f.x * nvec[col + 2 * j] + f.y * nvec[col + 2 * j + 1];
-        }
+        const float4 n0 = *reinterpret_cast<const float4*>(nvec + col);
+        const float4 n1 = *reinterpret_cast<const float4*>(nvec + col + 4);
+        float2 f = __bfloat1622float2(b2[0]);
+        a += f.x * n0.x + f.y * n0.y;
+        f = __bfloat1622float2(b2[1]);
+        a += f.x * n0.z + f.y * n0.w;
+        f = __bfloat1622float2(b2[2]);
+        a += f.x * n1.x + f.y * n1.y;
+        f = __bfloat1622float2(b2[3]);
+        a += f.x * n1.z + f.y * n1.w;
       }
       a += __shfl_xor_sync(0xffffffffu, a, 1);
-      if (half == 0) nq[t] = a;
+      a += __shfl_xor_sync(0xffffffffu, a, 2);
+      if (part == 0) nq[t] = a;
     }
-    for (int i = tid; i < L * (DVT / 8); i += NT) {
+    for (int i = tid; i < L * (DVT / 8); i += NTW) {
       const int row = i / (DVT / 8), ch = i % (DVT / 8);
       const int off = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
       uint4 u = *reinterpret_cast<const uint4*>(Vs + off);
@@ -500,114 +575,147 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
     if (abort_flag) break;
     tc_fence_after();
-    // ---- P = S o D' (bf16, K-major rows t), row sums, denominators
+    // ---- P = S o D' (bf16, rows t), half the columns per warp half; row-sum halves
     {
-      const int t = acc_row<64>(warp, lane);
-      float rs = 0.f;
-      for (int s0 = 0; s0 < L; s0 += 16) {
-        float r[16];
-        tmem_ld16(tm + lane_off + TM_S + s0, r);
-        tmem_wait_ld();
-        if (t >= 0) {
-          float pv[16];
+      const int t = acc_row<64>(quarter, lane);
+      float r[32];
+      tmem_ld32(tm + lane_off + TM_S + half * 32, r);
+      tmem_wait_ld();
+      if (t >= 0) {
+        const float ct = (bl[t] - mt[t]) * LOG2E;
+        float rs = 0.f;
+        uint32_t pk[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int s = s0 + j;
-            float v = 0.f;
-            if (s <= t && t < Lc) v = r[j] * expf(bl[t] - bl[s] + li[s] - mt[t]);
-            pv[j] = v;
-            rs += v;
-          }
-          const uint32_t base = smem_u32(Ps);
-          st_shared_v4(base + sw128_offset(t, s0), pack_bf16(pv[0], pv[1]), pack_bf16(pv[2], pv[3]),
-                       pack_bf16(pv[4], pv[5]), pack_bf16(pv[6], pv[7]));
-          st_shared_v4(base + sw128_offset(t, s0 + 8), pack_bf16(pv[8], pv[9]), pack_bf16(pv[10], pv[11]),
-                       pack_bf16(pv[12], pv[13]), pack_bf16(pv[14], pv[15]));
+        for (int j = 0; j < 32; j += 2) {
+          const int s = half * 32 + j;
+          const float e0 = (s <= t && t < Lc) ? r[j] * exp2f(ct + cs[s]) : 0.f;
+          const float e1 = (s + 1 <= t && t < Lc) ? r[j + 1] * exp2f(ct + cs[s + 1]) : 0.f;
+          rs += e0 + e1;
+          pk[j / 2] = pack_bf16(e0, e1);
         }
+        const uint32_t base = smem_u32(Ps);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+          st_shared_v4(base + sw128_offset(t, half * 32 + 8 * q4), pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2],
+                       pk[4 * q4 + 3]);
+        rs2[half * L + t] = rs;
       }
-      if (t >= 0 && !ret) den[t] = fmaxf(fabsf(rs + sint[t] * nq[t]), expf(-mt[t]));
     }
-    // ---- C round trip: bf16 copy of C_c for the read-out, C <- a C in TMEM
-    {
-      const int row = acc_row<DVT>(warp, lane);
-      const float a = scal[0];
-      const uint32_t cb = smem_u32(Cb);
-      for (int c0 = 0; c0 < DK; c0 += 16) {
-        float r[16];
-        tmem_ld16(tm + lane_off + TM_C + c0, r);
-        tmem_wait_ld();
-        if (row >= 0) {
-          const uint32_t base = cb + (c0 >> 6) * (DVT * 128);
-          st_shared_v4(base + sw128_offset(row, c0 & 63), pack_bf16(r[0], r[1]), pack_bf16(r[2], r[3]),
-                       pack_bf16(r[4], r[5]), pack_bf16(r[6], r[7]));
-          st_shared_v4(base + sw128_offset(row, (c0 & 63) + 8), pack_bf16(r[8], r[9]), pack_bf16(r[10], r[11]),
-                       pack_bf16(r[12], r[13]), pack_bf16(r[14], r[15]));
-        }
+    // ---- Q <- e^{b_t+m_c-m_t} Q (the inter-chunk read-out then shares the accumulator)
+    for (int i = tid; i < L * (DK / 8); i += NTW) {
+      const int row = i / (DK / 8), ch = i % (DK / 8);
+      const int off = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
+      uint4 u = *reinterpret_cast<const uint4*>(Qs + off);
+      __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&u);
+      const float w = sint[row];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) r[j] *= a;
-        tmem_st16(tm + lane_off + TM_C + c0, r);
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(b2[j]);
+        b2[j] = __floats2bfloat162_rn(f.x * w, f.y * w);
+      }
+      *reinterpret_cast<uint4*>(Qs + off) = u;
+    }
+    // ---- C round trip: bf16 copy of C_c into TMEM (MMA operand), C <- a C
+    {
+      const float a = scal[0];
+      for (int c0 = half * (DK / 2); c0 < (half + 1) * (DK / 2); c0 += 32) {
+        float r[32];
+        tmem_ld32(tm + lane_off + TM_C + c0, r);
+        tmem_wait_ld();
+        float pk[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const uint32_t u = pack_bf16(r[2 * j], r[2 * j + 1]);
+          pk[j] = __uint_as_float(u);
+        }
+        tmem_st16(tm + lane_off + TM_CB + c0 / 2, pk);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) pk[j] = r[j] * a;
+        tmem_st16(tm + lane_off + TM_C + c0, pk);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) pk[j] = r[16 + j] * a;
+        tmem_st16(tm + lane_off + TM_C + c0 + 16, pk);
       }
       tmem_wait_st();
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    // ---- read-out, intra-chunk and state-update MMAs
+    // ---- read-out + intra-chunk into H, state update into C
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
-      for (int k = 0; k < DK; k += 16) {
-        const uint32_t aoff = (k >> 6) * (DVT * 128) + (k & 63) * 2;
-        const uint32_t boff = (k >> 6) * 8192 + (k & 63) * 2;
-        mma_bf16_ss(tm + TM_I, smem_desc_sw128(smem_u32(Cb) + aoff, 16, 1024),
-                    smem_desc_sw128(smem_u32(Qs) + boff, 16, 1024), id_ro, k > 0 ? 1u : 0u);
-      }
+      for (int k = 0; k < DK; k += 16)
+        mma_bf16_ts(tm + TM_H, tm + TM_CB + k / 2,
+                    smem_desc_sw128(smem_u32(Qs) + (k >> 6) * 8192 + (k & 63) * 2, 16, 1024), id_ro,
+                    k > 0 ? 1u : 0u);
 #pragma unroll
       for (int ks = 0; ks < L / 16; ++ks)
-        mma_bf16_ss(tm + TM_J, smem_desc_sw128(smem_u32(Vs) + ks * 2048, 8192, 1024),
-                    smem_desc_sw128(smem_u32(Ps) + ks * 32, 16, 1024), id_pv, ks > 0 ? 1u : 0u);
+        mma_bf16_ss(tm + TM_H, smem_desc_sw128(smem_u32(Vs) + ks * 2048, 8192, 1024),
+                    smem_desc_sw128(smem_u32(Ps) + ks * 32, 16, 1024), id_pv, 1u);
 #pragma unroll
       for (int ks = 0; ks < L / 16; ++ks)
         mma_bf16_ss(tm + TM_C, smem_desc_sw128(smem_u32(Vw) + ks * 2048, 8192, 1024),
                     smem_desc_sw128(smem_u32(Ks) + ks * 2048, 8192, 1024), id_up, 1u);
       mma_commit(&bar_mma);
     }
-    // ---- normaliser update n <- a n + sum_s w_s k_s (reads K while the MMAs run)
+    // ---- denominators and the normaliser update n <- a n + sum_s w_s k_s
     if (!ret) {
-      const float a = scal[0];
-      for (int col = tid; col < DK; col += NT) {
-        float acc = 0.f;
-        const uint8_t* kt = Ks + (col >> 6) * 8192;
-        for (int s = 0; s < Lc; ++s) acc += wv[s] * bf16_at(kt, s, col & 63);
-        nvec[col] = a * nvec[col] + acc;
+      if (tid < L) {
+        const int t = tid;
+        const float den = fmaxf(fabsf(rs2[t] + rs2[L + t] + sint[t] * nq[t]), expf(-mt[t]));
+        rden[t] = 1.f / den;
       }
+      constexpr int NCG = DK / 8, NRG = NTW / NCG, RPG = L / NRG;
+      const int cg = tid % NCG, rg = tid / NCG;
+      float acc[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+      const int col = 8 * cg;
+      const uint8_t* kt = Ks + (col >> 6) * 8192;
+      for (int s = rg * RPG; s < (rg + 1) * RPG; ++s) {
+        const uint4 u = *reinterpret_cast<const uint4*>(kt + sw128_offset(s, col & 63));
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+        const float w = wv[s];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __bfloat1622float2(b2[j]);
+          acc[2 * j] += w * f.x;
+          acc[2 * j + 1] += w * f.y;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) npart[tid * 8 + j] = acc[j];
+      __syncthreads();
+      const float a = scal[0];
+      for (int c = tid; c < DK; c += NTW) {
+        float x = 0.f;
+        for (int r = 0; r < NRG; ++r) x += npart[(r * NCG + c / 8) * 8 + (c & 7)];
+        nvec[c] = a * nvec[c] + x;
+      }
+    } else if (tid < L) {
+      rden[tid] = 1.f;
     }
     if (!mbar_wait(&bar_mma, it & 1, WAIT)) atomicOr(&abort_flag, 1);
     __syncthreads();
     if (abort_flag) break;
     tc_fence_after();
-    // ---- outputs h_t for this value tile
+    // ---- outputs h_t for this value tile: H^T rows = value rows, columns = tokens
     {
-      const int row = acc_row<DVT>(warp, lane);
+      const int row = acc_row<DVT>(quarter, lane);
       const size_t hcol = (size_t)blk * p.dv + v0 + (row >= 0 ? row : 0);
-      for (int tt = 0; tt < L; tt += 16) {
-        float ri[16], rj[16];
-        tmem_ld16(tm + lane_off + TM_I + tt, ri);
-        tmem_ld16(tm + lane_off + TM_J + tt, rj);
-        tmem_wait_ld();
-        if (row >= 0) {
+      float r[32];
+      tmem_ld32(tm + lane_off + TM_H + half * 32, r);
+      tmem_wait_ld();
+      if (row >= 0) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int t = tt + j;
-            if (t < Lc) {
-              float hv = sint[t] * ri[j] + rj[j];
-              const size_t idx = (tok0 + t) * p.DHV + hcol;
-              if (!ret) {
-                hv = hv / den[t];
-                if (p.og) hv *= __bfloat162float(p.og[idx]);
-              }
-              p.h[idx] = __float2bfloat16_rn(hv);
-            }
+        for (int j = 0; j < 32; ++j) {
+          const int t = half * 32 + j;
+          if (t < Lc) {
+            const size_t idx = (tok0 + t) * p.DHV + hcol;
+            float hv = r[j] * rden[t];
+            if (p.og && !ret) hv *= __bfloat162float(p.og[idx]);
+            p.h[idx] = __float2bfloat16_rn(hv);
           }
         }
       }
@@ -615,29 +723,27 @@ __global__ void __launch_bounds__(NT, 1)
     if (tid == 0) scal[1] = scal[2];
     tc_fence_before();
     __syncthreads();
-    // next chunk's operands
-    if (tid == 0 && t0 + L < T1) issue(t0 + L);
   }
 
   // ---- final state (last segment)
   tc_fence_after();
   if (!abort_flag && last_seg) {
-    const int row = acc_row<DVT>(warp, lane);
+    const int row = acc_row<DVT>(quarter, lane);
     if (p.C_out)
-      for (int c0 = 0; c0 < DK; c0 += 16) {
-        float r[16];
-        tmem_ld16(tm + lane_off + TM_C + c0, r);
+      for (int c0 = half * (DK / 2); c0 < (half + 1) * (DK / 2); c0 += 32) {
+        float r[32];
+        tmem_ld32(tm + lane_off + TM_C + c0, r);
         tmem_wait_ld();
         if (row >= 0) {
           float* dst = p.C_out + ((size_t)slice * p.dv + v0 + row) * p.dk + c0;
 #pragma unroll
-          for (int j = 0; j < 16; j += 4)
+          for (int j = 0; j < 32; j += 4)
             *reinterpret_cast<float4*>(dst + j) = make_float4(r[j], r[j + 1], r[j + 2], r[j + 3]);
         }
       }
     if (!ret && tile == 0) {
       if (p.n_out)
-        for (int col = tid; col < DK; col += NT) p.n_out[(size_t)slice * p.dk + col] = nvec[col];
+        for (int col = tid; col < DK; col += NTW) p.n_out[(size_t)slice * p.dk + col] = nvec[col];
       if (p.m_out && blk == 0 && tid == 0) p.m_out[bh] = scal[1];
     }
   }
@@ -695,7 +801,7 @@ static cudaError_t launch_tc_dk(const TcPlan& pl, const TcParams& prm, const CUt
                                 cudaEvent_t ev1) {
   cudaError_t e;
   if (pl.G > 1) {
-    const int smemA = 2 * DK * 128 + 2 * DVT * 128 + pl.seg_chunks * L * 4 + 1024;
+    const int smemA = 2 * DK * 128 + 2 * DVT * 128 + (NT * 8 + pl.seg_chunks * L) * 4 + 1024;
     e = cudaFuncSetAttribute(tc_segment_kernel<DK, DVT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemA);
     if (e != cudaSuccess) return e;
     dim3 gridA(pl.n_tiles, pl.G - 1, (unsigned)slices);
@@ -708,7 +814,7 @@ static cudaError_t launch_tc_dk(const TcPlan& pl, const TcParams& prm, const CUt
   if (e != cudaSuccess) return e;
   if (ev0) cudaEventRecord(ev0, stream);
   dim3 gridC(pl.n_tiles, pl.G, (unsigned)slices);
-  tc_walk_kernel<DK, DVT><<<gridC, NT, smemC, stream>>>(mq, mk, mv, prm);
+  tc_walk_kernel<DK, DVT><<<gridC, NTW, smemC, stream>>>(mq, mk, mv, prm);
   e = cudaGetLastError();
   if (ev1) cudaEventRecord(ev1, stream);
   return e;
