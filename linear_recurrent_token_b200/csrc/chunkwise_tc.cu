@@ -68,6 +68,27 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+__device__ __forceinline__ void st_shared_b16(uint32_t addr, __nv_bfloat16 v) {
+  asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(*reinterpret_cast<uint16_t*>(&v)) : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 u;
+  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "r"(addr));
+  return u;
+}
+__device__ __forceinline__ void st_shared_v4u(uint32_t addr, uint4 u) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w) : "memory");
+}
+// Scales the 8 bf16 of a 16-byte chunk by w.
+__device__ __forceinline__ uint4 scale_bf16x8(uint4 u, float w) {
+  __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __bfloat1622float2(b2[j]);
+    b2[j] = __floats2bfloat162_rn(f.x * w, f.y * w);
+  }
+  return u;
+}
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
@@ -92,13 +113,13 @@ __global__ void __launch_bounds__(NT, 1)
     tc_segment_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV, TcParams p) {
   constexpr int KB = DK * 128;   // bytes of one K chunk tile (DK/64 boxes of 8 KiB)
   constexpr int VB = DVT * 128;  // bytes of one V chunk tile
+  constexpr int NS = 3;          // TMA stages
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* Ks[2] = {sm, sm + KB};
-  uint8_t* Vs[2] = {sm + 2 * KB, sm + 2 * KB + VB};
-  float* dnp = reinterpret_cast<float*>(sm + 2 * KB + 2 * VB);  // [NT * 8] partial sums of dn
-  float* omega = dnp + NT * 8;                                   // [seg_chunks * L]
-  __shared__ uint64_t bar_load[2], bar_mma[2];
+  // stage i: K at sm + i*(KB+VB), V right after it
+  float* dnp = reinterpret_cast<float*>(sm + NS * (KB + VB));  // [NT * 8] partial sums of dn
+  float* omega = dnp + NT * 8;                                  // [seg_chunks * L]
+  __shared__ uint64_t bar_load[NS], bar_mma[NS];
   __shared__ uint32_t tmem_base;
   __shared__ float red[NT / 32];
   __shared__ int abort_flag;
@@ -115,10 +136,10 @@ __global__ void __launch_bounds__(NT, 1)
   const bool do_dn = !p.retention && dn0 < DK;
 
   if (tid == 0) {
-    mbar_init(&bar_load[0], 1);
-    mbar_init(&bar_load[1], 1);
-    mbar_init(&bar_mma[0], 1);
-    mbar_init(&bar_mma[1], 1);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&bar_load[i], 1);
+      mbar_init(&bar_mma[i], 1);
+    }
     abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&mapK);
@@ -131,17 +152,16 @@ __global__ void __launch_bounds__(NT, 1)
 
   const int nck = p.seg_chunks;
   auto issue = [&](int c) {
-    const int st = c & 1;
+    const int st = c % NS;
+    uint8_t* kb = sm + st * (KB + VB);
     mbar_arrive_expect_tx(&bar_load[st], KB + VB);
     for (int j = 0; j < DK / 64; ++j)
-      tma_load_3d(Ks[st] + j * 8192, &mapK, blk * p.dk + 64 * j, T0 + c * L, bh, &bar_load[st]);
+      tma_load_3d(kb + j * 8192, &mapK, blk * p.dk + 64 * j, T0 + c * L, bh, &bar_load[st]);
     for (int j = 0; j < DVT / 64; ++j)
-      tma_load_3d(Vs[st] + j * 8192, &mapV, blk * p.dv + v0 + 64 * j, T0 + c * L, bh, &bar_load[st]);
+      tma_load_3d(kb + KB + j * 8192, &mapV, blk * p.dv + v0 + 64 * j, T0 + c * L, bh, &bar_load[st]);
   };
-  if (tid == 0) {
-    issue(0);
-    if (nck > 1) issue(1);
-  }
+  if (tid == 0)
+    for (int c = 0; c < NS - 1 && c < nck; ++c) issue(c);
 
   // ---- gates: G_s (inclusive cumulative log f), Gtot, M, omega_s
   const size_t tok0 = (size_t)bh * p.S + T0;
@@ -199,14 +219,16 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
   for (int j = 0; j < 8; ++j) dacc[j] = 0.f;
   for (int c = 0; c < nck; ++c) {
-    const int st = c & 1;
-    if (!abort_flag && !mbar_wait(&bar_load[st], (c >> 1) & 1, WAIT)) atomicOr(&abort_flag, 1);
+    const int st = c % NS;
+    uint8_t* Kst = sm + st * (KB + VB);
+    uint8_t* Vst = Kst + KB;
+    if (!abort_flag && !mbar_wait(&bar_load[st], (c / NS) & 1, WAIT)) atomicOr(&abort_flag, 1);
     __syncthreads();
     if (abort_flag) break;
     const float* om = omega + c * L;
     for (int i = tid; i < L * (DVT / 8); i += NT) {
       const int row = i / (DVT / 8), ch = i % (DVT / 8);
-      uint8_t* ptr = Vs[st] + (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
+      uint8_t* ptr = Vst + (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
       uint4 u = *reinterpret_cast<uint4*>(ptr);
       __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&u);
       const float w = om[row];
@@ -218,7 +240,7 @@ __global__ void __launch_bounds__(NT, 1)
       *reinterpret_cast<uint4*>(ptr) = u;
     }
     if (do_dn && rg < nrg && dcol < DK) {
-      const uint8_t* kt = Ks[st] + (dcol >> 6) * 8192;
+      const uint8_t* kt = Kst + (dcol >> 6) * 8192;
       for (int s = rg * rows_per; s < min(L, (rg + 1) * rows_per); ++s) {
         const uint4 u = *reinterpret_cast<const uint4*>(kt + sw128_offset(s, dcol & 63));
         const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
@@ -235,22 +257,23 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
     if (tid == 0) {
       tc_fence_after();
+      const uint32_t va = smem_u32(Vst), ka = smem_u32(Kst);
 #pragma unroll
-      for (int ks = 0; ks < L / 16; ++ks) {
-        const uint64_t ad = smem_desc_sw128(smem_u32(Vs[st]) + ks * 2048, 8192, 1024);
-        const uint64_t bd = smem_desc_sw128(smem_u32(Ks[st]) + ks * 2048, 8192, 1024);
-        mma_bf16_ss(tm, ad, bd, idesc, (c > 0 || ks > 0) ? 1u : 0u);
-      }
+      for (int ks = 0; ks < L / 16; ++ks)
+        mma_bf16_ss(tm, smem_desc_sw128(va + ks * 2048, 8192, 1024), smem_desc_sw128(ka + ks * 2048, 8192, 1024),
+                    idesc, (c > 0 || ks > 0) ? 1u : 0u);
       mma_commit(&bar_mma[st]);
-    }
-    // stage st is reloaded with chunk c+2 once this chunk's MMAs have read it
-    if (c + 2 < nck) {
-      if (!abort_flag && !mbar_wait(&bar_mma[st], (c >> 1) & 1, WAIT)) atomicOr(&abort_flag, 1);
-      __syncthreads();
-      if (tid == 0 && !abort_flag) issue(c + 2);
+      // stage (c + NS - 1) % NS was last read by the MMAs of chunk c - 1 (queued before
+      // this chunk's): refill it once they are done; the other threads move on
+      if (c + NS - 1 < nck) {
+        if (c >= 1 && !mbar_wait(&bar_mma[(c - 1) % NS], ((c - 1) / NS) & 1, WAIT))
+          atomicOr(&abort_flag, 1);
+        else
+          issue(c + NS - 1);
+      }
     }
   }
-  if (!abort_flag && !mbar_wait(&bar_mma[(nck - 1) & 1], ((nck - 1) >> 1) & 1, WAIT)) atomicOr(&abort_flag, 1);
+  if (!abort_flag && !mbar_wait(&bar_mma[(nck - 1) % NS], ((nck - 1) / NS) & 1, WAIT)) atomicOr(&abort_flag, 1);
   __syncthreads();
   tc_fence_after();
   if (!abort_flag) {
@@ -284,48 +307,72 @@ __global__ void __launch_bounds__(NT, 1)
 }
 
 // ===================================================================== phase C
-constexpr int NTW = 256;  // walk kernel: 8 warps; warps w and w+4 share TMEM lane quarter w%4
+// Warp-specialised walk: 10 warps.
+//   warps 0-3  state group: C round trip (bf16 copy into TMEM, C <- a C), n . q_t, n update
+//   warps 4-7  output group: V o w, P = S o D', Q scaling, denominators, h (TMA store)
+//   warp 8     MMA issue (one elected lane, fully unrolled, descriptors from constants)
+//   warp 9     producer: TMA loads of Q/K/V (two stages) and the per-chunk gate scan
+// Hand-offs are mbarriers; every wait is bounded, and a group decides to abort as one.
+constexpr int NTW = 320;
+constexpr int WG_STATE = 1, WG_OUT = 2;  // named barrier ids of the two 128-thread groups
 
 template <int DK, int DVT>
 struct WalkSmem {
-  static constexpr int QB = DK * 128, KB = DK * 128, VB = DVT * 128, PB = 64 * 128;
+  static constexpr int QB = DK * 128, KB = DK * 128, VB = DVT * 128, PB = 64 * 128, HB = DVT * 128;
   static constexpr int STAGE = QB + KB + VB;
-  static constexpr int OS0 = 0, OS1 = STAGE, OVW = 2 * STAGE, OP = OVW + VB;
-  static constexpr int OF = OP + PB;                                  // floats start here
-  static constexpr int NF = DK + NTW * 8 + 10 * L + 16;               // n, n partials, per-token, scalars
-  static constexpr int BYTES = OF + NF * 4 + 1024;                    // + alignment slack
+  static constexpr int OVW = 2 * STAGE, OP = OVW + VB, OH = OP + PB;
+  static constexpr int OF = OH + HB;  // floats start here
+  // n [DK], n partials [128*8], gate buffers [2][6][L], nq / rden / row sums [3][L], gate scalars [2][4]
+  static constexpr int NF = DK + 128 * 8 + 2 * 6 * L + 3 * L + 8;
+  static constexpr int BYTES = OF + NF * 4 + 1024;  // + alignment slack
+};
+
+// Per-chunk gate quantities (double-buffered).  b: inclusive cumulative log f; m: stabiliser
+// per token; sint = e^{b_t+m_c-m_t}; w = e^{g-b_s+itilde_s-m_next}; cs = (itilde_s - b_s) log2 e.
+struct GateBuf {
+  float* bl;
+  float* li;
+  float* mt;
+  float* sint;
+  float* wv;
+  float* cs;
+  float* scal;  // [0] decay a, [1] m_c, [2] m_next
+};
+
+struct WalkBars {
+  uint64_t full[2], empty[2], gfull[2], gempty[2];
+  uint64_t s_full, s_empty, e1_done, vw_full, pq_full, h_empty, mm_done, nq_done;
 };
 
 template <int DK, int DVT>
 __global__ void __launch_bounds__(NTW, 1)
     tc_walk_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
-                   const __grid_constant__ CUtensorMap mapV, TcParams p) {
+                   const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapH, TcParams p) {
   using SM = WalkSmem<DK, DVT>;
   // TMEM columns: C fp32 [DK], bf16 copy of C as MMA operand [DK/2], S [64], H [64]
   constexpr uint32_t TM_C = 0, TM_CB = DK, TM_S = DK + DK / 2, TM_H = TM_S + 64;
   constexpr uint32_t TM_COLS = (TM_H + 64 <= 256) ? 256 : 512;
+  constexpr float LOG2E = 1.4426950408889634f;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* stage_base[2] = {sm + SM::OS0, sm + SM::OS1};
-  uint8_t *Vw = sm + SM::OVW, *Ps = sm + SM::OP;
+  uint8_t *Vw = sm + SM::OVW, *Ps = sm + SM::OP, *Hs = sm + SM::OH;
   float* nvec = reinterpret_cast<float*>(sm + SM::OF);
-  float* npart = nvec + DK;  // [NTW * 8]
-  float* bl = npart + NTW * 8;
-  float* li = bl + L;
-  float* mt = li + L;
-  float* sint = mt + L;
-  float* wv = sint + L;
-  float* rden = wv + L;
-  float* nq = rden + L;
-  float* rs2 = nq + L;       // [2][L] row-sum halves
-  float* cs = rs2 + 2 * L;   // li - bl (per column s of P)
-  float* scal = cs + L;      // [0] decay a, [1] m_c, [2] m_next
-  __shared__ uint64_t bar_load[2], bar_s, bar_mma;
+  float* npart = nvec + DK;  // [128 * 8]
+  float* gmem = npart + 128 * 8;
+  float* nq = gmem + 2 * 6 * L;
+  float* rden = nq + L;
+  float* rsum = rden + L;
+  float* gscal = rsum + L;  // [2][4]
+  auto gbuf = [&](int b) {
+    float* base = gmem + b * 6 * L;
+    return GateBuf{base, base + L, base + 2 * L, base + 3 * L, base + 4 * L, base + 5 * L, gscal + 4 * b};
+  };
+  __shared__ WalkBars bars;
   __shared__ uint32_t tmem_base;
-  __shared__ int abort_flag;
+  __shared__ volatile int abort_flag;
+  __shared__ volatile int group_flag[2];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int quarter = warp & 3, half = warp >> 2;
   const int tile = blockIdx.x, g = blockIdx.y, slice = blockIdx.z;
   const int blk = slice % p.nb, bh = slice / p.nb, head = bh % p.NH;
   const int v0 = tile * DVT;
@@ -334,55 +381,37 @@ __global__ void __launch_bounds__(NTW, 1)
   const int nck = (T1 - T0 + L - 1) / L;
   const bool ret = p.retention != 0;
   const bool last_seg = g == p.G - 1;
-  const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+  const uint32_t sm_u = smem_u32(sm);
 
   if (tid == 0) {
-    mbar_init(&bar_load[0], 1);
-    mbar_init(&bar_load[1], 1);
-    mbar_init(&bar_s, 1);
-    mbar_init(&bar_mma, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.full[i], 1);
+      mbar_init(&bars.empty[i], 3);
+      mbar_init(&bars.gfull[i], 1);
+      mbar_init(&bars.gempty[i], 2);
+    }
+    mbar_init(&bars.s_full, 1);
+    mbar_init(&bars.s_empty, 1);
+    mbar_init(&bars.e1_done, 1);
+    mbar_init(&bars.vw_full, 1);
+    mbar_init(&bars.pq_full, 1);
+    mbar_init(&bars.h_empty, 1);
+    mbar_init(&bars.mm_done, 1);
+    mbar_init(&bars.nq_done, 1);
     abort_flag = 0;
+    group_flag[0] = group_flag[1] = 0;
     fence_mbar_init();
     prefetch_tensormap(&mapQ);
     prefetch_tensormap(&mapK);
     prefetch_tensormap(&mapV);
+    prefetch_tensormap(&mapH);
   }
   if (warp == 0) tmem_alloc(&tmem_base, TM_COLS);
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = tmem_base;
 
-  auto issue = [&](int c) {
-    const int st = c & 1;
-    uint8_t* base = stage_base[st];
-    const int t0 = T0 + c * L;
-    mbar_arrive_expect_tx(&bar_load[st], SM::STAGE);
-    for (int j = 0; j < DK / 64; ++j) {
-      tma_load_3d(base + j * 8192, &mapQ, blk * p.dk + 64 * j, t0, bh, &bar_load[st]);
-      tma_load_3d(base + SM::QB + j * 8192, &mapK, blk * p.dk + 64 * j, t0, bh, &bar_load[st]);
-    }
-    for (int j = 0; j < DVT / 64; ++j)
-      tma_load_3d(base + SM::QB + SM::KB + j * 8192, &mapV, blk * p.dv + v0 + 64 * j, t0, bh, &bar_load[st]);
-  };
-  if (tid == 0) issue(0);
-
-  // raw gates of the next chunk, held by warp 0 (two tokens per lane)
-  float rfa = 0.f, ria = 0.f, rfb = 0.f, rib = 0.f;
-  auto fetch_gates = [&](int c) {
-    const int t0 = T0 + c * L;
-    const int Lc = min(L, T1 - t0);
-    const size_t tok = (size_t)bh * p.S + t0;
-    const int ta = 2 * lane, tb = 2 * lane + 1;
-    if (!ret) {
-      rfa = ta < Lc ? p.fg[tok + ta] : 0.f;
-      ria = ta < Lc ? p.ig[tok + ta] : 0.f;
-      rfb = tb < Lc ? p.fg[tok + tb] : 0.f;
-      rib = tb < Lc ? p.ig[tok + tb] : 0.f;
-    }
-  };
-  if (warp == 0) fetch_gates(0);
-
-  // ---- start state of the segment (see the file header)
+  // ---- start state of the segment (see the file header); warps 0-7 fill TMEM and n
   float m_start = ret ? 0.f : (p.m0 ? p.m0[bh] : 0.f);
   const float m_init = m_start;
   float gsum = 0.f;
@@ -391,7 +420,9 @@ __global__ void __launch_bounds__(NTW, 1)
     if (!ret) m_start = fmaxf(A + m_start, Bm);
     gsum += A;
   }
-  {
+  if (warp < 8) {
+    const int quarter = warp & 3, half = warp >> 2;
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     const int row = acc_row<DVT>(quarter, lane);
     const float wc0 = expf(gsum + m_init - m_start);
     for (int c0 = half * (DK / 2); c0 < (half + 1) * (DK / 2); c0 += 16) {
@@ -430,7 +461,7 @@ __global__ void __launch_bounds__(NTW, 1)
     }
     tmem_wait_st();
     if (!ret)
-      for (int col = tid; col < DK; col += NTW) {
+      for (int col = tid; col < DK; col += 256) {
         float x = p.n0 ? wc0 * p.n0[(size_t)slice * p.dk + col] : 0.f;
         float after = gsum;
         for (int jg = 0; jg < g; ++jg) {
@@ -441,31 +472,67 @@ __global__ void __launch_bounds__(NTW, 1)
         nvec[col] = x;
       }
   }
-  if (tid == 0) scal[1] = m_start;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
 
-  const uint32_t id_s = idesc_bf16(64, 64, 0, 0);
-  const uint32_t id_ro = idesc_bf16(DVT, 64, 0, 0);
-  const uint32_t id_pv = idesc_bf16(DVT, 64, 1, 0);
-  const uint32_t id_up = idesc_bf16(DVT, DK, 1, 1);
-  const float lg = ret ? retention_log_gamma(head) : 0.f;
-  constexpr float LOG2E = 1.4426950408889634f;
+  // group-uniform bounded wait: the group's first thread waits, the group follows its verdict
+  auto group_wait = [&](uint64_t* bar, uint32_t parity, int gi, bool first) -> bool {
+    if (first && (abort_flag || !mbar_wait(bar, parity, WAIT))) {
+      group_flag[gi] = 1;
+      abort_flag = 1;
+    }
+    named_bar(gi == 0 ? WG_STATE : WG_OUT, 128);
+    return group_flag[gi] == 0;
+  };
+  // warp-uniform bounded wait (one lane waits)
+  auto warp_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    int ok = 1;
+    if (lane == 0 && (abort_flag || !mbar_wait(bar, parity, WAIT))) {
+      ok = 0;
+      abort_flag = 1;
+    }
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+  };
 
-  for (int it = 0; it < nck; ++it) {
-    const int st = it & 1;
-    const int t0 = T0 + it * L;
-    const int Lc = min(L, T1 - t0);
-    const size_t tok0 = (size_t)bh * p.S + t0;
-    uint8_t* Qs = stage_base[st];
-    uint8_t* Ks = Qs + SM::QB;
-    uint8_t* Vs = Ks + SM::KB;
-    // the other stage was released at the end of the previous chunk: prefetch chunk it+1
-    if (tid == 0 && it + 1 < nck && !abort_flag) issue(it + 1);
-    // ---- per-token gate quantities (warp 0): b (cumulative log f), m_t, scales
-    if (warp == 0) {
-      const float mc = scal[1];
+  if (warp == 9) {
+    // =============================================================== producer
+    const float lg = ret ? retention_log_gamma(head) : 0.f;
+    float rfa = 0.f, ria = 0.f, rfb = 0.f, rib = 0.f;
+    auto fetch_gates = [&](int c) {
+      const int t0 = T0 + c * L;
+      const int Lc = min(L, T1 - t0);
+      const size_t tok = (size_t)bh * p.S + t0;
+      const int ta = 2 * lane, tb = 2 * lane + 1;
+      if (!ret) {
+        rfa = ta < Lc ? p.fg[tok + ta] : 0.f;
+        ria = ta < Lc ? p.ig[tok + ta] : 0.f;
+        rfb = tb < Lc ? p.fg[tok + tb] : 0.f;
+        rib = tb < Lc ? p.ig[tok + tb] : 0.f;
+      }
+    };
+    fetch_gates(0);
+    float mc = m_start;
+    for (int c = 0; c < nck; ++c) {
+      const int b = c & 1;
+      // operands of chunk c into stage b once its previous user (chunk c-2) released it
+      if (!warp_wait(&bars.empty[b], ((c >> 1) & 1) ^ 1)) break;
+      if (lane == 0) {
+        uint8_t* base = sm + b * SM::STAGE;
+        const int t0 = T0 + c * L;
+        mbar_arrive_expect_tx(&bars.full[b], SM::STAGE);
+        for (int j = 0; j < DK / 64; ++j) {
+          tma_load_3d(base + j * 8192, &mapQ, blk * p.dk + 64 * j, t0, bh, &bars.full[b]);
+          tma_load_3d(base + SM::QB + j * 8192, &mapK, blk * p.dk + 64 * j, t0, bh, &bars.full[b]);
+        }
+        for (int j = 0; j < DVT / 64; ++j)
+          tma_load_3d(base + SM::QB + SM::KB + j * 8192, &mapV, blk * p.dv + v0 + 64 * j, t0, bh, &bars.full[b]);
+      }
+      // gate quantities of chunk c into buffer b
+      if (!warp_wait(&bars.gempty[b], ((c >> 1) & 1) ^ 1)) break;
+      GateBuf G = gbuf(b);
+      const int t0 = T0 + c * L;
+      const int Lc = min(L, T1 - t0);
       const int ta = 2 * lane, tb = 2 * lane + 1;
       float lfa, lia, lfb, lib;
       if (ret) {
@@ -477,7 +544,7 @@ __global__ void __launch_bounds__(NTW, 1)
         lfb = tb < Lc ? log_sigmoid(rfb) : 0.f;
         lib = tb < Lc ? rib : -INFINITY;
       }
-      if (it + 1 < nck) fetch_gates(it + 1);
+      if (c + 1 < nck) fetch_gates(c + 1);
       float isum = lfa + lfb;
       MaxPlus imp = mp_then(MaxPlus{lfa, lia}, MaxPlus{lfb, lib});
 #pragma unroll
@@ -502,251 +569,364 @@ __global__ void __launch_bounds__(NTW, 1)
         ma = mp_apply(pa, mc);
         mb = mp_apply(mp_then(pa, MaxPlus{lfb, lib}), mc);
       }
-      bl[ta] = ba;
-      bl[tb] = bb;
-      li[ta] = ret ? 0.f : lia;
-      li[tb] = ret ? 0.f : lib;
-      mt[ta] = ma;
-      mt[tb] = mb;
-      __syncwarp();
-      const float gtot = bl[Lc - 1];
-      const float mn = mt[Lc - 1];
-      sint[ta] = expf(ba + mc - ma);
-      sint[tb] = expf(bb + mc - mb);
-      wv[ta] = ta < Lc ? expf(gtot - ba + li[ta] - mn) : 0.f;
-      wv[tb] = tb < Lc ? expf(gtot - bb + li[tb] - mn) : 0.f;
-      cs[ta] = ta < Lc ? (li[ta] - ba) * LOG2E : -INFINITY;
-      cs[tb] = tb < Lc ? (li[tb] - bb) * LOG2E : -INFINITY;
+      const float lia_ = ret ? 0.f : lia, lib_ = ret ? 0.f : lib;
+      const int lt = (Lc - 1) >> 1;
+      const float gtot = __shfl_sync(0xffffffffu, ((Lc - 1) & 1) ? bb : ba, lt);
+      const float mn = __shfl_sync(0xffffffffu, ((Lc - 1) & 1) ? mb : ma, lt);
+      G.bl[ta] = ba;
+      G.bl[tb] = bb;
+      G.li[ta] = lia_;
+      G.li[tb] = lib_;
+      G.mt[ta] = ma;
+      G.mt[tb] = mb;
+      G.sint[ta] = expf(ba + mc - ma);
+      G.sint[tb] = expf(bb + mc - mb);
+      G.wv[ta] = ta < Lc ? expf(gtot - ba + lia_ - mn) : 0.f;
+      G.wv[tb] = tb < Lc ? expf(gtot - bb + lib_ - mn) : 0.f;
+      G.cs[ta] = ta < Lc ? (lia_ - ba) * LOG2E : -INFINITY;
+      G.cs[tb] = tb < Lc ? (lib_ - bb) * LOG2E : -INFINITY;
       if (lane == 0) {
-        scal[0] = expf(gtot + mc - mn);
-        scal[2] = mn;
+        G.scal[0] = expf(gtot + mc - mn);
+        G.scal[1] = mc;
+        G.scal[2] = mn;
       }
+      mc = mn;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.gfull[b]);
     }
-    if (!abort_flag && !mbar_wait(&bar_load[st], (it >> 1) & 1, WAIT)) atomicOr(&abort_flag, 1);
-    __syncthreads();
-    if (abort_flag) break;
-    // ---- S = Q K^T
-    if (tid == 0) {
+    if (lane == 0 && !abort_flag && last_seg && !ret && tile == 0 && blk == 0 && p.m_out) p.m_out[bh] = mc;
+  } else if (warp == 8) {
+    // =============================================================== MMA issue
+    const uint32_t id_s = idesc_bf16(64, 64, 0, 0);
+    const uint32_t id_ro = idesc_bf16(DVT, 64, 0, 0);
+    const uint32_t id_pv = idesc_bf16(DVT, 64, 1, 0);
+    const uint32_t id_up = idesc_bf16(DVT, DK, 1, 1);
+    const uint64_t ps_k = smem_desc_sw128(sm_u + SM::OP, 16, 1024);       // P, K-major rows t
+    const uint64_t vw_mn = smem_desc_sw128(sm_u + SM::OVW, 8192, 1024);  // V o w, MN-major
+    for (int c = 0; c < nck; ++c) {
+      const int b = c & 1;
+      const uint32_t q_u = sm_u + b * SM::STAGE, k_u = q_u + SM::QB, v_u = k_u + SM::KB;
+      const uint64_t q_k = smem_desc_sw128(q_u, 16, 1024);     // Q (or scaled Q), K-major rows t
+      const uint64_t k_k = smem_desc_sw128(k_u, 16, 1024);     // K, K-major rows s
+      const uint64_t k_mn = smem_desc_sw128(k_u, 8192, 1024);  // K, MN-major (rows s = K dim)
+      const uint64_t v_mn = smem_desc_sw128(v_u, 8192, 1024);  // V, MN-major
+      if (!warp_wait(&bars.full[b], (c >> 1) & 1)) break;
+      if (c > 0 && !warp_wait(&bars.s_empty, (c - 1) & 1)) break;
       tc_fence_after();
+      if (elect_one()) {
 #pragma unroll
-      for (int k = 0; k < DK; k += 16) {
-        const uint32_t off = (k >> 6) * 8192 + (k & 63) * 2;
-        mma_bf16_ss(tm + TM_S, smem_desc_sw128(smem_u32(Qs) + off, 16, 1024),
-                    smem_desc_sw128(smem_u32(Ks) + off, 16, 1024), id_s, k > 0 ? 1u : 0u);
-      }
-      mma_commit(&bar_s);
-    }
-    // ---- n . q_t (four threads per token) and V o w
-    if (!ret) {
-      const int t = tid >> 2, part = tid & 3;
-      float a = 0.f;
-      for (int col = part * (DK / 4); col < (part + 1) * (DK / 4); col += 8) {
-        const uint4 u = *reinterpret_cast<const uint4*>(Qs + (col >> 6) * 8192 + sw128_offset(t, col & 63));
-        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-        const float4 n0 = *reinterpret_cast<const float4*>(nvec + col);
-        const float4 n1 = *reinterpret_cast<const float4*>(nvec + col + 4);
-        float2 f = __bfloat1622float2(b2[0]);
-        a += f.x * n0.x + f.y * n0.y;
-        f = __bfloat1622float2(b2[1]);
-        a += f.x * n0.z + f.y * n0.w;
-        f = __bfloat1622float2(b2[2]);
-        a += f.x * n1.x + f.y * n1.y;
-        f = __bfloat1622float2(b2[3]);
-        a += f.x * n1.z + f.y * n1.w;
-      }
-      a += __shfl_xor_sync(0xffffffffu, a, 1);
-      a += __shfl_xor_sync(0xffffffffu, a, 2);
-      if (part == 0) nq[t] = a;
-    }
-    for (int i = tid; i < L * (DVT / 8); i += NTW) {
-      const int row = i / (DVT / 8), ch = i % (DVT / 8);
-      const int off = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
-      uint4 u = *reinterpret_cast<const uint4*>(Vs + off);
-      __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&u);
-      const float w = wv[row];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = __bfloat1622float2(b2[j]);
-        b2[j] = __floats2bfloat162_rn(f.x * w, f.y * w);
-      }
-      *reinterpret_cast<uint4*>(Vw + off) = u;
-    }
-    if (!mbar_wait(&bar_s, it & 1, WAIT)) atomicOr(&abort_flag, 1);
-    __syncthreads();
-    if (abort_flag) break;
-    tc_fence_after();
-    // ---- P = S o D' (bf16, rows t), half the columns per warp half; row-sum halves
-    {
-      const int t = acc_row<64>(quarter, lane);
-      float r[32];
-      tmem_ld32(tm + lane_off + TM_S + half * 32, r);
-      tmem_wait_ld();
-      if (t >= 0) {
-        const float ct = (bl[t] - mt[t]) * LOG2E;
-        float rs = 0.f;
-        uint32_t pk[16];
-#pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const int s = half * 32 + j;
-          const float e0 = (s <= t && t < Lc) ? r[j] * exp2f(ct + cs[s]) : 0.f;
-          const float e1 = (s + 1 <= t && t < Lc) ? r[j + 1] * exp2f(ct + cs[s + 1]) : 0.f;
-          rs += e0 + e1;
-          pk[j / 2] = pack_bf16(e0, e1);
+        for (int k = 0; k < DK; k += 16) {
+          const uint64_t off = (uint64_t)(((k >> 6) * 8192 + (k & 63) * 2) >> 4);
+          mma_bf16_ss(tm + TM_S, q_k + off, k_k + off, id_s, k > 0 ? 1u : 0u);
         }
-        const uint32_t base = smem_u32(Ps);
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-          st_shared_v4(base + sw128_offset(t, half * 32 + 8 * q4), pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2],
-                       pk[4 * q4 + 3]);
-        rs2[half * L + t] = rs;
+        mma_commit(&bars.s_full);
       }
-    }
-    // ---- Q <- e^{b_t+m_c-m_t} Q (the inter-chunk read-out then shares the accumulator)
-    for (int i = tid; i < L * (DK / 8); i += NTW) {
-      const int row = i / (DK / 8), ch = i % (DK / 8);
-      const int off = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
-      uint4 u = *reinterpret_cast<const uint4*>(Qs + off);
-      __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&u);
-      const float w = sint[row];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = __bfloat1622float2(b2[j]);
-        b2[j] = __floats2bfloat162_rn(f.x * w, f.y * w);
-      }
-      *reinterpret_cast<uint4*>(Qs + off) = u;
-    }
-    // ---- C round trip: bf16 copy of C_c into TMEM (MMA operand), C <- a C
-    {
-      const float a = scal[0];
-      for (int c0 = half * (DK / 2); c0 < (half + 1) * (DK / 2); c0 += 32) {
-        float r[32];
-        tmem_ld32(tm + lane_off + TM_C + c0, r);
-        tmem_wait_ld();
-        float pk[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const uint32_t u = pack_bf16(r[2 * j], r[2 * j + 1]);
-          pk[j] = __uint_as_float(u);
-        }
-        tmem_st16(tm + lane_off + TM_CB + c0 / 2, pk);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) pk[j] = r[j] * a;
-        tmem_st16(tm + lane_off + TM_C + c0, pk);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) pk[j] = r[16 + j] * a;
-        tmem_st16(tm + lane_off + TM_C + c0 + 16, pk);
-      }
-      tmem_wait_st();
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    // ---- read-out + intra-chunk into H, state update into C
-    if (tid == 0) {
+      __syncwarp();
+      if (!warp_wait(&bars.e1_done, c & 1)) break;
+      if (!warp_wait(&bars.vw_full, c & 1)) break;
       tc_fence_after();
+      if (elect_one()) {
 #pragma unroll
-      for (int k = 0; k < DK; k += 16)
-        mma_bf16_ts(tm + TM_H, tm + TM_CB + k / 2,
-                    smem_desc_sw128(smem_u32(Qs) + (k >> 6) * 8192 + (k & 63) * 2, 16, 1024), id_ro,
-                    k > 0 ? 1u : 0u);
-#pragma unroll
-      for (int ks = 0; ks < L / 16; ++ks)
-        mma_bf16_ss(tm + TM_H, smem_desc_sw128(smem_u32(Vs) + ks * 2048, 8192, 1024),
-                    smem_desc_sw128(smem_u32(Ps) + ks * 32, 16, 1024), id_pv, 1u);
-#pragma unroll
-      for (int ks = 0; ks < L / 16; ++ks)
-        mma_bf16_ss(tm + TM_C, smem_desc_sw128(smem_u32(Vw) + ks * 2048, 8192, 1024),
-                    smem_desc_sw128(smem_u32(Ks) + ks * 2048, 8192, 1024), id_up, 1u);
-      mma_commit(&bar_mma);
-    }
-    // ---- denominators and the normaliser update n <- a n + sum_s w_s k_s
-    if (!ret) {
-      if (tid < L) {
-        const int t = tid;
-        const float den = fmaxf(fabsf(rs2[t] + rs2[L + t] + sint[t] * nq[t]), expf(-mt[t]));
-        rden[t] = 1.f / den;
+        for (int ks = 0; ks < L / 16; ++ks)
+          mma_bf16_ss(tm + TM_C, vw_mn + (uint64_t)(ks * 128), k_mn + (uint64_t)(ks * 128), id_up, 1u);
       }
-      constexpr int NCG = DK / 8, NRG = NTW / NCG, RPG = L / NRG;
-      const int cg = tid % NCG, rg = tid / NCG;
-      float acc[8];
+      __syncwarp();
+      if (!warp_wait(&bars.pq_full, c & 1)) break;
+      if (c > 0 && !warp_wait(&bars.h_empty, (c - 1) & 1)) break;
+      tc_fence_after();
+      if (elect_one()) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-      const int col = 8 * cg;
-      const uint8_t* kt = Ks + (col >> 6) * 8192;
-      for (int s = rg * RPG; s < (rg + 1) * RPG; ++s) {
-        const uint4 u = *reinterpret_cast<const uint4*>(kt + sw128_offset(s, col & 63));
-        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-        const float w = wv[s];
+        for (int k = 0; k < DK; k += 16)
+          mma_bf16_ts(tm + TM_H, tm + TM_CB + k / 2, q_k + (uint64_t)(((k >> 6) * 8192 + (k & 63) * 2) >> 4), id_ro,
+                      k > 0 ? 1u : 0u);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float2 f = __bfloat1622float2(b2[j]);
-          acc[2 * j] += w * f.x;
-          acc[2 * j + 1] += w * f.y;
+        for (int ks = 0; ks < L / 16; ++ks)
+          mma_bf16_ss(tm + TM_H, v_mn + (uint64_t)(ks * 128), ps_k + (uint64_t)(ks * 2), id_pv, 1u);
+        mma_commit(&bars.mm_done);
+        mma_commit(&bars.empty[b]);
+      }
+      __syncwarp();
+    }
+  } else if (warp < 4) {
+    // =============================================================== state group
+    const int quarter = warp;
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+    const bool first = tid == 0;
+    for (int c = 0; c < nck; ++c) {
+      const int b = c & 1;
+      const GateBuf G = gbuf(b);
+      uint8_t* Qs = sm + b * SM::STAGE;
+      uint8_t* Ks = Qs + SM::QB;
+      if (!group_wait(&bars.gfull[b], (c >> 1) & 1, 0, first)) break;
+      if (c > 0 && !group_wait(&bars.mm_done, (c - 1) & 1, 0, first)) break;
+      tc_fence_after();
+      // C round trip: bf16 copy of C_c into TMEM (read-out operand), C <- a C
+      {
+        const float a = G.scal[0];
+        for (int c0 = 0; c0 < DK; c0 += 32) {
+          float r[32];
+          tmem_ld32(tm + lane_off + TM_C + c0, r);
+          tmem_wait_ld();
+          float pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) pk[j] = __uint_as_float(pack_bf16(r[2 * j], r[2 * j + 1]));
+          tmem_st16(tm + lane_off + TM_CB + c0 / 2, pk);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) pk[j] = r[j] * a;
+          tmem_st16(tm + lane_off + TM_C + c0, pk);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) pk[j] = r[16 + j] * a;
+          tmem_st16(tm + lane_off + TM_C + c0 + 16, pk);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      named_bar(WG_STATE, 128);
+      if (first) mbar_arrive(&bars.e1_done);
+      if (!group_wait(&bars.full[b], (c >> 1) & 1, 0, first)) break;
+      if (!ret) {
+        // n . q_t: two threads per token, DK/2 columns each (loads batched)
+        const int t = tid >> 1, part = tid & 1;
+        const uint32_t qs_u = smem_u32(Qs);
+        constexpr int NCH = DK / 16;
+        constexpr int BATCH = NCH < 8 ? NCH : 8;
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int j0 = 0; j0 < NCH; j0 += BATCH) {
+          uint4 u[BATCH];
+#pragma unroll
+          for (int j = 0; j < BATCH; ++j) {
+            const int col = part * (DK / 2) + 8 * (j0 + j);
+            u[j] = ld_shared_v4(qs_u + (col >> 6) * 8192 + sw128_offset(t, col & 63));
+          }
+#pragma unroll
+          for (int j = 0; j < BATCH; ++j) {
+            const int col = part * (DK / 2) + 8 * (j0 + j);
+            const float4 n0 = *reinterpret_cast<const float4*>(nvec + col);
+            const float4 n1 = *reinterpret_cast<const float4*>(nvec + col + 4);
+            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u[j]);
+            float2 f = __bfloat1622float2(b2[0]);
+            a0 += f.x * n0.x + f.y * n0.y;
+            f = __bfloat1622float2(b2[1]);
+            a1 += f.x * n0.z + f.y * n0.w;
+            f = __bfloat1622float2(b2[2]);
+            a0 += f.x * n1.x + f.y * n1.y;
+            f = __bfloat1622float2(b2[3]);
+            a1 += f.x * n1.z + f.y * n1.w;
+          }
+        }
+        float a = a0 + a1;
+        a += __shfl_xor_sync(0xffffffffu, a, 1);
+        if (part == 0) nq[t] = a;
+      }
+      named_bar(WG_STATE, 128);
+      if (first) mbar_arrive(&bars.nq_done);
+      if (!ret) {
+        // n <- a n + sum_s w_s k_s
+        constexpr int NCG = DK / 8, NRG = 128 / NCG, RPG = L / NRG;
+        const int cg = tid % NCG, rg = tid / NCG;
+        const int col = 8 * cg;
+        const uint8_t* kt = Ks + (col >> 6) * 8192;
+        float acc[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+#pragma unroll 4
+        for (int j = 0; j < RPG; ++j) {
+          const int srow = rg * RPG + j;
+          const uint4 u = *reinterpret_cast<const uint4*>(kt + sw128_offset(srow, col & 63));
+          const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+          const float w = G.wv[srow];
+#pragma unroll
+          for (int q2 = 0; q2 < 4; ++q2) {
+            const float2 f = __bfloat1622float2(b2[q2]);
+            acc[2 * q2] += w * f.x;
+            acc[2 * q2 + 1] += w * f.y;
+          }
+        }
+        *reinterpret_cast<float4*>(npart + tid * 8) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4*>(npart + tid * 8 + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        named_bar(WG_STATE, 128);
+        const float a = G.scal[0];
+        for (int cc = tid; cc < DK; cc += 128) {
+          float x = 0.f;
+#pragma unroll
+          for (int r = 0; r < NRG; ++r) x += npart[(r * NCG + cc / 8) * 8 + (cc & 7)];
+          nvec[cc] = a * nvec[cc] + x;
         }
       }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) npart[tid * 8 + j] = acc[j];
-      __syncthreads();
-      const float a = scal[0];
-      for (int c = tid; c < DK; c += NTW) {
-        float x = 0.f;
-        for (int r = 0; r < NRG; ++r) x += npart[(r * NCG + c / 8) * 8 + (c & 7)];
-        nvec[c] = a * nvec[c] + x;
+      named_bar(WG_STATE, 128);
+      if (first) {
+        mbar_arrive(&bars.empty[b]);
+        mbar_arrive(&bars.gempty[b]);
       }
-    } else if (tid < L) {
-      rden[tid] = 1.f;
     }
-    if (!mbar_wait(&bar_mma, it & 1, WAIT)) atomicOr(&abort_flag, 1);
-    __syncthreads();
-    if (abort_flag) break;
-    tc_fence_after();
-    // ---- outputs h_t for this value tile: H^T rows = value rows, columns = tokens
-    {
+    // final state after the last update
+    if (group_wait(&bars.mm_done, (nck - 1) & 1, 0, first) && last_seg) {
+      tc_fence_after();
       const int row = acc_row<DVT>(quarter, lane);
-      const size_t hcol = (size_t)blk * p.dv + v0 + (row >= 0 ? row : 0);
-      float r[32];
-      tmem_ld32(tm + lane_off + TM_H + half * 32, r);
-      tmem_wait_ld();
-      if (row >= 0) {
+      if (p.C_out)
+        for (int c0 = 0; c0 < DK; c0 += 32) {
+          float r[32];
+          tmem_ld32(tm + lane_off + TM_C + c0, r);
+          tmem_wait_ld();
+          if (row >= 0) {
+            float* dst = p.C_out + ((size_t)slice * p.dv + v0 + row) * p.dk + c0;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int t = half * 32 + j;
-          if (t < Lc) {
-            const size_t idx = (tok0 + t) * p.DHV + hcol;
-            float hv = r[j] * rden[t];
-            if (p.og && !ret) hv *= __bfloat162float(p.og[idx]);
-            p.h[idx] = __float2bfloat16_rn(hv);
+            for (int j = 0; j < 32; j += 4)
+              *reinterpret_cast<float4*>(dst + j) = make_float4(r[j], r[j + 1], r[j + 2], r[j + 3]);
+          }
+        }
+      if (!ret && tile == 0 && p.n_out)
+        for (int col = tid; col < DK; col += 128) p.n_out[(size_t)slice * p.dk + col] = nvec[col];
+    }
+  } else {
+    // =============================================================== output group
+    const int quarter = warp - 4;
+    const int gt = tid - 128;  // 0..127
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+    const bool first = gt == 0;
+    const uint32_t ps_u = sm_u + SM::OP;
+    for (int c = 0; c < nck; ++c) {
+      const int b = c & 1;
+      const GateBuf G = gbuf(b);
+      const int t0 = T0 + c * L;
+      const int Lc = min(L, T1 - t0);
+      const size_t tok0 = (size_t)bh * p.S + t0;
+      uint8_t* Qs = sm + b * SM::STAGE;
+      uint8_t* Vs = Qs + SM::QB + SM::KB;
+      if (!group_wait(&bars.gfull[b], (c >> 1) & 1, 1, first)) break;
+      if (!group_wait(&bars.full[b], (c >> 1) & 1, 1, first)) break;
+      if (c > 0 && !group_wait(&bars.mm_done, (c - 1) & 1, 1, first)) break;
+      // V o w for the state update (loads batched ahead of the stores)
+      {
+        constexpr int NV = L * (DVT / 8) / 128;  // 16-byte chunks per thread
+        const uint32_t vs_u = smem_u32(Vs), vw_u2 = smem_u32(Vw);
+        uint4 u[NV];
+        float wr[NV];
+        int offs[NV];
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+          const int i = k * 128 + gt;
+          const int row = i / (DVT / 8), ch = i % (DVT / 8);
+          offs[k] = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
+          u[k] = ld_shared_v4(vs_u + offs[k]);
+          wr[k] = G.wv[row];
+        }
+#pragma unroll
+        for (int k = 0; k < NV; ++k) st_shared_v4u(vw_u2 + offs[k], scale_bf16x8(u[k], wr[k]));
+      }
+      fence_proxy_async_smem();
+      named_bar(WG_OUT, 128);
+      if (first) mbar_arrive(&bars.vw_full);
+      // P = S o D' (bf16, rows t) and its row sums
+      if (!group_wait(&bars.s_full, c & 1, 1, first)) break;
+      tc_fence_after();
+      {
+        const int t = acc_row<64>(quarter, lane);
+        const int tt = t >= 0 ? t : 0;
+        const float ct = (G.bl[tt] - G.mt[tt]) * LOG2E;
+        float rs = 0.f;
+        float r[32], csr[32];
+#pragma unroll
+        for (int s0 = 0; s0 < L; s0 += 32) {
+          tmem_ld32(tm + lane_off + TM_S + s0, r);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) csr[j] = G.cs[s0 + j];
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const int s = s0 + j;
+            const float e0 = (s <= t && t < Lc) ? r[j] * exp2f(ct + csr[j]) : 0.f;
+            const float e1 = (s + 1 <= t && t < Lc) ? r[j + 1] * exp2f(ct + csr[j + 1]) : 0.f;
+            rs += e0 + e1;
+            pk[j / 2] = pack_bf16(e0, e1);
+          }
+          if (t >= 0) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+              st_shared_v4(ps_u + sw128_offset(t, s0 + 8 * q4), pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2],
+                           pk[4 * q4 + 3]);
+          }
+        }
+        if (t >= 0) rsum[t] = rs;
+      }
+      tc_fence_before();
+      named_bar(WG_OUT, 128);
+      if (first) mbar_arrive(&bars.s_empty);
+      // Q <- e^{b_t+m_c-m_t} Q (after the state group has read the raw Q), denominators
+      if (!group_wait(&bars.nq_done, c & 1, 1, first)) break;
+      {
+        constexpr int NQ = L * (DK / 8) / 128;  // 16-byte chunks per thread
+        constexpr int BATCH = NQ < 8 ? NQ : 8;
+        const uint32_t qs_u = smem_u32(Qs);
+#pragma unroll
+        for (int k0 = 0; k0 < NQ; k0 += BATCH) {
+          uint4 u[BATCH];
+          float wr[BATCH];
+          int offs[BATCH];
+#pragma unroll
+          for (int k = 0; k < BATCH; ++k) {
+            const int i = (k0 + k) * 128 + gt;
+            const int row = i / (DK / 8), ch = i % (DK / 8);
+            offs[k] = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
+            u[k] = ld_shared_v4(qs_u + offs[k]);
+            wr[k] = G.sint[row];
+          }
+#pragma unroll
+          for (int k = 0; k < BATCH; ++k) st_shared_v4u(qs_u + offs[k], scale_bf16x8(u[k], wr[k]));
+        }
+      }
+      if (gt < L) {
+        const int t = gt;
+        rden[t] = ret ? 1.f : 1.f / fmaxf(fabsf(rsum[t] + G.sint[t] * nq[t]), expf(-G.mt[t]));
+      }
+      fence_proxy_async_smem();
+      named_bar(WG_OUT, 128);
+      if (first) {
+        mbar_arrive(&bars.pq_full);
+        mbar_arrive(&bars.empty[b]);
+      }
+      // h_t = H_t / den_t (x o_t): stage the tile in shared memory, TMA store
+      if (first) bulk_wait_read_all();
+      if (!group_wait(&bars.mm_done, c & 1, 1, first)) break;
+      tc_fence_after();
+      {
+        const int row = acc_row<DVT>(quarter, lane);
+        const int rr = row >= 0 ? row : 0;
+        const uint32_t hb_u = smem_u32(Hs) + (rr >> 6) * 8192 + (rr & 63) * 2;
+        const size_t hcol = (size_t)blk * p.dv + v0 + rr;
+        float r[32], rd[32];
+#pragma unroll
+        for (int tt = 0; tt < L; tt += 32) {
+          tmem_ld32(tm + lane_off + TM_H + tt, r);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) rd[j] = rden[tt + j];
+          tmem_wait_ld();
+          if (p.og && !ret) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (tt + j < Lc) rd[j] *= __bfloat162float(p.og[(tok0 + tt + j) * p.DHV + hcol]);
+          }
+          if (row >= 0) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) st_shared_b16(hb_u + (tt + j) * 128, __float2bfloat16_rn(r[j] * rd[j]));
           }
         }
       }
+      tc_fence_before();
+      fence_proxy_async_smem();
+      named_bar(WG_OUT, 128);
+      if (first) {
+        mbar_arrive(&bars.h_empty);
+        for (int j = 0; j < DVT / 64; ++j) tma_store_3d(&mapH, Hs + j * 8192, blk * p.dv + v0 + 64 * j, t0, bh);
+        bulk_commit();
+        mbar_arrive(&bars.gempty[b]);
+      }
     }
-    if (tid == 0) scal[1] = scal[2];
-    tc_fence_before();
-    __syncthreads();
+    if (first) bulk_wait_all();
   }
 
-  // ---- final state (last segment)
-  tc_fence_after();
-  if (!abort_flag && last_seg) {
-    const int row = acc_row<DVT>(quarter, lane);
-    if (p.C_out)
-      for (int c0 = half * (DK / 2); c0 < (half + 1) * (DK / 2); c0 += 32) {
-        float r[32];
-        tmem_ld32(tm + lane_off + TM_C + c0, r);
-        tmem_wait_ld();
-        if (row >= 0) {
-          float* dst = p.C_out + ((size_t)slice * p.dv + v0 + row) * p.dk + c0;
-#pragma unroll
-          for (int j = 0; j < 32; j += 4)
-            *reinterpret_cast<float4*>(dst + j) = make_float4(r[j], r[j + 1], r[j + 2], r[j + 3]);
-        }
-      }
-    if (!ret && tile == 0) {
-      if (p.n_out)
-        for (int col = tid; col < DK; col += NTW) p.n_out[(size_t)slice * p.dk + col] = nvec[col];
-      if (p.m_out && blk == 0 && tid == 0) p.m_out[bh] = scal[1];
-    }
-  }
   if (abort_flag && tid == 0) atomicOr(p.err, 2u);
   tc_fence_before();
   __syncthreads();
@@ -797,11 +977,11 @@ size_t tc_workspace_bytes(const TcPlan& pl, long long BH, int nb, int dk, int dv
 
 template <int DK, int DVT>
 static cudaError_t launch_tc_dk(const TcPlan& pl, const TcParams& prm, const CUtensorMap& mq, const CUtensorMap& mk,
-                                const CUtensorMap& mv, long long slices, cudaStream_t stream, cudaEvent_t ev0,
-                                cudaEvent_t ev1) {
+                                const CUtensorMap& mv, const CUtensorMap& mh, long long slices, cudaStream_t stream,
+                                cudaEvent_t ev0, cudaEvent_t ev1) {
   cudaError_t e;
   if (pl.G > 1) {
-    const int smemA = 2 * DK * 128 + 2 * DVT * 128 + (NT * 8 + pl.seg_chunks * L) * 4 + 1024;
+    const int smemA = 3 * (DK * 128 + DVT * 128) + (NT * 8 + pl.seg_chunks * L) * 4 + 1024;
     e = cudaFuncSetAttribute(tc_segment_kernel<DK, DVT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemA);
     if (e != cudaSuccess) return e;
     dim3 gridA(pl.n_tiles, pl.G - 1, (unsigned)slices);
@@ -814,7 +994,7 @@ static cudaError_t launch_tc_dk(const TcPlan& pl, const TcParams& prm, const CUt
   if (e != cudaSuccess) return e;
   if (ev0) cudaEventRecord(ev0, stream);
   dim3 gridC(pl.n_tiles, pl.G, (unsigned)slices);
-  tc_walk_kernel<DK, DVT><<<gridC, NTW, smemC, stream>>>(mq, mk, mv, prm);
+  tc_walk_kernel<DK, DVT><<<gridC, NTW, smemC, stream>>>(mq, mk, mv, mh, prm);
   e = cudaGetLastError();
   if (ev1) cudaEventRecord(ev1, stream);
   return e;
@@ -824,9 +1004,10 @@ cudaError_t launch_tc(const WalkArgs& a, const TcPlan& pl, void* ws, cudaStream_
                       cudaEvent_t ev1) {
   const long long BH = (long long)a.B * a.NH, slices = BH * a.nb;
   if (slices == 0 || a.S == 0) return cudaSuccess;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mh;
   if (!make_map_bf16_3d(&mq, a.q, a.DHQK, a.S, BH, L) || !make_map_bf16_3d(&mk, a.k, a.DHQK, a.S, BH, L) ||
-      !make_map_bf16_3d(&mv, a.v, a.DHV, a.S, BH, L))
+      !make_map_bf16_3d(&mv, a.v, a.DHV, a.S, BH, L) ||
+      !make_map_bf16_3d(&mh, a.h, a.DHV, a.S, BH, L, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   TcParams prm;
   prm.S = a.S;
@@ -864,12 +1045,12 @@ cudaError_t launch_tc(const WalkArgs& a, const TcPlan& pl, void* ws, cudaStream_
   prm.segB = reinterpret_cast<float*>(w + off);
   cudaError_t e = cudaMemsetAsync(w, 0, 4, stream);
   if (e != cudaSuccess) return e;
-  if (a.dk == 256 && pl.dvt == 128) return launch_tc_dk<256, 128>(pl, prm, mq, mk, mv, slices, stream, ev0, ev1);
-  if (a.dk == 256 && pl.dvt == 64) return launch_tc_dk<256, 64>(pl, prm, mq, mk, mv, slices, stream, ev0, ev1);
-  if (a.dk == 128 && pl.dvt == 128) return launch_tc_dk<128, 128>(pl, prm, mq, mk, mv, slices, stream, ev0, ev1);
-  if (a.dk == 128 && pl.dvt == 64) return launch_tc_dk<128, 64>(pl, prm, mq, mk, mv, slices, stream, ev0, ev1);
-  if (a.dk == 64 && pl.dvt == 128) return launch_tc_dk<64, 128>(pl, prm, mq, mk, mv, slices, stream, ev0, ev1);
-  if (a.dk == 64 && pl.dvt == 64) return launch_tc_dk<64, 64>(pl, prm, mq, mk, mv, slices, stream, ev0, ev1);
+  if (a.dk == 256 && pl.dvt == 128) return launch_tc_dk<256, 128>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
+  if (a.dk == 256 && pl.dvt == 64) return launch_tc_dk<256, 64>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
+  if (a.dk == 128 && pl.dvt == 128) return launch_tc_dk<128, 128>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
+  if (a.dk == 128 && pl.dvt == 64) return launch_tc_dk<128, 64>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
+  if (a.dk == 64 && pl.dvt == 128) return launch_tc_dk<64, 128>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
+  if (a.dk == 64 && pl.dvt == 64) return launch_tc_dk<64, 64>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
   return cudaErrorInvalidValue;
 }
 

@@ -24,10 +24,10 @@ inline EncodeTiledFn encode_tiled_fn() {
   return fn;
 }
 
-// 3-D bf16 tensor [d2][d1][d0] (d0 contiguous), box {64, box_rows, 1}, 128-byte swizzle,
-// zero fill out of bounds.  Row stride d0 * 2 bytes must be a multiple of 16.
+// 3-D bf16 tensor [d2][d1][d0] (d0 contiguous), box {64, box_rows, 1}, 128-byte swizzle
+// unless given, zero fill out of bounds on loads (stores skip out-of-bounds elements).  Row stride d0 * 2 bytes must be a multiple of 16.
 inline bool make_map_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
-                             uint32_t box_rows) {
+                             uint32_t box_rows, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_tiled_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {d0, d1, d2};
@@ -35,7 +35,7 @@ inline bool make_map_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, ui
   const cuuint32_t box[3] = {64, box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
