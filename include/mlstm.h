@@ -153,6 +153,30 @@ mlstm_status_t mlstm_fwd_chunkwise_timed(const mlstm_fwd_params_t* p,
                                          mlstm_event_t main_begin, mlstm_event_t main_end);
 
 /*
+ * mlstm_fwd_chunkwise without a caller workspace (the pages have no counterpart; this
+ * is a deployment convenience).  For callers that cannot call cudaMalloc -- for example
+ * code running inside a host framework that owns all device memory and forbids outside
+ * allocations, or a loop where an allocation's implicit device synchronisation is not
+ * acceptable.  The scratch memory comes from one fixed buffer compiled into the library
+ * (mlstm_noalloc_scratch_bytes() bytes, 32 MiB), which every GPU that loads the library
+ * holds until the process exits.  Arguments are those of mlstm_fwd_chunkwise minus the
+ * workspace.  Returns MLSTM_ERR_WORKSPACE if the sizes need more scratch than the buffer
+ * holds (see mlstm_fwd_chunkwise_workspace_size).  The first call on a device looks up
+ * the buffer's device address (cudaGetSymbolAddress) and caches it; make that first
+ * call before any stream capture.  Nothing is allocated or freed.  All calls share the
+ * buffer: calls whose GPU work overlaps (other streams, other host threads) race.
+ */
+mlstm_status_t mlstm_fwd_chunkwise_noalloc(const mlstm_fwd_params_t* p,
+                                           const void* q, const void* k, const void* v,
+                                           const float* igate, const float* fgate, const void* ogate,
+                                           const float* C0, const float* n0, const float* m0,
+                                           void* h, float* C_out, float* n_out, float* m_out,
+                                           mlstm_stream_t stream);
+
+/* Size in bytes of the built-in scratch buffer used by mlstm_fwd_chunkwise_noalloc. */
+size_t mlstm_noalloc_scratch_bytes(void);
+
+/*
  * One recurrent decode step for every sequence of the batch, state updated in
  * place (RetNet recurrent_retention_step: O(1) per token; burn-gdn2 Gdn2Mode
  * FusedRecurrent: state [B,H,K,V] carried across tokens and updated in place).

@@ -359,3 +359,66 @@ mlstm_status_t mlstm_step(const mlstm_step_params_t* p, const void* q, const voi
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// Prefill without a caller workspace.  Some callers cannot call cudaMalloc at all
+// (their host framework owns every byte of device memory, or an allocation's implicit
+// device synchronisation is not acceptable where they run), so this entry point takes
+// its scratch memory from a fixed buffer compiled into the library instead.
+//
+// The buffer is a file-scope __device__ array: every GPU that loads the library holds
+// MLSTM_NOALLOC_SCRATCH_BYTES of it until the process exits.  All calls share it and it
+// keeps whatever the previous call left there; the kernels write every scratch byte they
+// read except the error word, which each call clears on its stream.  Two calls whose
+// GPU work overlaps (different streams, or different host threads) race on the buffer.
+#include <mutex>
+
+#define MLSTM_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MLSTM_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  The host-side name of a
+// __device__ array is only a stand-in, so the address is looked up once per device,
+// with that device current, and cached.
+mlstm_status_t noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLSTM_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return MLSTM_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MLSTM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mlstm_noalloc_scratch_bytes(void) { return MLSTM_NOALLOC_SCRATCH_BYTES; }
+
+mlstm_status_t mlstm_fwd_chunkwise_noalloc(const mlstm_fwd_params_t* p, const void* q, const void* k, const void* v,
+                                           const float* igate, const float* fgate, const void* ogate,
+                                           const float* C0, const float* n0, const float* m0, void* h, float* C_out,
+                                           float* n_out, float* m_out, mlstm_stream_t stream) {
+  FwdShape s;
+  mlstm_status_t st = check_fwd(p, &s);
+  if (st != MLSTM_OK) return st;
+  const size_t need = fwd_layout(s).total;
+  if (need > MLSTM_NOALLOC_SCRATCH_BYTES) return MLSTM_ERR_WORKSPACE;  // too large for the built-in buffer
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != MLSTM_OK) return st;
+  return fwd_impl(p, q, k, v, igate, fgate, ogate, C0, n0, m0, h, C_out, n_out, m_out, scratch,
+                  MLSTM_NOALLOC_SCRATCH_BYTES, (cudaStream_t)stream, nullptr, nullptr);
+}
+
+}  // extern "C"

@@ -62,6 +62,10 @@ def lib():
         L.mlstm_fwd_chunkwise.restype = I
         L.mlstm_fwd_chunkwise_timed.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 14 + [Z, P, P, P]
         L.mlstm_fwd_chunkwise_timed.restype = I
+        L.mlstm_fwd_chunkwise_noalloc.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 13 + [P]
+        L.mlstm_fwd_chunkwise_noalloc.restype = I
+        L.mlstm_noalloc_scratch_bytes.argtypes = []
+        L.mlstm_noalloc_scratch_bytes.restype = Z
         L.mlstm_step.argtypes = [ctypes.POINTER(StepParams)] + [P] * 10 + [P]
         L.mlstm_step.restype = I
         L.mlstm_status_string.argtypes = [I]
@@ -157,6 +161,37 @@ def fwd_chunkwise(q, k, v, igate=None, fgate=None, ogate=None, C0=None, n0=None,
                                              ctypes.c_void_p(events[1].cuda_event))
     if st != 0:
         raise MlstmError(st, "mlstm_fwd_chunkwise")
+    if retention:
+        return h, C_out, None, None
+    return h, C_out, n_out, m_out
+
+
+def fwd_chunkwise_noalloc(q, k, v, igate=None, fgate=None, ogate=None, C0=None, n0=None, m0=None, *,
+                          chunk: int = 64, num_blocks: int = 1, retention: bool = False,
+                          h=None, C_out=None, n_out=None, m_out=None, stream=None):
+    """mlstm_fwd_chunkwise_noalloc: the prefill with the library's built-in scratch buffer
+    instead of a workspace (for callers that cannot allocate device memory).  Outputs not
+    passed in are allocated here with torch, as in fwd_chunkwise; the library allocates
+    nothing.  Calls that overlap on the GPU share the buffer and race."""
+    B, NH, S, DHQK = q.shape
+    DHV = v.shape[-1]
+    nb = int(num_blocks)
+    p = fwd_params(B, NH, S, DHQK, DHV, chunk, nb, q.dtype, retention)
+    dev = q.device
+    if h is None:
+        h = torch.empty((B, NH, S, DHV), dtype=q.dtype, device=dev)
+    if C_out is None:
+        C_out = torch.empty((B, NH, nb, DHV // nb, DHQK // nb), dtype=torch.float32, device=dev)
+    if not retention:
+        if n_out is None:
+            n_out = torch.empty((B, NH, nb, DHQK // nb), dtype=torch.float32, device=dev)
+        if m_out is None:
+            m_out = torch.empty((B, NH), dtype=torch.float32, device=dev)
+    st = lib().mlstm_fwd_chunkwise_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(igate), _ptr(fgate),
+                                           _ptr(ogate), _ptr(C0), _ptr(n0), _ptr(m0), _ptr(h), _ptr(C_out),
+                                           _ptr(n_out), _ptr(m_out), _stream_ptr(stream))
+    if st != 0:
+        raise MlstmError(st, "mlstm_fwd_chunkwise_noalloc")
     if retention:
         return h, C_out, None, None
     return h, C_out, n_out, m_out
