@@ -226,18 +226,23 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
     if (abort_flag) break;
     const float* om = omega + c * L;
-    for (int i = tid; i < L * (DVT / 8); i += NT) {
-      const int row = i / (DVT / 8), ch = i % (DVT / 8);
-      uint8_t* ptr = Vst + (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
-      uint4 u = *reinterpret_cast<uint4*>(ptr);
-      __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&u);
-      const float w = om[row];
+    {
+      // V rows scaled in place by omega (loads batched ahead of the stores)
+      constexpr int NV = L * (DVT / 8) / NT;
+      const uint32_t v_u = smem_u32(Vst);
+      uint4 u[NV];
+      float wr[NV];
+      int offs[NV];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = __bfloat1622float2(b2[j]);
-        b2[j] = __floats2bfloat162_rn(f.x * w, f.y * w);
+      for (int k = 0; k < NV; ++k) {
+        const int i = k * NT + tid;
+        const int row = i / (DVT / 8), ch = i % (DVT / 8);
+        offs[k] = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
+        u[k] = ld_shared_v4(v_u + offs[k]);
+        wr[k] = om[row];
       }
-      *reinterpret_cast<uint4*>(ptr) = u;
+#pragma unroll
+      for (int k = 0; k < NV; ++k) st_shared_v4u(v_u + offs[k], scale_bf16x8(u[k], wr[k]));
     }
     if (do_dn && rg < nrg && dcol < DK) {
       const uint8_t* kt = Kst + (dcol >> 6) * 8192;
@@ -255,22 +260,25 @@ __global__ void __launch_bounds__(NT, 1)
     }
     fence_proxy_async_smem();
     __syncthreads();
-    if (tid == 0) {
+    if (warp == 0) {
       tc_fence_after();
-      const uint32_t va = smem_u32(Vst), ka = smem_u32(Kst);
+      const uint64_t ad = smem_desc_sw128(smem_u32(Vst), 8192, 1024);
+      const uint64_t bd = smem_desc_sw128(smem_u32(Kst), 8192, 1024);
+      if (elect_one()) {
 #pragma unroll
-      for (int ks = 0; ks < L / 16; ++ks)
-        mma_bf16_ss(tm, smem_desc_sw128(va + ks * 2048, 8192, 1024), smem_desc_sw128(ka + ks * 2048, 8192, 1024),
-                    idesc, (c > 0 || ks > 0) ? 1u : 0u);
-      mma_commit(&bar_mma[st]);
-      // stage (c + NS - 1) % NS was last read by the MMAs of chunk c - 1 (queued before
-      // this chunk's): refill it once they are done; the other threads move on
-      if (c + NS - 1 < nck) {
-        if (c >= 1 && !mbar_wait(&bar_mma[(c - 1) % NS], ((c - 1) / NS) & 1, WAIT))
-          atomicOr(&abort_flag, 1);
-        else
-          issue(c + NS - 1);
+        for (int ks = 0; ks < L / 16; ++ks)
+          mma_bf16_ss(tm, ad + (uint64_t)(ks * 128), bd + (uint64_t)(ks * 128), idesc, (c > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(&bar_mma[st]);
+        // stage (c + NS - 1) % NS was last read by the MMAs of chunk c - 1 (queued before
+        // this chunk's): refill it once they are done; the other warps move on
+        if (c + NS - 1 < nck) {
+          if (c >= 1 && !mbar_wait(&bar_mma[(c - 1) % NS], ((c - 1) / NS) & 1, WAIT))
+            atomicOr(&abort_flag, 1);
+          else
+            issue(c + NS - 1);
+        }
       }
+      __syncwarp();
     }
   }
   if (!abort_flag && !mbar_wait(&bar_mma[(nck - 1) % NS], ((nck - 1) / NS) & 1, WAIT)) atomicOr(&abort_flag, 1);
@@ -341,7 +349,7 @@ struct GateBuf {
 
 struct WalkBars {
   uint64_t full[2], empty[2], gfull[2], gempty[2];
-  uint64_t s_full, s_empty, e1_done, vw_full, pq_full, h_empty, mm_done, nq_done;
+  uint64_t s_full, s_empty, e1_done, vw_full, upd_done, q_ready, p_full, h_empty, mm_done, nq_done;
 };
 
 template <int DK, int DVT>
@@ -394,7 +402,9 @@ __global__ void __launch_bounds__(NTW, 1)
     mbar_init(&bars.s_empty, 1);
     mbar_init(&bars.e1_done, 1);
     mbar_init(&bars.vw_full, 1);
-    mbar_init(&bars.pq_full, 1);
+    mbar_init(&bars.upd_done, 1);
+    mbar_init(&bars.q_ready, 1);
+    mbar_init(&bars.p_full, 1);
     mbar_init(&bars.h_empty, 1);
     mbar_init(&bars.mm_done, 1);
     mbar_init(&bars.nq_done, 1);
@@ -629,9 +639,10 @@ __global__ void __launch_bounds__(NTW, 1)
 #pragma unroll
         for (int ks = 0; ks < L / 16; ++ks)
           mma_bf16_ss(tm + TM_C, vw_mn + (uint64_t)(ks * 128), k_mn + (uint64_t)(ks * 128), id_up, 1u);
+        mma_commit(&bars.upd_done);
       }
       __syncwarp();
-      if (!warp_wait(&bars.pq_full, c & 1)) break;
+      if (!warp_wait(&bars.q_ready, c & 1)) break;
       if (c > 0 && !warp_wait(&bars.h_empty, (c - 1) & 1)) break;
       tc_fence_after();
       if (elect_one()) {
@@ -639,6 +650,11 @@ __global__ void __launch_bounds__(NTW, 1)
         for (int k = 0; k < DK; k += 16)
           mma_bf16_ts(tm + TM_H, tm + TM_CB + k / 2, q_k + (uint64_t)(((k >> 6) * 8192 + (k & 63) * 2) >> 4), id_ro,
                       k > 0 ? 1u : 0u);
+      }
+      __syncwarp();
+      if (!warp_wait(&bars.p_full, c & 1)) break;
+      tc_fence_after();
+      if (elect_one()) {
 #pragma unroll
         for (int ks = 0; ks < L / 16; ++ks)
           mma_bf16_ss(tm + TM_H, v_mn + (uint64_t)(ks * 128), ps_k + (uint64_t)(ks * 2), id_pv, 1u);
@@ -721,6 +737,34 @@ __global__ void __launch_bounds__(NTW, 1)
       }
       named_bar(WG_STATE, 128);
       if (first) mbar_arrive(&bars.nq_done);
+      // Q <- e^{b_t+m_c-m_t} Q once the S MMA has read the raw Q (read-out and intra-chunk
+      // then share one accumulator)
+      if (!group_wait(&bars.s_full, c & 1, 0, first)) break;
+      {
+        const int gt = tid;
+        constexpr int NQ = L * (DK / 8) / 128;  // 16-byte chunks per thread
+        constexpr int BATCH = NQ < 8 ? NQ : 8;
+        const uint32_t qs_u = smem_u32(Qs);
+#pragma unroll
+        for (int k0 = 0; k0 < NQ; k0 += BATCH) {
+          uint4 u[BATCH];
+          float wr[BATCH];
+          int offs[BATCH];
+#pragma unroll
+          for (int k = 0; k < BATCH; ++k) {
+            const int i = (k0 + k) * 128 + gt;
+            const int row = i / (DK / 8), ch = i % (DK / 8);
+            offs[k] = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
+            u[k] = ld_shared_v4(qs_u + offs[k]);
+            wr[k] = G.sint[row];
+          }
+#pragma unroll
+          for (int k = 0; k < BATCH; ++k) st_shared_v4u(qs_u + offs[k], scale_bf16x8(u[k], wr[k]));
+        }
+      }
+      fence_proxy_async_smem();
+      named_bar(WG_STATE, 128);
+      if (first) mbar_arrive(&bars.q_ready);
       if (!ret) {
         // n <- a n + sum_s w_s k_s
         constexpr int NCG = DK / 8, NRG = 128 / NCG, RPG = L / NRG;
@@ -796,7 +840,7 @@ __global__ void __launch_bounds__(NTW, 1)
       uint8_t* Vs = Qs + SM::QB + SM::KB;
       if (!group_wait(&bars.gfull[b], (c >> 1) & 1, 1, first)) break;
       if (!group_wait(&bars.full[b], (c >> 1) & 1, 1, first)) break;
-      if (c > 0 && !group_wait(&bars.mm_done, (c - 1) & 1, 1, first)) break;
+      if (c > 0 && !group_wait(&bars.upd_done, (c - 1) & 1, 1, first)) break;
       // V o w for the state update (loads batched ahead of the stores)
       {
         constexpr int NV = L * (DVT / 8) / 128;  // 16-byte chunks per thread
@@ -818,75 +862,57 @@ __global__ void __launch_bounds__(NTW, 1)
       fence_proxy_async_smem();
       named_bar(WG_OUT, 128);
       if (first) mbar_arrive(&bars.vw_full);
-      // P = S o D' (bf16, rows t) and its row sums
+      // P = S o D' (bf16, rows t) and its row sums; P V of the previous chunk must be done
+      if (c > 0 && !group_wait(&bars.mm_done, (c - 1) & 1, 1, first)) break;
       if (!group_wait(&bars.s_full, c & 1, 1, first)) break;
       tc_fence_after();
       {
-        const int t = acc_row<64>(quarter, lane);
-        const int tt = t >= 0 ? t : 0;
-        const float ct = (G.bl[tt] - G.mt[tt]) * LOG2E;
-        float rs = 0.f;
-        float r[32], csr[32];
+        // 16x256b load: thread -> rows 16q + lane/4 and +8, column pairs 8j + 2(lane%4)
+        const int r_lo = 16 * quarter + (lane >> 2), r_hi = r_lo + 8, cp = 2 * (lane & 3);
+        float r[32], csr[16];
+        tmem_ld16x256_x8(tm + lane_off + TM_S, r);
 #pragma unroll
-        for (int s0 = 0; s0 < L; s0 += 32) {
-          tmem_ld32(tm + lane_off + TM_S + s0, r);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) csr[j] = G.cs[s0 + j];
-          tmem_wait_ld();
-          uint32_t pk[16];
-#pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const int s = s0 + j;
-            const float e0 = (s <= t && t < Lc) ? r[j] * exp2f(ct + csr[j]) : 0.f;
-            const float e1 = (s + 1 <= t && t < Lc) ? r[j + 1] * exp2f(ct + csr[j + 1]) : 0.f;
-            rs += e0 + e1;
-            pk[j / 2] = pack_bf16(e0, e1);
-          }
-          if (t >= 0) {
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-              st_shared_v4(ps_u + sw128_offset(t, s0 + 8 * q4), pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2],
-                           pk[4 * q4 + 3]);
-          }
+        for (int j = 0; j < 8; ++j) {
+          csr[2 * j] = G.cs[8 * j + cp];
+          csr[2 * j + 1] = G.cs[8 * j + cp + 1];
         }
-        if (t >= 0) rsum[t] = rs;
+        const float ct_lo = (G.bl[r_lo] - G.mt[r_lo]) * LOG2E, ct_hi = (G.bl[r_hi] - G.mt[r_hi]) * LOG2E;
+        tmem_wait_ld();
+        float rs_lo = 0.f, rs_hi = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int s0 = 8 * j + cp;
+          const float a0 = (s0 <= r_lo && r_lo < Lc) ? r[2 * j] * exp2f(ct_lo + csr[2 * j]) : 0.f;
+          const float a1 = (s0 + 1 <= r_lo && r_lo < Lc) ? r[2 * j + 1] * exp2f(ct_lo + csr[2 * j + 1]) : 0.f;
+          const float b0 = (s0 <= r_hi && r_hi < Lc) ? r[16 + 2 * j] * exp2f(ct_hi + csr[2 * j]) : 0.f;
+          const float b1 = (s0 + 1 <= r_hi && r_hi < Lc) ? r[16 + 2 * j + 1] * exp2f(ct_hi + csr[2 * j + 1]) : 0.f;
+          rs_lo += a0 + a1;
+          rs_hi += b0 + b1;
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(ps_u + sw128_offset(r_lo, s0)), "r"(pack_bf16(a0, a1)) : "memory");
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(ps_u + sw128_offset(r_hi, s0)), "r"(pack_bf16(b0, b1)) : "memory");
+        }
+        rs_lo += __shfl_xor_sync(0xffffffffu, rs_lo, 1);
+        rs_lo += __shfl_xor_sync(0xffffffffu, rs_lo, 2);
+        rs_hi += __shfl_xor_sync(0xffffffffu, rs_hi, 1);
+        rs_hi += __shfl_xor_sync(0xffffffffu, rs_hi, 2);
+        if ((lane & 3) == 0) {
+          rsum[r_lo] = rs_lo;
+          rsum[r_hi] = rs_hi;
+        }
       }
+      fence_proxy_async_smem();
       tc_fence_before();
       named_bar(WG_OUT, 128);
       if (first) mbar_arrive(&bars.s_empty);
-      // Q <- e^{b_t+m_c-m_t} Q (after the state group has read the raw Q), denominators
+      if (first) mbar_arrive(&bars.p_full);
+      // denominators (need n . q_t from the state group)
       if (!group_wait(&bars.nq_done, c & 1, 1, first)) break;
-      {
-        constexpr int NQ = L * (DK / 8) / 128;  // 16-byte chunks per thread
-        constexpr int BATCH = NQ < 8 ? NQ : 8;
-        const uint32_t qs_u = smem_u32(Qs);
-#pragma unroll
-        for (int k0 = 0; k0 < NQ; k0 += BATCH) {
-          uint4 u[BATCH];
-          float wr[BATCH];
-          int offs[BATCH];
-#pragma unroll
-          for (int k = 0; k < BATCH; ++k) {
-            const int i = (k0 + k) * 128 + gt;
-            const int row = i / (DK / 8), ch = i % (DK / 8);
-            offs[k] = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
-            u[k] = ld_shared_v4(qs_u + offs[k]);
-            wr[k] = G.sint[row];
-          }
-#pragma unroll
-          for (int k = 0; k < BATCH; ++k) st_shared_v4u(qs_u + offs[k], scale_bf16x8(u[k], wr[k]));
-        }
-      }
       if (gt < L) {
         const int t = gt;
         rden[t] = ret ? 1.f : 1.f / fmaxf(fabsf(rsum[t] + G.sint[t] * nq[t]), expf(-G.mt[t]));
       }
-      fence_proxy_async_smem();
       named_bar(WG_OUT, 128);
-      if (first) {
-        mbar_arrive(&bars.pq_full);
-        mbar_arrive(&bars.empty[b]);
-      }
+      if (first) mbar_arrive(&bars.empty[b]);
       // h_t = H_t / den_t (x o_t): stage the tile in shared memory, TMA store
       if (first) bulk_wait_read_all();
       if (!group_wait(&bars.mm_done, c & 1, 1, first)) break;
