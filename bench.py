@@ -31,6 +31,39 @@ sys.path.insert(0, ROOT)
 METRIC = "mLSTM chunkwise-fwd tokens/s (% bf16 TC peak); decode-step state GB/s (% HBM)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch, from one ncu
+# capture, with the sha256 of the kernel's sources at capture time.  Reported only while
+# the sources still hash the same; otherwise the counters are stale and traffic is null.
+CSRC = os.path.join(ROOT, "linear_recurrent_token_b200", "csrc")
+RECORDED_TRAFFIC = {
+    ("tc_walk", "large_head"): {
+        "bytes": 147_525_376 + 40_239_360,
+        "sources": ("chunkwise_tc.cu", "sm100.cuh", "common.cuh", "kernels.h"),
+        "sha256": "366332cd36de00b259675ce76f41d1fff928990c31b4a7b403b997256832aa7d",
+    },
+    ("step", "decode"): {
+        "bytes": 540_051_712 + 480_060_160,
+        "sources": ("step.cu", "common.cuh", "kernels.h"),
+        "sha256": "b64fcb693c657680bc53ef26ac8af0727bb74fef23054abb5c4655cf58c4773c",
+    },
+}
+
+
+def sources_sha256(names) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(CSRC, n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel: str, workload: str):
+    r = RECORDED_TRAFFIC.get((kernel, workload))
+    if r is None or sources_sha256(r["sources"]) != r["sha256"]:
+        return None
+    return r["bytes"]
+
 
 # ------------------------------------------------------------------ work accounting
 def chunkwise_flops(B, NH, S, dk, dv, L, nb=1, retention=False):
@@ -358,9 +391,13 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=3, help="chunkwise workload index (default 3)")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--legs", choices=["both", "chunkwise", "decode"], default="both",
+                    help="run only one leg (for profiling); the default runs both")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.legs == "chunkwise":
+        args.no_decode = True
 
     from linear_recurrent_token_b200 import inputs
     w = inputs.WORKLOADS[args.workload]
@@ -398,6 +435,13 @@ def main():
     try:
         dist_barrier(world)
         torch.cuda.synchronize()
+        if args.legs == "decode":
+            dec = run_decode(wd, args.steps, args.warmup, clocks)
+            ms = dist_max(statistics.mean(dec["step_ms"]), world)
+            dbytes = decode_step_bytes(wd.B, wd.NH, wd.DHQK, wd.DHV, 2, wd.num_blocks)
+            if rank == 0:
+                print(json.dumps({"leg": "decode", "ms_per_step": ms, "GB/s": dbytes / (ms * 1e-3) / 1e9}))
+            return
         cw = run_chunkwise(w, args.steps, args.warmup, 256 << 20, clocks)
         dist_barrier(world)
         torch.cuda.synchronize()
@@ -428,7 +472,8 @@ def main():
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
         "config": config,
         "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": achieved_tf / peaks["bf16_tflops"], "traffic": None,
+                     "frac": achieved_tf / peaks["bf16_tflops"],
+                     "traffic": recorded_traffic("tc_walk", w.name) if cw["plan"]["tensor_core"] else None,
                      "kernel": "chunkwise walk" + (" (tcgen05)" if cw["plan"]["tensor_core"] else " (SIMT)"),
                      "kernel_ms": main_ms, "flops_per_launch": flops, "peak_source": f"{peak_src} bf16 burst",
                      "hbm_frac": mbytes / (main_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
@@ -449,7 +494,8 @@ def main():
             "value": gbs, "unit": "GB/s", "ms_per_step": dms_max, "steps": len(dec["step_ms"]),
             "tokens_per_s": wd.B * world / (dms_max * 1e-3),
             "roofline": {"bound": "hbm", "achieved": per_rank_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": per_rank_gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "step_kernel<256>",
+                         "frac": per_rank_gbs / peaks["hbm_gbs"], "traffic": recorded_traffic("step", wd.name),
+                         "kernel": "step_kernel<256>",
                          "bytes_per_launch": dbytes, "peak_source": f"{peak_src} copy bandwidth"},
             "e2e": {"value": wd.B * world / (dec["e2e_ms"] * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": dec["h2d"], "d2h_bytes_per_step": dec["d2h"]},

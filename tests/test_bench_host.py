@@ -60,3 +60,14 @@ def test_two_replicas_report_the_slowest_rank():
         out = mgr.dict()
         mp.spawn(_rank_main, args=(world, port, out), nprocs=world, join=True)
         assert dict(out) == {0: 2.5, 1: 2.5}
+
+
+def test_recorded_traffic_is_null_once_sources_change(monkeypatch):
+    import bench
+    key = ("tc_walk", "large_head")
+    rec = dict(bench.RECORDED_TRAFFIC[key])
+    monkeypatch.setitem(bench.RECORDED_TRAFFIC, key, dict(rec, sha256="0" * 64))
+    assert bench.recorded_traffic(*key) is None
+    monkeypatch.setitem(bench.RECORDED_TRAFFIC, key, dict(rec, sha256=bench.sources_sha256(rec["sources"])))
+    assert bench.recorded_traffic(*key) == rec["bytes"]
+    assert bench.recorded_traffic("tc_walk", "retention") is None
