@@ -54,6 +54,11 @@ struct TcParams {
   __nv_bfloat16* h;
   float *C_out, *n_out, *m_out;
   float *dC, *dn, *segA, *segB;  // workspace: summaries of segments 0..G-2
+  // workspace: prepared gate planes [BH][sp] (sp = G * seg_chunks * L, one row per (b, h)):
+  // b_t (inclusive cumulative log f inside the chunk), X_t = itilde_t - b_t and its running
+  // maximum inside the chunk; per chunk [BH][ncp] its total log f and max X
+  float *gb, *gx, *gxc, *cg, *cxm;
+  int sp, ncp;
   unsigned int* err;
 };
 
@@ -89,9 +94,6 @@ __device__ __forceinline__ uint4 scale_bf16x8(uint4 u, float w) {
   }
   return u;
 }
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
 
 // Gate values of token t (global index) for head `head`: (log f, itilde).
 __device__ __forceinline__ void gate_vals(const TcParams& p, size_t tok, int head, float& lf, float& li) {
@@ -106,6 +108,54 @@ __device__ __forceinline__ void gate_vals(const TcParams& p, size_t tok, int hea
 
 }  // namespace
 
+// ===================================================================== gate preparation
+// One warp per (b, h, chunk): the within-chunk scans both kernels below need, computed once.
+// Token t of the chunk (lane t/2): b_t = sum_{s<=t} log f_s, X_t = itilde_t - b_t,
+// Xc_t = max_{s<=t} X_s.  Tokens past the end of the sequence carry log f = 0 and
+// itilde = -inf (b and Xc keep the last token's values, X = -inf), so consumers need no
+// bounds logic; the chunk totals are the values of token 63.
+__global__ void __launch_bounds__(256) tc_gate_prep_kernel(TcParams p, int BH) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long wid = (long long)blockIdx.x * 8 + warp;
+  if (wid >= (long long)BH * p.ncp) return;
+  const int bh = (int)(wid / p.ncp), c = (int)(wid % p.ncp);
+  const int t0 = c * L;
+  if (t0 >= p.S) return;
+  const int Lc = min(L, p.S - t0);
+  const size_t tok = (size_t)bh * p.S + t0;
+  const int ta = 2 * lane, tb = ta + 1;
+  float lfa = 0.f, lfb = 0.f, lia = -INFINITY, lib = -INFINITY;
+  if (ta < Lc) gate_vals(p, tok + ta, bh % p.NH, lfa, lia);
+  if (tb < Lc) gate_vals(p, tok + tb, bh % p.NH, lfb, lib);
+  float isum = lfa + lfb;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float u = __shfl_up_sync(0xffffffffu, isum, o);
+    if (lane >= o) isum += u;
+  }
+  float esum = __shfl_up_sync(0xffffffffu, isum, 1);
+  if (lane == 0) esum = 0.f;
+  const float ba = esum + lfa, bb = ba + lfb;
+  const float xa = lia - ba, xb = lib - bb;
+  float mx = fmaxf(xa, xb);
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float u = __shfl_up_sync(0xffffffffu, mx, o);
+    if (lane >= o) mx = fmaxf(mx, u);
+  }
+  float ex = __shfl_up_sync(0xffffffffu, mx, 1);
+  if (lane == 0) ex = -INFINITY;
+  const float xca = fmaxf(ex, xa), xcb = fmaxf(xca, xb);
+  const size_t r = (size_t)bh * p.sp + t0 + ta;
+  *reinterpret_cast<float2*>(p.gb + r) = make_float2(ba, bb);
+  *reinterpret_cast<float2*>(p.gx + r) = make_float2(xa, xb);
+  *reinterpret_cast<float2*>(p.gxc + r) = make_float2(xca, xcb);
+  if (lane == 31) {
+    p.cg[(size_t)bh * p.ncp + c] = bb;
+    p.cxm[(size_t)bh * p.ncp + c] = xcb;
+  }
+}
+
 // ===================================================================== phase A
 // CTA = (value tile, segment < G-1, slice); 128 threads.  Two TMA stages of (K, V).
 template <int DK, int DVT>
@@ -119,6 +169,7 @@ __global__ void __launch_bounds__(NT, 1)
   // stage i: K at sm + i*(KB+VB), V right after it
   float* dnp = reinterpret_cast<float*>(sm + NS * (KB + VB));  // [NT * 8] partial sums of dn
   float* omega = dnp + NT * 8;                                  // [seg_chunks * L]
+  float* coff = omega + p.seg_chunks * L;                       // [seg_chunks]
   __shared__ uint64_t bar_load[NS], bar_mma[NS];
   __shared__ uint32_t tmem_base;
   __shared__ float red[NT / 32];
@@ -126,7 +177,7 @@ __global__ void __launch_bounds__(NT, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.x, g = blockIdx.y, slice = blockIdx.z;
-  const int blk = slice % p.nb, bh = slice / p.nb, head = bh % p.NH;
+  const int blk = slice % p.nb, bh = slice / p.nb;
   const int seg_len = p.seg_chunks * L;
   const int T0 = g * seg_len;  // phase A covers full segments only
   const int v0 = tile * DVT;
@@ -163,51 +214,44 @@ __global__ void __launch_bounds__(NT, 1)
   if (tid == 0)
     for (int c = 0; c < NS - 1 && c < nck; ++c) issue(c);
 
-  // ---- gates: G_s (inclusive cumulative log f), Gtot, M, omega_s
-  const size_t tok0 = (size_t)bh * p.S + T0;
-  const int per = (seg_len + NT - 1) / NT;
-  const int r0 = min(seg_len, tid * per), r1 = min(seg_len, r0 + per);
-  float run = 0.f;
-  for (int t = r0; t < r1; ++t) {
-    float lf, li;
-    gate_vals(p, tok0 + t, head, lf, li);
-    omega[t] = lf;
-    run += lf;
+  // ---- gates: Gtot = sum of the chunk totals, and for token s of chunk c the log weight
+  // Gtot - G_s + itilde_s = Gtot - Gpre_c + X_s (Gpre_c: totals of the earlier chunks of the
+  // segment); M = its maximum = max_c (Gtot - Gpre_c + max X of chunk c); omega_s = e^{. - M}
+  {
+    const size_t crow = (size_t)bh * p.ncp + (size_t)g * p.seg_chunks;
+    const float gcv = tid < nck ? p.cg[crow + tid] : 0.f;
+    const float xmv = tid < nck ? p.cxm[crow + tid] : -INFINITY;
+    float inc = gcv;
+    for (int o = 1; o < 32; o <<= 1) {
+      const float u = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += u;
+    }
+    if (lane == 31) red[warp] = inc;
+    __syncthreads();
+    float wexcl = 0.f, total = 0.f;
+    for (int w = 0; w < NT / 32; ++w) {
+      if (w < warp) wexcl += red[w];
+      total += red[w];
+    }
+    const float gpre = wexcl + inc - gcv;
+    float lmax = tid < nck ? total - gpre + xmv : -INFINITY;
+    for (int o = 16; o >= 1; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+    __syncthreads();
+    if (lane == 0) red[warp] = lmax;
+    __syncthreads();
+    float Mg = -INFINITY;
+    for (int w = 0; w < NT / 32; ++w) Mg = fmaxf(Mg, red[w]);
+    if (p.retention) Mg = 0.f;
+    if (tid < nck) coff[tid] = total - gpre - Mg;
+    if (tile == 0 && blk == 0 && tid == 0) {
+      p.segA[(size_t)bh * (p.G - 1) + g] = total;
+      p.segB[(size_t)bh * (p.G - 1) + g] = Mg;
+    }
+    __syncthreads();
+    const float* gxr = p.gx + (size_t)bh * p.sp + T0;
+    for (int t = tid; t < seg_len; t += NT) omega[t] = expf(coff[t / L] + gxr[t]);
+    __syncthreads();
   }
-  float inc = run;
-  for (int o = 1; o < 32; o <<= 1) {
-    const float u = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += u;
-  }
-  if (lane == 31) red[warp] = inc;
-  __syncthreads();
-  float wexcl = 0.f, total = 0.f;
-  for (int w = 0; w < NT / 32; ++w) {
-    if (w < warp) wexcl += red[w];
-    total += red[w];
-  }
-  float Gs = wexcl + inc - run;
-  float lmax = -INFINITY;
-  for (int t = r0; t < r1; ++t) {
-    Gs += omega[t];
-    const float li = p.retention ? 0.f : p.ig[tok0 + t];
-    const float x = li - Gs;  // log weight minus Gtot
-    omega[t] = x;
-    lmax = fmaxf(lmax, total + x);
-  }
-  for (int o = 16; o >= 1; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
-  __syncthreads();
-  if (lane == 0) red[warp] = lmax;
-  __syncthreads();
-  float Mg = -INFINITY;
-  for (int w = 0; w < NT / 32; ++w) Mg = fmaxf(Mg, red[w]);
-  if (p.retention) Mg = 0.f;
-  for (int t = r0; t < r1; ++t) omega[t] = expf(total + omega[t] - Mg);
-  if (tile == 0 && blk == 0 && tid == 0) {
-    p.segA[(size_t)bh * (p.G - 1) + g] = total;
-    p.segB[(size_t)bh * (p.G - 1) + g] = Mg;
-  }
-  __syncthreads();
 
   // ---- main loop: D[dv, dk] += (V o omega)^T K over the segment
   const uint32_t idesc = idesc_bf16(DVT, DK, 1, 1);
@@ -316,13 +360,33 @@ __global__ void __launch_bounds__(NT, 1)
 
 // ===================================================================== phase C
 // Warp-specialised walk: 10 warps.
-//   warps 0-3  state group: C round trip (bf16 copy into TMEM, C <- a C), n . q_t, n update
-//   warps 4-7  output group: V o w, P = S o D', Q scaling, denominators, h (TMA store)
-//   warp 8     MMA issue (one elected lane, fully unrolled, descriptors from constants)
-//   warp 9     producer: TMA loads of Q/K/V (two stages) and the per-chunk gate scan
+//   warp 0     producer: TMA loads of Q/K/V (two stages) and the per-chunk gate quantities
+//   warp 1     MMA issue (one elected lane, fully unrolled, descriptors from constants)
+//   warps 2-5  state group: bf16 snapshot of C into TMEM (the read-out operand), n . q_t,
+//              Q scaling (guarded chunks only), n update
+//   warps 6-9  output group: P, V o u for the next chunk, denominators, h (TMA store)
+// The two single-warp roles have the lowest warp ids: a warp scheduler favours its older
+// warps, and with the groups' long instruction runs on the same sub-partitions the producer
+// and the MMA issuer otherwise wait thousands of cycles for issue slots.  A group's warps
+// cover the four TMEM lane quarters (warp % 4).
 // Hand-offs are mbarriers; every wait is bounded, and a group decides to abort as one.
+//
+// Lazily scaled state.  TMEM holds C_st with C_unstabilised = e^{lam} C_st (n likewise),
+// lam a scalar every role tracks identically.  With X_s = itilde_s - b_s (b the inclusive
+// cumulative log f inside the chunk) and S = Q K^T:
+//   h_t (stabilised numerator) = E_t [ C_st q_t + sum_{s<=t} u_s S_ts v_s ],
+//   E_t = e^{b_t + lam - m_t},  u_s = e^{X_s - lam},
+//   C_st <- C_st + (V o u)^T K,  lam <- lam + g      (g = b of the chunk's last token)
+// so C is never rescaled in place: the chunk recurrence is one TMEM snapshot and two MMAs.
+// lam is moved up to the stabiliser m_c (one extra TMEM pass over C) when m_c - lam > 20.
+// A chunk with max_s X_s - lam > 60 (an input gate far above the running stabiliser) is
+// "guarded": it uses the per-element stabilised form instead (C rescaled to units of
+// e^{m}, Q scaled by e^{b_t + m_c - m_t}, P = S o e^{b_t - m_t + X_s}, update weights
+// e^{g + X_s - m_next}); every fp32 / bf16 value then stays within e^{+-60} of 1.
 constexpr int NTW = 320;
 constexpr int WG_STATE = 1, WG_OUT = 2;  // named barrier ids of the two 128-thread groups
+constexpr float LAM_RENORM = 20.f;       // renormalise lam when the stabiliser is this far above
+constexpr float U_MAX_LOG = 60.f;        // largest log u_s a fast chunk may use
 
 template <int DK, int DVT>
 struct WalkSmem {
@@ -330,26 +394,30 @@ struct WalkSmem {
   static constexpr int STAGE = QB + KB + VB;
   static constexpr int OVW = 2 * STAGE, OP = OVW + VB, OH = OP + PB;
   static constexpr int OF = OH + HB;  // floats start here
-  // n [DK], n partials [128*8], gate buffers [2][6][L], nq / rden / row sums [3][L], gate scalars [2][4]
-  static constexpr int NF = DK + 128 * 8 + 2 * 6 * L + 3 * L + 8;
+  // n [DK], n partials [128*8], gate buffers [2][8][L], row sums / reciprocal denominators [2][L],
+  // gate scalars [2][8]
+  static constexpr int NF = DK + 128 * 8 + 2 * 8 * L + 2 * L + 16;
   static constexpr int BYTES = OF + NF * 4 + 1024;  // + alignment slack
 };
 
-// Per-chunk gate quantities (double-buffered).  b: inclusive cumulative log f; m: stabiliser
-// per token; sint = e^{b_t+m_c-m_t}; w = e^{g-b_s+itilde_s-m_next}; cs = (itilde_s - b_s) log2 e.
+// Per-chunk quantities (double-buffered), written by the producer except nq (state group).
+//   al, be : log2 row / column factors of P (fast: 0 and log2 u_s; guarded: (b_t - m_t) log2 e
+//            and X_s log2 e); be = -inf for tokens past the end
+//   u      : weight of v_s k_s in the update (and of k_s in the n update)
+//   E, F   : h_t = E_t H_t / max(|E_t rowsum_t + F_t nq_t|, e^{-m_t}),  nq_t = n_st . q_t
+//   emt    : e^{-m_t};  sq : Q scale of a guarded chunk
+//   scal   : [0] flags (bit 0 guarded, bit 1 rewrite C), [1] scale of the bf16 snapshot,
+//            [2] scale of the C rewrite, [3] scale of n before the n update,
+//            [4] e^{lam - m} after the chunk (final-state scale)
 struct GateBuf {
-  float* bl;
-  float* li;
-  float* mt;
-  float* sint;
-  float* wv;
-  float* cs;
-  float* scal;  // [0] decay a, [1] m_c, [2] m_next
+  float *al, *be, *u, *E, *F, *emt, *sq, *nq;
+  float* scal;
 };
+constexpr int GF_GUARD = 1, GF_STORE_C = 2;
 
 struct WalkBars {
-  uint64_t full[2], empty[2], gfull[2], gempty[2];
-  uint64_t s_full, s_empty, e1_done, vw_full, upd_done, q_ready, p_full, h_empty, mm_done, nq_done;
+  uint64_t full[2], empty[2], gfull[2], gempty[2], q_ready[2];
+  uint64_t s_full, s_empty, cb_ready, vw_full, upd_done, ro_done, p_full, h_empty, mm_done;
 };
 
 template <int DK, int DVT>
@@ -357,23 +425,23 @@ __global__ void __launch_bounds__(NTW, 1)
     tc_walk_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                    const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapH, TcParams p) {
   using SM = WalkSmem<DK, DVT>;
-  // TMEM columns: C fp32 [DK], bf16 copy of C as MMA operand [DK/2], S [64], H [64]
+  // TMEM columns: C fp32 [DK], bf16 snapshot of C as MMA operand [DK/2], S [64], H [64]
   constexpr uint32_t TM_C = 0, TM_CB = DK, TM_S = DK + DK / 2, TM_H = TM_S + 64;
   constexpr uint32_t TM_COLS = (TM_H + 64 <= 256) ? 256 : 512;
   constexpr float LOG2E = 1.4426950408889634f;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *Vw = sm + SM::OVW, *Ps = sm + SM::OP, *Hs = sm + SM::OH;
+  uint8_t *Vw = sm + SM::OVW, *Hs = sm + SM::OH;
   float* nvec = reinterpret_cast<float*>(sm + SM::OF);
   float* npart = nvec + DK;  // [128 * 8]
   float* gmem = npart + 128 * 8;
-  float* nq = gmem + 2 * 6 * L;
-  float* rden = nq + L;
-  float* rsum = rden + L;
-  float* gscal = rsum + L;  // [2][4]
+  float* rsum = gmem + 2 * 8 * L;
+  float* rden = rsum + L;
+  float* gscal = rden + L;  // [2][8]
   auto gbuf = [&](int b) {
-    float* base = gmem + b * 6 * L;
-    return GateBuf{base, base + L, base + 2 * L, base + 3 * L, base + 4 * L, base + 5 * L, gscal + 4 * b};
+    float* base = gmem + b * 8 * L;
+    return GateBuf{base,         base + L,     base + 2 * L, base + 3 * L, base + 4 * L,
+                   base + 5 * L, base + 6 * L, base + 7 * L, gscal + 8 * b};
   };
   __shared__ WalkBars bars;
   __shared__ uint32_t tmem_base;
@@ -382,7 +450,7 @@ __global__ void __launch_bounds__(NTW, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.x, g = blockIdx.y, slice = blockIdx.z;
-  const int blk = slice % p.nb, bh = slice / p.nb, head = bh % p.NH;
+  const int blk = slice % p.nb, bh = slice / p.nb;
   const int v0 = tile * DVT;
   const int seg_len = p.seg_chunks * L;
   const int T0 = g * seg_len, T1 = min(p.S, T0 + seg_len);
@@ -397,17 +465,17 @@ __global__ void __launch_bounds__(NTW, 1)
       mbar_init(&bars.empty[i], 3);
       mbar_init(&bars.gfull[i], 1);
       mbar_init(&bars.gempty[i], 2);
+      mbar_init(&bars.q_ready[i], 1);
     }
     mbar_init(&bars.s_full, 1);
     mbar_init(&bars.s_empty, 1);
-    mbar_init(&bars.e1_done, 1);
+    mbar_init(&bars.cb_ready, 1);
     mbar_init(&bars.vw_full, 1);
     mbar_init(&bars.upd_done, 1);
-    mbar_init(&bars.q_ready, 1);
+    mbar_init(&bars.ro_done, 1);
     mbar_init(&bars.p_full, 1);
     mbar_init(&bars.h_empty, 1);
     mbar_init(&bars.mm_done, 1);
-    mbar_init(&bars.nq_done, 1);
     abort_flag = 0;
     group_flag[0] = group_flag[1] = 0;
     fence_mbar_init();
@@ -421,7 +489,8 @@ __global__ void __launch_bounds__(NTW, 1)
   tc_fence_after();
   const uint32_t tm = tmem_base;
 
-  // ---- start state of the segment (see the file header); warps 0-7 fill TMEM and n
+  // ---- start state of the segment (see the file header); warps 0-7 fill TMEM and n.
+  // It is stabilised at m_start, so lam starts at m_start.
   float m_start = ret ? 0.f : (p.m0 ? p.m0[bh] : 0.f);
   const float m_init = m_start;
   float gsum = 0.f;
@@ -430,8 +499,8 @@ __global__ void __launch_bounds__(NTW, 1)
     if (!ret) m_start = fmaxf(A + m_start, Bm);
     gsum += A;
   }
-  if (warp < 8) {
-    const int quarter = warp & 3, half = warp >> 2;
+  if (warp >= 2) {
+    const int quarter = warp & 3, half = (warp - 2) >> 2;
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     const int row = acc_row<DVT>(quarter, lane);
     const float wc0 = expf(gsum + m_init - m_start);
@@ -471,7 +540,7 @@ __global__ void __launch_bounds__(NTW, 1)
     }
     tmem_wait_st();
     if (!ret)
-      for (int col = tid; col < DK; col += 256) {
+      for (int col = tid - 64; col < DK; col += 256) {
         float x = p.n0 ? wc0 * p.n0[(size_t)slice * p.dk + col] : 0.f;
         float after = gsum;
         for (int jg = 0; jg < g; ++jg) {
@@ -505,24 +574,28 @@ __global__ void __launch_bounds__(NTW, 1)
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
   };
 
-  if (warp == 9) {
+  if (warp == 0) {
     // =============================================================== producer
-    const float lg = ret ? retention_log_gamma(head) : 0.f;
-    float rfa = 0.f, ria = 0.f, rfb = 0.f, rib = 0.f;
+    // gate values of the next chunk are loaded into registers right after this chunk's
+    // hand-off, so their latency never sits in front of an mbarrier arrive
+    float pba = 0.f, pbb = 0.f, pxa = 0.f, pxb = 0.f, pca = 0.f, pcb = 0.f, pg = 0.f, pxm = 0.f;
     auto fetch_gates = [&](int c) {
-      const int t0 = T0 + c * L;
-      const int Lc = min(L, T1 - t0);
-      const size_t tok = (size_t)bh * p.S + t0;
-      const int ta = 2 * lane, tb = 2 * lane + 1;
-      if (!ret) {
-        rfa = ta < Lc ? p.fg[tok + ta] : 0.f;
-        ria = ta < Lc ? p.ig[tok + ta] : 0.f;
-        rfb = tb < Lc ? p.fg[tok + tb] : 0.f;
-        rib = tb < Lc ? p.ig[tok + tb] : 0.f;
-      }
+      const size_t r = (size_t)bh * p.sp + T0 + c * L + 2 * lane;
+      const float2 b2 = *reinterpret_cast<const float2*>(p.gb + r);
+      const float2 x2 = *reinterpret_cast<const float2*>(p.gx + r);
+      const float2 c2 = *reinterpret_cast<const float2*>(p.gxc + r);
+      const size_t cr = (size_t)bh * p.ncp + (size_t)g * p.seg_chunks + c;
+      pba = b2.x;
+      pbb = b2.y;
+      pxa = x2.x;
+      pxb = x2.y;
+      pca = c2.x;
+      pcb = c2.y;
+      pg = p.cg[cr];
+      pxm = p.cxm[cr];
     };
-    fetch_gates(0);
-    float mc = m_start;
+    if (nck > 0) fetch_gates(0);
+    float mc = m_start, lam = m_start;
     for (int c = 0; c < nck; ++c) {
       const int b = c & 1;
       // operands of chunk c into stage b once its previous user (chunk c-2) released it
@@ -538,90 +611,82 @@ __global__ void __launch_bounds__(NTW, 1)
         for (int j = 0; j < DVT / 64; ++j)
           tma_load_3d(base + SM::QB + SM::KB + j * 8192, &mapV, blk * p.dv + v0 + 64 * j, t0, bh, &bars.full[b]);
       }
-      // gate quantities of chunk c into buffer b
+      // gate quantities of chunk c into buffer b (lane: tokens 2 lane, 2 lane + 1)
       if (!warp_wait(&bars.gempty[b], ((c >> 1) & 1) ^ 1)) break;
       GateBuf G = gbuf(b);
-      const int t0 = T0 + c * L;
-      const int Lc = min(L, T1 - t0);
       const int ta = 2 * lane, tb = 2 * lane + 1;
-      float lfa, lia, lfb, lib;
-      if (ret) {
-        lfa = lfb = lg;
-        lia = lib = 0.f;
+      const float ba = pba, bb = pbb, xa = pxa, xb = pxb, gtot = pg, xmax = pxm;
+      // m_t = b_t + max(m_c, Xc_t): the stabiliser recurrence unrolled over the chunk
+      const float ma = ret ? 0.f : ba + fmaxf(mc, pca);
+      const float mb = ret ? 0.f : bb + fmaxf(mc, pcb);
+      const float mn = ret ? 0.f : gtot + fmaxf(mc, xmax);
+      const bool renorm = mc - lam > LAM_RENORM;
+      const float lam_eff = renorm ? mc : lam;
+      const bool guard = !ret && xmax - lam_eff > U_MAX_LOG;
+      float nu, csc, lam_next;
+      if (guard) {
+        nu = expf(lam - mc);
+        csc = expf(lam + gtot - mn);
+        lam_next = mn;
       } else {
-        lfa = ta < Lc ? log_sigmoid(rfa) : 0.f;
-        lia = ta < Lc ? ria : -INFINITY;
-        lfb = tb < Lc ? log_sigmoid(rfb) : 0.f;
-        lib = tb < Lc ? rib : -INFINITY;
+        nu = renorm ? expf(lam - mc) : 1.f;
+        csc = nu;
+        lam_next = lam_eff + gtot;
       }
-      if (c + 1 < nck) fetch_gates(c + 1);
-      float isum = lfa + lfb;
-      MaxPlus imp = mp_then(MaxPlus{lfa, lia}, MaxPlus{lfb, lib});
+      // tokens past the end have X = -inf: weight 0, column factor 0
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float us = __shfl_up_sync(0xffffffffu, isum, o);
-        const MaxPlus um{__shfl_up_sync(0xffffffffu, imp.A, o), __shfl_up_sync(0xffffffffu, imp.Bm, o)};
-        if (lane >= o) {
-          isum += us;
-          imp = mp_then(um, imp);
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int t = h2 ? tb : ta;
+        const float bt = h2 ? bb : ba, mt = h2 ? mb : ma, xt = h2 ? xb : xa;
+        if (guard) {
+          const float sint = expf(bt + mc - mt);
+          G.al[t] = (bt - mt) * LOG2E;
+          G.be[t] = xt * LOG2E;
+          G.u[t] = expf(gtot + xt - mn);
+          G.E[t] = 1.f;
+          G.F[t] = sint * nu;
+          G.sq[t] = sint;
+        } else {
+          const float et = expf(bt + lam_eff - mt);
+          G.al[t] = 0.f;
+          G.be[t] = (xt - lam_eff) * LOG2E;
+          G.u[t] = expf(xt - lam_eff);
+          G.E[t] = et;
+          G.F[t] = et * nu;
+          G.sq[t] = 1.f;
         }
+        G.emt[t] = expf(-mt);
       }
-      float esum = __shfl_up_sync(0xffffffffu, isum, 1);
-      MaxPlus emp{__shfl_up_sync(0xffffffffu, imp.A, 1), __shfl_up_sync(0xffffffffu, imp.Bm, 1)};
       if (lane == 0) {
-        esum = 0.f;
-        emp = MaxPlus{0.f, -INFINITY};
-      }
-      const float ba = esum + lfa, bb = esum + lfa + lfb;
-      float ma = 0.f, mb = 0.f;
-      if (!ret) {
-        const MaxPlus pa = mp_then(emp, MaxPlus{lfa, lia});
-        ma = mp_apply(pa, mc);
-        mb = mp_apply(mp_then(pa, MaxPlus{lfb, lib}), mc);
-      }
-      const float lia_ = ret ? 0.f : lia, lib_ = ret ? 0.f : lib;
-      const int lt = (Lc - 1) >> 1;
-      const float gtot = __shfl_sync(0xffffffffu, ((Lc - 1) & 1) ? bb : ba, lt);
-      const float mn = __shfl_sync(0xffffffffu, ((Lc - 1) & 1) ? mb : ma, lt);
-      G.bl[ta] = ba;
-      G.bl[tb] = bb;
-      G.li[ta] = lia_;
-      G.li[tb] = lib_;
-      G.mt[ta] = ma;
-      G.mt[tb] = mb;
-      G.sint[ta] = expf(ba + mc - ma);
-      G.sint[tb] = expf(bb + mc - mb);
-      G.wv[ta] = ta < Lc ? expf(gtot - ba + lia_ - mn) : 0.f;
-      G.wv[tb] = tb < Lc ? expf(gtot - bb + lib_ - mn) : 0.f;
-      G.cs[ta] = ta < Lc ? (lia_ - ba) * LOG2E : -INFINITY;
-      G.cs[tb] = tb < Lc ? (lib_ - bb) * LOG2E : -INFINITY;
-      if (lane == 0) {
-        G.scal[0] = expf(gtot + mc - mn);
-        G.scal[1] = mc;
-        G.scal[2] = mn;
+        G.scal[0] = __int_as_float((guard ? GF_GUARD : 0) | ((guard || renorm) ? GF_STORE_C : 0));
+        G.scal[1] = nu;
+        G.scal[2] = csc;
+        G.scal[3] = csc;
+        G.scal[4] = expf(lam_next - mn);
       }
       mc = mn;
+      lam = lam_next;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.gfull[b]);
+      if (c + 1 < nck) fetch_gates(c + 1);
     }
     if (lane == 0 && !abort_flag && last_seg && !ret && tile == 0 && blk == 0 && p.m_out) p.m_out[bh] = mc;
-  } else if (warp == 8) {
+  } else if (warp == 1) {
     // =============================================================== MMA issue
+    // per chunk: update (C += (V o u)^T K), read-out (H = Cb Q^T), next chunk's S = Q K^T,
+    // then P V (H += V^T P^T).  The update and read-out are the chunk recurrence.
     const uint32_t id_s = idesc_bf16(64, 64, 0, 0);
     const uint32_t id_ro = idesc_bf16(DVT, 64, 0, 0);
     const uint32_t id_pv = idesc_bf16(DVT, 64, 1, 0);
     const uint32_t id_up = idesc_bf16(DVT, DK, 1, 1);
     const uint64_t ps_k = smem_desc_sw128(sm_u + SM::OP, 16, 1024);       // P, K-major rows t
-    const uint64_t vw_mn = smem_desc_sw128(sm_u + SM::OVW, 8192, 1024);  // V o w, MN-major
-    for (int c = 0; c < nck; ++c) {
+    const uint64_t vw_mn = smem_desc_sw128(sm_u + SM::OVW, 8192, 1024);  // V o u, MN-major
+    auto issue_s = [&](int c) -> bool {
       const int b = c & 1;
-      const uint32_t q_u = sm_u + b * SM::STAGE, k_u = q_u + SM::QB, v_u = k_u + SM::KB;
-      const uint64_t q_k = smem_desc_sw128(q_u, 16, 1024);     // Q (or scaled Q), K-major rows t
-      const uint64_t k_k = smem_desc_sw128(k_u, 16, 1024);     // K, K-major rows s
-      const uint64_t k_mn = smem_desc_sw128(k_u, 8192, 1024);  // K, MN-major (rows s = K dim)
-      const uint64_t v_mn = smem_desc_sw128(v_u, 8192, 1024);  // V, MN-major
-      if (!warp_wait(&bars.full[b], (c >> 1) & 1)) break;
-      if (c > 0 && !warp_wait(&bars.s_empty, (c - 1) & 1)) break;
+      const uint64_t q_k = smem_desc_sw128(sm_u + b * SM::STAGE, 16, 1024);
+      const uint64_t k_k = smem_desc_sw128(sm_u + b * SM::STAGE + SM::QB, 16, 1024);
+      if (!warp_wait(&bars.full[b], (c >> 1) & 1)) return false;
+      if (c > 0 && !warp_wait(&bars.s_empty, (c - 1) & 1)) return false;
       tc_fence_after();
       if (elect_one()) {
 #pragma unroll
@@ -632,77 +697,102 @@ __global__ void __launch_bounds__(NTW, 1)
         mma_commit(&bars.s_full);
       }
       __syncwarp();
-      if (!warp_wait(&bars.e1_done, c & 1)) break;
-      if (!warp_wait(&bars.vw_full, c & 1)) break;
-      tc_fence_after();
-      if (elect_one()) {
+      return true;
+    };
+    if (nck > 0 && issue_s(0))
+      for (int c = 0; c < nck; ++c) {
+        const int b = c & 1;
+        const uint32_t q_u = sm_u + b * SM::STAGE, k_u = q_u + SM::QB, v_u = k_u + SM::KB;
+        const uint64_t q_k = smem_desc_sw128(q_u, 16, 1024);     // Q, K-major rows t
+        const uint64_t k_mn = smem_desc_sw128(k_u, 8192, 1024);  // K, MN-major (rows s = K dim)
+        const uint64_t v_mn = smem_desc_sw128(v_u, 8192, 1024);  // V, MN-major
+        if (!warp_wait(&bars.cb_ready, c & 1)) break;
+        if (!warp_wait(&bars.vw_full, c & 1)) break;
+        tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int ks = 0; ks < L / 16; ++ks)
-          mma_bf16_ss(tm + TM_C, vw_mn + (uint64_t)(ks * 128), k_mn + (uint64_t)(ks * 128), id_up, 1u);
-        mma_commit(&bars.upd_done);
-      }
-      __syncwarp();
-      if (!warp_wait(&bars.q_ready, c & 1)) break;
-      if (c > 0 && !warp_wait(&bars.h_empty, (c - 1) & 1)) break;
-      tc_fence_after();
-      if (elect_one()) {
+          for (int ks = 0; ks < L / 16; ++ks)
+            mma_bf16_ss(tm + TM_C, vw_mn + (uint64_t)(ks * 128), k_mn + (uint64_t)(ks * 128), id_up, 1u);
+          mma_commit(&bars.upd_done);
+        }
+        __syncwarp();
+        if (!warp_wait(&bars.q_ready[b], (c >> 1) & 1)) break;
+        if (c > 0 && !warp_wait(&bars.h_empty, (c - 1) & 1)) break;
+        tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int k = 0; k < DK; k += 16)
-          mma_bf16_ts(tm + TM_H, tm + TM_CB + k / 2, q_k + (uint64_t)(((k >> 6) * 8192 + (k & 63) * 2) >> 4), id_ro,
-                      k > 0 ? 1u : 0u);
-      }
-      __syncwarp();
-      if (!warp_wait(&bars.p_full, c & 1)) break;
-      tc_fence_after();
-      if (elect_one()) {
+          for (int k = 0; k < DK; k += 16)
+            mma_bf16_ts(tm + TM_H, tm + TM_CB + k / 2, q_k + (uint64_t)(((k >> 6) * 8192 + (k & 63) * 2) >> 4),
+                        id_ro, k > 0 ? 1u : 0u);
+          mma_commit(&bars.ro_done);
+        }
+        __syncwarp();
+        if (c + 1 < nck && !issue_s(c + 1)) break;
+        if (!warp_wait(&bars.p_full, c & 1)) break;
+        tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int ks = 0; ks < L / 16; ++ks)
-          mma_bf16_ss(tm + TM_H, v_mn + (uint64_t)(ks * 128), ps_k + (uint64_t)(ks * 2), id_pv, 1u);
-        mma_commit(&bars.mm_done);
-        mma_commit(&bars.empty[b]);
+          for (int ks = 0; ks < L / 16; ++ks)
+            mma_bf16_ss(tm + TM_H, v_mn + (uint64_t)(ks * 128), ps_k + (uint64_t)(ks * 2), id_pv, 1u);
+          mma_commit(&bars.mm_done);
+          mma_commit(&bars.empty[b]);
+        }
+        __syncwarp();
       }
-      __syncwarp();
-    }
-  } else if (warp < 4) {
+  } else if (warp < 6) {
     // =============================================================== state group
-    const int quarter = warp;
+    const int quarter = warp & 3;
+    const int st = tid - 64;  // 0..127
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
-    const bool first = tid == 0;
+    const bool first = st == 0;
+    float fin = 1.f;
     for (int c = 0; c < nck; ++c) {
       const int b = c & 1;
       const GateBuf G = gbuf(b);
       uint8_t* Qs = sm + b * SM::STAGE;
       uint8_t* Ks = Qs + SM::QB;
       if (!group_wait(&bars.gfull[b], (c >> 1) & 1, 0, first)) break;
-      if (c > 0 && !group_wait(&bars.mm_done, (c - 1) & 1, 0, first)) break;
+      // the previous read-out has read the snapshot and the previous update has written C
+      if (c > 0 && !group_wait(&bars.ro_done, (c - 1) & 1, 0, first)) break;
       tc_fence_after();
-      // C round trip: bf16 copy of C_c into TMEM (read-out operand), C <- a C
+      const int flags = __float_as_int(G.scal[0]);
+      fin = G.scal[4];
       {
-        const float a = G.scal[0];
-        for (int c0 = 0; c0 < DK; c0 += 32) {
-          float r[32];
-          tmem_ld32(tm + lane_off + TM_C + c0, r);
+        // bf16 snapshot of (scaled) C into TMEM; C itself rewritten only when lam moves
+        const float cbs = G.scal[1], csc = G.scal[2];
+        const bool store_c = (flags & GF_STORE_C) != 0;
+#pragma unroll 1
+        for (int c0 = 0; c0 < DK; c0 += 64) {
+          float r[64];
+          tmem_ld32(tm + lane_off + TM_C + c0, *reinterpret_cast<float(*)[32]>(r));
+          tmem_ld32(tm + lane_off + TM_C + c0 + 32, *reinterpret_cast<float(*)[32]>(r + 32));
           tmem_wait_ld();
           float pk[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) pk[j] = __uint_as_float(pack_bf16(r[2 * j], r[2 * j + 1]));
-          tmem_st16(tm + lane_off + TM_CB + c0 / 2, pk);
+          for (int h2 = 0; h2 < 2; ++h2) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) pk[j] = r[j] * a;
-          tmem_st16(tm + lane_off + TM_C + c0, pk);
+            for (int j = 0; j < 16; ++j)
+              pk[j] = __uint_as_float(pack_bf16(r[32 * h2 + 2 * j] * cbs, r[32 * h2 + 2 * j + 1] * cbs));
+            tmem_st16(tm + lane_off + TM_CB + c0 / 2 + 16 * h2, pk);
+          }
+          if (store_c) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) pk[j] = r[16 + j] * a;
-          tmem_st16(tm + lane_off + TM_C + c0 + 16, pk);
+            for (int h4 = 0; h4 < 4; ++h4) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) pk[j] = r[16 * h4 + j] * csc;
+              tmem_st16(tm + lane_off + TM_C + c0 + 16 * h4, pk);
+            }
+          }
         }
         tmem_wait_st();
       }
       tc_fence_before();
       named_bar(WG_STATE, 128);
-      if (first) mbar_arrive(&bars.e1_done);
+      if (first) mbar_arrive(&bars.cb_ready);
       if (!group_wait(&bars.full[b], (c >> 1) & 1, 0, first)) break;
       if (!ret) {
-        // n . q_t: two threads per token, DK/2 columns each (loads batched)
-        const int t = tid >> 1, part = tid & 1;
+        // nq_t = n_st . q_t: two threads per token, DK/2 columns each (loads batched)
+        const int t = st >> 1, part = st & 1;
         const uint32_t qs_u = smem_u32(Qs);
         constexpr int NCH = DK / 16;
         constexpr int BATCH = NCH < 8 ? NCH : 8;
@@ -733,15 +823,12 @@ __global__ void __launch_bounds__(NTW, 1)
         }
         float a = a0 + a1;
         a += __shfl_xor_sync(0xffffffffu, a, 1);
-        if (part == 0) nq[t] = a;
+        if (part == 0) G.nq[t] = a;
       }
-      named_bar(WG_STATE, 128);
-      if (first) mbar_arrive(&bars.nq_done);
-      // Q <- e^{b_t+m_c-m_t} Q once the S MMA has read the raw Q (read-out and intra-chunk
-      // then share one accumulator)
-      if (!group_wait(&bars.s_full, c & 1, 0, first)) break;
-      {
-        const int gt = tid;
+      if (flags & GF_GUARD) {
+        // guarded chunk: Q <- e^{b_t+m_c-m_t} Q once the S MMA has read the raw Q
+        if (!group_wait(&bars.s_full, c & 1, 0, first)) break;
+        const int gt = st;
         constexpr int NQ = L * (DK / 8) / 128;  // 16-byte chunks per thread
         constexpr int BATCH = NQ < 8 ? NQ : 8;
         const uint32_t qs_u = smem_u32(Qs);
@@ -756,19 +843,19 @@ __global__ void __launch_bounds__(NTW, 1)
             const int row = i / (DK / 8), ch = i % (DK / 8);
             offs[k] = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
             u[k] = ld_shared_v4(qs_u + offs[k]);
-            wr[k] = G.sint[row];
+            wr[k] = G.sq[row];
           }
 #pragma unroll
           for (int k = 0; k < BATCH; ++k) st_shared_v4u(qs_u + offs[k], scale_bf16x8(u[k], wr[k]));
         }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
       named_bar(WG_STATE, 128);
-      if (first) mbar_arrive(&bars.q_ready);
+      if (first) mbar_arrive(&bars.q_ready[b]);
       if (!ret) {
-        // n <- a n + sum_s w_s k_s
+        // n <- ns n + sum_s u_s k_s
         constexpr int NCG = DK / 8, NRG = 128 / NCG, RPG = L / NRG;
-        const int cg = tid % NCG, rg = tid / NCG;
+        const int cg = st % NCG, rg = st / NCG;
         const int col = 8 * cg;
         const uint8_t* kt = Ks + (col >> 6) * 8192;
         float acc[8];
@@ -779,7 +866,7 @@ __global__ void __launch_bounds__(NTW, 1)
           const int srow = rg * RPG + j;
           const uint4 u = *reinterpret_cast<const uint4*>(kt + sw128_offset(srow, col & 63));
           const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-          const float w = G.wv[srow];
+          const float w = G.u[srow];
 #pragma unroll
           for (int q2 = 0; q2 < 4; ++q2) {
             const float2 f = __bfloat1622float2(b2[q2]);
@@ -787,15 +874,15 @@ __global__ void __launch_bounds__(NTW, 1)
             acc[2 * q2 + 1] += w * f.y;
           }
         }
-        *reinterpret_cast<float4*>(npart + tid * 8) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        *reinterpret_cast<float4*>(npart + tid * 8 + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        *reinterpret_cast<float4*>(npart + st * 8) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4*>(npart + st * 8 + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
         named_bar(WG_STATE, 128);
-        const float a = G.scal[0];
-        for (int cc = tid; cc < DK; cc += 128) {
+        const float ns = G.scal[3];
+        for (int cc = st; cc < DK; cc += 128) {
           float x = 0.f;
 #pragma unroll
           for (int r = 0; r < NRG; ++r) x += npart[(r * NCG + cc / 8) * 8 + (cc & 7)];
-          nvec[cc] = a * nvec[cc] + x;
+          nvec[cc] = ns * nvec[cc] + x;
         }
       }
       named_bar(WG_STATE, 128);
@@ -804,8 +891,10 @@ __global__ void __launch_bounds__(NTW, 1)
         mbar_arrive(&bars.gempty[b]);
       }
     }
-    // final state after the last update
-    if (group_wait(&bars.mm_done, (nck - 1) & 1, 0, first) && last_seg) {
+    // final state after the last update, back in units of e^{m}.  The wait is on ro_done,
+    // whose every phase this group has waited for: a parity wait on a barrier two phases
+    // behind would return at once.
+    if (nck > 0 && group_wait(&bars.ro_done, (nck - 1) & 1, 0, first) && last_seg) {
       tc_fence_after();
       const int row = acc_row<DVT>(quarter, lane);
       if (p.C_out)
@@ -817,52 +906,54 @@ __global__ void __launch_bounds__(NTW, 1)
             float* dst = p.C_out + ((size_t)slice * p.dv + v0 + row) * p.dk + c0;
 #pragma unroll
             for (int j = 0; j < 32; j += 4)
-              *reinterpret_cast<float4*>(dst + j) = make_float4(r[j], r[j + 1], r[j + 2], r[j + 3]);
+              *reinterpret_cast<float4*>(dst + j) =
+                  make_float4(fin * r[j], fin * r[j + 1], fin * r[j + 2], fin * r[j + 3]);
           }
         }
       if (!ret && tile == 0 && p.n_out)
-        for (int col = tid; col < DK; col += 128) p.n_out[(size_t)slice * p.dk + col] = nvec[col];
+        for (int col = st; col < DK; col += 128) p.n_out[(size_t)slice * p.dk + col] = fin * nvec[col];
     }
   } else {
     // =============================================================== output group
-    const int quarter = warp - 4;
-    const int gt = tid - 128;  // 0..127
+    const int quarter = warp & 3;
+    const int gt = tid - 192;  // 0..127
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     const bool first = gt == 0;
     const uint32_t ps_u = sm_u + SM::OP;
-    for (int c = 0; c < nck; ++c) {
+    // V o u of chunk c into the update operand buffer (loads batched ahead of the stores)
+    auto scale_v = [&](int c) {
+      const GateBuf G = gbuf(c & 1);
+      const uint32_t vs_u = sm_u + (c & 1) * SM::STAGE + SM::QB + SM::KB, vw_u2 = smem_u32(Vw);
+      constexpr int NV = L * (DVT / 8) / 128;  // 16-byte chunks per thread
+      uint4 u[NV];
+      float wr[NV];
+      int offs[NV];
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        const int i = k * 128 + gt;
+        const int row = i / (DVT / 8), ch = i % (DVT / 8);
+        offs[k] = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
+        u[k] = ld_shared_v4(vs_u + offs[k]);
+        wr[k] = G.u[row];
+      }
+#pragma unroll
+      for (int k = 0; k < NV; ++k) st_shared_v4u(vw_u2 + offs[k], scale_bf16x8(u[k], wr[k]));
+      fence_proxy_async_smem();
+    };
+    bool ok = nck > 0 && group_wait(&bars.gfull[0], 0, 1, first) && group_wait(&bars.full[0], 0, 1, first);
+    if (ok) {
+      scale_v(0);
+      named_bar(WG_OUT, 128);
+      if (first) mbar_arrive(&bars.vw_full);
+    }
+    for (int c = 0; ok && c < nck; ++c) {
       const int b = c & 1;
       const GateBuf G = gbuf(b);
       const int t0 = T0 + c * L;
       const int Lc = min(L, T1 - t0);
       const size_t tok0 = (size_t)bh * p.S + t0;
-      uint8_t* Qs = sm + b * SM::STAGE;
-      uint8_t* Vs = Qs + SM::QB + SM::KB;
-      if (!group_wait(&bars.gfull[b], (c >> 1) & 1, 1, first)) break;
-      if (!group_wait(&bars.full[b], (c >> 1) & 1, 1, first)) break;
-      if (c > 0 && !group_wait(&bars.upd_done, (c - 1) & 1, 1, first)) break;
-      // V o w for the state update (loads batched ahead of the stores)
-      {
-        constexpr int NV = L * (DVT / 8) / 128;  // 16-byte chunks per thread
-        const uint32_t vs_u = smem_u32(Vs), vw_u2 = smem_u32(Vw);
-        uint4 u[NV];
-        float wr[NV];
-        int offs[NV];
-#pragma unroll
-        for (int k = 0; k < NV; ++k) {
-          const int i = k * 128 + gt;
-          const int row = i / (DVT / 8), ch = i % (DVT / 8);
-          offs[k] = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
-          u[k] = ld_shared_v4(vs_u + offs[k]);
-          wr[k] = G.wv[row];
-        }
-#pragma unroll
-        for (int k = 0; k < NV; ++k) st_shared_v4u(vw_u2 + offs[k], scale_bf16x8(u[k], wr[k]));
-      }
-      fence_proxy_async_smem();
-      named_bar(WG_OUT, 128);
-      if (first) mbar_arrive(&bars.vw_full);
-      // P = S o D' (bf16, rows t) and its row sums; P V of the previous chunk must be done
+      // P = S o e^{al_t + be_s} (bf16, rows t) and its row sums; P V of the previous chunk
+      // must be done with the P buffer
       if (c > 0 && !group_wait(&bars.mm_done, (c - 1) & 1, 1, first)) break;
       if (!group_wait(&bars.s_full, c & 1, 1, first)) break;
       tc_fence_after();
@@ -873,19 +964,22 @@ __global__ void __launch_bounds__(NTW, 1)
         tmem_ld16x256_x8(tm + lane_off + TM_S, r);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          csr[2 * j] = G.cs[8 * j + cp];
-          csr[2 * j + 1] = G.cs[8 * j + cp + 1];
+          csr[2 * j] = G.be[8 * j + cp];
+          csr[2 * j + 1] = G.be[8 * j + cp + 1];
         }
-        const float ct_lo = (G.bl[r_lo] - G.mt[r_lo]) * LOG2E, ct_hi = (G.bl[r_hi] - G.mt[r_hi]) * LOG2E;
+        const float al_lo = G.al[r_lo], al_hi = G.al[r_hi];
         tmem_wait_ld();
+        tc_fence_before();
+        named_bar(WG_OUT, 128);
+        if (first) mbar_arrive(&bars.s_empty);
         float rs_lo = 0.f, rs_hi = 0.f;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int s0 = 8 * j + cp;
-          const float a0 = (s0 <= r_lo && r_lo < Lc) ? r[2 * j] * exp2f(ct_lo + csr[2 * j]) : 0.f;
-          const float a1 = (s0 + 1 <= r_lo && r_lo < Lc) ? r[2 * j + 1] * exp2f(ct_lo + csr[2 * j + 1]) : 0.f;
-          const float b0 = (s0 <= r_hi && r_hi < Lc) ? r[16 + 2 * j] * exp2f(ct_hi + csr[2 * j]) : 0.f;
-          const float b1 = (s0 + 1 <= r_hi && r_hi < Lc) ? r[16 + 2 * j + 1] * exp2f(ct_hi + csr[2 * j + 1]) : 0.f;
+          const float a0 = (s0 <= r_lo && r_lo < Lc) ? r[2 * j] * exp2f(al_lo + csr[2 * j]) : 0.f;
+          const float a1 = (s0 + 1 <= r_lo && r_lo < Lc) ? r[2 * j + 1] * exp2f(al_lo + csr[2 * j + 1]) : 0.f;
+          const float b0 = (s0 <= r_hi && r_hi < Lc) ? r[16 + 2 * j] * exp2f(al_hi + csr[2 * j]) : 0.f;
+          const float b1 = (s0 + 1 <= r_hi && r_hi < Lc) ? r[16 + 2 * j + 1] * exp2f(al_hi + csr[2 * j + 1]) : 0.f;
           rs_lo += a0 + a1;
           rs_hi += b0 + b1;
           asm volatile("st.shared.b32 [%0], %1;" ::"r"(ps_u + sw128_offset(r_lo, s0)), "r"(pack_bf16(a0, a1)) : "memory");
@@ -901,19 +995,28 @@ __global__ void __launch_bounds__(NTW, 1)
         }
       }
       fence_proxy_async_smem();
-      tc_fence_before();
       named_bar(WG_OUT, 128);
-      if (first) mbar_arrive(&bars.s_empty);
       if (first) mbar_arrive(&bars.p_full);
-      // denominators (need n . q_t from the state group)
-      if (!group_wait(&bars.nq_done, c & 1, 1, first)) break;
+      // V o u of the next chunk once this chunk's update has read the buffer
+      if (c + 1 < nck) {
+        const int b1 = (c + 1) & 1;
+        if (!group_wait(&bars.gfull[b1], ((c + 1) >> 1) & 1, 1, first)) break;
+        if (!group_wait(&bars.full[b1], ((c + 1) >> 1) & 1, 1, first)) break;
+        if (!group_wait(&bars.upd_done, c & 1, 1, first)) break;
+        scale_v(c + 1);
+        named_bar(WG_OUT, 128);
+        if (first) mbar_arrive(&bars.vw_full);
+      }
+      // reciprocal denominators times the output scale E_t (nq_t from the state group)
+      if (!group_wait(&bars.q_ready[b], (c >> 1) & 1, 1, first)) break;
       if (gt < L) {
         const int t = gt;
-        rden[t] = ret ? 1.f : 1.f / fmaxf(fabsf(rsum[t] + G.sint[t] * nq[t]), expf(-G.mt[t]));
+        const float e = G.E[t];
+        rden[t] = ret ? e : e / fmaxf(fabsf(e * rsum[t] + G.F[t] * G.nq[t]), G.emt[t]);
       }
       named_bar(WG_OUT, 128);
       if (first) mbar_arrive(&bars.empty[b]);
-      // h_t = H_t / den_t (x o_t): stage the tile in shared memory, TMA store
+      // h_t = H_t rden_t (x o_t): H leaves TMEM first, then the tile is staged and TMA-stored
       if (first) bulk_wait_read_all();
       if (!group_wait(&bars.mm_done, c & 1, 1, first)) break;
       tc_fence_after();
@@ -922,13 +1025,18 @@ __global__ void __launch_bounds__(NTW, 1)
         const int rr = row >= 0 ? row : 0;
         const uint32_t hb_u = smem_u32(Hs) + (rr >> 6) * 8192 + (rr & 63) * 2;
         const size_t hcol = (size_t)blk * p.dv + v0 + rr;
-        float r[32], rd[32];
+        float r[64];
+        tmem_ld32(tm + lane_off + TM_H, *reinterpret_cast<float(*)[32]>(r));
+        tmem_ld32(tm + lane_off + TM_H + 32, *reinterpret_cast<float(*)[32]>(r + 32));
+        tmem_wait_ld();
+        tc_fence_before();
+        named_bar(WG_OUT, 128);
+        if (first) mbar_arrive(&bars.h_empty);
 #pragma unroll
         for (int tt = 0; tt < L; tt += 32) {
-          tmem_ld32(tm + lane_off + TM_H + tt, r);
+          float rd[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) rd[j] = rden[tt + j];
-          tmem_wait_ld();
           if (p.og && !ret) {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
@@ -936,15 +1044,14 @@ __global__ void __launch_bounds__(NTW, 1)
           }
           if (row >= 0) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) st_shared_b16(hb_u + (tt + j) * 128, __float2bfloat16_rn(r[j] * rd[j]));
+            for (int j = 0; j < 32; ++j)
+              st_shared_b16(hb_u + (tt + j) * 128, __float2bfloat16_rn(r[tt + j] * rd[j]));
           }
         }
       }
-      tc_fence_before();
       fence_proxy_async_smem();
       named_bar(WG_OUT, 128);
       if (first) {
-        mbar_arrive(&bars.h_empty);
         for (int j = 0; j < DVT / 64; ++j) tma_store_3d(&mapH, Hs + j * 8192, blk * p.dv + v0 + 64 * j, t0, bh);
         bulk_commit();
         mbar_arrive(&bars.gempty[b]);
@@ -998,6 +1105,9 @@ size_t tc_workspace_bytes(const TcPlan& pl, long long BH, int nb, int dk, int dv
   off += ((size_t)slices * G1 * dv * dk * 4 + 255) / 256 * 256;
   off += ((size_t)slices * G1 * dk * 4 + 255) / 256 * 256;
   off += 2 * (((size_t)BH * G1 * 4 + 255) / 256 * 256);
+  const size_t ncp = (size_t)pl.G * pl.seg_chunks, sp = ncp * L;
+  off += 3 * (((size_t)BH * sp * 4 + 255) / 256 * 256);
+  off += 2 * (((size_t)BH * ncp * 4 + 255) / 256 * 256);
   return off;
 }
 
@@ -1006,8 +1116,12 @@ static cudaError_t launch_tc_dk(const TcPlan& pl, const TcParams& prm, const CUt
                                 const CUtensorMap& mv, const CUtensorMap& mh, long long slices, cudaStream_t stream,
                                 cudaEvent_t ev0, cudaEvent_t ev1) {
   cudaError_t e;
+  const long long BH = slices / prm.nb;
+  tc_gate_prep_kernel<<<(unsigned)((BH * prm.ncp + 7) / 8), 256, 0, stream>>>(prm, (int)BH);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   if (pl.G > 1) {
-    const int smemA = 3 * (DK * 128 + DVT * 128) + (NT * 8 + pl.seg_chunks * L) * 4 + 1024;
+    const int smemA = 3 * (DK * 128 + DVT * 128) + (NT * 8 + pl.seg_chunks * L + pl.seg_chunks) * 4 + 1024;
     e = cudaFuncSetAttribute(tc_segment_kernel<DK, DVT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemA);
     if (e != cudaSuccess) return e;
     dim3 gridA(pl.n_tiles, pl.G - 1, (unsigned)slices);
@@ -1069,6 +1183,14 @@ cudaError_t launch_tc(const WalkArgs& a, const TcPlan& pl, void* ws, cudaStream_
   prm.segA = reinterpret_cast<float*>(w + off);
   off += ((size_t)BH * G1 * 4 + 255) / 256 * 256;
   prm.segB = reinterpret_cast<float*>(w + off);
+  off += ((size_t)BH * G1 * 4 + 255) / 256 * 256;
+  prm.ncp = pl.G * pl.seg_chunks;
+  prm.sp = prm.ncp * L;
+  float** planes[5] = {&prm.gb, &prm.gx, &prm.gxc, &prm.cg, &prm.cxm};
+  for (int i = 0; i < 5; ++i) {
+    *planes[i] = reinterpret_cast<float*>(w + off);
+    off += ((size_t)BH * (i < 3 ? prm.sp : prm.ncp) * 4 + 255) / 256 * 256;
+  }
   cudaError_t e = cudaMemsetAsync(w, 0, 4, stream);
   if (e != cudaSuccess) return e;
   if (a.dk == 256 && pl.dvt == 128) return launch_tc_dk<256, 128>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);

@@ -265,7 +265,7 @@ mlstm_status_t mlstm_fwd_chunkwise_plan(const mlstm_fwd_params_t* p, mlstm_fwd_p
     plan->segments = s.tcp.G;
     plan->dv_tile = s.tcp.dvt;
     plan->ctas_main = (int)(s.tcp.n_tiles * s.tcp.G * s.BH * s.nb);
-    plan->kernels = (s.BH == 0 || s.S == 0) ? 0 : (s.tcp.G > 1 ? 2 : 1);
+    plan->kernels = (s.BH == 0 || s.S == 0) ? 0 : (s.tcp.G > 1 ? 3 : 2);
     plan->workspace_bytes = fwd_layout(s).total;
     return MLSTM_OK;
   }

@@ -325,3 +325,43 @@ def test_tensor_core_state_in_place_across_segments():
     torch.cuda.synchronize()
     ref = oracle_fwd(inp, C0=C0, n0=n0, m0=m0)
     check((host(h), host(C), host(n), host(m)), ref, "bf16", what="tc in place")
+
+
+# Gate regimes for the tensor-core walk: the state is kept in a lazily scaled form and a
+# chunk whose input gate rises far above the running stabiliser is evaluated in the
+# per-element stabilised form.  q, k >= 0 keep n.q a sum of positive terms (see
+# test_large_input_gates_stay_finite), so the comparison measures the stabilisation.
+GATE_REGIMES = {
+    "spikes_80": dict(spikes=80.0),         # isolated input gates 80 above the rest
+    "spikes_40": dict(spikes=40.0),         # large but within the lazily scaled range
+    "shift_60": dict(shift=60.0),           # every input gate 60 above the initial stabiliser
+    "steep_forget": dict(fmean=-1.0),       # log f ~ -1.3 per token: ~-80 per chunk
+    "flat_forget": dict(fmean=8.0),         # f ~ 1: the scale barely moves
+    "negative_input": dict(shift=-30.0),    # input gates far below the carried state
+}
+
+
+@pytest.mark.parametrize("regime", list(GATE_REGIMES))
+def test_tensor_core_gate_regimes(regime):
+    cfg = GATE_REGIMES[regime]
+    B, NH, S, DHQK, DHV = 1, 2, 1536, 128, 128
+    w = inputs.Workload(3, "regime", B, NH, S, DHQK, DHV, 64, 1, "bf16", False, 1 / np.sqrt(DHQK))
+    assert mlstm.plan(mlstm.fwd_params(B, NH, S, DHQK, DHV, 64, 1, torch.bfloat16, False))["tensor_core"] == 1
+    inp = inputs.forward_inputs(w, seed=31)
+    inp["q"], inp["k"] = np.abs(inp["q"]), np.abs(inp["k"])
+    rng = np.random.default_rng(32)
+    if "spikes" in cfg:
+        idx = rng.choice(S, size=12, replace=False)
+        inp["igate"][:, :, idx] += cfg["spikes"]
+    if "shift" in cfg:
+        inp["igate"] = inp["igate"] + cfg["shift"]
+    if "fmean" in cfg:
+        inp["fgate"] = inp["fgate"] - 3.0 + cfg["fmean"]
+    rs = np.random.default_rng(33)
+    C0 = (rs.standard_normal((B, NH, 1, DHV, DHQK)) * 0.2).astype(np.float32)
+    n0 = np.abs(rs.standard_normal((B, NH, 1, DHQK)) * 0.2).astype(np.float32)
+    m0 = rs.standard_normal((B, NH)).astype(np.float32)
+    got = gpu_fwd(inp, "bf16", 64, C0=C0, n0=n0, m0=m0)
+    assert all(np.all(np.isfinite(x)) for x in got), regime
+    errs = check(got, oracle_fwd(inp, C0=C0, n0=n0, m0=m0), "bf16", what=regime)
+    print(regime, errs)
