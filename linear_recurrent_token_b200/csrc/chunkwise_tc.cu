@@ -73,9 +73,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
 }
-__device__ __forceinline__ void st_shared_b16(uint32_t addr, __nv_bfloat16 v) {
-  asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(*reinterpret_cast<uint16_t*>(&v)) : "memory");
-}
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 u;
   asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "r"(addr));
@@ -359,17 +356,23 @@ __global__ void __launch_bounds__(NT, 1)
 }
 
 // ===================================================================== phase C
-// Warp-specialised walk: 10 warps.
+// Warp-specialised walk: 11 warps.
 //   warp 0     producer: TMA loads of Q/K/V (two stages) and the per-chunk gate quantities
-//   warp 1     MMA issue (one elected lane, fully unrolled, descriptors from constants)
-//   warps 2-5  state group: bf16 snapshot of C into TMEM (the read-out operand), n . q_t,
+//              (up to four chunks ahead)
+//   warp 1     chain MMAs: the chunk's update (C += (V o u)^T K) and read-out (H = Cb Q^T)
+//   warp 2     output MMAs: S = Q K^T of the next chunk and P V (H += V^T P^T)
+//   warps 3-6  state group: bf16 snapshot of C into TMEM (the read-out operand), n . q_t,
 //              Q scaling (guarded chunks only), n update
-//   warps 6-9  output group: P, V o u for the next chunk, denominators, h (TMA store)
-// The two single-warp roles have the lowest warp ids: a warp scheduler favours its older
-// warps, and with the groups' long instruction runs on the same sub-partitions the producer
-// and the MMA issuer otherwise wait thousands of cycles for issue slots.  A group's warps
-// cover the four TMEM lane quarters (warp % 4).
-// Hand-offs are mbarriers; every wait is bounded, and a group decides to abort as one.
+//   warps 7-10 output group: P, V o u for the next chunk, denominators, h (TMA store)
+// MMAs are issued by warps that do nothing else: an issuing warp stalls for about the time
+// its MMAs take to execute, which would hold up a SIMT group.  Each issuing warp is
+// converged and one elected lane issues, with descriptors computed by the whole warp (an
+// MMA issued with per-lane operands from divergent code costs ~100 cycles more); the
+// elected lane is the same one every time, so each commit tracks all of the warp's earlier
+// MMAs.  The producer has the lowest warp id: a warp scheduler favours its older warps, and
+// the groups' long instruction runs would otherwise keep it waiting for issue slots.  A
+// group's warps cover the four TMEM lane quarters (warp % 4).  Waits are mbarriers, every
+// one bounded; a group decides to abort as one.
 //
 // Lazily scaled state.  TMEM holds C_st with C_unstabilised = e^{lam} C_st (n likewise),
 // lam a scalar every role tracks identically.  With X_s = itilde_s - b_s (b the inclusive
@@ -383,7 +386,8 @@ __global__ void __launch_bounds__(NT, 1)
 // "guarded": it uses the per-element stabilised form instead (C rescaled to units of
 // e^{m}, Q scaled by e^{b_t + m_c - m_t}, P = S o e^{b_t - m_t + X_s}, update weights
 // e^{g + X_s - m_next}); every fp32 / bf16 value then stays within e^{+-60} of 1.
-constexpr int NTW = 320;
+constexpr int NTW = 352;
+constexpr int NGB = 4;                   // gate buffers
 constexpr int WG_STATE = 1, WG_OUT = 2;  // named barrier ids of the two 128-thread groups
 constexpr float LAM_RENORM = 20.f;       // renormalise lam when the stabiliser is this far above
 constexpr float U_MAX_LOG = 60.f;        // largest log u_s a fast chunk may use
@@ -394,13 +398,13 @@ struct WalkSmem {
   static constexpr int STAGE = QB + KB + VB;
   static constexpr int OVW = 2 * STAGE, OP = OVW + VB, OH = OP + PB;
   static constexpr int OF = OH + HB;  // floats start here
-  // n [DK], n partials [128*8], gate buffers [2][8][L], row sums / reciprocal denominators [2][L],
-  // gate scalars [2][8]
-  static constexpr int NF = DK + 128 * 8 + 2 * 8 * L + 2 * L + 16;
+  // n [DK], n partials [128*8], gate buffers [NGB][8][L], row sums / reciprocal denominators
+  // [2][L], gate scalars [NGB][8]
+  static constexpr int NF = DK + 128 * 8 + NGB * 8 * L + 2 * L + NGB * 8;
   static constexpr int BYTES = OF + NF * 4 + 1024;  // + alignment slack
 };
 
-// Per-chunk quantities (double-buffered), written by the producer except nq (state group).
+// Per-chunk quantities (NGB buffers), written by the producer except nq (state group).
 //   al, be : log2 row / column factors of P (fast: 0 and log2 u_s; guarded: (b_t - m_t) log2 e
 //            and X_s log2 e); be = -inf for tokens past the end
 //   u      : weight of v_s k_s in the update (and of k_s in the n update)
@@ -416,8 +420,8 @@ struct GateBuf {
 constexpr int GF_GUARD = 1, GF_STORE_C = 2;
 
 struct WalkBars {
-  uint64_t full[2], empty[2], gfull[2], gempty[2], q_ready[2];
-  uint64_t s_full, s_empty, cb_ready, vw_full, upd_done, ro_done, p_full, h_empty, mm_done;
+  uint64_t full[2], empty[2], s_full[2], gfull[NGB], gempty[NGB], q_ready[NGB];
+  uint64_t cb_ready, vw_full, upd_done, ro_done, h_empty, s_empty, p_full, mm_done;
 };
 
 template <int DK, int DVT>
@@ -431,17 +435,17 @@ __global__ void __launch_bounds__(NTW, 1)
   constexpr float LOG2E = 1.4426950408889634f;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *Vw = sm + SM::OVW, *Hs = sm + SM::OH;
+  uint8_t* Vw = sm + SM::OVW;
   float* nvec = reinterpret_cast<float*>(sm + SM::OF);
   float* npart = nvec + DK;  // [128 * 8]
   float* gmem = npart + 128 * 8;
-  float* rsum = gmem + 2 * 8 * L;
+  float* rsum = gmem + NGB * 8 * L;
   float* rden = rsum + L;
-  float* gscal = rden + L;  // [2][8]
-  auto gbuf = [&](int b) {
-    float* base = gmem + b * 8 * L;
+  float* gscal = rden + L;  // [NGB][8]
+  auto gbuf = [&](int gi) {
+    float* base = gmem + gi * 8 * L;
     return GateBuf{base,         base + L,     base + 2 * L, base + 3 * L, base + 4 * L,
-                   base + 5 * L, base + 6 * L, base + 7 * L, gscal + 8 * b};
+                   base + 5 * L, base + 6 * L, base + 7 * L, gscal + 8 * gi};
   };
   __shared__ WalkBars bars;
   __shared__ uint32_t tmem_base;
@@ -463,18 +467,20 @@ __global__ void __launch_bounds__(NTW, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.full[i], 1);
       mbar_init(&bars.empty[i], 3);
+      mbar_init(&bars.s_full[i], 1);
+    }
+    for (int i = 0; i < NGB; ++i) {
       mbar_init(&bars.gfull[i], 1);
       mbar_init(&bars.gempty[i], 2);
       mbar_init(&bars.q_ready[i], 1);
     }
-    mbar_init(&bars.s_full, 1);
-    mbar_init(&bars.s_empty, 1);
     mbar_init(&bars.cb_ready, 1);
     mbar_init(&bars.vw_full, 1);
     mbar_init(&bars.upd_done, 1);
     mbar_init(&bars.ro_done, 1);
-    mbar_init(&bars.p_full, 1);
     mbar_init(&bars.h_empty, 1);
+    mbar_init(&bars.s_empty, 1);
+    mbar_init(&bars.p_full, 1);
     mbar_init(&bars.mm_done, 1);
     abort_flag = 0;
     group_flag[0] = group_flag[1] = 0;
@@ -489,7 +495,7 @@ __global__ void __launch_bounds__(NTW, 1)
   tc_fence_after();
   const uint32_t tm = tmem_base;
 
-  // ---- start state of the segment (see the file header); warps 0-7 fill TMEM and n.
+  // ---- start state of the segment (see the file header); warps 3-10 fill TMEM and n.
   // It is stabilised at m_start, so lam starts at m_start.
   float m_start = ret ? 0.f : (p.m0 ? p.m0[bh] : 0.f);
   const float m_init = m_start;
@@ -499,8 +505,8 @@ __global__ void __launch_bounds__(NTW, 1)
     if (!ret) m_start = fmaxf(A + m_start, Bm);
     gsum += A;
   }
-  if (warp >= 2) {
-    const int quarter = warp & 3, half = (warp - 2) >> 2;
+  if (warp >= 3) {
+    const int quarter = warp & 3, half = (warp - 3) >> 2;
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     const int row = acc_row<DVT>(quarter, lane);
     const float wc0 = expf(gsum + m_init - m_start);
@@ -540,7 +546,7 @@ __global__ void __launch_bounds__(NTW, 1)
     }
     tmem_wait_st();
     if (!ret)
-      for (int col = tid - 64; col < DK; col += 256) {
+      for (int col = tid - 96; col < DK; col += 256) {
         float x = p.n0 ? wc0 * p.n0[(size_t)slice * p.dk + col] : 0.f;
         float after = gsum;
         for (int jg = 0; jg < g; ++jg) {
@@ -573,6 +579,33 @@ __global__ void __launch_bounds__(NTW, 1)
     }
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
   };
+  const uint32_t id_s = idesc_bf16(64, 64, 0, 0);
+  const uint32_t id_ro = idesc_bf16(DVT, 64, 0, 0);
+  const uint32_t id_pv = idesc_bf16(DVT, 64, 1, 0);
+  const uint32_t id_up = idesc_bf16(DVT, DK, 1, 1);
+  // The issue helpers take descriptors computed by the whole (converged) warp, so the
+  // elected lane only adds constant offsets.
+  // S = Q K^T into the S columns; q_k, k_k: K-major descriptors of the chunk's Q and K
+  auto issue_s = [&](uint64_t q_k, uint64_t k_k, int b) {
+#pragma unroll
+    for (int k = 0; k < DK; k += 16) {
+      const uint64_t off = (uint64_t)(((k >> 6) * 8192 + (k & 63) * 2) >> 4);
+      mma_bf16_ss(tm + TM_S, q_k + off, k_k + off, id_s, k > 0 ? 1u : 0u);
+    }
+    mma_commit(&bars.s_full[b]);
+  };
+  // read-out H = Cb Q^T (A = the bf16 snapshot in TMEM); releases stage b with the update
+  auto issue_readout = [&](uint64_t q_k, int b) {
+#pragma unroll
+    for (int k = 0; k < DK; k += 16)
+      mma_bf16_ts(tm + TM_H, tm + TM_CB + k / 2, q_k + (uint64_t)(((k >> 6) * 8192 + (k & 63) * 2) >> 4), id_ro,
+                  k > 0 ? 1u : 0u);
+    mma_commit(&bars.ro_done);
+    mma_commit(&bars.empty[b]);
+  };
+  auto desc_k = [&](int c, int part) {  // part 0: Q, 1: K of chunk c's stage, K-major
+    return smem_desc_sw128(sm_u + (c & 1) * SM::STAGE + part * SM::QB, 16, 1024);
+  };
 
   if (warp == 0) {
     // =============================================================== producer
@@ -597,7 +630,7 @@ __global__ void __launch_bounds__(NTW, 1)
     if (nck > 0) fetch_gates(0);
     float mc = m_start, lam = m_start;
     for (int c = 0; c < nck; ++c) {
-      const int b = c & 1;
+      const int b = c & 1, gi = c % NGB;
       // operands of chunk c into stage b once its previous user (chunk c-2) released it
       if (!warp_wait(&bars.empty[b], ((c >> 1) & 1) ^ 1)) break;
       if (lane == 0) {
@@ -611,9 +644,9 @@ __global__ void __launch_bounds__(NTW, 1)
         for (int j = 0; j < DVT / 64; ++j)
           tma_load_3d(base + SM::QB + SM::KB + j * 8192, &mapV, blk * p.dv + v0 + 64 * j, t0, bh, &bars.full[b]);
       }
-      // gate quantities of chunk c into buffer b (lane: tokens 2 lane, 2 lane + 1)
-      if (!warp_wait(&bars.gempty[b], ((c >> 1) & 1) ^ 1)) break;
-      GateBuf G = gbuf(b);
+      // gate quantities of chunk c into buffer gi (lane: tokens 2 lane, 2 lane + 1)
+      if (!warp_wait(&bars.gempty[gi], ((c / NGB) & 1) ^ 1)) break;
+      GateBuf G = gbuf(gi);
       const int ta = 2 * lane, tb = 2 * lane + 1;
       const float ba = pba, bb = pbb, xa = pxa, xb = pxb, gtot = pg, xmax = pxm;
       // m_t = b_t + max(m_c, Xc_t): the stabiliser recurrence unrolled over the chunk
@@ -667,68 +700,61 @@ __global__ void __launch_bounds__(NTW, 1)
       mc = mn;
       lam = lam_next;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.gfull[b]);
+      if (lane == 0) mbar_arrive(&bars.gfull[gi]);
       if (c + 1 < nck) fetch_gates(c + 1);
     }
     if (lane == 0 && !abort_flag && last_seg && !ret && tile == 0 && blk == 0 && p.m_out) p.m_out[bh] = mc;
   } else if (warp == 1) {
-    // =============================================================== MMA issue
-    // per chunk: update (C += (V o u)^T K), read-out (H = Cb Q^T), next chunk's S = Q K^T,
-    // then P V (H += V^T P^T).  The update and read-out are the chunk recurrence.
-    const uint32_t id_s = idesc_bf16(64, 64, 0, 0);
-    const uint32_t id_ro = idesc_bf16(DVT, 64, 0, 0);
-    const uint32_t id_pv = idesc_bf16(DVT, 64, 1, 0);
-    const uint32_t id_up = idesc_bf16(DVT, DK, 1, 1);
-    const uint64_t ps_k = smem_desc_sw128(sm_u + SM::OP, 16, 1024);       // P, K-major rows t
+    // =============================================================== chain MMAs
     const uint64_t vw_mn = smem_desc_sw128(sm_u + SM::OVW, 8192, 1024);  // V o u, MN-major
-    auto issue_s = [&](int c) -> bool {
-      const int b = c & 1;
-      const uint64_t q_k = smem_desc_sw128(sm_u + b * SM::STAGE, 16, 1024);
-      const uint64_t k_k = smem_desc_sw128(sm_u + b * SM::STAGE + SM::QB, 16, 1024);
-      if (!warp_wait(&bars.full[b], (c >> 1) & 1)) return false;
-      if (c > 0 && !warp_wait(&bars.s_empty, (c - 1) & 1)) return false;
+    for (int c = 0; c < nck; ++c) {
+      const int b = c & 1, gi = c % NGB;
+      const uint64_t q_k = desc_k(c, 0);
+      const uint64_t k_mn = smem_desc_sw128(sm_u + b * SM::STAGE + SM::QB, 8192, 1024);  // K, MN-major
+      // update C += (V o u)^T K once the snapshot has read C and V o u is staged
+      if (!warp_wait(&bars.cb_ready, c & 1)) break;
+      if (!warp_wait(&bars.vw_full, c & 1)) break;
+      if (!warp_wait(&bars.full[b], (c >> 1) & 1)) break;
       tc_fence_after();
       if (elect_one()) {
 #pragma unroll
-        for (int k = 0; k < DK; k += 16) {
-          const uint64_t off = (uint64_t)(((k >> 6) * 8192 + (k & 63) * 2) >> 4);
-          mma_bf16_ss(tm + TM_S, q_k + off, k_k + off, id_s, k > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars.s_full);
+        for (int ks = 0; ks < L / 16; ++ks)
+          mma_bf16_ss(tm + TM_C, vw_mn + (uint64_t)(ks * 128), k_mn + (uint64_t)(ks * 128), id_up, 1u);
+        mma_commit(&bars.upd_done);
       }
       __syncwarp();
-      return true;
-    };
-    if (nck > 0 && issue_s(0))
+      // read-out of the snapshot; a guarded chunk first scales Q (the gate buffer is visible
+      // here through the state group's cb_ready, which it arrived after reading it)
+      const bool guard = (__float_as_int(gbuf(gi).scal[0]) & GF_GUARD) != 0;
+      if (guard && !warp_wait(&bars.q_ready[gi], (c / NGB) & 1)) break;
+      if (c > 0 && !warp_wait(&bars.h_empty, (c - 1) & 1)) break;
+      tc_fence_after();
+      if (elect_one()) issue_readout(q_k, b);
+      __syncwarp();
+    }
+  } else if (warp == 2) {
+    // =============================================================== output MMAs
+    const uint64_t ps_k = smem_desc_sw128(sm_u + SM::OP, 16, 1024);  // P, K-major rows t
+    if (nck > 0 && warp_wait(&bars.full[0], 0)) {
+      const uint64_t q_k = desc_k(0, 0), k_k = desc_k(0, 1);
+      tc_fence_after();
+      if (elect_one()) issue_s(q_k, k_k, 0);
+      __syncwarp();
       for (int c = 0; c < nck; ++c) {
         const int b = c & 1;
-        const uint32_t q_u = sm_u + b * SM::STAGE, k_u = q_u + SM::QB, v_u = k_u + SM::KB;
-        const uint64_t q_k = smem_desc_sw128(q_u, 16, 1024);     // Q, K-major rows t
-        const uint64_t k_mn = smem_desc_sw128(k_u, 8192, 1024);  // K, MN-major (rows s = K dim)
-        const uint64_t v_mn = smem_desc_sw128(v_u, 8192, 1024);  // V, MN-major
-        if (!warp_wait(&bars.cb_ready, c & 1)) break;
-        if (!warp_wait(&bars.vw_full, c & 1)) break;
-        tc_fence_after();
-        if (elect_one()) {
-#pragma unroll
-          for (int ks = 0; ks < L / 16; ++ks)
-            mma_bf16_ss(tm + TM_C, vw_mn + (uint64_t)(ks * 128), k_mn + (uint64_t)(ks * 128), id_up, 1u);
-          mma_commit(&bars.upd_done);
+        // S of the next chunk once this chunk's S has left TMEM
+        if (c + 1 < nck) {
+          const uint64_t q_k1 = desc_k(c + 1, 0), k_k1 = desc_k(c + 1, 1);
+          if (!warp_wait(&bars.s_empty, c & 1)) break;
+          if (!warp_wait(&bars.full[b ^ 1], ((c + 1) >> 1) & 1)) break;
+          tc_fence_after();
+          if (elect_one()) issue_s(q_k1, k_k1, b ^ 1);
+          __syncwarp();
         }
-        __syncwarp();
-        if (!warp_wait(&bars.q_ready[b], (c >> 1) & 1)) break;
-        if (c > 0 && !warp_wait(&bars.h_empty, (c - 1) & 1)) break;
-        tc_fence_after();
-        if (elect_one()) {
-#pragma unroll
-          for (int k = 0; k < DK; k += 16)
-            mma_bf16_ts(tm + TM_H, tm + TM_CB + k / 2, q_k + (uint64_t)(((k >> 6) * 8192 + (k & 63) * 2) >> 4),
-                        id_ro, k > 0 ? 1u : 0u);
-          mma_commit(&bars.ro_done);
-        }
-        __syncwarp();
-        if (c + 1 < nck && !issue_s(c + 1)) break;
+        // P V onto the read-out (same accumulator, issued by the chain warp)
+        const uint64_t v_mn = smem_desc_sw128(sm_u + b * SM::STAGE + SM::QB + SM::KB, 8192, 1024);
         if (!warp_wait(&bars.p_full, c & 1)) break;
+        if (!warp_wait(&bars.ro_done, c & 1)) break;
         tc_fence_after();
         if (elect_one()) {
 #pragma unroll
@@ -739,43 +765,60 @@ __global__ void __launch_bounds__(NTW, 1)
         }
         __syncwarp();
       }
-  } else if (warp < 6) {
+    }
+  } else if (warp < 7) {
     // =============================================================== state group
     const int quarter = warp & 3;
-    const int st = tid - 64;  // 0..127
+    const int st = tid - 96;  // 0..127
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     const bool first = st == 0;
     float fin = 1.f;
     for (int c = 0; c < nck; ++c) {
-      const int b = c & 1;
-      const GateBuf G = gbuf(b);
+      const int b = c & 1, gi = c % NGB;
+      const GateBuf G = gbuf(gi);
       uint8_t* Qs = sm + b * SM::STAGE;
       uint8_t* Ks = Qs + SM::QB;
-      if (!group_wait(&bars.gfull[b], (c >> 1) & 1, 0, first)) break;
+      if (!group_wait(&bars.gfull[gi], (c / NGB) & 1, 0, first)) break;
       // the previous read-out has read the snapshot and the previous update has written C
       if (c > 0 && !group_wait(&bars.ro_done, (c - 1) & 1, 0, first)) break;
       tc_fence_after();
       const int flags = __float_as_int(G.scal[0]);
+      const bool guard = (flags & GF_GUARD) != 0;
       fin = G.scal[4];
       {
         // bf16 snapshot of (scaled) C into TMEM; C itself rewritten only when lam moves
-        const float cbs = G.scal[1], csc = G.scal[2];
-        const bool store_c = (flags & GF_STORE_C) != 0;
+        if (!(flags & GF_STORE_C)) {
+          // the common case: C is already in the units of the snapshot
 #pragma unroll 1
-        for (int c0 = 0; c0 < DK; c0 += 64) {
-          float r[64];
-          tmem_ld32(tm + lane_off + TM_C + c0, *reinterpret_cast<float(*)[32]>(r));
-          tmem_ld32(tm + lane_off + TM_C + c0 + 32, *reinterpret_cast<float(*)[32]>(r + 32));
-          tmem_wait_ld();
-          float pk[16];
+          for (int c0 = 0; c0 < DK; c0 += 64) {
+            float r[64];
+            tmem_ld32(tm + lane_off + TM_C + c0, *reinterpret_cast<float(*)[32]>(r));
+            tmem_ld32(tm + lane_off + TM_C + c0 + 32, *reinterpret_cast<float(*)[32]>(r + 32));
+            tmem_wait_ld();
+            float pk[16];
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
+            for (int h2 = 0; h2 < 2; ++h2) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              pk[j] = __uint_as_float(pack_bf16(r[32 * h2 + 2 * j] * cbs, r[32 * h2 + 2 * j + 1] * cbs));
-            tmem_st16(tm + lane_off + TM_CB + c0 / 2 + 16 * h2, pk);
+              for (int j = 0; j < 16; ++j) pk[j] = __uint_as_float(pack_bf16(r[32 * h2 + 2 * j], r[32 * h2 + 2 * j + 1]));
+              tmem_st16(tm + lane_off + TM_CB + c0 / 2 + 16 * h2, pk);
+            }
           }
-          if (store_c) {
+        } else {
+          const float cbs = G.scal[1], csc = G.scal[2];
+#pragma unroll 1
+          for (int c0 = 0; c0 < DK; c0 += 64) {
+            float r[64];
+            tmem_ld32(tm + lane_off + TM_C + c0, *reinterpret_cast<float(*)[32]>(r));
+            tmem_ld32(tm + lane_off + TM_C + c0 + 32, *reinterpret_cast<float(*)[32]>(r + 32));
+            tmem_wait_ld();
+            float pk[16];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                pk[j] = __uint_as_float(pack_bf16(r[32 * h2 + 2 * j] * cbs, r[32 * h2 + 2 * j + 1] * cbs));
+              tmem_st16(tm + lane_off + TM_CB + c0 / 2 + 16 * h2, pk);
+            }
 #pragma unroll
             for (int h4 = 0; h4 < 4; ++h4) {
 #pragma unroll
@@ -825,9 +868,10 @@ __global__ void __launch_bounds__(NTW, 1)
         a += __shfl_xor_sync(0xffffffffu, a, 1);
         if (part == 0) G.nq[t] = a;
       }
-      if (flags & GF_GUARD) {
-        // guarded chunk: Q <- e^{b_t+m_c-m_t} Q once the S MMA has read the raw Q
-        if (!group_wait(&bars.s_full, c & 1, 0, first)) break;
+      if (guard) {
+        // guarded chunk: Q <- e^{b_t+m_c-m_t} Q once the S MMA has read the raw Q, then the
+        // read-out with the scaled Q
+        if (!group_wait(&bars.s_full[b], (c >> 1) & 1, 0, first)) break;
         const int gt = st;
         constexpr int NQ = L * (DK / 8) / 128;  // 16-byte chunks per thread
         constexpr int BATCH = NQ < 8 ? NQ : 8;
@@ -851,7 +895,7 @@ __global__ void __launch_bounds__(NTW, 1)
         fence_proxy_async_smem();
       }
       named_bar(WG_STATE, 128);
-      if (first) mbar_arrive(&bars.q_ready[b]);
+      if (first) mbar_arrive(&bars.q_ready[gi]);
       if (!ret) {
         // n <- ns n + sum_s u_s k_s
         constexpr int NCG = DK / 8, NRG = 128 / NCG, RPG = L / NRG;
@@ -888,12 +932,12 @@ __global__ void __launch_bounds__(NTW, 1)
       named_bar(WG_STATE, 128);
       if (first) {
         mbar_arrive(&bars.empty[b]);
-        mbar_arrive(&bars.gempty[b]);
+        mbar_arrive(&bars.gempty[gi]);
       }
     }
-    // final state after the last update, back in units of e^{m}.  The wait is on ro_done,
-    // whose every phase this group has waited for: a parity wait on a barrier two phases
-    // behind would return at once.
+    // final state after the last update, back in units of e^{m}.  ro_done is committed after
+    // the chunk's update, and this group has waited for each of its phases in turn (a parity
+    // wait on a barrier two phases behind would return at once).
     if (nck > 0 && group_wait(&bars.ro_done, (nck - 1) & 1, 0, first) && last_seg) {
       tc_fence_after();
       const int row = acc_row<DVT>(quarter, lane);
@@ -916,13 +960,13 @@ __global__ void __launch_bounds__(NTW, 1)
   } else {
     // =============================================================== output group
     const int quarter = warp & 3;
-    const int gt = tid - 192;  // 0..127
-    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+    const int gt = tid - 224;  // 0..127
     const bool first = gt == 0;
-    const uint32_t ps_u = sm_u + SM::OP;
+    const uint32_t ps_u = sm_u + SM::OP, hs_u = sm_u + SM::OH;
+    const bool use_og = p.og != nullptr && !ret;
     // V o u of chunk c into the update operand buffer (loads batched ahead of the stores)
     auto scale_v = [&](int c) {
-      const GateBuf G = gbuf(c & 1);
+      const GateBuf G = gbuf(c % NGB);
       const uint32_t vs_u = sm_u + (c & 1) * SM::STAGE + SM::QB + SM::KB, vw_u2 = smem_u32(Vw);
       constexpr int NV = L * (DVT / 8) / 128;  // 16-byte chunks per thread
       uint4 u[NV];
@@ -947,43 +991,65 @@ __global__ void __launch_bounds__(NTW, 1)
       if (first) mbar_arrive(&bars.vw_full);
     }
     for (int c = 0; ok && c < nck; ++c) {
-      const int b = c & 1;
-      const GateBuf G = gbuf(b);
+      const int b = c & 1, gi = c % NGB;
+      const GateBuf G = gbuf(gi);
       const int t0 = T0 + c * L;
       const int Lc = min(L, T1 - t0);
       const size_t tok0 = (size_t)bh * p.S + t0;
-      // P = S o e^{al_t + be_s} (bf16, rows t) and its row sums; P V of the previous chunk
-      // must be done with the P buffer
+      // P = S o e^{al_t + be_s} (bf16, rows t, 128-byte swizzled) and its row sums; P V of
+      // the previous chunk must be done with the P buffer
       if (c > 0 && !group_wait(&bars.mm_done, (c - 1) & 1, 1, first)) break;
-      if (!group_wait(&bars.s_full, c & 1, 1, first)) break;
+      if (!group_wait(&bars.s_full[b], (c >> 1) & 1, 1, first)) break;
       tc_fence_after();
       {
         // 16x256b load: thread -> rows 16q + lane/4 and +8, column pairs 8j + 2(lane%4)
         const int r_lo = 16 * quarter + (lane >> 2), r_hi = r_lo + 8, cp = 2 * (lane & 3);
-        float r[32], csr[16];
-        tmem_ld16x256_x8(tm + lane_off + TM_S, r);
+        float r[32], f_lo[16], f_hi[16];
+        tmem_ld16x256_x8(tm + ((uint32_t)(32 * quarter) << 16) + TM_S, r);
+        // element factors: fast chunk u_s (columns only); guarded e^{al_t + be_s}
+        if (!(__float_as_int(G.scal[0]) & GF_GUARD)) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          csr[2 * j] = G.be[8 * j + cp];
-          csr[2 * j + 1] = G.be[8 * j + cp + 1];
+          for (int j = 0; j < 8; ++j) {
+            const float2 u2 = *reinterpret_cast<const float2*>(G.u + 8 * j + cp);
+            f_lo[2 * j] = f_hi[2 * j] = u2.x;
+            f_lo[2 * j + 1] = f_hi[2 * j + 1] = u2.y;
+          }
+        } else {
+          const float al_lo = G.al[r_lo], al_hi = G.al[r_hi];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float2 be2 = *reinterpret_cast<const float2*>(G.be + 8 * j + cp);
+            f_lo[2 * j] = exp2f(al_lo + be2.x);
+            f_lo[2 * j + 1] = exp2f(al_lo + be2.y);
+            f_hi[2 * j] = exp2f(al_hi + be2.x);
+            f_hi[2 * j + 1] = exp2f(al_hi + be2.y);
+          }
         }
-        const float al_lo = G.al[r_lo], al_hi = G.al[r_hi];
         tmem_wait_ld();
         tc_fence_before();
         named_bar(WG_OUT, 128);
-        if (first) mbar_arrive(&bars.s_empty);
+        if (first) mbar_arrive(&bars.s_empty);  // S has left TMEM
         float rs_lo = 0.f, rs_hi = 0.f;
+        uint32_t plo[8], phi[8];
+        const int lim_lo = r_lo < Lc ? r_lo : -1, lim_hi = r_hi < Lc ? r_hi : -1;  // last column kept
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int s0 = 8 * j + cp;
-          const float a0 = (s0 <= r_lo && r_lo < Lc) ? r[2 * j] * exp2f(al_lo + csr[2 * j]) : 0.f;
-          const float a1 = (s0 + 1 <= r_lo && r_lo < Lc) ? r[2 * j + 1] * exp2f(al_lo + csr[2 * j + 1]) : 0.f;
-          const float b0 = (s0 <= r_hi && r_hi < Lc) ? r[16 + 2 * j] * exp2f(al_hi + csr[2 * j]) : 0.f;
-          const float b1 = (s0 + 1 <= r_hi && r_hi < Lc) ? r[16 + 2 * j + 1] * exp2f(al_hi + csr[2 * j + 1]) : 0.f;
+          const float a0 = s0 <= lim_lo ? r[2 * j] * f_lo[2 * j] : 0.f;
+          const float a1 = s0 + 1 <= lim_lo ? r[2 * j + 1] * f_lo[2 * j + 1] : 0.f;
+          const float b0 = s0 <= lim_hi ? r[16 + 2 * j] * f_hi[2 * j] : 0.f;
+          const float b1 = s0 + 1 <= lim_hi ? r[16 + 2 * j + 1] * f_hi[2 * j + 1] : 0.f;
           rs_lo += a0 + a1;
           rs_hi += b0 + b1;
-          asm volatile("st.shared.b32 [%0], %1;" ::"r"(ps_u + sw128_offset(r_lo, s0)), "r"(pack_bf16(a0, a1)) : "memory");
-          asm volatile("st.shared.b32 [%0], %1;" ::"r"(ps_u + sw128_offset(r_hi, s0)), "r"(pack_bf16(b0, b1)) : "memory");
+          plo[j] = pack_bf16(a0, a1);
+          phi[j] = pack_bf16(b0, b1);
+        }
+        // matrices (rows lo, cols 8j), (rows hi, 8j), (lo, 8j+8), (hi, 8j+8) per instruction
+        const int mrow = 16 * quarter + ((lane >> 3) & 1) * 8 + (lane & 7), mcol = lane >> 4;
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) {
+          const int cb = j + mcol;
+          stmatrix_x4(ps_u + mrow * 128 + ((cb ^ (mrow & 7)) << 4), plo[j], phi[j], plo[j + 1], phi[j + 1]);
         }
         rs_lo += __shfl_xor_sync(0xffffffffu, rs_lo, 1);
         rs_lo += __shfl_xor_sync(0xffffffffu, rs_lo, 2);
@@ -1000,7 +1066,7 @@ __global__ void __launch_bounds__(NTW, 1)
       // V o u of the next chunk once this chunk's update has read the buffer
       if (c + 1 < nck) {
         const int b1 = (c + 1) & 1;
-        if (!group_wait(&bars.gfull[b1], ((c + 1) >> 1) & 1, 1, first)) break;
+        if (!group_wait(&bars.gfull[(c + 1) % NGB], ((c + 1) / NGB) & 1, 1, first)) break;
         if (!group_wait(&bars.full[b1], ((c + 1) >> 1) & 1, 1, first)) break;
         if (!group_wait(&bars.upd_done, c & 1, 1, first)) break;
         scale_v(c + 1);
@@ -1008,53 +1074,83 @@ __global__ void __launch_bounds__(NTW, 1)
         if (first) mbar_arrive(&bars.vw_full);
       }
       // reciprocal denominators times the output scale E_t (nq_t from the state group)
-      if (!group_wait(&bars.q_ready[b], (c >> 1) & 1, 1, first)) break;
+      if (!group_wait(&bars.q_ready[gi], (c / NGB) & 1, 1, first)) break;
       if (gt < L) {
         const int t = gt;
         const float e = G.E[t];
         rden[t] = ret ? e : e / fmaxf(fabsf(e * rsum[t] + G.F[t] * G.nq[t]), G.emt[t]);
       }
-      named_bar(WG_OUT, 128);
-      if (first) mbar_arrive(&bars.empty[b]);
-      // h_t = H_t rden_t (x o_t): H leaves TMEM first, then the tile is staged and TMA-stored
+      // h_t = H_t rden_t (x o_t): H leaves TMEM first, then 8x8 tiles are stored transposed
+      // into the 128-byte swizzled staging tile and TMA-stored
       if (first) bulk_wait_read_all();
       if (!group_wait(&bars.mm_done, c & 1, 1, first)) break;
       tc_fence_after();
       {
-        const int row = acc_row<DVT>(quarter, lane);
-        const int rr = row >= 0 ? row : 0;
-        const uint32_t hb_u = smem_u32(Hs) + (rr >> 6) * 8192 + (rr & 63) * 2;
-        const size_t hcol = (size_t)blk * p.dv + v0 + rr;
-        float r[64];
-        tmem_ld32(tm + lane_off + TM_H, *reinterpret_cast<float(*)[32]>(r));
-        tmem_ld32(tm + lane_off + TM_H + 32, *reinterpret_cast<float(*)[32]>(r + 32));
+        constexpr int NH = DVT == 128 ? 2 : 1;  // 16-lane halves of this warp's quarter
+        float r[NH][32];
+#pragma unroll
+        for (int hf = 0; hf < NH; ++hf)
+          tmem_ld16x256_x8(tm + ((uint32_t)(32 * quarter + 16 * hf) << 16) + TM_H, r[hf]);
         tmem_wait_ld();
         tc_fence_before();
         named_bar(WG_OUT, 128);
         if (first) mbar_arrive(&bars.h_empty);
+        const int cp = 2 * (lane & 3);
+        float s0[8], s1[8];
 #pragma unroll
-        for (int tt = 0; tt < L; tt += 32) {
-          float rd[32];
+        for (int j = 0; j < 8; ++j) {
+          const float2 rd = *reinterpret_cast<const float2*>(rden + 8 * j + cp);
+          s0[j] = rd.x;
+          s1[j] = rd.y;
+        }
 #pragma unroll
-          for (int j = 0; j < 32; ++j) rd[j] = rden[tt + j];
-          if (p.og && !ret) {
+        for (int hf = 0; hf < NH; ++hf) {
+          // value rows of this half: d_lo = base + lane/4 (r[2j], r[2j+1]) and d_lo + 8 (r[16+..])
+          const int base = DVT == 128 ? 32 * quarter + 16 * hf : 16 * quarter;
+          const int d_lo = base + (lane >> 2), d_hi = d_lo + 8;
+          uint32_t plo[8], phi[8];
+          if (!use_og) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (tt + j < Lc) rd[j] *= __bfloat162float(p.og[(tok0 + tt + j) * p.DHV + hcol]);
+            for (int j = 0; j < 8; ++j) {
+              plo[j] = pack_bf16(r[hf][2 * j] * s0[j], r[hf][2 * j + 1] * s1[j]);
+              phi[j] = pack_bf16(r[hf][16 + 2 * j] * s0[j], r[hf][16 + 2 * j + 1] * s1[j]);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              float x0 = r[hf][2 * j] * s0[j], x1 = r[hf][2 * j + 1] * s1[j];
+              float y0 = r[hf][16 + 2 * j] * s0[j], y1 = r[hf][16 + 2 * j + 1] * s1[j];
+              const int ta = 8 * j + cp;
+              const size_t ra = (tok0 + ta) * p.DHV + (size_t)blk * p.dv + v0;
+              if (ta < Lc) {
+                x0 *= __bfloat162float(p.og[ra + d_lo]);
+                y0 *= __bfloat162float(p.og[ra + d_hi]);
+              }
+              if (ta + 1 < Lc) {
+                x1 *= __bfloat162float(p.og[ra + p.DHV + d_lo]);
+                y1 *= __bfloat162float(p.og[ra + p.DHV + d_hi]);
+              }
+              plo[j] = pack_bf16(x0, x1);
+              phi[j] = pack_bf16(y0, y1);
+            }
           }
-          if (row >= 0) {
+          // transposed: matrices (values lo, tokens 8j), (hi, 8j), (lo, 8j+8), (hi, 8j+8)
+          const int d0 = base + ((lane >> 3) & 1) * 8;
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              st_shared_b16(hb_u + (tt + j) * 128, __float2bfloat16_rn(r[tt + j] * rd[j]));
+          for (int j = 0; j < 8; j += 2) {
+            const int t = 8 * (j + (lane >> 4)) + (lane & 7);
+            const uint32_t addr = hs_u + (d0 >> 6) * 8192 + t * 128 + ((((d0 & 63) >> 3) ^ (t & 7)) << 4);
+            stmatrix_x4_trans(addr, plo[j], phi[j], plo[j + 1], phi[j + 1]);
           }
         }
       }
       fence_proxy_async_smem();
       named_bar(WG_OUT, 128);
       if (first) {
-        for (int j = 0; j < DVT / 64; ++j) tma_store_3d(&mapH, Hs + j * 8192, blk * p.dv + v0 + 64 * j, t0, bh);
+        for (int j = 0; j < DVT / 64; ++j)
+          tma_store_3d(&mapH, sm + SM::OH + j * 8192, blk * p.dv + v0 + 64 * j, t0, bh);
         bulk_commit();
-        mbar_arrive(&bars.gempty[b]);
+        mbar_arrive(&bars.gempty[gi]);
       }
     }
     if (first) bulk_wait_all();
@@ -1147,7 +1243,7 @@ cudaError_t launch_tc(const WalkArgs& a, const TcPlan& pl, void* ws, cudaStream_
   CUtensorMap mq, mk, mv, mh;
   if (!make_map_bf16_3d(&mq, a.q, a.DHQK, a.S, BH, L) || !make_map_bf16_3d(&mk, a.k, a.DHQK, a.S, BH, L) ||
       !make_map_bf16_3d(&mv, a.v, a.DHV, a.S, BH, L) ||
-      !make_map_bf16_3d(&mh, a.h, a.DHV, a.S, BH, L, CU_TENSOR_MAP_SWIZZLE_NONE))
+      !make_map_bf16_3d(&mh, a.h, a.DHV, a.S, BH, L))
     return cudaErrorInvalidValue;
   TcParams prm;
   prm.S = a.S;

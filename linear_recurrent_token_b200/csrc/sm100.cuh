@@ -199,6 +199,20 @@ __device__ __forceinline__ void tmem_ld16x256_x8(uint32_t taddr, float (&r)[32])
     u[16 + 2 * j + 1] = a[4 * j + 3];
   }
 }
+// stmatrix: four 8x8 b16 matrices.  Thread t gives the shared address of row t%8 of matrix
+// t/8 and holds in r_k its fragment of matrix k: row t/4, columns 2(t%4) (low half) and
+// 2(t%4)+1.  The .trans form stores the transpose: the row at thread t's address receives
+// column t%8 of matrix t/8.
+__device__ __forceinline__ void stmatrix_x4(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(r0), "r"(r1), "r"(r2),
+               "r"(r3)
+               : "memory");
+}
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(r0), "r"(r1),
+               "r"(r2), "r"(r3)
+               : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
