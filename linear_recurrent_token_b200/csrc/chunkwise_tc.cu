@@ -847,7 +847,7 @@ __global__ void __launch_bounds__(NTW, 1)
         constexpr int NCH = DK / 16;
         constexpr int BATCH = NCH < 8 ? NCH : 8;
         float a0 = 0.f, a1 = 0.f;
-#pragma unroll
+#pragma unroll 1
         for (int j0 = 0; j0 < NCH; j0 += BATCH) {
           uint4 u[BATCH];
 #pragma unroll
@@ -976,19 +976,23 @@ __global__ void __launch_bounds__(NTW, 1)
       const GateBuf G = gbuf(c % NGB);
       const uint32_t vs_u = sm_u + (c & 1) * SM::STAGE + SM::QB + SM::KB, vw_u2 = smem_u32(Vw);
       constexpr int NV = L * (DVT / 8) / 128;  // 16-byte chunks per thread
-      uint4 u[NV];
-      float wr[NV];
-      int offs[NV];
+      constexpr int NB = NV < 4 ? NV : 4;       // per pass; the pass loop keeps the code small
+#pragma unroll 1
+      for (int k0 = 0; k0 < NV; k0 += NB) {
+        uint4 u[NB];
+        float wr[NB];
+        int offs[NB];
 #pragma unroll
-      for (int k = 0; k < NV; ++k) {
-        const int i = k * 128 + gt;
-        const int row = i / (DVT / 8), ch = i % (DVT / 8);
-        offs[k] = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
-        u[k] = ld_shared_v4(vs_u + offs[k]);
-        wr[k] = G.u[row];
+        for (int k = 0; k < NB; ++k) {
+          const int i = (k0 + k) * 128 + gt;
+          const int row = i / (DVT / 8), ch = i % (DVT / 8);
+          offs[k] = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
+          u[k] = ld_shared_v4(vs_u + offs[k]);
+          wr[k] = G.u[row];
+        }
+#pragma unroll
+        for (int k = 0; k < NB; ++k) st_shared_v4u(vw_u2 + offs[k], scale_bf16x8(u[k], wr[k]));
       }
-#pragma unroll
-      for (int k = 0; k < NV; ++k) st_shared_v4u(vw_u2 + offs[k], scale_bf16x8(u[k], wr[k]));
       fence_proxy_async_smem();
     };
     bool ok = nck > 0 && group_wait(&bars.gfull[0], 0, 1, first) && group_wait(&bars.full[0], 0, 1, first);
@@ -1094,10 +1098,9 @@ __global__ void __launch_bounds__(NTW, 1)
       tc_fence_after();
       {
         constexpr int NH = DVT == 128 ? 2 : 1;  // 16-lane halves of this warp's quarter
-        float r[NH][32];
-#pragma unroll
-        for (int hf = 0; hf < NH; ++hf)
-          tmem_ld16x256_x8(tm + ((uint32_t)(32 * quarter + 16 * hf) << 16) + TM_H, r[hf]);
+        float r[32], r2[32];
+        tmem_ld16x256_x8(tm + ((uint32_t)(32 * quarter) << 16) + TM_H, r);
+        if (NH == 2) tmem_ld16x256_x8(tm + ((uint32_t)(32 * quarter + 16) << 16) + TM_H, r2);
         tmem_wait_ld();
         tc_fence_before();
         named_bar(WG_OUT, 128);
@@ -1110,8 +1113,14 @@ __global__ void __launch_bounds__(NTW, 1)
           s0[j] = rd.x;
           s1[j] = rd.y;
         }
-#pragma unroll
+        // one loop body for both halves (the second half's registers move into r), which
+        // keeps this hot code short
+#pragma unroll 1
         for (int hf = 0; hf < NH; ++hf) {
+          if (hf == 1) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) r[j] = r2[j];
+          }
           // value rows of this half: d_lo = base + lane/4 (r[2j], r[2j+1]) and d_lo + 8 (r[16+..])
           const int base = DVT == 128 ? 32 * quarter + 16 * hf : 16 * quarter;
           const int d_lo = base + (lane >> 2), d_hi = d_lo + 8;
@@ -1119,14 +1128,14 @@ __global__ void __launch_bounds__(NTW, 1)
           if (!use_og) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-              plo[j] = pack_bf16(r[hf][2 * j] * s0[j], r[hf][2 * j + 1] * s1[j]);
-              phi[j] = pack_bf16(r[hf][16 + 2 * j] * s0[j], r[hf][16 + 2 * j + 1] * s1[j]);
+              plo[j] = pack_bf16(r[2 * j] * s0[j], r[2 * j + 1] * s1[j]);
+              phi[j] = pack_bf16(r[16 + 2 * j] * s0[j], r[16 + 2 * j + 1] * s1[j]);
             }
           } else {
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-              float x0 = r[hf][2 * j] * s0[j], x1 = r[hf][2 * j + 1] * s1[j];
-              float y0 = r[hf][16 + 2 * j] * s0[j], y1 = r[hf][16 + 2 * j + 1] * s1[j];
+              float x0 = r[2 * j] * s0[j], x1 = r[2 * j + 1] * s1[j];
+              float y0 = r[16 + 2 * j] * s0[j], y1 = r[16 + 2 * j + 1] * s1[j];
               const int ta = 8 * j + cp;
               const size_t ra = (tok0 + ta) * p.DHV + (size_t)blk * p.dv + v0;
               if (ta < Lc) {
