@@ -104,6 +104,56 @@ __device__ __forceinline__ void gate_vals(const TcParams& p, size_t tok, int hea
   }
 }
 
+// ---- rarely taken walk steps, kept out of line so that the per-chunk code stays compact
+// (it is executed once per chunk by each role and must stay in the instruction cache).
+// rows t of a 64 x DK bf16 tile (128-byte swizzled 64-column blocks) scaled by w[t]; the
+// threads gt = 0..nthreads-1 of a group share the work
+template <int DK>
+__device__ __noinline__ void scale_rows_bf16(uint32_t base_u, const float* w, int gt, int nthreads) {
+  constexpr int NCH = DK / 8;  // 16-byte chunks per row
+  for (int i = gt; i < L * NCH; i += nthreads) {
+    const int row = i / NCH, ch = i % NCH;
+    const uint32_t a = base_u + (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
+    st_shared_v4u(a, scale_bf16x8(ld_shared_v4(a), w[row]));
+  }
+}
+// the DK fp32 columns of this thread's TMEM lane (address taddr) scaled by f; called by the
+// whole warp
+template <int DK>
+__device__ __noinline__ void scale_tmem_lane(uint32_t taddr, float f) {
+  for (int c0 = 0; c0 < DK; c0 += 32) {
+    float r[32];
+    tmem_ld32(taddr + c0, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 32; ++j) r[j] *= f;
+    tmem_st16(taddr + c0, *reinterpret_cast<float(*)[16]>(r));
+    tmem_st16(taddr + c0 + 16, *reinterpret_cast<float(*)[16]>(r + 16));
+  }
+  tmem_wait_st();
+}
+// h tile staged in shared memory (64 tokens x DVT values, 128-byte swizzled 64-value blocks)
+// multiplied by the output gate og[t][d] (og points at token t0, value column v0; row stride
+// ld), tokens t < Lc; the 128 threads of the output group share the work
+template <int DVT>
+__device__ __noinline__ void apply_ogate(uint32_t hs_u, const __nv_bfloat16* og, size_t ld, int Lc, int gt) {
+  constexpr int NCH = DVT / 8;
+  for (int i = gt; i < Lc * NCH; i += 128) {
+    const int t = i / NCH, d = 8 * (i % NCH);
+    const uint32_t a = hs_u + (d >> 6) * 8192 + t * 128 + ((((d & 63) >> 3) ^ (t & 7)) << 4);
+    uint4 h = ld_shared_v4(a);
+    const uint4 o = *reinterpret_cast<const uint4*>(og + t * ld + d);
+    __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&h);
+    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&o);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 x = __bfloat1622float2(h2[j]), y = __bfloat1622float2(o2[j]);
+      h2[j] = __floats2bfloat162_rn(x.x * y.x, x.y * y.y);
+    }
+    st_shared_v4u(a, h);
+  }
+}
+
 }  // namespace
 
 // ===================================================================== gate preparation
@@ -793,46 +843,27 @@ __global__ void __launch_bounds__(NTW, 1)
       const bool guard = (flags & GF_GUARD) != 0;
       fin = G.scal[4];
       {
-        // bf16 snapshot of (scaled) C into TMEM; C itself rewritten only when lam moves
-        if (!(flags & GF_STORE_C)) {
-          // the common case: C is already in the units of the snapshot
+        // bf16 snapshot of C into TMEM.  When lam moves (rare) C is first rescaled in place
+        // to the snapshot's units, and after the snapshot to the units of the update.
+        const float cbs = G.scal[1], csc = G.scal[2];
+        if (flags & GF_STORE_C) scale_tmem_lane<DK>(tm + lane_off + TM_C, cbs);
 #pragma unroll 1
-          for (int c0 = 0; c0 < DK; c0 += 64) {
-            float r[64];
-            tmem_ld32(tm + lane_off + TM_C + c0, *reinterpret_cast<float(*)[32]>(r));
-            tmem_ld32(tm + lane_off + TM_C + c0 + 32, *reinterpret_cast<float(*)[32]>(r + 32));
-            tmem_wait_ld();
-            float pk[16];
+        for (int c0 = 0; c0 < DK; c0 += 64) {
+          float r[64];
+          tmem_ld32(tm + lane_off + TM_C + c0, *reinterpret_cast<float(*)[32]>(r));
+          tmem_ld32(tm + lane_off + TM_C + c0 + 32, *reinterpret_cast<float(*)[32]>(r + 32));
+          tmem_wait_ld();
+          float pk[16];
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
+          for (int h2 = 0; h2 < 2; ++h2) {
 #pragma unroll
-              for (int j = 0; j < 16; ++j) pk[j] = __uint_as_float(pack_bf16(r[32 * h2 + 2 * j], r[32 * h2 + 2 * j + 1]));
-              tmem_st16(tm + lane_off + TM_CB + c0 / 2 + 16 * h2, pk);
-            }
+            for (int j = 0; j < 16; ++j) pk[j] = __uint_as_float(pack_bf16(r[32 * h2 + 2 * j], r[32 * h2 + 2 * j + 1]));
+            tmem_st16(tm + lane_off + TM_CB + c0 / 2 + 16 * h2, pk);
           }
-        } else {
-          const float cbs = G.scal[1], csc = G.scal[2];
-#pragma unroll 1
-          for (int c0 = 0; c0 < DK; c0 += 64) {
-            float r[64];
-            tmem_ld32(tm + lane_off + TM_C + c0, *reinterpret_cast<float(*)[32]>(r));
-            tmem_ld32(tm + lane_off + TM_C + c0 + 32, *reinterpret_cast<float(*)[32]>(r + 32));
-            tmem_wait_ld();
-            float pk[16];
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-#pragma unroll
-              for (int j = 0; j < 16; ++j)
-                pk[j] = __uint_as_float(pack_bf16(r[32 * h2 + 2 * j] * cbs, r[32 * h2 + 2 * j + 1] * cbs));
-              tmem_st16(tm + lane_off + TM_CB + c0 / 2 + 16 * h2, pk);
-            }
-#pragma unroll
-            for (int h4 = 0; h4 < 4; ++h4) {
-#pragma unroll
-              for (int j = 0; j < 16; ++j) pk[j] = r[16 * h4 + j] * csc;
-              tmem_st16(tm + lane_off + TM_C + c0 + 16 * h4, pk);
-            }
-          }
+        }
+        if ((flags & GF_STORE_C) && csc != cbs) {
+          tmem_wait_st();
+          scale_tmem_lane<DK>(tm + lane_off + TM_C, csc / cbs);
         }
         tmem_wait_st();
       }
@@ -879,26 +910,7 @@ __global__ void __launch_bounds__(NTW, 1)
         // guarded chunk: Q <- e^{b_t+m_c-m_t} Q once the S MMA has read the raw Q, then the
         // read-out with the scaled Q
         if (!group_wait(&bars.s_full[b], (c >> 1) & 1, 0, first)) break;
-        const int gt = st;
-        constexpr int NQ = L * (DK / 8) / 128;  // 16-byte chunks per thread
-        constexpr int BATCH = NQ < 8 ? NQ : 8;
-        const uint32_t qs_u = smem_u32(Qs);
-#pragma unroll
-        for (int k0 = 0; k0 < NQ; k0 += BATCH) {
-          uint4 u[BATCH];
-          float wr[BATCH];
-          int offs[BATCH];
-#pragma unroll
-          for (int k = 0; k < BATCH; ++k) {
-            const int i = (k0 + k) * 128 + gt;
-            const int row = i / (DK / 8), ch = i % (DK / 8);
-            offs[k] = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
-            u[k] = ld_shared_v4(qs_u + offs[k]);
-            wr[k] = G.sq[row];
-          }
-#pragma unroll
-          for (int k = 0; k < BATCH; ++k) st_shared_v4u(qs_u + offs[k], scale_bf16x8(u[k], wr[k]));
-        }
+        scale_rows_bf16<DK>(smem_u32(Qs), G.sq, st, 128);
         fence_proxy_async_smem();
       }
       named_bar(WG_STATE, 128);
@@ -1017,15 +1029,8 @@ __global__ void __launch_bounds__(NTW, 1)
         const int r_lo = 16 * quarter + (lane >> 2), r_hi = r_lo + 8, cp = 2 * (lane & 3);
         float r[32], f_lo[16], f_hi[16];
         tmem_ld16x256_x8(tm + ((uint32_t)(32 * quarter) << 16) + TM_S, r);
-        // element factors: fast chunk u_s (columns only); guarded e^{al_t + be_s}
-        if (!(__float_as_int(G.scal[0]) & GF_GUARD)) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float2 u2 = *reinterpret_cast<const float2*>(G.u + 8 * j + cp);
-            f_lo[2 * j] = f_hi[2 * j] = u2.x;
-            f_lo[2 * j + 1] = f_hi[2 * j + 1] = u2.y;
-          }
-        } else {
+        // element factors e^{al_t + be_s} (a fast chunk has al = 0, be = log2 u_s)
+        {
           const float al_lo = G.al[r_lo], al_hi = G.al[r_hi];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
@@ -1121,34 +1126,13 @@ __global__ void __launch_bounds__(NTW, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) r[j] = r2[j];
           }
-          // value rows of this half: d_lo = base + lane/4 (r[2j], r[2j+1]) and d_lo + 8 (r[16+..])
+          // value rows of this half: base + lane/4 (r[2j], r[2j+1]) and base + lane/4 + 8 (r[16+..])
           const int base = DVT == 128 ? 32 * quarter + 16 * hf : 16 * quarter;
-          const int d_lo = base + (lane >> 2), d_hi = d_lo + 8;
           uint32_t plo[8], phi[8];
-          if (!use_og) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              plo[j] = pack_bf16(r[2 * j] * s0[j], r[2 * j + 1] * s1[j]);
-              phi[j] = pack_bf16(r[16 + 2 * j] * s0[j], r[16 + 2 * j + 1] * s1[j]);
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              float x0 = r[2 * j] * s0[j], x1 = r[2 * j + 1] * s1[j];
-              float y0 = r[16 + 2 * j] * s0[j], y1 = r[16 + 2 * j + 1] * s1[j];
-              const int ta = 8 * j + cp;
-              const size_t ra = (tok0 + ta) * p.DHV + (size_t)blk * p.dv + v0;
-              if (ta < Lc) {
-                x0 *= __bfloat162float(p.og[ra + d_lo]);
-                y0 *= __bfloat162float(p.og[ra + d_hi]);
-              }
-              if (ta + 1 < Lc) {
-                x1 *= __bfloat162float(p.og[ra + p.DHV + d_lo]);
-                y1 *= __bfloat162float(p.og[ra + p.DHV + d_hi]);
-              }
-              plo[j] = pack_bf16(x0, x1);
-              phi[j] = pack_bf16(y0, y1);
-            }
+          for (int j = 0; j < 8; ++j) {
+            plo[j] = pack_bf16(r[2 * j] * s0[j], r[2 * j + 1] * s1[j]);
+            phi[j] = pack_bf16(r[16 + 2 * j] * s0[j], r[16 + 2 * j + 1] * s1[j]);
           }
           // transposed: matrices (values lo, tokens 8j), (hi, 8j), (lo, 8j+8), (hi, 8j+8)
           const int d0 = base + ((lane >> 3) & 1) * 8;
@@ -1159,6 +1143,10 @@ __global__ void __launch_bounds__(NTW, 1)
             stmatrix_x4_trans(addr, plo[j], phi[j], plo[j + 1], phi[j + 1]);
           }
         }
+      }
+      if (use_og) {  // h <- h o o_t on the staged tile
+        named_bar(WG_OUT, 128);
+        apply_ogate<DVT>(hs_u, p.og + tok0 * p.DHV + (size_t)blk * p.dv + v0, p.DHV, Lc, gt);
       }
       fence_proxy_async_smem();
       named_bar(WG_OUT, 128);

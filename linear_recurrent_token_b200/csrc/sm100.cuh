@@ -53,12 +53,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 // Bounded wait on phase `parity`.  Gives up after ~`limit_cycles` SM cycles and
 // returns false (the caller records an error and winds down instead of hanging).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit_cycles = 4000000000LL) {
-  if (mbar_try_wait(bar, parity)) return true;
+// The polling loop is out of line: kernels with many wait sites keep one copy of it, which
+// stays in the instruction cache.
+__device__ __noinline__ bool mbar_wait_loop(uint64_t* bar, uint32_t parity, long long limit_cycles) {
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity))
     if (clock64() - t0 > limit_cycles) return false;
   return true;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit_cycles = 4000000000LL) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_loop(bar, parity, limit_cycles);
 }
 
 // One lane of the (fully active) warp returns true.
