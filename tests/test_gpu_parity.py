@@ -272,6 +272,10 @@ TC_CASES = [
     (1, 1, 64, 64, 64, 1, False, False, False),
     (1, 2, 130, 64, 128, 1, False, True, False),
     (1, 8, 4096, 256, 512, 1, False, True, True),
+    # two / four value tiles of a head run as a cluster and share the key-side work
+    (1, 2, 1000, 128, 256, 1, False, True, True),
+    (2, 2, 700, 64, 256, 1, True, True, False),
+    (1, 3, 777, 64, 512, 1, False, True, True),
 ]
 
 
@@ -341,10 +345,11 @@ GATE_REGIMES = {
 }
 
 
+@pytest.mark.parametrize("DHV", [128, 512])
 @pytest.mark.parametrize("regime", list(GATE_REGIMES))
-def test_tensor_core_gate_regimes(regime):
+def test_tensor_core_gate_regimes(regime, DHV):
     cfg = GATE_REGIMES[regime]
-    B, NH, S, DHQK, DHV = 1, 2, 1536, 128, 128
+    B, NH, S, DHQK = 1, 2, 1536, 128
     w = inputs.Workload(3, "regime", B, NH, S, DHQK, DHV, 64, 1, "bf16", False, 1 / np.sqrt(DHQK))
     assert mlstm.plan(mlstm.fwd_params(B, NH, S, DHQK, DHV, 64, 1, torch.bfloat16, False))["tensor_core"] == 1
     inp = inputs.forward_inputs(w, seed=31)
