@@ -346,11 +346,12 @@ __global__ void __launch_bounds__(NT, 1)
         const uint4 u = *reinterpret_cast<const uint4*>(kt + sw128_offset(s, dcol & 63));
         const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
         const float w = om[s];
+        const float2 w2 = make_float2(w, w);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float2 f = __bfloat1622float2(b2[j]);
-          dacc[2 * j] += w * f.x;
-          dacc[2 * j + 1] += w * f.y;
+          const float2 d = __ffma2_rn(__bfloat1622float2(b2[j]), w2, make_float2(dacc[2 * j], dacc[2 * j + 1]));
+          dacc[2 * j] = d.x;
+          dacc[2 * j + 1] = d.y;
         }
       }
     }
@@ -877,7 +878,7 @@ __global__ void __launch_bounds__(NTW, 1)
         const uint32_t qs_u = smem_u32(Qs);
         constexpr int NCH = DK / 16;
         constexpr int BATCH = NCH < 8 ? NCH : 8;
-        float a0 = 0.f, a1 = 0.f;
+        float2 a0 = make_float2(0.f, 0.f), a1 = a0;  // packed fp32 accumulators
 #pragma unroll 1
         for (int j0 = 0; j0 < NCH; j0 += BATCH) {
           uint4 u[BATCH];
@@ -892,17 +893,13 @@ __global__ void __launch_bounds__(NTW, 1)
             const float4 n0 = *reinterpret_cast<const float4*>(nvec + col);
             const float4 n1 = *reinterpret_cast<const float4*>(nvec + col + 4);
             const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u[j]);
-            float2 f = __bfloat1622float2(b2[0]);
-            a0 += f.x * n0.x + f.y * n0.y;
-            f = __bfloat1622float2(b2[1]);
-            a1 += f.x * n0.z + f.y * n0.w;
-            f = __bfloat1622float2(b2[2]);
-            a0 += f.x * n1.x + f.y * n1.y;
-            f = __bfloat1622float2(b2[3]);
-            a1 += f.x * n1.z + f.y * n1.w;
+            a0 = __ffma2_rn(__bfloat1622float2(b2[0]), make_float2(n0.x, n0.y), a0);
+            a1 = __ffma2_rn(__bfloat1622float2(b2[1]), make_float2(n0.z, n0.w), a1);
+            a0 = __ffma2_rn(__bfloat1622float2(b2[2]), make_float2(n1.x, n1.y), a0);
+            a1 = __ffma2_rn(__bfloat1622float2(b2[3]), make_float2(n1.z, n1.w), a1);
           }
         }
-        float a = a0 + a1;
+        float a = (a0.x + a0.y) + (a1.x + a1.y);
         a += __shfl_xor_sync(0xffffffffu, a, 1);
         if (part == 0) G.nq[t] = a;
       }
@@ -921,24 +918,21 @@ __global__ void __launch_bounds__(NTW, 1)
         const int cg = st % NCG, rg = st / NCG;
         const int col = 8 * cg;
         const uint8_t* kt = Ks + (col >> 6) * 8192;
-        float acc[8];
+        float2 acc[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+        for (int j = 0; j < 4; ++j) acc[j] = make_float2(0.f, 0.f);
 #pragma unroll 4
         for (int j = 0; j < RPG; ++j) {
           const int srow = rg * RPG + j;
           const uint4 u = *reinterpret_cast<const uint4*>(kt + sw128_offset(srow, col & 63));
           const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
           const float w = G.u[srow];
+          const float2 w2 = make_float2(w, w);
 #pragma unroll
-          for (int q2 = 0; q2 < 4; ++q2) {
-            const float2 f = __bfloat1622float2(b2[q2]);
-            acc[2 * q2] += w * f.x;
-            acc[2 * q2 + 1] += w * f.y;
-          }
+          for (int q2 = 0; q2 < 4; ++q2) acc[q2] = __ffma2_rn(__bfloat1622float2(b2[q2]), w2, acc[q2]);
         }
-        *reinterpret_cast<float4*>(npart + st * 8) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        *reinterpret_cast<float4*>(npart + st * 8 + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        *reinterpret_cast<float4*>(npart + st * 8) = make_float4(acc[0].x, acc[0].y, acc[1].x, acc[1].y);
+        *reinterpret_cast<float4*>(npart + st * 8 + 4) = make_float4(acc[2].x, acc[2].y, acc[3].x, acc[3].y);
         named_bar(WG_STATE, 128);
         const float ns = G.scal[3];
         for (int cc = st; cc < DK; cc += 128) {
@@ -1051,10 +1045,13 @@ __global__ void __launch_bounds__(NTW, 1)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int s0 = 8 * j + cp;
-          const float a0 = s0 <= lim_lo ? r[2 * j] * f_lo[2 * j] : 0.f;
-          const float a1 = s0 + 1 <= lim_lo ? r[2 * j + 1] * f_lo[2 * j + 1] : 0.f;
-          const float b0 = s0 <= lim_hi ? r[16 + 2 * j] * f_hi[2 * j] : 0.f;
-          const float b1 = s0 + 1 <= lim_hi ? r[16 + 2 * j + 1] * f_hi[2 * j + 1] : 0.f;
+          const float2 pa = __fmul2_rn(make_float2(r[2 * j], r[2 * j + 1]), make_float2(f_lo[2 * j], f_lo[2 * j + 1]));
+          const float2 pb =
+              __fmul2_rn(make_float2(r[16 + 2 * j], r[16 + 2 * j + 1]), make_float2(f_hi[2 * j], f_hi[2 * j + 1]));
+          const float a0 = s0 <= lim_lo ? pa.x : 0.f;
+          const float a1 = s0 + 1 <= lim_lo ? pa.y : 0.f;
+          const float b0 = s0 <= lim_hi ? pb.x : 0.f;
+          const float b1 = s0 + 1 <= lim_hi ? pb.y : 0.f;
           rs_lo += a0 + a1;
           rs_hi += b0 + b1;
           plo[j] = pack_bf16(a0, a1);
@@ -1131,8 +1128,11 @@ __global__ void __launch_bounds__(NTW, 1)
           uint32_t plo[8], phi[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            plo[j] = pack_bf16(r[2 * j] * s0[j], r[2 * j + 1] * s1[j]);
-            phi[j] = pack_bf16(r[16 + 2 * j] * s0[j], r[16 + 2 * j + 1] * s1[j]);
+            const float2 sc = make_float2(s0[j], s1[j]);
+            const float2 x = __fmul2_rn(make_float2(r[2 * j], r[2 * j + 1]), sc);
+            const float2 y = __fmul2_rn(make_float2(r[16 + 2 * j], r[16 + 2 * j + 1]), sc);
+            plo[j] = pack_bf16(x.x, x.y);
+            phi[j] = pack_bf16(y.x, y.y);
           }
           // transposed: matrices (values lo, tokens 8j), (hi, 8j), (lo, 8j+8), (hi, 8j+8)
           const int d0 = base + ((lane >> 3) & 1) * 8;
