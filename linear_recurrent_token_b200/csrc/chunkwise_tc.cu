@@ -30,6 +30,8 @@
 // workspace error word, stops issuing work, frees its TMEM and returns.
 #include <cuda_bf16.h>
 
+#include <utility>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -163,6 +165,7 @@ __device__ __noinline__ void apply_ogate(uint32_t hs_u, const __nv_bfloat16* og,
 // itilde = -inf (b and Xc keep the last token's values, X = -inf), so consumers need no
 // bounds logic; the chunk totals are the values of token 63.
 __global__ void __launch_bounds__(256) tc_gate_prep_kernel(TcParams p, int BH) {
+  grid_dep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long wid = (long long)blockIdx.x * 8 + warp;
   if (wid >= (long long)BH * p.ncp) return;
@@ -262,6 +265,8 @@ __global__ void __launch_bounds__(NT, 1)
   if (tid == 0)
     for (int c = 0; c < NS - 1 && c < nck; ++c) issue(c);
 
+  grid_dep_launch();
+  grid_dep_wait();  // the gate planes come from the preparation kernel
   // ---- gates: Gtot = sum of the chunk totals, and for token s of chunk c the log weight
   // Gtot - G_s + itilde_s = Gtot - Gpre_c + X_s (Gpre_c: totals of the earlier chunks of the
   // segment); M = its maximum = max_c (Gtot - Gpre_c + max X of chunk c); omega_s = e^{. - M}
@@ -553,6 +558,7 @@ __global__ void __launch_bounds__(NTW, 1)
   tc_fence_after();
   const uint32_t tm = tmem_base;
 
+  grid_dep_wait();  // summaries and gate planes come from the kernels before this one
   // ---- start state of the segment (see the file header); warps 3-10 fill TMEM and n.
   // It is stabilised at m_start, so lam starts at m_start.
   float m_start = ret ? 0.f : (p.m0 ? p.m0[bh] : 0.f);
@@ -1211,6 +1217,24 @@ size_t tc_workspace_bytes(const TcPlan& pl, long long BH, int nb, int dk, int dv
   return off;
 }
 
+// Launch that may overlap the previous kernel of the stream (programmatic stream
+// serialization); the kernel waits (griddepcontrol.wait) before it reads that kernel's results.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, int smem, cudaStream_t stream,
+                                    Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <int DK, int DVT>
 static cudaError_t launch_tc_dk(const TcPlan& pl, const TcParams& prm, const CUtensorMap& mq, const CUtensorMap& mk,
                                 const CUtensorMap& mv, const CUtensorMap& mh, long long slices, cudaStream_t stream,
@@ -1225,8 +1249,7 @@ static cudaError_t launch_tc_dk(const TcPlan& pl, const TcParams& prm, const CUt
     e = cudaFuncSetAttribute(tc_segment_kernel<DK, DVT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemA);
     if (e != cudaSuccess) return e;
     dim3 gridA(pl.n_tiles, pl.G - 1, (unsigned)slices);
-    tc_segment_kernel<DK, DVT><<<gridA, NT, smemA, stream>>>(mk, mv, prm);
-    e = cudaGetLastError();
+    e = launch_dependent(tc_segment_kernel<DK, DVT>, gridA, dim3(NT), smemA, stream, mk, mv, prm);
     if (e != cudaSuccess) return e;
   }
   const int smemC = WalkSmem<DK, DVT>::BYTES;
@@ -1234,8 +1257,7 @@ static cudaError_t launch_tc_dk(const TcPlan& pl, const TcParams& prm, const CUt
   if (e != cudaSuccess) return e;
   if (ev0) cudaEventRecord(ev0, stream);
   dim3 gridC(pl.n_tiles, pl.G, (unsigned)slices);
-  tc_walk_kernel<DK, DVT><<<gridC, NTW, smemC, stream>>>(mq, mk, mv, mh, prm);
-  e = cudaGetLastError();
+  e = launch_dependent(tc_walk_kernel<DK, DVT>, gridC, dim3(NTW), smemC, stream, mq, mk, mv, mh, prm);
   if (ev1) cudaEventRecord(ev1, stream);
   return e;
 }

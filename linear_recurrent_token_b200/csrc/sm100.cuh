@@ -66,6 +66,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
   return mbar_wait_loop(bar, parity, limit_cycles);
 }
 
+// ------------------------------------------------------------------ dependent launches
+// A kernel launched with programmatic stream serialization may start before the previous
+// kernel of the stream has finished; it waits here before touching that kernel's results.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// lets the next kernel of the stream (if launched that way) start its setup now
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // One lane of the (fully active) warp returns true.
 __device__ __forceinline__ bool elect_one() {
   uint32_t pred = 0;
