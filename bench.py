@@ -288,8 +288,11 @@ def run_chunkwise(w, steps, warmup, flush_bytes, clocks):
 
 
 def run_chunkwise_e2e(w, steps, tensors):
-    """Same prefill through the public API with HOST buffers: pinned host inputs copied in,
-    the call, h and the final state copied back, all inside the timed region."""
+    """Same prefill through the public API with HOST buffers: every step copies its pinned
+    host inputs in, runs the call and copies h and the final state back, all inside the timed
+    region.  Steps are pipelined the way a serving loop would run them: step i+1's inputs
+    upload on one stream while step i computes on another and step i-1's outputs download on
+    a third (device inputs and outputs double-buffered); per step time = total / steps."""
     import torch
 
     from linear_recurrent_token_b200 import mlstm
@@ -297,32 +300,65 @@ def run_chunkwise_e2e(w, steps, tensors):
     pin = lambda t: t.cpu().pin_memory()
     hq, hk, hv, hig, hfg = pin(q), pin(k), pin(v), pin(ig), pin(fg)
     oh, oC, on_, om = (torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (h, C, n, m))
-    stream = torch.cuda.current_stream()
-    gi = (None, None) if w.retention else (ig, fg)
+    # second device copies of the per-step tensors
+    dev_in = [(q, k, v, ig, fg), tuple(torch.empty_like(t) for t in (q, k, v, ig, fg))]
+    dev_out = [(h, C, n, m), tuple(torch.empty_like(t) for t in (h, C, n, m))]
+    s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    in_free = [torch.cuda.Event() for _ in range(2)]
+    out_ready = [torch.cuda.Event() for _ in range(2)]
+    out_free = [torch.cuda.Event() for _ in range(2)]
 
-    def one():
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True)
-        if not w.retention:
-            ig.copy_(hig, non_blocking=True)
-            fg.copy_(hfg, non_blocking=True)
-        mlstm.fwd_chunkwise(q, k, v, *gi, chunk=w.chunk, num_blocks=w.num_blocks, retention=w.retention,
-                            h=h, C_out=C, n_out=None if w.retention else n, m_out=None if w.retention else m,
-                            workspace=ws, stream=stream)
-        oh.copy_(h, non_blocking=True)
-        oC.copy_(C, non_blocking=True)
-        if not w.retention:
-            on_.copy_(n, non_blocking=True)
-            om.copy_(m, non_blocking=True)
+    def upload(i):
+        b = i % 2
+        s_in.wait_event(in_free[b])
+        with torch.cuda.stream(s_in):
+            for d, hsrc in zip(dev_in[b], (hq, hk, hv, hig, hfg)):
+                if w.retention and d.dtype == torch.float32 and d.dim() == 3:
+                    continue
+                d.copy_(hsrc, non_blocking=True)
+        in_ready[b].record(s_in)
 
-    one()
+    def run(i):
+        b = i % 2
+        qq, kk, vv, gi_, gf_ = dev_in[b]
+        hh, CC, nn, mm = dev_out[b]
+        s_run.wait_event(in_ready[b])
+        s_run.wait_event(out_free[b])
+        gates = (None, None) if w.retention else (gi_, gf_)
+        mlstm.fwd_chunkwise(qq, kk, vv, *gates, chunk=w.chunk, num_blocks=w.num_blocks, retention=w.retention,
+                            h=hh, C_out=CC, n_out=None if w.retention else nn, m_out=None if w.retention else mm,
+                            workspace=ws, stream=s_run)
+        in_free[b].record(s_run)
+        out_ready[b].record(s_run)
+
+    def download(i):
+        b = i % 2
+        s_out.wait_event(out_ready[b])
+        with torch.cuda.stream(s_out):
+            outs = (oh, oC) + (() if w.retention else (on_, om))
+            for dst, src in zip(outs, dev_out[b]):
+                dst.copy_(src, non_blocking=True)
+        out_free[b].record(s_out)
+
+    def pipeline(nsteps):
+        upload(0)
+        for i in range(nsteps):
+            if i + 1 < nsteps:
+                upload(i + 1)
+            run(i)
+            download(i)
+
+    for b in range(2):  # events start signalled
+        in_free[b].record(s_run)
+        out_free[b].record(s_out)
+    pipeline(2)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        one()
-    e1.record(stream)
+    e0.record(s_in)
+    pipeline(steps)
+    s_in.wait_stream(s_out)
+    e1.record(s_in)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
     h2d = sum(t.numel() * t.element_size() for t in ((hq, hk, hv) + (() if w.retention else (hig, hfg))))
@@ -362,21 +398,56 @@ def run_decode(w, steps, warmup, clocks):
     clocks.mark(False)
     step_ms = [e_a.elapsed_time(e_b) / steps] * steps
 
-    # end to end: per step, pinned host q/k/v/gates in, the step, h out
+    # end to end: per step, pinned host q/k/v/gates in, the step, h out; pipelined as in a
+    # serving loop (step t+1's inputs upload while step t runs and step t-1's h downloads)
     hq, hk, hv = (x[:1].cpu().pin_memory() for x in (q, k, v))
     hig, hfg = (x[:1].cpu().pin_memory() for x in (ig, fg))
     oh = torch.empty(h[0].shape, dtype=td).pin_memory()
+    s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_ran = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for b_ in range(2):
+        ev_ran[b_].record(s_run)
+        ev_out[b_].record(s_out)
+
+    def upload(i):
+        b_ = i % 2
+        s_in.wait_event(ev_ran[b_])  # step i-2 is done with slot b_
+        with torch.cuda.stream(s_in):
+            for d, src in zip((q, k, v, ig, fg), (hq, hk, hv, hig, hfg)):
+                d[b_].copy_(src[0], non_blocking=True)
+        ev_in[b_].record(s_in)
+
+    def run(i):
+        b_ = i % 2
+        s_run.wait_event(ev_in[b_])
+        s_run.wait_event(ev_out[b_])  # h slot b_ has been downloaded
+        mlstm.step(q[b_], k[b_], v[b_], ig[b_], fg[b_], C, n, m, h=h[b_], stream=s_run)
+        ev_ran[b_].record(s_run)
+
+    def download(i):
+        b_ = i % 2
+        s_out.wait_event(ev_ran[b_])
+        with torch.cuda.stream(s_out):
+            oh.copy_(h[b_], non_blocking=True)
+        ev_out[b_].record(s_out)
+
+    def pipeline(nsteps):
+        upload(0)
+        for i in range(nsteps):
+            if i + 1 < nsteps:
+                upload(i + 1)
+            run(i)
+            download(i)
+
+    pipeline(2)
+    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(steps):
-        q[0].copy_(hq[0], non_blocking=True)
-        k[0].copy_(hk[0], non_blocking=True)
-        v[0].copy_(hv[0], non_blocking=True)
-        ig[0].copy_(hig[0], non_blocking=True)
-        fg[0].copy_(hfg[0], non_blocking=True)
-        mlstm.step(q[0], k[0], v[0], ig[0], fg[0], C, n, m, h=h[0], stream=stream)
-        oh.copy_(h[0], non_blocking=True)
-    e1.record(stream)
+    e0.record(s_in)
+    pipeline(steps)
+    s_in.wait_stream(s_out)
+    e1.record(s_in)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / steps
     h2d = sum(x[0].numel() * x.element_size() for x in (hq, hk, hv, hig, hfg))
@@ -456,7 +527,7 @@ def main():
         mbytes = chunkwise_min_bytes(w.B, w.NH, w.S, w.DHQK, w.DHV, 2 if w.dtype == "bf16" else 4,
                                      w.num_blocks, w.retention)
         achieved_tf = flops / (main_ms * 1e-3) / 1e12
-        e2e_ms, h2d, d2h = run_chunkwise_e2e(w, max(3, args.steps // 4), cw["tensors"])
+        e2e_ms, h2d, d2h = run_chunkwise_e2e(w, max(8, args.steps // 2), cw["tensors"])
         e2e_ms = dist_max(e2e_ms, world)
         del cw["tensors"]
         torch.cuda.empty_cache()

@@ -1029,8 +1029,16 @@ __global__ void __launch_bounds__(NTW, 1)
         const int r_lo = 16 * quarter + (lane >> 2), r_hi = r_lo + 8, cp = 2 * (lane & 3);
         float r[32], f_lo[16], f_hi[16];
         tmem_ld16x256_x8(tm + ((uint32_t)(32 * quarter) << 16) + TM_S, r);
-        // element factors e^{al_t + be_s} (a fast chunk has al = 0, be = log2 u_s)
-        {
+        // element factors: u_s in a fast chunk (column factors only), e^{al_t + be_s} in a
+        // guarded one
+        if (!(__float_as_int(G.scal[0]) & GF_GUARD)) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float2 u2 = *reinterpret_cast<const float2*>(G.u + 8 * j + cp);
+            f_lo[2 * j] = f_hi[2 * j] = u2.x;
+            f_lo[2 * j + 1] = f_hi[2 * j + 1] = u2.y;
+          }
+        } else {
           const float al_lo = G.al[r_lo], al_hi = G.al[r_hi];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
