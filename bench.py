@@ -37,14 +37,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 CSRC = os.path.join(ROOT, "linear_recurrent_token_b200", "csrc")
 RECORDED_TRAFFIC = {
     ("tc_walk", "large_head"): {
-        "bytes": 147_772_672 + 40_033_536,
+        "bytes": 147_740_416 + 39_798_528,
         "sources": ("chunkwise_tc.cu", "sm100.cuh", "common.cuh", "kernels.h"),
-        "sha256": "979c5c2c01c90dd6a5829ab4e3df4e7f4d389cd157ba3b5db7ca1cfb83fab7bc",
+        "sha256": "96772aff29aced5d25e4279f3cc2916e5f147eba7dd7aa8fc48a87680352ef5b",
     },
     ("step", "decode"): {
-        "bytes": 540_051_712 + 480_060_160,
+        "bytes": 540_096_256 + 480_655_616,
         "sources": ("step.cu", "common.cuh", "kernels.h"),
-        "sha256": "b64fcb693c657680bc53ef26ac8af0727bb74fef23054abb5c4655cf58c4773c",
+        "sha256": "5bc4a28dcea130bc462276a009b0ebffab3b6b8680c42dcacd5b1d3fb15e6dc5",
     },
 }
 
