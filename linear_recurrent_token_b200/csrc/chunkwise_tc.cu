@@ -634,14 +634,21 @@ __global__ void __launch_bounds__(NTW, 1)
     named_bar(gi == 0 ? WG_STATE : WG_OUT, 128);
     return group_flag[gi] == 0;
   };
-  // warp-uniform bounded wait (one lane waits)
+  // warp-uniform bounded wait.  Every lane tests the barrier and a vote makes the verdict, so
+  // a phase that is already complete costs one shared-memory round trip (a lane-0 wait
+  // followed by a shuffle costs several, and under the SIMT groups' load each takes hundreds
+  // of cycles); otherwise the lanes poll with the bounded wait.
   auto warp_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
-    int ok = 1;
-    if (lane == 0 && (abort_flag || !mbar_wait(bar, parity, WAIT))) {
-      ok = 0;
-      abort_flag = 1;
-    }
-    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;
+    const bool ok = !abort_flag && mbar_wait(bar, parity, WAIT);
+    if (!ok) abort_flag = 1;
+    return __all_sync(0xffffffffu, ok);
+  };
+  // two barriers tested at once (both tests in flight together)
+  auto warp_wait2 = [&](uint64_t* b1, uint32_t p1, uint64_t* b2, uint32_t p2) -> bool {
+    const bool x = mbar_test_wait(b1, p1), y = mbar_test_wait(b2, p2);
+    if (__all_sync(0xffffffffu, x && y)) return true;
+    return warp_wait(b1, p1) && warp_wait(b2, p2);
   };
   const uint32_t id_s = idesc_bf16(64, 64, 0, 0);
   const uint32_t id_ro = idesc_bf16(DVT, 64, 0, 0);
@@ -776,9 +783,13 @@ __global__ void __launch_bounds__(NTW, 1)
       const uint64_t q_k = desc_k(c, 0);
       const uint64_t k_mn = smem_desc_sw128(sm_u + b * SM::STAGE + SM::QB, 8192, 1024);  // K, MN-major
       // update C += (V o u)^T K once the snapshot has read C and V o u is staged
-      if (!warp_wait(&bars.cb_ready, c & 1)) break;
-      if (!warp_wait(&bars.vw_full, c & 1)) break;
-      if (!warp_wait(&bars.full[b], (c >> 1) & 1)) break;
+      {
+        const bool x = mbar_test_wait(&bars.cb_ready, c & 1), y = mbar_test_wait(&bars.vw_full, c & 1),
+                   z = mbar_test_wait(&bars.full[b], (c >> 1) & 1);
+        if (!__all_sync(0xffffffffu, x && y && z) &&
+            !(warp_wait2(&bars.cb_ready, c & 1, &bars.vw_full, c & 1) && warp_wait(&bars.full[b], (c >> 1) & 1)))
+          break;
+      }
       tc_fence_after();
       if (elect_one()) {
 #pragma unroll
@@ -790,8 +801,13 @@ __global__ void __launch_bounds__(NTW, 1)
       // read-out of the snapshot; a guarded chunk first scales Q (the gate buffer is visible
       // here through the state group's cb_ready, which it arrived after reading it)
       const bool guard = (__float_as_int(gbuf(gi).scal[0]) & GF_GUARD) != 0;
-      if (guard && !warp_wait(&bars.q_ready[gi], (c / NGB) & 1)) break;
-      if (c > 0 && !warp_wait(&bars.h_empty, (c - 1) & 1)) break;
+      if (guard && c > 0) {
+        if (!warp_wait2(&bars.q_ready[gi], (c / NGB) & 1, &bars.h_empty, (c - 1) & 1)) break;
+      } else if (guard) {
+        if (!warp_wait(&bars.q_ready[gi], (c / NGB) & 1)) break;
+      } else if (c > 0 && !warp_wait(&bars.h_empty, (c - 1) & 1)) {
+        break;
+      }
       tc_fence_after();
       if (elect_one()) issue_readout(q_k, b);
       __syncwarp();
@@ -809,16 +825,14 @@ __global__ void __launch_bounds__(NTW, 1)
         // S of the next chunk once this chunk's S has left TMEM
         if (c + 1 < nck) {
           const uint64_t q_k1 = desc_k(c + 1, 0), k_k1 = desc_k(c + 1, 1);
-          if (!warp_wait(&bars.s_empty, c & 1)) break;
-          if (!warp_wait(&bars.full[b ^ 1], ((c + 1) >> 1) & 1)) break;
+          if (!warp_wait2(&bars.s_empty, c & 1, &bars.full[b ^ 1], ((c + 1) >> 1) & 1)) break;
           tc_fence_after();
           if (elect_one()) issue_s(q_k1, k_k1, b ^ 1);
           __syncwarp();
         }
         // P V onto the read-out (same accumulator, issued by the chain warp)
         const uint64_t v_mn = smem_desc_sw128(sm_u + b * SM::STAGE + SM::QB + SM::KB, 8192, 1024);
-        if (!warp_wait(&bars.p_full, c & 1)) break;
-        if (!warp_wait(&bars.ro_done, c & 1)) break;
+        if (!warp_wait2(&bars.p_full, c & 1, &bars.ro_done, c & 1)) break;
         tc_fence_after();
         if (elect_one()) {
 #pragma unroll
