@@ -108,13 +108,14 @@ __device__ __forceinline__ void gate_vals(const TcParams& p, size_t tok, int hea
 
 // ---- rarely taken walk steps, kept out of line so that the per-chunk code stays compact
 // (it is executed once per chunk by each role and must stay in the instruction cache).
-// rows t of a 64 x DK bf16 tile (128-byte swizzled 64-column blocks) scaled by w[t]; the
-// threads gt = 0..nthreads-1 of a group share the work
+// rows row0 .. row0+rows-1 of a 64 x DK bf16 tile (128-byte swizzled 64-column blocks), row t
+// scaled by w[t]; the threads gt = 0..nthreads-1 share the work
 template <int DK>
-__device__ __noinline__ void scale_rows_bf16(uint32_t base_u, const float* w, int gt, int nthreads) {
+__device__ __noinline__ void scale_rows_bf16(uint32_t base_u, const float* w, int gt, int nthreads, int row0,
+                                             int rows) {
   constexpr int NCH = DK / 8;  // 16-byte chunks per row
-  for (int i = gt; i < L * NCH; i += nthreads) {
-    const int row = i / NCH, ch = i % NCH;
+  for (int i = gt; i < rows * NCH; i += nthreads) {
+    const int row = row0 + i / NCH, ch = i % NCH;
     const uint32_t a = base_u + (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
     st_shared_v4u(a, scale_bf16x8(ld_shared_v4(a), w[row]));
   }
@@ -535,15 +536,15 @@ __global__ void __launch_bounds__(NTW, 1)
     for (int i = 0; i < NGB; ++i) {
       mbar_init(&bars.gfull[i], 1);
       mbar_init(&bars.gempty[i], 2);
-      mbar_init(&bars.q_ready[i], 1);
+      mbar_init(&bars.q_ready[i], 4);
     }
-    mbar_init(&bars.cb_ready, 1);
-    mbar_init(&bars.vw_full, 1);
+    mbar_init(&bars.cb_ready, 4);
+    mbar_init(&bars.vw_full, 4);
     mbar_init(&bars.upd_done, 1);
     mbar_init(&bars.ro_done, 1);
-    mbar_init(&bars.h_empty, 1);
-    mbar_init(&bars.s_empty, 1);
-    mbar_init(&bars.p_full, 1);
+    mbar_init(&bars.h_empty, 4);
+    mbar_init(&bars.s_empty, 4);
+    mbar_init(&bars.p_full, 4);
     mbar_init(&bars.mm_done, 1);
     abort_flag = 0;
     group_flag[0] = group_flag[1] = 0;
@@ -643,6 +644,15 @@ __global__ void __launch_bounds__(NTW, 1)
     const bool ok = !abort_flag && mbar_wait(bar, parity, WAIT);
     if (!ok) abort_flag = 1;
     return __all_sync(0xffffffffu, ok);
+  };
+  // wait of one warp of a SIMT group.  Warps of a group wait independently (no verdict is
+  // shared), so group code never leaves its loop on a failed wait: it runs on, every later
+  // wait returns at once, and the error flag reports the failure.  Named barriers stay only
+  // where data crosses warps.
+  auto gwait = [&](uint64_t* bar, uint32_t parity) {
+    if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return;
+    if (abort_flag || !mbar_wait(bar, parity, WAIT)) abort_flag = 1;
+    __syncwarp();
   };
   // two barriers tested at once (both tests in flight together)
   auto warp_wait2 = [&](uint64_t* b1, uint32_t p1, uint64_t* b2, uint32_t p2) -> bool {
@@ -856,9 +866,17 @@ __global__ void __launch_bounds__(NTW, 1)
       const GateBuf G = gbuf(gi);
       uint8_t* Qs = sm + b * SM::STAGE;
       uint8_t* Ks = Qs + SM::QB;
-      if (!group_wait(&bars.gfull[gi], (c / NGB) & 1, 0, first)) break;
-      // the previous read-out has read the snapshot and the previous update has written C
-      if (c > 0 && !group_wait(&bars.ro_done, (c - 1) & 1, 0, first)) break;
+      // the gate values, and (the previous read-out has read the snapshot and the previous
+      // update has written C)
+      if (c > 0) {
+        const bool x = mbar_test_wait(&bars.gfull[gi], (c / NGB) & 1), y = mbar_test_wait(&bars.ro_done, (c - 1) & 1);
+        if (!__all_sync(0xffffffffu, x && y)) {
+          gwait(&bars.gfull[gi], (c / NGB) & 1);
+          gwait(&bars.ro_done, (c - 1) & 1);
+        }
+      } else {
+        gwait(&bars.gfull[gi], 0);
+      }
       tc_fence_after();
       const int flags = __float_as_int(G.scal[0]);
       const bool guard = (flags & GF_GUARD) != 0;
@@ -889,9 +907,9 @@ __global__ void __launch_bounds__(NTW, 1)
         tmem_wait_st();
       }
       tc_fence_before();
-      named_bar(WG_STATE, 128);
-      if (first) mbar_arrive(&bars.cb_ready);
-      if (!group_wait(&bars.full[b], (c >> 1) & 1, 0, first)) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.cb_ready);  // this warp's lanes of the snapshot are written
+      gwait(&bars.full[b], (c >> 1) & 1);
       if (!ret) {
         // nq_t = n_st . q_t: two threads per token, DK/2 columns each (loads batched)
         const int t = st >> 1, part = st & 1;
@@ -925,13 +943,13 @@ __global__ void __launch_bounds__(NTW, 1)
       }
       if (guard) {
         // guarded chunk: Q <- e^{b_t+m_c-m_t} Q once the S MMA has read the raw Q, then the
-        // read-out with the scaled Q
-        if (!group_wait(&bars.s_full[b], (c >> 1) & 1, 0, first)) break;
-        scale_rows_bf16<DK>(smem_u32(Qs), G.sq, st, 128);
+        // read-out with the scaled Q.  A warp's n . q read exactly the 16 rows it scales.
+        gwait(&bars.s_full[b], (c >> 1) & 1);
+        scale_rows_bf16<DK>(smem_u32(Qs), G.sq, lane, 32, 16 * (st >> 5), 16);
         fence_proxy_async_smem();
       }
-      named_bar(WG_STATE, 128);
-      if (first) mbar_arrive(&bars.q_ready[gi]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.q_ready[gi]);  // this warp's tokens: n . q (and scaled Q)
       if (!ret) {
         // n <- ns n + sum_s u_s k_s
         constexpr int NCG = DK / 8, NRG = 128 / NCG, RPG = L / NRG;
@@ -953,7 +971,7 @@ __global__ void __launch_bounds__(NTW, 1)
         }
         *reinterpret_cast<float4*>(npart + st * 8) = make_float4(acc[0].x, acc[0].y, acc[1].x, acc[1].y);
         *reinterpret_cast<float4*>(npart + st * 8 + 4) = make_float4(acc[2].x, acc[2].y, acc[3].x, acc[3].y);
-        named_bar(WG_STATE, 128);
+        named_bar(WG_STATE, 128);  // the partials of all warps are stored
         const float ns = G.scal[3];
         for (int cc = st; cc < DK; cc += 128) {
           float x = 0.f;
@@ -962,7 +980,7 @@ __global__ void __launch_bounds__(NTW, 1)
           nvec[cc] = ns * nvec[cc] + x;
         }
       }
-      named_bar(WG_STATE, 128);
+      named_bar(WG_STATE, 128);  // n updated for the next chunk; the group is done with the stage
       if (first) {
         mbar_arrive(&bars.empty[b]);
         mbar_arrive(&bars.gempty[gi]);
@@ -1021,13 +1039,14 @@ __global__ void __launch_bounds__(NTW, 1)
       }
       fence_proxy_async_smem();
     };
-    bool ok = nck > 0 && group_wait(&bars.gfull[0], 0, 1, first) && group_wait(&bars.full[0], 0, 1, first);
-    if (ok) {
+    if (nck > 0) {
+      gwait(&bars.gfull[0], 0);
+      gwait(&bars.full[0], 0);
       scale_v(0);
-      named_bar(WG_OUT, 128);
-      if (first) mbar_arrive(&bars.vw_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.vw_full);  // this warp's share of V o u is stored
     }
-    for (int c = 0; ok && c < nck; ++c) {
+    for (int c = 0; c < nck; ++c) {
       const int b = c & 1, gi = c % NGB;
       const GateBuf G = gbuf(gi);
       const int t0 = T0 + c * L;
@@ -1035,8 +1054,15 @@ __global__ void __launch_bounds__(NTW, 1)
       const size_t tok0 = (size_t)bh * p.S + t0;
       // P = S o e^{al_t + be_s} (bf16, rows t, 128-byte swizzled) and its row sums; P V of
       // the previous chunk must be done with the P buffer
-      if (c > 0 && !group_wait(&bars.mm_done, (c - 1) & 1, 1, first)) break;
-      if (!group_wait(&bars.s_full[b], (c >> 1) & 1, 1, first)) break;
+      if (c > 0) {
+        const bool x = mbar_test_wait(&bars.mm_done, (c - 1) & 1), y = mbar_test_wait(&bars.s_full[b], (c >> 1) & 1);
+        if (!__all_sync(0xffffffffu, x && y)) {
+          gwait(&bars.mm_done, (c - 1) & 1);
+          gwait(&bars.s_full[b], (c >> 1) & 1);
+        }
+      } else {
+        gwait(&bars.s_full[b], 0);
+      }
       tc_fence_after();
       {
         // 16x256b load: thread -> rows 16q + lane/4 and +8, column pairs 8j + 2(lane%4)
@@ -1065,8 +1091,8 @@ __global__ void __launch_bounds__(NTW, 1)
         }
         tmem_wait_ld();
         tc_fence_before();
-        named_bar(WG_OUT, 128);
-        if (first) mbar_arrive(&bars.s_empty);  // S has left TMEM
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.s_empty);  // this warp's rows of S have left TMEM
         float rs_lo = 0.f, rs_hi = 0.f;
         uint32_t plo[8], phi[8];
         const int lim_lo = r_lo < Lc ? r_lo : -1, lim_hi = r_hi < Lc ? r_hi : -1;  // last column kept
@@ -1102,20 +1128,26 @@ __global__ void __launch_bounds__(NTW, 1)
         }
       }
       fence_proxy_async_smem();
-      named_bar(WG_OUT, 128);
-      if (first) mbar_arrive(&bars.p_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.p_full);  // this warp's rows of P are stored
       // V o u of the next chunk once this chunk's update has read the buffer
       if (c + 1 < nck) {
-        const int b1 = (c + 1) & 1;
-        if (!group_wait(&bars.gfull[(c + 1) % NGB], ((c + 1) / NGB) & 1, 1, first)) break;
-        if (!group_wait(&bars.full[b1], ((c + 1) >> 1) & 1, 1, first)) break;
-        if (!group_wait(&bars.upd_done, c & 1, 1, first)) break;
-        scale_v(c + 1);
-        named_bar(WG_OUT, 128);
-        if (first) mbar_arrive(&bars.vw_full);
+        const int c1 = c + 1, b1 = c1 & 1;
+        const bool x = mbar_test_wait(&bars.gfull[c1 % NGB], (c1 / NGB) & 1),
+                   y = mbar_test_wait(&bars.full[b1], (c1 >> 1) & 1), z = mbar_test_wait(&bars.upd_done, c & 1);
+        if (!__all_sync(0xffffffffu, x && y && z)) {
+          gwait(&bars.gfull[c1 % NGB], (c1 / NGB) & 1);
+          gwait(&bars.full[b1], (c1 >> 1) & 1);
+          gwait(&bars.upd_done, c & 1);
+        }
+        scale_v(c1);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.vw_full);
       }
-      // reciprocal denominators times the output scale E_t (nq_t from the state group)
-      if (!group_wait(&bars.q_ready[gi], (c / NGB) & 1, 1, first)) break;
+      // reciprocal denominators times the output scale E_t (nq_t from the state group, the row
+      // sums from all warps of this group)
+      gwait(&bars.q_ready[gi], (c / NGB) & 1);
+      named_bar(WG_OUT, 128);
       if (gt < L) {
         const int t = gt;
         const float e = G.E[t];
@@ -1124,7 +1156,8 @@ __global__ void __launch_bounds__(NTW, 1)
       // h_t = H_t rden_t (x o_t): H leaves TMEM first, then 8x8 tiles are stored transposed
       // into the 128-byte swizzled staging tile and TMA-stored
       if (first) bulk_wait_read_all();
-      if (!group_wait(&bars.mm_done, c & 1, 1, first)) break;
+      named_bar(WG_OUT, 128);  // rden is written and the previous h tile has left the staging tile
+      gwait(&bars.mm_done, c & 1);
       tc_fence_after();
       {
         constexpr int NH = DVT == 128 ? 2 : 1;  // 16-lane halves of this warp's quarter
@@ -1133,8 +1166,8 @@ __global__ void __launch_bounds__(NTW, 1)
         if (NH == 2) tmem_ld16x256_x8(tm + ((uint32_t)(32 * quarter + 16) << 16) + TM_H, r2);
         tmem_wait_ld();
         tc_fence_before();
-        named_bar(WG_OUT, 128);
-        if (first) mbar_arrive(&bars.h_empty);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.h_empty);  // this warp's lanes of H have left TMEM
         const int cp = 2 * (lane & 3);
         float s0[8], s1[8];
 #pragma unroll
