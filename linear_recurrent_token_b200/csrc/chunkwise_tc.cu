@@ -106,6 +106,27 @@ __device__ __forceinline__ void gate_vals(const TcParams& p, size_t tok, int hea
   }
 }
 
+// n as the B operand of warp-level m16n8k16 MMAs for n . q_t: n = hi + lo (two bf16 values,
+// so the products keep fp32 accuracy) in columns 0 and 1 of B.  Lane 4j + t (j = 0 hi, 1 lo,
+// t = (k%8)/2) holds, for each 16-row step kk = k/16, the pairs (16kk+2t, +1) and
+// (16kk+2t+8, +9); a lane's DK/4 values are contiguous, lanes DK/4 + 8 apart (16 bytes of
+// padding put the eight lanes' loads in different banks).
+template <int DK>
+__device__ __forceinline__ void store_nfrag(__nv_bfloat16* nf, int k, float v) {
+  const int kk = k >> 4, r = k & 15;
+  const int i = ((r & 7) >> 1) * (DK / 4 + 8) + kk * 4 + ((r >> 3) << 1) + (r & 1);
+  const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+  nf[i] = hi;
+  nf[i + 4 * (DK / 4 + 8)] = __float2bfloat16_rn(v - __bfloat162float(hi));
+}
+// bf16 pair (a, b) split as hi + lo: returns hi, lo in *lo
+__device__ __forceinline__ uint32_t split_bf16x2(float a, float b, uint32_t* lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const float2 f = __bfloat1622float2(h);
+  *lo = pack_bf16(a - f.x, b - f.y);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 // ---- rarely taken walk steps, kept out of line so that the per-chunk code stays compact
 // (it is executed once per chunk by each role and must stay in the instruction cache).
 // rows row0 .. row0+rows-1 of a 64 x DK bf16 tile (128-byte swizzled 64-column blocks), row t
@@ -462,9 +483,11 @@ struct WalkSmem {
   static constexpr int STAGE = QB + KB + VB;
   static constexpr int OVW = 2 * STAGE, OP = OVW + VB, OH = OP + PB;
   static constexpr int OF = OH + HB;  // floats start here
-  // n [DK], n partials [128*8], gate buffers [NGB][8][L], row sums / reciprocal denominators
-  // [2][L], gate scalars [NGB][8]
-  static constexpr int NF = DK + 128 * 8 + NGB * 8 * L + 2 * L + NGB * 8;
+  // n as a bf16 pair (hi + lo) in warp-MMA fragment order: 8 lanes x (DK/4 + 8 padding)
+  static constexpr int NFRAG = 8 * (DK / 4 + 8);
+  // n [DK], n fragments [2 buffers][NFRAG bf16], gate buffers [NGB][8][L], row sums / reciprocal
+  // denominators [2][L], gate scalars [NGB][8]
+  static constexpr int NF = DK + NFRAG + NGB * 8 * L + 2 * L + NGB * 8;
   static constexpr int BYTES = OF + NF * 4 + 1024;  // + alignment slack
 };
 
@@ -501,8 +524,8 @@ __global__ void __launch_bounds__(NTW, 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* Vw = sm + SM::OVW;
   float* nvec = reinterpret_cast<float*>(sm + SM::OF);
-  float* npart = nvec + DK;  // [128 * 8]
-  float* gmem = npart + 128 * 8;
+  __nv_bfloat16* nfrag = reinterpret_cast<__nv_bfloat16*>(nvec + DK);  // [2][NFRAG]
+  float* gmem = nvec + DK + SM::NFRAG;
   float* rsum = gmem + NGB * 8 * L;
   float* rden = rsum + L;
   float* gscal = rden + L;  // [NGB][8]
@@ -620,6 +643,7 @@ __global__ void __launch_bounds__(NTW, 1)
                p.dn[((size_t)slice * (p.G - 1) + jg) * p.dk + col];
         }
         nvec[col] = x;
+        store_nfrag<DK>(nfrag, col, x);
       }
   }
   tc_fence_before();
@@ -911,35 +935,29 @@ __global__ void __launch_bounds__(NTW, 1)
       if (lane == 0) mbar_arrive(&bars.cb_ready);  // this warp's lanes of the snapshot are written
       gwait(&bars.full[b], (c >> 1) & 1);
       if (!ret) {
-        // nq_t = n_st . q_t: two threads per token, DK/2 columns each (loads batched)
-        const int t = st >> 1, part = st & 1;
-        const uint32_t qs_u = smem_u32(Qs);
-        constexpr int NCH = DK / 16;
-        constexpr int BATCH = NCH < 8 ? NCH : 8;
-        float2 a0 = make_float2(0.f, 0.f), a1 = a0;  // packed fp32 accumulators
-#pragma unroll 1
-        for (int j0 = 0; j0 < NCH; j0 += BATCH) {
-          uint4 u[BATCH];
+        // nq_t = n_st . q_t for this warp's 16 tokens as warp-level MMAs: A = the Q rows
+        // (ldmatrix from the swizzled tile), B = n as hi + lo in columns 0 and 1 (lanes 0-7)
+        const int mi = lane >> 3, arow = 16 * (st >> 5) + (mi & 1) * 8 + (lane & 7);
+        const uint32_t a_row = smem_u32(Qs) + arow * 128;
+        const __nv_bfloat16* nf = nfrag + (c & 1) * SM::NFRAG + (lane & 7) * (DK / 4 + 8);
+        float d[4][4] = {};
 #pragma unroll
-          for (int j = 0; j < BATCH; ++j) {
-            const int col = part * (DK / 2) + 8 * (j0 + j);
-            u[j] = ld_shared_v4(qs_u + (col >> 6) * 8192 + sw128_offset(t, col & 63));
-          }
+        for (int kk = 0; kk < DK / 16; kk += 2) {
+          const uint4 bv = *reinterpret_cast<const uint4*>(nf + 4 * kk);
 #pragma unroll
-          for (int j = 0; j < BATCH; ++j) {
-            const int col = part * (DK / 2) + 8 * (j0 + j);
-            const float4 n0 = *reinterpret_cast<const float4*>(nvec + col);
-            const float4 n1 = *reinterpret_cast<const float4*>(nvec + col + 4);
-            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u[j]);
-            a0 = __ffma2_rn(__bfloat1622float2(b2[0]), make_float2(n0.x, n0.y), a0);
-            a1 = __ffma2_rn(__bfloat1622float2(b2[1]), make_float2(n0.z, n0.w), a1);
-            a0 = __ffma2_rn(__bfloat1622float2(b2[2]), make_float2(n1.x, n1.y), a0);
-            a1 = __ffma2_rn(__bfloat1622float2(b2[3]), make_float2(n1.z, n1.w), a1);
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int col = 16 * (kk + h2) + (mi >> 1) * 8;
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4(a_row + (col >> 6) * 8192 + ((((col & 63) >> 3) ^ (arow & 7)) << 4), a0, a1, a2, a3);
+            const uint32_t b0 = lane < 8 ? (h2 ? bv.z : bv.x) : 0u, b1 = lane < 8 ? (h2 ? bv.w : bv.y) : 0u;
+            mma_m16n8k16_bf16(d[(kk + h2) & 3], a0, a1, a2, a3, b0, b1);
           }
         }
-        float a = (a0.x + a0.y) + (a1.x + a1.y);
-        a += __shfl_xor_sync(0xffffffffu, a, 1);
-        if (part == 0) G.nq[t] = a;
+        if ((lane & 3) == 0) {
+          const int t = 16 * (st >> 5) + (lane >> 2);
+          G.nq[t] = ((d[0][0] + d[1][0]) + (d[2][0] + d[3][0])) + ((d[0][1] + d[1][1]) + (d[2][1] + d[3][1]));
+          G.nq[t + 8] = ((d[0][2] + d[1][2]) + (d[2][2] + d[3][2])) + ((d[0][3] + d[1][3]) + (d[2][3] + d[3][3]));
+        }
       }
       if (guard) {
         // guarded chunk: Q <- e^{b_t+m_c-m_t} Q once the S MMA has read the raw Q, then the
@@ -951,33 +969,44 @@ __global__ void __launch_bounds__(NTW, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.q_ready[gi]);  // this warp's tokens: n . q (and scaled Q)
       if (!ret) {
-        // n <- ns n + sum_s u_s k_s
-        constexpr int NCG = DK / 8, NRG = 128 / NCG, RPG = L / NRG;
-        const int cg = st % NCG, rg = st / NCG;
-        const int col = 8 * cg;
-        const uint8_t* kt = Ks + (col >> 6) * 8192;
-        float2 acc[4];
+        // n <- ns n + K^T u for this warp's DK/4 entries of n as warp-level MMAs: A = K^T
+        // (ldmatrix.trans of the swizzled K tile), B = u as hi + lo in columns 0 and 1 (lanes 0-7)
+        constexpr int MT = DK / 64;  // 16-entry tiles per warp
+        const int mi = lane >> 3, tq = lane & 3, k0 = (DK / 4) * (st >> 5);
+        uint32_t ub[L / 16][2];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[j] = make_float2(0.f, 0.f);
-#pragma unroll 4
-        for (int j = 0; j < RPG; ++j) {
-          const int srow = rg * RPG + j;
-          const uint4 u = *reinterpret_cast<const uint4*>(kt + sw128_offset(srow, col & 63));
-          const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-          const float w = G.u[srow];
-          const float2 w2 = make_float2(w, w);
-#pragma unroll
-          for (int q2 = 0; q2 < 4; ++q2) acc[q2] = __ffma2_rn(__bfloat1622float2(b2[q2]), w2, acc[q2]);
+        for (int ks = 0; ks < L / 16; ++ks) {
+          const float2 x = *reinterpret_cast<const float2*>(G.u + 16 * ks + 2 * tq);
+          const float2 y = *reinterpret_cast<const float2*>(G.u + 16 * ks + 2 * tq + 8);
+          uint32_t xl, yl;
+          const uint32_t xh = split_bf16x2(x.x, x.y, &xl), yh = split_bf16x2(y.x, y.y, &yl);
+          ub[ks][0] = lane < 4 ? xh : lane < 8 ? xl : 0u;
+          ub[ks][1] = lane < 4 ? yh : lane < 8 ? yl : 0u;
         }
-        *reinterpret_cast<float4*>(npart + st * 8) = make_float4(acc[0].x, acc[0].y, acc[1].x, acc[1].y);
-        *reinterpret_cast<float4*>(npart + st * 8 + 4) = make_float4(acc[2].x, acc[2].y, acc[3].x, acc[3].y);
-        named_bar(WG_STATE, 128);  // the partials of all warps are stored
-        const float ns = G.scal[3];
-        for (int cc = st; cc < DK; cc += 128) {
-          float x = 0.f;
+        const uint32_t ks_u = smem_u32(Ks);
+        float d[MT][4] = {};
 #pragma unroll
-          for (int r = 0; r < NRG; ++r) x += npart[(r * NCG + cc / 8) * 8 + (cc & 7)];
-          nvec[cc] = ns * nvec[cc] + x;
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+          for (int ks = 0; ks < L / 16; ++ks) {
+            const int srow = 16 * ks + (mi >> 1) * 8 + (lane & 7), m = k0 + 16 * mt + (mi & 1) * 8;
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4_trans(ks_u + (m >> 6) * 8192 + srow * 128 + ((((m & 63) >> 3) ^ (srow & 7)) << 4), a0, a1, a2,
+                              a3);
+            mma_m16n8k16_bf16(d[mt], a0, a1, a2, a3, ub[ks][0], ub[ks][1]);
+          }
+        if (tq == 0) {
+          const float ns = G.scal[3];
+          __nv_bfloat16* nf = nfrag + ((c + 1) & 1) * SM::NFRAG;
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int k = k0 + 16 * mt + (lane >> 2) + 8 * h2;
+              const float v = ns * nvec[k] + (d[mt][2 * h2] + d[mt][2 * h2 + 1]);
+              nvec[k] = v;
+              store_nfrag<DK>(nf, k, v);
+            }
         }
       }
       named_bar(WG_STATE, 128);  // n updated for the next chunk; the group is done with the stage
