@@ -127,6 +127,16 @@ __device__ __forceinline__ uint32_t split_bf16x2(float a, float b, uint32_t* lo)
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// Slow path of a warp's barrier wait (the phase was not complete when the warp tested it):
+// every lane polls with the bounded wait unless a failure is already recorded; returns the
+// warp's verdict and records a failure.  Out of line, so the per-chunk code keeps only the
+// test and the vote.
+__device__ __noinline__ bool warp_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  const bool ok = !*abort_flag && mbar_wait(bar, parity, WAIT);
+  if (!ok) *abort_flag = 1;
+  return __all_sync(0xffffffffu, ok);
+}
+
 // ---- rarely taken walk steps, kept out of line so that the per-chunk code stays compact
 // (it is executed once per chunk by each role and must stay in the instruction cache).
 // rows row0 .. row0+rows-1 of a 64 x DK bf16 tile (128-byte swizzled 64-column blocks), row t
@@ -664,25 +674,20 @@ __global__ void __launch_bounds__(NTW, 1)
   // followed by a shuffle costs several, and under the SIMT groups' load each takes hundreds
   // of cycles); otherwise the lanes poll with the bounded wait.
   auto warp_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
-    if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;
-    const bool ok = !abort_flag && mbar_wait(bar, parity, WAIT);
-    if (!ok) abort_flag = 1;
-    return __all_sync(0xffffffffu, ok);
+    return __all_sync(0xffffffffu, mbar_test_wait(bar, parity)) || warp_wait_slow(bar, parity, &abort_flag);
   };
   // wait of one warp of a SIMT group.  Warps of a group wait independently (no verdict is
   // shared), so group code never leaves its loop on a failed wait: it runs on, every later
   // wait returns at once, and the error flag reports the failure.  Named barriers stay only
   // where data crosses warps.
   auto gwait = [&](uint64_t* bar, uint32_t parity) {
-    if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return;
-    if (abort_flag || !mbar_wait(bar, parity, WAIT)) abort_flag = 1;
-    __syncwarp();
+    if (!__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) warp_wait_slow(bar, parity, &abort_flag);
   };
   // two barriers tested at once (both tests in flight together)
   auto warp_wait2 = [&](uint64_t* b1, uint32_t p1, uint64_t* b2, uint32_t p2) -> bool {
     const bool x = mbar_test_wait(b1, p1), y = mbar_test_wait(b2, p2);
     if (__all_sync(0xffffffffu, x && y)) return true;
-    return warp_wait(b1, p1) && warp_wait(b2, p2);
+    return warp_wait_slow(b1, p1, &abort_flag) && warp_wait_slow(b2, p2, &abort_flag);
   };
   const uint32_t id_s = idesc_bf16(64, 64, 0, 0);
   const uint32_t id_ro = idesc_bf16(DVT, 64, 0, 0);
@@ -692,7 +697,7 @@ __global__ void __launch_bounds__(NTW, 1)
   // elected lane only adds constant offsets.
   // S = Q K^T into the S columns; q_k, k_k: K-major descriptors of the chunk's Q and K
   auto issue_s = [&](uint64_t q_k, uint64_t k_k, int b) {
-#pragma unroll
+#pragma unroll 1
     for (int k = 0; k < DK; k += 16) {
       const uint64_t off = (uint64_t)(((k >> 6) * 8192 + (k & 63) * 2) >> 4);
       mma_bf16_ss(tm + TM_S, q_k + off, k_k + off, id_s, k > 0 ? 1u : 0u);
@@ -701,7 +706,7 @@ __global__ void __launch_bounds__(NTW, 1)
   };
   // read-out H = Cb Q^T (A = the bf16 snapshot in TMEM); releases stage b with the update
   auto issue_readout = [&](uint64_t q_k, int b) {
-#pragma unroll
+#pragma unroll 1
     for (int k = 0; k < DK; k += 16)
       mma_bf16_ts(tm + TM_H, tm + TM_CB + k / 2, q_k + (uint64_t)(((k >> 6) * 8192 + (k & 63) * 2) >> 4), id_ro,
                   k > 0 ? 1u : 0u);
@@ -816,15 +821,22 @@ __global__ void __launch_bounds__(NTW, 1)
       const int b = c & 1, gi = c % NGB;
       const uint64_t q_k = desc_k(c, 0);
       const uint64_t k_mn = smem_desc_sw128(sm_u + b * SM::STAGE + SM::QB, 8192, 1024);  // K, MN-major
-      // update C += (V o u)^T K once the snapshot has read C and V o u is staged
+      // update C += (V o u)^T K once the snapshot has read C and V o u is staged; whether the
+      // previous h has left TMEM (for the read-out) is tested in the same batch
+      bool h_free;
       {
         const bool x = mbar_test_wait(&bars.cb_ready, c & 1), y = mbar_test_wait(&bars.vw_full, c & 1),
                    z = mbar_test_wait(&bars.full[b], (c >> 1) & 1);
+        h_free = c == 0 || mbar_test_wait(&bars.h_empty, (c - 1) & 1);
         if (!__all_sync(0xffffffffu, x && y && z) &&
-            !(warp_wait2(&bars.cb_ready, c & 1, &bars.vw_full, c & 1) && warp_wait(&bars.full[b], (c >> 1) & 1)))
+            !(warp_wait_slow(&bars.cb_ready, c & 1, &abort_flag) && warp_wait_slow(&bars.vw_full, c & 1, &abort_flag) &&
+              warp_wait_slow(&bars.full[b], (c >> 1) & 1, &abort_flag)))
           break;
       }
       tc_fence_after();
+      // the gate buffer is visible here through the state group's cb_ready, which it arrived
+      // after reading the buffer; a guarded chunk scales Q before its read-out
+      const int flags = __float_as_int(gbuf(gi).scal[0]);
       if (elect_one()) {
 #pragma unroll
         for (int ks = 0; ks < L / 16; ++ks)
@@ -832,17 +844,12 @@ __global__ void __launch_bounds__(NTW, 1)
         mma_commit(&bars.upd_done);
       }
       __syncwarp();
-      // read-out of the snapshot; a guarded chunk first scales Q (the gate buffer is visible
-      // here through the state group's cb_ready, which it arrived after reading it)
-      const bool guard = (__float_as_int(gbuf(gi).scal[0]) & GF_GUARD) != 0;
-      if (guard && c > 0) {
-        if (!warp_wait2(&bars.q_ready[gi], (c / NGB) & 1, &bars.h_empty, (c - 1) & 1)) break;
-      } else if (guard) {
-        if (!warp_wait(&bars.q_ready[gi], (c / NGB) & 1)) break;
-      } else if (c > 0 && !warp_wait(&bars.h_empty, (c - 1) & 1)) {
-        break;
+      const bool guard = (flags & GF_GUARD) != 0;
+      if (guard || !__all_sync(0xffffffffu, h_free)) {
+        if (guard && !warp_wait_slow(&bars.q_ready[gi], (c / NGB) & 1, &abort_flag)) break;
+        if (c > 0 && !warp_wait_slow(&bars.h_empty, (c - 1) & 1, &abort_flag)) break;
+        tc_fence_after();
       }
-      tc_fence_after();
       if (elect_one()) issue_readout(q_k, b);
       __syncwarp();
     }
@@ -856,14 +863,6 @@ __global__ void __launch_bounds__(NTW, 1)
       __syncwarp();
       for (int c = 0; c < nck; ++c) {
         const int b = c & 1;
-        // S of the next chunk once this chunk's S has left TMEM
-        if (c + 1 < nck) {
-          const uint64_t q_k1 = desc_k(c + 1, 0), k_k1 = desc_k(c + 1, 1);
-          if (!warp_wait2(&bars.s_empty, c & 1, &bars.full[b ^ 1], ((c + 1) >> 1) & 1)) break;
-          tc_fence_after();
-          if (elect_one()) issue_s(q_k1, k_k1, b ^ 1);
-          __syncwarp();
-        }
         // P V onto the read-out (same accumulator, issued by the chain warp)
         const uint64_t v_mn = smem_desc_sw128(sm_u + b * SM::STAGE + SM::QB + SM::KB, 8192, 1024);
         if (!warp_wait2(&bars.p_full, c & 1, &bars.ro_done, c & 1)) break;
@@ -876,6 +875,15 @@ __global__ void __launch_bounds__(NTW, 1)
           mma_commit(&bars.empty[b]);
         }
         __syncwarp();
+        // S of the next chunk after this chunk's read-out and P V in the tensor pipe (the
+        // recurrence's MMAs never queue behind it), once this chunk's S has left TMEM
+        if (c + 1 < nck) {
+          const uint64_t q_k1 = desc_k(c + 1, 0), k_k1 = desc_k(c + 1, 1);
+          if (!warp_wait2(&bars.s_empty, c & 1, &bars.full[b ^ 1], ((c + 1) >> 1) & 1)) break;
+          tc_fence_after();
+          if (elect_one()) issue_s(q_k1, k_k1, b ^ 1);
+          __syncwarp();
+        }
       }
     }
   } else if (warp < 7) {
@@ -895,8 +903,8 @@ __global__ void __launch_bounds__(NTW, 1)
       if (c > 0) {
         const bool x = mbar_test_wait(&bars.gfull[gi], (c / NGB) & 1), y = mbar_test_wait(&bars.ro_done, (c - 1) & 1);
         if (!__all_sync(0xffffffffu, x && y)) {
-          gwait(&bars.gfull[gi], (c / NGB) & 1);
-          gwait(&bars.ro_done, (c - 1) & 1);
+          warp_wait_slow(&bars.gfull[gi], (c / NGB) & 1, &abort_flag);
+          warp_wait_slow(&bars.ro_done, (c - 1) & 1, &abort_flag);
         }
       } else {
         gwait(&bars.gfull[gi], 0);
@@ -1086,8 +1094,8 @@ __global__ void __launch_bounds__(NTW, 1)
       if (c > 0) {
         const bool x = mbar_test_wait(&bars.mm_done, (c - 1) & 1), y = mbar_test_wait(&bars.s_full[b], (c >> 1) & 1);
         if (!__all_sync(0xffffffffu, x && y)) {
-          gwait(&bars.mm_done, (c - 1) & 1);
-          gwait(&bars.s_full[b], (c >> 1) & 1);
+          warp_wait_slow(&bars.mm_done, (c - 1) & 1, &abort_flag);
+          warp_wait_slow(&bars.s_full[b], (c >> 1) & 1, &abort_flag);
         }
       } else {
         gwait(&bars.s_full[b], 0);
@@ -1165,9 +1173,9 @@ __global__ void __launch_bounds__(NTW, 1)
         const bool x = mbar_test_wait(&bars.gfull[c1 % NGB], (c1 / NGB) & 1),
                    y = mbar_test_wait(&bars.full[b1], (c1 >> 1) & 1), z = mbar_test_wait(&bars.upd_done, c & 1);
         if (!__all_sync(0xffffffffu, x && y && z)) {
-          gwait(&bars.gfull[c1 % NGB], (c1 / NGB) & 1);
-          gwait(&bars.full[b1], (c1 >> 1) & 1);
-          gwait(&bars.upd_done, c & 1);
+          warp_wait_slow(&bars.gfull[c1 % NGB], (c1 / NGB) & 1, &abort_flag);
+          warp_wait_slow(&bars.full[b1], (c1 >> 1) & 1, &abort_flag);
+          warp_wait_slow(&bars.upd_done, c & 1, &abort_flag);
         }
         scale_v(c1);
         __syncwarp();
