@@ -44,7 +44,7 @@ using namespace sm100;
 namespace {
 
 constexpr int L = 64;            // chunk length of the tensor-core path
-constexpr int NT = 256;          // phase A threads per CTA (2 warps per TMEM lane quarter)
+constexpr int NTA = 192;         // phase A threads per CTA (producer, MMA warp, 4 SIMT warps)
 constexpr int NSA = 4;           // phase A TMA stages
 constexpr long long WAIT = 4000000000LL;
 
@@ -133,6 +133,21 @@ __device__ __forceinline__ uint32_t split_bf16x2(float a, float b, uint32_t* lo)
 // test and the vote.
 __device__ __noinline__ bool warp_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   const bool ok = !*abort_flag && mbar_wait(bar, parity, WAIT);
+  if (!ok) *abort_flag = 1;
+  return __all_sync(0xffffffffu, ok);
+}
+// The same for up to three barriers (unused ones null): each round tests all of them at once,
+// so the warp resumes one shared-memory round trip after the last phase completes.
+__device__ __noinline__ bool warp_wait_slow3(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1, uint64_t* b2,
+                                             uint32_t p2, volatile int* abort_flag) {
+  bool ok = !*abort_flag;
+  const long long t0 = clock64();
+  while (ok) {
+    const bool x = mbar_test_wait(b0, p0), y = b1 == nullptr || mbar_test_wait(b1, p1),
+               z = b2 == nullptr || mbar_test_wait(b2, p2);
+    if (x && y && z) break;
+    if (clock64() - t0 > WAIT) ok = false;
+  }
   if (!ok) *abort_flag = 1;
   return __all_sync(0xffffffffu, ok);
 }
@@ -240,9 +255,16 @@ __global__ void __launch_bounds__(256) tc_gate_prep_kernel(TcParams p, int BH) {
 }
 
 // ===================================================================== phase A
-// CTA = (value tile, segment < G-1, slice); 256 threads.  Four TMA stages of (K, V).
+// CTA = (value tile, segment < G-1, slice); 192 threads in three roles, four TMA stages of
+// (K, V) with per-stage barriers:
+//   warp 0     producer: TMA loads of stage c % NS once the MMAs of chunk c - NS are done,
+//              then the chunk's weights omega_s (second arrival on the stage's full barrier)
+//   warp 1     MMA warp: D[dv, dk] += (V o omega)^T K once the SIMT group has scaled V
+//   warps 2-5  SIMT group: V rows scaled in place by omega, dn partials (this tile's share of
+//              the key columns); at the end the TMEM accumulator and dn go to global memory
+// The roles only meet at mbarriers, so the SIMT work of later stages overlaps the MMAs.
 template <int DK, int DVT>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NTA, 1)
     tc_segment_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV, TcParams p) {
   constexpr int KB = DK * 128;   // bytes of one K chunk tile (DK/64 boxes of 8 KiB)
   constexpr int VB = DVT * 128;  // bytes of one V chunk tile
@@ -250,13 +272,13 @@ __global__ void __launch_bounds__(NT, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // stage i: K at sm + i*(KB+VB), V right after it
-  float* dnp = reinterpret_cast<float*>(sm + NS * (KB + VB));  // [NT * 8] partial sums of dn
-  float* omb = dnp + NT * 8;                                    // [2][L] weights of the chunk
-  float* coff = omb + 2 * L;                                    // [seg_chunks]
-  __shared__ uint64_t bar_load[NS], bar_mma[NS];
+  float* dnp = reinterpret_cast<float*>(sm + NS * (KB + VB));  // [128 * 8] partial sums of dn
+  float* omb = dnp + 128 * 8;                                   // [NS][L] weights of the stage's chunk
+  float* coff = omb + NS * L;                                   // [seg_chunks]
+  __shared__ uint64_t full[NS], scaled[NS], mma_done[NS], all_done;
   __shared__ uint32_t tmem_base;
-  __shared__ float red[NT / 32];
-  __shared__ int abort_flag;
+  __shared__ float red[NTA / 32];
+  __shared__ volatile int abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.x, g = blockIdx.y, slice = blockIdx.z;
@@ -268,12 +290,15 @@ __global__ void __launch_bounds__(NT, 1)
   const int dnw = ((DK + p.n_tiles - 1) / p.n_tiles + 7) / 8 * 8;
   const int dn0 = tile * dnw;
   const bool do_dn = !p.retention && dn0 < DK;
+  const int nck = p.seg_chunks;
 
   if (tid == 0) {
     for (int i = 0; i < NS; ++i) {
-      mbar_init(&bar_load[i], 1);
-      mbar_init(&bar_mma[i], 1);
+      mbar_init(&full[i], 2);  // the TMA arrival (with its bytes) and the weights
+      mbar_init(&scaled[i], 4);
+      mbar_init(&mma_done[i], 1);
     }
+    mbar_init(&all_done, 1);
     abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&mapK);
@@ -284,18 +309,18 @@ __global__ void __launch_bounds__(NT, 1)
   tc_fence_after();
   const uint32_t tm = tmem_base;
 
-  const int nck = p.seg_chunks;
-  auto issue = [&](int c) {
+  auto issue = [&](int c) {  // one lane
     const int st = c % NS;
     uint8_t* kb = sm + st * (KB + VB);
-    mbar_arrive_expect_tx(&bar_load[st], KB + VB);
+    mbar_arrive_expect_tx(&full[st], KB + VB);
     for (int j = 0; j < DK / 64; ++j)
-      tma_load_3d(kb + j * 8192, &mapK, blk * p.dk + 64 * j, T0 + c * L, bh, &bar_load[st]);
+      tma_load_3d(kb + j * 8192, &mapK, blk * p.dk + 64 * j, T0 + c * L, bh, &full[st]);
     for (int j = 0; j < DVT / 64; ++j)
-      tma_load_3d(kb + KB + j * 8192, &mapV, blk * p.dv + v0 + 64 * j, T0 + c * L, bh, &bar_load[st]);
+      tma_load_3d(kb + KB + j * 8192, &mapV, blk * p.dv + v0 + 64 * j, T0 + c * L, bh, &full[st]);
   };
+  // K and V are inputs: the first stages load while the previous kernel finishes
   if (tid == 0)
-    for (int c = 0; c < NS - 1 && c < nck; ++c) issue(c);
+    for (int c = 0; c < NS && c < nck; ++c) issue(c);
 
   grid_dep_launch();
   grid_dep_wait();  // the gate planes come from the preparation kernel
@@ -314,7 +339,7 @@ __global__ void __launch_bounds__(NT, 1)
     if (lane == 31) red[warp] = inc;
     __syncthreads();
     float wexcl = 0.f, total = 0.f;
-    for (int w = 0; w < NT / 32; ++w) {
+    for (int w = 0; w < NTA / 32; ++w) {
       if (w < warp) wexcl += red[w];
       total += red[w];
     }
@@ -325,7 +350,7 @@ __global__ void __launch_bounds__(NT, 1)
     if (lane == 0) red[warp] = lmax;
     __syncthreads();
     float Mg = -INFINITY;
-    for (int w = 0; w < NT / 32; ++w) Mg = fmaxf(Mg, red[w]);
+    for (int w = 0; w < NTA / 32; ++w) Mg = fmaxf(Mg, red[w]);
     if (p.retention) Mg = 0.f;
     if (tid < nck) coff[tid] = total - gpre - Mg;
     if (tile == 0 && blk == 0 && tid == 0) {
@@ -334,119 +359,132 @@ __global__ void __launch_bounds__(NT, 1)
     }
     __syncthreads();
   }
-  // omega_s = e^{coff_c + X_s}, formed per chunk (the X_s of the next chunk in a register)
-  const float* gxr = p.gx + (size_t)bh * p.sp + T0;
-  float gxn = tid < L ? gxr[tid] : 0.f;
+  // warp-uniform test of a barrier, bounded wait out of line when the phase is not complete
+  auto warp_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    return __all_sync(0xffffffffu, mbar_test_wait(bar, parity)) || warp_wait_slow(bar, parity, &abort_flag);
+  };
 
-  // ---- main loop: D[dv, dk] += (V o omega)^T K over the segment
-  const uint32_t idesc = idesc_bf16(DVT, DK, 1, 1);
-  // dn partials: thread -> (column group of 8 inside this tile's columns, row group)
-  const int ncg = dnw / 8 < NT ? dnw / 8 : NT, nrg = NT / ncg, rows_per = (L + nrg - 1) / nrg;
-  const int cg = tid % ncg, rg = tid / ncg;
-  const int dcol = dn0 + 8 * cg;  // first of this thread's 8 columns
-  float dacc[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) dacc[j] = 0.f;
-  for (int c = 0; c < nck; ++c) {
-    const int st = c % NS;
-    uint8_t* Kst = sm + st * (KB + VB);
-    uint8_t* Vst = Kst + KB;
-    float* om = omb + (c & 1) * L;
-    if (tid < L) {
-      om[tid] = expf(coff[c] + gxn);
-      if (c + 1 < nck) gxn = gxr[(c + 1) * L + tid];
-    }
-    if (!abort_flag && !mbar_wait(&bar_load[st], (c / NS) & 1, WAIT)) atomicOr(&abort_flag, 1);
-    __syncthreads();
-    if (abort_flag) break;
-    {
-      // V rows scaled in place by omega (loads batched ahead of the stores)
-      constexpr int NV = L * (DVT / 8) / NT;
-      const uint32_t v_u = smem_u32(Vst);
-      uint4 u[NV];
-      float wr[NV];
-      int offs[NV];
-#pragma unroll
-      for (int k = 0; k < NV; ++k) {
-        const int i = k * NT + tid;
-        const int row = i / (DVT / 8), ch = i % (DVT / 8);
-        offs[k] = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
-        u[k] = ld_shared_v4(v_u + offs[k]);
-        wr[k] = om[row];
+  if (warp == 0) {
+    // =============================================================== producer
+    // omega_s = e^{coff_c + X_s}: lane -> tokens 2 lane, 2 lane + 1 (X of the next chunk
+    // prefetched into registers)
+    const float* gxr = p.gx + (size_t)bh * p.sp + T0 + 2 * lane;
+    float2 gxn = *reinterpret_cast<const float2*>(gxr);
+    for (int c = 0; c < nck; ++c) {
+      const int st = c % NS;
+      if (c >= NS) {
+        // the stage's previous chunk has been read by its MMAs (and by the SIMT group before)
+        if (!warp_wait(&mma_done[st], ((c / NS) - 1) & 1)) break;
+        if (lane == 0) issue(c);
       }
-#pragma unroll
-      for (int k = 0; k < NV; ++k) st_shared_v4u(v_u + offs[k], scale_bf16x8(u[k], wr[k]));
+      const float cf = coff[c];
+      *reinterpret_cast<float2*>(omb + st * L + 2 * lane) = make_float2(expf(cf + gxn.x), expf(cf + gxn.y));
+      if (c + 1 < nck) gxn = *reinterpret_cast<const float2*>(gxr + (size_t)(c + 1) * L);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full[st]);
     }
-    if (do_dn && rg < nrg && dcol < DK) {
-      const uint8_t* kt = Kst + (dcol >> 6) * 8192;
-      for (int s = rg * rows_per; s < min(L, (rg + 1) * rows_per); ++s) {
-        const uint4 u = *reinterpret_cast<const uint4*>(kt + sw128_offset(s, dcol & 63));
-        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-        const float w = om[s];
-        const float2 w2 = make_float2(w, w);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float2 d = __ffma2_rn(__bfloat1622float2(b2[j]), w2, make_float2(dacc[2 * j], dacc[2 * j + 1]));
-          dacc[2 * j] = d.x;
-          dacc[2 * j + 1] = d.y;
-        }
-      }
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (warp == 0) {
-      tc_fence_after();
-      const uint64_t ad = smem_desc_sw128(smem_u32(Vst), 8192, 1024);
+  } else if (warp == 1) {
+    // =============================================================== MMA warp
+    const uint32_t idesc = idesc_bf16(DVT, DK, 1, 1);
+    for (int c = 0; c < nck; ++c) {
+      const int st = c % NS;
+      uint8_t* Kst = sm + st * (KB + VB);
+      const uint64_t ad = smem_desc_sw128(smem_u32(Kst + KB), 8192, 1024);
       const uint64_t bd = smem_desc_sw128(smem_u32(Kst), 8192, 1024);
+      if (!warp_wait(&scaled[st], (c / NS) & 1)) break;
+      tc_fence_after();
       if (elect_one()) {
 #pragma unroll
         for (int ks = 0; ks < L / 16; ++ks)
           mma_bf16_ss(tm, ad + (uint64_t)(ks * 128), bd + (uint64_t)(ks * 128), idesc, (c > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(&bar_mma[st]);
-        // stage (c + NS - 1) % NS was last read by the MMAs of chunk c - 1 (queued before
-        // this chunk's): refill it once they are done; the other warps move on
-        if (c + NS - 1 < nck) {
-          if (c >= 1 && !mbar_wait(&bar_mma[(c - 1) % NS], ((c - 1) / NS) & 1, WAIT))
-            atomicOr(&abort_flag, 1);
-          else
-            issue(c + NS - 1);
-        }
+        mma_commit(&mma_done[st]);
+        if (c == nck - 1) mma_commit(&all_done);
       }
       __syncwarp();
     }
-  }
-  if (!abort_flag && !mbar_wait(&bar_mma[(nck - 1) % NS], ((nck - 1) / NS) & 1, WAIT)) atomicOr(&abort_flag, 1);
-  __syncthreads();
-  tc_fence_after();
-  if (!abort_flag) {
-    // warp w: TMEM lane quarter w % 4, column half w / 4
-    const int quarter = warp & 3, half = warp >> 2;
+  } else {
+    // =============================================================== SIMT group
+    const int gt = tid - 64;  // 0..127
+    // dn partials: thread -> (column group of 8 inside this tile's columns, row group)
+    const int ncg = dnw / 8 < 128 ? dnw / 8 : 128, nrg = 128 / ncg, rows_per = (L + nrg - 1) / nrg;
+    const int cg = gt % ncg, rg = gt / ncg;
+    const int dcol = dn0 + 8 * cg;  // first of this thread's 8 columns
+    float2 dacc[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) dacc[j] = make_float2(0.f, 0.f);
+    for (int c = 0; c < nck; ++c) {
+      const int st = c % NS;
+      uint8_t* Kst = sm + st * (KB + VB);
+      const float* om = omb + st * L;
+      // a failed wait leaves the loop of no warp: it runs on (later waits return at once)
+      // and the error flag reports it
+      if (!__all_sync(0xffffffffu, mbar_test_wait(&full[st], (c / NS) & 1)))
+        warp_wait_slow(&full[st], (c / NS) & 1, &abort_flag);
+      {
+        // V rows scaled in place by omega (loads batched ahead of the stores)
+        constexpr int NV = L * (DVT / 8) / 128;
+        const uint32_t v_u = smem_u32(Kst + KB);
+        uint4 u[NV];
+        float wr[NV];
+        int offs[NV];
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+          const int i = k * 128 + gt;
+          const int row = i / (DVT / 8), ch = i % (DVT / 8);
+          offs[k] = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
+          u[k] = ld_shared_v4(v_u + offs[k]);
+          wr[k] = om[row];
+        }
+#pragma unroll
+        for (int k = 0; k < NV; ++k) st_shared_v4u(v_u + offs[k], scale_bf16x8(u[k], wr[k]));
+      }
+      if (do_dn && rg < nrg && dcol < DK) {
+        const uint8_t* kt = Kst + (dcol >> 6) * 8192;
+        const int s1 = min(L, (rg + 1) * rows_per);
+#pragma unroll 4
+        for (int s = rg * rows_per; s < s1; ++s) {
+          const uint4 u = *reinterpret_cast<const uint4*>(kt + sw128_offset(s, dcol & 63));
+          const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+          const float w = om[s];
+          const float2 w2 = make_float2(w, w);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) dacc[j] = __ffma2_rn(__bfloat1622float2(b2[j]), w2, dacc[j]);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&scaled[st]);
+    }
+    // ---- epilogue: the accumulator (warp w reads TMEM lane quarter w % 4) and dn
+    if (!__all_sync(0xffffffffu, mbar_test_wait(&all_done, 0))) warp_wait_slow(&all_done, 0, &abort_flag);
+    tc_fence_after();
+    const int quarter = warp & 3;
     const int row = acc_row<DVT>(quarter, lane);
     float* dst = row >= 0 ? p.dC + (((size_t)slice * (p.G - 1) + g) * p.dv + v0 + row) * p.dk : nullptr;
-    for (int c0 = half * (DK / 2); c0 < (half + 1) * (DK / 2); c0 += 32) {
+#pragma unroll 1
+    for (int c0 = 0; c0 < DK; c0 += 32) {
       float r[32];
       tmem_ld32(tm + ((uint32_t)(32 * quarter) << 16) + c0, r);
       tmem_wait_ld();
-      if (dst)
+      if (dst && !abort_flag)
 #pragma unroll
         for (int j = 0; j < 32; j += 4)
           *reinterpret_cast<float4*>(dst + c0 + j) = make_float4(r[j], r[j + 1], r[j + 2], r[j + 3]);
     }
     if (do_dn) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) dnp[tid * 8 + j] = dacc[j];
-      __syncthreads();
-      for (int col = tid; col < ncg * 8 && dn0 + col < DK; col += NT) {
+      *reinterpret_cast<float4*>(dnp + gt * 8) = make_float4(dacc[0].x, dacc[0].y, dacc[1].x, dacc[1].y);
+      *reinterpret_cast<float4*>(dnp + gt * 8 + 4) = make_float4(dacc[2].x, dacc[2].y, dacc[3].x, dacc[3].y);
+      named_bar(1, 128);
+      for (int col = gt; col < ncg * 8 && dn0 + col < DK; col += 128) {
         float x = 0.f;
         for (int r = 0; r < nrg; ++r) x += dnp[(r * ncg + col / 8) * 8 + (col & 7)];
-        p.dn[((size_t)slice * (p.G - 1) + g) * p.dk + dn0 + col] = x;
+        if (!abort_flag) p.dn[((size_t)slice * (p.G - 1) + g) * p.dk + dn0 + col] = x;
       }
     }
-  } else if (tid == 0) {
-    atomicOr(p.err, 1u);
   }
   tc_fence_before();
   __syncthreads();
+  if (abort_flag && tid == 0) atomicOr(p.err, 1u);
   if (warp == 0) tmem_dealloc(tm, DK);
 }
 
@@ -687,7 +725,7 @@ __global__ void __launch_bounds__(NTW, 1)
   auto warp_wait2 = [&](uint64_t* b1, uint32_t p1, uint64_t* b2, uint32_t p2) -> bool {
     const bool x = mbar_test_wait(b1, p1), y = mbar_test_wait(b2, p2);
     if (__all_sync(0xffffffffu, x && y)) return true;
-    return warp_wait_slow(b1, p1, &abort_flag) && warp_wait_slow(b2, p2, &abort_flag);
+    return warp_wait_slow3(b1, p1, b2, p2, nullptr, 0, &abort_flag);
   };
   const uint32_t id_s = idesc_bf16(64, 64, 0, 0);
   const uint32_t id_ro = idesc_bf16(DVT, 64, 0, 0);
@@ -829,8 +867,7 @@ __global__ void __launch_bounds__(NTW, 1)
                    z = mbar_test_wait(&bars.full[b], (c >> 1) & 1);
         h_free = c == 0 || mbar_test_wait(&bars.h_empty, (c - 1) & 1);
         if (!__all_sync(0xffffffffu, x && y && z) &&
-            !(warp_wait_slow(&bars.cb_ready, c & 1, &abort_flag) && warp_wait_slow(&bars.vw_full, c & 1, &abort_flag) &&
-              warp_wait_slow(&bars.full[b], (c >> 1) & 1, &abort_flag)))
+            !warp_wait_slow3(&bars.cb_ready, c & 1, &bars.vw_full, c & 1, &bars.full[b], (c >> 1) & 1, &abort_flag))
           break;
       }
       tc_fence_after();
@@ -846,8 +883,9 @@ __global__ void __launch_bounds__(NTW, 1)
       __syncwarp();
       const bool guard = (flags & GF_GUARD) != 0;
       if (guard || !__all_sync(0xffffffffu, h_free)) {
-        if (guard && !warp_wait_slow(&bars.q_ready[gi], (c / NGB) & 1, &abort_flag)) break;
-        if (c > 0 && !warp_wait_slow(&bars.h_empty, (c - 1) & 1, &abort_flag)) break;
+        if (!warp_wait_slow3(&bars.h_empty, (c - 1) & 1, guard ? &bars.q_ready[gi] : nullptr, (c / NGB) & 1, nullptr, 0,
+                             &abort_flag))
+          break;
         tc_fence_after();
       }
       if (elect_one()) issue_readout(q_k, b);
@@ -902,10 +940,8 @@ __global__ void __launch_bounds__(NTW, 1)
       // update has written C)
       if (c > 0) {
         const bool x = mbar_test_wait(&bars.gfull[gi], (c / NGB) & 1), y = mbar_test_wait(&bars.ro_done, (c - 1) & 1);
-        if (!__all_sync(0xffffffffu, x && y)) {
-          warp_wait_slow(&bars.gfull[gi], (c / NGB) & 1, &abort_flag);
-          warp_wait_slow(&bars.ro_done, (c - 1) & 1, &abort_flag);
-        }
+        if (!__all_sync(0xffffffffu, x && y))
+          warp_wait_slow3(&bars.gfull[gi], (c / NGB) & 1, &bars.ro_done, (c - 1) & 1, nullptr, 0, &abort_flag);
       } else {
         gwait(&bars.gfull[gi], 0);
       }
@@ -1093,10 +1129,8 @@ __global__ void __launch_bounds__(NTW, 1)
       // the previous chunk must be done with the P buffer
       if (c > 0) {
         const bool x = mbar_test_wait(&bars.mm_done, (c - 1) & 1), y = mbar_test_wait(&bars.s_full[b], (c >> 1) & 1);
-        if (!__all_sync(0xffffffffu, x && y)) {
-          warp_wait_slow(&bars.mm_done, (c - 1) & 1, &abort_flag);
-          warp_wait_slow(&bars.s_full[b], (c >> 1) & 1, &abort_flag);
-        }
+        if (!__all_sync(0xffffffffu, x && y))
+          warp_wait_slow3(&bars.mm_done, (c - 1) & 1, &bars.s_full[b], (c >> 1) & 1, nullptr, 0, &abort_flag);
       } else {
         gwait(&bars.s_full[b], 0);
       }
@@ -1172,11 +1206,9 @@ __global__ void __launch_bounds__(NTW, 1)
         const int c1 = c + 1, b1 = c1 & 1;
         const bool x = mbar_test_wait(&bars.gfull[c1 % NGB], (c1 / NGB) & 1),
                    y = mbar_test_wait(&bars.full[b1], (c1 >> 1) & 1), z = mbar_test_wait(&bars.upd_done, c & 1);
-        if (!__all_sync(0xffffffffu, x && y && z)) {
-          warp_wait_slow(&bars.gfull[c1 % NGB], (c1 / NGB) & 1, &abort_flag);
-          warp_wait_slow(&bars.full[b1], (c1 >> 1) & 1, &abort_flag);
-          warp_wait_slow(&bars.upd_done, c & 1, &abort_flag);
-        }
+        if (!__all_sync(0xffffffffu, x && y && z))
+          warp_wait_slow3(&bars.gfull[c1 % NGB], (c1 / NGB) & 1, &bars.full[b1], (c1 >> 1) & 1, &bars.upd_done, c & 1,
+                          &abort_flag);
         scale_v(c1);
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.vw_full);
@@ -1337,11 +1369,11 @@ static cudaError_t launch_tc_dk(const TcPlan& pl, const TcParams& prm, const CUt
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (pl.G > 1) {
-    const int smemA = NSA * (DK * 128 + DVT * 128) + (NT * 8 + 2 * L + pl.seg_chunks) * 4 + 1024;
+    const int smemA = NSA * (DK * 128 + DVT * 128) + (128 * 8 + NSA * L + pl.seg_chunks) * 4 + 1024;
     e = cudaFuncSetAttribute(tc_segment_kernel<DK, DVT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemA);
     if (e != cudaSuccess) return e;
     dim3 gridA(pl.n_tiles, pl.G - 1, (unsigned)slices);
-    e = launch_dependent(tc_segment_kernel<DK, DVT>, gridA, dim3(NT), smemA, stream, mk, mv, prm);
+    e = launch_dependent(tc_segment_kernel<DK, DVT>, gridA, dim3(NTA), smemA, stream, mk, mv, prm);
     if (e != cudaSuccess) return e;
   }
   const int smemC = WalkSmem<DK, DVT>::BYTES;
