@@ -489,14 +489,15 @@ __global__ void __launch_bounds__(NTA, 1)
 }
 
 // ===================================================================== phase C
-// Warp-specialised walk: 11 warps.
-//   warp 0     producer: TMA loads of Q/K/V (two stages) and the per-chunk gate quantities
-//              (up to four chunks ahead)
-//   warp 1     chain MMAs: the chunk's update (C += (V o u)^T K) and read-out (H = Cb Q^T)
-//   warp 2     output MMAs: S = Q K^T of the next chunk and P V (H += V^T P^T)
-//   warps 3-6  state group: bf16 snapshot of C into TMEM (the read-out operand), n . q_t,
-//              Q scaling (guarded chunks only), n update
-//   warps 7-10 output group: P, V o u for the next chunk, denominators, h (TMA store)
+// Warp-specialised walk: 15 warps.
+//   warp 0       producer: TMA loads of Q/K/V (two stages) and the per-chunk gate quantities
+//                (up to four chunks ahead)
+//   warp 1       chain MMAs: the chunk's update (C += (V o u)^T K) and read-out (H = Cb Q^T)
+//   warp 2       output MMAs: P V (H += V^T P^T), then S = Q K^T of the next chunk
+//   warps 3-6    state group: bf16 snapshot of C into TMEM (the read-out operand), then
+//                V o u of the next chunk while the MMAs run
+//   warps 7-10   output group: P, denominators, h (TMA store)
+//   warps 11-14  n group: n . q_t, Q scaling (guarded chunks only), n update
 // MMAs are issued by warps that do nothing else: an issuing warp stalls for about the time
 // its MMAs take to execute, which would hold up a SIMT group.  Each issuing warp is
 // converged and one elected lane issues, with descriptors computed by the whole warp (an
@@ -519,9 +520,9 @@ __global__ void __launch_bounds__(NTA, 1)
 // "guarded": it uses the per-element stabilised form instead (C rescaled to units of
 // e^{m}, Q scaled by e^{b_t + m_c - m_t}, P = S o e^{b_t - m_t + X_s}, update weights
 // e^{g + X_s - m_next}); every fp32 / bf16 value then stays within e^{+-60} of 1.
-constexpr int NTW = 352;
-constexpr int NGB = 4;                   // gate buffers
-constexpr int WG_STATE = 1, WG_OUT = 2;  // named barrier ids of the two 128-thread groups
+constexpr int NTW = 480;
+constexpr int NGB = 4;                             // gate buffers
+constexpr int WG_STATE = 1, WG_OUT = 2, WG_N = 3;  // named barrier ids of the 128-thread groups
 constexpr float LAM_RENORM = 20.f;       // renormalise lam when the stabiliser is this far above
 constexpr float U_MAX_LOG = 60.f;        // largest log u_s a fast chunk may use
 
@@ -606,7 +607,7 @@ __global__ void __launch_bounds__(NTW, 1)
     }
     for (int i = 0; i < NGB; ++i) {
       mbar_init(&bars.gfull[i], 1);
-      mbar_init(&bars.gempty[i], 2);
+      mbar_init(&bars.gempty[i], 6);  // four state warps, the n and output groups
       mbar_init(&bars.q_ready[i], 4);
     }
     mbar_init(&bars.cb_ready, 4);
@@ -641,7 +642,7 @@ __global__ void __launch_bounds__(NTW, 1)
     if (!ret) m_start = fmaxf(A + m_start, Bm);
     gsum += A;
   }
-  if (warp >= 3) {
+  if (warp >= 3 && warp < 11) {
     const int quarter = warp & 3, half = (warp - 3) >> 2;
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     const int row = acc_row<DVT>(quarter, lane);
@@ -931,11 +932,40 @@ __global__ void __launch_bounds__(NTW, 1)
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     const bool first = st == 0;
     float fin = 1.f;
+    // V o u of chunk c into the update operand buffer (loads batched ahead of the stores)
+    auto scale_v = [&](int c) {
+      const GateBuf G = gbuf(c % NGB);
+      const uint32_t vs_u = sm_u + (c & 1) * SM::STAGE + SM::QB + SM::KB, vw_u2 = smem_u32(Vw);
+      constexpr int NV = L * (DVT / 8) / 128;  // 16-byte chunks per thread
+      constexpr int NB = NV < 4 ? NV : 4;       // per pass; the pass loop keeps the code small
+#pragma unroll 1
+      for (int k0 = 0; k0 < NV; k0 += NB) {
+        uint4 u[NB];
+        float wr[NB];
+        int offs[NB];
+#pragma unroll
+        for (int k = 0; k < NB; ++k) {
+          const int i = (k0 + k) * 128 + st;
+          const int row = i / (DVT / 8), ch = i % (DVT / 8);
+          offs[k] = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
+          u[k] = ld_shared_v4(vs_u + offs[k]);
+          wr[k] = G.u[row];
+        }
+#pragma unroll
+        for (int k = 0; k < NB; ++k) st_shared_v4u(vw_u2 + offs[k], scale_bf16x8(u[k], wr[k]));
+      }
+      fence_proxy_async_smem();
+    };
+    if (nck > 0) {
+      gwait(&bars.gfull[0], 0);
+      gwait(&bars.full[0], 0);
+      scale_v(0);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.vw_full);  // this warp's share of V o u is stored
+    }
     for (int c = 0; c < nck; ++c) {
-      const int b = c & 1, gi = c % NGB;
+      const int gi = c % NGB;
       const GateBuf G = gbuf(gi);
-      uint8_t* Qs = sm + b * SM::STAGE;
-      uint8_t* Ks = Qs + SM::QB;
       // the gate values, and (the previous read-out has read the snapshot and the previous
       // update has written C)
       if (c > 0) {
@@ -947,7 +977,6 @@ __global__ void __launch_bounds__(NTW, 1)
       }
       tc_fence_after();
       const int flags = __float_as_int(G.scal[0]);
-      const bool guard = (flags & GF_GUARD) != 0;
       fin = G.scal[4];
       {
         // bf16 snapshot of C into TMEM.  When lam moves (rare) C is first rescaled in place
@@ -976,163 +1005,63 @@ __global__ void __launch_bounds__(NTW, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.cb_ready);  // this warp's lanes of the snapshot are written
-      gwait(&bars.full[b], (c >> 1) & 1);
-      if (!ret) {
-        // nq_t = n_st . q_t for this warp's 16 tokens as warp-level MMAs: A = the Q rows
-        // (ldmatrix from the swizzled tile), B = n as hi + lo in columns 0 and 1 (lanes 0-7)
-        const int mi = lane >> 3, arow = 16 * (st >> 5) + (mi & 1) * 8 + (lane & 7);
-        const uint32_t a_row = smem_u32(Qs) + arow * 128;
-        const __nv_bfloat16* nf = nfrag + (c & 1) * SM::NFRAG + (lane & 7) * (DK / 4 + 8);
-        float d[4][4] = {};
-#pragma unroll
-        for (int kk = 0; kk < DK / 16; kk += 2) {
-          const uint4 bv = *reinterpret_cast<const uint4*>(nf + 4 * kk);
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int col = 16 * (kk + h2) + (mi >> 1) * 8;
-            uint32_t a0, a1, a2, a3;
-            ldmatrix_x4(a_row + (col >> 6) * 8192 + ((((col & 63) >> 3) ^ (arow & 7)) << 4), a0, a1, a2, a3);
-            const uint32_t b0 = lane < 8 ? (h2 ? bv.z : bv.x) : 0u, b1 = lane < 8 ? (h2 ? bv.w : bv.y) : 0u;
-            mma_m16n8k16_bf16(d[(kk + h2) & 3], a0, a1, a2, a3, b0, b1);
-          }
-        }
-        if ((lane & 3) == 0) {
-          const int t = 16 * (st >> 5) + (lane >> 2);
-          G.nq[t] = ((d[0][0] + d[1][0]) + (d[2][0] + d[3][0])) + ((d[0][1] + d[1][1]) + (d[2][1] + d[3][1]));
-          G.nq[t + 8] = ((d[0][2] + d[1][2]) + (d[2][2] + d[3][2])) + ((d[0][3] + d[1][3]) + (d[2][3] + d[3][3]));
-        }
+      if (lane == 0) {
+        mbar_arrive(&bars.cb_ready);  // this warp's lanes of the snapshot are written
+        mbar_arrive(&bars.gempty[gi]);  // and it is done with the chunk's gate buffer
       }
-      if (guard) {
-        // guarded chunk: Q <- e^{b_t+m_c-m_t} Q once the S MMA has read the raw Q, then the
-        // read-out with the scaled Q.  A warp's n . q read exactly the 16 rows it scales.
-        gwait(&bars.s_full[b], (c >> 1) & 1);
-        scale_rows_bf16<DK>(smem_u32(Qs), G.sq, lane, 32, 16 * (st >> 5), 16);
-        fence_proxy_async_smem();
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.q_ready[gi]);  // this warp's tokens: n . q (and scaled Q)
-      if (!ret) {
-        // n <- ns n + K^T u for this warp's DK/4 entries of n as warp-level MMAs: A = K^T
-        // (ldmatrix.trans of the swizzled K tile), B = u as hi + lo in columns 0 and 1 (lanes 0-7)
-        constexpr int MT = DK / 64;  // 16-entry tiles per warp
-        const int mi = lane >> 3, tq = lane & 3, k0 = (DK / 4) * (st >> 5);
-        uint32_t ub[L / 16][2];
-#pragma unroll
-        for (int ks = 0; ks < L / 16; ++ks) {
-          const float2 x = *reinterpret_cast<const float2*>(G.u + 16 * ks + 2 * tq);
-          const float2 y = *reinterpret_cast<const float2*>(G.u + 16 * ks + 2 * tq + 8);
-          uint32_t xl, yl;
-          const uint32_t xh = split_bf16x2(x.x, x.y, &xl), yh = split_bf16x2(y.x, y.y, &yl);
-          ub[ks][0] = lane < 4 ? xh : lane < 8 ? xl : 0u;
-          ub[ks][1] = lane < 4 ? yh : lane < 8 ? yl : 0u;
-        }
-        const uint32_t ks_u = smem_u32(Ks);
-        float d[MT][4] = {};
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-          for (int ks = 0; ks < L / 16; ++ks) {
-            const int srow = 16 * ks + (mi >> 1) * 8 + (lane & 7), m = k0 + 16 * mt + (mi & 1) * 8;
-            uint32_t a0, a1, a2, a3;
-            ldmatrix_x4_trans(ks_u + (m >> 6) * 8192 + srow * 128 + ((((m & 63) >> 3) ^ (srow & 7)) << 4), a0, a1, a2,
-                              a3);
-            mma_m16n8k16_bf16(d[mt], a0, a1, a2, a3, ub[ks][0], ub[ks][1]);
-          }
-        if (tq == 0) {
-          const float ns = G.scal[3];
-          __nv_bfloat16* nf = nfrag + ((c + 1) & 1) * SM::NFRAG;
-#pragma unroll
-          for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const int k = k0 + 16 * mt + (lane >> 2) + 8 * h2;
-              const float v = ns * nvec[k] + (d[mt][2 * h2] + d[mt][2 * h2 + 1]);
-              nvec[k] = v;
-              store_nfrag<DK>(nf, k, v);
-            }
-        }
-      }
-      named_bar(WG_STATE, 128);  // n updated for the next chunk; the group is done with the stage
-      if (first) {
-        mbar_arrive(&bars.empty[b]);
-        mbar_arrive(&bars.gempty[gi]);
+      // V o u of the next chunk once this chunk's update has read the buffer
+      if (c + 1 < nck) {
+        const int c1 = c + 1, b1 = c1 & 1;
+        const bool x = mbar_test_wait(&bars.gfull[c1 % NGB], (c1 / NGB) & 1),
+                   y = mbar_test_wait(&bars.full[b1], (c1 >> 1) & 1), z = mbar_test_wait(&bars.upd_done, c & 1);
+        if (!__all_sync(0xffffffffu, x && y && z))
+          warp_wait_slow3(&bars.gfull[c1 % NGB], (c1 / NGB) & 1, &bars.full[b1], (c1 >> 1) & 1, &bars.upd_done, c & 1,
+                          &abort_flag);
+        scale_v(c1);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.vw_full);
       }
     }
     // final state after the last update, back in units of e^{m}.  ro_done is committed after
     // the chunk's update, and this group has waited for each of its phases in turn (a parity
     // wait on a barrier two phases behind would return at once).
-    if (nck > 0 && group_wait(&bars.ro_done, (nck - 1) & 1, 0, first) && last_seg) {
+    if (nck > 0 && group_wait(&bars.ro_done, (nck - 1) & 1, 0, first) && last_seg && p.C_out) {
       tc_fence_after();
       const int row = acc_row<DVT>(quarter, lane);
-      if (p.C_out)
-        for (int c0 = 0; c0 < DK; c0 += 32) {
-          float r[32];
-          tmem_ld32(tm + lane_off + TM_C + c0, r);
-          tmem_wait_ld();
-          if (row >= 0) {
-            float* dst = p.C_out + ((size_t)slice * p.dv + v0 + row) * p.dk + c0;
+      for (int c0 = 0; c0 < DK; c0 += 32) {
+        float r[32];
+        tmem_ld32(tm + lane_off + TM_C + c0, r);
+        tmem_wait_ld();
+        if (row >= 0) {
+          float* dst = p.C_out + ((size_t)slice * p.dv + v0 + row) * p.dk + c0;
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
-              *reinterpret_cast<float4*>(dst + j) =
-                  make_float4(fin * r[j], fin * r[j + 1], fin * r[j + 2], fin * r[j + 3]);
-          }
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(dst + j) = make_float4(fin * r[j], fin * r[j + 1], fin * r[j + 2], fin * r[j + 3]);
         }
-      if (!ret && tile == 0 && p.n_out)
-        for (int col = st; col < DK; col += 128) p.n_out[(size_t)slice * p.dk + col] = fin * nvec[col];
+      }
     }
-  } else {
+  } else if (warp < 11) {
     // =============================================================== output group
     const int quarter = warp & 3;
     const int gt = tid - 224;  // 0..127
     const bool first = gt == 0;
     const uint32_t ps_u = sm_u + SM::OP, hs_u = sm_u + SM::OH;
     const bool use_og = p.og != nullptr && !ret;
-    // V o u of chunk c into the update operand buffer (loads batched ahead of the stores)
-    auto scale_v = [&](int c) {
-      const GateBuf G = gbuf(c % NGB);
-      const uint32_t vs_u = sm_u + (c & 1) * SM::STAGE + SM::QB + SM::KB, vw_u2 = smem_u32(Vw);
-      constexpr int NV = L * (DVT / 8) / 128;  // 16-byte chunks per thread
-      constexpr int NB = NV < 4 ? NV : 4;       // per pass; the pass loop keeps the code small
-#pragma unroll 1
-      for (int k0 = 0; k0 < NV; k0 += NB) {
-        uint4 u[NB];
-        float wr[NB];
-        int offs[NB];
-#pragma unroll
-        for (int k = 0; k < NB; ++k) {
-          const int i = (k0 + k) * 128 + gt;
-          const int row = i / (DVT / 8), ch = i % (DVT / 8);
-          offs[k] = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
-          u[k] = ld_shared_v4(vs_u + offs[k]);
-          wr[k] = G.u[row];
-        }
-#pragma unroll
-        for (int k = 0; k < NB; ++k) st_shared_v4u(vw_u2 + offs[k], scale_bf16x8(u[k], wr[k]));
-      }
-      fence_proxy_async_smem();
-    };
-    if (nck > 0) {
-      gwait(&bars.gfull[0], 0);
-      gwait(&bars.full[0], 0);
-      scale_v(0);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.vw_full);  // this warp's share of V o u is stored
-    }
     for (int c = 0; c < nck; ++c) {
       const int b = c & 1, gi = c % NGB;
       const GateBuf G = gbuf(gi);
       const int t0 = T0 + c * L;
       const int Lc = min(L, T1 - t0);
       const size_t tok0 = (size_t)bh * p.S + t0;
-      // P = S o e^{al_t + be_s} (bf16, rows t, 128-byte swizzled) and its row sums; P V of
-      // the previous chunk must be done with the P buffer
-      if (c > 0) {
-        const bool x = mbar_test_wait(&bars.mm_done, (c - 1) & 1), y = mbar_test_wait(&bars.s_full[b], (c >> 1) & 1);
-        if (!__all_sync(0xffffffffu, x && y))
-          warp_wait_slow3(&bars.mm_done, (c - 1) & 1, &bars.s_full[b], (c >> 1) & 1, nullptr, 0, &abort_flag);
-      } else {
-        gwait(&bars.s_full[b], 0);
+      // P = S o e^{al_t + be_s} (bf16, rows t, 128-byte swizzled) and its row sums, once the
+      // chunk's gate values are written (the producer loads a stage before it writes them)
+      // and P V of the previous chunk is done with the P buffer
+      {
+        const bool x = c == 0 || mbar_test_wait(&bars.mm_done, (c - 1) & 1),
+                   y = mbar_test_wait(&bars.s_full[b], (c >> 1) & 1), z = mbar_test_wait(&bars.gfull[gi], (c / NGB) & 1);
+        if (!__all_sync(0xffffffffu, x && y && z))
+          warp_wait_slow3(&bars.s_full[b], (c >> 1) & 1, &bars.gfull[gi], (c / NGB) & 1,
+                          c > 0 ? &bars.mm_done : nullptr, (c - 1) & 1, &abort_flag);
       }
       tc_fence_after();
       {
@@ -1201,18 +1130,6 @@ __global__ void __launch_bounds__(NTW, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.p_full);  // this warp's rows of P are stored
-      // V o u of the next chunk once this chunk's update has read the buffer
-      if (c + 1 < nck) {
-        const int c1 = c + 1, b1 = c1 & 1;
-        const bool x = mbar_test_wait(&bars.gfull[c1 % NGB], (c1 / NGB) & 1),
-                   y = mbar_test_wait(&bars.full[b1], (c1 >> 1) & 1), z = mbar_test_wait(&bars.upd_done, c & 1);
-        if (!__all_sync(0xffffffffu, x && y && z))
-          warp_wait_slow3(&bars.gfull[c1 % NGB], (c1 / NGB) & 1, &bars.full[b1], (c1 >> 1) & 1, &bars.upd_done, c & 1,
-                          &abort_flag);
-        scale_v(c1);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.vw_full);
-      }
       // reciprocal denominators times the output scale E_t (nq_t from the state group, the row
       // sums from all warps of this group)
       gwait(&bars.q_ready[gi], (c / NGB) & 1);
@@ -1288,6 +1205,107 @@ __global__ void __launch_bounds__(NTW, 1)
       }
     }
     if (first) bulk_wait_all();
+  } else {
+    // =============================================================== n group
+    const int nt = tid - 352, wq = nt >> 5;  // 0..127, 0..3
+    const bool first = nt == 0;
+    float fin = 1.f;
+    for (int c = 0; c < nck; ++c) {
+      const int b = c & 1, gi = c % NGB;
+      const GateBuf G = gbuf(gi);
+      uint8_t* Qs = sm + b * SM::STAGE;
+      uint8_t* Ks = Qs + SM::QB;
+      {
+        const bool x = mbar_test_wait(&bars.gfull[gi], (c / NGB) & 1), y = mbar_test_wait(&bars.full[b], (c >> 1) & 1);
+        if (!__all_sync(0xffffffffu, x && y))
+          warp_wait_slow3(&bars.gfull[gi], (c / NGB) & 1, &bars.full[b], (c >> 1) & 1, nullptr, 0, &abort_flag);
+      }
+      const bool guard = (__float_as_int(G.scal[0]) & GF_GUARD) != 0;
+      fin = G.scal[4];
+      if (!ret) {
+        // nq_t = n_st . q_t for this warp's 16 tokens as warp-level MMAs: A = the Q rows
+        // (ldmatrix from the swizzled tile), B = n as hi + lo in columns 0 and 1 (lanes 0-7)
+        const int mi = lane >> 3, arow = 16 * wq + (mi & 1) * 8 + (lane & 7);
+        const uint32_t a_row = smem_u32(Qs) + arow * 128;
+        const __nv_bfloat16* nf = nfrag + (c & 1) * SM::NFRAG + (lane & 7) * (DK / 4 + 8);
+        float d[4][4] = {};
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; kk += 2) {
+          const uint4 bv = *reinterpret_cast<const uint4*>(nf + 4 * kk);
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int col = 16 * (kk + h2) + (mi >> 1) * 8;
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4(a_row + (col >> 6) * 8192 + ((((col & 63) >> 3) ^ (arow & 7)) << 4), a0, a1, a2, a3);
+            const uint32_t b0 = lane < 8 ? (h2 ? bv.z : bv.x) : 0u, b1 = lane < 8 ? (h2 ? bv.w : bv.y) : 0u;
+            mma_m16n8k16_bf16(d[(kk + h2) & 3], a0, a1, a2, a3, b0, b1);
+          }
+        }
+        if ((lane & 3) == 0) {
+          const int t = 16 * wq + (lane >> 2);
+          G.nq[t] = ((d[0][0] + d[1][0]) + (d[2][0] + d[3][0])) + ((d[0][1] + d[1][1]) + (d[2][1] + d[3][1]));
+          G.nq[t + 8] = ((d[0][2] + d[1][2]) + (d[2][2] + d[3][2])) + ((d[0][3] + d[1][3]) + (d[2][3] + d[3][3]));
+        }
+      }
+      if (guard) {
+        // guarded chunk: Q <- e^{b_t+m_c-m_t} Q once the S MMA has read the raw Q, then the
+        // read-out with the scaled Q.  A warp's n . q read exactly the 16 rows it scales.
+        gwait(&bars.s_full[b], (c >> 1) & 1);
+        scale_rows_bf16<DK>(smem_u32(Qs), G.sq, lane, 32, 16 * wq, 16);
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.q_ready[gi]);  // this warp's tokens: n . q (and scaled Q)
+      if (!ret) {
+        // n <- ns n + K^T u for this warp's DK/4 entries of n as warp-level MMAs: A = K^T
+        // (ldmatrix.trans of the swizzled K tile), B = u as hi + lo in columns 0 and 1 (lanes 0-7)
+        constexpr int MT = DK / 64;  // 16-entry tiles per warp
+        const int mi = lane >> 3, tq = lane & 3, k0 = (DK / 4) * wq;
+        uint32_t ub[L / 16][2];
+#pragma unroll
+        for (int ks = 0; ks < L / 16; ++ks) {
+          const float2 x = *reinterpret_cast<const float2*>(G.u + 16 * ks + 2 * tq);
+          const float2 y = *reinterpret_cast<const float2*>(G.u + 16 * ks + 2 * tq + 8);
+          uint32_t xl, yl;
+          const uint32_t xh = split_bf16x2(x.x, x.y, &xl), yh = split_bf16x2(y.x, y.y, &yl);
+          ub[ks][0] = lane < 4 ? xh : lane < 8 ? xl : 0u;
+          ub[ks][1] = lane < 4 ? yh : lane < 8 ? yl : 0u;
+        }
+        const uint32_t ks_u = smem_u32(Ks);
+        float d[MT][4] = {};
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+          for (int ks = 0; ks < L / 16; ++ks) {
+            const int srow = 16 * ks + (mi >> 1) * 8 + (lane & 7), m = k0 + 16 * mt + (mi & 1) * 8;
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4_trans(ks_u + (m >> 6) * 8192 + srow * 128 + ((((m & 63) >> 3) ^ (srow & 7)) << 4), a0, a1, a2,
+                              a3);
+            mma_m16n8k16_bf16(d[mt], a0, a1, a2, a3, ub[ks][0], ub[ks][1]);
+          }
+        if (tq == 0) {
+          const float ns = G.scal[3];
+          __nv_bfloat16* nf = nfrag + ((c + 1) & 1) * SM::NFRAG;
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int k = k0 + 16 * mt + (lane >> 2) + 8 * h2;
+              const float v = ns * nvec[k] + (d[mt][2 * h2] + d[mt][2 * h2 + 1]);
+              nvec[k] = v;
+              store_nfrag<DK>(nf, k, v);
+            }
+        }
+      }
+      named_bar(WG_N, 128);  // n updated for the next chunk; the group is done with the stage
+      if (first) {
+        mbar_arrive(&bars.empty[b]);
+        mbar_arrive(&bars.gempty[gi]);
+      }
+    }
+    // final n after the last update, back in units of e^{m}
+    if (nck > 0 && last_seg && !ret && tile == 0 && p.n_out && !abort_flag)
+      for (int col = nt; col < DK; col += 128) p.n_out[(size_t)slice * p.dk + col] = fin * nvec[col];
   }
 
   if (abort_flag && tid == 0) atomicOr(p.err, 2u);
