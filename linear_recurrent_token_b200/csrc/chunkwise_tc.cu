@@ -610,7 +610,7 @@ __global__ void __launch_bounds__(NTW, 1)
       mbar_init(&bars.gempty[i], 6);  // four state warps, the n and output groups
       mbar_init(&bars.q_ready[i], 4);
     }
-    mbar_init(&bars.cb_ready, 4);
+    mbar_init(&bars.cb_ready, 8);  // the state and n groups' warps
     mbar_init(&bars.vw_full, 4);
     mbar_init(&bars.upd_done, 1);
     mbar_init(&bars.ro_done, 1);
@@ -745,7 +745,7 @@ __global__ void __launch_bounds__(NTW, 1)
   };
   // read-out H = Cb Q^T (A = the bf16 snapshot in TMEM); releases stage b with the update
   auto issue_readout = [&](uint64_t q_k, int b) {
-#pragma unroll 1
+#pragma unroll 4
     for (int k = 0; k < DK; k += 16)
       mma_bf16_ts(tm + TM_H, tm + TM_CB + k / 2, q_k + (uint64_t)(((k >> 6) * 8192 + (k & 63) * 2) >> 4), id_ro,
                   k > 0 ? 1u : 0u);
@@ -754,6 +754,34 @@ __global__ void __launch_bounds__(NTW, 1)
   };
   auto desc_k = [&](int c, int part) {  // part 0: Q, 1: K of chunk c's stage, K-major
     return smem_desc_sw128(sm_u + (c & 1) * SM::STAGE + part * SM::QB, 16, 1024);
+  };
+  // bf16 snapshot of C into TMEM for this warp's lanes, columns [c_lo, c_lo + DK/2) (the state
+  // and n groups take one half each).  When lam moves (rare) C is first rescaled in place to
+  // the snapshot's units, and after the snapshot to the units of the update.
+  auto snapshot_half = [&](const GateBuf& G, int flags, uint32_t lane_off, int c_lo) {
+    constexpr int HALF = DK / 2, SB = HALF >= 64 ? 64 : 32;
+    const float cbs = G.scal[1], csc = G.scal[2];
+    if (flags & GF_STORE_C) scale_tmem_lane<HALF>(tm + lane_off + TM_C + c_lo, cbs);
+#pragma unroll 1
+    for (int c0 = c_lo; c0 < c_lo + HALF; c0 += SB) {
+      float r[SB];
+#pragma unroll
+      for (int h2 = 0; h2 < SB / 32; ++h2)
+        tmem_ld32(tm + lane_off + TM_C + c0 + 32 * h2, *reinterpret_cast<float(*)[32]>(r + 32 * h2));
+      tmem_wait_ld();
+      float pk[16];
+#pragma unroll
+      for (int h2 = 0; h2 < SB / 32; ++h2) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) pk[j] = __uint_as_float(pack_bf16(r[32 * h2 + 2 * j], r[32 * h2 + 2 * j + 1]));
+        tmem_st16(tm + lane_off + TM_CB + c0 / 2 + 16 * h2, pk);
+      }
+    }
+    if ((flags & GF_STORE_C) && csc != cbs) {
+      tmem_wait_st();
+      scale_tmem_lane<HALF>(tm + lane_off + TM_C + c_lo, csc / cbs);
+    }
+    tmem_wait_st();
   };
 
   if (warp == 0) {
@@ -978,31 +1006,7 @@ __global__ void __launch_bounds__(NTW, 1)
       tc_fence_after();
       const int flags = __float_as_int(G.scal[0]);
       fin = G.scal[4];
-      {
-        // bf16 snapshot of C into TMEM.  When lam moves (rare) C is first rescaled in place
-        // to the snapshot's units, and after the snapshot to the units of the update.
-        const float cbs = G.scal[1], csc = G.scal[2];
-        if (flags & GF_STORE_C) scale_tmem_lane<DK>(tm + lane_off + TM_C, cbs);
-#pragma unroll 1
-        for (int c0 = 0; c0 < DK; c0 += 64) {
-          float r[64];
-          tmem_ld32(tm + lane_off + TM_C + c0, *reinterpret_cast<float(*)[32]>(r));
-          tmem_ld32(tm + lane_off + TM_C + c0 + 32, *reinterpret_cast<float(*)[32]>(r + 32));
-          tmem_wait_ld();
-          float pk[16];
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) pk[j] = __uint_as_float(pack_bf16(r[32 * h2 + 2 * j], r[32 * h2 + 2 * j + 1]));
-            tmem_st16(tm + lane_off + TM_CB + c0 / 2 + 16 * h2, pk);
-          }
-        }
-        if ((flags & GF_STORE_C) && csc != cbs) {
-          tmem_wait_st();
-          scale_tmem_lane<DK>(tm + lane_off + TM_C, csc / cbs);
-        }
-        tmem_wait_st();
-      }
+      snapshot_half(G, flags, lane_off, 0);  // columns [0, DK/2); the n group takes the rest
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -1209,18 +1213,30 @@ __global__ void __launch_bounds__(NTW, 1)
     // =============================================================== n group
     const int nt = tid - 352, wq = nt >> 5;  // 0..127, 0..3
     const bool first = nt == 0;
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     float fin = 1.f;
     for (int c = 0; c < nck; ++c) {
       const int b = c & 1, gi = c % NGB;
       const GateBuf G = gbuf(gi);
       uint8_t* Qs = sm + b * SM::STAGE;
       uint8_t* Ks = Qs + SM::QB;
+      // the upper half of the snapshot first: it is on the recurrence's path, n is not
       {
-        const bool x = mbar_test_wait(&bars.gfull[gi], (c / NGB) & 1), y = mbar_test_wait(&bars.full[b], (c >> 1) & 1);
+        const bool x = mbar_test_wait(&bars.gfull[gi], (c / NGB) & 1),
+                   y = c == 0 || mbar_test_wait(&bars.ro_done, (c - 1) & 1);
         if (!__all_sync(0xffffffffu, x && y))
-          warp_wait_slow3(&bars.gfull[gi], (c / NGB) & 1, &bars.full[b], (c >> 1) & 1, nullptr, 0, &abort_flag);
+          warp_wait_slow3(&bars.gfull[gi], (c / NGB) & 1, c > 0 ? &bars.ro_done : nullptr, (c - 1) & 1, nullptr, 0,
+                          &abort_flag);
       }
-      const bool guard = (__float_as_int(G.scal[0]) & GF_GUARD) != 0;
+      tc_fence_after();
+      const int flags = __float_as_int(G.scal[0]);
+      snapshot_half(G, flags, lane_off, DK / 2);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.cb_ready);
+      if (!__all_sync(0xffffffffu, mbar_test_wait(&bars.full[b], (c >> 1) & 1)))
+        warp_wait_slow(&bars.full[b], (c >> 1) & 1, &abort_flag);
+      const bool guard = (flags & GF_GUARD) != 0;
       fin = G.scal[4];
       if (!ret) {
         // nq_t = n_st . q_t for this warp's 16 tokens as warp-level MMAs: A = the Q rows
