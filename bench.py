@@ -37,9 +37,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 CSRC = os.path.join(ROOT, "linear_recurrent_token_b200", "csrc")
 RECORDED_TRAFFIC = {
     ("tc_walk", "large_head"): {
-        "bytes": 147_738_624 + 39_954_944,
+        "bytes": 147_769_088 + 40_159_232,
         "sources": ("chunkwise_tc.cu", "sm100.cuh", "common.cuh", "kernels.h"),
-        "sha256": "9c5759c49c9962f3823cf0d9fd1848dd4efc0804380ea8990002520eead289fe",
+        "sha256": "723b5dcbb74d2f28ab7d9033bbdaf79adfa53b55c87c89179a6abd1cafdfe927",
     },
     ("step", "decode"): {
         "bytes": 540_096_256 + 480_655_616,
