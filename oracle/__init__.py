@@ -18,6 +18,9 @@ Contents
 ``unstabilised``     numpy, fp64, the recurrence with raw exponential gates and
                      the floor 1 of the mLSTM read-out, no stabiliser at all.
 ``state_bytes``      size of a model's recurrent state (xLSTM 7B "Modelled costs").
+``sequential_backward``  numpy, fp64, gradients of ``sequential`` by reverse-mode
+                     differentiation of its steps in reverse order (backpropagation
+                     through time); pinned by central finite differences.
 
 Pins (tests/test_oracle_*.py) tie every function to something other than
 itself: closed forms, brute-force double loops, special cases and invariants.
@@ -28,6 +31,7 @@ for those two readings (their self-consistency is still tested).
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import subprocess
 
@@ -294,6 +298,124 @@ def unstabilised(q, k, v, igate, fgate, ogate=None, C0=None, n0=None, num_blocks
             ht = ht * _split_blocks(np.asarray(ogate[:, :, t], dtype=np.float64), nb)
         h[:, :, t] = ht
     return h.reshape(B, NH, S, DHV), C, n
+
+
+def sequential_backward(q, k, v, dh, igate=None, fgate=None, ogate=None, C0=None, n0=None, m0=None,
+                        dC=None, dn=None, num_blocks: int = 1, retention: bool = False):
+    """Gradients of the sequential recurrence, fp64: its steps differentiated in reverse order.
+
+    The forward step (mLSTM "Core idea", gates stabilised in log space) is
+        lf = logsigmoid(ftilde);  m_t = max(lf + m_{t-1}, itilde_t)
+        f' = exp(lf + m_{t-1} - m_t);  i' = exp(itilde_t - m_t)
+        C'_t = f' C'_{t-1} + i' v_t k_t^T;  n'_t = f' n'_{t-1} + i' k_t
+        h_t = o_t * (C'_t q_t) / max(|n'_t . q_t|, exp(-m_t))
+    (retention: f' = gamma_h, i' = 1, h_t = C'_t q_t).  h does not depend on the stabiliser:
+    with C'_t = exp(-m_t) C_t the division removes exp(-m_t) for any sequence m, so the steps
+    are differentiated with m held at its forward values and the result is the exact gradient.
+    The returned final state (C'_S, n'_S) is differentiated with m_S held fixed as well (dC, dn
+    are the gradients of a loss on exp(m_S) C'_S, n'_S written in stabilised units); the
+    initial state enters as exp(m0) C0, so dm0 = <dC0, C0> + dn0 . n0.
+
+    dh: [B,NH,S,DHV]; dC: [B,NH,nb,dv,dk]; dn: [B,NH,nb,dk] (None = 0).
+    Returns dict(dq, dk, dv, di, df, do, dC0, dn0, dm0); di, df, dn0, dm0 are None in retention
+    mode, do is None without an output gate (or in retention mode).
+    """
+    q, k, v, dh = (np.asarray(a, dtype=np.float64) for a in (q, k, v, dh))
+    B, NH, S, DHQK = q.shape
+    DHV = v.shape[-1]
+    nb = num_blocks
+    dk, dv = DHQK // nb, DHV // nb
+    use_o = ogate is not None and not retention
+    og = np.asarray(ogate, dtype=np.float64) if use_o else None
+    C0 = np.zeros((B, NH, nb, dv, dk)) if C0 is None else np.asarray(C0, dtype=np.float64)
+    n0 = np.zeros((B, NH, nb, dk)) if n0 is None else np.asarray(n0, dtype=np.float64)
+    m0 = np.zeros((B, NH)) if m0 is None else np.asarray(m0, dtype=np.float64)
+    dCS = np.zeros((B, NH, nb, dv, dk)) if dC is None else np.asarray(dC, dtype=np.float64)
+    dnS = np.zeros((B, NH, nb, dk)) if dn is None else np.asarray(dn, dtype=np.float64)
+    gam = retention_gamma(NH)
+    out = {key: np.zeros_like(x) for key, x in (("dq", q), ("dk", k), ("dv", v))}
+    out["do"] = np.zeros_like(dh) if use_o else None
+    out["dC0"] = np.zeros((B, NH, nb, dv, dk))
+    di = np.zeros((B, NH, S)) if not retention else None
+    df = np.zeros((B, NH, S)) if not retention else None
+    dn0 = np.zeros((B, NH, nb, dk)) if not retention else None
+    dm0 = np.zeros((B, NH)) if not retention else None
+    for b in range(B):
+        for hd in range(NH):
+            # gate quantities shared by the blocks of the head
+            if retention:
+                fp = np.full(S, gam[hd])
+                ip = np.ones(S)
+                mt = np.zeros(S)
+            else:
+                lf = log_sigmoid(fgate[b, hd])
+                li = np.asarray(igate[b, hd], dtype=np.float64)
+                mt = np.zeros(S)
+                mprev = m0[b, hd]
+                fp = np.zeros(S)
+                ip = np.zeros(S)
+                for t in range(S):
+                    mt[t] = max(lf[t] + mprev, li[t])
+                    fp[t] = math.exp(lf[t] + mprev - mt[t])
+                    ip[t] = math.exp(li[t] - mt[t])
+                    mprev = mt[t]
+            dlf = np.zeros(S)
+            dli = np.zeros(S)
+            for j in range(nb):
+                sk, sv = slice(j * dk, (j + 1) * dk), slice(j * dv, (j + 1) * dv)
+                Q, K, V = q[b, hd, :, sk], k[b, hd, :, sk], v[b, hd, :, sv]
+                dH = dh[b, hd, :, sv]
+                O = og[b, hd, :, sv] if use_o else np.ones((S, dv))
+                # forward, keeping every state
+                Cs = np.zeros((S + 1, dv, dk))
+                ns = np.zeros((S + 1, dk))
+                Cs[0], ns[0] = C0[b, hd, j], n0[b, hd, j]
+                num = np.zeros((S, dv))
+                dd = np.zeros(S)
+                den = np.ones(S)
+                for t in range(S):
+                    Cs[t + 1] = fp[t] * Cs[t] + ip[t] * np.outer(V[t], K[t])
+                    ns[t + 1] = fp[t] * ns[t] + ip[t] * K[t]
+                    num[t] = Cs[t + 1] @ Q[t]
+                    if not retention:
+                        dd[t] = ns[t + 1] @ Q[t]
+                        den[t] = max(abs(dd[t]), math.exp(-mt[t]))
+                # backward, t = S-1 .. 0; D, G: gradients of C'_t, n'_t accumulated so far
+                D = dCS[b, hd, j].copy()
+                G = dnS[b, hd, j].copy()
+                for t in range(S - 1, -1, -1):
+                    # h_t = o * num_t / den_t
+                    dnum = O[t] * dH[t] / den[t]
+                    if use_o:
+                        out["do"][b, hd, t, sv] = dH[t] * num[t] / den[t]
+                    ddd = 0.0
+                    if not retention and abs(dd[t]) > math.exp(-mt[t]):
+                        dden = -np.sum(O[t] * dH[t] * num[t]) / den[t] ** 2
+                        ddd = dden * math.copysign(1.0, dd[t])
+                    # num_t = C'_t q_t, d_t = n'_t . q_t
+                    D = D + np.outer(dnum, Q[t])
+                    G = G + ddd * Q[t]
+                    out["dq"][b, hd, t, sk] = Cs[t + 1].T @ dnum + ddd * ns[t + 1]
+                    # C'_t = f' C'_{t-1} + i' v k^T, n'_t = f' n'_{t-1} + i' k
+                    out["dv"][b, hd, t, sv] = ip[t] * (D @ K[t])
+                    out["dk"][b, hd, t, sk] = ip[t] * (D.T @ V[t]) + (0.0 if retention else ip[t]) * G
+                    if not retention:
+                        dip = V[t] @ D @ K[t] + G @ K[t]
+                        dfp = np.sum(D * Cs[t]) + G @ ns[t]
+                        dli[t] += ip[t] * dip  # d i'/d itilde = i'
+                        dlf[t] += fp[t] * dfp  # d f'/d lf = f'
+                    D = fp[t] * D
+                    G = fp[t] * G
+                out["dC0"][b, hd, j] = D
+                if not retention:
+                    dn0[b, hd, j] = G
+                    dm0[b, hd] += np.sum(D * C0[b, hd, j]) + G @ n0[b, hd, j]
+            if not retention:
+                di[b, hd] = dli
+                # d logsigmoid(x)/dx = sigmoid(-x)
+                df[b, hd] = dlf / (1.0 + np.exp(np.asarray(fgate[b, hd], dtype=np.float64)))
+    out.update(di=di, df=df, dn0=dn0, dm0=dm0)
+    return out
 
 
 def state_bytes(layers: int, heads: int, dqk: int, dv: int, bytes_per_value: int) -> int:
