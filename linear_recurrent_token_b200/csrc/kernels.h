@@ -62,4 +62,18 @@ struct StepArgs {
 bool step_supported_dk(int dk);
 cudaError_t launch_step(const StepArgs& a, cudaStream_t stream);
 
+// Backward (gradients of h and of the final state).  One CTA per (batch, head).
+struct BwdArgs {
+  int B, NH, S, DHQK, DHV, nb, retention, dtype;
+  int dk, dv;
+  const void *q, *k, *v, *og, *dh;
+  const float *ig, *fg, *C0, *n0, *m0, *dC, *dn;
+  float *dq, *dk_out, *dv_out, *dig, *dfg, *dog, *dC0, *dn0, *dm0;
+  float* ws;  // bwd_workspace_bytes
+};
+size_t bwd_smem_bytes(int dk, int dv);
+size_t bwd_workspace_bytes(long long BH, int S);
+bool bwd_supported(int dk, int dv);
+cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream);
+
 }  // namespace mlstm

@@ -228,6 +228,31 @@ mlstm_status_t fwd_impl(const mlstm_fwd_params_t* p, const void* q, const void* 
   return MLSTM_OK;
 }
 
+// Sizes of a backward call; MLSTM_OK when the kernel supports them.
+mlstm_status_t check_bwd(const mlstm_fwd_params_t* p, FwdShape* s) {
+  if (!p) return MLSTM_ERR_NULL;
+  if (p->dtype != MLSTM_F32 && p->dtype != MLSTM_BF16) return MLSTM_ERR_DTYPE;
+  if (p->B < 0 || p->NH < 0 || p->S < 0 || p->DHQK < 1 || p->DHV < 1 || p->num_blocks < 1)
+    return MLSTM_ERR_SHAPE;
+  if (p->DHQK % p->num_blocks || p->DHV % p->num_blocks) return MLSTM_ERR_SHAPE;
+  memset(s, 0, sizeof(*s));
+  s->B = p->B;
+  s->NH = p->NH;
+  s->S = p->S;
+  s->DHQK = p->DHQK;
+  s->DHV = p->DHV;
+  s->nb = p->num_blocks;
+  s->dk = p->DHQK / p->num_blocks;
+  s->dv = p->DHV / p->num_blocks;
+  s->retention = p->retention ? 1 : 0;
+  s->dtype = p->dtype == MLSTM_BF16 ? 1 : 0;
+  s->esize = p->dtype == MLSTM_BF16 ? 2 : 4;
+  s->BH = (long long)p->B * p->NH;
+  if (s->BH > 0x7fffffffLL || (long long)s->S * s->BH > (1LL << 40)) return MLSTM_ERR_SHAPE;
+  if (!bwd_supported(s->dk, s->dv)) return MLSTM_ERR_SHAPE;
+  return MLSTM_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -293,6 +318,98 @@ mlstm_status_t mlstm_fwd_chunkwise_timed(const mlstm_fwd_params_t* p, const void
                                          mlstm_stream_t stream, mlstm_event_t main_begin, mlstm_event_t main_end) {
   return fwd_impl(p, q, k, v, igate, fgate, ogate, C0, n0, m0, h, C_out, n_out, m_out, workspace, workspace_bytes,
                   (cudaStream_t)stream, (cudaEvent_t)main_begin, (cudaEvent_t)main_end);
+}
+
+size_t mlstm_bwd_workspace_size(const mlstm_fwd_params_t* p) {
+  FwdShape s;
+  if (check_bwd(p, &s) != MLSTM_OK) return 0;
+  return bwd_workspace_bytes(s.BH, s.S);
+}
+
+mlstm_status_t mlstm_bwd(const mlstm_fwd_params_t* p, const void* q, const void* k, const void* v,
+                         const float* igate, const float* fgate, const void* ogate, const float* C0,
+                         const float* n0, const float* m0, const void* dh, const float* dC, const float* dn,
+                         float* dq, float* dk, float* dv, float* digate, float* dfgate, float* dogate,
+                         float* dC0, float* dn0, float* dm0, void* workspace, size_t workspace_bytes,
+                         mlstm_stream_t stream) {
+  FwdShape s;
+  mlstm_status_t st = check_bwd(p, &s);
+  if (st != MLSTM_OK) return st;
+  const bool ret = s.retention != 0;
+  if (ret) {
+    igate = fgate = nullptr;
+    ogate = nullptr;
+    n0 = m0 = dn = nullptr;
+    digate = dfgate = dogate = dn0 = dm0 = nullptr;
+  }
+  if (!ogate) dogate = nullptr;
+  const size_t BH = (size_t)s.BH, S = (size_t)s.S;
+  const bool work = BH > 0 && S > 0;
+  if (work) {
+    if (!q || !k || !v || !dh || !dq || !dk || !dv) return MLSTM_ERR_NULL;
+    if (!ret && (!igate || !fgate)) return MLSTM_ERR_NULL;
+  }
+  const void* all[] = {q,  k,  v,  igate,  fgate,  ogate,  C0,  n0,  m0,  dh,  dC,
+                       dn, dq, dk, dv, digate, dfgate, dogate, dC0, dn0, dm0, workspace};
+  for (const void* ptr : all)
+    if (ptr && misaligned(ptr)) return MLSTM_ERR_ALIGN;
+  const size_t es = s.esize, nbs = BH * s.nb;
+  const size_t cbytes = nbs * s.dv * s.dk * 4, nbytes = nbs * s.dk * 4;
+  const Range ins[] = {{q, BH * S * s.DHQK * es}, {k, BH * S * s.DHQK * es}, {v, BH * S * s.DHV * es},
+                       {igate, BH * S * 4},       {fgate, BH * S * 4},       {ogate, BH * S * s.DHV * es},
+                       {C0, cbytes},              {n0, nbytes},              {m0, BH * 4},
+                       {dh, BH * S * s.DHV * es}, {dC, cbytes},              {dn, nbytes}};
+  const Range outs[] = {{dq, BH * S * s.DHQK * 4}, {dk, BH * S * s.DHQK * 4}, {dv, BH * S * s.DHV * 4},
+                        {digate, BH * S * 4},      {dfgate, BH * S * 4},      {dogate, BH * S * s.DHV * 4},
+                        {dC0, cbytes},             {dn0, nbytes},             {dm0, BH * 4}};
+  const int nout = (int)(sizeof(outs) / sizeof(outs[0]));
+  const size_t need = bwd_workspace_bytes(s.BH, s.S);
+  const Range rws{work ? workspace : nullptr, need};
+  for (int a = 0; a < nout; ++a) {
+    for (const Range& i : ins)
+      if (overlaps(outs[a], i)) return MLSTM_ERR_ALIAS;
+    for (int b = a + 1; b < nout; ++b)
+      if (overlaps(outs[a], outs[b])) return MLSTM_ERR_ALIAS;
+    if (overlaps(outs[a], rws)) return MLSTM_ERR_ALIAS;
+  }
+  if (work && (!workspace || workspace_bytes < need)) return MLSTM_ERR_WORKSPACE;
+  cudaStream_t cs = (cudaStream_t)stream;
+  if (BH == 0) return MLSTM_OK;  // with S == 0 the kernel still forms the initial-state gradients
+  BwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = s.B;
+  a.NH = s.NH;
+  a.S = s.S;
+  a.DHQK = s.DHQK;
+  a.DHV = s.DHV;
+  a.nb = s.nb;
+  a.retention = s.retention;
+  a.dtype = s.dtype;
+  a.dk = s.dk;
+  a.dv = s.dv;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.og = ogate;
+  a.dh = dh;
+  a.ig = igate;
+  a.fg = fgate;
+  a.C0 = C0;
+  a.n0 = n0;
+  a.m0 = m0;
+  a.dC = dC;
+  a.dn = dn;
+  a.dq = dq;
+  a.dk_out = dk;
+  a.dv_out = dv;
+  a.dig = digate;
+  a.dfg = dfgate;
+  a.dog = dogate;
+  a.dC0 = dC0;
+  a.dn0 = dn0;
+  a.dm0 = dm0;
+  a.ws = static_cast<float*>(workspace);
+  return launch_bwd(a, cs) == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA;
 }
 
 mlstm_status_t mlstm_step(const mlstm_step_params_t* p, const void* q, const void* k, const void* v,

@@ -66,6 +66,10 @@ def lib():
         L.mlstm_fwd_chunkwise_noalloc.restype = I
         L.mlstm_noalloc_scratch_bytes.argtypes = []
         L.mlstm_noalloc_scratch_bytes.restype = Z
+        L.mlstm_bwd_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
+        L.mlstm_bwd_workspace_size.restype = Z
+        L.mlstm_bwd.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 22 + [Z, P]
+        L.mlstm_bwd.restype = I
         L.mlstm_step.argtypes = [ctypes.POINTER(StepParams)] + [P] * 10 + [P]
         L.mlstm_step.restype = I
         L.mlstm_status_string.argtypes = [I]
@@ -164,6 +168,44 @@ def fwd_chunkwise(q, k, v, igate=None, fgate=None, ogate=None, C0=None, n0=None,
     if retention:
         return h, C_out, None, None
     return h, C_out, n_out, m_out
+
+
+def bwd_workspace_size(params: FwdParams) -> int:
+    return int(lib().mlstm_bwd_workspace_size(ctypes.byref(params)))
+
+
+def bwd(q, k, v, dh, igate=None, fgate=None, ogate=None, C0=None, n0=None, m0=None, dC=None, dn=None, *,
+        num_blocks: int = 1, retention: bool = False, workspace=None, stream=None):
+    """Backward of the recurrence (mlstm_bwd).  CUDA tensors, contiguous; the forward's inputs
+    plus dh [B,NH,S,DHV] (the input dtype) and optional dC, dn (gradients of the final state,
+    fp32).  Returns a dict of fp32 gradients dq, dk, dv, di, df (None in retention mode), do
+    (None without ogate), dC0, dn0 and dm0 (the last two None in retention mode)."""
+    B, NH, S, DHQK = q.shape
+    DHV = v.shape[-1]
+    nb = int(num_blocks)
+    p = fwd_params(B, NH, S, DHQK, DHV, 64, nb, q.dtype, retention)
+    dev = q.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {"dq": torch.empty((B, NH, S, DHQK), **f32), "dk": torch.empty((B, NH, S, DHQK), **f32),
+           "dv": torch.empty((B, NH, S, DHV), **f32),
+           "di": None if retention else torch.empty((B, NH, S), **f32),
+           "df": None if retention else torch.empty((B, NH, S), **f32),
+           "do": torch.empty((B, NH, S, DHV), **f32) if (ogate is not None and not retention) else None,
+           "dC0": torch.empty((B, NH, nb, DHV // nb, DHQK // nb), **f32),
+           "dn0": None if retention else torch.empty((B, NH, nb, DHQK // nb), **f32),
+           "dm0": None if retention else torch.empty((B, NH), **f32)}
+    ws_bytes = bwd_workspace_size(p)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().mlstm_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(igate), _ptr(fgate), _ptr(ogate),
+                         _ptr(C0), _ptr(n0), _ptr(m0), _ptr(dh), _ptr(dC), _ptr(dn),
+                         _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["di"]), _ptr(out["df"]),
+                         _ptr(out["do"]), _ptr(out["dC0"]), _ptr(out["dn0"]), _ptr(out["dm0"]),
+                         _ptr(workspace), ctypes.c_size_t(ws_len), _stream_ptr(stream))
+    if st != 0:
+        raise MlstmError(st, "mlstm_bwd")
+    return out
 
 
 def fwd_chunkwise_noalloc(q, k, v, igate=None, fgate=None, ogate=None, C0=None, n0=None, m0=None, *,

@@ -131,3 +131,36 @@ def test_step_null_and_alias():
     assert step_call(sparams(), h=F_) == 7        # h on top of C
     assert step_call(sparams(), C=A) == 7         # state on top of q
     assert step_call(sparams(), q=A + 4) == 4
+
+
+# ---------------------------------------------------------------- backward
+def bwd_call(p, q=A, k=B_, v=C_, ig=D_, fg=E_, og=None, C0=None, n0=None, m0=None, dh=F_, dC=None, dn=None,
+             dq=0x9000000, dk=0xA000000, dv=0xB000000, di=None, df=None, do=None, dC0=None, dn0=None, dm0=None,
+             ws=0xC000000, ws_bytes=1 << 40):
+    return mlstm.lib().mlstm_bwd(ctypes.byref(p), q, k, v, ig, fg, og, C0, n0, m0, dh, dC, dn, dq, dk, dv, di, df,
+                                 do, dC0, dn0, dm0, ws, ctypes.c_size_t(ws_bytes), ctypes.c_void_p(0))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=-1), 2), (dict(S=-1), 2), (dict(DHQK=0), 2), (dict(num_blocks=3), 2), (dict(dtype=7), 3),
+    (dict(DHQK=512, DHV=16), 2),              # block key width above 256
+    (dict(DHQK=256, DHV=256), 2),             # state of one block beyond shared memory
+])
+def test_bwd_rejects_bad_params(kw, status):
+    assert bwd_call(params(**kw)) == status
+
+
+def test_bwd_null_align_alias_workspace():
+    p = params()
+    assert bwd_call(p, dh=None) == 1
+    assert bwd_call(p, fg=None) == 1
+    assert bwd_call(p, dq=None) == 1
+    assert bwd_call(params(retention=True), ig=None, fg=None) != 1  # gates ignored in retention
+    assert bwd_call(p, q=A + 8) == 4
+    assert bwd_call(p, dq=A) == 7                  # dq on top of q
+    assert bwd_call(p, dk=0x9000000) == 7          # dk on top of dq
+    assert bwd_call(p, ws=0x9000000) == 7          # workspace on top of dq
+    assert bwd_call(p, ws_bytes=16) == 5
+    assert bwd_call(p, ws=None) == 5
+    assert mlstm.bwd_workspace_size(p) == 2 * 2 * 8 * 64 * 4
+    assert mlstm.bwd_workspace_size(params(DHQK=512)) == 0
