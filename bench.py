@@ -39,12 +39,12 @@ RECORDED_TRAFFIC = {
     ("tc_walk", "large_head"): {
         "bytes": 147_769_088 + 40_159_232,
         "sources": ("chunkwise_tc.cu", "sm100.cuh", "common.cuh", "kernels.h"),
-        "sha256": "723b5dcbb74d2f28ab7d9033bbdaf79adfa53b55c87c89179a6abd1cafdfe927",
+        "sha256": "b0ef1a9b6e7b1aac4b20a8e7990724c34500f309eea0a7ddf3b63575a6ce5846",
     },
     ("step", "decode"): {
         "bytes": 540_096_256 + 480_655_616,
         "sources": ("step.cu", "common.cuh", "kernels.h"),
-        "sha256": "5bc4a28dcea130bc462276a009b0ebffab3b6b8680c42dcacd5b1d3fb15e6dc5",
+        "sha256": "45215b51f32ce50a67dcd31064196f32c13182bf3f4189cf139d1f7115cd65f1",
     },
 }
 
@@ -95,6 +95,18 @@ def decode_step_bytes(B, NH, DHQK, DHV, esize, nb=1):
 def decode_step_flops(B, NH, DHQK, DHV, nb=1):
     """Update (f'C + i' v k^T: 3 flops/element) plus read-out (2 per element) plus n."""
     return B * NH * (5 * DHV * DHQK // nb + 6 * DHQK)
+
+
+def backward_flops(B, NH, S, dk, dv, nb=1):
+    """Algorithmic flops of the backward as the sequential reverse-mode evaluation does them:
+    per token and block six dk x dv products or rank-1 updates (state update, read-out, dq,
+    update of dL/dC, dv, dk), 2 flops per element; vector terms omitted."""
+    return B * NH * S * nb * 12 * dk * dv
+
+
+def fp32_simt_peak_tflops(sm_mhz):
+    """B200 fp32 FMA throughput from unit counts: 148 SMs x 128 fp32 lanes x 2 flops x clock."""
+    return 148 * 128 * 2 * (sm_mhz or 1965.0) * 1e6 / 1e12
 
 
 def load_peaks():
@@ -455,6 +467,76 @@ def run_decode(w, steps, warmup, clocks):
     return dict(step_ms=step_ms, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h)
 
 
+def oracle_backward_sample(w, tokens: int, heads: int):
+    """The fp64 backward oracle on the first `tokens` positions of `heads` (batch, head)
+    sequences of the workload; returns (seconds, tokens processed)."""
+    import oracle
+    from linear_recurrent_token_b200 import inputs
+    inp = inputs.forward_inputs(w, S=tokens)
+    rng = np.random.default_rng(3000)
+    sel = lambda x: None if x is None else x[:1, :heads]
+    dh = rng.standard_normal((1, heads, tokens, w.DHV))
+    t0 = time.perf_counter()
+    oracle.sequential_backward(sel(inp["q"]), sel(inp["k"]), sel(inp["v"]), dh, sel(inp.get("igate")),
+                               sel(inp.get("fgate")), num_blocks=w.num_blocks, retention=w.retention)
+    return time.perf_counter() - t0, tokens * heads
+
+
+def run_backward(w, steps, warmup, flush_bytes, clocks):
+    """The backward (mlstm_bwd) on the workload's shapes, inputs resident, L2 flushed
+    between steps; returns per-step milliseconds."""
+    import torch
+
+    from linear_recurrent_token_b200 import inputs, mlstm
+    td = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    inp = inputs.forward_inputs(w)
+    rng = np.random.default_rng(3001)
+    d = lambda x, dt=torch.float32: None if x is None else torch.from_numpy(np.ascontiguousarray(x)).to("cuda", dt)
+    q, k, v = d(inp["q"], td), d(inp["k"], td), d(inp["v"], td)
+    ig, fg = d(inp.get("igate")), d(inp.get("fgate"))
+    dh = d(rng.standard_normal((w.B, w.NH, w.S, w.DHV)), td)
+    p = mlstm.fwd_params(w.B, w.NH, w.S, w.DHQK, w.DHV, w.chunk, w.num_blocks, td, w.retention)
+    ws = torch.empty(max(mlstm.bwd_workspace_size(p), 16), dtype=torch.uint8, device="cuda")
+    flush = torch.empty(flush_bytes // 4, dtype=torch.float32, device="cuda")
+    for _ in range(warmup):
+        mlstm.bwd(q, k, v, dh, ig, fg, num_blocks=w.num_blocks, retention=w.retention, workspace=ws)
+    torch.cuda.synchronize()
+    ms = []
+    clocks.mark(True)
+    for _ in range(steps):
+        flush.fill_(1.0)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        mlstm.bwd(q, k, v, dh, ig, fg, num_blocks=w.num_blocks, retention=w.retention, workspace=ws)
+        b.record()
+        torch.cuda.synchronize()
+        ms.append(a.elapsed_time(b))
+    clocks.mark(False)
+    return ms
+
+
+def backward_line(w, ms, sm_mhz, cpu: bool):
+    step_ms = statistics.median(ms)
+    flops = backward_flops(w.B, w.NH, w.S, w.dk, w.dv, w.num_blocks)
+    peak = fp32_simt_peak_tflops(sm_mhz)
+    tf = flops / (step_ms * 1e-3) / 1e12
+    out = {"workload": w.describe(), "value": w.B * w.S / (step_ms * 1e-3), "unit": "tokens/s",
+           "ms_per_step": step_ms, "steps": len(ms), "dtype": "f32 (inputs " + w.dtype + ")",
+           "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                        "traffic": None, "kernel": "bwd_kernel (SIMT, one CTA per head)",
+                        "flops_per_launch": flops,
+                        "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x median SM clock"}}
+    if cpu:
+        tokens = min(w.S, 64)
+        heads = min(w.NH, 2)
+        secs, done = oracle_backward_sample(w, tokens, heads)
+        out["cpu_baseline"] = {"value": done / secs, "unit": "tokens/s (one sequence)", "cores": 1,
+                               "kind": "oracle",
+                               "sample": f"first {tokens} positions of {heads} (batch, head) sequences of "
+                                         f"{w.describe()}, fp64 reverse-mode sequential recurrence"}
+    return out
+
+
 # ------------------------------------------------------------------ main
 def main():
     ap = argparse.ArgumentParser()
@@ -464,7 +546,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=3, help="chunkwise workload index (default 3)")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--legs", choices=["both", "chunkwise", "decode"], default="both",
+    ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--legs", choices=["both", "chunkwise", "decode", "backward"], default="both",
                     help="run only one leg (for profiling); the default runs both")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -508,6 +591,13 @@ def main():
     try:
         dist_barrier(world)
         torch.cuda.synchronize()
+        if args.legs == "backward":
+            for idx in (1, 2):
+                wb = inputs.WORKLOADS[idx]
+                ms = run_backward(wb, args.steps, args.warmup, 256 << 20, clocks)
+                if rank == 0:
+                    print(json.dumps({"leg": "backward", "workload": wb.describe(), "ms_per_step": statistics.median(ms)}))
+            return
         if args.legs == "decode":
             dec = run_decode(wd, args.steps, args.warmup, clocks)
             ms = dist_max(statistics.mean(dec["step_ms"]), world)
@@ -535,6 +625,12 @@ def main():
         if not args.no_decode:
             dist_barrier(world)
             dec = run_decode(wd, args.steps * 5, args.warmup, clocks)
+            dist_barrier(world)
+        bwd = []
+        if not args.no_backward and args.legs == "both":
+            for idx in (1, 2):
+                wb = inputs.WORKLOADS[idx]
+                bwd.append((wb, run_backward(wb, max(3, args.steps // 4), args.warmup, 256 << 20, clocks)))
             dist_barrier(world)
     finally:
         clocks.stop()
@@ -574,6 +670,11 @@ def main():
                     "h2d_bytes_per_step": dec["h2d"], "d2h_bytes_per_step": dec["d2h"]},
         }
         line["gpu_launches"] += len(dec["step_ms"])
+    if bwd:
+        sm_mhz = line["clocks"].get("sm_mhz")
+        line["backward"] = [backward_line(wb, ms, sm_mhz, rank == 0 and world == 1 and not args.no_cpu_baseline)
+                            for wb, ms in bwd]
+        line["gpu_launches"] += sum(len(ms) for _, ms in bwd)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(w)
         line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}

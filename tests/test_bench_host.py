@@ -71,3 +71,10 @@ def test_recorded_traffic_is_null_once_sources_change(monkeypatch):
     monkeypatch.setitem(bench.RECORDED_TRAFFIC, key, dict(rec, sha256=bench.sources_sha256(rec["sources"])))
     assert bench.recorded_traffic(*key) == rec["bytes"]
     assert bench.recorded_traffic("tc_walk", "retention") is None
+
+
+def test_backward_flop_count_and_simt_peak():
+    # six dk x dv products / rank-1 updates per token and block, 2 flops per element
+    assert bench.backward_flops(1, 1, 1, 64, 32, 1) == 6 * 2 * 64 * 32
+    assert bench.backward_flops(4, 4, 512, 32, 32, 2) == 4 * 4 * 512 * 2 * 12 * 32 * 32
+    assert abs(bench.fp32_simt_peak_tflops(1965.0) - 148 * 128 * 2 * 1.965e9 / 1e12) < 1e-9
