@@ -49,6 +49,46 @@ __device__ __forceinline__ float block_sum(float x, float* red) {
   return s;
 }
 
+// Products over the block state St [dv][dk + 1] with all threads.  Thread t owns key column
+// c = t % dk and the value rows r = t / dk (mod NTB / dk) (column map), or value row
+// r = t % dv and the key columns c = t / dv (mod NTB / dv) (row map); partial sums meet in
+// `part` [NTB] and one thread per output adds them.  Each call ends with a barrier.
+//   col_prod: out[c] = sum_r St[r][c] x[r]      row_prod: out[r] = sum_c St[r][c] x[c]
+__device__ __forceinline__ void col_prod(const float* St, int ld, int dk, int dv, const float* x, float* part,
+                                         float* out) {
+  const int t = threadIdx.x, rg = NTB / dk;
+  if (t < rg * dk) {
+    const int c = t % dk;
+    float s = 0.f;
+    for (int r = t / dk; r < dv; r += rg) s += St[r * ld + c] * x[r];
+    part[t] = s;
+  }
+  __syncthreads();
+  if (t < dk) {
+    float s = 0.f;
+    for (int j = 0; j < rg; ++j) s += part[j * dk + t];
+    out[t] = s;
+  }
+  __syncthreads();
+}
+__device__ __forceinline__ void row_prod(const float* St, int ld, int dk, int dv, const float* x, float* part,
+                                         float* out) {
+  const int t = threadIdx.x, sl = NTB / dv;
+  if (t < sl * dv) {
+    const int r = t % dv;
+    float s = 0.f;
+    for (int c = t / dv; c < dk; c += sl) s += St[r * ld + c] * x[c];
+    part[t] = s;
+  }
+  __syncthreads();
+  if (t < dv) {
+    float s = 0.f;
+    for (int j = 0; j < sl; ++j) s += part[j * dv + t];
+    out[t] = s;
+  }
+  __syncthreads();
+}
+
 template <typename T>
 __global__ void __launch_bounds__(NTB, 1) bwd_kernel(BwdArgs a) {
   extern __shared__ float smf[];
@@ -62,10 +102,15 @@ __global__ void __launch_bounds__(NTB, 1) bwd_kernel(BwdArgs a) {
   float* os = dhs + dv;          // [dv]
   float* dnum = os + dv;         // [dv]
   float* red = dnum + dv;        // [NTB / 32]
+  float* part = red + NTB / 32;  // [NTB] partial sums of the state products
+  float* rowv = part + NTB;      // [dv] row products
+  float* colv = rowv + dv;       // [dk] column products
   __shared__ float sc[4];
 
   const int tid = threadIdx.x;
   const int bh = blockIdx.x, head = bh % a.NH;
+  // column map of the state loops: column tid % dk, rows tid / dk + j * cstep
+  const int cstep = NTB / dk, ccol = tid % dk, crow0 = tid / dk;
   const bool ret = a.retention != 0;
   const T* q = static_cast<const T*>(a.q);
   const T* k = static_cast<const T*>(a.k);
@@ -126,21 +171,40 @@ __global__ void __launch_bounds__(NTB, 1) bwd_kernel(BwdArgs a) {
     }
     for (int c = tid; c < dk; c += NTB) nv[c] = (!ret && a.n0) ? a.n0[slice * dk + c] : 0.f;
     __syncthreads();
-    for (int t = 0; t < S; ++t) {
-      const float fp = wf[t], ip = wi[t];
-      for (int c = tid; c < dk; c += NTB) {
-        qs[c] = io<T>::load(q, qoff + (size_t)t * a.DHQK + c);
-        ks[c] = io<T>::load(k, qoff + (size_t)t * a.DHQK + c);
+    // the next token's inputs are loaded into registers while this token is worked on
+    // (dk, dv <= NTB: one element of each vector per thread)
+    float pq = 0.f, pk = 0.f, pv = 0.f, pdh = 0.f, po = 1.f, pfp = 0.f, pip = 0.f, pmt = 0.f;
+    auto fetch1 = [&](int t) {
+      if (tid < dk) {
+        pq = io<T>::load(q, qoff + (size_t)t * a.DHQK + tid);
+        pk = io<T>::load(k, qoff + (size_t)t * a.DHQK + tid);
       }
-      for (int r = tid; r < dv; r += NTB) {
-        vs[r] = io<T>::load(v, voff + (size_t)t * a.DHV + r);
-        dhs[r] = io<T>::load(dh, voff + (size_t)t * a.DHV + r);
-        os[r] = og ? io<T>::load(og, voff + (size_t)t * a.DHV + r) : 1.f;
+      if (tid < dv) {
+        pv = io<T>::load(v, voff + (size_t)t * a.DHV + tid);
+        pdh = io<T>::load(dh, voff + (size_t)t * a.DHV + tid);
+        po = og ? io<T>::load(og, voff + (size_t)t * a.DHV + tid) : 1.f;
+      }
+      pfp = wf[t];
+      pip = wi[t];
+      pmt = wm[t];
+    };
+    if (S > 0) fetch1(0);
+    for (int t = 0; t < S; ++t) {
+      const float fp = pfp, ip = pip, mt = pmt;
+      if (tid < dk) {
+        qs[tid] = pq;
+        ks[tid] = pk;
+      }
+      if (tid < dv) {
+        vs[tid] = pv;
+        dhs[tid] = pdh;
+        os[tid] = po;
       }
       __syncthreads();
-      for (int e = tid; e < dv * dk; e += NTB) {
-        const int r = e / dk, c = e % dk;
-        St[r * ld + c] = fp * St[r * ld + c] + ip * vs[r] * ks[c];
+      if (t + 1 < S) fetch1(t + 1);
+      if (tid < cstep * dk) {
+        const float kc = ip * ks[ccol];
+        for (int r = crow0; r < dv; r += cstep) St[r * ld + ccol] = fp * St[r * ld + ccol] + vs[r] * kc;
       }
       if (!ret)
         for (int c = tid; c < dk; c += NTB) nv[c] = fp * nv[c] + ip * ks[c];
@@ -150,25 +214,21 @@ __global__ void __launch_bounds__(NTB, 1) bwd_kernel(BwdArgs a) {
       if (!ret)
         for (int c = tid; c < dk; c += NTB) dpart += nv[c] * qs[c];
       const float d = ret ? 0.f : block_sum(dpart, red);
-      const float den = ret ? 1.f : fmaxf(fabsf(d), expf(-wm[t]));
+      const float den = ret ? 1.f : fmaxf(fabsf(d), expf(-mt));
       // read-out rows: num_r = C'_t[r,:] . q_t
+      row_prod(St, ld, dk, dv, qs, part, rowv);
       float ppart = 0.f;
       for (int r = tid; r < dv; r += NTB) {
-        float num = 0.f;
-        for (int c = 0; c < dk; ++c) num += St[r * ld + c] * qs[c];
-        const float hn = num / den;
+        const float hn = rowv[r] / den;
         dnum[r] = os[r] * dhs[r] / den;
         ppart += os[r] * dhs[r] * hn;
         if (a.dog) a.dog[voff + (size_t)t * a.DHV + r] = dhs[r] * hn;
       }
       const float P = ret ? 0.f : block_sum(ppart, red);  // also orders the dnum stores
       if (ret) __syncthreads();
-      const float dd = (!ret && fabsf(d) > expf(-wm[t])) ? -P / den * copysignf(1.f, d) : 0.f;
-      for (int c = tid; c < dk; c += NTB) {
-        float g = 0.f;
-        for (int r = 0; r < dv; ++r) g += St[r * ld + c] * dnum[r];
-        a.dq[qoff + (size_t)t * a.DHQK + c] = g + dd * nv[c];
-      }
+      const float dd = (!ret && fabsf(d) > expf(-mt)) ? -P / den * copysignf(1.f, d) : 0.f;
+      col_prod(St, ld, dk, dv, dnum, part, colv);
+      for (int c = tid; c < dk; c += NTB) a.dq[qoff + (size_t)t * a.DHQK + c] = colv[c] + dd * nv[c];
       if (tid == 0) {
         wden[t] = den;
         wd[t] = d;
@@ -195,38 +255,43 @@ __global__ void __launch_bounds__(NTB, 1) bwd_kernel(BwdArgs a) {
     }
     for (int c = tid; c < dk; c += NTB) nv[c] = (!ret && a.dn) ? a.dn[slice * dk + c] : 0.f;
     __syncthreads();
+    float pden = 1.f, pdd = 0.f;
+    auto fetch2 = [&](int t) {
+      fetch1(t);
+      pden = wden[t];
+      pdd = wdd[t];
+    };
+    if (S > 0) fetch2(S - 1);
     for (int t = S - 1; t >= 0; --t) {
-      const float fp = wf[t], ip = wi[t], den = wden[t], dd = wdd[t];
-      for (int c = tid; c < dk; c += NTB) {
-        qs[c] = io<T>::load(q, qoff + (size_t)t * a.DHQK + c);
-        ks[c] = io<T>::load(k, qoff + (size_t)t * a.DHQK + c);
+      const float fp = pfp, ip = pip, den = pden, dd = pdd;
+      if (tid < dk) {
+        qs[tid] = pq;
+        ks[tid] = pk;
       }
-      for (int r = tid; r < dv; r += NTB) {
-        vs[r] = io<T>::load(v, voff + (size_t)t * a.DHV + r);
-        const float o = og ? io<T>::load(og, voff + (size_t)t * a.DHV + r) : 1.f;
-        dnum[r] = o * io<T>::load(dh, voff + (size_t)t * a.DHV + r) / den;
+      if (tid < dv) {
+        vs[tid] = pv;
+        dnum[tid] = po * pdh / den;
       }
       __syncthreads();
-      for (int e = tid; e < dv * dk; e += NTB) {
-        const int r = e / dk, c = e % dk;
-        St[r * ld + c] += dnum[r] * qs[c];
+      if (t > 0) fetch2(t - 1);
+      if (tid < cstep * dk) {
+        const float qc = qs[ccol];
+        for (int r = crow0; r < dv; r += cstep) St[r * ld + ccol] += dnum[r] * qc;
       }
       if (!ret)
         for (int c = tid; c < dk; c += NTB) nv[c] += dd * qs[c];
       __syncthreads();
+      row_prod(St, ld, dk, dv, ks, part, rowv);
+      col_prod(St, ld, dk, dv, vs, part, colv);
       float bpart = 0.f;
       for (int r = tid; r < dv; r += NTB) {
-        float x = 0.f;
-        for (int c = 0; c < dk; ++c) x += St[r * ld + c] * ks[c];
-        const float g = ip * x;
+        const float g = ip * rowv[r];
         a.dv_out[voff + (size_t)t * a.DHV + r] = g;
         bpart += vs[r] * g;
       }
       for (int c = tid; c < dk; c += NTB) {
-        float x = 0.f;
-        for (int r = 0; r < dv; ++r) x += St[r * ld + c] * vs[r];
         const float gn = ret ? 0.f : ip * nv[c];
-        a.dk_out[qoff + (size_t)t * a.DHQK + c] = ip * x + gn;
+        a.dk_out[qoff + (size_t)t * a.DHQK + c] = ip * colv[c] + gn;
         bpart += gn * ks[c];
       }
       if (!ret) {
@@ -237,10 +302,8 @@ __global__ void __launch_bounds__(NTB, 1) bwd_kernel(BwdArgs a) {
         }
       }
       __syncthreads();
-      for (int e = tid; e < dv * dk; e += NTB) {
-        const int r = e / dk, c = e % dk;
-        St[r * ld + c] *= fp;
-      }
+      if (tid < cstep * dk)
+        for (int r = crow0; r < dv; r += cstep) St[r * ld + ccol] *= fp;
       if (!ret)
         for (int c = tid; c < dk; c += NTB) nv[c] *= fp;
       __syncthreads();
@@ -279,7 +342,7 @@ __global__ void __launch_bounds__(NTB, 1) bwd_kernel(BwdArgs a) {
 }  // namespace
 
 size_t bwd_smem_bytes(int dk, int dv) {
-  return ((size_t)dv * (dk + 1) + 3 * (size_t)dk + 4 * (size_t)dv + NTB / 32) * sizeof(float);
+  return ((size_t)dv * (dk + 1) + 4 * (size_t)dk + 5 * (size_t)dv + NTB / 32 + NTB) * sizeof(float);
 }
 
 size_t bwd_workspace_bytes(long long BH, int S) { return (size_t)BH * 8 * (size_t)S * sizeof(float); }
