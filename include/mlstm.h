@@ -177,6 +177,68 @@ mlstm_status_t mlstm_fwd_chunkwise_noalloc(const mlstm_fwd_params_t* p,
 size_t mlstm_noalloc_scratch_bytes(void);
 
 /*
+ * The same prefill over the reversed sequence: token S-1 is read first and token 0 last;
+ * h[t] is written at the token's own position t, and the final state is the state after
+ * token 0.  This is the backward direction of a bidirectional encoder (DeepChrInteract-v2
+ * "mLSTM Model": a bidirectional wrapper so that the encoder sees context from both sides);
+ * a caller combines it with mlstm_fwd_chunkwise as it likes.  Arguments as for
+ * mlstm_fwd_chunkwise; the workspace (mlstm_fwd_chunkwise_reversed_workspace_size bytes)
+ * also holds reversed copies of the inputs and of h, and must not overlap any argument.
+ */
+size_t mlstm_fwd_chunkwise_reversed_workspace_size(const mlstm_fwd_params_t* p);
+mlstm_status_t mlstm_fwd_chunkwise_reversed(const mlstm_fwd_params_t* p,
+                                            const void* q, const void* k, const void* v,
+                                            const float* igate, const float* fgate, const void* ogate,
+                                            const float* C0, const float* n0, const float* m0,
+                                            void* h, float* C_out, float* n_out, float* m_out,
+                                            void* workspace, size_t workspace_bytes,
+                                            mlstm_stream_t stream);
+
+/*
+ * Backward of the recurrence: gradients of a loss with respect to the inputs of
+ * mlstm_fwd_chunkwise, given its gradient dh with respect to h (and optionally dC, dn
+ * with respect to the final state).  Reverse-mode differentiation of the sequential
+ * steps (RetNet "Triple Paradigm": the parallel / chunkwise form is the training mode;
+ * this computes its gradients).  h does not depend on the stabiliser m, so the steps
+ * are differentiated with m held fixed, which is exact; the final state (C'_S, n'_S) is
+ * differentiated in stabilised units with m_S fixed (dC = exp(m_S) dL/dC_S for a loss on
+ * the raw state C_S = exp(m_S) C'_S), and the initial state enters as exp(m0) C0, so
+ * dm0 = <dC0, C0> + dn0 . n0.
+ *
+ *   p                       sizes as for the forward (chunk is ignored).  Supported: block
+ *                           key and value widths DHQK/nb, DHV/nb <= 256 with
+ *                           (DHV/nb) x (DHQK/nb + 1) fp32 of state in one CTA's shared memory
+ *                           (about 48 K values), else MLSTM_ERR_SHAPE.
+ *   q, k, v, igate, fgate,  the forward's inputs, same layouts and rules (ogate, C0, n0,
+ *   ogate, C0, n0, m0       m0 may be NULL)
+ *   dh      [B,NH,S,DHV]   dtype   gradient of h; required (if S > 0)
+ *   dC      [B,NH,nb,DHV/nb,DHQK/nb] fp32  gradient of C_out (stabilised units); NULL = 0
+ *   dn      [B,NH,nb,DHQK/nb]        fp32  gradient of n_out; NULL = 0; ignored in retention
+ *   dq, dk  [B,NH,S,DHQK]  fp32    required (if S > 0)
+ *   dv      [B,NH,S,DHV]   fp32    required (if S > 0)
+ *   digate, dfgate [B,NH,S] fp32   gradients of the gate pre-activations; NULL = not
+ *                                  written; not written in retention mode
+ *   dogate  [B,NH,S,DHV]   fp32    gradient of the output gate; written only if ogate
+ *                                  is given (and not in retention mode)
+ *   dC0 [B,NH,nb,DHV/nb,DHQK/nb], dn0 [B,NH,nb,DHQK/nb], dm0 [B,NH]  fp32  gradients of the
+ *                                  initial state; NULL = not written; dn0 and dm0 not in
+ *                                  retention mode
+ *   workspace, workspace_bytes     at least mlstm_bwd_workspace_size(p) bytes, 16-byte
+ *                                  aligned; contents need not be initialised
+ * Outputs must not overlap the inputs, each other or the workspace (MLSTM_ERR_ALIAS).
+ * Other conventions as for the forward.
+ */
+size_t mlstm_bwd_workspace_size(const mlstm_fwd_params_t* p);
+mlstm_status_t mlstm_bwd(const mlstm_fwd_params_t* p,
+                         const void* q, const void* k, const void* v,
+                         const float* igate, const float* fgate, const void* ogate,
+                         const float* C0, const float* n0, const float* m0,
+                         const void* dh, const float* dC, const float* dn,
+                         float* dq, float* dk, float* dv, float* digate, float* dfgate, float* dogate,
+                         float* dC0, float* dn0, float* dm0,
+                         void* workspace, size_t workspace_bytes, mlstm_stream_t stream);
+
+/*
  * One recurrent decode step for every sequence of the batch, state updated in
  * place (RetNet recurrent_retention_step: O(1) per token; burn-gdn2 Gdn2Mode
  * FusedRecurrent: state [B,H,K,V] carried across tokens and updated in place).

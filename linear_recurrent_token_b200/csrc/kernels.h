@@ -62,6 +62,10 @@ struct StepArgs {
 bool step_supported_dk(int dk);
 cudaError_t launch_step(const StepArgs& a, cudaStream_t stream);
 
+// dst[bh][S-1-t] = src[bh][t] for [BH, S, row_bytes] tensors (row_bytes a multiple of 2).
+cudaError_t launch_reverse_rows(const void* src, void* dst, long long BH, long long S, long long row_bytes,
+                                cudaStream_t stream);
+
 // Backward (gradients of h and of the final state).  One CTA per (batch, head).
 struct BwdArgs {
   int B, NH, S, DHQK, DHV, nb, retention, dtype;

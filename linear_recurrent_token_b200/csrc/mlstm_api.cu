@@ -105,7 +105,7 @@ mlstm_status_t fwd_impl(const mlstm_fwd_params_t* p, const void* q, const void* 
                         const float* igate, const float* fgate, const void* ogate, const float* C0,
                         const float* n0, const float* m0, void* h, float* C_out, float* n_out, float* m_out,
                         void* workspace, size_t workspace_bytes, cudaStream_t stream, cudaEvent_t ev0,
-                        cudaEvent_t ev1) {
+                        cudaEvent_t ev1, bool launch = true) {
   FwdShape s;
   mlstm_status_t st = check_fwd(p, &s);
   if (st != MLSTM_OK) return st;
@@ -154,7 +154,7 @@ mlstm_status_t fwd_impl(const mlstm_fwd_params_t* p, const void* q, const void* 
       if (overlaps(so, si) && !exact) return MLSTM_ERR_ALIAS;
     }
   }
-  if (s.BH == 0) return MLSTM_OK;
+  if (s.BH == 0 || !launch) return MLSTM_OK;
 
   cudaError_t e = cudaSuccess;
   if (s.S == 0) {  // nothing to read: the final state is the initial state
@@ -318,6 +318,95 @@ mlstm_status_t mlstm_fwd_chunkwise_timed(const mlstm_fwd_params_t* p, const void
                                          mlstm_stream_t stream, mlstm_event_t main_begin, mlstm_event_t main_end) {
   return fwd_impl(p, q, k, v, igate, fgate, ogate, C0, n0, m0, h, C_out, n_out, m_out, workspace, workspace_bytes,
                   (cudaStream_t)stream, (cudaEvent_t)main_begin, (cudaEvent_t)main_end);
+}
+
+// Workspace of the reversed-sequence pass: the forward's, then reversed copies of the
+// inputs and of h.
+struct RevLayout {
+  size_t fwd, q, k, v, o, ig, fg, h, total;
+};
+RevLayout rev_layout(const FwdShape& s) {
+  RevLayout r = {};
+  const size_t tok = (size_t)s.BH * s.S;
+  const size_t bq = tok * s.DHQK * s.esize, bv = tok * s.DHV * s.esize, bg = tok * sizeof(float);
+  r.fwd = 0;  // the forward's own workspace comes first
+  size_t off = align_up(fwd_layout(s).total);
+  r.q = off;
+  off = align_up(off + bq);
+  r.k = off;
+  off = align_up(off + bq);
+  r.v = off;
+  off = align_up(off + bv);
+  if (!s.retention) {
+    r.o = off;
+    off = align_up(off + bv);
+    r.ig = off;
+    off = align_up(off + bg);
+    r.fg = off;
+    off = align_up(off + bg);
+  }
+  r.h = off;
+  off = align_up(off + bv);
+  r.total = off;
+  return r;
+}
+
+size_t mlstm_fwd_chunkwise_reversed_workspace_size(const mlstm_fwd_params_t* p) {
+  FwdShape s;
+  if (check_fwd(p, &s) != MLSTM_OK) return 0;
+  return s.BH == 0 || s.S == 0 ? fwd_layout(s).total : rev_layout(s).total;
+}
+
+mlstm_status_t mlstm_fwd_chunkwise_reversed(const mlstm_fwd_params_t* p, const void* q, const void* k,
+                                            const void* v, const float* igate, const float* fgate,
+                                            const void* ogate, const float* C0, const float* n0, const float* m0,
+                                            void* h, float* C_out, float* n_out, float* m_out, void* workspace,
+                                            size_t workspace_bytes, mlstm_stream_t stream) {
+  FwdShape s;
+  mlstm_status_t st = check_fwd(p, &s);
+  if (st != MLSTM_OK) return st;
+  cudaStream_t cs = (cudaStream_t)stream;
+  if (s.BH == 0 || s.S == 0)  // nothing to reverse
+    return fwd_impl(p, q, k, v, igate, fgate, ogate, C0, n0, m0, h, C_out, n_out, m_out, workspace,
+                    workspace_bytes, cs, nullptr, nullptr);
+  const RevLayout r = rev_layout(s);
+  const size_t fwd_bytes = fwd_layout(s).total;
+  // the caller's buffers, validated as for the forward (with the forward's part of the workspace)
+  st = fwd_impl(p, q, k, v, igate, fgate, ogate, C0, n0, m0, h, C_out, n_out, m_out, workspace,
+                workspace_bytes, cs, nullptr, nullptr, false);
+  if (st != MLSTM_OK) return st;
+  if (!workspace || workspace_bytes < r.total) return MLSTM_ERR_WORKSPACE;
+  const bool ret = s.retention != 0;
+  if (ret) {
+    igate = fgate = nullptr;
+    ogate = nullptr;
+  }
+  const size_t tok = (size_t)s.BH * s.S;
+  const size_t bq = tok * s.DHQK * s.esize, bv = tok * s.DHV * s.esize, bg = tok * sizeof(float);
+  const size_t bC = (size_t)s.BH * s.nb * s.dv * s.dk * sizeof(float);
+  const size_t bn = (size_t)s.BH * s.nb * s.dk * sizeof(float), bm = (size_t)s.BH * sizeof(float);
+  const Range wsr{workspace, r.total};
+  const Range user[] = {{q, bq},   {k, bq},    {v, bv},     {igate, bg}, {fgate, bg}, {ogate, bv}, {C0, bC},
+                        {n0, bn},  {m0, bm},   {h, bv},     {C_out, bC}, {n_out, bn}, {m_out, bm}};
+  for (const Range& u : user)
+    if (overlaps(wsr, u)) return MLSTM_ERR_ALIAS;
+  char* w = static_cast<char*>(workspace);
+  void *qr = w + r.q, *kr = w + r.k, *vr = w + r.v, *hr = w + r.h;
+  void* orv = (!ret && ogate) ? static_cast<void*>(w + r.o) : nullptr;
+  float* igr = ret ? nullptr : reinterpret_cast<float*>(w + r.ig);
+  float* fgr = ret ? nullptr : reinterpret_cast<float*>(w + r.fg);
+  const long long BH = s.BH, S = s.S;
+  cudaError_t e = launch_reverse_rows(q, qr, BH, S, (long long)s.DHQK * s.esize, cs);
+  if (e == cudaSuccess) e = launch_reverse_rows(k, kr, BH, S, (long long)s.DHQK * s.esize, cs);
+  if (e == cudaSuccess) e = launch_reverse_rows(v, vr, BH, S, (long long)s.DHV * s.esize, cs);
+  if (e == cudaSuccess && orv) e = launch_reverse_rows(ogate, orv, BH, S, (long long)s.DHV * s.esize, cs);
+  if (e == cudaSuccess && igr) e = launch_reverse_rows(igate, igr, BH, S, 4, cs);
+  if (e == cudaSuccess && fgr) e = launch_reverse_rows(fgate, fgr, BH, S, 4, cs);
+  if (e != cudaSuccess) return MLSTM_ERR_CUDA;
+  st = fwd_impl(p, qr, kr, vr, igr, fgr, orv, C0, n0, m0, hr, C_out, n_out, m_out, w + r.fwd, fwd_bytes, cs, nullptr,
+                nullptr);
+  if (st != MLSTM_OK) return st;
+  return launch_reverse_rows(hr, h, BH, S, (long long)s.DHV * s.esize, cs) == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA;
 }
 
 size_t mlstm_bwd_workspace_size(const mlstm_fwd_params_t* p) {

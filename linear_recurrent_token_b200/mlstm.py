@@ -66,6 +66,10 @@ def lib():
         L.mlstm_fwd_chunkwise_noalloc.restype = I
         L.mlstm_noalloc_scratch_bytes.argtypes = []
         L.mlstm_noalloc_scratch_bytes.restype = Z
+        L.mlstm_fwd_chunkwise_reversed_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
+        L.mlstm_fwd_chunkwise_reversed_workspace_size.restype = Z
+        L.mlstm_fwd_chunkwise_reversed.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 14 + [Z, P]
+        L.mlstm_fwd_chunkwise_reversed.restype = I
         L.mlstm_bwd_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
         L.mlstm_bwd_workspace_size.restype = Z
         L.mlstm_bwd.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 22 + [Z, P]
@@ -125,7 +129,7 @@ def plan(params: FwdParams) -> dict:
 def fwd_chunkwise(q, k, v, igate=None, fgate=None, ogate=None, C0=None, n0=None, m0=None, *,
                   chunk: int = 64, num_blocks: int = 1, retention: bool = False,
                   h=None, C_out=None, n_out=None, m_out=None, workspace=None,
-                  return_state: bool = True, stream=None, events=None):
+                  return_state: bool = True, stream=None, events=None, reverse: bool = False):
     """Chunkwise-parallel prefill (mlstm_fwd_chunkwise).  CUDA tensors, contiguous.
 
     q, k [B,NH,S,DHQK], v [B,NH,S,DHV] (fp32 or bf16); igate, fgate [B,NH,S] fp32;
@@ -133,6 +137,8 @@ def fwd_chunkwise(q, k, v, igate=None, fgate=None, ogate=None, C0=None, n0=None,
     m0 [B,NH] fp32 or None (zeros).  Returns (h, C, n, m); n, m are None in
     retention mode and the state is None when return_state is False.
     ``events`` = (begin, end) torch.cuda.Event pair recorded around the main kernel.
+    ``reverse``: the reversed-sequence pass (mlstm_fwd_chunkwise_reversed): token S-1 first,
+    h at the original positions, the final state after token 0.
     """
     B, NH, S, DHQK = q.shape
     DHV = v.shape[-1]
@@ -148,13 +154,20 @@ def fwd_chunkwise(q, k, v, igate=None, fgate=None, ogate=None, C0=None, n0=None,
             n_out = torch.empty((B, NH, nb, DHQK // nb), dtype=torch.float32, device=dev)
         if m_out is None:
             m_out = torch.empty((B, NH), dtype=torch.float32, device=dev)
-    ws_bytes = workspace_size(p)
+    ws_bytes = reversed_workspace_size(p) if reverse else workspace_size(p)
     if workspace is None and ws_bytes > 0:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
     args = [ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(igate), _ptr(fgate), _ptr(ogate),
             _ptr(C0), _ptr(n0), _ptr(m0), _ptr(h), _ptr(C_out), _ptr(n_out), _ptr(m_out),
             _ptr(workspace), ctypes.c_size_t(ws_len), _stream_ptr(stream)]
+    if reverse:
+        if events is not None:
+            raise ValueError("events are not supported with reverse=True")
+        st = lib().mlstm_fwd_chunkwise_reversed(*args)
+        if st != 0:
+            raise MlstmError(st, "mlstm_fwd_chunkwise_reversed")
+        return (h, C_out, None, None) if retention else (h, C_out, n_out, m_out)
     if events is None:
         st = lib().mlstm_fwd_chunkwise(*args)
     else:
@@ -168,6 +181,10 @@ def fwd_chunkwise(q, k, v, igate=None, fgate=None, ogate=None, C0=None, n0=None,
     if retention:
         return h, C_out, None, None
     return h, C_out, n_out, m_out
+
+
+def reversed_workspace_size(params: FwdParams) -> int:
+    return int(lib().mlstm_fwd_chunkwise_reversed_workspace_size(ctypes.byref(params)))
 
 
 def bwd_workspace_size(params: FwdParams) -> int:

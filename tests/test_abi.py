@@ -164,3 +164,25 @@ def test_bwd_null_align_alias_workspace():
     assert bwd_call(p, ws=None) == 5
     assert mlstm.bwd_workspace_size(p) == 2 * 2 * 8 * 64 * 4
     assert mlstm.bwd_workspace_size(params(DHQK=512)) == 0
+
+
+# ---------------------------------------------------------------- reversed-sequence pass
+def rev_call(p, q=A, k=B_, v=C_, ig=D_, fg=E_, og=None, C0=None, n0=None, m0=None, h=F_, C=None, n=None, m=None,
+             ws=G_, ws_bytes=1 << 40):
+    return mlstm.lib().mlstm_fwd_chunkwise_reversed(ctypes.byref(p), q, k, v, ig, fg, og, C0, n0, m0, h, C, n, m, ws,
+                                                    ctypes.c_size_t(ws_bytes), ctypes.c_void_p(0))
+
+
+def test_reversed_validates_like_the_forward_and_checks_its_workspace():
+    p = params()
+    assert rev_call(params(B=-1)) == 2
+    assert rev_call(p, q=None) == 1
+    assert rev_call(p, h=A) == 7                     # h on top of q
+    assert rev_call(p, q=A + 8) == 4
+    need = mlstm.reversed_workspace_size(p)
+    # the reversed copies of q, k, v, gates, o and h come on top of the forward's workspace
+    tok = 2 * 2 * 64
+    assert need >= mlstm.workspace_size(p) + 2 * tok * 16 * 4 + 3 * tok * 16 * 4 + 2 * tok * 4
+    assert rev_call(p, ws_bytes=need - 1) == 5
+    assert rev_call(p, ws=C_ - 256) == 7             # workspace overlapping v
+    assert mlstm.reversed_workspace_size(params(S=0)) == mlstm.workspace_size(params(S=0))

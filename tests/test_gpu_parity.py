@@ -272,7 +272,7 @@ TC_CASES = [
     (1, 1, 64, 64, 64, 1, False, False, False),
     (1, 2, 130, 64, 128, 1, False, True, False),
     (1, 8, 4096, 256, 512, 1, False, True, True),
-    # two / four value tiles of a head run as a cluster and share the key-side work
+    # heads of two and four value tiles
     (1, 2, 1000, 128, 256, 1, False, True, True),
     (2, 2, 700, 64, 256, 1, True, True, False),
     (1, 3, 777, 64, 512, 1, False, True, True),
@@ -370,3 +370,38 @@ def test_tensor_core_gate_regimes(regime, DHV):
     assert all(np.all(np.isfinite(x)) for x in got), regime
     errs = check(got, oracle_fwd(inp, C0=C0, n0=n0, m0=m0), "bf16", what=regime)
     print(regime, errs)
+
+
+@pytest.mark.parametrize("dtype,chunk,nb,retention,with_o", [
+    ("bf16", 64, 1, False, True),    # tensor-core path
+    ("bf16", 64, 1, True, False),    # tensor-core path, retention
+    ("f32", 16, 2, False, False),    # SIMT path, block-diagonal
+])
+def test_reversed_sequence_pass(dtype, chunk, nb, retention, with_o):
+    """mlstm_fwd_chunkwise_reversed == the oracle on the sequence read backwards, with h put
+    back at the original positions and the final state after token 0."""
+    B, NH, S, DHQK, DHV = 2, 2, 333, 64, 128
+    w = inputs.Workload(3, "rev", B, NH, S, DHQK, DHV, chunk, nb, dtype, retention, 1 / np.sqrt(DHQK // nb))
+    inp = inputs.forward_inputs(w, seed=41)
+    rng = np.random.default_rng(8)
+    dk, dv = DHQK // nb, DHV // nb
+    C0 = (rng.standard_normal((B, NH, nb, dv, dk)) * 0.2).astype(np.float32)
+    n0 = None if retention else (rng.standard_normal((B, NH, nb, dk)) * 0.2).astype(np.float32)
+    m0 = None if retention else rng.standard_normal((B, NH)).astype(np.float32)
+    og = None
+    if with_o:
+        og = (1 / (1 + np.exp(-rng.standard_normal((B, NH, S, DHV))))).astype(np.float32)
+        og = torch.from_numpy(og).to(TORCH_DTYPE[dtype]).float().numpy()
+    td = TORCH_DTYPE[dtype]
+    q, k, v = (dev(inp[x], td) for x in ("q", "k", "v"))
+    ig = None if retention else dev(inp["igate"])
+    fg = None if retention else dev(inp["fgate"])
+    h, C, n, m = mlstm.fwd_chunkwise(q, k, v, ig, fg, dev(og, td) if og is not None else None, dev(C0), dev(n0),
+                                     dev(m0), chunk=chunk, num_blocks=nb, retention=retention, reverse=True)
+    torch.cuda.synchronize()
+    flip = lambda x: None if x is None else np.ascontiguousarray(np.flip(x, axis=2))
+    ref = oracle_fwd({"q": flip(inp["q"]), "k": flip(inp["k"]), "v": flip(inp["v"]),
+                      "igate": flip(inp.get("igate")), "fgate": flip(inp.get("fgate"))},
+                     nb, retention, flip(og), C0, n0, m0)
+    ref = (flip(ref[0]),) + tuple(ref[1:])
+    check((host(h), host(C), host(n), host(m)), ref, dtype, retention, what="reversed")
