@@ -515,6 +515,38 @@ def run_backward(w, steps, warmup, flush_bytes, clocks):
     return ms
 
 
+def run_reversed(w, steps, warmup, flush_bytes):
+    """The reversed-sequence prefill (mlstm_fwd_chunkwise_reversed) on the workload, inputs
+    resident, L2 flushed between steps; returns per-step milliseconds."""
+    import torch
+
+    from linear_recurrent_token_b200 import inputs, mlstm
+    td = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    inp = inputs.forward_inputs(w)
+    d = lambda x, dt=torch.float32: None if x is None else torch.from_numpy(np.ascontiguousarray(x)).to("cuda", dt)
+    q, k, v = d(inp["q"], td), d(inp["k"], td), d(inp["v"], td)
+    ig, fg = d(inp.get("igate")), d(inp.get("fgate"))
+    p = mlstm.fwd_params(w.B, w.NH, w.S, w.DHQK, w.DHV, w.chunk, w.num_blocks, td, w.retention)
+    ws = torch.empty(mlstm.reversed_workspace_size(p), dtype=torch.uint8, device="cuda")
+    h = torch.empty((w.B, w.NH, w.S, w.DHV), dtype=td, device="cuda")
+    flush = torch.empty(flush_bytes // 4, dtype=torch.float32, device="cuda")
+    call = lambda: mlstm.fwd_chunkwise(q, k, v, ig, fg, chunk=w.chunk, num_blocks=w.num_blocks,
+                                       retention=w.retention, h=h, workspace=ws, reverse=True)
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        flush.fill_(1.0)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        call()
+        b.record()
+        torch.cuda.synchronize()
+        ms.append(a.elapsed_time(b))
+    return ms
+
+
 def backward_line(w, ms, sm_mhz, cpu: bool):
     step_ms = statistics.median(ms)
     flops = backward_flops(w.B, w.NH, w.S, w.dk, w.dv, w.num_blocks)
@@ -626,6 +658,9 @@ def main():
             dist_barrier(world)
             dec = run_decode(wd, args.steps * 5, args.warmup, clocks)
             dist_barrier(world)
+        rev_ms = None
+        if args.legs == "both":
+            rev_ms = run_reversed(w, max(3, args.steps // 4), args.warmup, 256 << 20)
         bwd = []
         if not args.no_backward and args.legs == "both":
             for idx in (1, 2):
@@ -670,6 +705,16 @@ def main():
                     "h2d_bytes_per_step": dec["h2d"], "d2h_bytes_per_step": dec["d2h"]},
         }
         line["gpu_launches"] += len(dec["step_ms"])
+    if rev_ms:
+        rms = dist_max(statistics.median(rev_ms), world)
+        esz = 2 if w.dtype == "bf16" else 4
+        copy_bytes = 2 * w.B * w.NH * w.S * ((2 * w.DHQK + 2 * w.DHV) * esz + (0 if w.retention else 8))
+        line["reversed"] = {"workload": w.describe(), "value": w.B * w.S * world / (rms * 1e-3), "unit": "tokens/s",
+                            "ms_per_step": rms, "steps": len(rev_ms),
+                            "note": "the forward kernels on reversed copies of q, k, v and the gates, h reversed "
+                                    "back; the copies move reversal_bytes through HBM on top of the forward",
+                            "reversal_bytes": copy_bytes}
+        line["gpu_launches"] += len(rev_ms) * (cw["plan"]["kernels"] + (4 if w.retention else 6))
     if bwd:
         sm_mhz = line["clocks"].get("sm_mhz")
         line["backward"] = [backward_line(wb, ms, sm_mhz, rank == 0 and world == 1 and not args.no_cpu_baseline)
