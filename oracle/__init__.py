@@ -18,6 +18,8 @@ Contents
 ``unstabilised``     numpy, fp64, the recurrence with raw exponential gates and
                      the floor 1 of the mLSTM read-out, no stabiliser at all.
 ``state_bytes``      size of a model's recurrent state (xLSTM 7B "Modelled costs").
+``sequential_scalar_normaliser``  numpy, fp64, the variant with a scalar normaliser and a
+                     learnable bias (Edifice.Recurrent.XLSTMv2, "Key Improvements" #2).
 ``sequential_backward``  numpy, fp64, gradients of ``sequential`` by reverse-mode
                      differentiation of its steps in reverse order (backpropagation
                      through time); pinned by central finite differences.
@@ -298,6 +300,56 @@ def unstabilised(q, k, v, igate, fgate, ogate=None, C0=None, n0=None, num_blocks
             ht = ht * _split_blocks(np.asarray(ogate[:, :, t], dtype=np.float64), nb)
         h[:, :, t] = ht
     return h.reshape(B, NH, S, DHV), C, n
+
+
+def sequential_scalar_normaliser(q, k, v, igate, fgate, bias, ogate=None, C0=None, n0=None, m0=None,
+                                  num_blocks: int = 1):
+    """The mLSTM with the normaliser of Edifice.Recurrent.XLSTMv2 "Key Improvements" #2: a
+    scalar n_t = f_t n_{t-1} + i_t (no key vector) and a learnable bias in the denominator,
+    h_t = o_t * (C_t q_t) / max(|n_t + bias|, 1), fp64, one token at a time.  Gates and their
+    stabiliser as in ``sequential``; in stabilised units n'_t = f' n'_{t-1} + i' and the
+    denominator is max(|n'_t + bias e^{-m_t}|, e^{-m_t}).  n is per head (it depends on the
+    gates only, so the blocks of a head share it).
+
+    bias: [NH]; n0: [B,NH] stabilised; other arguments as for ``sequential``.
+    Returns (h, C, n [B,NH], m [B,NH]).
+    """
+    q, k, v = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
+    B, NH, S, DHQK = q.shape
+    DHV = v.shape[-1]
+    nb = num_blocks
+    dk, dv = DHQK // nb, DHV // nb
+    C0 = np.zeros((B, NH, nb, dv, dk)) if C0 is None else np.asarray(C0, dtype=np.float64)
+    n0 = np.zeros((B, NH)) if n0 is None else np.asarray(n0, dtype=np.float64)
+    m0 = np.zeros((B, NH)) if m0 is None else np.asarray(m0, dtype=np.float64)
+    bias = np.asarray(bias, dtype=np.float64)
+    h = np.zeros((B, NH, S, DHV))
+    C = np.zeros((B, NH, nb, dv, dk))
+    n = np.zeros((B, NH))
+    m = np.zeros((B, NH))
+    for b in range(B):
+        for hd in range(NH):
+            Cs = [C0[b, hd, j].copy() for j in range(nb)]
+            ns, mt = n0[b, hd], m0[b, hd]
+            for t in range(S):
+                lf = float(log_sigmoid(fgate[b, hd, t]))
+                li = float(igate[b, hd, t])
+                m_new = max(lf + mt, li)
+                fp, ip = math.exp(lf + mt - m_new), math.exp(li - m_new)
+                mt = m_new
+                ns = fp * ns + ip
+                den = max(abs(ns + bias[hd] * math.exp(-mt)), math.exp(-mt))
+                for j in range(nb):
+                    sk, sv = slice(j * dk, (j + 1) * dk), slice(j * dv, (j + 1) * dv)
+                    Cs[j] = fp * Cs[j] + ip * np.outer(v[b, hd, t, sv], k[b, hd, t, sk])
+                    ht = Cs[j] @ q[b, hd, t, sk] / den
+                    if ogate is not None:
+                        ht = ht * np.asarray(ogate[b, hd, t, sv], dtype=np.float64)
+                    h[b, hd, t, sv] = ht
+            for j in range(nb):
+                C[b, hd, j] = Cs[j]
+            n[b, hd], m[b, hd] = ns, mt
+    return h, C, n, m
 
 
 def sequential_backward(q, k, v, dh, igate=None, fgate=None, ogate=None, C0=None, n0=None, m0=None,
