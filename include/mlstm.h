@@ -195,6 +195,27 @@ mlstm_status_t mlstm_fwd_chunkwise_reversed(const mlstm_fwd_params_t* p,
                                             mlstm_stream_t stream);
 
 /*
+ * The prefill with the normaliser of Edifice.Recurrent.XLSTMv2 ("Key Improvements" #2): a
+ * scalar n_t = f_t n_{t-1} + i_t and a learnable bias,  h_t = o_t (C_t q_t) / max(|n_t + bias|, 1)
+ * (gates and stabiliser as above; in stabilised units the denominator is
+ * max(|n'_t + bias e^{-m_t}|, e^{-m_t})).  n depends on the gates only, so it is one value per
+ * (batch, head), shared by the head's blocks.  Arguments as for mlstm_fwd_chunkwise, except:
+ *   bias    [NH]   fp32   required (if S > 0)
+ *   n0, n_out [B,NH] fp32 stabilised scalar normaliser (NULL = zero / not written)
+ * retention is rejected (MLSTM_ERR_SHAPE: retention has no normaliser).  Runs on the SIMT fp32
+ * kernels for every dtype; workspace: mlstm_fwd_chunkwise_scalar_normaliser_workspace_size.
+ */
+size_t mlstm_fwd_chunkwise_scalar_normaliser_workspace_size(const mlstm_fwd_params_t* p);
+mlstm_status_t mlstm_fwd_chunkwise_scalar_normaliser(const mlstm_fwd_params_t* p,
+                                                     const void* q, const void* k, const void* v,
+                                                     const float* igate, const float* fgate, const void* ogate,
+                                                     const float* bias,
+                                                     const float* C0, const float* n0, const float* m0,
+                                                     void* h, float* C_out, float* n_out, float* m_out,
+                                                     void* workspace, size_t workspace_bytes,
+                                                     mlstm_stream_t stream);
+
+/*
  * Backward of the recurrence: gradients of a loss with respect to the inputs of
  * mlstm_fwd_chunkwise, given its gradient dh with respect to h (and optionally dC, dn
  * with respect to the final state).  Reverse-mode differentiation of the sequential

@@ -13,6 +13,9 @@
 //   C     <- e^{g+m_c-m_next} C + sum_s e^{g-b_s+itilde_s-m_next} v_s k_s^T   (same for n)
 // Retention replaces the gate weights by powers of gamma_h and drops the normaliser
 // (RetNet "Key Innovation": D[n,m] = gamma^(n-m)).
+// With a.nbias set, the normaliser is the scalar n_t = f n_{t-1} + i of Edifice.Recurrent.
+// XLSTMv2 ("Key Improvements" #2) and the denominator max(|n_t + bias|, 1), i.e. in these units
+//   max(|sum_s exp(b_t - b_s + itilde_s - m_t) + e^{b_t+m_c-m_t} n + bias e^{-m_t}|, e^{-m_t}).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -69,7 +72,13 @@ __global__ void __launch_bounds__(256) simt_walk_kernel(WalkArgs a) {
     const int r = i / dk, c = i % dk;
     Cs[r * ldk + c] = a.C0 ? a.C0[((size_t)slice * dv + v0 + r) * dk + c] : 0.f;
   }
-  for (int c = tid; c < dk; c += nt) ns[c] = ret ? 0.f : a.n_init[(size_t)slice * dk + c];
+  const bool scalar_n = a.nbias != nullptr && !ret;
+  const float nbias = scalar_n ? a.nbias[head] : 0.f;
+  if (scalar_n) {
+    if (tid == 0) ns[0] = a.n_init[bh];
+  } else {
+    for (int c = tid; c < dk; c += nt) ns[c] = ret ? 0.f : a.n_init[(size_t)slice * dk + c];
+  }
   float m_c = ret ? 0.f : a.m_init[bh];
 
   for (int c0 = 0; c0 < S; c0 += L) {
@@ -124,7 +133,14 @@ __global__ void __launch_bounds__(256) simt_walk_kernel(WalkArgs a) {
       Ps[t * (L + 1) + s] = p;
     }
     __syncthreads();
-    if (!ret) {
+    if (scalar_n) {
+      for (int t = tid; t < Lc; t += nt) {
+        float rs = 0.f;
+        for (int s = 0; s <= t; ++s) rs += expf(bl[t] - bl[s] + li[s] - mt[t]);
+        const float emt = expf(-mt[t]);
+        den[t] = fmaxf(fabsf(rs + sint[t] * ns[0] + nbias * emt), emt);
+      }
+    } else if (!ret) {
       for (int t = tid; t < Lc; t += nt) {
         float rs = 0.f, qn = 0.f;
         for (int s = 0; s <= t; ++s) rs += Ps[t * (L + 1) + s];
@@ -153,7 +169,13 @@ __global__ void __launch_bounds__(256) simt_walk_kernel(WalkArgs a) {
       for (int s = 0; s < Lc; ++s) acc += wv[s] * Vs[s * TV + r] * Ks[s * ldk + c];
       Cs[r * ldk + c] = decay * Cs[r * ldk + c] + acc;
     }
-    if (!ret) {
+    if (scalar_n) {
+      if (tid == 0) {
+        float acc = 0.f;
+        for (int s = 0; s < Lc; ++s) acc += wv[s];
+        ns[0] = decay * ns[0] + acc;
+      }
+    } else if (!ret) {
       for (int c = tid; c < dk; c += nt) {
         float acc = 0.f;
         for (int s = 0; s < Lc; ++s) acc += wv[s] * Ks[s * ldk + c];
@@ -170,8 +192,11 @@ __global__ void __launch_bounds__(256) simt_walk_kernel(WalkArgs a) {
       a.C_out[((size_t)slice * dv + v0 + r) * dk + c] = Cs[r * ldk + c];
     }
   if (!ret && blockIdx.x == 0) {
-    if (a.n_out)
+    if (a.n_out && scalar_n) {
+      if (blk == 0 && tid == 0) a.n_out[bh] = ns[0];
+    } else if (a.n_out) {
       for (int c = tid; c < dk; c += nt) a.n_out[(size_t)slice * dk + c] = ns[c];
+    }
     if (a.m_out && blk == 0 && tid == 0) a.m_out[bh] = m_c;
   }
 }

@@ -18,6 +18,8 @@ struct WalkArgs {
   const float *n_init;       // [BH*nb, dk] snapshot of n0 (never NULL for mLSTM)
   const float *m_init;       // [BH] snapshot of m0 (never NULL for mLSTM)
   const float *m_tok;        // [BH, S] stabiliser per token (mLSTM)
+  const float *nbias;        // [NH]: scalar normaliser with this bias (NULL = vector n . q);
+                             // then n_init / n_out hold one value per (batch, head)
   void *h;
   float *C_out, *n_out, *m_out;
 };

@@ -409,6 +409,105 @@ mlstm_status_t mlstm_fwd_chunkwise_reversed(const mlstm_fwd_params_t* p, const v
   return launch_reverse_rows(hr, h, BH, S, (long long)s.DHV * s.esize, cs) == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA;
 }
 
+// Workspace of the scalar-normaliser prefill (SIMT walk): per-token stabiliser and snapshots
+// of m0 and of the per-head n0.
+static size_t scalar_norm_ws(const FwdShape& s) {
+  if (s.BH == 0 || s.S == 0) return 0;
+  return align_up(sizeof(float) * (size_t)s.BH * s.S) + 2 * align_up(sizeof(float) * (size_t)s.BH);
+}
+
+size_t mlstm_fwd_chunkwise_scalar_normaliser_workspace_size(const mlstm_fwd_params_t* p) {
+  FwdShape s;
+  if (check_fwd(p, &s) != MLSTM_OK || p->retention) return 0;
+  return scalar_norm_ws(s);
+}
+
+mlstm_status_t mlstm_fwd_chunkwise_scalar_normaliser(const mlstm_fwd_params_t* p, const void* q, const void* k,
+                                                     const void* v, const float* igate, const float* fgate,
+                                                     const void* ogate, const float* bias, const float* C0,
+                                                     const float* n0, const float* m0, void* h, float* C_out,
+                                                     float* n_out, float* m_out, void* workspace,
+                                                     size_t workspace_bytes, mlstm_stream_t stream) {
+  FwdShape s;
+  mlstm_status_t st = check_fwd(p, &s);
+  if (st != MLSTM_OK) return st;
+  if (p->retention) return MLSTM_ERR_SHAPE;  // retention has no normaliser
+  if (s.BH > 0 && s.S > 0 && simt_walk_pick_tile(s.chunk, s.dk, s.dv) == 0) return MLSTM_ERR_SHAPE;
+  const size_t tok = (size_t)s.BH * s.S;
+  const size_t bq = tok * s.DHQK * s.esize, bv = tok * s.DHV * s.esize, bg = tok * sizeof(float);
+  const size_t bC = (size_t)s.BH * s.nb * s.dv * s.dk * sizeof(float), bh4 = (size_t)s.BH * sizeof(float);
+  if (tok > 0 && (!q || !k || !v || !h || !igate || !fgate || !bias)) return MLSTM_ERR_NULL;
+  const void* all[] = {q, k, v, igate, fgate, ogate, bias, C0, n0, m0, h, C_out, n_out, m_out, workspace};
+  for (const void* ptr : all)
+    if (ptr && misaligned(ptr)) return MLSTM_ERR_ALIGN;
+  const size_t need = scalar_norm_ws(s);
+  const Range inputs[] = {{q, bq}, {k, bq}, {v, bv}, {igate, bg}, {fgate, bg}, {ogate, bv}, {bias, (size_t)s.NH * 4}};
+  const Range outs[] = {{h, bv}, {C_out, bC}, {n_out, bh4}, {m_out, bh4}, {workspace, need}};
+  for (const Range& o : outs)
+    for (const Range& i : inputs)
+      if (overlaps(o, i)) return MLSTM_ERR_ALIAS;
+  for (int a = 0; a < 5; ++a)
+    for (int b = a + 1; b < 5; ++b)
+      if (overlaps(outs[a], outs[b])) return MLSTM_ERR_ALIAS;
+  const Range states_in[] = {{C0, bC}, {n0, bh4}, {m0, bh4}};
+  for (int i = 0; i < 3; ++i) {
+    if (overlaps(outs[0], states_in[i]) || overlaps(outs[4], states_in[i])) return MLSTM_ERR_ALIAS;
+    for (int j = 1; j < 4; ++j) {
+      const bool exact = outs[j].p == states_in[i].p && outs[j].n == states_in[i].n && j == i + 1;
+      if (overlaps(outs[j], states_in[i]) && !exact) return MLSTM_ERR_ALIAS;
+    }
+  }
+  if (need > 0 && (!workspace || workspace_bytes < need)) return MLSTM_ERR_WORKSPACE;
+  if (s.BH == 0) return MLSTM_OK;
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  if (s.S == 0) {  // the final state is the initial state
+    if (C_out && C_out != C0)
+      e = C0 ? cudaMemcpyAsync(C_out, C0, bC, cudaMemcpyDeviceToDevice, cs) : cudaMemsetAsync(C_out, 0, bC, cs);
+    if (e == cudaSuccess && n_out && n_out != n0)
+      e = n0 ? cudaMemcpyAsync(n_out, n0, bh4, cudaMemcpyDeviceToDevice, cs) : cudaMemsetAsync(n_out, 0, bh4, cs);
+    if (e == cudaSuccess && m_out && m_out != m0)
+      e = m0 ? cudaMemcpyAsync(m_out, m0, bh4, cudaMemcpyDeviceToDevice, cs) : cudaMemsetAsync(m_out, 0, bh4, cs);
+    return e == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA;
+  }
+  char* w = static_cast<char*>(workspace);
+  float* m_tok = reinterpret_cast<float*>(w);
+  float* m_init = reinterpret_cast<float*>(w + align_up(sizeof(float) * tok));
+  float* n_init = reinterpret_cast<float*>(w + align_up(sizeof(float) * tok) + align_up(bh4));
+  e = launch_gate_prep((int)s.BH, s.S, 1, igate, fgate, m0, n0, m_tok, m_init, n_init, cs);
+  if (e != cudaSuccess) return MLSTM_ERR_CUDA;
+  WalkArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = s.B;
+  a.NH = s.NH;
+  a.S = s.S;
+  a.DHQK = s.DHQK;
+  a.DHV = s.DHV;
+  a.chunk = s.chunk;
+  a.nb = s.nb;
+  a.retention = 0;
+  a.dk = s.dk;
+  a.dv = s.dv;
+  a.dtype = s.dtype;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.og = ogate;
+  a.ig = igate;
+  a.fg = fgate;
+  a.C0 = C0;
+  a.n_init = n_init;
+  a.m_init = m_init;
+  a.m_tok = m_tok;
+  a.nbias = bias;
+  a.h = h;
+  a.C_out = C_out;
+  a.n_out = n_out;
+  a.m_out = m_out;
+  a.dv_tile = simt_walk_pick_tile(s.chunk, s.dk, s.dv);
+  return launch_simt_walk(a, cs) == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA;
+}
+
 size_t mlstm_bwd_workspace_size(const mlstm_fwd_params_t* p) {
   FwdShape s;
   if (check_bwd(p, &s) != MLSTM_OK) return 0;

@@ -70,6 +70,10 @@ def lib():
         L.mlstm_fwd_chunkwise_reversed_workspace_size.restype = Z
         L.mlstm_fwd_chunkwise_reversed.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 14 + [Z, P]
         L.mlstm_fwd_chunkwise_reversed.restype = I
+        L.mlstm_fwd_chunkwise_scalar_normaliser_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
+        L.mlstm_fwd_chunkwise_scalar_normaliser_workspace_size.restype = Z
+        L.mlstm_fwd_chunkwise_scalar_normaliser.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 15 + [Z, P]
+        L.mlstm_fwd_chunkwise_scalar_normaliser.restype = I
         L.mlstm_bwd_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
         L.mlstm_bwd_workspace_size.restype = Z
         L.mlstm_bwd.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 22 + [Z, P]
@@ -180,6 +184,33 @@ def fwd_chunkwise(q, k, v, igate=None, fgate=None, ogate=None, C0=None, n0=None,
         raise MlstmError(st, "mlstm_fwd_chunkwise")
     if retention:
         return h, C_out, None, None
+    return h, C_out, n_out, m_out
+
+
+def fwd_chunkwise_scalar_normaliser(q, k, v, igate, fgate, bias, ogate=None, C0=None, n0=None, m0=None, *,
+                                    chunk: int = 64, num_blocks: int = 1, workspace=None, stream=None):
+    """The prefill with a scalar normaliser and a learnable bias
+    (mlstm_fwd_chunkwise_scalar_normaliser): bias [NH] fp32, n0 [B,NH] fp32 or None.
+    Returns (h, C, n [B,NH], m [B,NH])."""
+    B, NH, S, DHQK = q.shape
+    DHV = v.shape[-1]
+    nb = int(num_blocks)
+    p = fwd_params(B, NH, S, DHQK, DHV, chunk, nb, q.dtype, False)
+    dev = q.device
+    h = torch.empty((B, NH, S, DHV), dtype=q.dtype, device=dev)
+    C_out = torch.empty((B, NH, nb, DHV // nb, DHQK // nb), dtype=torch.float32, device=dev)
+    n_out = torch.empty((B, NH), dtype=torch.float32, device=dev)
+    m_out = torch.empty((B, NH), dtype=torch.float32, device=dev)
+    ws_bytes = int(lib().mlstm_fwd_chunkwise_scalar_normaliser_workspace_size(ctypes.byref(p)))
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().mlstm_fwd_chunkwise_scalar_normaliser(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(igate), _ptr(fgate), _ptr(ogate), _ptr(bias), _ptr(C0),
+        _ptr(n0), _ptr(m0), _ptr(h), _ptr(C_out), _ptr(n_out), _ptr(m_out), _ptr(workspace), ctypes.c_size_t(ws_len),
+        _stream_ptr(stream))
+    if st != 0:
+        raise MlstmError(st, "mlstm_fwd_chunkwise_scalar_normaliser")
     return h, C_out, n_out, m_out
 
 

@@ -155,7 +155,9 @@ def test_bwd_null_align_alias_workspace():
     assert bwd_call(p, dh=None) == 1
     assert bwd_call(p, fg=None) == 1
     assert bwd_call(p, dq=None) == 1
-    assert bwd_call(params(retention=True), ig=None, fg=None) != 1  # gates ignored in retention
+    # gates are ignored in retention mode: validation passes them and stops at the (too small)
+    # workspace, so nothing is launched with these fake pointers
+    assert bwd_call(params(retention=True), ig=None, fg=None, ws_bytes=16) == 5
     assert bwd_call(p, q=A + 8) == 4
     assert bwd_call(p, dq=A) == 7                  # dq on top of q
     assert bwd_call(p, dk=0x9000000) == 7          # dk on top of dq
@@ -186,3 +188,25 @@ def test_reversed_validates_like_the_forward_and_checks_its_workspace():
     assert rev_call(p, ws_bytes=need - 1) == 5
     assert rev_call(p, ws=C_ - 256) == 7             # workspace overlapping v
     assert mlstm.reversed_workspace_size(params(S=0)) == mlstm.workspace_size(params(S=0))
+
+
+# ---------------------------------------------------------------- scalar-normaliser prefill
+def sn_call(p, q=A, k=B_, v=C_, ig=D_, fg=E_, og=None, bias=0xD000000, C0=None, n0=None, m0=None, h=F_, C=None, n=None,
+            m=None, ws=G_, ws_bytes=1 << 40):
+    return mlstm.lib().mlstm_fwd_chunkwise_scalar_normaliser(ctypes.byref(p), q, k, v, ig, fg, og, bias, C0, n0, m0,
+                                                             h, C, n, m, ws, ctypes.c_size_t(ws_bytes),
+                                                             ctypes.c_void_p(0))
+
+
+def test_scalar_normaliser_validation():
+    p = params()
+    assert sn_call(params(retention=True)) == 2        # retention has no normaliser
+    assert sn_call(p, bias=None) == 1
+    assert sn_call(p, fg=None) == 1
+    assert sn_call(p, bias=0xD000000 + 4) == 4
+    assert sn_call(p, h=A) == 7
+    assert sn_call(p, n=0xD000000) == 7                 # n_out on top of the bias
+    # an in-place state passes the alias checks and stops at the (too small) workspace
+    assert sn_call(p, C=0xE000000, C0=0xE000000, ws_bytes=16) == 5
+    need = mlstm.lib().mlstm_fwd_chunkwise_scalar_normaliser_workspace_size(ctypes.byref(p))
+    assert need > 0 and sn_call(p, ws_bytes=need - 1) == 5

@@ -405,3 +405,38 @@ def test_reversed_sequence_pass(dtype, chunk, nb, retention, with_o):
                      nb, retention, flip(og), C0, n0, m0)
     ref = (flip(ref[0]),) + tuple(ref[1:])
     check((host(h), host(C), host(n), host(m)), ref, dtype, retention, what="reversed")
+
+
+@pytest.mark.parametrize("dtype,chunk,nb,with_o,with_state", [
+    ("f32", 16, 1, False, True),
+    ("bf16", 64, 2, True, True),
+    ("bf16", 32, 1, False, False),
+])
+def test_scalar_normaliser_prefill(dtype, chunk, nb, with_o, with_state):
+    """mlstm_fwd_chunkwise_scalar_normaliser == oracle.sequential_scalar_normaliser (scalar
+    n_t = f n + i, denominator max(|n + bias|, 1)), h and final state."""
+    B, NH, S, DHQK, DHV = 2, 3, 301, 64, 64
+    w = inputs.Workload(1, "sn", B, NH, S, DHQK, DHV, chunk, nb, dtype, False, 1 / np.sqrt(DHQK // nb))
+    inp = inputs.forward_inputs(w, seed=51)
+    rng = np.random.default_rng(9)
+    dk, dv = DHQK // nb, DHV // nb
+    bias = rng.standard_normal(NH).astype(np.float32) * 2.0
+    C0 = n0 = m0 = og = None
+    if with_state:
+        C0 = (rng.standard_normal((B, NH, nb, dv, dk)) * 0.2).astype(np.float32)
+        n0 = (rng.standard_normal((B, NH)) * 0.5).astype(np.float32)
+        m0 = rng.standard_normal((B, NH)).astype(np.float32)
+    if with_o:
+        og = (1 / (1 + np.exp(-rng.standard_normal((B, NH, S, DHV))))).astype(np.float32)
+        og = torch.from_numpy(og).to(TORCH_DTYPE[dtype]).float().numpy()
+    td = TORCH_DTYPE[dtype]
+    h, C, n, m = mlstm.fwd_chunkwise_scalar_normaliser(
+        dev(inp["q"], td), dev(inp["k"], td), dev(inp["v"], td), dev(inp["igate"]), dev(inp["fgate"]), dev(bias),
+        dev(og, td) if og is not None else None, dev(C0), dev(n0), dev(m0), chunk=chunk, num_blocks=nb)
+    torch.cuda.synchronize()
+    hr, Cr, nr, mr = oracle.sequential_scalar_normaliser(inp["q"], inp["k"], inp["v"], inp["igate"], inp["fgate"],
+                                                         bias, og, C0, n0, m0, num_blocks=nb)
+    tol = TOL[dtype]
+    errs = {"h": slice_relerr(host(h), hr, 2), "C": slice_relerr(host(C), Cr, 3),
+            "n": float(np.max(np.abs(host(n) - nr)) / max(np.max(np.abs(nr)), 1e-30)), "m": m_err(host(m), mr)}
+    assert all(e <= tol for e in errs.values()), errs
