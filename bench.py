@@ -39,12 +39,12 @@ RECORDED_TRAFFIC = {
     ("tc_walk", "large_head"): {
         "bytes": 147_769_088 + 40_159_232,
         "sources": ("chunkwise_tc.cu", "sm100.cuh", "common.cuh", "kernels.h"),
-        "sha256": "b0ef1a9b6e7b1aac4b20a8e7990724c34500f309eea0a7ddf3b63575a6ce5846",
+        "sha256": "f1bffa7263213551f2c2ba8c787e48d21cc7ce845f47fdb6f6f5b5cef9109063",
     },
     ("step", "decode"): {
         "bytes": 540_096_256 + 480_655_616,
         "sources": ("step.cu", "common.cuh", "kernels.h"),
-        "sha256": "45215b51f32ce50a67dcd31064196f32c13182bf3f4189cf139d1f7115cd65f1",
+        "sha256": "7fabfb5c78ac0ae706a843259d2689de36ebce8ec00e52aec5ff53012b012fc1",
     },
 }
 
