@@ -547,6 +547,39 @@ def run_reversed(w, steps, warmup, flush_bytes):
     return ms
 
 
+def run_scalar_normaliser(w, steps, warmup, flush_bytes):
+    """The scalar-normaliser prefill (mlstm_fwd_chunkwise_scalar_normaliser, one n per head
+    and a per-head bias) on the workload, inputs resident, L2 flushed between steps; returns
+    per-step milliseconds."""
+    import torch
+
+    from linear_recurrent_token_b200 import inputs, mlstm
+    td = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    inp = inputs.forward_inputs(w)
+    d = lambda x, dt=torch.float32: None if x is None else torch.from_numpy(np.ascontiguousarray(x)).to("cuda", dt)
+    q, k, v = d(inp["q"], td), d(inp["k"], td), d(inp["v"], td)
+    ig, fg = d(inp["igate"]), d(inp["fgate"])
+    bias = torch.full((w.NH,), 0.5, dtype=torch.float32, device="cuda")
+    p = mlstm.fwd_params(w.B, w.NH, w.S, w.DHQK, w.DHV, w.chunk, w.num_blocks, td, False)
+    ws = torch.empty(max(1, mlstm.scalar_normaliser_workspace_size(p)), dtype=torch.uint8, device="cuda")
+    flush = torch.empty(flush_bytes // 4, dtype=torch.float32, device="cuda")
+    call = lambda: mlstm.fwd_chunkwise_scalar_normaliser(q, k, v, ig, fg, bias, chunk=w.chunk,
+                                                         num_blocks=w.num_blocks, workspace=ws)
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        flush.fill_(1.0)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        call()
+        b.record()
+        torch.cuda.synchronize()
+        ms.append(a.elapsed_time(b))
+    return ms
+
+
 def backward_line(w, ms, sm_mhz, cpu: bool):
     step_ms = statistics.median(ms)
     flops = backward_flops(w.B, w.NH, w.S, w.dk, w.dv, w.num_blocks)
@@ -661,6 +694,11 @@ def main():
         rev_ms = None
         if args.legs == "both":
             rev_ms = run_reversed(w, max(3, args.steps // 4), args.warmup, 256 << 20)
+        sn = []
+        if args.legs == "both":
+            for idx in (1, 3):
+                wn = inputs.WORKLOADS[idx]
+                sn.append((wn, run_scalar_normaliser(wn, max(3, args.steps // 4), args.warmup, 256 << 20)))
         bwd = []
         if not args.no_backward and args.legs == "both":
             for idx in (1, 2):
@@ -715,6 +753,22 @@ def main():
                                     "back; the copies move reversal_bytes through HBM on top of the forward",
                             "reversal_bytes": copy_bytes}
         line["gpu_launches"] += len(rev_ms) * (cw["plan"]["kernels"] + (4 if w.retention else 6))
+    if sn:
+        sm_mhz = line["clocks"].get("sm_mhz")
+        line["scalar_normaliser"] = []
+        for wn, ms in sn:
+            nms = dist_max(statistics.median(ms), world)
+            flops = chunkwise_flops(wn.B, wn.NH, wn.S, wn.dk, wn.dv, wn.chunk, wn.num_blocks, False)
+            tf = flops / (nms * 1e-3) / 1e12
+            peak = fp32_simt_peak_tflops(sm_mhz)
+            line["scalar_normaliser"].append({
+                "workload": wn.describe(), "value": wn.B * wn.S * world / (nms * 1e-3), "unit": "tokens/s",
+                "ms_per_step": nms, "steps": len(ms),
+                "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                             "traffic": None, "kernel": "SIMT chunkwise walk, scalar normaliser",
+                             "flops_per_launch": flops,
+                             "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x median SM clock"}})
+            line["gpu_launches"] += len(ms) * 2
     if bwd:
         sm_mhz = line["clocks"].get("sm_mhz")
         line["backward"] = [backward_line(wb, ms, sm_mhz, rank == 0 and world == 1 and not args.no_cpu_baseline)

@@ -218,6 +218,10 @@ def reversed_workspace_size(params: FwdParams) -> int:
     return int(lib().mlstm_fwd_chunkwise_reversed_workspace_size(ctypes.byref(params)))
 
 
+def scalar_normaliser_workspace_size(params: FwdParams) -> int:
+    return int(lib().mlstm_fwd_chunkwise_scalar_normaliser_workspace_size(ctypes.byref(params)))
+
+
 def bwd_workspace_size(params: FwdParams) -> int:
     return int(lib().mlstm_bwd_workspace_size(ctypes.byref(params)))
 

@@ -20,6 +20,9 @@ Contents
 ``state_bytes``      size of a model's recurrent state (xLSTM 7B "Modelled costs").
 ``sequential_scalar_normaliser``  numpy, fp64, the variant with a scalar normaliser and a
                      learnable bias (Edifice.Recurrent.XLSTMv2, "Key Improvements" #2).
+``theta_rotate``, ``group_norm_gate``, ``retention_block``  numpy, fp64, the steps
+                     either side of retention (Edifice.Attention.RetNet): the rotation of
+                     q and k, the per-head GroupNorm and the SiLU gate, and their composition.
 ``sequential_backward``  numpy, fp64, gradients of ``sequential`` by reverse-mode
                      differentiation of its steps in reverse order (backpropagation
                      through time); pinned by central finite differences.
@@ -468,6 +471,84 @@ def sequential_backward(q, k, v, dh, igate=None, fgate=None, ogate=None, C0=None
                 df[b, hd] = dlf / (1.0 + np.exp(np.asarray(fgate[b, hd], dtype=np.float64)))
     out.update(di=di, df=df, dn0=dn0, dm0=dm0)
     return out
+
+
+def theta_rotate(x, pos0=None, base: float = 10000.0):
+    """The relative-position rotation Theta that RetNet applies to queries and keys before
+    retention (Edifice.Attention.RetNet, "Key Innovation": Y = (Q Theta) D (K Theta)^T V),
+    fp64.  Theta is not spelled out on the page; the reading built here is the complex form
+    Theta_n = e^{i n theta}: the head vector's entries (2j, 2j+1) are one complex number,
+    multiplied by e^{i p theta_j} at sequence position p, theta_j = base^{-2j/D}.  The same
+    rotation on q and k makes (Q Theta)(K Theta)^T depend on positions only through n - m.
+
+    x: [B,NH,S,D], D even; pos0: [B] position of token 0 of each sequence (None = 0).
+    Returns the rotated x, fp64.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    B, NH, S, D = x.shape
+    pos0 = np.zeros(B, dtype=np.int64) if pos0 is None else np.asarray(pos0, dtype=np.int64)
+    theta = base ** (-2.0 * np.arange(D // 2) / D)
+    out = np.empty_like(x)
+    for b in range(B):
+        pos = (pos0[b] + np.arange(S)).astype(np.float64)
+        ang = pos[:, None] * theta[None, :]                # [S, D/2]
+        c, s_ = np.cos(ang), np.sin(ang)
+        x0, x1 = x[b, :, :, 0::2], x[b, :, :, 1::2]        # [NH, S, D/2]
+        out[b, :, :, 0::2] = x0 * c - x1 * s_
+        out[b, :, :, 1::2] = x0 * s_ + x1 * c
+    return out
+
+
+def silu(x):
+    """x sigmoid(x), fp64."""
+    x = np.asarray(x, dtype=np.float64)
+    return x / (1.0 + np.exp(-x))
+
+
+def group_norm_gate(h, g=None, weight=None, bias=None, eps: float = 1e-5):
+    """Per-head GroupNorm of the retention output followed by the SiLU gate
+    (Edifice.Attention.RetNet, "Multi-Scale Retention (MSR)": GroupNorm over heads, then
+    Y = SiLU(X W_G) * GroupNorm(Retention(X))), fp64.  Each (batch, head, token) row of DHV
+    values is one group: y = (h - mean) / sqrt(var + eps) * weight + bias with the biased
+    variance, then y *= silu(g).  The projections X W_G (given here as g) and W_O are
+    matrix products outside the recurrence.
+
+    h, g: [B,NH,S,DHV] (g None = no gate); weight, bias: [NH*DHV] per channel (None = 1, 0).
+    Returns y, fp64.
+    """
+    h = np.asarray(h, dtype=np.float64)
+    B, NH, S, DHV = h.shape
+    mu = h.mean(axis=-1, keepdims=True)
+    var = ((h - mu) ** 2).mean(axis=-1, keepdims=True)
+    y = (h - mu) / np.sqrt(var + eps)
+    if weight is not None:
+        y = y * np.asarray(weight, dtype=np.float64).reshape(1, NH, 1, DHV)
+    if bias is not None:
+        y = y + np.asarray(bias, dtype=np.float64).reshape(1, NH, 1, DHV)
+    if g is not None:
+        y = y * silu(g)
+    return y
+
+
+def retention_block(q, k, v, igate=None, fgate=None, g=None, gn_weight=None, gn_bias=None,
+                    C0=None, n0=None, m0=None, *, pos0=None, theta_base: float = 10000.0,
+                    eps: float = 1e-5, num_blocks: int = 1, retention: bool = True, rounding=None):
+    """The multi-scale retention block around the recurrence, in the page's order
+    (Edifice.Attention.RetNet, "Key Innovation" and "Multi-Scale Retention (MSR)"): rotate q
+    and k by Theta, run the recurrence (``sequential``), GroupNorm each head's output and
+    gate it with SiLU(g).  ``rounding`` (None or a function) is applied to the rotated q, k
+    and to h before the GroupNorm, to model a storage precision between the steps.
+
+    Returns (y, C, n, m) as ``sequential`` does (n, m None in retention mode).
+    """
+    qr, kr = theta_rotate(q, pos0, theta_base), theta_rotate(k, pos0, theta_base)
+    if rounding is not None:
+        qr, kr = rounding(qr), rounding(kr)
+    h, C, n, m = sequential(qr, kr, v, igate, fgate, None, C0, n0, m0, num_blocks=num_blocks,
+                            retention=retention)
+    if rounding is not None:
+        h = rounding(h)
+    return group_norm_gate(h, g, gn_weight, gn_bias, eps), C, n, m
 
 
 def state_bytes(layers: int, heads: int, dqk: int, dv: int, bytes_per_value: int) -> int:
