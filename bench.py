@@ -580,6 +580,71 @@ def run_scalar_normaliser(w, steps, warmup, flush_bytes):
     return ms
 
 
+def run_msr(w, steps, warmup, flush_bytes, hbm_peak):
+    """The multi-scale retention block (mlstm_fwd_chunkwise_msr: rotation of q and k, the
+    recurrence, GroupNorm + SiLU gate) on the workload, inputs resident, L2 flushed between
+    steps; also the plain forward, and the rotation and GroupNorm kernels alone with their
+    bytes against the HBM peak.  Returns a dict for the JSON line."""
+    import torch
+
+    from linear_recurrent_token_b200 import inputs, mlstm
+    td = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    esz = 2 if w.dtype == "bf16" else 4
+    inp = inputs.forward_inputs(w)
+    d = lambda x, dt=torch.float32: None if x is None else torch.from_numpy(np.ascontiguousarray(x)).to("cuda", dt)
+    q, k, v = d(inp["q"], td), d(inp["k"], td), d(inp["v"], td)
+    ig = None if w.retention else d(inp["igate"])
+    fg = None if w.retention else d(inp["fgate"])
+    rng = np.random.default_rng(7)
+    g = torch.from_numpy(rng.standard_normal((w.B, w.NH, w.S, w.DHV)).astype(np.float32)).to("cuda", td)
+    gw = torch.ones(w.NH * w.DHV, dtype=torch.float32, device="cuda")
+    gb = torch.zeros(w.NH * w.DHV, dtype=torch.float32, device="cuda")
+    pos0 = torch.zeros(w.B, dtype=torch.int64, device="cuda")
+    p = mlstm.fwd_params(w.B, w.NH, w.S, w.DHQK, w.DHV, w.chunk, w.num_blocks, td, w.retention)
+    ws = torch.empty(max(1, mlstm.msr_workspace_size(p)), dtype=torch.uint8, device="cuda")
+    wsf = torch.empty(max(1, mlstm.workspace_size(p)), dtype=torch.uint8, device="cuda")
+    y = torch.empty((w.B, w.NH, w.S, w.DHV), dtype=td, device="cuda")
+    qo, ko = torch.empty_like(q), torch.empty_like(k)
+    flush = torch.empty(flush_bytes // 4, dtype=torch.float32, device="cuda")
+    calls = {
+        "block": lambda: mlstm.fwd_chunkwise_msr(q, k, v, ig, fg, g, gw, gb, pos0=pos0, chunk=w.chunk,
+                                                 num_blocks=w.num_blocks, retention=w.retention, y=y, workspace=ws),
+        "forward": lambda: mlstm.fwd_chunkwise(q, k, v, ig, fg, chunk=w.chunk, num_blocks=w.num_blocks,
+                                               retention=w.retention, h=y, workspace=wsf, return_state=False),
+        "rotate": lambda: mlstm.theta_rotate(q, k, pos0, q_out=qo, k_out=ko),
+        "gn_gate": lambda: mlstm.group_norm_gate(v, g, gw, gb, 1e-5, y=y),
+    }
+    out = {}
+    for name, call in calls.items():
+        for _ in range(warmup):
+            call()
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(steps):
+            flush.fill_(1.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            call()
+            b.record()
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        out[name] = statistics.median(ms)
+    tok = w.B * w.NH * w.S
+    rot_bytes = 4 * tok * w.DHQK * esz
+    gn_bytes = 3 * tok * w.DHV * esz + 2 * w.NH * w.DHV * 4
+    return {"block_ms": out["block"], "forward_ms": out["forward"], "steps": steps,
+            "rotate": {"ms": out["rotate"], "bytes_per_launch": rot_bytes,
+                       "roofline": {"bound": "hbm", "achieved": rot_bytes / (out["rotate"] * 1e-3) / 1e9,
+                                    "peak": hbm_peak, "unit": "GB/s",
+                                    "frac": rot_bytes / (out["rotate"] * 1e-3) / 1e9 / hbm_peak, "traffic": None,
+                                    "kernel": "theta_rotate_kernel"}},
+            "gn_gate": {"ms": out["gn_gate"], "bytes_per_launch": gn_bytes,
+                        "roofline": {"bound": "hbm", "achieved": gn_bytes / (out["gn_gate"] * 1e-3) / 1e9,
+                                     "peak": hbm_peak, "unit": "GB/s",
+                                     "frac": gn_bytes / (out["gn_gate"] * 1e-3) / 1e9 / hbm_peak, "traffic": None,
+                                     "kernel": "gn_gate_kernel (standalone; v as h)"}}}
+
+
 def backward_line(w, ms, sm_mhz, cpu: bool):
     step_ms = statistics.median(ms)
     flops = backward_flops(w.B, w.NH, w.S, w.dk, w.dv, w.num_blocks)
@@ -612,7 +677,7 @@ def main():
     ap.add_argument("--workload", type=int, default=3, help="chunkwise workload index (default 3)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
-    ap.add_argument("--legs", choices=["both", "chunkwise", "decode", "backward"], default="both",
+    ap.add_argument("--legs", choices=["both", "chunkwise", "decode", "backward", "msr"], default="both",
                     help="run only one leg (for profiling); the default runs both")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -663,6 +728,11 @@ def main():
                 if rank == 0:
                     print(json.dumps({"leg": "backward", "workload": wb.describe(), "ms_per_step": statistics.median(ms)}))
             return
+        if args.legs == "msr":
+            r = run_msr(inputs.WORKLOADS[2], args.steps, args.warmup, 256 << 20, peaks["hbm_gbs"])
+            if rank == 0:
+                print(json.dumps({"leg": "msr", "workload": inputs.WORKLOADS[2].describe(), **r}))
+            return
         if args.legs == "decode":
             dec = run_decode(wd, args.steps, args.warmup, clocks)
             ms = dist_max(statistics.mean(dec["step_ms"]), world)
@@ -694,6 +764,10 @@ def main():
         rev_ms = None
         if args.legs == "both":
             rev_ms = run_reversed(w, max(3, args.steps // 4), args.warmup, 256 << 20)
+        msr = None
+        if args.legs in ("both", "msr"):
+            msr = (inputs.WORKLOADS[2], run_msr(inputs.WORKLOADS[2], max(3, args.steps // 2), args.warmup, 256 << 20,
+                                                 peaks["hbm_gbs"]))
         sn = []
         if args.legs == "both":
             for idx in (1, 3):
@@ -753,6 +827,14 @@ def main():
                                     "back; the copies move reversal_bytes through HBM on top of the forward",
                             "reversal_bytes": copy_bytes}
         line["gpu_launches"] += len(rev_ms) * (cw["plan"]["kernels"] + (4 if w.retention else 6))
+    if msr:
+        wm, r = msr
+        bms = dist_max(r["block_ms"], world)
+        line["msr_block"] = {"workload": wm.describe(), "value": wm.B * wm.S * world / (bms * 1e-3), "unit": "tokens/s",
+                             "ms_per_step": bms, **{k: v for k, v in r.items() if k != "block_ms"},
+                             "note": "rotation of q and k, the recurrence, GroupNorm + SiLU gate (three kernels "
+                                     "in sequence), against the plain forward (forward_ms) on the same inputs"}
+        line["gpu_launches"] += r["steps"] * (cw["plan"]["kernels"] + 2) + r["steps"] * (cw["plan"]["kernels"] + 2)
     if sn:
         sm_mhz = line["clocks"].get("sm_mhz")
         line["scalar_normaliser"] = []

@@ -260,6 +260,56 @@ mlstm_status_t mlstm_bwd(const mlstm_fwd_params_t* p,
                          void* workspace, size_t workspace_bytes, mlstm_stream_t stream);
 
 /*
+ * The steps either side of retention in a multi-scale retention block
+ * (Edifice.Attention.RetNet, "Key Innovation": Y = (Q Theta) D (K Theta)^T V; "Multi-Scale
+ * Retention (MSR)": GroupNorm over heads, Y = SiLU(X W_G) * GroupNorm(Retention(X))).  The
+ * projections X W_G and W_O are matrix products outside the library.
+ *
+ * mlstm_theta_rotate: q_out = q Theta, k_out = k Theta.  Entries (2j, 2j+1) of each head
+ * vector are one complex number, multiplied by e^{i p theta_j} at sequence position
+ * p = pos0[b] + t, theta_j = theta_base^{-2j/DHQK}; the same rotation on q and k makes the
+ * scores depend on positions only through their difference.
+ *   p            B, NH, S, DHQK, dtype used (the rest ignored but validated as for the
+ *                forward).  DHQK a multiple of 8 (bf16) or 4 (fp32), at most 2048 / 1024.
+ *   q, k         [B,NH,S,DHQK]  dtype   required (if the tensor is not empty)
+ *   pos0         [B]  int64, device, 8-byte aligned: position of token 0 of each sequence
+ *                (a decode step passes the sequence's current length); NULL = 0
+ *   theta_base   > 0 (10000 is the common choice)
+ *   q_out, k_out [B,NH,S,DHQK]  dtype   may equal q / k exactly (in place); no other overlap
+ *
+ * mlstm_group_norm_gate: each (batch, head, token) row of DHV values is one group,
+ * y = (h - mean) / sqrt(var + eps) * weight + bias (biased variance), then y *= silu(g).
+ *   p            B, NH, S, DHV, dtype used.  DHV = 8 x 2^k (bf16) or 4 x 2^k (fp32), k <= 8.
+ *   h, y         [B,NH,S,DHV]  dtype   y may equal h exactly (in place)
+ *   g            [B,NH,S,DHV]  dtype   gate pre-activation X W_G; NULL = no gate
+ *   weight, bias [NH*DHV] fp32 per channel; NULL = 1 / 0
+ *   eps          >= 0
+ *
+ * mlstm_fwd_chunkwise_msr: the block in one call: rotate q and k (into the workspace), run
+ * mlstm_fwd_chunkwise on them (retention or mLSTM per p->retention; no ogate), GroupNorm
+ * and gate h into y (the kernel of mlstm_group_norm_gate, in place on y).  Other
+ * arguments as for mlstm_fwd_chunkwise and the two calls
+ * above; workspace: mlstm_fwd_chunkwise_msr_workspace_size (rotated q and k plus the
+ * forward's).  g, weight, bias, pos0, q and k must not overlap y, the state outputs or the
+ * workspace (MLSTM_ERR_ALIAS).
+ */
+mlstm_status_t mlstm_theta_rotate(const mlstm_fwd_params_t* p, const void* q, const void* k,
+                                  const long long* pos0, float theta_base, void* q_out, void* k_out,
+                                  mlstm_stream_t stream);
+mlstm_status_t mlstm_group_norm_gate(const mlstm_fwd_params_t* p, const void* h, const void* g,
+                                     const float* weight, const float* bias, float eps, void* y,
+                                     mlstm_stream_t stream);
+size_t mlstm_fwd_chunkwise_msr_workspace_size(const mlstm_fwd_params_t* p);
+mlstm_status_t mlstm_fwd_chunkwise_msr(const mlstm_fwd_params_t* p,
+                                       const void* q, const void* k, const void* v,
+                                       const float* igate, const float* fgate,
+                                       const long long* pos0, float theta_base,
+                                       const void* g, const float* gn_weight, const float* gn_bias, float eps,
+                                       const float* C0, const float* n0, const float* m0,
+                                       void* y, float* C_out, float* n_out, float* m_out,
+                                       void* workspace, size_t workspace_bytes, mlstm_stream_t stream);
+
+/*
  * One recurrent decode step for every sequence of the batch, state updated in
  * place (RetNet recurrent_retention_step: O(1) per token; burn-gdn2 Gdn2Mode
  * FusedRecurrent: state [B,H,K,V] carried across tokens and updated in place).

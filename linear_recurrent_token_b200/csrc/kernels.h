@@ -24,6 +24,16 @@ struct WalkArgs {
   float *C_out, *n_out, *m_out;
 };
 
+// The steps either side of retention (msr.cu): the rotation Theta of q and k by position
+// (in place allowed: qo == q, ko == k), and the per-head GroupNorm + SiLU gate (y == h
+// allowed).  *_supported: the head width fits the kernel's vector layout.
+bool theta_rotate_supported(int D, int dtype);
+bool gn_gate_supported(int DHV, int dtype);
+cudaError_t launch_theta_rotate(int B, int NH, int S, int D, int dtype, const void* q, const void* k, void* qo,
+                                void* ko, const long long* pos0, float base, cudaStream_t stream);
+cudaError_t launch_gn_gate(long long rows, int NH, int S, int DHV, int dtype, const void* h, const void* g,
+                           const float* w, const float* b, float eps, void* y, cudaStream_t stream);
+
 cudaError_t launch_gate_prep(int BH, int S, int n_per_head, const float* ig, const float* fg,
                              const float* m0, const float* n0, float* m_tok, float* m_init,
                              float* n_init, cudaStream_t stream);

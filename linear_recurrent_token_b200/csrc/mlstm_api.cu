@@ -101,11 +101,18 @@ bool overlaps(Range a, Range b) {
   return a0 < b0 + b.n && b0 < a0 + a.n;
 }
 
+// GroupNorm + SiLU gate applied to h after the recurrence: one more kernel over h in place
+struct GnArgs {
+  const void* g;
+  const float *w, *b;
+  float eps;
+};
+
 mlstm_status_t fwd_impl(const mlstm_fwd_params_t* p, const void* q, const void* k, const void* v,
                         const float* igate, const float* fgate, const void* ogate, const float* C0,
                         const float* n0, const float* m0, void* h, float* C_out, float* n_out, float* m_out,
                         void* workspace, size_t workspace_bytes, cudaStream_t stream, cudaEvent_t ev0,
-                        cudaEvent_t ev1, bool launch = true) {
+                        cudaEvent_t ev1, bool launch = true, const GnArgs* gn = nullptr) {
   FwdShape s;
   mlstm_status_t st = check_fwd(p, &s);
   if (st != MLSTM_OK) return st;
@@ -209,6 +216,8 @@ mlstm_status_t fwd_impl(const mlstm_fwd_params_t* p, const void* q, const void* 
     }
     if (e != cudaSuccess) return MLSTM_ERR_CUDA;
     e = launch_tc(a, s.tcp, wsb + ws.tc, stream, ev0, ev1);
+    if (e == cudaSuccess && gn)
+      e = launch_gn_gate((long long)s.BH * s.S, s.NH, s.S, s.DHV, s.dtype, h, gn->g, gn->w, gn->b, gn->eps, h, stream);
     return e == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA;
   }
   if (!ret) {
@@ -225,6 +234,44 @@ mlstm_status_t fwd_impl(const mlstm_fwd_params_t* p, const void* q, const void* 
   e = launch_simt_walk(a, stream);
   if (e != cudaSuccess) return MLSTM_ERR_CUDA;
   if (ev1 && cudaEventRecord(ev1, stream) != cudaSuccess) return MLSTM_ERR_CUDA;
+  if (gn && launch_gn_gate((long long)s.BH * s.S, s.NH, s.S, s.DHV, s.dtype, h, gn->g, gn->w, gn->b, gn->eps, h,
+                           stream) != cudaSuccess)
+    return MLSTM_ERR_CUDA;
+  return MLSTM_OK;
+}
+
+// Workspace of the multi-scale retention block: rotated q and k, then the forward's own.
+struct MsrLayout {
+  size_t qr, kr, fwd, total;
+};
+MsrLayout msr_layout(const FwdShape& s) {
+  MsrLayout r = {0, 0, 0, 0};
+  const size_t bq = (size_t)s.BH * s.S * s.DHQK * s.esize;
+  r.qr = 0;
+  r.kr = align_up(bq);
+  r.fwd = r.kr + align_up(bq);
+  r.total = r.fwd + fwd_layout(s).total;
+  return r;
+}
+
+bool finite_nonneg(float x) { return x >= 0.f && x <= 3.4e38f; }
+
+// Sizes of the element-wise entries (rotation, GroupNorm): no recurrence kernel involved, so
+// only the dimensions themselves and the grid limits are checked.
+mlstm_status_t check_dims(const mlstm_fwd_params_t* p, FwdShape* s) {
+  if (!p) return MLSTM_ERR_NULL;
+  if (p->dtype != MLSTM_F32 && p->dtype != MLSTM_BF16) return MLSTM_ERR_DTYPE;
+  if (p->B < 0 || p->NH < 0 || p->S < 0 || p->DHQK < 1 || p->DHV < 1) return MLSTM_ERR_SHAPE;
+  memset(s, 0, sizeof(*s));
+  s->B = p->B;
+  s->NH = p->NH;
+  s->S = p->S;
+  s->DHQK = p->DHQK;
+  s->DHV = p->DHV;
+  s->dtype = p->dtype == MLSTM_BF16 ? 1 : 0;
+  s->esize = p->dtype == MLSTM_BF16 ? 2 : 4;
+  s->BH = (long long)p->B * p->NH;
+  if (s->B > 65535 || (long long)s->S * s->BH > (1LL << 40)) return MLSTM_ERR_SHAPE;
   return MLSTM_OK;
 }
 
@@ -661,6 +708,102 @@ mlstm_status_t mlstm_step(const mlstm_step_params_t* p, const void* q, const voi
   a.m = m;
   a.h = h;
   return launch_step(a, (cudaStream_t)stream) == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA;
+}
+
+
+mlstm_status_t mlstm_theta_rotate(const mlstm_fwd_params_t* p, const void* q, const void* k, const long long* pos0,
+                                  float theta_base, void* q_out, void* k_out, cudaStream_t stream) {
+  FwdShape s;
+  mlstm_status_t st = check_dims(p, &s);
+  if (st != MLSTM_OK) return st;
+  if (!theta_rotate_supported(s.DHQK, s.dtype) || !(theta_base > 0.f) || !finite_nonneg(theta_base))
+    return MLSTM_ERR_SHAPE;
+  const size_t bq = (size_t)s.BH * s.S * s.DHQK * s.esize;
+  if (bq == 0) return MLSTM_OK;
+  if (!q || !k || !q_out || !k_out) return MLSTM_ERR_NULL;
+  const void* all[] = {q, k, q_out, k_out, pos0};
+  for (const void* ptr : all)
+    if (ptr && ((uintptr_t)ptr & (ptr == pos0 ? 7 : 15))) return MLSTM_ERR_ALIGN;
+  const Range rq{q, bq}, rk{k, bq}, oq{q_out, bq}, ok{k_out, bq}, rp{pos0, (size_t)s.B * 8};
+  // in place only exactly (q_out == q, k_out == k); no other overlap
+  if ((overlaps(oq, rq) && q_out != q) || overlaps(oq, rk) || overlaps(ok, rq) || (overlaps(ok, rk) && k_out != k) ||
+      overlaps(oq, ok) || overlaps(oq, rp) || overlaps(ok, rp))
+    return MLSTM_ERR_ALIAS;
+  return launch_theta_rotate(s.B, s.NH, s.S, s.DHQK, s.dtype, q, k, q_out, k_out, pos0, theta_base,
+                             (cudaStream_t)stream) == cudaSuccess
+             ? MLSTM_OK
+             : MLSTM_ERR_CUDA;
+}
+
+mlstm_status_t mlstm_group_norm_gate(const mlstm_fwd_params_t* p, const void* h, const void* g, const float* weight,
+                                     const float* bias, float eps, void* y, cudaStream_t stream) {
+  FwdShape s;
+  mlstm_status_t st = check_dims(p, &s);
+  if (st != MLSTM_OK) return st;
+  if (!gn_gate_supported(s.DHV, s.dtype) || !finite_nonneg(eps)) return MLSTM_ERR_SHAPE;
+  const size_t bv = (size_t)s.BH * s.S * s.DHV * s.esize, bw = (size_t)s.NH * s.DHV * sizeof(float);
+  if (bv == 0) return MLSTM_OK;
+  if (!h || !y) return MLSTM_ERR_NULL;
+  const void* all[] = {h, g, weight, bias, y};
+  for (const void* ptr : all)
+    if (ptr && misaligned(ptr)) return MLSTM_ERR_ALIGN;
+  const Range rh{h, bv}, ry{y, bv}, rg{g, bv}, rw{weight, bw}, rb{bias, bw};
+  if ((overlaps(ry, rh) && y != h) || overlaps(ry, rg) || overlaps(ry, rw) || overlaps(ry, rb)) return MLSTM_ERR_ALIAS;
+  return launch_gn_gate((long long)s.BH * s.S, s.NH, s.S, s.DHV, s.dtype, h, g, weight, bias, eps, y,
+                        (cudaStream_t)stream) == cudaSuccess
+             ? MLSTM_OK
+             : MLSTM_ERR_CUDA;
+}
+
+size_t mlstm_fwd_chunkwise_msr_workspace_size(const mlstm_fwd_params_t* p) {
+  FwdShape s;
+  if (check_fwd(p, &s) != MLSTM_OK) return 0;
+  return msr_layout(s).total;
+}
+
+mlstm_status_t mlstm_fwd_chunkwise_msr(const mlstm_fwd_params_t* p, const void* q, const void* k, const void* v,
+                                       const float* igate, const float* fgate, const long long* pos0,
+                                       float theta_base, const void* g, const float* gn_weight,
+                                       const float* gn_bias, float eps, const float* C0, const float* n0,
+                                       const float* m0, void* y, float* C_out, float* n_out, float* m_out,
+                                       void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  FwdShape s;
+  mlstm_status_t st = check_fwd(p, &s);
+  if (st != MLSTM_OK) return st;
+  if (!theta_rotate_supported(s.DHQK, s.dtype) || !gn_gate_supported(s.DHV, s.dtype) || !(theta_base > 0.f) ||
+      !finite_nonneg(theta_base) || !finite_nonneg(eps))
+    return MLSTM_ERR_SHAPE;
+  const MsrLayout r = msr_layout(s);
+  const size_t tok = (size_t)s.BH * s.S;
+  const size_t bq = tok * s.DHQK * s.esize, bv = tok * s.DHV * s.esize, bw = (size_t)s.NH * s.DHV * sizeof(float);
+  if (tok > 0 && (!q || !k)) return MLSTM_ERR_NULL;
+  const void* extra[] = {g, gn_weight, gn_bias, workspace};
+  for (const void* ptr : extra)
+    if (ptr && misaligned(ptr)) return MLSTM_ERR_ALIGN;
+  if (pos0 && ((uintptr_t)pos0 & 7)) return MLSTM_ERR_ALIGN;
+  // the block's own inputs must not overlap what the forward writes (y, state, workspace)
+  const size_t bC = (size_t)s.BH * s.nb * s.dv * s.dk * sizeof(float);
+  const size_t bn = s.retention ? 0 : (size_t)s.BH * s.nb * s.dk * sizeof(float), bm = s.retention ? 0 : (size_t)s.BH * 4;
+  const Range outs[] = {{y, bv}, {C_out, bC}, {n_out, bn}, {m_out, bm}, {workspace, r.total}};
+  const Range ins[] = {{g, bv}, {gn_weight, bw}, {gn_bias, bw}, {pos0, (size_t)s.B * 8}, {q, bq}, {k, bq}};
+  for (const Range& o : outs)
+    for (const Range& i : ins)
+      if (overlaps(o, i)) return MLSTM_ERR_ALIAS;
+  if (r.total > 0 && (!workspace || workspace_bytes < r.total)) return MLSTM_ERR_WORKSPACE;
+  char* w = static_cast<char*>(workspace);
+  void* qr = tok ? w + r.qr : nullptr;
+  void* kr = tok ? w + r.kr : nullptr;
+  // validate the forward (with the rotated copies as its q, k) before launching anything
+  const GnArgs gn{g, gn_weight, gn_bias, eps};
+  st = fwd_impl(p, qr, kr, v, igate, fgate, nullptr, C0, n0, m0, y, C_out, n_out, m_out, w ? w + r.fwd : nullptr,
+                workspace_bytes > r.fwd ? workspace_bytes - r.fwd : 0, (cudaStream_t)stream, nullptr, nullptr, false,
+                &gn);
+  if (st != MLSTM_OK || s.BH == 0) return st;
+  if (s.S > 0 && launch_theta_rotate(s.B, s.NH, s.S, s.DHQK, s.dtype, q, k, qr, kr, pos0, theta_base,
+                                     (cudaStream_t)stream) != cudaSuccess)
+    return MLSTM_ERR_CUDA;
+  return fwd_impl(p, qr, kr, v, igate, fgate, nullptr, C0, n0, m0, y, C_out, n_out, m_out, w + r.fwd,
+                  workspace_bytes - r.fwd, (cudaStream_t)stream, nullptr, nullptr, true, &gn);
 }
 
 }  // extern "C"

@@ -74,6 +74,16 @@ def lib():
         L.mlstm_fwd_chunkwise_scalar_normaliser_workspace_size.restype = Z
         L.mlstm_fwd_chunkwise_scalar_normaliser.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 15 + [Z, P]
         L.mlstm_fwd_chunkwise_scalar_normaliser.restype = I
+        F = ctypes.c_float
+        L.mlstm_theta_rotate.argtypes = [ctypes.POINTER(FwdParams), P, P, P, F, P, P, P]
+        L.mlstm_theta_rotate.restype = I
+        L.mlstm_group_norm_gate.argtypes = [ctypes.POINTER(FwdParams), P, P, P, P, F, P, P]
+        L.mlstm_group_norm_gate.restype = I
+        L.mlstm_fwd_chunkwise_msr_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
+        L.mlstm_fwd_chunkwise_msr_workspace_size.restype = Z
+        L.mlstm_fwd_chunkwise_msr.argtypes = [ctypes.POINTER(FwdParams), P, P, P, P, P, P, F, P, P, P, F, P, P, P,
+                                              P, P, P, P, P, Z, P]
+        L.mlstm_fwd_chunkwise_msr.restype = I
         L.mlstm_bwd_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
         L.mlstm_bwd_workspace_size.restype = Z
         L.mlstm_bwd.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 22 + [Z, P]
@@ -212,6 +222,66 @@ def fwd_chunkwise_scalar_normaliser(q, k, v, igate, fgate, bias, ogate=None, C0=
     if st != 0:
         raise MlstmError(st, "mlstm_fwd_chunkwise_scalar_normaliser")
     return h, C_out, n_out, m_out
+
+
+def theta_rotate(q, k, pos0=None, theta_base: float = 10000.0, *, q_out=None, k_out=None, stream=None):
+    """The rotation Theta of q and k by position (mlstm_theta_rotate): q, k [B,NH,S,DHQK];
+    pos0 [B] int64 (position of token 0 of each sequence) or None.  q_out / k_out may be q / k
+    (in place).  Returns (q_out, k_out)."""
+    B, NH, S, DHQK = q.shape
+    p = fwd_params(B, NH, S, DHQK, DHQK, 64, 1, q.dtype, True)
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    st = lib().mlstm_theta_rotate(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(pos0), ctypes.c_float(theta_base),
+                                  _ptr(q_out), _ptr(k_out), _stream_ptr(stream))
+    if st != 0:
+        raise MlstmError(st, "mlstm_theta_rotate")
+    return q_out, k_out
+
+
+def group_norm_gate(h, g=None, weight=None, bias=None, eps: float = 1e-5, *, y=None, stream=None):
+    """Per-head GroupNorm of h [B,NH,S,DHV] and the SiLU gate g (mlstm_group_norm_gate);
+    weight, bias [NH*DHV] fp32 or None.  y may be h (in place).  Returns y."""
+    B, NH, S, DHV = h.shape
+    p = fwd_params(B, NH, S, DHV, DHV, 64, 1, h.dtype, True)
+    y = torch.empty_like(h) if y is None else y
+    st = lib().mlstm_group_norm_gate(ctypes.byref(p), _ptr(h), _ptr(g), _ptr(weight), _ptr(bias),
+                                     ctypes.c_float(eps), _ptr(y), _stream_ptr(stream))
+    if st != 0:
+        raise MlstmError(st, "mlstm_group_norm_gate")
+    return y
+
+
+def msr_workspace_size(params: FwdParams) -> int:
+    return int(lib().mlstm_fwd_chunkwise_msr_workspace_size(ctypes.byref(params)))
+
+
+def fwd_chunkwise_msr(q, k, v, igate=None, fgate=None, g=None, gn_weight=None, gn_bias=None, C0=None, n0=None,
+                      m0=None, *, pos0=None, theta_base: float = 10000.0, eps: float = 1e-5, chunk: int = 64,
+                      num_blocks: int = 1, retention: bool = True, y=None, workspace=None, stream=None):
+    """The multi-scale retention block in one call (mlstm_fwd_chunkwise_msr): rotate q, k,
+    the recurrence, GroupNorm and the SiLU gate.  Returns (y, C, n, m); n, m None in
+    retention mode."""
+    B, NH, S, DHQK = q.shape
+    DHV = v.shape[-1]
+    nb = int(num_blocks)
+    p = fwd_params(B, NH, S, DHQK, DHV, chunk, nb, q.dtype, retention)
+    dev = q.device
+    y = torch.empty((B, NH, S, DHV), dtype=q.dtype, device=dev) if y is None else y
+    C_out = torch.empty((B, NH, nb, DHV // nb, DHQK // nb), dtype=torch.float32, device=dev)
+    n_out = None if retention else torch.empty((B, NH, nb, DHQK // nb), dtype=torch.float32, device=dev)
+    m_out = None if retention else torch.empty((B, NH), dtype=torch.float32, device=dev)
+    ws_bytes = msr_workspace_size(p)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().mlstm_fwd_chunkwise_msr(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(igate), _ptr(fgate), _ptr(pos0), ctypes.c_float(theta_base),
+        _ptr(g), _ptr(gn_weight), _ptr(gn_bias), ctypes.c_float(eps), _ptr(C0), _ptr(n0), _ptr(m0), _ptr(y),
+        _ptr(C_out), _ptr(n_out), _ptr(m_out), _ptr(workspace), ctypes.c_size_t(ws_len), _stream_ptr(stream))
+    if st != 0:
+        raise MlstmError(st, "mlstm_fwd_chunkwise_msr")
+    return y, C_out, n_out, m_out
 
 
 def reversed_workspace_size(params: FwdParams) -> int:

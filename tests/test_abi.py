@@ -210,3 +210,59 @@ def test_scalar_normaliser_validation():
     assert sn_call(p, C=0xE000000, C0=0xE000000, ws_bytes=16) == 5
     need = mlstm.lib().mlstm_fwd_chunkwise_scalar_normaliser_workspace_size(ctypes.byref(p))
     assert need > 0 and sn_call(p, ws_bytes=need - 1) == 5
+
+
+# ---------------------------------------------------------------- multi-scale retention block
+def rot_call(p, q=A, k=B_, pos0=None, base=10000.0, qo=C_, ko=D_):
+    return mlstm.lib().mlstm_theta_rotate(ctypes.byref(p), q, k, pos0, ctypes.c_float(base), qo, ko,
+                                          ctypes.c_void_p(0))
+
+
+def gn_call(p, h=A, g=B_, w=None, b=None, eps=1e-5, y=C_):
+    return mlstm.lib().mlstm_group_norm_gate(ctypes.byref(p), h, g, w, b, ctypes.c_float(eps), y, ctypes.c_void_p(0))
+
+
+def msr_call(p, q=A, k=B_, v=C_, ig=D_, fg=E_, pos0=None, base=10000.0, g=H_, w=None, b=None, eps=1e-5, C0=None,
+             n0=None, m0=None, y=F_, C=None, n=None, m=None, ws=G_, ws_bytes=1 << 40):
+    return mlstm.lib().mlstm_fwd_chunkwise_msr(ctypes.byref(p), q, k, v, ig, fg, pos0, ctypes.c_float(base), g, w, b,
+                                               ctypes.c_float(eps), C0, n0, m0, y, C, n, m, ws,
+                                               ctypes.c_size_t(ws_bytes), ctypes.c_void_p(0))
+
+
+def test_theta_rotate_validation():
+    # every call here fails validation: none reaches a launch
+    p = params()
+    assert rot_call(params(DHQK=18)) == 2                   # not a whole number of 16-byte vectors
+    assert rot_call(params(DHQK=12, dtype=torch.bfloat16)) == 2   # 12 bf16 = 1.5 vectors
+    assert rot_call(p, base=0.0) == 2 and rot_call(p, base=float("nan")) == 2
+    assert rot_call(p, q=None) == 1 and rot_call(p, ko=None) == 1
+    assert rot_call(p, q=A + 4) == 4 and rot_call(p, pos0=E_ + 4) == 4
+    assert rot_call(p, qo=A + 16) == 7                      # overlaps q without being q
+    assert rot_call(p, qo=B_) == 7 and rot_call(p, ko=C_) == 7
+    assert rot_call(p, pos0=C_) == 7                        # positions under an output
+
+
+def test_group_norm_gate_validation():
+    p = params()
+    assert gn_call(params(DHV=24)) == 2                     # 6 vectors per row: not a power of two
+    assert gn_call(p, eps=-1.0) == 2
+    assert gn_call(p, h=None) == 1 and gn_call(p, y=None) == 1
+    assert gn_call(p, w=E_ + 8) == 4
+    assert gn_call(p, y=B_) == 7 and gn_call(p, y=A + 16) == 7
+    assert gn_call(p, w=C_ + 16) == 7                       # weights under y
+
+
+def test_msr_block_validation_and_workspace():
+    p = params(retention=True)
+    need = mlstm.msr_workspace_size(p)
+    tok = 2 * 2 * 64
+    assert need >= mlstm.workspace_size(p) + 2 * tok * 16 * 4
+    assert msr_call(p, ws_bytes=need - 1) == 5
+    assert msr_call(params(DHQK=18, retention=True)) == 2
+    assert msr_call(params(DHV=24, retention=True)) == 2
+    assert msr_call(p, q=None) == 1
+    assert msr_call(p, g=F_) == 7                           # gate under y
+    assert msr_call(p, ws=A) == 7                           # workspace under q
+    assert msr_call(p, pos0=G_ + 8) == 7                    # positions inside the workspace
+    assert msr_call(p, g=H_ + 4) == 4
+    assert msr_call(params(), ig=None, ws_bytes=16) == 5  # mLSTM mode: workspace checked first
