@@ -23,6 +23,8 @@ Contents
 ``theta_rotate``, ``group_norm_gate``, ``retention_block``  numpy, fp64, the steps
                      either side of retention (Edifice.Attention.RetNet): the rotation of
                      q and k, the per-head GroupNorm and the SiLU gate, and their composition.
+``gdn2_sequential``, ``gdn2_chunk``  numpy, fp64, Gated DeltaNet-2 (burn-gdn2): the
+                     token-by-token recurrence and its chunked (triangular-solve) evaluation.
 ``sequential_backward``  numpy, fp64, gradients of ``sequential`` by reverse-mode
                      differentiation of its steps in reverse order (backpropagation
                      through time); pinned by central finite differences.
@@ -549,6 +551,81 @@ def retention_block(q, k, v, igate=None, fgate=None, g=None, gn_weight=None, gn_
     if rounding is not None:
         h = rounding(h)
     return group_norm_gate(h, g, gn_weight, gn_bias, eps), C, n, m
+
+
+def gdn2_sequential(q, k, v, g, b, w, S0=None):
+    """Gated DeltaNet-2 (burn-gdn2 config.rs: channel-wise erase gate b in [0,1]^{d_k}, write
+    gate w in [0,1]^{d_v}, state S [B,H,K,V] carried token by token), fp64, one token at a time.
+    The page gives the gates' roles and the reductions (b = w = beta 1 is KDA; a scalar decay
+    on top is Gated DeltaNet), not the update itself; the reading built here is the KDA step
+    with its erase and write strengths split by channel:
+
+        S'_t = Diag(alpha_t) S_{t-1}                 (alpha_t = exp(g_t), per key channel)
+        r_t  = S'_t^T k_t                            (the value stored under k_t)
+        S_t  = S'_t - (b_t o k_t) r_t^T + k_t (w_t o v_t)^T
+        o_t  = S_t^T q_t
+
+    q, k, g, b: [B,H,T,K] (g = log alpha <= 0); v, w: [B,H,T,V]; S0: [B,H,K,V] or None.
+    Returns (o [B,H,T,V], S_T [B,H,K,V]).
+    """
+    q, k, v, g, b, w = (np.asarray(x, dtype=np.float64) for x in (q, k, v, g, b, w))
+    B, H, T, K = q.shape
+    V = v.shape[-1]
+    S = np.zeros((B, H, K, V)) if S0 is None else np.array(S0, dtype=np.float64)
+    o = np.zeros((B, H, T, V))
+    for t in range(T):
+        Sd = np.exp(g[:, :, t])[..., None] * S
+        r = np.einsum("bhkv,bhk->bhv", Sd, k[:, :, t])
+        S = Sd - np.einsum("bhk,bhv->bhkv", b[:, :, t] * k[:, :, t], r) \
+            + np.einsum("bhk,bhv->bhkv", k[:, :, t], w[:, :, t] * v[:, :, t])
+        o[:, :, t] = np.einsum("bhkv,bhk->bhv", S, q[:, :, t])
+    return o, S
+
+
+def gdn2_chunk(q, k, v, g, b, w, S0=None, chunk: int = 64):
+    """The chunked evaluation of ``gdn2_sequential`` (burn-gdn2 Gdn2Mode::Chunk: intra-chunk
+    interactions as dense products with a WY-like triangular solve, the state carried between
+    chunks), fp64, written from this derivation.  Inside a chunk with cumulative log decay
+    G_t = sum_{s<=t} g_s (per key channel) and carried state S0:
+
+        r_t = (k_t o e^{G_t})^T S0 + sum_{s<t} [sum_i k_ti k_si e^{G_ti-G_si}] u_s
+                                   - sum_{s<t} [sum_i k_ti bk_si e^{G_ti-G_si}] r_s
+        (u = w o v, bk = b o k), i.e. (I + L_E) R = C S0 + L_A U with strictly lower
+        triangular L_A, L_E: R comes from one unit-lower-triangular solve;
+        o_t = (q_t o e^{G_t})^T S0 + sum_{s<=t} [q.k weights] u_s - sum_{s<=t} [q.bk weights] r_s
+        S_L = e^{G_L} o S0 + sum_s (e^{G_L - G_s} o k_s) u_s^T - sum_s (e^{G_L - G_s} o bk_s) r_s^T
+
+    Every exponent above is <= 0.  Returns (o, S_T) like ``gdn2_sequential``.
+    """
+    q, k, v, g, b, w = (np.asarray(x, dtype=np.float64) for x in (q, k, v, g, b, w))
+    B, H, T, K = q.shape
+    V = v.shape[-1]
+    S = np.zeros((B, H, K, V)) if S0 is None else np.array(S0, dtype=np.float64)
+    o = np.zeros((B, H, T, V))
+    for bb in range(B):
+        for hh in range(H):
+            St = S[bb, hh].copy()
+            for c0 in range(0, T, chunk):
+                sl = slice(c0, min(T, c0 + chunk))
+                qc, kc, gc = q[bb, hh, sl], k[bb, hh, sl], g[bb, hh, sl]
+                u = w[bb, hh, sl] * v[bb, hh, sl]
+                bk = b[bb, hh, sl] * kc
+                G = np.cumsum(gc, axis=0)                        # [L, K]
+                Lc = G.shape[0]
+                dec = np.exp(np.minimum(G[:, None, :] - G[None, :, :], 0.0))  # [t, s, K]; s <= t used
+                low = np.tril(np.ones((Lc, Lc)), -1)
+                incl = np.tril(np.ones((Lc, Lc)))
+                LA = np.einsum("ti,si,tsi->ts", kc, kc, np.where(low[..., None] > 0, dec, 0.0))
+                LE = np.einsum("ti,si,tsi->ts", kc, bk, np.where(low[..., None] > 0, dec, 0.0))
+                rhs = (kc * np.exp(G)) @ St + LA @ u
+                R = np.linalg.solve(np.eye(Lc) + LE, rhs)
+                QA = np.einsum("ti,si,tsi->ts", qc, kc, np.where(incl[..., None] > 0, dec, 0.0))
+                QE = np.einsum("ti,si,tsi->ts", qc, bk, np.where(incl[..., None] > 0, dec, 0.0))
+                o[bb, hh, sl] = (qc * np.exp(G)) @ St + QA @ u - QE @ R
+                tail = np.exp(G[-1][None, :] - G)                # [L, K]
+                St = np.exp(G[-1])[:, None] * St + (tail * kc).T @ u - (tail * bk).T @ R
+            S[bb, hh] = St
+    return o, S
 
 
 def state_bytes(layers: int, heads: int, dqk: int, dv: int, bytes_per_value: int) -> int:
