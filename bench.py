@@ -645,6 +645,74 @@ def run_msr(w, steps, warmup, flush_bytes, hbm_peak):
                                      "kernel": "gn_gate_kernel (standalone; v as h)"}}}
 
 
+def gdn2_flops(B, H, T, K, V):
+    """Algorithmic flops of the GDN-2 recurrence: per token and head the decay (K V), the
+    read-out r = S'^T k (2 K V), the erase and write (4 K V) and o = S^T q (2 K V)."""
+    return B * H * T * 9 * K * V
+
+
+def run_gdn2(steps, warmup, flush_bytes, peaks, sm_mhz):
+    """Gated DeltaNet-2: the prefill workload in both modes (fused recurrent, chunk) and the
+    decode workload (one token per sequence, state in place), inputs resident, L2 flushed
+    between steps.  Returns the dict for the JSON line."""
+    import torch
+
+    from linear_recurrent_token_b200 import inputs, mlstm
+    out = {}
+    flush = torch.empty(flush_bytes // 4, dtype=torch.float32, device="cuda")
+
+    def timed(call):
+        for _ in range(warmup):
+            call()
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(steps):
+            flush.fill_(1.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            call()
+            b.record()
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        return statistics.median(ms)
+
+    for wl in inputs.GDN2_WORKLOADS:
+        td = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+        inp = inputs.gdn2_inputs(wl.B, wl.H, wl.T, wl.K, wl.V, wl.dtype, seed=7)
+        d = lambda x, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(x)).to("cuda", dt)
+        q, k, v = d(inp["q"], td), d(inp["k"], td), d(inp["v"], td)
+        g, b, w, S0 = d(inp["g"]), d(inp["b"]), d(inp["w"]), d(inp["S0"])
+        o = torch.empty((wl.B, wl.H, wl.T, wl.V), dtype=td, device="cuda")
+        esz = 2 if wl.dtype == "bf16" else 4
+        flops = gdn2_flops(wl.B, wl.H, wl.T, wl.K, wl.V)
+        fp32_peak = fp32_simt_peak_tflops(sm_mhz)
+        if wl.T > 1:
+            S_out = torch.empty_like(S0)
+            modes = {}
+            for mode in ("recurrent", "chunk"):
+                ms = timed(lambda: mlstm.gdn2_fwd(q, k, v, g, b, w, S0, mode=mode, chunk=wl.chunk, o=o, S_out=S_out))
+                tf = flops / (ms * 1e-3) / 1e12
+                modes[mode] = {"value": wl.B * wl.T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+                               "roofline": {"bound": "alu", "achieved": tf, "peak": fp32_peak, "unit": "TFLOP/s",
+                                            "frac": tf / fp32_peak, "traffic": None,
+                                            "kernel": "gdn2_%s_kernel (fp32 SIMT)" % mode, "flops_per_launch": flops,
+                                            "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x median SM clock"}}
+            out[wl.name] = {"workload": wl.describe(), **modes}
+        else:
+            S = S0.clone()
+            ms = timed(lambda: mlstm.gdn2_fwd(q, k, v, g, b, w, S, o=o, S_out=S))
+            nbytes = 2 * wl.B * wl.H * wl.K * wl.V * 4 + wl.B * wl.H * (2 * wl.K * esz + 2 * wl.K * 4 + wl.V * (2 * esz + 4))
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            out[wl.name] = {"workload": wl.describe(), "value": gbs, "unit": "GB/s", "ms_per_step": ms,
+                            "tokens_per_s": wl.B / (ms * 1e-3),
+                            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                         "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                                         "kernel": "gdn2_recurrent_kernel (T = 1, state in place)",
+                                         "bytes_per_launch": nbytes}}
+    out["steps"] = steps
+    return out
+
+
 def backward_line(w, ms, sm_mhz, cpu: bool):
     step_ms = statistics.median(ms)
     flops = backward_flops(w.B, w.NH, w.S, w.dk, w.dv, w.num_blocks)
@@ -677,7 +745,7 @@ def main():
     ap.add_argument("--workload", type=int, default=3, help="chunkwise workload index (default 3)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
-    ap.add_argument("--legs", choices=["both", "chunkwise", "decode", "backward", "msr"], default="both",
+    ap.add_argument("--legs", choices=["both", "chunkwise", "decode", "backward", "msr", "gdn2"], default="both",
                     help="run only one leg (for profiling); the default runs both")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -728,6 +796,11 @@ def main():
                 if rank == 0:
                     print(json.dumps({"leg": "backward", "workload": wb.describe(), "ms_per_step": statistics.median(ms)}))
             return
+        if args.legs == "gdn2":
+            r = run_gdn2(args.steps, args.warmup, 256 << 20, peaks, clocks.summary().get("sm_mhz"))
+            if rank == 0:
+                print(json.dumps({"leg": "gdn2", **r}))
+            return
         if args.legs == "msr":
             r = run_msr(inputs.WORKLOADS[2], args.steps, args.warmup, 256 << 20, peaks["hbm_gbs"])
             if rank == 0:
@@ -764,6 +837,9 @@ def main():
         rev_ms = None
         if args.legs == "both":
             rev_ms = run_reversed(w, max(3, args.steps // 4), args.warmup, 256 << 20)
+        gdn2 = None
+        if args.legs == "both":
+            gdn2 = run_gdn2(max(3, args.steps // 4), args.warmup, 256 << 20, peaks, None)
         msr = None
         if args.legs in ("both", "msr"):
             msr = (inputs.WORKLOADS[2], run_msr(inputs.WORKLOADS[2], max(3, args.steps // 2), args.warmup, 256 << 20,
@@ -827,6 +903,15 @@ def main():
                                     "back; the copies move reversal_bytes through HBM on top of the forward",
                             "reversal_bytes": copy_bytes}
         line["gpu_launches"] += len(rev_ms) * (cw["plan"]["kernels"] + (4 if w.retention else 6))
+    if gdn2:
+        for val in gdn2.values():  # the fp32 peak at the clock seen during the run
+            for mode in ("recurrent", "chunk"):
+                if isinstance(val, dict) and mode in val:
+                    r = val[mode]["roofline"]
+                    r["peak"] = fp32_simt_peak_tflops(line["clocks"].get("sm_mhz"))
+                    r["frac"] = r["achieved"] / r["peak"]
+        line["gdn2"] = gdn2
+        line["gpu_launches"] += gdn2["steps"] * 3
     if msr:
         wm, r = msr
         bms = dist_max(r["block_ms"], world)

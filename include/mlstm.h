@@ -310,6 +310,44 @@ mlstm_status_t mlstm_fwd_chunkwise_msr(const mlstm_fwd_params_t* p,
                                        void* workspace, size_t workspace_bytes, mlstm_stream_t stream);
 
 /*
+ * Gated DeltaNet-2 (burn-gdn2 config.rs): the delta rule with a per-key-channel decay and two
+ * channel-wise gates, an erase gate b (how much of each key channel to erase) and a write
+ * gate w (how much of each value channel to write); b = w = beta 1 is KDA, and a scalar decay
+ * on top is Gated DeltaNet.  Per (batch, head), state S [K, V] fp32, for each token t:
+ *     S' = Diag(exp(g_t)) S;   r = S'^T k_t;   S = S' - (b_t o k_t) r^T + k_t (w_t o v_t)^T;
+ *     o_t = S^T q_t
+ * (the page names the gates and modes but prints no update; this is the KDA step with its
+ * erase and write strengths split by channel).  Projections, the short convolution, key
+ * normalisation and the output norm are outside the library.
+ *
+ *   p->mode   MLSTM_GDN2_RECURRENT: token by token, the state on chip for the whole sequence
+ *             (Gdn2Mode::FusedRecurrent; with T = 1 and S_out == S0 it is the decode step);
+ *             K in {32, 64, 128, 256}.
+ *             MLSTM_GDN2_CHUNK: chunks of p->chunk tokens (a multiple of 4, at most 64), dense
+ *             products and one triangular solve per chunk (Gdn2Mode::Chunk); needs g <= 0.
+ *             Unsupported sizes: MLSTM_ERR_SHAPE.
+ *   q, k      [B,H,T,K]  dtype       required (if T > 0); k usually unit-norm (caller's choice)
+ *   v         [B,H,T,V]  dtype       required
+ *   g         [B,H,T,K]  fp32        log decay (log alpha), <= 0 for a decay
+ *   b         [B,H,T,K]  fp32        erase gate (in [0,1], or [0,2] with negative eigenvalues)
+ *   w         [B,H,T,V]  fp32        write gate in [0,1]
+ *   S0        [B,H,K,V]  fp32        initial state; NULL = zeros
+ *   o         [B,H,T,V]  dtype       output, required (if T > 0)
+ *   S_out     [B,H,K,V]  fp32        final state; NULL = not written; may equal S0 exactly
+ * No workspace.  Outputs must not overlap the inputs or each other (MLSTM_ERR_ALIAS).
+ */
+typedef enum { MLSTM_GDN2_RECURRENT = 0, MLSTM_GDN2_CHUNK = 1 } mlstm_gdn2_mode_t;
+typedef struct {
+  int B, H, T, K, V;
+  mlstm_dtype_t dtype;
+  int mode;  /* mlstm_gdn2_mode_t */
+  int chunk; /* chunk mode only */
+} mlstm_gdn2_params_t;
+mlstm_status_t mlstm_gdn2_fwd(const mlstm_gdn2_params_t* p, const void* q, const void* k, const void* v,
+                              const float* g, const float* b, const float* w, const float* S0, void* o,
+                              float* S_out, mlstm_stream_t stream);
+
+/*
  * One recurrent decode step for every sequence of the batch, state updated in
  * place (RetNet recurrent_retention_step: O(1) per token; burn-gdn2 Gdn2Mode
  * FusedRecurrent: state [B,H,K,V] carried across tokens and updated in place).

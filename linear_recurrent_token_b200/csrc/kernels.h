@@ -34,6 +34,24 @@ cudaError_t launch_theta_rotate(int B, int NH, int S, int D, int dtype, const vo
 cudaError_t launch_gn_gate(long long rows, int NH, int S, int DHV, int dtype, const void* h, const void* g,
                            const float* w, const float* b, float eps, void* y, cudaStream_t stream);
 
+// Gated DeltaNet-2 (gdn2.cu).  q, k [B,H,T,K], v [B,H,T,V] (dtype 0 fp32, 1 bf16); g (log
+// decay), b (erase gate) [B,H,T,K] and w (write gate) [B,H,T,V] fp32; S0, S_out [B,H,K,V] fp32
+// (S0 NULL = zeros, S_out NULL = not written, S_out == S0 in place); o [B,H,T,V] dtype.
+struct Gdn2Args {
+  int B, H, T, K, V, dtype;
+  const void *q, *k, *v;
+  const float *g, *b, *w;
+  const float* S0;
+  void* o;
+  float* S_out;
+};
+bool gdn2_recurrent_supported(int K);
+// value-tile width of the chunk kernel for these sizes (0 = unsupported)
+int gdn2_chunk_vtile(int L, int K, int V);
+size_t gdn2_chunk_smem_bytes(int L, int K, int VT);
+// mode 0: fused recurrent (token by token); 1: chunk of `chunk` tokens
+cudaError_t launch_gdn2(const Gdn2Args& a, int mode, int chunk, cudaStream_t stream);
+
 cudaError_t launch_gate_prep(int BH, int S, int n_per_head, const float* ig, const float* fg,
                              const float* m0, const float* n0, float* m_tok, float* m_init,
                              float* n_init, cudaStream_t stream);

@@ -806,6 +806,44 @@ mlstm_status_t mlstm_fwd_chunkwise_msr(const mlstm_fwd_params_t* p, const void* 
                   workspace_bytes - r.fwd, (cudaStream_t)stream, nullptr, nullptr, true, &gn);
 }
 
+
+mlstm_status_t mlstm_gdn2_fwd(const mlstm_gdn2_params_t* p, const void* q, const void* k, const void* v,
+                              const float* g, const float* b, const float* w, const float* S0, void* o,
+                              float* S_out, cudaStream_t stream) {
+  if (!p) return MLSTM_ERR_NULL;
+  if (p->dtype != MLSTM_F32 && p->dtype != MLSTM_BF16) return MLSTM_ERR_DTYPE;
+  if (p->B < 0 || p->H < 0 || p->T < 0 || p->K < 1 || p->V < 1) return MLSTM_ERR_SHAPE;
+  if (p->mode != MLSTM_GDN2_RECURRENT && p->mode != MLSTM_GDN2_CHUNK) return MLSTM_ERR_SHAPE;
+  const long long BH = (long long)p->B * p->H;
+  if (BH > 65535 || (long long)p->T * BH > (1LL << 40)) return MLSTM_ERR_SHAPE;
+  if (p->mode == MLSTM_GDN2_RECURRENT ? !gdn2_recurrent_supported(p->K) : gdn2_chunk_vtile(p->chunk, p->K, p->V) == 0)
+    return MLSTM_ERR_SHAPE;
+  const size_t es = p->dtype == MLSTM_BF16 ? 2 : 4, tok = (size_t)BH * p->T;
+  const size_t bq = tok * p->K * es, bv = tok * p->V * es, bg = tok * p->K * 4, bw = tok * p->V * 4;
+  const size_t bS = (size_t)BH * p->K * p->V * 4;
+  if (tok > 0 && (!q || !k || !v || !g || !b || !w || !o)) return MLSTM_ERR_NULL;
+  const void* all[] = {q, k, v, g, b, w, S0, o, S_out};
+  for (const void* ptr : all)
+    if (ptr && misaligned(ptr)) return MLSTM_ERR_ALIGN;
+  const Range ins[] = {{q, bq}, {k, bq}, {v, bv}, {g, bg}, {b, bg}, {w, bw}};
+  const Range ro{o, bv}, rS{S_out, bS}, r0{S0, bS};
+  for (const Range& i : ins)
+    if (overlaps(ro, i) || overlaps(rS, i)) return MLSTM_ERR_ALIAS;
+  if (overlaps(ro, rS) || overlaps(ro, r0) || (overlaps(rS, r0) && S_out != S0)) return MLSTM_ERR_ALIAS;
+  if (BH == 0) return MLSTM_OK;
+  Gdn2Args a;
+  a.B = p->B, a.H = p->H, a.T = p->T, a.K = p->K, a.V = p->V, a.dtype = p->dtype == MLSTM_BF16 ? 1 : 0;
+  a.q = q, a.k = k, a.v = v, a.g = g, a.b = b, a.w = w, a.S0 = S0, a.o = o, a.S_out = S_out;
+  if (p->T == 0) {  // the final state is the initial state
+    cudaError_t e = cudaSuccess;
+    if (S_out && S_out != S0)
+      e = S0 ? cudaMemcpyAsync(S_out, S0, bS, cudaMemcpyDeviceToDevice, (cudaStream_t)stream)
+             : cudaMemsetAsync(S_out, 0, bS, (cudaStream_t)stream);
+    return e == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA;
+  }
+  return launch_gdn2(a, p->mode, p->chunk, (cudaStream_t)stream) == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA;
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------------

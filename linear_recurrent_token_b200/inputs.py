@@ -128,3 +128,43 @@ def decode_sequence_inputs(w: Workload, steps: int, B: int | None = None):
     """Steps 0..steps-1 stacked along a sequence axis: q [B,NH,steps,DHQK] etc."""
     per = [decode_step_inputs(w, t, B) for t in range(steps)]
     return {key: np.stack([p[key] for p in per], axis=2) for key in per[0]}
+
+
+# Gated DeltaNet-2 workloads (burn-gdn2 config.rs defaults: 16 heads of 128, value head 128,
+# chunk 64): a prefill batch and a decode batch (one token per sequence, state in place).
+@dataclasses.dataclass(frozen=True)
+class Gdn2Workload:
+    name: str
+    B: int
+    H: int
+    T: int
+    K: int
+    V: int
+    chunk: int
+    dtype: str
+
+    def describe(self) -> str:
+        return f"{self.name}: B{self.B} H{self.H} T{self.T} K{self.K} V{self.V} chunk{self.chunk} {self.dtype}"
+
+
+GDN2_WORKLOADS = [
+    Gdn2Workload("gdn2_prefill", 8, 16, 2048, 128, 128, 64, "bf16"),
+    Gdn2Workload("gdn2_decode", 256, 16, 1, 128, 128, 64, "bf16"),
+]
+
+
+def gdn2_inputs(B, H, T, K, V, dtype, seed, with_state=True):
+    """Inputs of a GDN-2 call: q, v ~ N(0,1); k ~ N(0,1) scaled to unit length per token (the
+    usual key normalisation, done by the caller); log decay g = -exp(N(-3, 1)) (alpha near
+    0.95 on average, a few channels much lower); erase and write gates b, w ~ U(0,1); S0 ~
+    N(0, 0.1^2).  Dict of float32 numpy arrays holding the exact stored values."""
+    rng = np.random.default_rng(seed)
+    q = _draw(rng, (B, H, T, K), dtype)
+    kr = rng.standard_normal((B, H, T, K))
+    k = round_to(kr / np.maximum(np.linalg.norm(kr, axis=-1, keepdims=True), 1e-12), dtype)
+    v = _draw(rng, (B, H, T, V), dtype)
+    g = round_to(-np.exp(rng.standard_normal((B, H, T, K)) - 3.0), "f32")
+    b = round_to(rng.uniform(0, 1, (B, H, T, K)), "f32")
+    w = round_to(rng.uniform(0, 1, (B, H, T, V)), "f32")
+    S0 = _draw(rng, (B, H, K, V), "f32", scale=0.1) if with_state else None
+    return dict(q=q, k=k, v=v, g=g, b=b, w=w, S0=S0)

@@ -31,6 +31,14 @@ class StepParams(ctypes.Structure):
                 ("num_blocks", ctypes.c_int), ("dtype", ctypes.c_int), ("retention", ctypes.c_int)]
 
 
+class Gdn2Params(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int), ("K", ctypes.c_int),
+                ("V", ctypes.c_int), ("dtype", ctypes.c_int), ("mode", ctypes.c_int), ("chunk", ctypes.c_int)]
+
+
+GDN2_RECURRENT, GDN2_CHUNK = 0, 1
+
+
 class FwdPlan(ctypes.Structure):
     _fields_ = [("tensor_core", ctypes.c_int), ("segments", ctypes.c_int), ("dv_tile", ctypes.c_int),
                 ("ctas_main", ctypes.c_int), ("kernels", ctypes.c_int), ("workspace_bytes", ctypes.c_size_t)]
@@ -84,6 +92,8 @@ def lib():
         L.mlstm_fwd_chunkwise_msr.argtypes = [ctypes.POINTER(FwdParams), P, P, P, P, P, P, F, P, P, P, F, P, P, P,
                                               P, P, P, P, P, Z, P]
         L.mlstm_fwd_chunkwise_msr.restype = I
+        L.mlstm_gdn2_fwd.argtypes = [ctypes.POINTER(Gdn2Params)] + [P] * 9 + [P]
+        L.mlstm_gdn2_fwd.restype = I
         L.mlstm_bwd_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
         L.mlstm_bwd_workspace_size.restype = Z
         L.mlstm_bwd.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 22 + [Z, P]
@@ -282,6 +292,26 @@ def fwd_chunkwise_msr(q, k, v, igate=None, fgate=None, g=None, gn_weight=None, g
     if st != 0:
         raise MlstmError(st, "mlstm_fwd_chunkwise_msr")
     return y, C_out, n_out, m_out
+
+
+def gdn2_fwd(q, k, v, g, b, w, S0=None, *, mode: str = "recurrent", chunk: int = 64, o=None, S_out=None,
+             return_state: bool = True, stream=None):
+    """Gated DeltaNet-2 (mlstm_gdn2_fwd): q, k [B,H,T,K], v [B,H,T,V] (fp32 or bf16); g, b
+    [B,H,T,K] and w [B,H,T,V] fp32; S0 [B,H,K,V] fp32 or None.  mode "recurrent" or "chunk".
+    S_out may be S0 (in place: the decode step).  Returns (o, S_out)."""
+    B, H, T, K = q.shape
+    V = v.shape[-1]
+    p = Gdn2Params(int(B), int(H), int(T), int(K), int(V), _dtype_code(q),
+                   GDN2_CHUNK if mode == "chunk" else GDN2_RECURRENT, int(chunk))
+    if o is None:
+        o = torch.empty((B, H, T, V), dtype=q.dtype, device=q.device)
+    if return_state and S_out is None:
+        S_out = torch.empty((B, H, K, V), dtype=torch.float32, device=q.device)
+    st = lib().mlstm_gdn2_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0),
+                              _ptr(o), _ptr(S_out), _stream_ptr(stream))
+    if st != 0:
+        raise MlstmError(st, "mlstm_gdn2_fwd")
+    return o, S_out
 
 
 def reversed_workspace_size(params: FwdParams) -> int:

@@ -266,3 +266,24 @@ def test_msr_block_validation_and_workspace():
     assert msr_call(p, pos0=G_ + 8) == 7                    # positions inside the workspace
     assert msr_call(p, g=H_ + 4) == 4
     assert msr_call(params(), ig=None, ws_bytes=16) == 5  # mLSTM mode: workspace checked first
+
+
+# ---------------------------------------------------------------- Gated DeltaNet-2
+def gdn2_call(B=2, H=2, T=16, K=64, V=64, dtype=0, mode=0, chunk=16, q=A, k=B_, v=C_, g=D_, b=E_, w=F_, S0=None,
+              o=G_, S=None):
+    p = mlstm.Gdn2Params(B, H, T, K, V, dtype, mode, chunk)
+    return mlstm.lib().mlstm_gdn2_fwd(ctypes.byref(p), q, k, v, g, b, w, S0, o, S, ctypes.c_void_p(0))
+
+
+def test_gdn2_validation():
+    # every call here fails validation: none reaches a launch
+    assert gdn2_call(K=48) == 2                     # recurrent: K in {32, 64, 128, 256}
+    assert gdn2_call(mode=1, chunk=66) == 2         # chunk length over 64
+    assert gdn2_call(mode=1, chunk=6) == 2          # not a multiple of 4
+    assert gdn2_call(mode=2) == 2 and gdn2_call(dtype=5) == 3 and gdn2_call(T=-1) == 2
+    assert gdn2_call(q=None) == 1 and gdn2_call(w=None) == 1 and gdn2_call(o=None) == 1
+    assert gdn2_call(g=D_ + 4) == 4
+    assert gdn2_call(o=A) == 7                      # o on top of q
+    assert gdn2_call(S=G_ + 64) == 7                # state inside o
+    assert gdn2_call(S0=H_, S=H_ + 16) == 7         # state overlapping the initial state, not equal
+    assert gdn2_call(S0=G_, S=None) == 7            # initial state under o
