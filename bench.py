@@ -707,7 +707,7 @@ def run_gdn2(steps, warmup, flush_bytes, peaks, sm_mhz):
                             "tokens_per_s": wl.B / (ms * 1e-3),
                             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                          "frac": gbs / peaks["hbm_gbs"], "traffic": None,
-                                         "kernel": "gdn2_recurrent_kernel (T = 1, state in place)",
+                                         "kernel": "gdn2_step_kernel (T = 1, state in place)",
                                          "bytes_per_launch": nbytes}}
     out["steps"] = steps
     return out

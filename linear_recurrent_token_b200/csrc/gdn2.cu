@@ -8,7 +8,7 @@
 //   for the whole sequence; lane l holds key rows l, l+32, ... of those columns in registers,
 //   so the two reductions over K per token (r and o) are warp shuffles and the state never
 //   leaves the chip between tokens.  With T = 1 and the state in place this is the decode step
-//   (one HBM read and write of S).
+//   (one HBM read and write of S); gdn2_step_kernel below lays the state out for that case.
 // gdn2_chunk_kernel  Gdn2Mode::Chunk.  One CTA owns a (head, value tile) and walks the chunks;
 //   per chunk, with G the cumulative log decay inside the chunk (every exponent below <= 0):
 //     LA[t,s] = sum_i k_ti k_si e^{G_ti-G_si} (s<t),  LE[t,s] = sum_i k_ti bk_si e^{..} (s<t),
@@ -126,6 +126,67 @@ __global__ void __launch_bounds__(32 * REC_WARPS) gdn2_recurrent_kernel(Gdn2Args
 #pragma unroll
       for (int c = 0; c < REC_C; ++c)
         if (c < nc) So[(size_t)(lane + 32 * m) * a.V + j0 + c] = S[m][c];
+  }
+}
+
+// ------------------------------------------------------------------ decode step (T = 1)
+// One token per sequence: the state is read and written once, so the layout is chosen for
+// HBM: lane = value column (a warp reads 128 contiguous bytes of a state row), the 8 warps
+// split the key rows, and the two reductions over K go through shared memory.
+constexpr int STEP_WARPS = 8;
+
+template <typename T, int RPW>
+__global__ void __launch_bounds__(32 * STEP_WARPS) gdn2_step_kernel(Gdn2Args a) {
+  constexpr int K = RPW * STEP_WARPS;
+  __shared__ float qs[K], ks[K], es[K], bks[K], red[2][STEP_WARPS][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long long bh = blockIdx.y;
+  const int j = blockIdx.x * 32 + lane;
+  const bool col = j < a.V;
+  const int i0 = warp * RPW;
+  const float* S0 = a.S0 ? a.S0 + bh * K * a.V : nullptr;
+  float S[RPW];
+#pragma unroll
+  for (int m = 0; m < RPW; ++m) S[m] = (S0 && col) ? S0[(size_t)(i0 + m) * a.V + j] : 0.f;
+  for (int i = threadIdx.x; i < K; i += 32 * STEP_WARPS) {
+    const size_t x = bh * K + i;
+    const float kk = ld_in(static_cast<const T*>(a.k) + x);
+    qs[i] = ld_in(static_cast<const T*>(a.q) + x);
+    ks[i] = kk;
+    es[i] = expf(a.g[x]);
+    bks[i] = a.b[x] * kk;
+  }
+  const float u = col ? a.w[bh * a.V + j] * ld_in(static_cast<const T*>(a.v) + bh * a.V + j) : 0.f;
+  __syncthreads();
+  float r = 0.f;
+#pragma unroll
+  for (int m = 0; m < RPW; ++m) {
+    S[m] *= es[i0 + m];
+    r = fmaf(ks[i0 + m], S[m], r);
+  }
+  red[0][warp][lane] = r;
+  __syncthreads();
+  r = 0.f;
+#pragma unroll
+  for (int x = 0; x < STEP_WARPS; ++x) r += red[0][x][lane];
+  float y = 0.f;
+#pragma unroll
+  for (int m = 0; m < RPW; ++m) {
+    S[m] = fmaf(ks[i0 + m], u, fmaf(-bks[i0 + m], r, S[m]));
+    y = fmaf(qs[i0 + m], S[m], y);
+  }
+  if (a.S_out && col) {
+    float* So = a.S_out + bh * K * a.V;
+#pragma unroll
+    for (int m = 0; m < RPW; ++m) So[(size_t)(i0 + m) * a.V + j] = S[m];
+  }
+  red[1][warp][lane] = y;
+  __syncthreads();
+  if (warp == 0 && col) {
+    y = 0.f;
+#pragma unroll
+    for (int x = 0; x < STEP_WARPS; ++x) y += red[1][x][lane];
+    st_out(static_cast<T*>(a.o) + bh * a.V + j, y);
   }
 }
 
@@ -330,6 +391,23 @@ cudaError_t launch_gdn2(const Gdn2Args& a, int mode, int chunk, cudaStream_t str
   const long long BH = (long long)a.B * a.H;
   if (BH == 0 || (a.T == 0 && !a.S_out)) return cudaSuccess;
   if (BH > 65535) return cudaErrorInvalidValue;
+  if (mode == 0 && a.T == 1) {
+    const dim3 grid((a.V + 31) / 32, (unsigned)BH);
+#define STEP(RPW)                                                                         \
+  if (a.dtype == 0)                                                                       \
+    gdn2_step_kernel<float, RPW><<<grid, 32 * STEP_WARPS, 0, stream>>>(a);                \
+  else                                                                                    \
+    gdn2_step_kernel<__nv_bfloat16, RPW><<<grid, 32 * STEP_WARPS, 0, stream>>>(a);
+    switch (a.K) {
+      case 32: STEP(4) break;
+      case 64: STEP(8) break;
+      case 128: STEP(16) break;
+      case 256: STEP(32) break;
+      default: return cudaErrorInvalidValue;
+    }
+#undef STEP
+    return cudaGetLastError();
+  }
   if (mode == 0) {
     const dim3 grid((a.V + REC_WARPS * REC_C - 1) / (REC_WARPS * REC_C), (unsigned)BH);
     const dim3 block(32 * REC_WARPS);

@@ -68,8 +68,19 @@ def test_decode_steps_match_the_prefill():
                               dev(inp["b"][sl]), dev(inp["w"][sl]), S, S_out=S)
         outs.append(o)
     torch.cuda.synchronize()
-    assert slice_relerr(host(torch.cat(outs, dim=2)), o_ref, 2) <= 1e-6
-    assert slice_relerr(host(S), S_ref, 2) <= 1e-6
+    # the single-token calls run the decode kernel (another reduction order): o within one
+    # bf16 rounding, the fp32 state within fp32 rounding; both against the oracle as well
+    assert slice_relerr(host(torch.cat(outs, dim=2)), o_ref, 2) <= 1e-2
+    assert slice_relerr(host(S), S_ref, 2) <= 1e-5
+    check(inp, "bf16", host(torch.cat(outs, dim=2)), host(S))
+
+
+@pytest.mark.parametrize("dtype,K,V,state", [("f32", 64, 40, True), ("bf16", 256, 96, False), ("f32", 32, 32, True)])
+def test_decode_step(dtype, K, V, state):
+    """One token per sequence (the decode kernel), state in place, ragged value tile."""
+    inp = inputs.gdn2_inputs(5, 3, 1, K, V, dtype, seed=76, with_state=state)
+    o, S = run(inp, dtype, "recurrent", inplace=state)
+    check(inp, dtype, o, S)
 
 
 def test_empty_sequence_copies_the_state():
