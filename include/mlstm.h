@@ -334,7 +334,10 @@ mlstm_status_t mlstm_fwd_chunkwise_msr(const mlstm_fwd_params_t* p,
  *   S0        [B,H,K,V]  fp32        initial state; NULL = zeros
  *   o         [B,H,T,V]  dtype       output, required (if T > 0)
  *   S_out     [B,H,K,V]  fp32        final state; NULL = not written; may equal S0 exactly
- * No workspace.  Outputs must not overlap the inputs or each other (MLSTM_ERR_ALIAS).
+ *   workspace, workspace_bytes  chunk mode: at least mlstm_gdn2_workspace_size(p) bytes, 16-byte
+ *             aligned (one prepared slot of per-chunk matrices per batch, head and chunk);
+ *             recurrent mode: none needed (size 0), may be NULL
+ * Outputs and the workspace must not overlap the inputs or each other (MLSTM_ERR_ALIAS).
  */
 typedef enum { MLSTM_GDN2_RECURRENT = 0, MLSTM_GDN2_CHUNK = 1 } mlstm_gdn2_mode_t;
 typedef struct {
@@ -343,9 +346,10 @@ typedef struct {
   int mode;  /* mlstm_gdn2_mode_t */
   int chunk; /* chunk mode only */
 } mlstm_gdn2_params_t;
+size_t mlstm_gdn2_workspace_size(const mlstm_gdn2_params_t* p);
 mlstm_status_t mlstm_gdn2_fwd(const mlstm_gdn2_params_t* p, const void* q, const void* k, const void* v,
                               const float* g, const float* b, const float* w, const float* S0, void* o,
-                              float* S_out, mlstm_stream_t stream);
+                              float* S_out, void* workspace, size_t workspace_bytes, mlstm_stream_t stream);
 
 /*
  * One recurrent decode step for every sequence of the batch, state updated in

@@ -9,15 +9,18 @@
 //   so the two reductions over K per token (r and o) are warp shuffles and the state never
 //   leaves the chip between tokens.  With T = 1 and the state in place this is the decode step
 //   (one HBM read and write of S); gdn2_step_kernel below lays the state out for that case.
-// gdn2_chunk_kernel  Gdn2Mode::Chunk.  One CTA owns a (head, value tile) and walks the chunks;
-//   per chunk, with G the cumulative log decay inside the chunk (every exponent below <= 0):
+// gdn2_chunk_prep_kernel + gdn2_chunk_scan_kernel  Gdn2Mode::Chunk.  Per chunk, with G the
+//   cumulative log decay inside the chunk (every exponent below <= 0):
 //     LA[t,s] = sum_i k_ti k_si e^{G_ti-G_si} (s<t),  LE[t,s] = sum_i k_ti bk_si e^{..} (s<t),
 //     QA, QE the same with q_t (s<=t);
 //     R = (I + LE)^{-1} (k e^{G} S + LA U)            (U = w o v; one triangular solve)
 //     o = (q e^{G}) S + QA U - QE R
 //     S <- e^{G_L} o S + (k e^{G_L-G})^T U - (bk e^{G_L-G})^T R
 //   i.e. the WY-style block form of the recurrence: dense products inside the chunk, the state
-//   carried between chunks.  fp32 SIMT, state tile in shared memory.
+//   carried between chunks.  The prep kernel builds every chunk's L x L matrices, the inverse
+//   of I + LE and the decayed rows at once (one CTA per chunk) into the workspace; the scan
+//   kernel (one CTA per head and value tile, chunks in order) is left with dense products.
+//   fp32 SIMT, the state tile in shared memory.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -193,177 +196,247 @@ __global__ void __launch_bounds__(32 * STEP_WARPS) gdn2_step_kernel(Gdn2Args a) 
 // ------------------------------------------------------------------ chunk (WY block form)
 constexpr int CH_THREADS = 256;
 
-struct ChunkSmem {
-  int L, K, VT, lk, ll;
-  // offsets in floats
-  size_t G, Kc, Bk, Qc, S, U, R, LA, LE, QA, QE, gL, total;
-};
-__host__ __device__ inline ChunkSmem chunk_smem(int L, int K, int VT) {
-  ChunkSmem m;
-  m.L = L;
-  m.K = K;
-  m.VT = VT;
-  m.lk = K + 1;  // padded rows: threads on different tokens read different banks
-  m.ll = L + 1;
-  size_t o = 0;
-  m.G = o, o += (size_t)L * m.lk;
-  m.Kc = o, o += (size_t)L * m.lk;
-  m.Bk = o, o += (size_t)L * m.lk;
-  m.Qc = o, o += (size_t)L * m.lk;
-  m.S = o, o += (size_t)K * VT;
-  m.U = o, o += (size_t)L * VT;
-  m.R = o, o += (size_t)L * VT;
-  m.LA = o, o += (size_t)L * m.ll;
-  m.LE = o, o += (size_t)L * m.ll;
-  m.QA = o, o += (size_t)L * m.ll;
-  m.QE = o, o += (size_t)L * m.ll;
-  m.gL = o, o += (size_t)K;
-  m.total = o;
-  return m;
+// Per-chunk slot of the workspace written by the prep kernel (floats, unpadded rows):
+//   Qd = q e^{G}, Kd = k e^{G}, Kt = k e^{G_L-G}, Bt = bk e^{G_L-G}   [L][K] each
+//   LA, Tinv = (I + LE)^{-1}, QA, QE                                   [L][L] each
+//   eGL = e^{G_L}                                                      [K]
+__host__ __device__ inline size_t chunk_slot_floats(int L, int K) { return (size_t)4 * L * K + (size_t)4 * L * L + K; }
+
+// shared-memory plans (floats; rows padded by one against bank conflicts)
+__host__ __device__ inline size_t prep_smem_floats(int L, int K) {
+  return (size_t)4 * L * (K + 1) + (size_t)5 * L * (L + 1) + K;
+}
+__host__ __device__ inline size_t scan_smem_floats(int L, int K, int VT) {
+  return (size_t)4 * L * (K + 1) + (size_t)4 * L * (L + 1) + K + (size_t)K * VT + (size_t)3 * L * VT;
 }
 
+// Prep: one CTA per (chunk, head), every chunk at once.  Builds the chunk's weight matrices
+// (the exponential-heavy part, e^{G_t - G_s} per pair and key channel, every exponent <= 0),
+// the inverse of the unit lower-triangular I + LE, and the decayed row forms.
 template <typename T>
-__global__ void __launch_bounds__(CH_THREADS) gdn2_chunk_kernel(Gdn2Args a, int L, int VT) {
+__global__ void __launch_bounds__(CH_THREADS) gdn2_chunk_prep_kernel(Gdn2Args a, int L, float* ws) {
   extern __shared__ float sm[];
-  const int K = a.K, tid = threadIdx.x;
-  const ChunkSmem M = chunk_smem(L, K, VT);
-  const int lk = M.lk, ll = M.ll;
-  float *G = sm + M.G, *Kc = sm + M.Kc, *Bk = sm + M.Bk, *Qc = sm + M.Qc, *S = sm + M.S, *U = sm + M.U,
-        *R = sm + M.R, *LA = sm + M.LA, *LE = sm + M.LE, *QA = sm + M.QA, *QE = sm + M.QE, *gL = sm + M.gL;
+  const int K = a.K, tid = threadIdx.x, lk = K + 1, ll = L + 1;
+  float *G = sm, *Kc = G + L * lk, *Bk = Kc + L * lk, *Qc = Bk + L * lk, *LA = Qc + L * lk, *LE = LA + L * ll,
+        *QA = LE + L * ll, *QE = QA + L * ll, *TI = QE + L * ll, *gL = TI + L * ll;
   const long long bh = blockIdx.y;
-  const int j0 = blockIdx.x * VT;
+  const int c = blockIdx.x, t0 = c * L, Lc = min(L, a.T - t0);
+  const int nch = (a.T + L - 1) / L;
   const T* q = static_cast<const T*>(a.q) + bh * a.T * K;
   const T* k = static_cast<const T*>(a.k) + bh * a.T * K;
-  const T* v = static_cast<const T*>(a.v) + bh * a.T * a.V + j0;
   const float* g = a.g + bh * a.T * K;
   const float* b = a.b + bh * a.T * K;
+  for (int e = tid; e < L * K; e += CH_THREADS) {
+    const int t = e / K, i = e % K;
+    float qq = 0.f, kk = 0.f, gg = 0.f, bb = 0.f;
+    if (t < Lc) {
+      const size_t x = (size_t)(t0 + t) * K + i;
+      qq = ld_in(q + x), kk = ld_in(k + x), gg = g[x], bb = b[x];
+    }
+    Qc[t * lk + i] = qq, Kc[t * lk + i] = kk, G[t * lk + i] = gg, Bk[t * lk + i] = bb * kk;
+  }
+  __syncthreads();
+  for (int i = tid; i < K; i += CH_THREADS) {  // cumulative log decay per key channel
+    float s = 0.f;
+    for (int t = 0; t < L; ++t) {
+      s += G[t * lk + i];
+      G[t * lk + i] = s;
+    }
+    gL[i] = s;
+  }
+  __syncthreads();
+  // the four L x L weight matrices, 4 x 4 (t, s) blocks per thread, lower triangle only
+  const int nb4 = L / 4;
+  for (int blk = tid; blk < nb4 * nb4; blk += CH_THREADS) {
+    const int tb = blk / nb4, sb = blk % nb4;
+    float la[4][4] = {}, le[4][4] = {}, qa[4][4] = {}, qe[4][4] = {};
+    if (sb <= tb) {
+      for (int i = 0; i < K; ++i) {
+        float gt[4], kt[4], qt[4], gs[4], ks[4], bs[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const int t = 4 * tb + x, s2 = 4 * sb + x;
+          gt[x] = G[t * lk + i], kt[x] = Kc[t * lk + i], qt[x] = Qc[t * lk + i];
+          gs[x] = G[s2 * lk + i], ks[x] = Kc[s2 * lk + i], bs[x] = Bk[s2 * lk + i];
+        }
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+          for (int y = 0; y < 4; ++y) {
+            const float e = expf(fminf(gt[x] - gs[y], 0.f));
+            const float ek = e * ks[y], eb = e * bs[y];
+            la[x][y] = fmaf(kt[x], ek, la[x][y]);
+            le[x][y] = fmaf(kt[x], eb, le[x][y]);
+            qa[x][y] = fmaf(qt[x], ek, qa[x][y]);
+            qe[x][y] = fmaf(qt[x], eb, qe[x][y]);
+          }
+      }
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int y = 0; y < 4; ++y) {
+        const int t = 4 * tb + x, s2 = 4 * sb + y;
+        LA[t * ll + s2] = s2 < t ? la[x][y] : 0.f;
+        LE[t * ll + s2] = s2 < t ? le[x][y] : 0.f;
+        QA[t * ll + s2] = s2 <= t ? qa[x][y] : 0.f;
+        QE[t * ll + s2] = s2 <= t ? qe[x][y] : 0.f;
+      }
+  }
+  __syncthreads();
+  // inverse of I + LE, one column per thread: TI[t][col] = -sum_{col<=s<t} LE[t][s] TI[s][col]
+  for (int col = tid; col < L; col += CH_THREADS) {
+    for (int t = 0; t < L; ++t) {
+      if (t < col) {
+        TI[t * ll + col] = 0.f;
+        continue;
+      }
+      if (t == col) {
+        TI[t * ll + col] = 1.f;
+        continue;
+      }
+      float a0 = 0.f, a1 = 0.f;
+      int s2 = col;
+      for (; s2 + 1 < t; s2 += 2) {
+        a0 = fmaf(LE[t * ll + s2], TI[s2 * ll + col], a0);
+        a1 = fmaf(LE[t * ll + s2 + 1], TI[(s2 + 1) * ll + col], a1);
+      }
+      if (s2 < t) a0 = fmaf(LE[t * ll + s2], TI[s2 * ll + col], a0);
+      TI[t * ll + col] = -(a0 + a1);
+    }
+  }
+  // the slot: decayed rows, then the L x L matrices and e^{G_L}
+  float* slot = ws + ((size_t)bh * nch + c) * chunk_slot_floats(L, K);
+  float *oQd = slot, *oKd = oQd + L * K, *oKt = oKd + L * K, *oBt = oKt + L * K, *oLA = oBt + L * K,
+        *oTI = oLA + L * L, *oQA = oTI + L * L, *oQE = oQA + L * L, *oGL = oQE + L * L;
+  for (int e = tid; e < L * K; e += CH_THREADS) {
+    const int t = e / K, i = e % K, x = t * lk + i;
+    const float gg = G[x], up = expf(gg), tail = expf(gL[i] - gg);
+    oQd[e] = Qc[x] * up;
+    oKd[e] = Kc[x] * up;
+    oKt[e] = Kc[x] * tail;
+    oBt[e] = Bk[x] * tail;
+  }
+  for (int i = tid; i < K; i += CH_THREADS) oGL[i] = expf(gL[i]);
+  __syncthreads();  // TI complete
+  for (int e = tid; e < L * L; e += CH_THREADS) {
+    const int t = e / L, s2 = e % L;
+    oLA[e] = LA[t * ll + s2];
+    oTI[e] = TI[t * ll + s2];
+    oQA[e] = QA[t * ll + s2];
+    oQE[e] = QE[t * ll + s2];
+  }
+}
+
+// Scan: one CTA per (value tile, head) walks the chunks in order; per chunk only dense
+// products on the prepared slot:
+//   R = Tinv (Kd S + LA U),  o = Qd S + QA U - QE R,  S <- e^{G_L} o S + Kt^T U - Bt^T R
+template <typename T>
+__global__ void __launch_bounds__(CH_THREADS) gdn2_chunk_scan_kernel(Gdn2Args a, int L, int VT, const float* ws) {
+  extern __shared__ float sm[];
+  const int K = a.K, tid = threadIdx.x, lk = K + 1, ll = L + 1;
+  float *Qd = sm, *Kd = Qd + L * lk, *Kt = Kd + L * lk, *Bt = Kt + L * lk, *LA = Bt + L * lk, *TI = LA + L * ll,
+        *QA = TI + L * ll, *QE = QA + L * ll, *eGL = QE + L * ll, *S = eGL + K, *U = S + K * VT, *X = U + L * VT,
+        *R = X + L * VT;
+  const long long bh = blockIdx.y;
+  const int j0 = blockIdx.x * VT, nch = (a.T + L - 1) / L;
+  const T* v = static_cast<const T*>(a.v) + bh * a.T * a.V + j0;
   const float* w = a.w + bh * a.T * a.V + j0;
   T* o = static_cast<T*>(a.o) + bh * a.T * a.V + j0;
   for (int e = tid; e < K * VT; e += CH_THREADS) {
     const int i = e / VT, j = e % VT;
     S[e] = a.S0 ? a.S0[(bh * K + i) * a.V + j0 + j] : 0.f;
   }
-  for (int t0 = 0; t0 < a.T; t0 += L) {
-    const int Lc = min(L, a.T - t0);
+  for (int c = 0; c < nch; ++c) {
+    const int t0 = c * L, Lc = min(L, a.T - t0);
+    const float* slot = ws + ((size_t)bh * nch + c) * chunk_slot_floats(L, K);
     __syncthreads();  // the previous chunk is done with every buffer
-    // 1. inputs of the chunk (rows past the end: zeros, which add nothing below)
     for (int e = tid; e < L * K; e += CH_THREADS) {
-      const int t = e / K, i = e % K;
-      float qq = 0.f, kk = 0.f, gg = 0.f, bb = 0.f;
-      if (t < Lc) {
-        const size_t x = (size_t)(t0 + t) * K + i;
-        qq = ld_in(q + x), kk = ld_in(k + x), gg = g[x], bb = b[x];
-      }
-      Qc[t * lk + i] = qq, Kc[t * lk + i] = kk, G[t * lk + i] = gg, Bk[t * lk + i] = bb * kk;
+      const int t = e / K, i = e % K, x = t * lk + i;
+      Qd[x] = slot[e];
+      Kd[x] = slot[L * K + e];
+      Kt[x] = slot[2 * L * K + e];
+      Bt[x] = slot[3 * L * K + e];
     }
+    const float* sl2 = slot + 4 * L * K;
+    for (int e = tid; e < L * L; e += CH_THREADS) {
+      const int t = e / L, s2 = e % L, x = t * ll + s2;
+      LA[x] = sl2[e];
+      TI[x] = sl2[L * L + e];
+      QA[x] = sl2[2 * L * L + e];
+      QE[x] = sl2[3 * L * L + e];
+    }
+    for (int i = tid; i < K; i += CH_THREADS) eGL[i] = sl2[4 * L * L + i];
     for (int e = tid; e < L * VT; e += CH_THREADS) {
       const int t = e / VT, j = e % VT;
       U[e] = t < Lc ? w[(size_t)(t0 + t) * a.V + j] * ld_in(v + (size_t)(t0 + t) * a.V + j) : 0.f;
     }
     __syncthreads();
-    // 2. cumulative log decay per key channel
-    for (int i = tid; i < K; i += CH_THREADS) {
-      float s = 0.f;
-      for (int t = 0; t < L; ++t) {
-        s += G[t * lk + i];
-        G[t * lk + i] = s;
+    // Each thread computes four rows t, t + L/4, t + L/2, t + 3L/4 of one column j with
+    // independent accumulators, so the column operand is loaded once per four FMAs and the
+    // four dependency chains overlap.
+    const int L4 = L / 4, K4 = K / 4;
+    for (int e = tid; e < L4 * VT; e += CH_THREADS) {  // X = Kd S + LA U
+      const int t = e / VT, j = e % VT;
+      float acc[4] = {};
+      for (int i = 0; i < K; ++i) {
+        const float sv = S[i * VT + j];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) acc[x] = fmaf(Kd[(t + x * L4) * lk + i], sv, acc[x]);
       }
-      gL[i] = s;
+      for (int s2 = 0; s2 < t + 3 * L4; ++s2) {
+        const float uv = U[s2 * VT + j];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) acc[x] = fmaf(LA[(t + x * L4) * ll + s2], uv, acc[x]);  // LA = 0 for s >= t
+      }
+#pragma unroll
+      for (int x = 0; x < 4; ++x) X[(t + x * L4) * VT + j] = acc[x];
     }
     __syncthreads();
-    // 3. the four L x L weight matrices, 4 x 4 (t, s) blocks per thread, lower triangle only
-    {
-      const int nb4 = L / 4;
-      for (int blk = tid; blk < nb4 * nb4; blk += CH_THREADS) {
-        const int tb = blk / nb4, sb = blk % nb4;
-        if (sb > tb) continue;
-        float la[4][4] = {}, le[4][4] = {}, qa[4][4] = {}, qe[4][4] = {};
-        for (int i = 0; i < K; ++i) {
-          float gt[4], kt[4], qt[4], gs[4], ks[4], bs[4];
+    for (int e = tid; e < L4 * VT; e += CH_THREADS) {  // R = Tinv X
+      const int t = e / VT, j = e % VT;
+      float acc[4] = {};
+      for (int s2 = 0; s2 <= t + 3 * L4; ++s2) {
+        const float xv = X[s2 * VT + j];
 #pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            const int t = 4 * tb + x, s = 4 * sb + x;
-            gt[x] = G[t * lk + i], kt[x] = Kc[t * lk + i], qt[x] = Qc[t * lk + i];
-            gs[x] = G[s * lk + i], ks[x] = Kc[s * lk + i], bs[x] = Bk[s * lk + i];
-          }
+        for (int x = 0; x < 4; ++x) acc[x] = fmaf(TI[(t + x * L4) * ll + s2], xv, acc[x]);  // TI = 0 above the diagonal
+      }
 #pragma unroll
-          for (int x = 0; x < 4; ++x)
+      for (int x = 0; x < 4; ++x) R[(t + x * L4) * VT + j] = acc[x];
+    }
+    __syncthreads();
+    for (int e = tid; e < L4 * VT; e += CH_THREADS) {  // o = Qd S + QA U - QE R
+      const int t = e / VT, j = e % VT;
+      float acc[4] = {};
+      for (int i = 0; i < K; ++i) {
+        const float sv = S[i * VT + j];
 #pragma unroll
-            for (int y = 0; y < 4; ++y) {
-              const float e = expf(fminf(gt[x] - gs[y], 0.f));
-              const float ek = e * ks[y], eb = e * bs[y];
-              la[x][y] = fmaf(kt[x], ek, la[x][y]);
-              le[x][y] = fmaf(kt[x], eb, le[x][y]);
-              qa[x][y] = fmaf(qt[x], ek, qa[x][y]);
-              qe[x][y] = fmaf(qt[x], eb, qe[x][y]);
-            }
-        }
+        for (int x = 0; x < 4; ++x) acc[x] = fmaf(Qd[(t + x * L4) * lk + i], sv, acc[x]);
+      }
+      for (int s2 = 0; s2 <= t + 3 * L4; ++s2) {
+        const float uv = U[s2 * VT + j], rv = R[s2 * VT + j];
+#pragma unroll
+        for (int x = 0; x < 4; ++x)  // QA, QE = 0 above the diagonal
+          acc[x] = fmaf(QA[(t + x * L4) * ll + s2], uv, fmaf(-QE[(t + x * L4) * ll + s2], rv, acc[x]));
+      }
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+        if (t + x * L4 < Lc) st_out(o + (size_t)(t0 + t + x * L4) * a.V + j, acc[x]);
+    }
+    __syncthreads();  // every read of S for o is done
+    for (int e = tid; e < K4 * VT; e += CH_THREADS) {  // S <- e^{G_L} S + Kt^T U - Bt^T R
+      const int i = e / VT, j = e % VT;
+      float acc[4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) acc[x] = eGL[i + x * K4] * S[(i + x * K4) * VT + j];
+      for (int s2 = 0; s2 < L; ++s2) {
+        const float uv = U[s2 * VT + j], rv = R[s2 * VT + j];
 #pragma unroll
         for (int x = 0; x < 4; ++x)
+          acc[x] = fmaf(Kt[s2 * lk + i + x * K4], uv, fmaf(-Bt[s2 * lk + i + x * K4], rv, acc[x]));
+      }
 #pragma unroll
-          for (int y = 0; y < 4; ++y) {
-            const int t = 4 * tb + x, s = 4 * sb + y;
-            LA[t * ll + s] = s < t ? la[x][y] : 0.f;
-            LE[t * ll + s] = s < t ? le[x][y] : 0.f;
-            QA[t * ll + s] = s <= t ? qa[x][y] : 0.f;
-            QE[t * ll + s] = s <= t ? qe[x][y] : 0.f;
-          }
-      }
-    }
-    __syncthreads();
-    // 4. decayed forms of the rows: Qc <- q e^{G}, G <- k e^{G} (read-out and right-hand side),
-    //    Kc <- k e^{G_L - G}, Bk <- bk e^{G_L - G} (state update)
-    for (int e = tid; e < L * K; e += CH_THREADS) {
-      const int t = e / K, i = e % K, x = t * lk + i;
-      const float gg = G[x], up = expf(gg), tail = expf(gL[i] - gg);
-      Qc[x] *= up;
-      G[x] = Kc[x] * up;
-      Kc[x] *= tail;
-      Bk[x] *= tail;
-    }
-    __syncthreads();
-    // 5. right-hand side of the solve: R = (k e^G) S + LA U
-    for (int e = tid; e < L * VT; e += CH_THREADS) {
-      const int t = e / VT, j = e % VT;
-      float acc = 0.f;
-      for (int i = 0; i < K; ++i) acc = fmaf(G[t * lk + i], S[i * VT + j], acc);
-      for (int s = 0; s < t; ++s) acc = fmaf(LA[t * ll + s], U[s * VT + j], acc);
-      R[e] = acc;
-    }
-    __syncthreads();
-    // 6. unit lower-triangular solve (I + LE) R = rhs, column by column
-    for (int j = tid; j < VT; j += CH_THREADS) {
-      for (int t = 1; t < L; ++t) {
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-        int s = 0;
-        for (; s + 3 < t; s += 4) {
-          a0 = fmaf(LE[t * ll + s], R[s * VT + j], a0);
-          a1 = fmaf(LE[t * ll + s + 1], R[(s + 1) * VT + j], a1);
-          a2 = fmaf(LE[t * ll + s + 2], R[(s + 2) * VT + j], a2);
-          a3 = fmaf(LE[t * ll + s + 3], R[(s + 3) * VT + j], a3);
-        }
-        for (; s < t; ++s) a0 = fmaf(LE[t * ll + s], R[s * VT + j], a0);
-        R[t * VT + j] -= (a0 + a1) + (a2 + a3);
-      }
-    }
-    __syncthreads();
-    // 7. outputs: o = (q e^G) S + QA U - QE R
-    for (int e = tid; e < L * VT; e += CH_THREADS) {
-      const int t = e / VT, j = e % VT;
-      if (t >= Lc) continue;
-      float acc = 0.f;
-      for (int i = 0; i < K; ++i) acc = fmaf(Qc[t * lk + i], S[i * VT + j], acc);
-      for (int s = 0; s <= t; ++s) acc = fmaf(QA[t * ll + s], U[s * VT + j], fmaf(-QE[t * ll + s], R[s * VT + j], acc));
-      st_out(o + (size_t)(t0 + t) * a.V + j, acc);
-    }
-    // 8. state: S <- e^{G_L} S + (k e^{G_L-G})^T U - (bk e^{G_L-G})^T R  (reads S, R, U only
-    //    after step 7 read them: each thread updates the elements no other thread reads here)
-    __syncthreads();
-    for (int e = tid; e < K * VT; e += CH_THREADS) {
-      const int i = e / VT, j = e % VT;
-      float acc = expf(gL[i]) * S[e];
-      for (int s = 0; s < L; ++s) acc = fmaf(Kc[s * lk + i], U[s * VT + j], fmaf(-Bk[s * lk + i], R[s * VT + j], acc));
-      S[e] = acc;
+      for (int x = 0; x < 4; ++x) S[(i + x * K4) * VT + j] = acc[x];
     }
   }
   __syncthreads();
@@ -379,15 +452,19 @@ __global__ void __launch_bounds__(CH_THREADS) gdn2_chunk_kernel(Gdn2Args a, int 
 bool gdn2_recurrent_supported(int K) { return K == 32 || K == 64 || K == 128 || K == 256; }
 
 int gdn2_chunk_vtile(int L, int K, int V) {
-  if (L < 4 || L > 64 || L % 4 || K < 1 || V < 1) return 0;
+  if (L < 4 || L > 64 || L % 4 || K < 4 || K % 4 || V < 1) return 0;
+  if (prep_smem_floats(L, K) * sizeof(float) > 227 * 1024) return 0;
   for (int vt = 64; vt >= 1; vt /= 2)
-    if (V % vt == 0 && chunk_smem(L, K, vt).total * sizeof(float) <= 227 * 1024) return vt;
+    if (V % vt == 0 && scan_smem_floats(L, K, vt) * sizeof(float) <= 227 * 1024) return vt;
   return 0;
 }
 
-size_t gdn2_chunk_smem_bytes(int L, int K, int VT) { return chunk_smem(L, K, VT).total * sizeof(float); }
+size_t gdn2_chunk_workspace_bytes(long long BH, int T, int L, int K) {
+  const long long nch = (T + L - 1) / L;
+  return (size_t)BH * nch * chunk_slot_floats(L, K) * sizeof(float);
+}
 
-cudaError_t launch_gdn2(const Gdn2Args& a, int mode, int chunk, cudaStream_t stream) {
+cudaError_t launch_gdn2(const Gdn2Args& a, int mode, int chunk, void* ws, cudaStream_t stream) {
   const long long BH = (long long)a.B * a.H;
   if (BH == 0 || (a.T == 0 && !a.S_out)) return cudaSuccess;
   if (BH > 65535) return cudaErrorInvalidValue;
@@ -427,19 +504,30 @@ cudaError_t launch_gdn2(const Gdn2Args& a, int mode, int chunk, cudaStream_t str
     return cudaGetLastError();
   }
   const int VT = gdn2_chunk_vtile(chunk, a.K, a.V);
-  if (VT == 0) return cudaErrorInvalidValue;
-  const size_t smem = gdn2_chunk_smem_bytes(chunk, a.K, VT);
-  const dim3 grid(a.V / VT, (unsigned)BH);
+  if (VT == 0 || !ws) return cudaErrorInvalidValue;
+  const long long nch = (a.T + chunk - 1) / chunk;
+  if (nch > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const int smem_p = (int)(prep_smem_floats(chunk, a.K) * sizeof(float));
+  const int smem_s = (int)(scan_smem_floats(chunk, a.K, VT) * sizeof(float));
+  float* wsf = static_cast<float*>(ws);
+  const dim3 grid_p((unsigned)nch, (unsigned)BH), grid_s(a.V / VT, (unsigned)BH);
   cudaError_t e;
   if (a.dtype == 0) {
-    e = cudaFuncSetAttribute(gdn2_chunk_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(gdn2_chunk_prep_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_p);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gdn2_chunk_scan_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_s);
     if (e != cudaSuccess) return e;
-    gdn2_chunk_kernel<float><<<grid, CH_THREADS, smem, stream>>>(a, chunk, VT);
+    gdn2_chunk_prep_kernel<float><<<grid_p, CH_THREADS, smem_p, stream>>>(a, chunk, wsf);
+    gdn2_chunk_scan_kernel<float><<<grid_s, CH_THREADS, smem_s, stream>>>(a, chunk, VT, wsf);
   } else {
-    e = cudaFuncSetAttribute(gdn2_chunk_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
+    e = cudaFuncSetAttribute(gdn2_chunk_prep_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem_p);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gdn2_chunk_scan_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               smem_s);
     if (e != cudaSuccess) return e;
-    gdn2_chunk_kernel<__nv_bfloat16><<<grid, CH_THREADS, smem, stream>>>(a, chunk, VT);
+    gdn2_chunk_prep_kernel<__nv_bfloat16><<<grid_p, CH_THREADS, smem_p, stream>>>(a, chunk, wsf);
+    gdn2_chunk_scan_kernel<__nv_bfloat16><<<grid_s, CH_THREADS, smem_s, stream>>>(a, chunk, VT, wsf);
   }
   return cudaGetLastError();
 }

@@ -46,11 +46,12 @@ struct Gdn2Args {
   float* S_out;
 };
 bool gdn2_recurrent_supported(int K);
-// value-tile width of the chunk kernel for these sizes (0 = unsupported)
+// value-tile width of the chunk scan kernel for these sizes (0 = unsupported)
 int gdn2_chunk_vtile(int L, int K, int V);
-size_t gdn2_chunk_smem_bytes(int L, int K, int VT);
-// mode 0: fused recurrent (token by token); 1: chunk of `chunk` tokens
-cudaError_t launch_gdn2(const Gdn2Args& a, int mode, int chunk, cudaStream_t stream);
+// workspace of the chunk mode: one prepared slot per (batch, head, chunk)
+size_t gdn2_chunk_workspace_bytes(long long BH, int T, int L, int K);
+// mode 0: fused recurrent (token by token); 1: chunk of `chunk` tokens (needs ws)
+cudaError_t launch_gdn2(const Gdn2Args& a, int mode, int chunk, void* ws, cudaStream_t stream);
 
 cudaError_t launch_gate_prep(int BH, int S, int n_per_head, const float* ig, const float* fg,
                              const float* m0, const float* n0, float* m_tok, float* m_init,

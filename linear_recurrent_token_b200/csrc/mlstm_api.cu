@@ -807,9 +807,15 @@ mlstm_status_t mlstm_fwd_chunkwise_msr(const mlstm_fwd_params_t* p, const void* 
 }
 
 
+size_t mlstm_gdn2_workspace_size(const mlstm_gdn2_params_t* p) {
+  if (!p || p->mode != MLSTM_GDN2_CHUNK || p->B < 0 || p->H < 0 || p->T < 0 || p->K < 1) return 0;
+  if (p->chunk < 4 || p->chunk > 64 || p->chunk % 4) return 0;
+  return gdn2_chunk_workspace_bytes((long long)p->B * p->H, p->T, p->chunk, p->K);
+}
+
 mlstm_status_t mlstm_gdn2_fwd(const mlstm_gdn2_params_t* p, const void* q, const void* k, const void* v,
                               const float* g, const float* b, const float* w, const float* S0, void* o,
-                              float* S_out, cudaStream_t stream) {
+                              float* S_out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (!p) return MLSTM_ERR_NULL;
   if (p->dtype != MLSTM_F32 && p->dtype != MLSTM_BF16) return MLSTM_ERR_DTYPE;
   if (p->B < 0 || p->H < 0 || p->T < 0 || p->K < 1 || p->V < 1) return MLSTM_ERR_SHAPE;
@@ -822,14 +828,17 @@ mlstm_status_t mlstm_gdn2_fwd(const mlstm_gdn2_params_t* p, const void* q, const
   const size_t bq = tok * p->K * es, bv = tok * p->V * es, bg = tok * p->K * 4, bw = tok * p->V * 4;
   const size_t bS = (size_t)BH * p->K * p->V * 4;
   if (tok > 0 && (!q || !k || !v || !g || !b || !w || !o)) return MLSTM_ERR_NULL;
-  const void* all[] = {q, k, v, g, b, w, S0, o, S_out};
+  const void* all[] = {q, k, v, g, b, w, S0, o, S_out, workspace};
   for (const void* ptr : all)
     if (ptr && misaligned(ptr)) return MLSTM_ERR_ALIGN;
+  const size_t need = mlstm_gdn2_workspace_size(p);
   const Range ins[] = {{q, bq}, {k, bq}, {v, bv}, {g, bg}, {b, bg}, {w, bw}};
-  const Range ro{o, bv}, rS{S_out, bS}, r0{S0, bS};
+  const Range ro{o, bv}, rS{S_out, bS}, r0{S0, bS}, rw{workspace, need};
   for (const Range& i : ins)
-    if (overlaps(ro, i) || overlaps(rS, i)) return MLSTM_ERR_ALIAS;
+    if (overlaps(ro, i) || overlaps(rS, i) || overlaps(rw, i)) return MLSTM_ERR_ALIAS;
   if (overlaps(ro, rS) || overlaps(ro, r0) || (overlaps(rS, r0) && S_out != S0)) return MLSTM_ERR_ALIAS;
+  if (overlaps(rw, ro) || overlaps(rw, rS) || overlaps(rw, r0)) return MLSTM_ERR_ALIAS;
+  if (need > 0 && (!workspace || workspace_bytes < need)) return MLSTM_ERR_WORKSPACE;
   if (BH == 0) return MLSTM_OK;
   Gdn2Args a;
   a.B = p->B, a.H = p->H, a.T = p->T, a.K = p->K, a.V = p->V, a.dtype = p->dtype == MLSTM_BF16 ? 1 : 0;
@@ -841,7 +850,8 @@ mlstm_status_t mlstm_gdn2_fwd(const mlstm_gdn2_params_t* p, const void* q, const
              : cudaMemsetAsync(S_out, 0, bS, (cudaStream_t)stream);
     return e == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA;
   }
-  return launch_gdn2(a, p->mode, p->chunk, (cudaStream_t)stream) == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA;
+  return launch_gdn2(a, p->mode, p->chunk, workspace, (cudaStream_t)stream) == cudaSuccess ? MLSTM_OK
+                                                                                             : MLSTM_ERR_CUDA;
 }
 
 }  // extern "C"

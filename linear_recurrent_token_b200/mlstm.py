@@ -92,7 +92,9 @@ def lib():
         L.mlstm_fwd_chunkwise_msr.argtypes = [ctypes.POINTER(FwdParams), P, P, P, P, P, P, F, P, P, P, F, P, P, P,
                                               P, P, P, P, P, Z, P]
         L.mlstm_fwd_chunkwise_msr.restype = I
-        L.mlstm_gdn2_fwd.argtypes = [ctypes.POINTER(Gdn2Params)] + [P] * 9 + [P]
+        L.mlstm_gdn2_workspace_size.argtypes = [ctypes.POINTER(Gdn2Params)]
+        L.mlstm_gdn2_workspace_size.restype = Z
+        L.mlstm_gdn2_fwd.argtypes = [ctypes.POINTER(Gdn2Params)] + [P] * 10 + [Z, P]
         L.mlstm_gdn2_fwd.restype = I
         L.mlstm_bwd_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
         L.mlstm_bwd_workspace_size.restype = Z
@@ -294,8 +296,12 @@ def fwd_chunkwise_msr(q, k, v, igate=None, fgate=None, g=None, gn_weight=None, g
     return y, C_out, n_out, m_out
 
 
+def gdn2_workspace_size(params: Gdn2Params) -> int:
+    return int(lib().mlstm_gdn2_workspace_size(ctypes.byref(params)))
+
+
 def gdn2_fwd(q, k, v, g, b, w, S0=None, *, mode: str = "recurrent", chunk: int = 64, o=None, S_out=None,
-             return_state: bool = True, stream=None):
+             return_state: bool = True, workspace=None, stream=None):
     """Gated DeltaNet-2 (mlstm_gdn2_fwd): q, k [B,H,T,K], v [B,H,T,V] (fp32 or bf16); g, b
     [B,H,T,K] and w [B,H,T,V] fp32; S0 [B,H,K,V] fp32 or None.  mode "recurrent" or "chunk".
     S_out may be S0 (in place: the decode step).  Returns (o, S_out)."""
@@ -307,8 +313,12 @@ def gdn2_fwd(q, k, v, g, b, w, S0=None, *, mode: str = "recurrent", chunk: int =
         o = torch.empty((B, H, T, V), dtype=q.dtype, device=q.device)
     if return_state and S_out is None:
         S_out = torch.empty((B, H, K, V), dtype=torch.float32, device=q.device)
+    ws_bytes = gdn2_workspace_size(p)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib().mlstm_gdn2_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0),
-                              _ptr(o), _ptr(S_out), _stream_ptr(stream))
+                              _ptr(o), _ptr(S_out), _ptr(workspace), ctypes.c_size_t(ws_len), _stream_ptr(stream))
     if st != 0:
         raise MlstmError(st, "mlstm_gdn2_fwd")
     return o, S_out

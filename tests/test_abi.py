@@ -270,9 +270,10 @@ def test_msr_block_validation_and_workspace():
 
 # ---------------------------------------------------------------- Gated DeltaNet-2
 def gdn2_call(B=2, H=2, T=16, K=64, V=64, dtype=0, mode=0, chunk=16, q=A, k=B_, v=C_, g=D_, b=E_, w=F_, S0=None,
-              o=G_, S=None):
+              o=G_, S=None, ws=None, ws_bytes=0):
     p = mlstm.Gdn2Params(B, H, T, K, V, dtype, mode, chunk)
-    return mlstm.lib().mlstm_gdn2_fwd(ctypes.byref(p), q, k, v, g, b, w, S0, o, S, ctypes.c_void_p(0))
+    return mlstm.lib().mlstm_gdn2_fwd(ctypes.byref(p), q, k, v, g, b, w, S0, o, S, ws, ctypes.c_size_t(ws_bytes),
+                                      ctypes.c_void_p(0))
 
 
 def test_gdn2_validation():
@@ -287,3 +288,10 @@ def test_gdn2_validation():
     assert gdn2_call(S=G_ + 64) == 7                # state inside o
     assert gdn2_call(S0=H_, S=H_ + 16) == 7         # state overlapping the initial state, not equal
     assert gdn2_call(S0=G_, S=None) == 7            # initial state under o
+    # chunk mode: one prepared slot per (batch, head, chunk) of 4 L K + 4 L^2 + K floats
+    p = mlstm.Gdn2Params(2, 2, 16, 64, 64, 0, 1, 8)
+    assert mlstm.gdn2_workspace_size(p) == 2 * 2 * 2 * (4 * 8 * 64 + 4 * 64 + 64) * 4
+    assert mlstm.gdn2_workspace_size(mlstm.Gdn2Params(2, 2, 16, 64, 64, 0, 0, 8)) == 0
+    assert gdn2_call(mode=1, chunk=8) == 5                          # no workspace
+    assert gdn2_call(mode=1, chunk=8, ws=H_, ws_bytes=16) == 5      # too small
+    assert gdn2_call(mode=1, chunk=8, ws=A, ws_bytes=1 << 30) == 7  # workspace over q
