@@ -6,7 +6,8 @@
 //
 // gdn2_recurrent_kernel  Gdn2Mode::FusedRecurrent.  One warp owns C value columns of one head
 //   for the whole sequence; lane l holds key rows l, l+32, ... of those columns in registers,
-//   so the two reductions over K per token (r and o) are warp shuffles and the state never
+//   so the two reductions over K per token (r and o) are warp shuffles (the eight columns
+//   reduced together in 9 shuffles, r broadcast back in 8) and the state never
 //   leaves the chip between tokens.  With T = 1 and the state in place this is the decode step
 //   (one HBM read and write of S); gdn2_step_kernel below lays the state out for that case.
 // gdn2_chunk_prep_kernel + gdn2_chunk_scan_kernel  Gdn2Mode::Chunk.  Per chunk, with G the
@@ -39,8 +40,31 @@ __device__ __forceinline__ void st_out(__nv_bfloat16* p, float x) { *p = __float
 constexpr int REC_WARPS = 4;
 constexpr int REC_C = 8;  // value columns per warp
 
+// Sums of 8 values over the 32 lanes of a warp in 9 shuffles: at each of the offsets 16, 8, 4
+// a lane keeps half of its values and adds its partner's copy of them, then offsets 2 and 1
+// finish the sum.  Lane l returns the total of value (l >> 2) & 7.
+__device__ __forceinline__ float warp_sum8(const float (&v)[8], int lane) {
+  const bool h4 = lane & 16, h3 = lane & 8, h2 = lane & 4;
+  float a[4], b[2];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float send = h4 ? v[i] : v[i + 4];
+    a[i] = (h4 ? v[i + 4] : v[i]) + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float send = h3 ? a[i] : a[i + 2];
+    b[i] = (h3 ? a[i + 2] : a[i]) + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+  float c = (h2 ? b[1] : b[0]) + __shfl_xor_sync(0xffffffffu, h2 ? b[0] : b[1], 4);
+  c += __shfl_xor_sync(0xffffffffu, c, 2);
+  c += __shfl_xor_sync(0xffffffffu, c, 1);
+  return c;
+}
+
 template <typename T, int KPL>
 __global__ void __launch_bounds__(32 * REC_WARPS) gdn2_recurrent_kernel(Gdn2Args a) {
+  static_assert(REC_C == 8, "warp_sum8 reduces eight columns");
   constexpr int K = 32 * KPL;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long bh = blockIdx.y;
@@ -99,10 +123,11 @@ __global__ void __launch_bounds__(32 * REC_WARPS) gdn2_recurrent_kernel(Gdn2Args
       }
       r[c] = s;
     }
+    {  // r of column c sits in lanes 4c..4c+3; every lane needs all eight
+      const float rs = warp_sum8(r, lane);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-#pragma unroll
-      for (int c = 0; c < REC_C; ++c) r[c] += __shfl_xor_sync(0xffffffffu, r[c], off);
+      for (int c = 0; c < REC_C; ++c) r[c] = __shfl_sync(0xffffffffu, rs, 4 * c);
+    }
     float y[REC_C];
 #pragma unroll
     for (int c = 0; c < REC_C; ++c) {
@@ -114,13 +139,8 @@ __global__ void __launch_bounds__(32 * REC_WARPS) gdn2_recurrent_kernel(Gdn2Args
       }
       y[c] = s;
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-#pragma unroll
-      for (int c = 0; c < REC_C; ++c) y[c] += __shfl_xor_sync(0xffffffffu, y[c], off);
-#pragma unroll
-    for (int c = 0; c < REC_C; ++c)
-      if (lane == c && c < nc) st_out(o + (size_t)t * a.V + c, y[c]);
+    const float ys = warp_sum8(y, lane);
+    if ((lane & 3) == 0 && (lane >> 2) < nc) st_out(o + (size_t)t * a.V + (lane >> 2), ys);
   }
   if (a.S_out) {
     float* So = a.S_out + bh * K * a.V;
