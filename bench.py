@@ -912,7 +912,7 @@ def main():
                     r["peak"] = fp32_simt_peak_tflops(line["clocks"].get("sm_mhz"))
                     r["frac"] = r["achieved"] / r["peak"]
         line["gdn2"] = gdn2
-        line["gpu_launches"] += gdn2["steps"] * 3
+        line["gpu_launches"] += gdn2["steps"] * 4  # recurrent, chunk prep + scan, decode step
     if msr:
         wm, r = msr
         bms = dist_max(r["block_ms"], world)
