@@ -714,6 +714,39 @@ def run_gdn2(steps, warmup, flush_bytes, peaks, sm_mhz):
     return out
 
 
+def gdn2_over_ranks(gdn2, world, sm_mhz):
+    """The GDN-2 leg's numbers as the job's: each time is the slowest rank's (every rank runs
+    the same leg, so the all-reduces line up), throughputs summed over ranks, and the fp32
+    peak taken at the clock seen during the run."""
+    out = dict(gdn2)
+    for name, val in gdn2.items():
+        if not isinstance(val, dict):
+            continue
+        val = dict(val)
+        entries = [(mode, dict(val[mode])) for mode in ("recurrent", "chunk") if mode in val]
+        if not entries:  # decode: one entry at the top level
+            entries = [(None, val)]
+        for mode, e in entries:
+            ms_max = dist_max(e["ms_per_step"], world)
+            scale = e["ms_per_step"] / ms_max
+            e["ms_per_step"] = ms_max
+            e["value"] = e["value"] * scale * world
+            if "tokens_per_s" in e:
+                e["tokens_per_s"] = e["tokens_per_s"] * scale * world
+            r = dict(e["roofline"])
+            if r["bound"] == "alu":
+                r["peak"] = fp32_simt_peak_tflops(sm_mhz)
+            r["achieved"] = r["achieved"] * scale
+            r["frac"] = r["achieved"] / r["peak"]
+            e["roofline"] = r
+            if mode is None:
+                val = e
+            else:
+                val[mode] = e
+        out[name] = val
+    return out
+
+
 def backward_line(w, ms, sm_mhz, cpu: bool):
     step_ms = statistics.median(ms)
     flops = backward_flops(w.B, w.NH, w.S, w.dk, w.dv, w.num_blocks)
@@ -905,13 +938,7 @@ def main():
                             "reversal_bytes": copy_bytes}
         line["gpu_launches"] += len(rev_ms) * (cw["plan"]["kernels"] + (4 if w.retention else 6))
     if gdn2:
-        for val in gdn2.values():  # the fp32 peak at the clock seen during the run
-            for mode in ("recurrent", "chunk"):
-                if isinstance(val, dict) and mode in val:
-                    r = val[mode]["roofline"]
-                    r["peak"] = fp32_simt_peak_tflops(line["clocks"].get("sm_mhz"))
-                    r["frac"] = r["achieved"] / r["peak"]
-        line["gdn2"] = gdn2
+        line["gdn2"] = gdn2_over_ranks(gdn2, world, line["clocks"].get("sm_mhz"))
         line["gpu_launches"] += gdn2["steps"] * 4  # recurrent, chunk prep + scan, decode step
     if msr:
         wm, r = msr

@@ -78,3 +78,51 @@ def test_backward_flop_count_and_simt_peak():
     assert bench.backward_flops(1, 1, 1, 64, 32, 1) == 6 * 2 * 64 * 32
     assert bench.backward_flops(4, 4, 512, 32, 32, 2) == 4 * 4 * 512 * 2 * 12 * 32 * 32
     assert abs(bench.fp32_simt_peak_tflops(1965.0) - 148 * 128 * 2 * 1.965e9 / 1e12) < 1e-9
+
+
+def _fake_gdn2(rank):
+    ms_p, ms_c, ms_d = 2.0 + rank, 4.0 + 2 * rank, 0.1 * (1 + rank)
+    tokens, flops, nbytes = 1000.0, 9e9, 5e8
+    alu = lambda ms: {"bound": "alu", "achieved": flops / (ms * 1e-3) / 1e12, "peak": 1.0, "unit": "TFLOP/s",
+                      "frac": 0.0, "traffic": None}
+    return {"gdn2_prefill": {"workload": "w", "recurrent": {"value": tokens / (ms_p * 1e-3), "unit": "tokens/s",
+                                                            "ms_per_step": ms_p, "roofline": alu(ms_p)},
+                             "chunk": {"value": tokens / (ms_c * 1e-3), "unit": "tokens/s", "ms_per_step": ms_c,
+                                       "roofline": alu(ms_c)}},
+            "gdn2_decode": {"workload": "d", "value": nbytes / (ms_d * 1e-3) / 1e9, "unit": "GB/s",
+                            "ms_per_step": ms_d, "tokens_per_s": 256 / (ms_d * 1e-3),
+                            "roofline": {"bound": "hbm", "achieved": nbytes / (ms_d * 1e-3) / 1e9, "peak": 6535.4,
+                                         "unit": "GB/s", "frac": 0.0, "traffic": None}},
+            "steps": 5}
+
+
+def _gdn2_rank_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    bench.dist_setup(world)
+    out[rank] = bench.gdn2_over_ranks(_fake_gdn2(rank), world, 1965.0)
+    import torch.distributed as dist
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(120)
+def test_gdn2_leg_reports_the_slowest_rank_and_the_job_throughput():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_gdn2_rank_main, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    assert res[0] == res[1]
+    rec = res[0]["gdn2_prefill"]["recurrent"]
+    assert rec["ms_per_step"] == 3.0 and abs(rec["value"] - 2 * 1000 / 3e-3) < 1e-6 * rec["value"]
+    assert abs(rec["roofline"]["peak"] - bench.fp32_simt_peak_tflops(1965.0)) < 1e-9
+    assert abs(rec["roofline"]["achieved"] - 9e9 / 3e-3 / 1e12) < 1e-9
+    assert res[0]["gdn2_prefill"]["chunk"]["ms_per_step"] == 6.0
+    dec = res[0]["gdn2_decode"]
+    assert abs(dec["ms_per_step"] - 0.2) < 1e-12 and abs(dec["value"] - 2 * 5e8 / 0.2e-3 / 1e9) < 1e-6
+    assert abs(dec["roofline"]["achieved"] - 5e8 / 0.2e-3 / 1e9) < 1e-6 and dec["roofline"]["peak"] == 6535.4
+    # one rank: unchanged times and values
+    one = bench.gdn2_over_ranks(_fake_gdn2(0), 1, 1965.0)
+    assert one["gdn2_prefill"]["recurrent"]["ms_per_step"] == 2.0
+    assert abs(one["gdn2_prefill"]["recurrent"]["value"] - 1000 / 2e-3) < 1e-6
