@@ -33,7 +33,14 @@ Pins (tests/test_oracle_*.py) tie every function to something other than
 itself: closed forms, brute-force double loops, special cases and invariants.
 The per-block normaliser (num_blocks > 1) and the optional output gate o_t are
 fixed by this project's reading of the pages, not by them: parity unpinned
-for those two readings (their self-consistency is still tested).
+for those two readings (their self-consistency is still tested).  Likewise for
+the NEXT-row readings: the frequencies of Theta (theta_j = base^{-2j/D} on
+interleaved pairs; the pins fix the rotation's form and its relative-position
+property, not the frequency choice), and the GDN-2 update beyond what the page
+states (the pins fix the per-channel roles of the erase and write gates and the
+delta-rule property of the KDA reduction it names; the order decay -> erase ->
+write and the erase vector b o k are readings): parity unpinned by the pages
+for those parts.  GroupNorm and SiLU are pinned by torch's routines.
 """
 from __future__ import annotations
 
