@@ -295,3 +295,23 @@ def test_gdn2_validation():
     assert gdn2_call(mode=1, chunk=8) == 5                          # no workspace
     assert gdn2_call(mode=1, chunk=8, ws=H_, ws_bytes=16) == 5      # too small
     assert gdn2_call(mode=1, chunk=8, ws=A, ws_bytes=1 << 30) == 7  # workspace over q
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/mlstm.h is a C header: it compiles as pedantic C99 with no CUDA headers and
+    declares every type the entry points use."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "mlstm.h"\n'
+                   "int main(void) {\n"
+                   "  mlstm_fwd_params_t f; mlstm_step_params_t s; mlstm_gdn2_params_t g; mlstm_fwd_plan_t p;\n"
+                   "  (void)f; (void)s; (void)g; (void)p;\n"
+                   "  return (int)MLSTM_OK + (int)MLSTM_GDN2_CHUNK * 0;\n"
+                   "}\n")
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", f"{ROOT}/include",
+                        "-fsyntax-only", str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
