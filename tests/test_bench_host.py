@@ -126,3 +126,22 @@ def test_gdn2_leg_reports_the_slowest_rank_and_the_job_throughput():
     one = bench.gdn2_over_ranks(_fake_gdn2(0), 1, 1965.0)
     assert one["gdn2_prefill"]["recurrent"]["ms_per_step"] == 2.0
     assert abs(one["gdn2_prefill"]["recurrent"]["value"] - 1000 / 2e-3) < 1e-6
+
+
+def test_gdn2_inputs_follow_their_recipe():
+    from linear_recurrent_token_b200 import inputs
+    x = inputs.gdn2_inputs(2, 3, 50, 16, 8, "bf16", seed=1)
+    import numpy as np
+    assert x["q"].shape == (2, 3, 50, 16) and x["v"].shape == (2, 3, 50, 8) and x["S0"].shape == (2, 3, 16, 8)
+    np.testing.assert_allclose(np.linalg.norm(x["k"], axis=-1), 1.0, rtol=1e-2)  # unit keys (bf16-rounded)
+    assert np.all(x["g"] < 0) and np.all((x["b"] >= 0) & (x["b"] <= 1)) and np.all((x["w"] >= 0) & (x["w"] <= 1))
+    # stored values are exact in the storage type
+    import torch
+    assert np.array_equal(torch.from_numpy(x["q"]).to(torch.bfloat16).float().numpy(), x["q"])
+    assert inputs.gdn2_inputs(1, 1, 3, 8, 8, "f32", seed=1, with_state=False)["S0"] is None
+
+
+def test_gdn2_flop_count():
+    # decay K V, read-out 2 K V, erase + write 4 K V, output 2 K V per token and head
+    assert bench.gdn2_flops(1, 1, 1, 128, 128) == 9 * 128 * 128
+    assert bench.gdn2_flops(8, 16, 2048, 128, 128) == 38_654_705_664
