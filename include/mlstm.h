@@ -31,7 +31,9 @@
  *   - Every data pointer is DEVICE memory owned by the caller.  The library never
  *     allocates, frees or keeps a pointer past the call.  Scratch memory of the
  *     prefill is a caller-supplied workspace sized by
- *     mlstm_fwd_chunkwise_workspace_size().
+ *     mlstm_fwd_chunkwise_workspace_size().  (One exception, for callers that cannot
+ *     allocate: mlstm_fwd_chunkwise_noalloc uses a scratch buffer built into the
+ *     library instead; see there.)
  *   - All tensors are dense, row-major (last index fastest), 16-byte aligned.
  *   - q, k, v, o, h use the dtype of the params (fp32 or bf16); gates are always
  *     fp32; the state (C, n, m) is always fp32.
@@ -39,8 +41,16 @@
  *   - Arguments are validated on the host before anything is enqueued; on any
  *     error nothing is enqueued and no output is touched.  Errors raised by the
  *     CUDA runtime at launch are returned as MLSTM_ERR_CUDA.
+ *   - Device-side waits are bounded.  The tensor-core prefill kernels wait on
+ *     mbarriers for their own copies and tensor-core results; each wait gives up
+ *     after params->wait_limit_cycles SM cycles (0 = about 4e9, ~2 s).  A wait that
+ *     runs out is reported after the work, by mlstm_fwd_chunkwise_status
+ *     (MLSTM_ERR_TIMEOUT), never by a hang: the kernel stops issuing work, waits for
+ *     the copies it has in flight, frees its tensor memory and returns.
  *   - Calls that share no output buffer may run concurrently on different
- *     streams.  The library holds no global mutable state.
+ *     streams.  The library holds no global mutable state, except the built-in
+ *     scratch buffer of mlstm_fwd_chunkwise_noalloc: calls of that entry point
+ *     whose GPU work overlaps race on it, so they must not overlap.
  */
 #ifndef MLSTM_H_
 #define MLSTM_H_
@@ -63,7 +73,9 @@ typedef enum {
   MLSTM_ERR_ALIGN = 4,      /* a pointer is not 16-byte aligned                    */
   MLSTM_ERR_WORKSPACE = 5,  /* workspace NULL or smaller than the size query       */
   MLSTM_ERR_CUDA = 6,       /* the CUDA runtime reported an error at launch        */
-  MLSTM_ERR_ALIAS = 7       /* an output overlaps an input it must not overlap     */
+  MLSTM_ERR_ALIAS = 7,      /* an output overlaps an input it must not overlap     */
+  MLSTM_ERR_TIMEOUT = 8     /* a bounded device-side wait ran out (reported by the
+                               status calls after the work has finished)           */
 } mlstm_status_t;
 
 typedef enum { MLSTM_F32 = 0, MLSTM_BF16 = 1 } mlstm_dtype_t;
@@ -71,13 +83,18 @@ typedef enum { MLSTM_F32 = 0, MLSTM_BF16 = 1 } mlstm_dtype_t;
 /* Sizes of one chunkwise prefill.  B, NH >= 0; S >= 0; DHQK, DHV >= 1 and
  * divisible by num_blocks (>= 1); chunk >= 1 (the intra-chunk tile length; the
  * result does not depend on it beyond rounding; S need not be a multiple of it).
- * retention: 0 = mLSTM, 1 = retention. */
+ * retention: 0 = mLSTM, 1 = retention.
+ * wait_limit_cycles: bound of each device-side wait of the tensor-core kernels in SM
+ * cycles; 0 (or negative) = the default, about 4e9 (~2 s).  Only tests and watchdogs
+ * set it: a limit shorter than a copy takes makes the call fail with MLSTM_ERR_TIMEOUT
+ * (see mlstm_fwd_chunkwise_status).  Ignored by the other entry points. */
 typedef struct {
   int B, NH, S, DHQK, DHV;
   int chunk;
   int num_blocks;
   mlstm_dtype_t dtype;
   int retention;
+  long long wait_limit_cycles;
 } mlstm_fwd_params_t;
 
 /* Sizes of one decode step (one token per sequence). */
@@ -164,7 +181,9 @@ mlstm_status_t mlstm_fwd_chunkwise_timed(const mlstm_fwd_params_t* p,
  * holds (see mlstm_fwd_chunkwise_workspace_size).  The first call on a device looks up
  * the buffer's device address (cudaGetSymbolAddress) and caches it; make that first
  * call before any stream capture.  Nothing is allocated or freed.  All calls share the
- * buffer: calls whose GPU work overlaps (other streams, other host threads) race.
+ * buffer: calls whose GPU work overlaps (other streams, other host threads) race.  The
+ * buffer used is the one of the CURRENT device, so every pointer must be memory of the
+ * current device.  Bounded-wait failures are read with mlstm_fwd_chunkwise_noalloc_status.
  */
 mlstm_status_t mlstm_fwd_chunkwise_noalloc(const mlstm_fwd_params_t* p,
                                            const void* q, const void* k, const void* v,
@@ -175,6 +194,26 @@ mlstm_status_t mlstm_fwd_chunkwise_noalloc(const mlstm_fwd_params_t* p,
 
 /* Size in bytes of the built-in scratch buffer used by mlstm_fwd_chunkwise_noalloc. */
 size_t mlstm_noalloc_scratch_bytes(void);
+
+/*
+ * Outcome of the bounded device-side waits of the last prefill enqueued on `stream` with
+ * `workspace` (mlstm_fwd_chunkwise, _timed, _reversed or _msr, called with the same params):
+ * synchronises `stream`, then reads the error word the tensor-core kernels keep in the first
+ * bytes of the workspace (each prefill call clears it first).
+ *   MLSTM_OK           no wait ran out (always, for sizes that run the SIMT kernels, which
+ *                      have no such waits)
+ *   MLSTM_ERR_TIMEOUT  a wait ran out (params->wait_limit_cycles); that call's outputs and
+ *                      final state are unspecified, the workspace can be used again
+ *   MLSTM_ERR_CUDA     the synchronisation or the read failed (for example an earlier
+ *                      asynchronous error on the stream)
+ *   MLSTM_ERR_NULL / _SHAPE / _DTYPE as for mlstm_fwd_chunkwise (workspace NULL: _NULL when
+ *                      the sizes have a workspace)
+ * mlstm_fwd_chunkwise_noalloc_status does the same for mlstm_fwd_chunkwise_noalloc, reading
+ * the built-in scratch buffer of the current device.
+ */
+mlstm_status_t mlstm_fwd_chunkwise_status(const mlstm_fwd_params_t* p, const void* workspace,
+                                          mlstm_stream_t stream);
+mlstm_status_t mlstm_fwd_chunkwise_noalloc_status(const mlstm_fwd_params_t* p, mlstm_stream_t stream);
 
 /*
  * The same prefill over the reversed sequence: token S-1 is read first and token 0 last;

@@ -46,7 +46,7 @@ namespace {
 constexpr int L = 64;            // chunk length of the tensor-core path
 constexpr int NTA = 192;         // phase A threads per CTA (producer, MMA warp, 4 SIMT warps)
 constexpr int NSA = 4;           // phase A TMA stages
-constexpr long long WAIT = 4000000000LL;
+constexpr long long WAIT_DEFAULT = 4000000000LL;  // bound of a wait unless the caller sets one (~2 s)
 
 struct TcParams {
   int S, NH, nb, dk, dv, DHQK, DHV, retention, dtype;
@@ -63,6 +63,7 @@ struct TcParams {
   float *gb, *gx, *gxc, *cg, *cxm;
   int sp, ncp;
   unsigned int* err;
+  long long wait;  // bound of every mbarrier wait, SM cycles
 };
 
 // Lane / row mapping of an M-row accumulator: thread (warp w, lane l) owns row
@@ -131,22 +132,23 @@ __device__ __forceinline__ uint32_t split_bf16x2(float a, float b, uint32_t* lo)
 // every lane polls with the bounded wait unless a failure is already recorded; returns the
 // warp's verdict and records a failure.  Out of line, so the per-chunk code keeps only the
 // test and the vote.
-__device__ __noinline__ bool warp_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  const bool ok = !*abort_flag && mbar_wait(bar, parity, WAIT);
+__device__ __noinline__ bool warp_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                            long long limit) {
+  const bool ok = !*abort_flag && mbar_wait(bar, parity, limit);
   if (!ok) *abort_flag = 1;
   return __all_sync(0xffffffffu, ok);
 }
 // The same for up to three barriers (unused ones null): each round tests all of them at once,
 // so the warp resumes one shared-memory round trip after the last phase completes.
 __device__ __noinline__ bool warp_wait_slow3(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1, uint64_t* b2,
-                                             uint32_t p2, volatile int* abort_flag) {
+                                             uint32_t p2, volatile int* abort_flag, long long limit) {
   bool ok = !*abort_flag;
   const long long t0 = clock64();
   while (ok) {
     const bool x = mbar_test_wait(b0, p0), y = b1 == nullptr || mbar_test_wait(b1, p1),
                z = b2 == nullptr || mbar_test_wait(b2, p2);
     if (x && y && z) break;
-    if (clock64() - t0 > WAIT) ok = false;
+    if (clock64() - t0 > limit) ok = false;
   }
   if (!ok) *abort_flag = 1;
   return __all_sync(0xffffffffu, ok);
@@ -275,7 +277,7 @@ __global__ void __launch_bounds__(NTA, 1)
   float* dnp = reinterpret_cast<float*>(sm + NS * (KB + VB));  // [128 * 8] partial sums of dn
   float* omb = dnp + 128 * 8;                                   // [NS][L] weights of the stage's chunk
   float* coff = omb + NS * L;                                   // [seg_chunks]
-  __shared__ uint64_t full[NS], scaled[NS], mma_done[NS], all_done;
+  __shared__ uint64_t full[NS], scaled[NS], mma_done[NS], all_done, drain;
   __shared__ uint32_t tmem_base;
   __shared__ float red[NTA / 32];
   __shared__ volatile int abort_flag;
@@ -299,6 +301,7 @@ __global__ void __launch_bounds__(NTA, 1)
       mbar_init(&mma_done[i], 1);
     }
     mbar_init(&all_done, 1);
+    mbar_init(&drain, 1);
     abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&mapK);
@@ -319,8 +322,12 @@ __global__ void __launch_bounds__(NTA, 1)
       tma_load_3d(kb + KB + j * 8192, &mapV, blk * p.dv + v0 + 64 * j, T0 + c * L, bh, &full[st]);
   };
   // K and V are inputs: the first stages load while the previous kernel finishes
+  int n_issued = 0;  // chunks whose loads thread 0 has issued
   if (tid == 0)
-    for (int c = 0; c < NS && c < nck; ++c) issue(c);
+    for (int c = 0; c < NS && c < nck; ++c) {
+      issue(c);
+      n_issued = c + 1;
+    }
 
   grid_dep_launch();
   grid_dep_wait();  // the gate planes come from the preparation kernel
@@ -361,7 +368,7 @@ __global__ void __launch_bounds__(NTA, 1)
   }
   // warp-uniform test of a barrier, bounded wait out of line when the phase is not complete
   auto warp_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
-    return __all_sync(0xffffffffu, mbar_test_wait(bar, parity)) || warp_wait_slow(bar, parity, &abort_flag);
+    return __all_sync(0xffffffffu, mbar_test_wait(bar, parity)) || warp_wait_slow(bar, parity, &abort_flag, p.wait);
   };
 
   if (warp == 0) {
@@ -375,7 +382,10 @@ __global__ void __launch_bounds__(NTA, 1)
       if (c >= NS) {
         // the stage's previous chunk has been read by its MMAs (and by the SIMT group before)
         if (!warp_wait(&mma_done[st], ((c / NS) - 1) & 1)) break;
-        if (lane == 0) issue(c);
+        if (lane == 0) {
+          issue(c);
+          n_issued = c + 1;
+        }
       }
       const float cf = coff[c];
       *reinterpret_cast<float2*>(omb + st * L + 2 * lane) = make_float2(expf(cf + gxn.x), expf(cf + gxn.y));
@@ -419,7 +429,7 @@ __global__ void __launch_bounds__(NTA, 1)
       // a failed wait leaves the loop of no warp: it runs on (later waits return at once)
       // and the error flag reports it
       if (!__all_sync(0xffffffffu, mbar_test_wait(&full[st], (c / NS) & 1)))
-        warp_wait_slow(&full[st], (c / NS) & 1, &abort_flag);
+        warp_wait_slow(&full[st], (c / NS) & 1, &abort_flag, p.wait);
       {
         // V rows scaled in place by omega (loads batched ahead of the stores)
         constexpr int NV = L * (DVT / 8) / 128;
@@ -456,7 +466,7 @@ __global__ void __launch_bounds__(NTA, 1)
       if (lane == 0) mbar_arrive(&scaled[st]);
     }
     // ---- epilogue: the accumulator (warp w reads TMEM lane quarter w % 4) and dn
-    if (!__all_sync(0xffffffffu, mbar_test_wait(&all_done, 0))) warp_wait_slow(&all_done, 0, &abort_flag);
+    if (!__all_sync(0xffffffffu, mbar_test_wait(&all_done, 0))) warp_wait_slow(&all_done, 0, &abort_flag, p.wait);
     tc_fence_after();
     const int quarter = warp & 3;
     const int row = acc_row<DVT>(quarter, lane);
@@ -482,9 +492,26 @@ __global__ void __launch_bounds__(NTA, 1)
       }
     }
   }
+  // Drain before TMEM is freed and the CTA exits: every MMA issued and every TMA load issued has
+  // completed (after an expired wait the loops above may have stopped early).  These waits use
+  // the default bound whatever the caller's limit: they end as soon as the copies land.
+  if (warp == 1) {
+    if (elect_one()) mma_commit(&drain);
+    __syncwarp();
+  }
   tc_fence_before();
   __syncthreads();
-  if (abort_flag && tid == 0) atomicOr(p.err, 1u);
+  if (tid == 0) {
+    bool ok = mbar_wait(&drain, 0, WAIT_DEFAULT);
+    for (int st = 0; st < NS; ++st)
+      if (n_issued > st) {
+        const int c_last = st + NS * ((n_issued - 1 - st) / NS);
+        ok = mbar_wait(&full[st], (c_last / NS) & 1, WAIT_DEFAULT) && ok;
+      }
+    if (!ok) abort_flag = 1;
+    if (abort_flag) atomicOr(p.err, 1u);
+  }
+  __syncthreads();
   if (warp == 0) tmem_dealloc(tm, DK);
 }
 
@@ -558,6 +585,7 @@ constexpr int GF_GUARD = 1, GF_STORE_C = 2;
 struct WalkBars {
   uint64_t full[2], empty[2], s_full[2], gfull[NGB], gempty[NGB], q_ready[NGB];
   uint64_t cb_ready, vw_full, upd_done, ro_done, h_empty, s_empty, p_full, mm_done;
+  uint64_t drain;  // both MMA warps' last commits, before TMEM is freed
 };
 
 template <int DK, int DVT>
@@ -618,6 +646,7 @@ __global__ void __launch_bounds__(NTW, 1)
     mbar_init(&bars.s_empty, 4);
     mbar_init(&bars.p_full, 4);
     mbar_init(&bars.mm_done, 1);
+    mbar_init(&bars.drain, 2);
     abort_flag = 0;
     group_flag[0] = group_flag[1] = 0;
     fence_mbar_init();
@@ -701,7 +730,7 @@ __global__ void __launch_bounds__(NTW, 1)
 
   // group-uniform bounded wait: the group's first thread waits, the group follows its verdict
   auto group_wait = [&](uint64_t* bar, uint32_t parity, int gi, bool first) -> bool {
-    if (first && (abort_flag || !mbar_wait(bar, parity, WAIT))) {
+    if (first && (abort_flag || !mbar_wait(bar, parity, p.wait))) {
       group_flag[gi] = 1;
       abort_flag = 1;
     }
@@ -713,21 +742,22 @@ __global__ void __launch_bounds__(NTW, 1)
   // followed by a shuffle costs several, and under the SIMT groups' load each takes hundreds
   // of cycles); otherwise the lanes poll with the bounded wait.
   auto warp_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
-    return __all_sync(0xffffffffu, mbar_test_wait(bar, parity)) || warp_wait_slow(bar, parity, &abort_flag);
+    return __all_sync(0xffffffffu, mbar_test_wait(bar, parity)) || warp_wait_slow(bar, parity, &abort_flag, p.wait);
   };
   // wait of one warp of a SIMT group.  Warps of a group wait independently (no verdict is
   // shared), so group code never leaves its loop on a failed wait: it runs on, every later
   // wait returns at once, and the error flag reports the failure.  Named barriers stay only
   // where data crosses warps.
   auto gwait = [&](uint64_t* bar, uint32_t parity) {
-    if (!__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) warp_wait_slow(bar, parity, &abort_flag);
+    if (!__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) warp_wait_slow(bar, parity, &abort_flag, p.wait);
   };
   // two barriers tested at once (both tests in flight together)
   auto warp_wait2 = [&](uint64_t* b1, uint32_t p1, uint64_t* b2, uint32_t p2) -> bool {
     const bool x = mbar_test_wait(b1, p1), y = mbar_test_wait(b2, p2);
     if (__all_sync(0xffffffffu, x && y)) return true;
-    return warp_wait_slow3(b1, p1, b2, p2, nullptr, 0, &abort_flag);
+    return warp_wait_slow3(b1, p1, b2, p2, nullptr, 0, &abort_flag, p.wait);
   };
+  int n_issued = 0;  // chunks whose Q/K/V loads the producer (thread 0) has issued
   const uint32_t id_s = idesc_bf16(64, 64, 0, 0);
   const uint32_t id_ro = idesc_bf16(DVT, 64, 0, 0);
   const uint32_t id_pv = idesc_bf16(DVT, 64, 1, 0);
@@ -820,6 +850,7 @@ __global__ void __launch_bounds__(NTW, 1)
         }
         for (int j = 0; j < DVT / 64; ++j)
           tma_load_3d(base + SM::QB + SM::KB + j * 8192, &mapV, blk * p.dv + v0 + 64 * j, t0, bh, &bars.full[b]);
+        n_issued = c + 1;
       }
       // gate quantities of chunk c into buffer gi (lane: tokens 2 lane, 2 lane + 1)
       if (!warp_wait(&bars.gempty[gi], ((c / NGB) & 1) ^ 1)) break;
@@ -896,7 +927,7 @@ __global__ void __launch_bounds__(NTW, 1)
                    z = mbar_test_wait(&bars.full[b], (c >> 1) & 1);
         h_free = c == 0 || mbar_test_wait(&bars.h_empty, (c - 1) & 1);
         if (!__all_sync(0xffffffffu, x && y && z) &&
-            !warp_wait_slow3(&bars.cb_ready, c & 1, &bars.vw_full, c & 1, &bars.full[b], (c >> 1) & 1, &abort_flag))
+            !warp_wait_slow3(&bars.cb_ready, c & 1, &bars.vw_full, c & 1, &bars.full[b], (c >> 1) & 1, &abort_flag, p.wait))
           break;
       }
       tc_fence_after();
@@ -913,7 +944,7 @@ __global__ void __launch_bounds__(NTW, 1)
       const bool guard = (flags & GF_GUARD) != 0;
       if (guard || !__all_sync(0xffffffffu, h_free)) {
         if (!warp_wait_slow3(&bars.h_empty, (c - 1) & 1, guard ? &bars.q_ready[gi] : nullptr, (c / NGB) & 1, nullptr, 0,
-                             &abort_flag))
+                             &abort_flag, p.wait))
           break;
         tc_fence_after();
       }
@@ -999,7 +1030,7 @@ __global__ void __launch_bounds__(NTW, 1)
       if (c > 0) {
         const bool x = mbar_test_wait(&bars.gfull[gi], (c / NGB) & 1), y = mbar_test_wait(&bars.ro_done, (c - 1) & 1);
         if (!__all_sync(0xffffffffu, x && y))
-          warp_wait_slow3(&bars.gfull[gi], (c / NGB) & 1, &bars.ro_done, (c - 1) & 1, nullptr, 0, &abort_flag);
+          warp_wait_slow3(&bars.gfull[gi], (c / NGB) & 1, &bars.ro_done, (c - 1) & 1, nullptr, 0, &abort_flag, p.wait);
       } else {
         gwait(&bars.gfull[gi], 0);
       }
@@ -1020,7 +1051,7 @@ __global__ void __launch_bounds__(NTW, 1)
                    y = mbar_test_wait(&bars.full[b1], (c1 >> 1) & 1), z = mbar_test_wait(&bars.upd_done, c & 1);
         if (!__all_sync(0xffffffffu, x && y && z))
           warp_wait_slow3(&bars.gfull[c1 % NGB], (c1 / NGB) & 1, &bars.full[b1], (c1 >> 1) & 1, &bars.upd_done, c & 1,
-                          &abort_flag);
+                          &abort_flag, p.wait);
         scale_v(c1);
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.vw_full);
@@ -1065,7 +1096,7 @@ __global__ void __launch_bounds__(NTW, 1)
                    y = mbar_test_wait(&bars.s_full[b], (c >> 1) & 1), z = mbar_test_wait(&bars.gfull[gi], (c / NGB) & 1);
         if (!__all_sync(0xffffffffu, x && y && z))
           warp_wait_slow3(&bars.s_full[b], (c >> 1) & 1, &bars.gfull[gi], (c / NGB) & 1,
-                          c > 0 ? &bars.mm_done : nullptr, (c - 1) & 1, &abort_flag);
+                          c > 0 ? &bars.mm_done : nullptr, (c - 1) & 1, &abort_flag, p.wait);
       }
       tc_fence_after();
       {
@@ -1226,7 +1257,7 @@ __global__ void __launch_bounds__(NTW, 1)
                    y = c == 0 || mbar_test_wait(&bars.ro_done, (c - 1) & 1);
         if (!__all_sync(0xffffffffu, x && y))
           warp_wait_slow3(&bars.gfull[gi], (c / NGB) & 1, c > 0 ? &bars.ro_done : nullptr, (c - 1) & 1, nullptr, 0,
-                          &abort_flag);
+                          &abort_flag, p.wait);
       }
       tc_fence_after();
       const int flags = __float_as_int(G.scal[0]);
@@ -1235,7 +1266,7 @@ __global__ void __launch_bounds__(NTW, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.cb_ready);
       if (!__all_sync(0xffffffffu, mbar_test_wait(&bars.full[b], (c >> 1) & 1)))
-        warp_wait_slow(&bars.full[b], (c >> 1) & 1, &abort_flag);
+        warp_wait_slow(&bars.full[b], (c >> 1) & 1, &abort_flag, p.wait);
       const bool guard = (flags & GF_GUARD) != 0;
       fin = G.scal[4];
       if (!ret) {
@@ -1324,8 +1355,25 @@ __global__ void __launch_bounds__(NTW, 1)
       for (int col = nt; col < DK; col += 128) p.n_out[(size_t)slice * p.dk + col] = fin * nvec[col];
   }
 
-  if (abort_flag && tid == 0) atomicOr(p.err, 2u);
+  // Drain before TMEM is freed and the CTA exits: every MMA issued and every Q/K/V load issued
+  // has completed (after an expired wait the role loops may have stopped early; the h stores
+  // were waited for by the output group).  Default bound whatever the caller's limit.
+  if (warp == 1 || warp == 2) {
+    if (elect_one()) mma_commit(&bars.drain);
+    __syncwarp();
+  }
   tc_fence_before();
+  __syncthreads();
+  if (tid == 0) {
+    bool ok = mbar_wait(&bars.drain, 0, WAIT_DEFAULT);
+    for (int b = 0; b < 2; ++b)
+      if (n_issued > b) {
+        const int c_last = b + 2 * ((n_issued - 1 - b) / 2);
+        ok = mbar_wait(&bars.full[b], (c_last >> 1) & 1, WAIT_DEFAULT) && ok;
+      }
+    if (!ok) abort_flag = 1;
+    if (abort_flag) atomicOr(p.err, 2u);
+  }
   __syncthreads();
   if (warp == 0) tmem_dealloc(tm, TM_COLS);
 }
@@ -1466,6 +1514,7 @@ cudaError_t launch_tc(const WalkArgs& a, const TcPlan& pl, void* ws, cudaStream_
   off += ((size_t)BH * G1 * 4 + 255) / 256 * 256;
   prm.ncp = pl.G * pl.seg_chunks;
   prm.sp = prm.ncp * L;
+  prm.wait = a.wait_cycles > 0 ? a.wait_cycles : WAIT_DEFAULT;
   float** planes[5] = {&prm.gb, &prm.gx, &prm.gxc, &prm.cg, &prm.cxm};
   for (int i = 0; i < 5; ++i) {
     *planes[i] = reinterpret_cast<float*>(w + off);

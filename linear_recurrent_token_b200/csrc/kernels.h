@@ -22,6 +22,7 @@ struct WalkArgs {
                              // then n_init / n_out hold one value per (batch, head)
   void *h;
   float *C_out, *n_out, *m_out;
+  long long wait_cycles;     // bound of each device-side wait (tensor-core path); 0 = default
 };
 
 // The steps either side of retention (msr.cu): the rotation Theta of q and k by position
@@ -76,7 +77,7 @@ int tc_num_sms();
 TcPlan tc_plan(int B, int NH, int S, int nb, int dk, int dv, int num_sms);
 size_t tc_workspace_bytes(const TcPlan& pl, long long BH, int nb, int dk, int dv);
 // ws: workspace of at least tc_workspace_bytes bytes; its first 4 bytes become an error
-// word (0 = ok; nonzero = a bounded wait expired).  ev0/ev1 (may be NULL) are recorded
+// word (0 = ok; nonzero = a bounded wait expired), cleared on the stream before the kernels.  ev0/ev1 (may be NULL) are recorded
 // around the walk kernel.
 cudaError_t launch_tc(const WalkArgs& a, const TcPlan& pl, void* ws, cudaStream_t stream, cudaEvent_t ev0,
                       cudaEvent_t ev1);

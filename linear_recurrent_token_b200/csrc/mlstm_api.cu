@@ -199,6 +199,7 @@ mlstm_status_t fwd_impl(const mlstm_fwd_params_t* p, const void* q, const void* 
   a.C_out = C_out;
   a.n_out = n_out;
   a.m_out = m_out;
+  a.wait_cycles = p->wait_limit_cycles;
   if (s.tc) {
     // snapshots: the walk writes n_out / m_out (and C_out across segments) while other
     // CTAs may still read n0 / m0 / C0, which the caller may have aliased to them
@@ -247,10 +248,10 @@ struct MsrLayout {
 MsrLayout msr_layout(const FwdShape& s) {
   MsrLayout r = {0, 0, 0, 0};
   const size_t bq = (size_t)s.BH * s.S * s.DHQK * s.esize;
-  r.qr = 0;
-  r.kr = align_up(bq);
-  r.fwd = r.kr + align_up(bq);
-  r.total = r.fwd + fwd_layout(s).total;
+  r.fwd = 0;  // first, so that its error word sits at the start (mlstm_fwd_chunkwise_status)
+  r.qr = align_up(fwd_layout(s).total);
+  r.kr = r.qr + align_up(bq);
+  r.total = r.kr + align_up(bq);
   return r;
 }
 
@@ -304,7 +305,7 @@ mlstm_status_t check_bwd(const mlstm_fwd_params_t* p, FwdShape* s) {
 
 extern "C" {
 
-int mlstm_abi_version(void) { return (1 << 16) | 0; }
+int mlstm_abi_version(void) { return (2 << 16) | 0; }
 
 const char* mlstm_status_string(mlstm_status_t s) {
   switch (s) {
@@ -316,6 +317,7 @@ const char* mlstm_status_string(mlstm_status_t s) {
     case MLSTM_ERR_WORKSPACE: return "workspace missing or too small";
     case MLSTM_ERR_CUDA: return "CUDA runtime error at launch";
     case MLSTM_ERR_ALIAS: return "an output overlaps an input";
+    case MLSTM_ERR_TIMEOUT: return "a bounded device-side wait ran out";
   }
   return "unknown status";
 }
@@ -365,6 +367,26 @@ mlstm_status_t mlstm_fwd_chunkwise_timed(const mlstm_fwd_params_t* p, const void
                                          mlstm_stream_t stream, mlstm_event_t main_begin, mlstm_event_t main_end) {
   return fwd_impl(p, q, k, v, igate, fgate, ogate, C0, n0, m0, h, C_out, n_out, m_out, workspace, workspace_bytes,
                   (cudaStream_t)stream, (cudaEvent_t)main_begin, (cudaEvent_t)main_end);
+}
+
+// Error word of the tensor-core kernels (0 = every bounded wait succeeded), read after the
+// stream's work has finished.  `ws` is the forward's workspace (its error word comes first).
+static mlstm_status_t read_error_word(const FwdShape& s, const void* ws, cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MLSTM_ERR_CUDA;
+  if (!s.tc || s.BH == 0 || s.S == 0) return MLSTM_OK;  // no bounded waits ran
+  unsigned int word = 0;
+  const char* base = static_cast<const char*>(ws) + fwd_layout(s).tc;
+  if (cudaMemcpy(&word, base, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return MLSTM_ERR_CUDA;
+  return word == 0 ? MLSTM_OK : MLSTM_ERR_TIMEOUT;
+}
+
+mlstm_status_t mlstm_fwd_chunkwise_status(const mlstm_fwd_params_t* p, const void* workspace,
+                                          mlstm_stream_t stream) {
+  FwdShape s;
+  mlstm_status_t st = check_fwd(p, &s);
+  if (st != MLSTM_OK) return st;
+  if (s.tc && s.BH > 0 && s.S > 0 && !workspace) return MLSTM_ERR_NULL;
+  return read_error_word(s, workspace, (cudaStream_t)stream);
 }
 
 // Workspace of the reversed-sequence pass: the forward's, then reversed copies of the
@@ -881,7 +903,8 @@ void* g_noalloc_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device.  The host-side name of a
 // __device__ array is only a stand-in, so the address is looked up once per device,
-// with that device current, and cached.
+// with that device current, and cached.  (A cudaDeviceReset would make the cached
+// address stale; the library's users do not reset devices while it is loaded.)
 mlstm_status_t noalloc_scratch(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLSTM_ERR_CUDA;
@@ -915,6 +938,16 @@ mlstm_status_t mlstm_fwd_chunkwise_noalloc(const mlstm_fwd_params_t* p, const vo
   if (st != MLSTM_OK) return st;
   return fwd_impl(p, q, k, v, igate, fgate, ogate, C0, n0, m0, h, C_out, n_out, m_out, scratch,
                   MLSTM_NOALLOC_SCRATCH_BYTES, (cudaStream_t)stream, nullptr, nullptr);
+}
+
+mlstm_status_t mlstm_fwd_chunkwise_noalloc_status(const mlstm_fwd_params_t* p, mlstm_stream_t stream) {
+  FwdShape s;
+  mlstm_status_t st = check_fwd(p, &s);
+  if (st != MLSTM_OK) return st;
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != MLSTM_OK) return st;
+  return read_error_word(s, scratch, (cudaStream_t)stream);
 }
 
 }  // extern "C"

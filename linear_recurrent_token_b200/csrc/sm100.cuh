@@ -50,31 +50,38 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+// The suspend-time hint (ns) lets the waiting thread sleep in hardware until the phase
+// completes instead of spinning on issue slots other warps need.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, uint32_t hint_ns = 1000000u) {
   uint32_t ok;
-  // the suspend-time hint (ns) lets the waiting thread sleep in hardware until the phase
-  // completes instead of spinning on issue slots other warps need
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
+}
+// Suspend hint for a wait bounded by `limit_cycles`: at most 1 ms, and never longer than the
+// limit itself (an SM cycle is at least half a nanosecond), so a short limit really ends the
+// wait after about that many cycles.
+__device__ __forceinline__ uint32_t wait_hint_ns(long long limit_cycles) {
+  return limit_cycles >= 2000000LL ? 1000000u : (uint32_t)(limit_cycles > 1 ? limit_cycles / 2 : 1);
 }
 // Bounded wait on phase `parity`.  Gives up after ~`limit_cycles` SM cycles and
 // returns false (the caller records an error and winds down instead of hanging).
 // The polling loop is out of line: kernels with many wait sites keep one copy of it, which
 // stays in the instruction cache.
 __device__ __noinline__ bool mbar_wait_loop(uint64_t* bar, uint32_t parity, long long limit_cycles) {
+  const uint32_t hint = wait_hint_ns(limit_cycles);
   const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity))
+  while (!mbar_try_wait(bar, parity, hint))
     if (clock64() - t0 > limit_cycles) return false;
   return true;
 }
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit_cycles = 4000000000LL) {
-  if (mbar_try_wait(bar, parity)) return true;
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit_cycles) {
+  if (mbar_try_wait(bar, parity, wait_hint_ns(limit_cycles))) return true;
   return mbar_wait_loop(bar, parity, limit_cycles);
 }
 

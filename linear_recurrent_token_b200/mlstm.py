@@ -23,7 +23,7 @@ _DTYPES = {torch.float32: MLSTM_F32, torch.bfloat16: MLSTM_BF16}
 class FwdParams(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("NH", ctypes.c_int), ("S", ctypes.c_int), ("DHQK", ctypes.c_int),
                 ("DHV", ctypes.c_int), ("chunk", ctypes.c_int), ("num_blocks", ctypes.c_int),
-                ("dtype", ctypes.c_int), ("retention", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("retention", ctypes.c_int), ("wait_limit_cycles", ctypes.c_longlong)]
 
 
 class StepParams(ctypes.Structure):
@@ -72,6 +72,10 @@ def lib():
         L.mlstm_fwd_chunkwise_timed.restype = I
         L.mlstm_fwd_chunkwise_noalloc.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 13 + [P]
         L.mlstm_fwd_chunkwise_noalloc.restype = I
+        L.mlstm_fwd_chunkwise_status.argtypes = [ctypes.POINTER(FwdParams), P, P]
+        L.mlstm_fwd_chunkwise_status.restype = I
+        L.mlstm_fwd_chunkwise_noalloc_status.argtypes = [ctypes.POINTER(FwdParams), P]
+        L.mlstm_fwd_chunkwise_noalloc_status.restype = I
         L.mlstm_noalloc_scratch_bytes.argtypes = []
         L.mlstm_noalloc_scratch_bytes.restype = Z
         L.mlstm_fwd_chunkwise_reversed_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
@@ -135,9 +139,21 @@ def _dtype_code(t: torch.Tensor) -> int:
         raise TypeError(f"q/k/v must be float32 or bfloat16, got {t.dtype}") from None
 
 
-def fwd_params(B, NH, S, DHQK, DHV, chunk=64, num_blocks=1, dtype=torch.bfloat16, retention=False) -> FwdParams:
+def fwd_params(B, NH, S, DHQK, DHV, chunk=64, num_blocks=1, dtype=torch.bfloat16, retention=False,
+               wait_limit_cycles: int = 0) -> FwdParams:
     return FwdParams(int(B), int(NH), int(S), int(DHQK), int(DHV), int(chunk), int(num_blocks),
-                     _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype), int(bool(retention)))
+                     _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype), int(bool(retention)),
+                     int(wait_limit_cycles))
+
+
+def fwd_status(params: FwdParams, workspace=None, stream=None, noalloc: bool = False) -> int:
+    """Outcome of the bounded device-side waits of the last prefill with these params and this
+    workspace (mlstm_fwd_chunkwise_status; noalloc=True: of the last mlstm_fwd_chunkwise_noalloc,
+    mlstm_fwd_chunkwise_noalloc_status).  Synchronises the stream.  Returns the status code:
+    0 = ok, 8 = a wait ran out (MLSTM_ERR_TIMEOUT)."""
+    if noalloc:
+        return int(lib().mlstm_fwd_chunkwise_noalloc_status(ctypes.byref(params), _stream_ptr(stream)))
+    return int(lib().mlstm_fwd_chunkwise_status(ctypes.byref(params), _ptr(workspace), _stream_ptr(stream)))
 
 
 def workspace_size(params: FwdParams) -> int:
@@ -155,7 +171,8 @@ def plan(params: FwdParams) -> dict:
 def fwd_chunkwise(q, k, v, igate=None, fgate=None, ogate=None, C0=None, n0=None, m0=None, *,
                   chunk: int = 64, num_blocks: int = 1, retention: bool = False,
                   h=None, C_out=None, n_out=None, m_out=None, workspace=None,
-                  return_state: bool = True, stream=None, events=None, reverse: bool = False):
+                  return_state: bool = True, stream=None, events=None, reverse: bool = False,
+                  wait_limit_cycles: int = 0):
     """Chunkwise-parallel prefill (mlstm_fwd_chunkwise).  CUDA tensors, contiguous.
 
     q, k [B,NH,S,DHQK], v [B,NH,S,DHV] (fp32 or bf16); igate, fgate [B,NH,S] fp32;
@@ -169,7 +186,7 @@ def fwd_chunkwise(q, k, v, igate=None, fgate=None, ogate=None, C0=None, n0=None,
     B, NH, S, DHQK = q.shape
     DHV = v.shape[-1]
     nb = int(num_blocks)
-    p = fwd_params(B, NH, S, DHQK, DHV, chunk, nb, q.dtype, retention)
+    p = fwd_params(B, NH, S, DHQK, DHV, chunk, nb, q.dtype, retention, wait_limit_cycles)
     dev = q.device
     if h is None:
         h = torch.empty((B, NH, S, DHV), dtype=q.dtype, device=dev)
@@ -376,7 +393,9 @@ def fwd_chunkwise_noalloc(q, k, v, igate=None, fgate=None, ogate=None, C0=None, 
     """mlstm_fwd_chunkwise_noalloc: the prefill with the library's built-in scratch buffer
     instead of a workspace (for callers that cannot allocate device memory).  Outputs not
     passed in are allocated here with torch, as in fwd_chunkwise; the library allocates
-    nothing.  Calls that overlap on the GPU share the buffer and race."""
+    nothing.  The call runs with q's device current (the library uses the buffer of the
+    current device) and, unless a stream is given, on that device's current stream.  Calls
+    that overlap on the GPU share the buffer and race."""
     B, NH, S, DHQK = q.shape
     DHV = v.shape[-1]
     nb = int(num_blocks)
@@ -391,9 +410,11 @@ def fwd_chunkwise_noalloc(q, k, v, igate=None, fgate=None, ogate=None, C0=None, 
             n_out = torch.empty((B, NH, nb, DHQK // nb), dtype=torch.float32, device=dev)
         if m_out is None:
             m_out = torch.empty((B, NH), dtype=torch.float32, device=dev)
-    st = lib().mlstm_fwd_chunkwise_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(igate), _ptr(fgate),
-                                           _ptr(ogate), _ptr(C0), _ptr(n0), _ptr(m0), _ptr(h), _ptr(C_out),
-                                           _ptr(n_out), _ptr(m_out), _stream_ptr(stream))
+    with torch.cuda.device(dev):
+        cs = _stream_ptr(stream if stream is not None else torch.cuda.current_stream(dev))
+        st = lib().mlstm_fwd_chunkwise_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(igate), _ptr(fgate),
+                                               _ptr(ogate), _ptr(C0), _ptr(n0), _ptr(m0), _ptr(h), _ptr(C_out),
+                                               _ptr(n_out), _ptr(m_out), cs)
     if st != 0:
         raise MlstmError(st, "mlstm_fwd_chunkwise_noalloc")
     if retention:

@@ -31,10 +31,30 @@ def test_library_builds_and_exports_every_declared_symbol():
 
 
 def test_status_strings_and_version():
-    for code in range(8):
-        assert mlstm.status_string(code)
+    for code in range(9):
+        assert mlstm.status_string(code) != "unknown status"
+    assert mlstm.status_string(8) == "a bounded device-side wait ran out"
     assert mlstm.status_string(99) == "unknown status"
-    assert mlstm.lib().mlstm_abi_version() >> 16 == 1
+    assert mlstm.lib().mlstm_abi_version() >> 16 == 2
+
+
+def test_params_struct_matches_header_layout():
+    # nine ints, then the 64-bit wait limit at offset 40 (C alignment of long long)
+    assert ctypes.sizeof(mlstm.FwdParams) == 48
+    assert mlstm.FwdParams.wait_limit_cycles.offset == 40
+    assert mlstm.fwd_params(1, 1, 1, 16, 16).wait_limit_cycles == 0
+
+
+def test_status_calls_validate_before_touching_the_device():
+    P = ctypes.c_void_p
+    L = mlstm.lib()
+    assert L.mlstm_fwd_chunkwise_status(None, P(G_), P(0)) == 1
+    assert L.mlstm_fwd_chunkwise_status(ctypes.byref(params(B=-1)), P(G_), P(0)) == 2
+    assert L.mlstm_fwd_chunkwise_status(ctypes.byref(params(dtype=7)), P(G_), P(0)) == 3
+    tc = mlstm.fwd_params(1, 2, 640, 128, 128, 64, 1, torch.bfloat16, False)
+    assert mlstm.plan(tc)["tensor_core"] == 1
+    assert L.mlstm_fwd_chunkwise_status(ctypes.byref(tc), None, P(0)) == 1  # its error word lives there
+    assert L.mlstm_fwd_chunkwise_noalloc_status(None, P(0)) == 1
 
 
 def fwd(p, q=A, k=B_, v=C_, ig=D_, fg=E_, og=None, C0=None, n0=None, m0=None, h=F_, C=None, n=None, m=None,

@@ -13,8 +13,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from linear_recurrent_token_b200 import inputs, mlstm
-from tests.helpers import TOL, TORCH_DTYPE, dev, host, slice_relerr
+from tests.helpers import TOL, TORCH_DTYPE, dev, host, m_err, slice_relerr
 
 SCRATCH = 32 << 20
 
@@ -60,5 +61,25 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(idx, S):
         errs = {"h": slice_relerr(host(got[0]), host(ref[0]), 2), "C": slice_relerr(host(got[1]), host(ref[1]), 3)}
         if not w.retention:
             errs["n"] = slice_relerr(host(got[2]), host(ref[2]), 3)
-            errs["m"] = float(np.max(np.abs(host(got[3]) - host(ref[3]))))
+            errs["m"] = m_err(host(got[3]), host(ref[3]))
         assert all(e <= tol for e in errs.values()), (call, errs)
+        # no bounded wait of the built-in buffer's call ran out
+        assert mlstm.fwd_status(p, noalloc=True) == 0
+
+
+@pytest.mark.gpu
+def test_noalloc_large_head_matches_the_oracle():
+    """One call on the full large-head workload (tensor-core path, 4 segments) against the fp64
+    oracle directly, so that the entry point is checked on its own and not only against the
+    workspace entry point."""
+    w = inputs.WORKLOADS[3]
+    td = TORCH_DTYPE[w.dtype]
+    inp = inputs.forward_inputs(w)
+    q, k, v = (dev(inp[x], td) for x in ("q", "k", "v"))
+    h, C, n, m = mlstm.fwd_chunkwise_noalloc(q, k, v, dev(inp["igate"]), dev(inp["fgate"]), chunk=w.chunk)
+    p = mlstm.fwd_params(w.B, w.NH, w.S, w.DHQK, w.DHV, w.chunk, w.num_blocks, td, w.retention)
+    assert mlstm.fwd_status(p, noalloc=True) == 0  # synchronises
+    hr, Cr, nr, mr = oracle.sequential(inp["q"], inp["k"], inp["v"], inp["igate"], inp["fgate"])
+    errs = {"h": slice_relerr(host(h), hr, 2), "C": slice_relerr(host(C), Cr, 3), "n": slice_relerr(host(n), nr, 3),
+            "m": m_err(host(m), mr)}
+    assert all(e <= TOL[w.dtype] for e in errs.values()), errs
