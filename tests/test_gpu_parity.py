@@ -10,9 +10,24 @@ import torch
 
 import oracle
 from linear_recurrent_token_b200 import inputs, mlstm
-from tests.helpers import TOL, TORCH_DTYPE, dev, host, m_err, slice_relerr
+from tests.helpers import (TOL, TORCH_DTYPE, Guarded, conditioned_excess, denominator_condition, dev, host,
+                           m_err, slice_relerr)
 
 pytestmark = pytest.mark.gpu
+
+
+def guarded_outputs(B, NH, S, DHQK, DHV, nb, td, retention):
+    """h and the final state as views into guard-banded buffers (tests.helpers.Guarded)."""
+    g = {"h": Guarded((B, NH, S, DHV), td), "C": Guarded((B, NH, nb, DHV // nb, DHQK // nb), torch.float32)}
+    if not retention:
+        g["n"] = Guarded((B, NH, nb, DHQK // nb), torch.float32)
+        g["m"] = Guarded((B, NH), torch.float32)
+    return g
+
+
+def assert_guards_intact(guards, what=""):
+    bad = [key for key, gd in guards.items() if not gd.intact()]
+    assert not bad, f"{what}: writes outside {bad}"
 
 
 def gpu_fwd(inp, dtype, chunk, nb=1, retention=False, ogate=None, C0=None, n0=None, m0=None):
@@ -20,9 +35,14 @@ def gpu_fwd(inp, dtype, chunk, nb=1, retention=False, ogate=None, C0=None, n0=No
     q, k, v = (dev(inp[x], td) for x in ("q", "k", "v"))
     ig = None if retention else dev(inp["igate"])
     fg = None if retention else dev(inp["fgate"])
+    B, NH, S, DHQK = q.shape
+    gd = guarded_outputs(B, NH, S, DHQK, v.shape[-1], nb, td, retention)
+    out = {key: gd[key].t if key in gd else None for key in ("h", "C", "n", "m")}
     h, C, n, m = mlstm.fwd_chunkwise(q, k, v, ig, fg, dev(ogate, td) if ogate is not None else None,
-                                     dev(C0), dev(n0), dev(m0), chunk=chunk, num_blocks=nb, retention=retention)
+                                     dev(C0), dev(n0), dev(m0), chunk=chunk, num_blocks=nb, retention=retention,
+                                     h=out["h"], C_out=out["C"], n_out=out["n"], m_out=out["m"])
     torch.cuda.synchronize()
+    assert_guards_intact(gd, f"S={S} chunk={chunk} nb={nb}")
     return host(h), host(C), host(n), host(m)
 
 
@@ -227,6 +247,26 @@ def test_large_input_gates_stay_finite():
     check(got, oracle_fwd(inp), "f32", what="large igate")
 
 
+def test_large_input_gates_signed_inputs_within_conditioned_bound():
+    # The same input gates with q and k of both signs.  n'.q can now cancel: a token whose
+    # denominator terms sum to kappa_t times the denominator loses kappa_t times the relative
+    # accuracy of those terms, in any fixed-precision evaluation.  The bound per token is the
+    # fp32 tolerance of the slice plus delta * kappa_t * |h_t|, with delta = 2^-20 (sixteen
+    # fp32 roundings: the recurrence of n' and a 16-term dot product).
+    w = inputs.WORKLOADS[0]
+    inp = inputs.forward_inputs(w, seed=80)
+    inp["igate"] = inp["igate"] + 60.0
+    got = gpu_fwd(inp, "f32", 16)
+    assert all(np.all(np.isfinite(x)) for x in got)
+    ref = oracle_fwd(inp)
+    kappa = denominator_condition(inp["q"], inp["k"], inp["igate"], inp["fgate"])
+    assert kappa.max() > 1e3  # the case really has cancelling denominators
+    excess = conditioned_excess(got[0], ref[0], kappa, TOL["f32"], 2.0 ** -20)
+    assert excess <= 1.0, (excess, kappa.max())
+    errs = {"C": slice_relerr(got[1], ref[1], 3), "n": slice_relerr(got[2], ref[2], 3), "m": m_err(got[3], ref[3])}
+    assert all(e <= TOL["f32"] for e in errs.values()), errs
+
+
 @pytest.fixture(scope="module")
 def decode_workload():
     w = inputs.WORKLOADS[4]
@@ -301,12 +341,15 @@ def test_tensor_core_path(case):
     td = torch.bfloat16
     ws = torch.zeros(plan["workspace_bytes"], dtype=torch.uint8, device="cuda")
     ws[:4] = 255
+    gd = guarded_outputs(B, NH, S, DHQK, DHV, nb, td, retention)
     h, C, n, m = mlstm.fwd_chunkwise(dev(inp["q"], td), dev(inp["k"], td), dev(inp["v"], td),
                                      None if retention else dev(inp["igate"]), None if retention else dev(inp["fgate"]),
                                      dev(og, td) if og is not None else None, dev(C0), dev(n0), dev(m0),
-                                     chunk=64, num_blocks=nb, retention=retention, workspace=ws)
-    torch.cuda.synchronize()
-    assert int(ws[:4].view(torch.int32).item()) == 0, "a bounded wait expired in the kernel"
+                                     chunk=64, num_blocks=nb, retention=retention, workspace=ws,
+                                     h=gd["h"].t, C_out=gd["C"].t, n_out=gd["n"].t if not retention else None,
+                                     m_out=gd["m"].t if not retention else None)
+    assert mlstm.fwd_status(p, ws) == 0, "a bounded wait expired in the kernel"
+    assert_guards_intact(gd, f"tc {case}")
     ref = oracle_fwd(inp, nb, retention, og, C0, n0, m0)
     errs = check((host(h), host(C), host(n), host(m)), ref, "bf16", retention, f"tc {case} plan {plan}")
     print(case, plan, errs)
@@ -331,10 +374,39 @@ def test_tensor_core_state_in_place_across_segments():
     check((host(h), host(C), host(n), host(m)), ref, "bf16", what="tc in place")
 
 
+def test_tensor_core_wait_limit_reports_timeout_then_workspace_is_reusable():
+    """A wait limit far shorter than a TMA load: the first wait on the loaded operands runs out,
+    the kernels stop, drain their own copies and free their tensor memory, and the status call
+    reports MLSTM_ERR_TIMEOUT promptly instead of hanging.  The same workspace then serves a
+    normal call, which matches the oracle and reports no timeout."""
+    import time
+    B, NH, S, DHQK, DHV = 1, 2, 640, 128, 128
+    w = inputs.Workload(3, "wait", B, NH, S, DHQK, DHV, 64, 1, "bf16", False, 1 / np.sqrt(DHQK))
+    p = mlstm.fwd_params(B, NH, S, DHQK, DHV, 64, 1, torch.bfloat16, False)
+    plan = mlstm.plan(p)
+    assert plan["tensor_core"] == 1 and plan["segments"] > 1  # both kernels with waits run
+    inp = inputs.forward_inputs(w, seed=3)
+    td = torch.bfloat16
+    args = (dev(inp["q"], td), dev(inp["k"], td), dev(inp["v"], td), dev(inp["igate"]), dev(inp["fgate"]))
+    ws = torch.zeros(plan["workspace_bytes"], dtype=torch.uint8, device="cuda")
+    short = mlstm.fwd_params(B, NH, S, DHQK, DHV, 64, 1, torch.bfloat16, False, wait_limit_cycles=256)
+    t0 = time.perf_counter()
+    mlstm.fwd_chunkwise(*args, chunk=64, workspace=ws, wait_limit_cycles=256)
+    st = mlstm.fwd_status(short, ws)
+    elapsed = time.perf_counter() - t0
+    assert st == 8, mlstm.status_string(st)  # MLSTM_ERR_TIMEOUT
+    assert elapsed < 5.0, elapsed
+    h, C, n, m = mlstm.fwd_chunkwise(*args, chunk=64, workspace=ws)
+    assert mlstm.fwd_status(p, ws) == 0
+    check((host(h), host(C), host(n), host(m)), oracle_fwd(inp), "bf16", what="after a timeout")
+
+
 # Gate regimes for the tensor-core walk: the state is kept in a lazily scaled form and a
 # chunk whose input gate rises far above the running stabiliser is evaluated in the
-# per-element stabilised form.  q, k >= 0 keep n.q a sum of positive terms (see
-# test_large_input_gates_stay_finite), so the comparison measures the stabilisation.
+# per-element stabilised form.  Each regime runs twice: with q, k and n0 >= 0 (n.q a sum of
+# positive terms, so the comparison isolates the stabilisation) and with q, k and n0 drawn
+# with both signs as in every other test (signs of the Q scaling, the column and row factors
+# and the guarded update weights all matter there).
 GATE_REGIMES = {
     "spikes_80": dict(spikes=80.0),         # isolated input gates 80 above the rest
     "spikes_40": dict(spikes=40.0),         # large but within the lazily scaled range
@@ -345,15 +417,17 @@ GATE_REGIMES = {
 }
 
 
+@pytest.mark.parametrize("signs", ["nonneg", "signed"])
 @pytest.mark.parametrize("DHV", [128, 512])
 @pytest.mark.parametrize("regime", list(GATE_REGIMES))
-def test_tensor_core_gate_regimes(regime, DHV):
+def test_tensor_core_gate_regimes(regime, DHV, signs):
     cfg = GATE_REGIMES[regime]
     B, NH, S, DHQK = 1, 2, 1536, 128
     w = inputs.Workload(3, "regime", B, NH, S, DHQK, DHV, 64, 1, "bf16", False, 1 / np.sqrt(DHQK))
     assert mlstm.plan(mlstm.fwd_params(B, NH, S, DHQK, DHV, 64, 1, torch.bfloat16, False))["tensor_core"] == 1
     inp = inputs.forward_inputs(w, seed=31)
-    inp["q"], inp["k"] = np.abs(inp["q"]), np.abs(inp["k"])
+    if signs == "nonneg":
+        inp["q"], inp["k"] = np.abs(inp["q"]), np.abs(inp["k"])
     rng = np.random.default_rng(32)
     if "spikes" in cfg:
         idx = rng.choice(S, size=12, replace=False)
@@ -364,12 +438,14 @@ def test_tensor_core_gate_regimes(regime, DHV):
         inp["fgate"] = inp["fgate"] - 3.0 + cfg["fmean"]
     rs = np.random.default_rng(33)
     C0 = (rs.standard_normal((B, NH, 1, DHV, DHQK)) * 0.2).astype(np.float32)
-    n0 = np.abs(rs.standard_normal((B, NH, 1, DHQK)) * 0.2).astype(np.float32)
+    n0 = (rs.standard_normal((B, NH, 1, DHQK)) * 0.2).astype(np.float32)
+    if signs == "nonneg":
+        n0 = np.abs(n0)
     m0 = rs.standard_normal((B, NH)).astype(np.float32)
     got = gpu_fwd(inp, "bf16", 64, C0=C0, n0=n0, m0=m0)
     assert all(np.all(np.isfinite(x)) for x in got), regime
-    errs = check(got, oracle_fwd(inp, C0=C0, n0=n0, m0=m0), "bf16", what=regime)
-    print(regime, errs)
+    errs = check(got, oracle_fwd(inp, C0=C0, n0=n0, m0=m0), "bf16", what=f"{regime} {signs}")
+    print(regime, signs, errs)
 
 
 @pytest.mark.parametrize("dtype,chunk,nb,retention,with_o", [
