@@ -769,6 +769,82 @@ def backward_line(w, ms, sm_mhz, cpu: bool):
     return out
 
 
+def forward_leg(w, steps, warmup, clocks, peaks, world, cpu: bool):
+    """The chunkwise prefill on one of the smaller workloads (block-diagonal, retention): step
+    time (every kernel of the call) with L2 flushed between steps, the roofline of the whole
+    step against HBM (these workloads are HBM-bound: their intensity is far below the ridge)
+    with the tensor fraction beside it, e2e through the API with host buffers, and the oracle
+    on a bounded sample."""
+    cw = run_chunkwise(w, steps, warmup, 256 << 20, clocks)
+    step_ms = dist_max(statistics.mean(cw["step_ms"]), world)
+    main_ms = statistics.mean(cw["main_ms"])
+    esz = 2 if w.dtype == "bf16" else 4
+    flops = chunkwise_flops(w.B, w.NH, w.S, w.dk, w.dv, w.chunk, w.num_blocks, w.retention)
+    mbytes = chunkwise_min_bytes(w.B, w.NH, w.S, w.DHQK, w.DHV, esz, w.num_blocks, w.retention)
+    e2e_ms, h2d, d2h = run_chunkwise_e2e(w, max(8, steps // 2), cw["tensors"])
+    e2e_ms = dist_max(e2e_ms, world)
+    del cw["tensors"]
+    gbs = mbytes / (step_ms * 1e-3) / 1e9
+    tf = flops / (step_ms * 1e-3) / 1e12
+    tc = cw["plan"]["tensor_core"]
+    out = {"workload": w.describe(), "value": w.B * w.S * world / (step_ms * 1e-3), "unit": "tokens/s",
+           "ms_per_step": step_ms, "steps": steps, "plan": cw["plan"],
+           "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                        "kernel": "whole prefill call (" + ("gate prep, segment summaries, tcgen05 walk"
+                                                            if tc else "gate prep, SIMT walk") + ")",
+                        "min_bytes_per_launch": mbytes, "walk_ms": main_ms,
+                        "tc_achieved_tflops": tf, "tc_frac": tf / peaks["bf16_tflops"], "flops_per_launch": flops},
+           "e2e": {"value": w.B * w.S * world / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                   "d2h_bytes_per_step": d2h}}
+    if cpu:
+        cb = cpu_baseline(w, budget_s=6.0)
+        out["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    return out
+
+
+def _r(x, digits=3):
+    """x rounded to `digits` significant digits (for the compact summary)."""
+    if x is None or not isinstance(x, (int, float)) or x == 0:
+        return x
+    import math
+    return round(x, -int(math.floor(math.log10(abs(x)))) + digits - 1)
+
+
+def compact_legs(line):
+    """Key figures of every leg, short: the headline line ends with them, so that a log that
+    keeps only the end of the output still shows each leg's number and roofline fraction."""
+    legs = {}
+    if "decode" in line:
+        d = line["decode"]
+        legs["decode"] = {"GB/s": _r(d["value"]), "hbm": _r(d["roofline"]["frac"]), "ms": _r(d["ms_per_step"])}
+    for key, name in (("fwd_blockdiag", "fwd_blockdiag"), ("fwd_retention", "fwd_retention")):
+        if key in line:
+            e = line[key]
+            legs[name] = {"tok/s": _r(e["value"]), "ms": _r(e["ms_per_step"]), "hbm": _r(e["roofline"]["frac"]),
+                          "tc": _r(e["roofline"]["tc_frac"])}
+    if "reversed" in line:
+        legs["reversed"] = {"tok/s": _r(line["reversed"]["value"]), "ms": _r(line["reversed"]["ms_per_step"])}
+    for e in line.get("backward", []):
+        legs["bwd_" + e["workload"].split(":")[0]] = {"tok/s": _r(e["value"]), "ms": _r(e["ms_per_step"]),
+                                                       "fp32": _r(e["roofline"]["frac"])}
+    for e in line.get("scalar_normaliser", []):
+        legs["scalar_norm_" + e["workload"].split(":")[0]] = {"tok/s": _r(e["value"]), "ms": _r(e["ms_per_step"])}
+    if "msr_block" in line:
+        e = line["msr_block"]
+        legs["msr_block"] = {"tok/s": _r(e["value"]), "ms": _r(e["ms_per_step"]), "fwd_ms": _r(e["forward_ms"])}
+    g = line.get("gdn2", {})
+    for name, val in g.items():
+        if not isinstance(val, dict):
+            continue
+        for mode in ("recurrent", "chunk"):
+            if mode in val:
+                legs[f"gdn2_{mode}"] = {"tok/s": _r(val[mode]["value"]), "ms": _r(val[mode]["ms_per_step"])}
+        if "recurrent" not in val and "roofline" in val:
+            legs["gdn2_decode"] = {"GB/s": _r(val["value"]), "hbm": _r(val["roofline"]["frac"])}
+    return legs
+
+
 # ------------------------------------------------------------------ main
 def main():
     ap = argparse.ArgumentParser()
@@ -779,8 +855,8 @@ def main():
     ap.add_argument("--workload", type=int, default=3, help="chunkwise workload index (default 3)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
-    ap.add_argument("--legs", choices=["both", "chunkwise", "decode", "backward", "msr", "gdn2"], default="both",
-                    help="run only one leg (for profiling); the default runs both")
+    ap.add_argument("--legs", choices=["both", "chunkwise", "decode", "backward", "msr", "gdn2", "forward"],
+                    default="both", help="run only one leg (for profiling); the default runs all of them")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
@@ -840,6 +916,12 @@ def main():
             if rank == 0:
                 print(json.dumps({"leg": "msr", "workload": inputs.WORKLOADS[2].describe(), **r}))
             return
+        if args.legs == "forward":
+            for idx in (1, 2):
+                r = forward_leg(inputs.WORKLOADS[idx], args.steps, args.warmup, clocks, peaks, world, False)
+                if rank == 0:
+                    print(json.dumps({"leg": "forward", **r}))
+            return
         if args.legs == "decode":
             dec = run_decode(wd, args.steps, args.warmup, clocks)
             ms = dist_max(statistics.mean(dec["step_ms"]), world)
@@ -868,6 +950,12 @@ def main():
             dist_barrier(world)
             dec = run_decode(wd, args.steps * 5, args.warmup, clocks)
             dist_barrier(world)
+        fwd_small = {}
+        if args.legs == "both":
+            for key, idx in (("fwd_blockdiag", 1), ("fwd_retention", 2)):
+                dist_barrier(world)
+                fwd_small[key] = forward_leg(inputs.WORKLOADS[idx], args.steps, args.warmup, clocks, peaks, world,
+                                             rank == 0 and world == 1 and not args.no_cpu_baseline)
         rev_ms = None
         if args.legs == "both":
             rev_ms = run_reversed(w, max(3, args.steps // 4), args.warmup, 256 << 20)
@@ -899,6 +987,7 @@ def main():
         "config": config,
         "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": achieved_tf / peaks["bf16_tflops"],
+                     "step_frac": flops / (slow_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
                      "traffic": recorded_traffic("tc_walk", w.name) if cw["plan"]["tensor_core"] else None,
                      "kernel": "chunkwise walk" + (" (tcgen05)" if cw["plan"]["tensor_core"] else " (SIMT)"),
                      "kernel_ms": main_ms, "flops_per_launch": flops, "peak_source": f"{peak_src} bf16 burst",
@@ -927,6 +1016,9 @@ def main():
                     "h2d_bytes_per_step": dec["h2d"], "d2h_bytes_per_step": dec["d2h"]},
         }
         line["gpu_launches"] += len(dec["step_ms"])
+    for key, r in fwd_small.items():
+        line[key] = r
+        line["gpu_launches"] += r["steps"] * r["plan"]["kernels"]
     if rev_ms:
         rms = dist_max(statistics.median(rev_ms), world)
         esz = 2 if w.dtype == "bf16" else 4
@@ -973,7 +1065,15 @@ def main():
         cb = cpu_baseline(w)
         line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
     if rank == 0:
-        print(json.dumps(line))
+        # every leg in full on one line, then the headline line, which ends with the key
+        # figures of each leg (so that the end of the output carries all of them)
+        standard = ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                    "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "cpu_baseline", "clocks", "e2e",
+                    "gpu_launches")
+        print(json.dumps({"detail": {k: v for k, v in line.items() if k not in standard}}))
+        head = {k: line[k] for k in standard if k in line}
+        head["legs"] = compact_legs(line)
+        print(json.dumps(head))
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
