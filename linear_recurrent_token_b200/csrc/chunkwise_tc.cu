@@ -64,6 +64,9 @@ struct TcParams {
   int sp, ncp;
   unsigned int* err;
   long long wait;  // bound of every mbarrier wait, SM cycles
+  // scalar normaliser with a learnable bias (NULL: the vector normaliser n . q): bias [NH];
+  // then n0 / n_out hold one value per (batch, head) and dn one value per (slice, segment)
+  const float* nbias;
 };
 
 // Lane / row mapping of an M-row accumulator: thread (warp w, lane l) owns row
@@ -291,7 +294,7 @@ __global__ void __launch_bounds__(NTA, 1)
   // this tile accumulates dn over key columns [dn0, min(DK, dn0 + dnw)), dnw a multiple of 8
   const int dnw = ((DK + p.n_tiles - 1) / p.n_tiles + 7) / 8 * 8;
   const int dn0 = tile * dnw;
-  const bool do_dn = !p.retention && dn0 < DK;
+  const bool do_dn = !p.retention && !p.nbias && dn0 < DK;
   const int nck = p.seg_chunks;
 
   if (tid == 0) {
@@ -377,6 +380,7 @@ __global__ void __launch_bounds__(NTA, 1)
     // prefetched into registers)
     const float* gxr = p.gx + (size_t)bh * p.sp + T0 + 2 * lane;
     float2 gxn = *reinterpret_cast<const float2*>(gxr);
+    float osum = 0.f;  // scalar normaliser: this lane's share of the segment's sum of weights
     for (int c = 0; c < nck; ++c) {
       const int st = c % NS;
       if (c >= NS) {
@@ -388,10 +392,17 @@ __global__ void __launch_bounds__(NTA, 1)
         }
       }
       const float cf = coff[c];
-      *reinterpret_cast<float2*>(omb + st * L + 2 * lane) = make_float2(expf(cf + gxn.x), expf(cf + gxn.y));
+      const float2 om2 = make_float2(expf(cf + gxn.x), expf(cf + gxn.y));
+      *reinterpret_cast<float2*>(omb + st * L + 2 * lane) = om2;
+      osum += om2.x + om2.y;
       if (c + 1 < nck) gxn = *reinterpret_cast<const float2*>(gxr + (size_t)(c + 1) * L);
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[st]);
+    }
+    if (p.nbias && !p.retention) {  // dn of the scalar normaliser: sum over the segment of omega_s
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) osum += __shfl_xor_sync(0xffffffffu, osum, o);
+      if (lane == 0 && tile == 0 && !abort_flag) p.dn[((size_t)slice * (p.G - 1) + g) * p.dk] = osum;
     }
   } else if (warp == 1) {
     // =============================================================== MMA warp
@@ -588,7 +599,7 @@ struct WalkBars {
   uint64_t drain;  // both MMA warps' last commits, before TMEM is freed
 };
 
-template <int DK, int DVT>
+template <int DK, int DVT, bool SN>
 __global__ void __launch_bounds__(NTW, 1)
     tc_walk_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                    const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapH, TcParams p) {
@@ -711,7 +722,18 @@ __global__ void __launch_bounds__(NTW, 1)
       tmem_st16(tm + lane_off + TM_C + c0, r);
     }
     tmem_wait_st();
-    if (!ret)
+    if (SN) {
+      if (tid == 96) {  // scalar normaliser: one value per (batch, head), in nvec[0]
+        float x = p.n0 ? wc0 * p.n0[bh] : 0.f;
+        float after = gsum;
+        for (int jg = 0; jg < g; ++jg) {
+          after -= p.segA[(size_t)bh * (p.G - 1) + jg];
+          x += expf(p.segB[(size_t)bh * (p.G - 1) + jg] + after - m_start) *
+               p.dn[((size_t)slice * (p.G - 1) + jg) * p.dk];
+        }
+        nvec[0] = x;
+      }
+    } else if (!ret)
       for (int col = tid - 96; col < DK; col += 256) {
         float x = p.n0 ? wc0 * p.n0[(size_t)slice * p.dk + col] : 0.f;
         float after = gsum;
@@ -1082,6 +1104,7 @@ __global__ void __launch_bounds__(NTW, 1)
     const bool first = gt == 0;
     const uint32_t ps_u = sm_u + SM::OP, hs_u = sm_u + SM::OH;
     const bool use_og = p.og != nullptr && !ret;
+    const float nbias_h = SN ? p.nbias[bh % p.NH] : 0.f;
     for (int c = 0; c < nck; ++c) {
       const int b = c & 1, gi = c % NGB;
       const GateBuf G = gbuf(gi);
@@ -1141,8 +1164,13 @@ __global__ void __launch_bounds__(NTW, 1)
           const float a1 = s0 + 1 <= lim_lo ? pa.y : 0.f;
           const float b0 = s0 <= lim_hi ? pb.x : 0.f;
           const float b1 = s0 + 1 <= lim_hi ? pb.y : 0.f;
-          rs_lo += a0 + a1;
-          rs_hi += b0 + b1;
+          if (SN) {  // scalar normaliser: sums of the weights themselves (no q . k factor)
+            rs_lo += (s0 <= lim_lo ? f_lo[2 * j] : 0.f) + (s0 + 1 <= lim_lo ? f_lo[2 * j + 1] : 0.f);
+            rs_hi += (s0 <= lim_hi ? f_hi[2 * j] : 0.f) + (s0 + 1 <= lim_hi ? f_hi[2 * j + 1] : 0.f);
+          } else {
+            rs_lo += a0 + a1;
+            rs_hi += b0 + b1;
+          }
           plo[j] = pack_bf16(a0, a1);
           phi[j] = pack_bf16(b0, b1);
         }
@@ -1172,7 +1200,10 @@ __global__ void __launch_bounds__(NTW, 1)
       if (gt < L) {
         const int t = gt;
         const float e = G.E[t];
-        rden[t] = ret ? e : e / fmaxf(fabsf(e * rsum[t] + G.F[t] * G.nq[t]), G.emt[t]);
+        if (SN)  // max(|n' + bias e^{-m}|, e^{-m}) in stabilised units
+          rden[t] = e / fmaxf(fabsf(e * rsum[t] + G.F[t] * G.nq[t] + nbias_h * G.emt[t]), G.emt[t]);
+        else
+          rden[t] = ret ? e : e / fmaxf(fabsf(e * rsum[t] + G.F[t] * G.nq[t]), G.emt[t]);
       }
       // h_t = H_t rden_t (x o_t): H leaves TMEM first, then 8x8 tiles are stored transposed
       // into the 128-byte swizzled staging tile and TMA-stored
@@ -1246,6 +1277,7 @@ __global__ void __launch_bounds__(NTW, 1)
     const bool first = nt == 0;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     float fin = 1.f;
+    float n_sc = SN ? nvec[0] : 0.f;  // scalar normaliser (lazily scaled like n)
     for (int c = 0; c < nck; ++c) {
       const int b = c & 1, gi = c % NGB;
       const GateBuf G = gbuf(gi);
@@ -1269,7 +1301,9 @@ __global__ void __launch_bounds__(NTW, 1)
         warp_wait_slow(&bars.full[b], (c >> 1) & 1, &abort_flag, p.wait);
       const bool guard = (flags & GF_GUARD) != 0;
       fin = G.scal[4];
-      if (!ret) {
+      if (SN) {
+        if (nt < L) G.nq[nt] = n_sc;  // scalar normaliser: the chunk's start value for every token
+      } else if (!ret) {
         // nq_t = n_st . q_t for this warp's 16 tokens as warp-level MMAs: A = the Q rows
         // (ldmatrix from the swizzled tile), B = n as hi + lo in columns 0 and 1 (lanes 0-7)
         const int mi = lane >> 3, arow = 16 * wq + (mi & 1) * 8 + (lane & 7);
@@ -1303,7 +1337,14 @@ __global__ void __launch_bounds__(NTW, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.q_ready[gi]);  // this warp's tokens: n . q (and scaled Q)
-      if (!ret) {
+      if (SN) {
+        // n <- ns n + sum_s u_s, the same in every thread of the group (no shared state)
+        const float2 u2 = *reinterpret_cast<const float2*>(G.u + 2 * lane);
+        float us = u2.x + u2.y;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) us += __shfl_xor_sync(0xffffffffu, us, o);
+        n_sc = G.scal[3] * n_sc + us;
+      } else if (!ret) {
         // n <- ns n + K^T u for this warp's DK/4 entries of n as warp-level MMAs: A = K^T
         // (ldmatrix.trans of the swizzled K tile), B = u as hi + lo in columns 0 and 1 (lanes 0-7)
         constexpr int MT = DK / 64;  // 16-entry tiles per warp
@@ -1351,7 +1392,9 @@ __global__ void __launch_bounds__(NTW, 1)
       }
     }
     // final n after the last update, back in units of e^{m}
-    if (nck > 0 && last_seg && !ret && tile == 0 && p.n_out && !abort_flag)
+    if (SN) {
+      if (nck > 0 && last_seg && tile == 0 && blk == 0 && p.n_out && !abort_flag && nt == 0) p.n_out[bh] = fin * n_sc;
+    } else if (nck > 0 && last_seg && !ret && tile == 0 && p.n_out && !abort_flag)
       for (int col = nt; col < DK; col += 128) p.n_out[(size_t)slice * p.dk + col] = fin * nvec[col];
   }
 
@@ -1441,7 +1484,7 @@ static cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 bl
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-template <int DK, int DVT>
+template <int DK, int DVT, bool SN>
 static cudaError_t launch_tc_dk(const TcPlan& pl, const TcParams& prm, const CUtensorMap& mq, const CUtensorMap& mk,
                                 const CUtensorMap& mv, const CUtensorMap& mh, long long slices, cudaStream_t stream,
                                 cudaEvent_t ev0, cudaEvent_t ev1) {
@@ -1459,11 +1502,11 @@ static cudaError_t launch_tc_dk(const TcPlan& pl, const TcParams& prm, const CUt
     if (e != cudaSuccess) return e;
   }
   const int smemC = WalkSmem<DK, DVT>::BYTES;
-  e = cudaFuncSetAttribute(tc_walk_kernel<DK, DVT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemC);
+  e = cudaFuncSetAttribute(tc_walk_kernel<DK, DVT, SN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemC);
   if (e != cudaSuccess) return e;
   if (ev0) cudaEventRecord(ev0, stream);
   dim3 gridC(pl.n_tiles, pl.G, (unsigned)slices);
-  e = launch_dependent(tc_walk_kernel<DK, DVT>, gridC, dim3(NTW), smemC, stream, mq, mk, mv, mh, prm);
+  e = launch_dependent(tc_walk_kernel<DK, DVT, SN>, gridC, dim3(NTW), smemC, stream, mq, mk, mv, mh, prm);
   if (ev1) cudaEventRecord(ev1, stream);
   return e;
 }
@@ -1515,6 +1558,7 @@ cudaError_t launch_tc(const WalkArgs& a, const TcPlan& pl, void* ws, cudaStream_
   prm.ncp = pl.G * pl.seg_chunks;
   prm.sp = prm.ncp * L;
   prm.wait = a.wait_cycles > 0 ? a.wait_cycles : WAIT_DEFAULT;
+  prm.nbias = a.retention ? nullptr : a.nbias;
   float** planes[5] = {&prm.gb, &prm.gx, &prm.gxc, &prm.cg, &prm.cxm};
   for (int i = 0; i < 5; ++i) {
     *planes[i] = reinterpret_cast<float*>(w + off);
@@ -1522,12 +1566,21 @@ cudaError_t launch_tc(const WalkArgs& a, const TcPlan& pl, void* ws, cudaStream_
   }
   cudaError_t e = cudaMemsetAsync(w, 0, 4, stream);
   if (e != cudaSuccess) return e;
-  if (a.dk == 256 && pl.dvt == 128) return launch_tc_dk<256, 128>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
-  if (a.dk == 256 && pl.dvt == 64) return launch_tc_dk<256, 64>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
-  if (a.dk == 128 && pl.dvt == 128) return launch_tc_dk<128, 128>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
-  if (a.dk == 128 && pl.dvt == 64) return launch_tc_dk<128, 64>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
-  if (a.dk == 64 && pl.dvt == 128) return launch_tc_dk<64, 128>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
-  if (a.dk == 64 && pl.dvt == 64) return launch_tc_dk<64, 64>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
+  if (prm.nbias) {
+    if (a.dk == 256 && pl.dvt == 128) return launch_tc_dk<256, 128, true>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
+    if (a.dk == 256 && pl.dvt == 64) return launch_tc_dk<256, 64, true>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
+    if (a.dk == 128 && pl.dvt == 128) return launch_tc_dk<128, 128, true>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
+    if (a.dk == 128 && pl.dvt == 64) return launch_tc_dk<128, 64, true>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
+    if (a.dk == 64 && pl.dvt == 128) return launch_tc_dk<64, 128, true>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
+    if (a.dk == 64 && pl.dvt == 64) return launch_tc_dk<64, 64, true>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
+    return cudaErrorInvalidValue;
+  }
+  if (a.dk == 256 && pl.dvt == 128) return launch_tc_dk<256, 128, false>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
+  if (a.dk == 256 && pl.dvt == 64) return launch_tc_dk<256, 64, false>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
+  if (a.dk == 128 && pl.dvt == 128) return launch_tc_dk<128, 128, false>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
+  if (a.dk == 128 && pl.dvt == 64) return launch_tc_dk<128, 64, false>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
+  if (a.dk == 64 && pl.dvt == 128) return launch_tc_dk<64, 128, false>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
+  if (a.dk == 64 && pl.dvt == 64) return launch_tc_dk<64, 64, false>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
   return cudaErrorInvalidValue;
 }
 

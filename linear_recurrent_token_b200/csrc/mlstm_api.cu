@@ -57,7 +57,8 @@ struct WsLayout {
   size_t tc, c_init;  // tensor-core path: its own area, snapshot of C0
 };
 
-WsLayout fwd_layout(const FwdShape& s) {
+// scalar_n: the scalar-normaliser variant (n0 one value per (batch, head)); tensor-core path only
+WsLayout fwd_layout(const FwdShape& s, bool scalar_n = false) {
   WsLayout w = {0, 0, 0, 0, 0, 0};
   if (s.BH == 0) return w;
   if (s.tc) {
@@ -66,7 +67,7 @@ WsLayout fwd_layout(const FwdShape& s) {
     off = align_up(off + tc_workspace_bytes(s.tcp, s.BH, s.nb, s.dk, s.dv));
     if (!s.retention) {
       w.n_init = off;
-      off = align_up(off + sizeof(float) * (size_t)s.BH * s.nb * s.dk);
+      off = align_up(off + sizeof(float) * (size_t)s.BH * (scalar_n ? 1 : (size_t)s.nb * s.dk));
       w.m_init = off;
       off = align_up(off + sizeof(float) * (size_t)s.BH);
     }
@@ -112,10 +113,15 @@ mlstm_status_t fwd_impl(const mlstm_fwd_params_t* p, const void* q, const void* 
                         const float* igate, const float* fgate, const void* ogate, const float* C0,
                         const float* n0, const float* m0, void* h, float* C_out, float* n_out, float* m_out,
                         void* workspace, size_t workspace_bytes, cudaStream_t stream, cudaEvent_t ev0,
-                        cudaEvent_t ev1, bool launch = true, const GnArgs* gn = nullptr) {
+                        cudaEvent_t ev1, bool launch = true, const GnArgs* gn = nullptr,
+                        const float* nbias = nullptr) {
+  // nbias != NULL: the scalar normaliser with this bias [NH] (tensor-core path only; n0 / n_out
+  // one value per (batch, head)); the caller has validated it
   FwdShape s;
   mlstm_status_t st = check_fwd(p, &s);
   if (st != MLSTM_OK) return st;
+  const bool scalar_n = nbias != nullptr;
+  if (scalar_n && (!s.tc || s.retention)) return MLSTM_ERR_SHAPE;
   const bool ret = s.retention != 0;
   if (ret) {
     igate = fgate = nullptr;
@@ -126,7 +132,8 @@ mlstm_status_t fwd_impl(const mlstm_fwd_params_t* p, const void* q, const void* 
   const size_t tok = (size_t)s.BH * s.S;
   const size_t bq = tok * s.DHQK * s.esize, bv = tok * s.DHV * s.esize, bg = tok * sizeof(float);
   const size_t bC = (size_t)s.BH * s.nb * s.dv * s.dk * sizeof(float);
-  const size_t bn = (size_t)s.BH * s.nb * s.dk * sizeof(float), bm = (size_t)s.BH * sizeof(float);
+  const size_t bn = (size_t)s.BH * (scalar_n ? 1 : (size_t)s.nb * s.dk) * sizeof(float);
+  const size_t bm = (size_t)s.BH * sizeof(float);
   if (tok > 0) {
     if (!q || !k || !v || !h) return MLSTM_ERR_NULL;
     if (!ret && (!igate || !fgate)) return MLSTM_ERR_NULL;
@@ -134,7 +141,7 @@ mlstm_status_t fwd_impl(const mlstm_fwd_params_t* p, const void* q, const void* 
   const void* all[] = {q, k, v, igate, fgate, ogate, C0, n0, m0, h, C_out, n_out, m_out, workspace};
   for (const void* ptr : all)
     if (ptr && misaligned(ptr)) return MLSTM_ERR_ALIGN;
-  const WsLayout ws = fwd_layout(s);
+  const WsLayout ws = fwd_layout(s, scalar_n);
   if (ws.total > 0 && (!workspace || workspace_bytes < ws.total)) return MLSTM_ERR_WORKSPACE;
 
   // aliasing: outputs may not overlap inputs, except the exact in-place state aliases
@@ -200,6 +207,7 @@ mlstm_status_t fwd_impl(const mlstm_fwd_params_t* p, const void* q, const void* 
   a.n_out = n_out;
   a.m_out = m_out;
   a.wait_cycles = p->wait_limit_cycles;
+  a.nbias = nbias;
   if (s.tc) {
     // snapshots: the walk writes n_out / m_out (and C_out across segments) while other
     // CTAs may still read n0 / m0 / C0, which the caller may have aliased to them
@@ -480,8 +488,11 @@ mlstm_status_t mlstm_fwd_chunkwise_reversed(const mlstm_fwd_params_t* p, const v
 
 // Workspace of the scalar-normaliser prefill (SIMT walk): per-token stabiliser and snapshots
 // of m0 and of the per-head n0.
+// On the tensor-core path (bf16, chunk 64, the shapes it covers) the walk's own workspace with
+// per-head n0 instead.
 static size_t scalar_norm_ws(const FwdShape& s) {
   if (s.BH == 0 || s.S == 0) return 0;
+  if (s.tc) return fwd_layout(s, true).total;
   return align_up(sizeof(float) * (size_t)s.BH * s.S) + 2 * align_up(sizeof(float) * (size_t)s.BH);
 }
 
@@ -501,7 +512,7 @@ mlstm_status_t mlstm_fwd_chunkwise_scalar_normaliser(const mlstm_fwd_params_t* p
   mlstm_status_t st = check_fwd(p, &s);
   if (st != MLSTM_OK) return st;
   if (p->retention) return MLSTM_ERR_SHAPE;  // retention has no normaliser
-  if (s.BH > 0 && s.S > 0 && simt_walk_pick_tile(s.chunk, s.dk, s.dv) == 0) return MLSTM_ERR_SHAPE;
+  if (s.BH > 0 && s.S > 0 && !s.tc && simt_walk_pick_tile(s.chunk, s.dk, s.dv) == 0) return MLSTM_ERR_SHAPE;
   const size_t tok = (size_t)s.BH * s.S;
   const size_t bq = tok * s.DHQK * s.esize, bv = tok * s.DHV * s.esize, bg = tok * sizeof(float);
   const size_t bC = (size_t)s.BH * s.nb * s.dv * s.dk * sizeof(float), bh4 = (size_t)s.BH * sizeof(float);
@@ -529,6 +540,9 @@ mlstm_status_t mlstm_fwd_chunkwise_scalar_normaliser(const mlstm_fwd_params_t* p
   if (need > 0 && (!workspace || workspace_bytes < need)) return MLSTM_ERR_WORKSPACE;
   if (s.BH == 0) return MLSTM_OK;
   cudaStream_t cs = (cudaStream_t)stream;
+  if (s.tc && s.S > 0)  // tensor-core kernels with the scalar normaliser
+    return fwd_impl(p, q, k, v, igate, fgate, ogate, C0, n0, m0, h, C_out, n_out, m_out, workspace,
+                    workspace_bytes, cs, nullptr, nullptr, true, nullptr, bias);
   cudaError_t e = cudaSuccess;
   if (s.S == 0) {  // the final state is the initial state
     if (C_out && C_out != C0)

@@ -42,17 +42,9 @@ def host(t):
     return None if t is None else t.detach().float().cpu().numpy()
 
 
-def denominator_condition(q, k, igate, fgate, n0=None, m0=None, num_blocks: int = 1):
-    """Condition number of each token's read-out denominator, fp64, [B, NH, nb, S]:
-
-        kappa_t = sum_i |n'_{t,i} q_{t,i}| / max(|n'_t . q_t|, exp(-m_t)).
-
-    A relative error delta in the terms of n'.q (rounding of n' and of the dot product)
-    moves the denominator by at most delta * kappa_t of itself, and h_t by the same
-    factor.  With q and k of both signs n'.q can cancel, so kappa_t is unbounded and no
-    fixed-precision evaluation keeps a fixed relative error on such a token.  Used only to
-    scale a tolerance, never as an expected value.
-    """
+def _denominators(q, k, igate, fgate, n0, m0, num_blocks):
+    """fp64 per token [B, NH, nb, S]: den_t = max(|n'_t . q_t|, e^{-m_t}) and the same with the
+    absolute values |n'_abs| . |q_t| (n'_abs the normaliser of |k| and |n0|, same gates)."""
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
     ig = np.asarray(igate, np.float64)
@@ -63,41 +55,68 @@ def denominator_condition(q, k, igate, fgate, n0=None, m0=None, num_blocks: int 
     kb = k.reshape(B, NH, S, num_blocks, dk)
     lf = np.minimum(fg, 0.0) - np.log1p(np.exp(-np.abs(fg)))
     n = np.zeros((B, NH, num_blocks, dk)) if n0 is None else np.asarray(n0, np.float64).reshape(B, NH, num_blocks, dk)
+    na = np.abs(n)
     m = np.zeros((B, NH)) if m0 is None else np.asarray(m0, np.float64).reshape(B, NH)
-    out = np.zeros((B, NH, num_blocks, S))
+    den = np.zeros((B, NH, num_blocks, S))
+    den_abs = np.zeros((B, NH, num_blocks, S))
     for t in range(S):
         m_new = np.maximum(lf[:, :, t] + m, ig[:, :, t])
         fp = np.exp(lf[:, :, t] + m - m_new)[..., None, None]
         ip = np.exp(ig[:, :, t] - m_new)[..., None, None]
         n = fp * n + ip * kb[:, :, t]
+        na = fp * na + ip * np.abs(kb[:, :, t])
         m = m_new
-        prod = n * qb[:, :, t]
-        out[..., t] = np.sum(np.abs(prod), -1) / np.maximum(np.abs(np.sum(prod, -1)), np.exp(-m)[..., None])
-    return out
+        floor = np.exp(-m)[..., None]
+        den[..., t] = np.maximum(np.abs(np.sum(n * qb[:, :, t], -1)), floor)
+        den_abs[..., t] = np.maximum(np.sum(na * np.abs(qb[:, :, t]), -1), floor)
+    return den, den_abs
 
 
-def conditioned_excess(h, ref, kappa, tol: float, delta: float) -> float:
-    """Largest ratio, over (batch, head, block) slices and tokens, of a token's error to its
-    bound tol * max|ref of the slice| + delta * kappa_t * max|ref_t|; <= 1 passes.
+def readout_scale(q, k, v, igate, fgate, C0=None, n0=None, m0=None, num_blocks: int = 1):
+    """What rounding the recurrence's terms can do to h, fp64: returns (kappa [B, NH, nb, S],
+    h_abs [B, NH, S, DHV]).  h_t = num_t / den_t with num_t = C'_t q_t and den_t =
+    max(|n'_t . q_t|, e^{-m_t}); if every element of the state (and of the intra-chunk terms)
+    carries a relative error delta, then
 
-    h, ref [B, NH, S, DHV] (DHV split into nb blocks as kappa's third axis); kappa from
-    denominator_condition.  The first term is the fixed tolerance of the comparison, the
-    second what a relative error delta in the denominator's terms costs a token whose
-    denominator cancels (see denominator_condition).
+        |d num_t,i| <= delta sum_j |C'_t,ij q_t,j| <= delta num_abs_t,i,
+        |d den_t|   <= delta sum_j |n'_t,j q_t,j|  <= delta den_abs_t,
+
+    where num_abs, den_abs are the same recurrence run on |q|, |k|, |v|, |C0|, |n0| (all gate
+    weights are positive).  With kappa_t = den_abs_t / den_t and h_abs = num_abs / den_abs (the
+    read-out of that absolute run):
+
+        |d h_t,i| <= delta (num_abs_t,i + |h_t,i| den_abs_t) / den_t
+                  =  delta kappa_t (h_abs_t,i + |h_t,i|).
+
+    With q and k of both signs, num and den can cancel, so kappa_t is unbounded and no
+    fixed-precision evaluation meets a fixed relative error on such tokens.  Used only to scale
+    a tolerance, never as an expected value.
     """
+    import oracle
+    den, den_abs = _denominators(q, k, igate, fgate, n0, m0, num_blocks)
+    a = lambda x: None if x is None else np.abs(x)
+    h_abs = oracle.sequential(a(q), a(k), a(v), igate, fgate, None, a(C0), a(n0), m0, num_blocks=num_blocks)[0]
+    return den_abs / den, np.abs(h_abs)
+
+
+def conditioned_excess(h, ref, kappa, h_abs, tol: float, delta: float) -> float:
+    """Largest ratio, over tokens and values, of an element's error |h_t,i - ref_t,i| to its
+    bound tol * max_i |ref_t,i| + delta * kappa_t * (h_abs_t,i + |ref_t,i|) (kappa, h_abs from
+    readout_scale); <= 1 passes.  The first term is the fixed tolerance relative to the token's
+    own read-out (stricter than relative to the whole slice, which one huge token of a slice
+    would make lenient on all the others), the second what a relative error delta in the terms
+    costs a token whose read-out cancels."""
     h = np.asarray(h, np.float64)
     ref = np.asarray(ref, np.float64)
     B, NH, S, DHV = ref.shape
     nb = kappa.shape[2]
-    hb = h.reshape(B, NH, S, nb, DHV // nb).transpose(0, 1, 3, 2, 4)
-    rb = ref.reshape(B, NH, S, nb, DHV // nb).transpose(0, 1, 3, 2, 4)
+    split = lambda x: np.asarray(x, np.float64).reshape(B, NH, S, nb, DHV // nb).transpose(0, 1, 3, 2, 4)
+    hb, rb, ab = split(h), split(ref), split(h_abs)
     if not np.all(np.isfinite(hb)):
         return float("inf")
-    err = np.max(np.abs(hb - rb), -1)                         # [B, NH, nb, S]
-    tok = np.max(np.abs(rb), -1)                              # [B, NH, nb, S]
-    scale = np.max(tok, -1, keepdims=True)                    # [B, NH, nb, 1]
-    bound = tol * np.maximum(scale, 1e-30) + delta * kappa * tok
-    return float(np.max(err / bound))
+    tok = np.max(np.abs(rb), axis=-1, keepdims=True)            # [B, NH, nb, S, 1]
+    bound = tol * tok + delta * kappa[..., None] * (ab + np.abs(rb))
+    return float(np.max(np.abs(hb - rb) / np.maximum(bound, 1e-300)))
 
 
 class Guarded:

@@ -10,8 +10,8 @@ import torch
 
 import oracle
 from linear_recurrent_token_b200 import inputs, mlstm
-from tests.helpers import (TOL, TORCH_DTYPE, Guarded, conditioned_excess, denominator_condition, dev, host,
-                           m_err, slice_relerr)
+from tests.helpers import (TOL, TORCH_DTYPE, Guarded, conditioned_excess, dev, host, m_err, readout_scale,
+                           slice_relerr)
 
 pytestmark = pytest.mark.gpu
 
@@ -248,21 +248,21 @@ def test_large_input_gates_stay_finite():
 
 
 def test_large_input_gates_signed_inputs_within_conditioned_bound():
-    # The same input gates with q and k of both signs.  n'.q can now cancel: a token whose
-    # denominator terms sum to kappa_t times the denominator loses kappa_t times the relative
-    # accuracy of those terms, in any fixed-precision evaluation.  The bound per token is the
-    # fp32 tolerance of the slice plus delta * kappa_t * |h_t|, with delta = 2^-20 (sixteen
-    # fp32 roundings: the recurrence of n' and a 16-term dot product).
+    # The same input gates with q and k of both signs.  n'.q (and C'q) can now cancel: a token
+    # whose read-out terms sum to many times the read-out loses that factor of the relative
+    # accuracy of those terms, in any fixed-precision evaluation (tests.helpers.readout_scale).
+    # The bound per element is the fp32 tolerance relative to the token's own read-out plus
+    # 2^-20 (sixteen fp32 roundings) kappa_t (h_abs + |h|).
     w = inputs.WORKLOADS[0]
     inp = inputs.forward_inputs(w, seed=80)
     inp["igate"] = inp["igate"] + 60.0
     got = gpu_fwd(inp, "f32", 16)
     assert all(np.all(np.isfinite(x)) for x in got)
     ref = oracle_fwd(inp)
-    kappa = denominator_condition(inp["q"], inp["k"], inp["igate"], inp["fgate"])
+    kappa, h_abs = readout_scale(inp["q"], inp["k"], inp["v"], inp["igate"], inp["fgate"])
     assert kappa.max() > 1e3  # the case really has cancelling denominators
-    excess = conditioned_excess(got[0], ref[0], kappa, TOL["f32"], 2.0 ** -20)
-    assert excess <= 1.0, (excess, kappa.max())
+    excess = conditioned_excess(got[0], ref[0], kappa, h_abs, TOL["f32"], 2.0 ** -20)
+    assert excess <= 1.0, excess
     errs = {"C": slice_relerr(got[1], ref[1], 3), "n": slice_relerr(got[2], ref[2], 3), "m": m_err(got[3], ref[3])}
     assert all(e <= TOL["f32"] for e in errs.values()), errs
 
@@ -444,8 +444,26 @@ def test_tensor_core_gate_regimes(regime, DHV, signs):
     m0 = rs.standard_normal((B, NH)).astype(np.float32)
     got = gpu_fwd(inp, "bf16", 64, C0=C0, n0=n0, m0=m0)
     assert all(np.all(np.isfinite(x)) for x in got), regime
-    errs = check(got, oracle_fwd(inp, C0=C0, n0=n0, m0=m0), "bf16", what=f"{regime} {signs}")
-    print(regime, signs, errs)
+    ref = oracle_fwd(inp, C0=C0, n0=n0, m0=m0)
+    if signs == "nonneg":
+        print(regime, signs, check(got, ref, "bf16", what=f"{regime} {signs}"))
+        return
+    # Signed inputs: the final state (no cancellation) at the flat bound; h per element at the flat
+    # bound relative to its own token plus 2^-8 kappa_t (h_abs + |h|) (tests.helpers.readout_scale),
+    # 2^-8 being two bf16
+    # roundings of the terms: the read-out reads a bf16 copy of the state, and the state itself
+    # accumulates bf16 products V o u.  An input spike makes the state one dominant rank-1 term,
+    # and a token whose query is nearly orthogonal to that key cancels it in num and den alike;
+    # an fp64 evaluation that rounds only the read-out's copy of the state to bf16 already misses
+    # the flat bound by 3x on the spike regimes (6.5 % at DHV 128, 20 % at 512).  Most tokens'
+    # kappa is small, so the bound stays the flat one for them (an h of the wrong sign on one
+    # token in twenty exceeds it 28-47 times in the spike and shift regimes).
+    errs = {"C": slice_relerr(got[1], ref[1], 3), "n": slice_relerr(got[2], ref[2], 3), "m": m_err(got[3], ref[3])}
+    assert all(e <= TOL["bf16"] for e in errs.values()), (regime, errs)
+    kappa, h_abs = readout_scale(inp["q"], inp["k"], inp["v"], inp["igate"], inp["fgate"], C0, n0, m0)
+    excess = conditioned_excess(got[0], ref[0], kappa, h_abs, TOL["bf16"], 2.0 ** -8)
+    assert excess <= 1.0, (regime, excess, slice_relerr(got[0], ref[0], 2))
+    print(regime, signs, errs, "h excess", excess, "flat h error", slice_relerr(got[0], ref[0], 2))
 
 
 @pytest.mark.parametrize("dtype,chunk,nb,retention,with_o", [
@@ -515,4 +533,57 @@ def test_scalar_normaliser_prefill(dtype, chunk, nb, with_o, with_state):
     tol = TOL[dtype]
     errs = {"h": slice_relerr(host(h), hr, 2), "C": slice_relerr(host(C), Cr, 3),
             "n": float(np.max(np.abs(host(n) - nr)) / max(np.max(np.abs(nr)), 1e-30)), "m": m_err(host(m), mr)}
+    assert all(e <= tol for e in errs.values()), errs
+
+
+SN_TC_CASES = [
+    # B, NH, S, DHQK, DHV, nb, with_o, with_state
+    (1, 2, 700, 128, 256, 1, True, True),      # several segments (segment summaries of the scalar n)
+    (2, 2, 333, 64, 128, 1, False, False),     # ragged last chunk, zero initial state
+    (1, 4, 2048, 256, 512, 1, False, True),    # the large-head shape
+    (2, 2, 640, 128, 128, 2, True, True),      # two blocks sharing the head's scalar n
+]
+
+
+@pytest.mark.parametrize("case", SN_TC_CASES, ids=[f"B{c[0]}NH{c[1]}S{c[2]}k{c[3]}v{c[4]}nb{c[5]}" for c in SN_TC_CASES])
+def test_scalar_normaliser_prefill_tensor_core(case):
+    """The scalar-normaliser variant on the tensor-core kernels (bf16, chunk 64) against
+    oracle.sequential_scalar_normaliser: h, C, the per-head n and m, outputs guard-banded."""
+    B, NH, S, DHQK, DHV, nb, with_o, with_state = case
+    assert mlstm.plan(mlstm.fwd_params(B, NH, S, DHQK, DHV, 64, nb, torch.bfloat16, False))["tensor_core"] == 1
+    w = inputs.Workload(3, "sn_tc", B, NH, S, DHQK, DHV, 64, nb, "bf16", False, 1 / np.sqrt(DHQK // nb))
+    inp = inputs.forward_inputs(w, seed=sum(case[:5]))
+    rng = np.random.default_rng(19)
+    dk, dv = DHQK // nb, DHV // nb
+    bias = (rng.standard_normal(NH) * 2.0).astype(np.float32)
+    C0 = n0 = m0 = og = None
+    if with_state:
+        C0 = (rng.standard_normal((B, NH, nb, dv, dk)) * 0.2).astype(np.float32)
+        n0 = (rng.standard_normal((B, NH)) * 0.5).astype(np.float32)
+        m0 = rng.standard_normal((B, NH)).astype(np.float32)
+    if with_o:
+        og = inputs.round_to(rng.uniform(0, 1, (B, NH, S, DHV)), "bf16")
+    td = torch.bfloat16
+    gd = {"h": Guarded((B, NH, S, DHV), td), "C": Guarded((B, NH, nb, dv, dk), torch.float32),
+          "n": Guarded((B, NH), torch.float32), "m": Guarded((B, NH), torch.float32)}
+    p = mlstm.fwd_params(B, NH, S, DHQK, DHV, 64, nb, td, False)
+    ws = torch.empty(mlstm.scalar_normaliser_workspace_size(p), dtype=torch.uint8, device="cuda")
+    lib = mlstm.lib()
+    ptr = lambda t: None if t is None else t.data_ptr()
+    args = [dev(inp[x], td) for x in ("q", "k", "v")] + [dev(inp["igate"]), dev(inp["fgate"]),
+                                                          dev(og, td) if og is not None else None, dev(bias),
+                                                          dev(C0), dev(n0), dev(m0)]
+    import ctypes
+    st = lib.mlstm_fwd_chunkwise_scalar_normaliser(
+        ctypes.byref(p), *[ptr(a) for a in args], gd["h"].t.data_ptr(), gd["C"].t.data_ptr(), gd["n"].t.data_ptr(),
+        gd["m"].t.data_ptr(), ws.data_ptr(), ctypes.c_size_t(ws.numel()), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0, mlstm.status_string(st)
+    assert mlstm.fwd_status(p, ws) == 0  # synchronises; no bounded wait ran out
+    assert_guards_intact(gd, f"scalar normaliser {case}")
+    hr, Cr, nr, mr = oracle.sequential_scalar_normaliser(inp["q"], inp["k"], inp["v"], inp["igate"], inp["fgate"],
+                                                         bias, og, C0, n0, m0, num_blocks=nb)
+    tol = TOL["bf16"]
+    errs = {"h": slice_relerr(host(gd["h"].t), hr, 2), "C": slice_relerr(host(gd["C"].t), Cr, 3),
+            "n": float(np.max(np.abs(host(gd["n"].t) - nr)) / max(np.max(np.abs(nr)), 1e-30)),
+            "m": m_err(host(gd["m"].t), mr)}
     assert all(e <= tol for e in errs.values()), errs
