@@ -747,17 +747,28 @@ def gdn2_over_ranks(gdn2, world, sm_mhz):
     return out
 
 
-def backward_line(w, ms, sm_mhz, cpu: bool):
+def backward_uses_cluster(dtype, dk, dv):
+    """Whether mlstm_bwd runs the cluster kernel (warp-level bf16 MMAs) for these block widths:
+    bf16, key width 64 / 128 / 256, value width a multiple of 64 up to 512 (the library's rule)."""
+    return dtype == "bf16" and dk in (64, 128, 256) and dv % 64 == 0 and 64 <= dv <= 512
+
+
+def backward_line(w, ms, sm_mhz, cpu: bool, peaks=None):
     step_ms = statistics.median(ms)
     flops = backward_flops(w.B, w.NH, w.S, w.dk, w.dv, w.num_blocks)
-    peak = fp32_simt_peak_tflops(sm_mhz)
     tf = flops / (step_ms * 1e-3) / 1e12
+    if backward_uses_cluster(w.dtype, w.dk, w.dv):
+        peak = (peaks or FALLBACK_PEAKS)["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                "traffic": None, "kernel": "bwd_cluster_kernel (warp-level bf16 MMAs, a cluster of dv/64 CTAs per head)",
+                "flops_per_launch": flops, "peak_source": "bf16 tensor peak (burst)"}
+    else:
+        peak = fp32_simt_peak_tflops(sm_mhz)
+        roof = {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                "traffic": None, "kernel": "bwd_kernel (SIMT, one CTA per head)", "flops_per_launch": flops,
+                "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x median SM clock"}
     out = {"workload": w.describe(), "value": w.B * w.S / (step_ms * 1e-3), "unit": "tokens/s",
-           "ms_per_step": step_ms, "steps": len(ms), "dtype": "f32 (inputs " + w.dtype + ")",
-           "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
-                        "traffic": None, "kernel": "bwd_kernel (SIMT, one CTA per head)",
-                        "flops_per_launch": flops,
-                        "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x median SM clock"}}
+           "ms_per_step": step_ms, "steps": len(ms), "dtype": "f32 (inputs " + w.dtype + ")", "roofline": roof}
     if cpu:
         tokens = min(w.S, 64)
         heads = min(w.NH, 2)
@@ -827,7 +838,7 @@ def compact_legs(line):
         legs["reversed"] = {"tok/s": _r(line["reversed"]["value"]), "ms": _r(line["reversed"]["ms_per_step"])}
     for e in line.get("backward", []):
         legs["bwd_" + e["workload"].split(":")[0]] = {"tok/s": _r(e["value"]), "ms": _r(e["ms_per_step"]),
-                                                       "fp32": _r(e["roofline"]["frac"])}
+                                                       e["roofline"]["bound"]: _r(e["roofline"]["frac"])}
     for e in line.get("scalar_normaliser", []):
         legs["scalar_norm_" + e["workload"].split(":")[0]] = {"tok/s": _r(e["value"]), "ms": _r(e["ms_per_step"])}
     if "msr_block" in line:
@@ -900,7 +911,7 @@ def main():
         dist_barrier(world)
         torch.cuda.synchronize()
         if args.legs == "backward":
-            for idx in (1, 2):
+            for idx in (1, 2, 3):
                 wb = inputs.WORKLOADS[idx]
                 ms = run_backward(wb, args.steps, args.warmup, 256 << 20, clocks)
                 if rank == 0:
@@ -973,7 +984,7 @@ def main():
                 sn.append((wn, run_scalar_normaliser(wn, max(3, args.steps // 4), args.warmup, 256 << 20)))
         bwd = []
         if not args.no_backward and args.legs == "both":
-            for idx in (1, 2):
+            for idx in (1, 2, 3):
                 wb = inputs.WORKLOADS[idx]
                 bwd.append((wb, run_backward(wb, max(3, args.steps // 4), args.warmup, 256 << 20, clocks)))
             dist_barrier(world)
@@ -1058,7 +1069,7 @@ def main():
             line["gpu_launches"] += len(ms) * 2
     if bwd:
         sm_mhz = line["clocks"].get("sm_mhz")
-        line["backward"] = [backward_line(wb, ms, sm_mhz, rank == 0 and world == 1 and not args.no_cpu_baseline)
+        line["backward"] = [backward_line(wb, ms, sm_mhz, rank == 0 and world == 1 and not args.no_cpu_baseline, peaks)
                             for wb, ms in bwd]
         line["gpu_launches"] += sum(len(ms) for _, ms in bwd)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

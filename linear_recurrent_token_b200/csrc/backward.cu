@@ -23,12 +23,14 @@
 // backward (D, G: dv, dk, ditilde); a last pass forms the gate gradients.  The state of one
 // block lives in shared memory (value rows padded by one column against bank conflicts):
 // a thread per value row for row products, a thread per key column for column products.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace mlstm {
 namespace {
@@ -735,6 +737,687 @@ __global__ void __launch_bounds__(NTB, 1) bwd_chunk_kernel(BwdArgs a) {
 
 }  // namespace
 
+// =======================================================================================
+// Cluster form of the chunked backward, for blocks whose state does not fit one CTA (the
+// 256 x 512 head): a thread-block cluster per (batch, head), CTA `rank` owning value rows
+// [64 rank, 64 rank + 64) of each block's state (C' in phase 1, D in phase 2) in registers
+// as warp-MMA accumulators, bf16 inputs.  The chunk algebra is the one of bwd_chunk_kernel
+// (32-token chunks); every product over the chunk is an m16n8k16 bf16 MMA with fp32
+// accumulation (operands from shared memory by ldmatrix), and the sums over value rows that
+// span the cluster meet in distributed shared memory:
+//   phase 1: P_t = sum_r o dh num / den (every CTA reads every CTA's partial, so each has
+//            dd_t), dq (each CTA adds the partials of its 1/NC of the key columns, plus the
+//            dd term);
+//   phase 2: dk (the same column split, plus the dd and G terms), ditilde_t by atomics on the
+//            per-head workspace.
+// n' / G (one key vector per block) is kept by every CTA.  Two cluster barriers per chunk:
+// after the partials are written, and before they are overwritten.
+namespace {
+
+namespace cg = cooperative_groups;
+using namespace sm100;
+typedef __nv_bfloat16 bf16_t;
+
+constexpr int BCL = 32;          // chunk length
+constexpr int BCV = 64;          // value rows per CTA
+constexpr int BCT = 256;         // threads per CTA
+constexpr int LDV = BCV + 8;     // bf16 row stride of [BCL][BCV] tiles (16-byte rows, odd 16-byte count)
+constexpr int LDL = BCL + 8;     // bf16 row stride of [BCL][BCL] tiles
+constexpr int LDF = BCV + 1;     // fp32 row stride of [BCL][BCV] tiles
+constexpr int LDW = BCL + 1;     // fp32 row stride of [BCL][BCL] tiles
+
+template <int DK>
+struct BcSmem {
+  static constexpr int LDK = DK + 8;  // bf16 row stride of [.][DK] tiles
+  static constexpr int Q = 0;                        // bf16 [BCL][LDK]
+  static constexpr int K = Q + BCL * LDK * 2;        // bf16 [BCL][LDK]
+  static constexpr int CB = K + BCL * LDK * 2;       // bf16 [BCV][LDK]: copy of the state (C' or D)
+  static constexpr int VB = CB + BCV * LDK * 2;      // bf16 [BCL][LDV]
+  static constexpr int AB = VB + BCL * LDV * 2;      // bf16 [BCL][LDV]: V o w (phase 1), dN o A (phase 2)
+  static constexpr int DNB = AB + BCL * LDV * 2;     // bf16 [BCL][LDV]: dN
+  static constexpr int PB = DNB + BCL * LDV * 2;     // bf16 [BCL][LDL]: P
+  static constexpr int XB = PB + BCL * LDL * 2;      // bf16 [BCL][LDL]: X = W o (dN V^T), this CTA's rows
+  static constexpr int DH = XB + BCL * LDL * 2;      // f32 [BCL][LDF]
+  static constexpr int O = DH + BCL * LDF * 4;       // f32 [BCL][LDF]
+  static constexpr int W = O + BCL * LDF * 4;        // f32 [BCL][LDW]
+  static constexpr int P = W + BCL * LDW * 4;        // f32 [BCL][LDW]
+  static constexpr int R = P + BCL * LDW * 4;        // f32 [BCL][DK]: this CTA's partial dq / dk
+  static constexpr int NV = R + BCL * DK * 4;        // f32 [DK]: n' (phase 1) / G (phase 2)
+  static constexpr int TOK = NV + DK * 4;            // f32 [12][BCL] per-token values
+  static constexpr int BYTES = TOK + 12 * BCL * 4;
+};
+
+// acc[NT] (16 x 8 tiles at rows m0.., columns n0 + 8 nt) += A[m0 : m0 + 16, 0 : K] B[0 : K, n0 : ..].
+// A bf16 in shared memory stored [m][k] (ATR false) or [k][m] (ATR true), row stride lda;
+// B stored [n][k] (BTR false) or [k][n] (BTR true), row stride ldb.  One warp.
+template <bool ATR, bool BTR, int NT>
+__device__ __forceinline__ void warp_mma(float (&acc)[NT][4], const bf16_t* A, int lda, const bf16_t* B, int ldb,
+                                         int m0, int n0, int K) {
+  const int lane = threadIdx.x & 31;
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    uint32_t a0, a1, a2, a3;
+    if (!ATR)
+      ldmatrix_x4(smem_u32(A + (m0 + (lane & 15)) * lda + k0 + ((lane >> 4) << 3)), a0, a1, a2, a3);
+    else
+      ldmatrix_x4_trans(smem_u32(A + (k0 + (lane & 7) + ((lane >> 4) << 3)) * lda + m0 + (((lane >> 3) & 1) << 3)), a0,
+                        a1, a2, a3);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      uint32_t b0, b1;
+      if (!BTR)
+        ldmatrix_x2(smem_u32(B + (n0 + 8 * nt + (lane & 7)) * ldb + k0 + (((lane >> 3) & 1) << 3)), b0, b1);
+      else
+        ldmatrix_x2_trans(smem_u32(B + (k0 + (lane & 15)) * ldb + n0 + 8 * nt), b0, b1);
+      mma_m16n8k16_bf16(acc[nt], a0, a1, a2, a3, b0, b1);
+    }
+  }
+}
+
+template <int NT>
+__device__ __forceinline__ void zero_acc(float (&acc)[NT][4]) {
+#pragma unroll
+  for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+}
+
+__device__ __forceinline__ uint32_t bf2(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float cl_block_sum(float x, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  __syncthreads();
+  if (lane == 0) red[warp] = x;
+  __syncthreads();
+  float s = 0.f;
+#pragma unroll
+  for (int w = 0; w < BCT / 32; ++w) s += red[w];
+  __syncthreads();
+  return s;
+}
+
+template <int DK>
+__global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
+  using SM = BcSmem<DK>;
+  constexpr int LDK = SM::LDK;
+  constexpr int NS = DK / 16;   // n8 tiles of a warp's share of the state (16 rows x DK/2 columns)
+  constexpr int NQ = DK / 32;   // n8 tiles of a warp's share of a [BCL][DK] product
+  extern __shared__ __align__(16) uint8_t smb[];
+  bf16_t* Qb = reinterpret_cast<bf16_t*>(smb + SM::Q);
+  bf16_t* Kb = reinterpret_cast<bf16_t*>(smb + SM::K);
+  bf16_t* Cb = reinterpret_cast<bf16_t*>(smb + SM::CB);
+  bf16_t* Vb = reinterpret_cast<bf16_t*>(smb + SM::VB);
+  bf16_t* Ab = reinterpret_cast<bf16_t*>(smb + SM::AB);
+  bf16_t* dNb = reinterpret_cast<bf16_t*>(smb + SM::DNB);
+  bf16_t* Pb = reinterpret_cast<bf16_t*>(smb + SM::PB);
+  bf16_t* Xb = reinterpret_cast<bf16_t*>(smb + SM::XB);
+  float* dHf = reinterpret_cast<float*>(smb + SM::DH);
+  float* Of = reinterpret_cast<float*>(smb + SM::O);
+  float* Wm = reinterpret_cast<float*>(smb + SM::W);
+  float* Pm = reinterpret_cast<float*>(smb + SM::P);
+  float* Rp = reinterpret_cast<float*>(smb + SM::R);
+  float* nv = reinterpret_cast<float*>(smb + SM::NV);
+  float* tok = reinterpret_cast<float*>(smb + SM::TOK);
+  float* lA = tok;              // log A_t (cumulative log f' inside the chunk)
+  float* eA = tok + BCL;        // A_t
+  float* li = tok + 2 * BCL;    // log i'_t (-inf past the end)
+  float* tmt = tok + 3 * BCL;   // m_t
+  float* td = tok + 4 * BCL;    // d_t = n'_t . q_t
+  float* tden = tok + 5 * BCL;  // den_t
+  float* tdd = tok + 6 * BCL;   // dd_t
+  float* tpp = tok + 7 * BCL;   // this CTA's partial of P_t; ditilde partials in phase 2
+  float* wv = tok + 8 * BCL;    // w_s = W[Lc-1][s]
+  float* tdn = tok + 9 * BCL;   // ditilde partial of the n part (phase 2)
+  float* red = tok + 10 * BCL;  // [8] block sums
+  float* scal = red + 8;        // [0] final-state term, [1] dm0 (partials of this CTA)
+
+  cg::cluster_group cl = cg::this_cluster();
+  const int NC = (int)cl.num_blocks(), rank = (int)cl.block_rank();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, tq = lane & 3;
+  const int bh = blockIdx.y, head = bh % a.NH;
+  const int dv = a.dv, S = a.S, r0 = rank * BCV;
+  const bool ret = a.retention != 0;
+  const bf16_t* q = static_cast<const bf16_t*>(a.q);
+  const bf16_t* k = static_cast<const bf16_t*>(a.k);
+  const bf16_t* v = static_cast<const bf16_t*>(a.v);
+  const bf16_t* dh = static_cast<const bf16_t*>(a.dh);
+  const bf16_t* og = ret ? nullptr : static_cast<const bf16_t*>(a.og);
+  float* wlf = a.ws + (size_t)bh * 8 * S;
+  float* wli = wlf + S;
+  float* wm = wli + S;
+  float* wr = wm + S;
+  float* wdi = wr + S;
+  float* wden = wdi + S;
+  float* wd = wden + S;
+  float* wdd = wd + S;
+  // this warp's share of the state: rows 16 rt .. +16, key columns hc DK/2 .. +DK/2
+  const int rt = warp & 3, hc = warp >> 2;
+  float st[NS][4];
+
+  // ---- gates (rank 0, warp 0: the stabiliser recurrence as a max-plus scan), workspace sums zeroed
+  if (rank == 0) {
+    if (warp == 0) {
+      if (ret) {
+        const float lg = retention_log_gamma(head);
+        for (int t = lane; t < S; t += 32) {
+          wlf[t] = lg;
+          wli[t] = 0.f;
+          wm[t] = 0.f;
+        }
+      } else {
+        const int seg = (S + 31) / 32, t_lo = lane * seg, t_hi = min(S, t_lo + seg);
+        MaxPlus mp{0.f, -INFINITY};
+        for (int t = t_lo; t < t_hi; ++t)
+          mp = mp_then(mp, MaxPlus{log_sigmoid(a.fg[(size_t)bh * S + t]), a.ig[(size_t)bh * S + t]});
+        for (int o = 1; o < 32; o <<= 1) {
+          const float A = __shfl_up_sync(0xffffffffu, mp.A, o), Bm = __shfl_up_sync(0xffffffffu, mp.Bm, o);
+          if (lane >= o) mp = mp_then(MaxPlus{A, Bm}, mp);
+        }
+        float ex_A = __shfl_up_sync(0xffffffffu, mp.A, 1), ex_B = __shfl_up_sync(0xffffffffu, mp.Bm, 1);
+        if (lane == 0) {
+          ex_A = 0.f;
+          ex_B = -INFINITY;
+        }
+        float m = mp_apply(MaxPlus{ex_A, ex_B}, a.m0 ? a.m0[bh] : 0.f);
+        for (int t = t_lo; t < t_hi; ++t) {
+          const float lf = log_sigmoid(a.fg[(size_t)bh * S + t]), it = a.ig[(size_t)bh * S + t];
+          const float mn = fmaxf(lf + m, it);
+          wlf[t] = lf + m - mn;
+          wli[t] = it - mn;
+          wm[t] = mn;
+          m = mn;
+        }
+      }
+    }
+    for (int t = tid; t < S; t += BCT) {
+      wr[t] = 0.f;
+      wdi[t] = 0.f;
+    }
+  }
+  if (tid == 0) {
+    scal[0] = 0.f;
+    scal[1] = 0.f;
+  }
+  cl.sync();
+
+  const int nck = (S + BCL - 1) / BCL;
+  for (int blk = 0; blk < a.nb; ++blk) {
+    const size_t slice = (size_t)bh * a.nb + blk;
+    const size_t qoff = (size_t)bh * S * a.DHQK + (size_t)blk * DK;
+    const size_t voff = (size_t)bh * S * a.DHV + (size_t)blk * dv + r0;
+    const size_t soff = slice * (size_t)dv * DK + (size_t)r0 * DK;  // this CTA's rows of a state
+
+    // chunk inputs, gate logs, W and P (every CTA: the key-side products are redundant)
+    auto load_chunk = [&](int t0, int Lc) {
+      for (int e = tid; e < BCL * (DK / 8); e += BCT) {
+        const int t = e / (DK / 8), c = (e % (DK / 8)) * 8;
+        uint4 uq = make_uint4(0, 0, 0, 0), uk = uq;
+        if (t < Lc) {
+          uq = *reinterpret_cast<const uint4*>(q + qoff + (size_t)(t0 + t) * a.DHQK + c);
+          uk = *reinterpret_cast<const uint4*>(k + qoff + (size_t)(t0 + t) * a.DHQK + c);
+        }
+        *reinterpret_cast<uint4*>(Qb + t * LDK + c) = uq;
+        *reinterpret_cast<uint4*>(Kb + t * LDK + c) = uk;
+      }
+      for (int e = tid; e < BCL * (BCV / 8); e += BCT) {
+        const int t = e / (BCV / 8), c = (e % (BCV / 8)) * 8;
+        uint4 uv = make_uint4(0, 0, 0, 0), uh = uv, uo = uv;
+        if (t < Lc) {
+          const size_t off = voff + (size_t)(t0 + t) * a.DHV + c;
+          uv = *reinterpret_cast<const uint4*>(v + off);
+          uh = *reinterpret_cast<const uint4*>(dh + off);
+          if (og) uo = *reinterpret_cast<const uint4*>(og + off);
+        }
+        *reinterpret_cast<uint4*>(Vb + t * LDV + c) = uv;
+        const bf16_t* hb = reinterpret_cast<const bf16_t*>(&uh);
+        const bf16_t* ob = reinterpret_cast<const bf16_t*>(&uo);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          dHf[t * LDF + c + j] = __bfloat162float(hb[j]);
+          Of[t * LDF + c + j] = og ? __bfloat162float(ob[j]) : 1.f;
+        }
+      }
+      if (warp == 0) {
+        float x = lane < Lc ? wlf[t0 + lane] : 0.f;
+        for (int o = 1; o < 32; o <<= 1) {
+          const float y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        lA[lane] = x;
+        eA[lane] = expf(x);
+        li[lane] = lane < Lc ? wli[t0 + lane] : -INFINITY;
+        tmt[lane] = lane < Lc ? wm[t0 + lane] : 0.f;
+      }
+      __syncthreads();
+      {  // S = Q K^T: warp -> rows 16 (w >> 2), columns 8 (w & 3)
+        float acc[1][4];
+        zero_acc(acc);
+        const int m0 = 16 * (warp >> 2), n0 = 8 * (warp & 3);
+        warp_mma<false, false, 1>(acc, Qb, LDK, Kb, LDK, m0, n0, DK);
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int t = m0 + g + 8 * h2, s0 = n0 + 2 * tq;
+          float wv2[2], pv2[2];
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int s2 = s0 + j;
+            const float w = (s2 <= t && t < Lc) ? expf(lA[t] - lA[s2] + li[s2]) : 0.f;
+            wv2[j] = w;
+            pv2[j] = w * acc[0][2 * h2 + j];
+            Wm[t * LDW + s2] = w;
+            Pm[t * LDW + s2] = pv2[j];
+          }
+          *reinterpret_cast<uint32_t*>(Pb + t * LDL + s0) = bf2(pv2[0], pv2[1]);
+        }
+      }
+      __syncthreads();
+      if (tid < BCL) wv[tid] = Wm[(Lc - 1) * LDW + tid];
+    };
+    // X = W o (dN V^T) over this CTA's value rows, into Xb: warp -> rows 16 (w >> 2), cols 8 (w & 3)
+    auto make_x = [&]() {
+      float acc[1][4];
+      zero_acc(acc);
+      const int m0 = 16 * (warp >> 2), n0 = 8 * (warp & 3);
+      warp_mma<false, false, 1>(acc, dNb, LDV, Vb, LDV, m0, n0, BCV);
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int t = m0 + g + 8 * h2, s0 = n0 + 2 * tq;
+        *reinterpret_cast<uint32_t*>(Xb + t * LDL + s0) =
+            bf2(Wm[t * LDW + s0] * acc[0][2 * h2], Wm[t * LDW + s0 + 1] * acc[0][2 * h2 + 1]);
+      }
+    };
+    // the bf16 copy of this CTA's state rows (the warps' accumulators) for the products
+    auto state_to_cb = [&]() {
+#pragma unroll
+      for (int nt = 0; nt < NS; ++nt) {
+        const int c = hc * (DK / 2) + 8 * nt + 2 * tq, r = 16 * rt + g;
+        *reinterpret_cast<uint32_t*>(Cb + r * LDK + c) = bf2(st[nt][0], st[nt][1]);
+        *reinterpret_cast<uint32_t*>(Cb + (r + 8) * LDK + c) = bf2(st[nt][2], st[nt][3]);
+      }
+    };
+    // a state (C0 or dC, [dv][DK] per slice) into the accumulators; NULL = zeros
+    auto load_state = [&](const float* src) {
+#pragma unroll
+      for (int nt = 0; nt < NS; ++nt) {
+        const int c = hc * (DK / 2) + 8 * nt + 2 * tq, r = 16 * rt + g;
+        float2 x = make_float2(0.f, 0.f), y = x;
+        if (src) {
+          x = *reinterpret_cast<const float2*>(src + soff + (size_t)r * DK + c);
+          y = *reinterpret_cast<const float2*>(src + soff + (size_t)(r + 8) * DK + c);
+        }
+        st[nt][0] = x.x;
+        st[nt][1] = x.y;
+        st[nt][2] = y.x;
+        st[nt][3] = y.y;
+      }
+    };
+    // <state, src> over this CTA's rows (src [dv][DK] per slice)
+    auto state_dot = [&](const float* src) {
+      float part = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < NS; ++nt) {
+        const int c = hc * (DK / 2) + 8 * nt + 2 * tq, r = 16 * rt + g;
+        const float2 x = *reinterpret_cast<const float2*>(src + soff + (size_t)r * DK + c);
+        const float2 y = *reinterpret_cast<const float2*>(src + soff + (size_t)(r + 8) * DK + c);
+        part += st[nt][0] * x.x + st[nt][1] * x.y + st[nt][2] * y.x + st[nt][3] * y.y;
+      }
+      return part;
+    };
+    const int CW = (DK + NC - 1) / NC;  // key columns this CTA reduces (the last rank may have fewer)
+
+    // ------------------------------------------------------------------ phase 1 (forward)
+    load_state(a.C0);
+    for (int c = tid; c < DK; c += BCT) nv[c] = (!ret && a.n0) ? a.n0[slice * DK + c] : 0.f;
+    for (int ch = 0; ch < nck; ++ch) {
+      const int t0 = ch * BCL, Lc = min(BCL, S - t0);
+      state_to_cb();
+      if (tid < BCL) tpp[tid] = 0.f;
+      load_chunk(t0, Lc);  // ends with a barrier after W, P
+      // d_t and den_t (every CTA; a warp per token)
+      for (int t = warp; t < BCL; t += BCT / 32) {
+        float x = 0.f;
+        if (!ret && t < Lc)
+          for (int c = lane; c < DK; c += 32) x += __bfloat162float(Qb[t * LDK + c]) * nv[c];
+        x *= eA[t];
+        if (!ret && t < Lc) x += Pm[t * LDW + lane];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        if (lane == 0) {
+          td[t] = ret ? 0.f : x;
+          tden[t] = ret ? 1.f : fmaxf(fabsf(x), expf(-tmt[t]));
+        }
+      }
+      __syncthreads();
+      {  // num = diag(A) Q C'^T + P V (this CTA's rows): warp -> tokens 16 (w & 1), rows 16 (w >> 1)
+        float acc[2][4];
+        zero_acc(acc);
+        const int m0 = 16 * (warp & 1), n0 = 16 * (warp >> 1);
+        warp_mma<false, false, 2>(acc, Qb, LDK, Cb, LDK, m0, n0, DK);
+        const float e_lo = eA[m0 + g], e_hi = eA[m0 + g + 8];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          acc[nt][0] *= e_lo;
+          acc[nt][1] *= e_lo;
+          acc[nt][2] *= e_hi;
+          acc[nt][3] *= e_hi;
+        }
+        warp_mma<false, true, 2>(acc, Pb, LDL, Vb, LDV, m0, n0, BCL);
+        float pp[2] = {0.f, 0.f};
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int t = m0 + g + 8 * h2;
+          const float den = tden[t];
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            const int r = n0 + 8 * nt + 2 * tq;
+            float dn2[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const float hn = acc[nt][2 * h2 + j] / den;
+              const float o = Of[t * LDF + r + j], dhv = dHf[t * LDF + r + j];
+              dn2[j] = t < Lc ? o * dhv / den : 0.f;
+              pp[h2] += o * dhv * hn;
+              if (a.dog && t < Lc) a.dog[voff + (size_t)(t0 + t) * a.DHV + r + j] = dhv * hn;
+            }
+            *reinterpret_cast<uint32_t*>(dNb + t * LDV + r) = bf2(dn2[0], dn2[1]);
+          }
+        }
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          pp[h2] += __shfl_xor_sync(0xffffffffu, pp[h2], 1);
+          pp[h2] += __shfl_xor_sync(0xffffffffu, pp[h2], 2);
+          if (tq == 0 && !ret) atomicAdd(&tpp[m0 + g + 8 * h2], pp[h2]);
+        }
+      }
+      cl.sync();  // every CTA's P partials (and this CTA's dN) are written
+      if (tid < BCL) {
+        const int t = tid;
+        float P = 0.f;
+        for (int i = 0; i < NC; ++i) P += cl.map_shared_rank(tpp, i)[t];
+        const float d = td[t], den = tden[t];
+        const float dd = (!ret && t < Lc && fabsf(d) > expf(-tmt[t])) ? -P / den * copysignf(1.f, d) : 0.f;
+        tdd[t] = dd;
+        if (rank == 0 && t < Lc) {
+          wden[t0 + t] = den;
+          wd[t0 + t] = d;
+          wdd[t0 + t] = dd;
+          if (!ret) atomicAdd(&wr[t0 + t], P + dd * d);
+        }
+      }
+      make_x();
+      // V o w for the state update
+      for (int e = tid; e < BCL * BCV / 2; e += BCT) {
+        const int s2 = e / (BCV / 2), r = 2 * (e % (BCV / 2));
+        const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(Vb + s2 * LDV + r));
+        *reinterpret_cast<uint32_t*>(Ab + s2 * LDV + r) = bf2(x.x * wv[s2], x.y * wv[s2]);
+      }
+      __syncthreads();
+      {  // partial dq = diag(A) dN C' + X K: warp -> tokens 16 (w & 1), key columns (w >> 1) DK/4
+        float acc[NQ][4];
+        zero_acc(acc);
+        const int m0 = 16 * (warp & 1), n0 = (warp >> 1) * (DK / 4);
+        warp_mma<false, true, NQ>(acc, dNb, LDV, Cb, LDK, m0, n0, BCV);
+        const float e_lo = eA[m0 + g], e_hi = eA[m0 + g + 8];
+#pragma unroll
+        for (int nt = 0; nt < NQ; ++nt) {
+          acc[nt][0] *= e_lo;
+          acc[nt][1] *= e_lo;
+          acc[nt][2] *= e_hi;
+          acc[nt][3] *= e_hi;
+        }
+        warp_mma<false, true, NQ>(acc, Xb, LDL, Kb, LDK, m0, n0, BCL);
+#pragma unroll
+        for (int nt = 0; nt < NQ; ++nt) {
+          const int c = n0 + 8 * nt + 2 * tq;
+          *reinterpret_cast<float2*>(Rp + (m0 + g) * DK + c) = make_float2(acc[nt][0], acc[nt][1]);
+          *reinterpret_cast<float2*>(Rp + (m0 + g + 8) * DK + c) = make_float2(acc[nt][2], acc[nt][3]);
+        }
+      }
+      cl.sync();  // every CTA's partial dq is written
+      for (int e = tid; e < BCL * CW; e += BCT) {
+        const int t = e / CW, c = rank * CW + e % CW;
+        if (t >= Lc || c >= DK) continue;
+        float x = 0.f;
+        for (int i = 0; i < NC; ++i) x += cl.map_shared_rank(Rp, i)[t * DK + c];
+        const float dd = tdd[t];
+        if (!ret && dd != 0.f) {
+          float wk = 0.f;
+          for (int s2 = 0; s2 <= t; ++s2) wk += Wm[t * LDW + s2] * __bfloat162float(Kb[s2 * LDK + c]);
+          x += dd * (eA[t] * nv[c] + wk);
+        }
+        a.dq[qoff + (size_t)(t0 + t) * a.DHQK + c] = x;
+      }
+      {  // state to the chunk end: C' <- A_L C' + (V o w)^T K
+        const float AL = eA[Lc - 1];
+#pragma unroll
+        for (int nt = 0; nt < NS; ++nt)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) st[nt][j] *= AL;
+        warp_mma<true, true, NS>(st, Ab, LDV, Kb, LDK, 16 * rt, hc * (DK / 2), BCL);
+      }
+      __syncthreads();  // n' is read above (dd term)
+      if (!ret) {
+        const float AL = eA[Lc - 1];
+        for (int c = tid; c < DK; c += BCT) {
+          float x = AL * nv[c];
+          for (int s2 = 0; s2 < Lc; ++s2) x += wv[s2] * __bfloat162float(Kb[s2 * LDK + c]);
+          nv[c] = x;
+        }
+      }
+      __syncthreads();
+    }
+    // final-state term <dC_S, C'_S> + dn_S . n'_S of the forget gradient
+    if (!ret && (a.dC || a.dn)) {
+      float part = a.dC ? state_dot(a.dC) : 0.f;
+      if (a.dn && rank == 0)
+        for (int c = tid; c < DK; c += BCT) part += a.dn[slice * DK + c] * nv[c];
+      const float s2 = cl_block_sum(part, red);
+      if (tid == 0) scal[0] += s2;
+    }
+    cl.sync();  // the per-token workspace of phase 1 is complete
+
+    // ------------------------------------------------------------------ phase 2 (backward)
+    load_state(a.dC);
+    for (int c = tid; c < DK; c += BCT) nv[c] = (!ret && a.dn) ? a.dn[slice * DK + c] : 0.f;
+    for (int ch = nck - 1; ch >= 0; --ch) {
+      const int t0 = ch * BCL, Lc = min(BCL, S - t0);
+      state_to_cb();  // D entering from the later chunks
+      if (tid < BCL) {
+        tpp[tid] = 0.f;
+        tdn[tid] = 0.f;
+      }
+      load_chunk(t0, Lc);
+      if (tid < BCL) {
+        tden[tid] = tid < Lc ? wden[t0 + tid] : 1.f;
+        tdd[tid] = tid < Lc ? wdd[t0 + tid] : 0.f;
+      }
+      __syncthreads();
+      for (int e = tid; e < BCL * BCV / 2; e += BCT) {
+        const int t = e / (BCV / 2), r = 2 * (e % (BCV / 2));
+        float d0 = 0.f, d1 = 0.f;
+        if (t < Lc) {
+          d0 = Of[t * LDF + r] * dHf[t * LDF + r] / tden[t];
+          d1 = Of[t * LDF + r + 1] * dHf[t * LDF + r + 1] / tden[t];
+        }
+        *reinterpret_cast<uint32_t*>(dNb + t * LDV + r) = bf2(d0, d1);
+        *reinterpret_cast<uint32_t*>(Ab + t * LDV + r) = bf2(d0 * eA[t], d1 * eA[t]);
+      }
+      __syncthreads();
+      make_x();
+      __syncthreads();
+      {  // dv = P^T dN + diag(w) K D^T (this CTA's rows): warp -> tokens 16 (w & 1), rows 16 (w >> 1)
+        float acc[2][4], acc2[2][4];
+        zero_acc(acc);
+        zero_acc(acc2);
+        const int m0 = 16 * (warp & 1), n0 = 16 * (warp >> 1);
+        warp_mma<false, false, 2>(acc2, Kb, LDK, Cb, LDK, m0, n0, DK);
+        warp_mma<true, true, 2>(acc, Pb, LDL, dNb, LDV, m0, n0, BCL);
+        float dip[2] = {0.f, 0.f};
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int s2 = m0 + g + 8 * h2;
+          const float w = wv[s2];
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            const int r = n0 + 8 * nt + 2 * tq;
+            const float x0 = acc[nt][2 * h2] + w * acc2[nt][2 * h2];
+            const float x1 = acc[nt][2 * h2 + 1] + w * acc2[nt][2 * h2 + 1];
+            if (s2 < Lc) {
+              *reinterpret_cast<float2*>(a.dv_out + voff + (size_t)(t0 + s2) * a.DHV + r) = make_float2(x0, x1);
+              const float2 vv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(Vb + s2 * LDV + r));
+              dip[h2] += vv.x * x0 + vv.y * x1;
+            }
+          }
+        }
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          dip[h2] += __shfl_xor_sync(0xffffffffu, dip[h2], 1);
+          dip[h2] += __shfl_xor_sync(0xffffffffu, dip[h2], 2);
+          if (tq == 0 && !ret) atomicAdd(&tpp[m0 + g + 8 * h2], dip[h2]);
+        }
+      }
+      {  // partial dk = diag(w) V D + X^T Q: warp -> tokens 16 (w & 1), key columns (w >> 1) DK/4
+        float acc[NQ][4];
+        zero_acc(acc);
+        const int m0 = 16 * (warp & 1), n0 = (warp >> 1) * (DK / 4);
+        warp_mma<false, true, NQ>(acc, Vb, LDV, Cb, LDK, m0, n0, BCV);
+        const float w_lo = wv[m0 + g], w_hi = wv[m0 + g + 8];
+#pragma unroll
+        for (int nt = 0; nt < NQ; ++nt) {
+          acc[nt][0] *= w_lo;
+          acc[nt][1] *= w_lo;
+          acc[nt][2] *= w_hi;
+          acc[nt][3] *= w_hi;
+        }
+        warp_mma<true, true, NQ>(acc, Xb, LDL, Qb, LDK, m0, n0, BCL);
+#pragma unroll
+        for (int nt = 0; nt < NQ; ++nt) {
+          const int c = n0 + 8 * nt + 2 * tq;
+          *reinterpret_cast<float2*>(Rp + (m0 + g) * DK + c) = make_float2(acc[nt][0], acc[nt][1]);
+          *reinterpret_cast<float2*>(Rp + (m0 + g + 8) * DK + c) = make_float2(acc[nt][2], acc[nt][3]);
+        }
+      }
+      cl.sync();  // every CTA's partial dk is written
+      for (int e = tid; e < BCL * CW; e += BCT) {
+        const int s2 = e / CW, c = rank * CW + e % CW;
+        if (s2 >= Lc || c >= DK) continue;
+        float x = 0.f;
+        for (int i = 0; i < NC; ++i) x += cl.map_shared_rank(Rp, i)[s2 * DK + c];
+        if (!ret) {
+          float xn = wv[s2] * nv[c];
+          for (int tau = s2; tau < Lc; ++tau)
+            xn += Wm[tau * LDW + s2] * tdd[tau] * __bfloat162float(Qb[tau * LDK + c]);
+          x += xn;
+          atomicAdd(&tdn[s2], xn * __bfloat162float(Kb[s2 * LDK + c]));
+        }
+        a.dk_out[qoff + (size_t)(t0 + s2) * a.DHQK + c] = x;
+      }
+      {  // D <- A_L D + (dN o A)^T Q
+        const float AL = eA[Lc - 1];
+#pragma unroll
+        for (int nt = 0; nt < NS; ++nt)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) st[nt][j] *= AL;
+        warp_mma<true, true, NS>(st, Ab, LDV, Qb, LDK, 16 * rt, hc * (DK / 2), BCL);
+      }
+      __syncthreads();  // G is read above; the ditilde partials are complete
+      if (!ret) {
+        const float AL = eA[Lc - 1];
+        for (int c = tid; c < DK; c += BCT) {
+          float x = AL * nv[c];
+          for (int tau = 0; tau < Lc; ++tau) x += eA[tau] * tdd[tau] * __bfloat162float(Qb[tau * LDK + c]);
+          nv[c] = x;
+        }
+        if (tid < Lc) {
+          const float di = tpp[tid] + tdn[tid];
+          atomicAdd(&wdi[t0 + tid], di);
+          atomicAdd(&wr[t0 + tid], -di);
+        }
+      }
+      cl.sync();  // the partials have been read before the next chunk overwrites them
+    }
+    // initial-state gradients: dC0 = D, dn0 = G; dm0 = <dC0, C0> + dn0 . n0
+    if (a.dC0) {
+#pragma unroll
+      for (int nt = 0; nt < NS; ++nt) {
+        const int c = hc * (DK / 2) + 8 * nt + 2 * tq, r = 16 * rt + g;
+        *reinterpret_cast<float2*>(a.dC0 + soff + (size_t)r * DK + c) = make_float2(st[nt][0], st[nt][1]);
+        *reinterpret_cast<float2*>(a.dC0 + soff + (size_t)(r + 8) * DK + c) = make_float2(st[nt][2], st[nt][3]);
+      }
+    }
+    if (!ret) {
+      float part = a.C0 ? state_dot(a.C0) : 0.f;
+      if (rank == 0)
+        for (int c = tid; c < DK; c += BCT) {
+          if (a.dn0) a.dn0[slice * DK + c] = nv[c];
+          if (a.n0) part += nv[c] * a.n0[slice * DK + c];
+        }
+      const float s2 = cl_block_sum(part, red);
+      if (tid == 0) scal[1] += s2;
+    }
+    cl.sync();
+  }
+  // ---- gate gradients (rank 0): dlf_t = sum_{tau >= t} r_tau + the final-state term
+  if (!ret && rank == 0 && warp == 0) {
+    float sc2 = 0.f, sc3 = 0.f;
+    for (int i = 0; i < NC; ++i) {
+      sc2 += cl.map_shared_rank(scal, i)[0];
+      sc3 += cl.map_shared_rank(scal, i)[1];
+    }
+    const int seg = (S + 31) / 32, t_lo = lane * seg, t_hi = min(S, t_lo + seg);
+    float sum = 0.f;
+    for (int t = t_lo; t < t_hi; ++t) sum += wr[t];
+    float later = sum;
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y = __shfl_down_sync(0xffffffffu, later, o);
+      if (lane + o < 32) later += y;
+    }
+    float acc = later - sum + sc2;
+    for (int t = t_hi - 1; t >= t_lo; --t) {
+      acc += wr[t];
+      const float ft = a.fg[(size_t)bh * S + t];
+      if (a.dfg) a.dfg[(size_t)bh * S + t] = acc / (1.f + expf(ft));
+      if (a.dig) a.dig[(size_t)bh * S + t] = wdi[t];
+    }
+    if (lane == 0 && a.dm0) a.dm0[bh] = sc3;
+  }
+  cl.sync();  // no CTA leaves while rank 0 may still read its shared memory
+}
+
+// value rows per CTA of the cluster kernel, and its cluster size for these widths (0: not
+// supported): bf16, block key width 64 / 128 / 256, value width a multiple of 64 up to 512
+int bwd_cluster_size(int dtype, int dk, int dv) {
+  if (dtype != 1) return 0;
+  if (dk != 64 && dk != 128 && dk != 256) return 0;
+  if (dv % BCV != 0 || dv / BCV > 8 || dv < BCV) return 0;
+  return dv / BCV;
+}
+
+template <int DK>
+cudaError_t launch_cluster_dk(const BwdArgs& a, long long BH, int nc, cudaStream_t stream) {
+  const int smem = BcSmem<DK>::BYTES;
+  cudaError_t e = cudaFuncSetAttribute(bwd_cluster_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)nc, (unsigned)BH, 1);
+  cfg.blockDim = dim3(BCT, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = (unsigned)nc;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, bwd_cluster_kernel<DK>, a);
+}
+
+}  // namespace
+
 size_t bwd_smem_bytes(int dk, int dv) {
   return ((size_t)dv * (dk + 1) + 4 * (size_t)dk + 5 * (size_t)dv + NTB / 32 + NTB) * sizeof(float);
 }
@@ -765,13 +1448,24 @@ cudaError_t launch_chunked(const BwdArgs& a, long long BH, cudaStream_t stream) 
 }
 }  // namespace
 
-bool bwd_supported(int dk, int dv) {
-  return dk >= 1 && dv >= 1 && dk <= NTB && dv <= NTB && bwd_smem_bytes(dk, dv) <= 200 * 1024;
+bool bwd_supported(int dk, int dv, int dtype) {
+  if (dk >= 1 && dv >= 1 && dk <= NTB && dv <= NTB && bwd_smem_bytes(dk, dv) <= 200 * 1024) return true;
+  return bwd_cluster_size(dtype, dk, dv) > 0;
 }
 
 cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream) {
   const long long BH = (long long)a.B * a.NH;
   if (BH == 0) return cudaSuccess;
+  // bf16 blocks of key width 64 / 128 / 256 and value width a multiple of 64 (up to 512): the
+  // cluster kernel (warp-level MMAs; one CTA per 64 value rows); everything else (fp32 inputs,
+  // narrower blocks): the SIMT kernels with the whole block state in one CTA
+  const int nc = bwd_cluster_size(a.dtype, a.dk, a.dv);
+  if (nc > 0) {
+    if (a.dk == 256) return launch_cluster_dk<256>(a, BH, nc, stream);
+    if (a.dk == 128) return launch_cluster_dk<128>(a, BH, nc, stream);
+    if (a.dk == 64) return launch_cluster_dk<64>(a, BH, nc, stream);
+    return cudaErrorInvalidValue;
+  }
   const int L = bwd_chunk_len(a.dk, a.dv);
   if (L == 32) return a.dtype == 1 ? launch_chunked<__nv_bfloat16, 32>(a, BH, stream) : launch_chunked<float, 32>(a, BH, stream);
   if (L == 16) return a.dtype == 1 ? launch_chunked<__nv_bfloat16, 16>(a, BH, stream) : launch_chunked<float, 16>(a, BH, stream);

@@ -109,7 +109,7 @@ struct BwdArgs {
 };
 size_t bwd_smem_bytes(int dk, int dv);
 size_t bwd_workspace_bytes(long long BH, int S);
-bool bwd_supported(int dk, int dv);
+bool bwd_supported(int dk, int dv, int dtype);
 cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream);
 
 }  // namespace mlstm

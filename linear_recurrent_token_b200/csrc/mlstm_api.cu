@@ -305,7 +305,7 @@ mlstm_status_t check_bwd(const mlstm_fwd_params_t* p, FwdShape* s) {
   s->esize = p->dtype == MLSTM_BF16 ? 2 : 4;
   s->BH = (long long)p->B * p->NH;
   if (s->BH > 0x7fffffffLL || (long long)s->S * s->BH > (1LL << 40)) return MLSTM_ERR_SHAPE;
-  if (!bwd_supported(s->dk, s->dv)) return MLSTM_ERR_SHAPE;
+  if (!bwd_supported(s->dk, s->dv, s->dtype)) return MLSTM_ERR_SHAPE;
   return MLSTM_OK;
 }
 

@@ -73,7 +73,7 @@ __device__ __forceinline__ uint32_t wait_hint_ns(long long limit_cycles) {
 // returns false (the caller records an error and winds down instead of hanging).
 // The polling loop is out of line: kernels with many wait sites keep one copy of it, which
 // stays in the instruction cache.
-__device__ __noinline__ bool mbar_wait_loop(uint64_t* bar, uint32_t parity, long long limit_cycles) {
+static __device__ __noinline__ bool mbar_wait_loop(uint64_t* bar, uint32_t parity, long long limit_cycles) {
   const uint32_t hint = wait_hint_ns(limit_cycles);
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity, hint))
@@ -257,6 +257,17 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, u
                                                   uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr)
+               : "memory");
+}
+// Two 8x8 b16 matrices (threads 0-7 address matrix 0, 8-15 matrix 1); the .trans form
+// delivers the fragments of the transposed matrices.
+__device__ __forceinline__ void ldmatrix_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr) : "memory");
+}
+__device__ __forceinline__ void ldmatrix_x2_trans(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r0), "=r"(r1)
                : "r"(addr)
                : "memory");
 }

@@ -115,3 +115,27 @@ def test_backward_retention_workload_sampled_heads():
     # the retention workload's shapes (64 x 64 per head), a few heads of the batch
     w = inputs.WORKLOADS[2]
     run_case(8, 1, 2, w.S // 4, w.DHQK, w.DHV, 1, w.dtype, retention=True)
+
+
+# ---------------------------------------------------------------- the cluster kernel
+# Blocks whose state does not fit one CTA (bf16, key width 64/128/256, value width a multiple
+# of 64 up to 512): a thread-block cluster per head, 64 value rows per CTA.
+@pytest.mark.parametrize("case", [
+    # seed, B, NH, S, DHQK, DHV, nb, retention, with_state, with_o, with_dstate
+    (11, 1, 2, 200, 256, 512, 1, False, True, True, True),     # the large-head shape, ragged last chunk
+    (12, 1, 1, 96, 256, 512, 1, True, True, False, True),      # retention
+    (13, 2, 1, 70, 128, 384, 1, False, False, False, False),   # six CTAs per cluster, no state
+    (14, 1, 1, 64, 512, 1024, 2, False, True, True, True),     # two blocks of 256 x 512
+])
+def test_backward_cluster_kernel_parity(case):
+    seed, B, NH, S, DHQK, DHV, nb, retention, with_state, with_o, with_dstate = case
+    run_case(seed, B, NH, S, DHQK, DHV, nb, "bf16", retention=retention, with_state=with_state, with_o=with_o,
+             with_dstate=with_dstate)
+
+
+def test_backward_large_head_workload_sampled_heads():
+    """The large-head workload's shapes (256 x 512 per head, bf16), two heads over 1024 tokens
+    (the fp64 oracle over the full 8192 x 8 heads would take minutes)."""
+    w = inputs.WORKLOADS[3]
+    errs = run_case(15, 1, 2, 1024, w.DHQK, w.DHV, 1, w.dtype, with_state=True, with_dstate=True)
+    print("large head backward", errs)
