@@ -1032,14 +1032,16 @@ def main():
         line["gpu_launches"] += r["steps"] * r["plan"]["kernels"]
     if rev_ms:
         rms = dist_max(statistics.median(rev_ms), world)
+        tc = cw["plan"]["tensor_core"]
         esz = 2 if w.dtype == "bf16" else 4
-        copy_bytes = 2 * w.B * w.NH * w.S * ((2 * w.DHQK + 2 * w.DHV) * esz + (0 if w.retention else 8))
+        copy_bytes = 0 if tc else 2 * w.B * w.NH * w.S * ((2 * w.DHQK + 2 * w.DHV) * esz + (0 if w.retention else 8))
         line["reversed"] = {"workload": w.describe(), "value": w.B * w.S * world / (rms * 1e-3), "unit": "tokens/s",
-                            "ms_per_step": rms, "steps": len(rev_ms),
-                            "note": "the forward kernels on reversed copies of q, k, v and the gates, h reversed "
-                                    "back; the copies move reversal_bytes through HBM on top of the forward",
+                            "ms_per_step": rms, "steps": len(rev_ms), "forward_ms": slow_ms,
+                            "note": ("the tensor-core kernels reading the chunks and their rows backwards in place"
+                                     if tc else "the forward kernels on reversed copies of q, k, v and the gates, h "
+                                                "reversed back"),
                             "reversal_bytes": copy_bytes}
-        line["gpu_launches"] += len(rev_ms) * (cw["plan"]["kernels"] + (4 if w.retention else 6))
+        line["gpu_launches"] += len(rev_ms) * (cw["plan"]["kernels"] + (0 if tc else (4 if w.retention else 6)))
     if gdn2:
         line["gdn2"] = gdn2_over_ranks(gdn2, world, line["clocks"].get("sm_mhz"))
         line["gpu_launches"] += gdn2["steps"] * 4  # recurrent, chunk prep + scan, decode step

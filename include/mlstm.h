@@ -221,8 +221,11 @@ mlstm_status_t mlstm_fwd_chunkwise_noalloc_status(const mlstm_fwd_params_t* p, m
  * token 0.  This is the backward direction of a bidirectional encoder (DeepChrInteract-v2
  * "mLSTM Model": a bidirectional wrapper so that the encoder sees context from both sides);
  * a caller combines it with mlstm_fwd_chunkwise as it likes.  Arguments as for
- * mlstm_fwd_chunkwise; the workspace (mlstm_fwd_chunkwise_reversed_workspace_size bytes)
- * also holds reversed copies of the inputs and of h, and must not overlap any argument.
+ * mlstm_fwd_chunkwise; workspace: mlstm_fwd_chunkwise_reversed_workspace_size bytes.  On the
+ * tensor-core path (bf16, chunk 64) the kernels read the chunks and their rows backwards in
+ * place (the chunks stay aligned to multiples of 64 rows from the start of the sequence, so a
+ * ragged chunk is the first one taken) and the workspace is the forward's; elsewhere it also
+ * holds reversed copies of the inputs and of h and must not overlap any argument.
  */
 size_t mlstm_fwd_chunkwise_reversed_workspace_size(const mlstm_fwd_params_t* p);
 mlstm_status_t mlstm_fwd_chunkwise_reversed(const mlstm_fwd_params_t* p,

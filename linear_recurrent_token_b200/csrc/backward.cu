@@ -813,6 +813,24 @@ __device__ __forceinline__ void warp_mma(float (&acc)[NT][4], const bf16_t* A, i
   }
 }
 
+// sum over the cluster's CTAs (nc <= 8) of four floats at the same shared-memory offset; the
+// remote loads are all issued before the first add
+__device__ __forceinline__ float4 sum_remote4(cg::cluster_group& cl, float* local, int nc) {
+  float4 v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    v[i] = i < nc ? *reinterpret_cast<const float4*>(cl.map_shared_rank(local, i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 s = v[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    s.x += v[i].x;
+    s.y += v[i].y;
+    s.z += v[i].z;
+    s.w += v[i].w;
+  }
+  return s;
+}
+
 template <int NT>
 __device__ __forceinline__ void zero_acc(float (&acc)[NT][4]) {
 #pragma unroll
@@ -952,24 +970,33 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
 
     // chunk inputs, gate logs, W and P (every CTA: the key-side products are redundant)
     auto load_chunk = [&](int t0, int Lc) {
-      for (int e = tid; e < BCL * (DK / 8); e += BCT) {
-        const int t = e / (DK / 8), c = (e % (DK / 8)) * 8;
-        uint4 uq = make_uint4(0, 0, 0, 0), uk = uq;
+      // every load of this thread is issued before the first store, so they are in flight together
+      constexpr int NQL = BCL * (DK / 8) / BCT;  // 16-byte pieces of Q (and of K) per thread
+      static_assert(NQL * BCT == BCL * (DK / 8) && BCL * (BCV / 8) == BCT, "chunk tiles map onto the threads");
+      uint4 uq[NQL], uk[NQL];
+#pragma unroll
+      for (int i = 0; i < NQL; ++i) {
+        const int e = tid + i * BCT, t = e / (DK / 8), c = (e % (DK / 8)) * 8;
+        uq[i] = uk[i] = make_uint4(0, 0, 0, 0);
         if (t < Lc) {
-          uq = *reinterpret_cast<const uint4*>(q + qoff + (size_t)(t0 + t) * a.DHQK + c);
-          uk = *reinterpret_cast<const uint4*>(k + qoff + (size_t)(t0 + t) * a.DHQK + c);
+          uq[i] = *reinterpret_cast<const uint4*>(q + qoff + (size_t)(t0 + t) * a.DHQK + c);
+          uk[i] = *reinterpret_cast<const uint4*>(k + qoff + (size_t)(t0 + t) * a.DHQK + c);
         }
-        *reinterpret_cast<uint4*>(Qb + t * LDK + c) = uq;
-        *reinterpret_cast<uint4*>(Kb + t * LDK + c) = uk;
       }
-      for (int e = tid; e < BCL * (BCV / 8); e += BCT) {
-        const int t = e / (BCV / 8), c = (e % (BCV / 8)) * 8;
+      {
+        const int t = tid / (BCV / 8), c = (tid % (BCV / 8)) * 8;
         uint4 uv = make_uint4(0, 0, 0, 0), uh = uv, uo = uv;
         if (t < Lc) {
           const size_t off = voff + (size_t)(t0 + t) * a.DHV + c;
           uv = *reinterpret_cast<const uint4*>(v + off);
           uh = *reinterpret_cast<const uint4*>(dh + off);
           if (og) uo = *reinterpret_cast<const uint4*>(og + off);
+        }
+#pragma unroll
+        for (int i = 0; i < NQL; ++i) {
+          const int e = tid + i * BCT, tt = e / (DK / 8), cc = (e % (DK / 8)) * 8;
+          *reinterpret_cast<uint4*>(Qb + tt * LDK + cc) = uq[i];
+          *reinterpret_cast<uint4*>(Kb + tt * LDK + cc) = uk[i];
         }
         *reinterpret_cast<uint4*>(Vb + t * LDV + c) = uv;
         const bf16_t* hb = reinterpret_cast<const bf16_t*>(&uh);
@@ -1066,7 +1093,8 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
       }
       return part;
     };
-    const int CW = (DK + NC - 1) / NC;  // key columns this CTA reduces (the last rank may have fewer)
+    // key columns this CTA reduces, in groups of four (the last rank may have fewer)
+    const int CW4 = (DK / 4 + NC - 1) / NC;
 
     // ------------------------------------------------------------------ phase 1 (forward)
     load_state(a.C0);
@@ -1135,8 +1163,12 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
       cl.sync();  // every CTA's P partials (and this CTA's dN) are written
       if (tid < BCL) {
         const int t = tid;
+        float part[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) part[i] = i < NC ? cl.map_shared_rank(tpp, i)[t] : 0.f;
         float P = 0.f;
-        for (int i = 0; i < NC; ++i) P += cl.map_shared_rank(tpp, i)[t];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) P += part[i];
         const float d = td[t], den = tden[t];
         const float dd = (!ret && t < Lc && fabsf(d) > expf(-tmt[t])) ? -P / den * copysignf(1.f, d) : 0.f;
         tdd[t] = dd;
@@ -1177,18 +1209,31 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
         }
       }
       cl.sync();  // every CTA's partial dq is written
-      for (int e = tid; e < BCL * CW; e += BCT) {
-        const int t = e / CW, c = rank * CW + e % CW;
+      for (int e = tid; e < BCL * CW4; e += BCT) {
+        const int t = e / CW4, c = rank * CW4 * 4 + (e % CW4) * 4;
         if (t >= Lc || c >= DK) continue;
-        float x = 0.f;
-        for (int i = 0; i < NC; ++i) x += cl.map_shared_rank(Rp, i)[t * DK + c];
+        const float4 x = sum_remote4(cl, Rp + t * DK + c, NC);
+        float4 y = x;
         const float dd = tdd[t];
         if (!ret && dd != 0.f) {
-          float wk = 0.f;
-          for (int s2 = 0; s2 <= t; ++s2) wk += Wm[t * LDW + s2] * __bfloat162float(Kb[s2 * LDK + c]);
-          x += dd * (eA[t] * nv[c] + wk);
+          float4 wk = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int s2 = 0; s2 <= t; ++s2) {
+            const float w = Wm[t * LDW + s2];
+            const uint2 kk = *reinterpret_cast<const uint2*>(Kb + s2 * LDK + c);
+            const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kk.x));
+            const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kk.y));
+            wk.x += w * k01.x;
+            wk.y += w * k01.y;
+            wk.z += w * k23.x;
+            wk.w += w * k23.y;
+          }
+          const float At = eA[t];
+          y.x += dd * (At * nv[c] + wk.x);
+          y.y += dd * (At * nv[c + 1] + wk.y);
+          y.z += dd * (At * nv[c + 2] + wk.z);
+          y.w += dd * (At * nv[c + 3] + wk.w);
         }
-        a.dq[qoff + (size_t)(t0 + t) * a.DHQK + c] = x;
+        *reinterpret_cast<float4*>(a.dq + qoff + (size_t)(t0 + t) * a.DHQK + c) = y;
       }
       {  // state to the chunk end: C' <- A_L C' + (V o w)^T K
         const float AL = eA[Lc - 1];
@@ -1301,19 +1346,33 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
         }
       }
       cl.sync();  // every CTA's partial dk is written
-      for (int e = tid; e < BCL * CW; e += BCT) {
-        const int s2 = e / CW, c = rank * CW + e % CW;
+      for (int e = tid; e < BCL * CW4; e += BCT) {
+        const int s2 = e / CW4, c = rank * CW4 * 4 + (e % CW4) * 4;
         if (s2 >= Lc || c >= DK) continue;
-        float x = 0.f;
-        for (int i = 0; i < NC; ++i) x += cl.map_shared_rank(Rp, i)[s2 * DK + c];
+        float4 x = sum_remote4(cl, Rp + s2 * DK + c, NC);
         if (!ret) {
-          float xn = wv[s2] * nv[c];
-          for (int tau = s2; tau < Lc; ++tau)
-            xn += Wm[tau * LDW + s2] * tdd[tau] * __bfloat162float(Qb[tau * LDK + c]);
-          x += xn;
-          atomicAdd(&tdn[s2], xn * __bfloat162float(Kb[s2 * LDK + c]));
+          const float w = wv[s2];
+          float4 xn = make_float4(w * nv[c], w * nv[c + 1], w * nv[c + 2], w * nv[c + 3]);
+          for (int tau = s2; tau < Lc; ++tau) {
+            const float f = Wm[tau * LDW + s2] * tdd[tau];
+            const uint2 qq = *reinterpret_cast<const uint2*>(Qb + tau * LDK + c);
+            const float2 q01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qq.x));
+            const float2 q23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qq.y));
+            xn.x += f * q01.x;
+            xn.y += f * q01.y;
+            xn.z += f * q23.x;
+            xn.w += f * q23.y;
+          }
+          x.x += xn.x;
+          x.y += xn.y;
+          x.z += xn.z;
+          x.w += xn.w;
+          const uint2 kk = *reinterpret_cast<const uint2*>(Kb + s2 * LDK + c);
+          const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kk.x));
+          const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kk.y));
+          atomicAdd(&tdn[s2], xn.x * k01.x + xn.y * k01.y + xn.z * k23.x + xn.w * k23.y);
         }
-        a.dk_out[qoff + (size_t)(t0 + s2) * a.DHQK + c] = x;
+        *reinterpret_cast<float4*>(a.dk_out + qoff + (size_t)(t0 + s2) * a.DHQK + c) = x;
       }
       {  // D <- A_L D + (dN o A)^T Q
         const float AL = eA[Lc - 1];

@@ -67,7 +67,18 @@ struct TcParams {
   // scalar normaliser with a learnable bias (NULL: the vector normaliser n . q): bias [NH];
   // then n0 / n_out hold one value per (batch, head) and dn one value per (slice, segment)
   const float* nbias;
+  // reversed sequence (token S-1 first): chunk c of the processing order is the original chunk
+  // nck_all-1-c (rows aligned to 64 from the start), its tokens taken from the last row back
+  int rev, nck_all;
 };
+
+// First original row of processing-order chunk c (global chunk index).
+__device__ __forceinline__ int chunk_row0(const TcParams& p, int c) {
+  return p.rev ? L * (p.nck_all - 1 - c) : L * c;
+}
+// Shared-memory row of position t (processing order) inside a chunk tile (the tile holds the
+// chunk's rows in original order).
+__device__ __forceinline__ int tile_row(const TcParams& p, int t) { return p.rev ? L - 1 - t : t; }
 
 // Lane / row mapping of an M-row accumulator: thread (warp w, lane l) owns row
 // 32w+l for M=128; row 16w+l for M=64 (lanes 16..31 hold no row).
@@ -222,14 +233,17 @@ __global__ void __launch_bounds__(256) tc_gate_prep_kernel(TcParams p, int BH) {
   const long long wid = (long long)blockIdx.x * 8 + warp;
   if (wid >= (long long)BH * p.ncp) return;
   const int bh = (int)(wid / p.ncp), c = (int)(wid % p.ncp);
-  const int t0 = c * L;
-  if (t0 >= p.S) return;
-  const int Lc = min(L, p.S - t0);
-  const size_t tok = (size_t)bh * p.S + t0;
+  if (c >= p.nck_all) return;
+  const int t0 = c * L;  // processing order
+  const int row0 = chunk_row0(p, c);
+  const size_t tok = (size_t)bh * p.S;
   const int ta = 2 * lane, tb = ta + 1;
+  // original rows of positions ta, tb (reversed: from the chunk's last row back; rows past the
+  // end are the identity step, first in the chunk when reversed)
+  const int ra = row0 + tile_row(p, ta), rb = row0 + tile_row(p, tb);
   float lfa = 0.f, lfb = 0.f, lia = -INFINITY, lib = -INFINITY;
-  if (ta < Lc) gate_vals(p, tok + ta, bh % p.NH, lfa, lia);
-  if (tb < Lc) gate_vals(p, tok + tb, bh % p.NH, lfb, lib);
+  if (ra < p.S) gate_vals(p, tok + ra, bh % p.NH, lfa, lia);
+  if (rb < p.S) gate_vals(p, tok + rb, bh % p.NH, lfb, lib);
   float isum = lfa + lfb;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -320,9 +334,10 @@ __global__ void __launch_bounds__(NTA, 1)
     uint8_t* kb = sm + st * (KB + VB);
     mbar_arrive_expect_tx(&full[st], KB + VB);
     for (int j = 0; j < DK / 64; ++j)
-      tma_load_3d(kb + j * 8192, &mapK, blk * p.dk + 64 * j, T0 + c * L, bh, &full[st]);
+      tma_load_3d(kb + j * 8192, &mapK, blk * p.dk + 64 * j, chunk_row0(p, g * p.seg_chunks + c), bh, &full[st]);
     for (int j = 0; j < DVT / 64; ++j)
-      tma_load_3d(kb + KB + j * 8192, &mapV, blk * p.dv + v0 + 64 * j, T0 + c * L, bh, &full[st]);
+      tma_load_3d(kb + KB + j * 8192, &mapV, blk * p.dv + v0 + 64 * j, chunk_row0(p, g * p.seg_chunks + c), bh,
+                  &full[st]);
   };
   // K and V are inputs: the first stages load while the previous kernel finishes
   int n_issued = 0;  // chunks whose loads thread 0 has issued
@@ -393,7 +408,10 @@ __global__ void __launch_bounds__(NTA, 1)
       }
       const float cf = coff[c];
       const float2 om2 = make_float2(expf(cf + gxn.x), expf(cf + gxn.y));
-      *reinterpret_cast<float2*>(omb + st * L + 2 * lane) = om2;
+      if (p.rev)  // positions 2 lane, 2 lane + 1 are tile rows 63 - 2 lane, 62 - 2 lane
+        *reinterpret_cast<float2*>(omb + st * L + L - 2 - 2 * lane) = make_float2(om2.y, om2.x);
+      else
+        *reinterpret_cast<float2*>(omb + st * L + 2 * lane) = om2;
       osum += om2.x + om2.y;
       if (c + 1 < nck) gxn = *reinterpret_cast<const float2*>(gxr + (size_t)(c + 1) * L);
       __syncwarp();
@@ -864,7 +882,7 @@ __global__ void __launch_bounds__(NTW, 1)
       if (!warp_wait(&bars.empty[b], ((c >> 1) & 1) ^ 1)) break;
       if (lane == 0) {
         uint8_t* base = sm + b * SM::STAGE;
-        const int t0 = T0 + c * L;
+        const int t0 = chunk_row0(p, g * p.seg_chunks + c);
         mbar_arrive_expect_tx(&bars.full[b], SM::STAGE);
         for (int j = 0; j < DK / 64; ++j) {
           tma_load_3d(base + j * 8192, &mapQ, blk * p.dk + 64 * j, t0, bh, &bars.full[b]);
@@ -899,7 +917,7 @@ __global__ void __launch_bounds__(NTW, 1)
       // tokens past the end have X = -inf: weight 0, column factor 0
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
-        const int t = h2 ? tb : ta;
+        const int t = tile_row(p, h2 ? tb : ta);  // the token's row in the chunk tiles
         const float bt = h2 ? bb : ba, mt = h2 ? mb : ma, xt = h2 ? xb : xa;
         if (guard) {
           const float sint = expf(bt + mc - mt);
@@ -1108,8 +1126,8 @@ __global__ void __launch_bounds__(NTW, 1)
     for (int c = 0; c < nck; ++c) {
       const int b = c & 1, gi = c % NGB;
       const GateBuf G = gbuf(gi);
-      const int t0 = T0 + c * L;
-      const int Lc = min(L, T1 - t0);
+      const int t0 = chunk_row0(p, g * p.seg_chunks + c);  // first original row of the chunk tile
+      const int Lc = min(L, p.S - t0);                        // rows of the tile inside the sequence
       const size_t tok0 = (size_t)bh * p.S + t0;
       // P = S o e^{al_t + be_s} (bf16, rows t, 128-byte swizzled) and its row sums, once the
       // chunk's gate values are written (the producer loads a stage before it writes them)
@@ -1153,20 +1171,26 @@ __global__ void __launch_bounds__(NTW, 1)
         if (lane == 0) mbar_arrive(&bars.s_empty);  // this warp's rows of S have left TMEM
         float rs_lo = 0.f, rs_hi = 0.f;
         uint32_t plo[8], phi[8];
-        const int lim_lo = r_lo < Lc ? r_lo : -1, lim_hi = r_hi < Lc ? r_hi : -1;  // last column kept
+        // columns kept: [lo, hi] (causal; forward: s <= t for rows inside the sequence, reversed:
+        // tile rows hold the positions backwards, so s >= t; the rows past the end there are the
+        // identity steps, whose columns carry factor 0 and whose h is not stored)
+        const int lo_lo = p.rev ? r_lo : 0, hi_lo = p.rev ? L - 1 : (r_lo < Lc ? r_lo : -1);
+        const int lo_hi = p.rev ? r_hi : 0, hi_hi = p.rev ? L - 1 : (r_hi < Lc ? r_hi : -1);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int s0 = 8 * j + cp;
           const float2 pa = __fmul2_rn(make_float2(r[2 * j], r[2 * j + 1]), make_float2(f_lo[2 * j], f_lo[2 * j + 1]));
           const float2 pb =
               __fmul2_rn(make_float2(r[16 + 2 * j], r[16 + 2 * j + 1]), make_float2(f_hi[2 * j], f_hi[2 * j + 1]));
-          const float a0 = s0 <= lim_lo ? pa.x : 0.f;
-          const float a1 = s0 + 1 <= lim_lo ? pa.y : 0.f;
-          const float b0 = s0 <= lim_hi ? pb.x : 0.f;
-          const float b1 = s0 + 1 <= lim_hi ? pb.y : 0.f;
+          const bool ka0 = s0 >= lo_lo && s0 <= hi_lo, ka1 = s0 + 1 >= lo_lo && s0 + 1 <= hi_lo;
+          const bool kb0 = s0 >= lo_hi && s0 <= hi_hi, kb1 = s0 + 1 >= lo_hi && s0 + 1 <= hi_hi;
+          const float a0 = ka0 ? pa.x : 0.f;
+          const float a1 = ka1 ? pa.y : 0.f;
+          const float b0 = kb0 ? pb.x : 0.f;
+          const float b1 = kb1 ? pb.y : 0.f;
           if (SN) {  // scalar normaliser: sums of the weights themselves (no q . k factor)
-            rs_lo += (s0 <= lim_lo ? f_lo[2 * j] : 0.f) + (s0 + 1 <= lim_lo ? f_lo[2 * j + 1] : 0.f);
-            rs_hi += (s0 <= lim_hi ? f_hi[2 * j] : 0.f) + (s0 + 1 <= lim_hi ? f_hi[2 * j + 1] : 0.f);
+            rs_lo += (ka0 ? f_lo[2 * j] : 0.f) + (ka1 ? f_lo[2 * j + 1] : 0.f);
+            rs_hi += (kb0 ? f_hi[2 * j] : 0.f) + (kb1 ? f_hi[2 * j + 1] : 0.f);
           } else {
             rs_lo += a0 + a1;
             rs_hi += b0 + b1;
@@ -1559,6 +1583,8 @@ cudaError_t launch_tc(const WalkArgs& a, const TcPlan& pl, void* ws, cudaStream_
   prm.sp = prm.ncp * L;
   prm.wait = a.wait_cycles > 0 ? a.wait_cycles : WAIT_DEFAULT;
   prm.nbias = a.retention ? nullptr : a.nbias;
+  prm.rev = a.reverse ? 1 : 0;
+  prm.nck_all = (a.S + L - 1) / L;
   float** planes[5] = {&prm.gb, &prm.gx, &prm.gxc, &prm.cg, &prm.cxm};
   for (int i = 0; i < 5; ++i) {
     *planes[i] = reinterpret_cast<float*>(w + off);

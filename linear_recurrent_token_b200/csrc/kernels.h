@@ -23,6 +23,7 @@ struct WalkArgs {
   void *h;
   float *C_out, *n_out, *m_out;
   long long wait_cycles;     // bound of each device-side wait (tensor-core path); 0 = default
+  int reverse;               // tensor-core path: the reversed sequence read in place (token S-1 first)
 };
 
 // The steps either side of retention (msr.cu): the rotation Theta of q and k by position

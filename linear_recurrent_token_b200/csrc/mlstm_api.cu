@@ -114,7 +114,9 @@ mlstm_status_t fwd_impl(const mlstm_fwd_params_t* p, const void* q, const void* 
                         const float* n0, const float* m0, void* h, float* C_out, float* n_out, float* m_out,
                         void* workspace, size_t workspace_bytes, cudaStream_t stream, cudaEvent_t ev0,
                         cudaEvent_t ev1, bool launch = true, const GnArgs* gn = nullptr,
-                        const float* nbias = nullptr) {
+                        const float* nbias = nullptr, bool reverse = false) {
+  // reverse: the reversed sequence read in place by the tensor-core kernels (the caller checks
+  // that the tensor-core path runs)
   // nbias != NULL: the scalar normaliser with this bias [NH] (tensor-core path only; n0 / n_out
   // one value per (batch, head)); the caller has validated it
   FwdShape s;
@@ -208,6 +210,7 @@ mlstm_status_t fwd_impl(const mlstm_fwd_params_t* p, const void* q, const void* 
   a.m_out = m_out;
   a.wait_cycles = p->wait_limit_cycles;
   a.nbias = nbias;
+  a.reverse = reverse ? 1 : 0;
   if (s.tc) {
     // snapshots: the walk writes n_out / m_out (and C_out across segments) while other
     // CTAs may still read n0 / m0 / C0, which the caller may have aliased to them
@@ -431,7 +434,8 @@ RevLayout rev_layout(const FwdShape& s) {
 size_t mlstm_fwd_chunkwise_reversed_workspace_size(const mlstm_fwd_params_t* p) {
   FwdShape s;
   if (check_fwd(p, &s) != MLSTM_OK) return 0;
-  return s.BH == 0 || s.S == 0 ? fwd_layout(s).total : rev_layout(s).total;
+  // the tensor-core kernels read the sequence backwards in place; the SIMT path runs on copies
+  return s.BH == 0 || s.S == 0 || s.tc ? fwd_layout(s).total : rev_layout(s).total;
 }
 
 mlstm_status_t mlstm_fwd_chunkwise_reversed(const mlstm_fwd_params_t* p, const void* q, const void* k,
@@ -446,6 +450,9 @@ mlstm_status_t mlstm_fwd_chunkwise_reversed(const mlstm_fwd_params_t* p, const v
   if (s.BH == 0 || s.S == 0)  // nothing to reverse
     return fwd_impl(p, q, k, v, igate, fgate, ogate, C0, n0, m0, h, C_out, n_out, m_out, workspace,
                     workspace_bytes, cs, nullptr, nullptr);
+  if (s.tc)  // the tensor-core kernels take the chunks and their rows backwards, no copies
+    return fwd_impl(p, q, k, v, igate, fgate, ogate, C0, n0, m0, h, C_out, n_out, m_out, workspace,
+                    workspace_bytes, cs, nullptr, nullptr, true, nullptr, nullptr, true);
   const RevLayout r = rev_layout(s);
   const size_t fwd_bytes = fwd_layout(s).total;
   // the caller's buffers, validated as for the forward (with the forward's part of the workspace)

@@ -587,3 +587,38 @@ def test_scalar_normaliser_prefill_tensor_core(case):
             "n": float(np.max(np.abs(host(gd["n"].t) - nr)) / max(np.max(np.abs(nr)), 1e-30)),
             "m": m_err(host(gd["m"].t), mr)}
     assert all(e <= tol for e in errs.values()), errs
+
+
+@pytest.mark.parametrize("retention,with_o,S", [(False, True, 1500), (True, False, 1000), (False, False, 2048)])
+def test_reversed_sequence_pass_several_segments(retention, with_o, S):
+    """The tensor-core reversed pass reads the chunks and their rows backwards in place; with
+    several sequence segments the segment summaries run backwards too.  Against the oracle on
+    the flipped sequence, outputs guard-banded."""
+    B, NH, DHQK, DHV = 1, 2, 128, 256
+    p = mlstm.fwd_params(B, NH, S, DHQK, DHV, 64, 1, torch.bfloat16, retention)
+    plan = mlstm.plan(p)
+    assert plan["tensor_core"] == 1 and plan["segments"] > 1, plan
+    assert mlstm.reversed_workspace_size(p) == mlstm.workspace_size(p)  # no copies on this path
+    w = inputs.Workload(3, "rev_seg", B, NH, S, DHQK, DHV, 64, 1, "bf16", retention, 1 / np.sqrt(DHQK))
+    inp = inputs.forward_inputs(w, seed=S)
+    rng = np.random.default_rng(S + 1)
+    C0 = (rng.standard_normal((B, NH, 1, DHV, DHQK)) * 0.2).astype(np.float32)
+    n0 = None if retention else (rng.standard_normal((B, NH, 1, DHQK)) * 0.2).astype(np.float32)
+    m0 = None if retention else rng.standard_normal((B, NH)).astype(np.float32)
+    og = inputs.round_to(rng.uniform(0, 1, (B, NH, S, DHV)), "bf16") if with_o else None
+    td = torch.bfloat16
+    gd = guarded_outputs(B, NH, S, DHQK, DHV, 1, td, retention)
+    ws = torch.empty(mlstm.reversed_workspace_size(p), dtype=torch.uint8, device="cuda")
+    h, C, n, m = mlstm.fwd_chunkwise(dev(inp["q"], td), dev(inp["k"], td), dev(inp["v"], td),
+                                     None if retention else dev(inp["igate"]), None if retention else dev(inp["fgate"]),
+                                     dev(og, td) if og is not None else None, dev(C0), dev(n0), dev(m0), chunk=64,
+                                     retention=retention, reverse=True, workspace=ws, h=gd["h"].t, C_out=gd["C"].t,
+                                     n_out=None if retention else gd["n"].t, m_out=None if retention else gd["m"].t)
+    assert mlstm.fwd_status(p, ws) == 0
+    assert_guards_intact(gd, "reversed")
+    flip = lambda x: None if x is None else np.ascontiguousarray(np.flip(x, axis=2))
+    ref = oracle_fwd({"q": flip(inp["q"]), "k": flip(inp["k"]), "v": flip(inp["v"]),
+                      "igate": flip(inp.get("igate")), "fgate": flip(inp.get("fgate"))},
+                     1, retention, flip(og), C0, n0, m0)
+    ref = (flip(ref[0]),) + tuple(ref[1:])
+    check((host(h), host(C), host(n), host(m)), ref, "bf16", retention, what=f"reversed S={S}")
