@@ -113,6 +113,10 @@ typedef struct {
   int ctas_main;        /* CTAs of the dominant (intra-chunk + state walk) kernel   */
   int kernels;          /* kernel launches one call enqueues                         */
   size_t workspace_bytes;
+  int seg0_chunks;      /* chunks of the first segment (tensor-core path; it walks while the
+                           others are summarised, so it may be longer)                */
+  int seg_chunks;       /* chunks of each later segment (the last may be shorter)    */
+  int summary_units;    /* segment summaries computed before the walk (0: one segment) */
 } mlstm_fwd_plan_t;
 
 /* Workspace bytes mlstm_fwd_chunkwise needs for these sizes (0 if none); returns

@@ -30,6 +30,8 @@
 // workspace error word, stops issuing work, frees its TMEM and returns.
 #include <cuda_bf16.h>
 
+#include <string.h>
+
 #include <utility>
 
 #include "common.cuh"
@@ -45,7 +47,6 @@ namespace {
 
 constexpr int L = 64;            // chunk length of the tensor-core path
 constexpr int NTA = 192;         // phase A threads per CTA (producer, MMA warp, 4 SIMT warps)
-constexpr int NSA = 4;           // phase A TMA stages
 constexpr long long WAIT_DEFAULT = 4000000000LL;  // bound of a wait unless the caller sets one (~2 s)
 
 struct TcParams {
@@ -70,7 +71,35 @@ struct TcParams {
   // reversed sequence (token S-1 first): chunk c of the processing order is the original chunk
   // nck_all-1-c (rows aligned to 64 from the start), its tokens taken from the last row back
   int rev, nck_all;
+  // segments: segment 0 has seg0_chunks chunks, the others seg_chunks (the last ends with the
+  // sequence); every segment but the last is summarised by phase A, segment 0 in ups units
+  // (halves when ups = 2), the others in one: NU units in all, by CTAs of dv / n_tiles_a value
+  // rows each
+  int seg0_chunks, ups, NU, n_tiles_a;
 };
+
+// Processing-order chunks [s0, s1) of segment g.
+__device__ __forceinline__ void seg_range(const TcParams& p, int g, int& s0, int& s1) {
+  s0 = g == 0 ? 0 : p.seg0_chunks + (g - 1) * p.seg_chunks;
+  s1 = g == p.G - 1 ? p.nck_all : s0 + (g == 0 ? p.seg0_chunks : p.seg_chunks);
+  s1 = min(s1, p.nck_all);
+  s0 = min(s0, s1);
+}
+// Processing-order chunks [u0, u1) of summary unit j: units 0 .. ups-1 are the parts of
+// segment 0, unit ups - 1 + g is segment g >= 1.
+__device__ __forceinline__ void unit_range(const TcParams& p, int j, int& u0, int& u1) {
+  int s0, s1;
+  if (j < p.ups) {
+    seg_range(p, 0, s0, s1);
+    const int n = s1 - s0;
+    u0 = s0 + j * n / p.ups;
+    u1 = s0 + (j + 1) * n / p.ups;
+  } else {
+    seg_range(p, j - p.ups + 1, u0, u1);
+  }
+}
+// Summary units before segment g.
+__device__ __forceinline__ int units_before(const TcParams& p, int g) { return g == 0 ? 0 : p.ups + g - 1; }
 
 // First original row of processing-order chunk c (global chunk index).
 __device__ __forceinline__ int chunk_row0(const TcParams& p, int c) {
@@ -79,6 +108,15 @@ __device__ __forceinline__ int chunk_row0(const TcParams& p, int c) {
 // Shared-memory row of position t (processing order) inside a chunk tile (the tile holds the
 // chunk's rows in original order).
 __device__ __forceinline__ int tile_row(const TcParams& p, int t) { return p.rev ? L - 1 - t : t; }
+// The same with the direction known at compile time (the walk's per-chunk code).
+template <bool REV>
+__device__ __forceinline__ int chunk_row0_c(const TcParams& p, int c) {
+  return REV ? L * (p.nck_all - 1 - c) : L * c;
+}
+template <bool REV>
+__device__ __forceinline__ int tile_row_c(int t) {
+  return REV ? L - 1 - t : t;
+}
 
 // Lane / row mapping of an M-row accumulator: thread (warp w, lane l) owns row
 // 32w+l for M=128; row 16w+l for M=64 (lanes 16..31 hold no row).
@@ -274,42 +312,54 @@ __global__ void __launch_bounds__(256) tc_gate_prep_kernel(TcParams p, int BH) {
 }
 
 // ===================================================================== phase A
-// CTA = (value tile, segment < G-1, slice); 192 threads in three roles, four TMA stages of
-// (K, V) with per-stage barriers:
+// CTA = (value rows [DVA r, DVA r + DVA), summary unit j, slice): the zero-start contribution of
+// the unit's chunks (a segment or half a segment, see seg_range / unit_range) to those rows of
+// the state.  192 threads in three roles, NS TMA stages of (K, V) with per-stage barriers:
 //   warp 0     producer: TMA loads of stage c % NS once the MMAs of chunk c - NS are done,
 //              then the chunk's weights omega_s (second arrival on the stage's full barrier)
-//   warp 1     MMA warp: D[dv, dk] += (V o omega)^T K once the SIMT group has scaled V
-//   warps 2-5  SIMT group: V rows scaled in place by omega, dn partials (this tile's share of
-//              the key columns); at the end the TMEM accumulator and dn go to global memory
+//   warp 1     MMA warp: D[rows, dk] += (V o omega)^T K once the SIMT group has scaled V; with
+//              DVA = 256 two M = 128 accumulators fill the tensor memory and share each K tile
+//   warps 2-5  SIMT group: V rows scaled in place by omega, dn partials (this CTA's share of
+//              the key columns); at the end the TMEM accumulators and dn go to global memory
 // The roles only meet at mbarriers, so the SIMT work of later stages overlaps the MMAs.
-template <int DK, int DVT>
+template <int DK, int DVA>
+struct SegCfg {
+  static constexpr int NACC = DVA == 256 ? 2 : 1;       // accumulators
+  static constexpr int MA = DVA == 256 ? 128 : DVA;     // MMA M
+  static constexpr int KB = DK * 128, VB = DVA * 128;   // bytes of one K / V chunk tile
+  static constexpr int STAGE = KB + VB;
+  static constexpr int NS = STAGE * 4 <= 200 * 1024 ? 4 : 3;  // TMA stages
+  static constexpr int BYTES_FIXED = NS * STAGE + (128 * 8 + NS * L) * 4 + 1024;
+};
+
+template <int DK, int DVA>
 __global__ void __launch_bounds__(NTA, 1)
     tc_segment_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV, TcParams p) {
-  constexpr int KB = DK * 128;   // bytes of one K chunk tile (DK/64 boxes of 8 KiB)
-  constexpr int VB = DVT * 128;  // bytes of one V chunk tile
-  constexpr int NS = NSA;        // TMA stages
+  using CF = SegCfg<DK, DVA>;
+  constexpr int KB = CF::KB, VB = CF::VB, NS = CF::NS, NACC = CF::NACC, MA = CF::MA;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // stage i: K at sm + i*(KB+VB), V right after it
   float* dnp = reinterpret_cast<float*>(sm + NS * (KB + VB));  // [128 * 8] partial sums of dn
   float* omb = dnp + 128 * 8;                                   // [NS][L] weights of the stage's chunk
-  float* coff = omb + NS * L;                                   // [seg_chunks]
+  float* coff = omb + NS * L;                                   // [unit chunks]
   __shared__ uint64_t full[NS], scaled[NS], mma_done[NS], all_done, drain;
   __shared__ uint32_t tmem_base;
   __shared__ float red[NTA / 32];
   __shared__ volatile int abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tile = blockIdx.x, g = blockIdx.y, slice = blockIdx.z;
+  const int tile = blockIdx.x, j = blockIdx.y, slice = blockIdx.z;
   const int blk = slice % p.nb, bh = slice / p.nb;
-  const int seg_len = p.seg_chunks * L;
-  const int T0 = g * seg_len;  // phase A covers full segments only
-  const int v0 = tile * DVT;
-  // this tile accumulates dn over key columns [dn0, min(DK, dn0 + dnw)), dnw a multiple of 8
-  const int dnw = ((DK + p.n_tiles - 1) / p.n_tiles + 7) / 8 * 8;
+  int u0, u1;
+  unit_range(p, j, u0, u1);  // processing-order chunks of this unit (all full: it precedes the last segment)
+  const int nck = u1 - u0;
+  const int T0 = u0 * L;
+  const int v0 = tile * DVA;
+  // this CTA accumulates dn over key columns [dn0, min(DK, dn0 + dnw)), dnw a multiple of 8
+  const int dnw = ((DK + p.n_tiles_a - 1) / p.n_tiles_a + 7) / 8 * 8;
   const int dn0 = tile * dnw;
   const bool do_dn = !p.retention && !p.nbias && dn0 < DK;
-  const int nck = p.seg_chunks;
 
   if (tid == 0) {
     for (int i = 0; i < NS; ++i) {
@@ -324,7 +374,7 @@ __global__ void __launch_bounds__(NTA, 1)
     prefetch_tensormap(&mapK);
     prefetch_tensormap(&mapV);
   }
-  if (warp == 0) tmem_alloc(&tmem_base, DK);
+  if (warp == 0) tmem_alloc(&tmem_base, NACC * DK);
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = tmem_base;
@@ -332,12 +382,12 @@ __global__ void __launch_bounds__(NTA, 1)
   auto issue = [&](int c) {  // one lane
     const int st = c % NS;
     uint8_t* kb = sm + st * (KB + VB);
+    const int row0 = chunk_row0(p, u0 + c);
     mbar_arrive_expect_tx(&full[st], KB + VB);
-    for (int j = 0; j < DK / 64; ++j)
-      tma_load_3d(kb + j * 8192, &mapK, blk * p.dk + 64 * j, chunk_row0(p, g * p.seg_chunks + c), bh, &full[st]);
-    for (int j = 0; j < DVT / 64; ++j)
-      tma_load_3d(kb + KB + j * 8192, &mapV, blk * p.dv + v0 + 64 * j, chunk_row0(p, g * p.seg_chunks + c), bh,
-                  &full[st]);
+    for (int jj = 0; jj < DK / 64; ++jj)
+      tma_load_3d(kb + jj * 8192, &mapK, blk * p.dk + 64 * jj, row0, bh, &full[st]);
+    for (int jj = 0; jj < DVA / 64; ++jj)
+      tma_load_3d(kb + KB + jj * 8192, &mapV, blk * p.dv + v0 + 64 * jj, row0, bh, &full[st]);
   };
   // K and V are inputs: the first stages load while the previous kernel finishes
   int n_issued = 0;  // chunks whose loads thread 0 has issued
@@ -347,40 +397,50 @@ __global__ void __launch_bounds__(NTA, 1)
       n_issued = c + 1;
     }
 
-  grid_dep_launch();
   grid_dep_wait();  // the gate planes come from the preparation kernel
+  grid_dep_launch();  // after the wait: a dependent grid that starts now finds the gate planes complete
   // ---- gates: Gtot = sum of the chunk totals, and for token s of chunk c the log weight
   // Gtot - G_s + itilde_s = Gtot - Gpre_c + X_s (Gpre_c: totals of the earlier chunks of the
-  // segment); M = its maximum = max_c (Gtot - Gpre_c + max X of chunk c); omega_s = e^{. - M}
+  // unit); M = its maximum = max_c (Gtot - Gpre_c + max X of chunk c); omega_s = e^{. - M}
   {
-    const size_t crow = (size_t)bh * p.ncp + (size_t)g * p.seg_chunks;
-    const float gcv = tid < nck ? p.cg[crow + tid] : 0.f;
-    const float xmv = tid < nck ? p.cxm[crow + tid] : -INFINITY;
-    float inc = gcv;
-    for (int o = 1; o < 32; o <<= 1) {
-      const float u = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += u;
+    const size_t crow = (size_t)bh * p.ncp + (size_t)u0;
+    float total = 0.f, Mg = -INFINITY;
+    // chunk totals in passes of NTA (a unit has at most a few hundred chunks)
+    for (int base = 0; base < nck; base += NTA) {
+      const int c = base + tid;
+      const float gcv = c < nck ? p.cg[crow + c] : 0.f;
+      const float xmv = c < nck ? p.cxm[crow + c] : -INFINITY;
+      float inc = gcv;
+      for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += u;
+      }
+      __syncthreads();
+      if (lane == 31) red[warp] = inc;
+      __syncthreads();
+      float wexcl = 0.f, ptotal = 0.f;
+      for (int w = 0; w < NTA / 32; ++w) {
+        if (w < warp) wexcl += red[w];
+        ptotal += red[w];
+      }
+      // gpre relative to the unit start: earlier passes' total plus this pass's exclusive sum
+      const float gpre = total + wexcl + inc - gcv;
+      if (c < nck) coff[c] = gpre;  // provisional: Gpre_c; turned into Gtot - Gpre_c - M below
+      float lm = c < nck ? xmv - gpre : -INFINITY;  // max_c (X max of chunk c - Gpre_c)
+      for (int o = 16; o >= 1; o >>= 1) lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, o));
+      __syncthreads();
+      if (lane == 0) red[warp] = lm;
+      __syncthreads();
+      for (int w = 0; w < NTA / 32; ++w) Mg = fmaxf(Mg, red[w]);
+      total += ptotal;
     }
-    if (lane == 31) red[warp] = inc;
-    __syncthreads();
-    float wexcl = 0.f, total = 0.f;
-    for (int w = 0; w < NTA / 32; ++w) {
-      if (w < warp) wexcl += red[w];
-      total += red[w];
-    }
-    const float gpre = wexcl + inc - gcv;
-    float lmax = tid < nck ? total - gpre + xmv : -INFINITY;
-    for (int o = 16; o >= 1; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
-    __syncthreads();
-    if (lane == 0) red[warp] = lmax;
-    __syncthreads();
-    float Mg = -INFINITY;
-    for (int w = 0; w < NTA / 32; ++w) Mg = fmaxf(Mg, red[w]);
+    Mg += total;  // M = Gtot + max_c (X max - Gpre_c)
     if (p.retention) Mg = 0.f;
-    if (tid < nck) coff[tid] = total - gpre - Mg;
+    __syncthreads();
+    for (int c = tid; c < nck; c += NTA) coff[c] = total - coff[c] - Mg;
     if (tile == 0 && blk == 0 && tid == 0) {
-      p.segA[(size_t)bh * (p.G - 1) + g] = total;
-      p.segB[(size_t)bh * (p.G - 1) + g] = Mg;
+      p.segA[(size_t)bh * p.NU + j] = total;
+      p.segB[(size_t)bh * p.NU + j] = Mg;
     }
     __syncthreads();
   }
@@ -395,7 +455,7 @@ __global__ void __launch_bounds__(NTA, 1)
     // prefetched into registers)
     const float* gxr = p.gx + (size_t)bh * p.sp + T0 + 2 * lane;
     float2 gxn = *reinterpret_cast<const float2*>(gxr);
-    float osum = 0.f;  // scalar normaliser: this lane's share of the segment's sum of weights
+    float osum = 0.f;  // scalar normaliser: this lane's share of the unit's sum of weights
     for (int c = 0; c < nck; ++c) {
       const int st = c % NS;
       if (c >= NS) {
@@ -417,25 +477,28 @@ __global__ void __launch_bounds__(NTA, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[st]);
     }
-    if (p.nbias && !p.retention) {  // dn of the scalar normaliser: sum over the segment of omega_s
+    if (p.nbias && !p.retention) {  // dn of the scalar normaliser: sum over the unit of omega_s
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) osum += __shfl_xor_sync(0xffffffffu, osum, o);
-      if (lane == 0 && tile == 0 && !abort_flag) p.dn[((size_t)slice * (p.G - 1) + g) * p.dk] = osum;
+      if (lane == 0 && tile == 0 && !abort_flag) p.dn[((size_t)slice * p.NU + j) * p.dk] = osum;
     }
   } else if (warp == 1) {
     // =============================================================== MMA warp
-    const uint32_t idesc = idesc_bf16(DVT, DK, 1, 1);
+    const uint32_t idesc = idesc_bf16(MA, DK, 1, 1);
     for (int c = 0; c < nck; ++c) {
       const int st = c % NS;
       uint8_t* Kst = sm + st * (KB + VB);
-      const uint64_t ad = smem_desc_sw128(smem_u32(Kst + KB), 8192, 1024);
       const uint64_t bd = smem_desc_sw128(smem_u32(Kst), 8192, 1024);
+      const uint64_t ad0 = smem_desc_sw128(smem_u32(Kst + KB), 8192, 1024);
       if (!warp_wait(&scaled[st], (c / NS) & 1)) break;
       tc_fence_after();
       if (elect_one()) {
 #pragma unroll
         for (int ks = 0; ks < L / 16; ++ks)
-          mma_bf16_ss(tm, ad + (uint64_t)(ks * 128), bd + (uint64_t)(ks * 128), idesc, (c > 0 || ks > 0) ? 1u : 0u);
+#pragma unroll
+          for (int a = 0; a < NACC; ++a)  // accumulator a: value rows 128 a .. (two 64-row blocks of V on)
+            mma_bf16_ss(tm + a * DK, ad0 + (uint64_t)(ks * 128) + (uint64_t)((a * 16384) >> 4),
+                        bd + (uint64_t)(ks * 128), idesc, (c > 0 || ks > 0) ? 1u : 0u);
         mma_commit(&mma_done[st]);
         if (c == nck - 1) mma_commit(&all_done);
       }
@@ -444,13 +507,13 @@ __global__ void __launch_bounds__(NTA, 1)
   } else {
     // =============================================================== SIMT group
     const int gt = tid - 64;  // 0..127
-    // dn partials: thread -> (column group of 8 inside this tile's columns, row group)
+    // dn partials: thread -> (column group of 8 inside this CTA's columns, row group)
     const int ncg = dnw / 8 < 128 ? dnw / 8 : 128, nrg = 128 / ncg, rows_per = (L + nrg - 1) / nrg;
     const int cg = gt % ncg, rg = gt / ncg;
     const int dcol = dn0 + 8 * cg;  // first of this thread's 8 columns
     float2 dacc[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) dacc[j] = make_float2(0.f, 0.f);
+    for (int jj = 0; jj < 4; ++jj) dacc[jj] = make_float2(0.f, 0.f);
     for (int c = 0; c < nck; ++c) {
       const int st = c % NS;
       uint8_t* Kst = sm + st * (KB + VB);
@@ -460,22 +523,26 @@ __global__ void __launch_bounds__(NTA, 1)
       if (!__all_sync(0xffffffffu, mbar_test_wait(&full[st], (c / NS) & 1)))
         warp_wait_slow(&full[st], (c / NS) & 1, &abort_flag, p.wait);
       {
-        // V rows scaled in place by omega (loads batched ahead of the stores)
-        constexpr int NV = L * (DVT / 8) / 128;
+        // V rows scaled in place by omega (loads batched ahead of the stores, in passes of 8)
+        constexpr int NV = L * (DVA / 8) / 128;
+        constexpr int NB = NV < 8 ? NV : 8;
         const uint32_t v_u = smem_u32(Kst + KB);
-        uint4 u[NV];
-        float wr[NV];
-        int offs[NV];
 #pragma unroll
-        for (int k = 0; k < NV; ++k) {
-          const int i = k * 128 + gt;
-          const int row = i / (DVT / 8), ch = i % (DVT / 8);
-          offs[k] = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
-          u[k] = ld_shared_v4(v_u + offs[k]);
-          wr[k] = om[row];
+        for (int k0 = 0; k0 < NV; k0 += NB) {
+          uint4 u[NB];
+          float wr[NB];
+          int offs[NB];
+#pragma unroll
+          for (int k = 0; k < NB; ++k) {
+            const int i = (k0 + k) * 128 + gt;
+            const int row = i / (DVA / 8), ch = i % (DVA / 8);
+            offs[k] = (ch >> 3) * 8192 + row * 128 + ((ch & 7) << 4);
+            u[k] = ld_shared_v4(v_u + offs[k]);
+            wr[k] = om[row];
+          }
+#pragma unroll
+          for (int k = 0; k < NB; ++k) st_shared_v4u(v_u + offs[k], scale_bf16x8(u[k], wr[k]));
         }
-#pragma unroll
-        for (int k = 0; k < NV; ++k) st_shared_v4u(v_u + offs[k], scale_bf16x8(u[k], wr[k]));
       }
       if (do_dn && rg < nrg && dcol < DK) {
         const uint8_t* kt = Kst + (dcol >> 6) * 8192;
@@ -487,28 +554,31 @@ __global__ void __launch_bounds__(NTA, 1)
           const float w = om[s];
           const float2 w2 = make_float2(w, w);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) dacc[j] = __ffma2_rn(__bfloat1622float2(b2[j]), w2, dacc[j]);
+          for (int jj = 0; jj < 4; ++jj) dacc[jj] = __ffma2_rn(__bfloat1622float2(b2[jj]), w2, dacc[jj]);
         }
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&scaled[st]);
     }
-    // ---- epilogue: the accumulator (warp w reads TMEM lane quarter w % 4) and dn
+    // ---- epilogue: the accumulators (warp w reads TMEM lane quarter w % 4) and dn
     if (!__all_sync(0xffffffffu, mbar_test_wait(&all_done, 0))) warp_wait_slow(&all_done, 0, &abort_flag, p.wait);
     tc_fence_after();
     const int quarter = warp & 3;
-    const int row = acc_row<DVT>(quarter, lane);
-    float* dst = row >= 0 ? p.dC + (((size_t)slice * (p.G - 1) + g) * p.dv + v0 + row) * p.dk : nullptr;
+    const int row = acc_row<MA>(quarter, lane);
 #pragma unroll 1
-    for (int c0 = 0; c0 < DK; c0 += 32) {
-      float r[32];
-      tmem_ld32(tm + ((uint32_t)(32 * quarter) << 16) + c0, r);
-      tmem_wait_ld();
-      if (dst && !abort_flag)
+    for (int a = 0; a < NACC; ++a) {
+      float* dst = row >= 0 ? p.dC + (((size_t)slice * p.NU + j) * p.dv + v0 + a * MA + row) * p.dk : nullptr;
+#pragma unroll 1
+      for (int c0 = 0; c0 < DK; c0 += 32) {
+        float r[32];
+        tmem_ld32(tm + ((uint32_t)(32 * quarter) << 16) + a * DK + c0, r);
+        tmem_wait_ld();
+        if (dst && !abort_flag)
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          *reinterpret_cast<float4*>(dst + c0 + j) = make_float4(r[j], r[j + 1], r[j + 2], r[j + 3]);
+          for (int jj = 0; jj < 32; jj += 4)
+            *reinterpret_cast<float4*>(dst + c0 + jj) = make_float4(r[jj], r[jj + 1], r[jj + 2], r[jj + 3]);
+      }
     }
     if (do_dn) {
       *reinterpret_cast<float4*>(dnp + gt * 8) = make_float4(dacc[0].x, dacc[0].y, dacc[1].x, dacc[1].y);
@@ -517,7 +587,7 @@ __global__ void __launch_bounds__(NTA, 1)
       for (int col = gt; col < ncg * 8 && dn0 + col < DK; col += 128) {
         float x = 0.f;
         for (int r = 0; r < nrg; ++r) x += dnp[(r * ncg + col / 8) * 8 + (col & 7)];
-        if (!abort_flag) p.dn[((size_t)slice * (p.G - 1) + g) * p.dk + dn0 + col] = x;
+        if (!abort_flag) p.dn[((size_t)slice * p.NU + j) * p.dk + dn0 + col] = x;
       }
     }
   }
@@ -541,7 +611,7 @@ __global__ void __launch_bounds__(NTA, 1)
     if (abort_flag) atomicOr(p.err, 1u);
   }
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tm, DK);
+  if (warp == 0) tmem_dealloc(tm, NACC * DK);
 }
 
 // ===================================================================== phase C
@@ -615,12 +685,14 @@ struct WalkBars {
   uint64_t full[2], empty[2], s_full[2], gfull[NGB], gempty[NGB], q_ready[NGB];
   uint64_t cb_ready, vw_full, upd_done, ro_done, h_empty, s_empty, p_full, mm_done;
   uint64_t drain;  // both MMA warps' last commits, before TMEM is freed
+  uint64_t comp;   // the summary tiles of the start state (prologue)
 };
 
-template <int DK, int DVT, bool SN>
+template <int DK, int DVT, bool SN, bool REV>
 __global__ void __launch_bounds__(NTW, 1)
     tc_walk_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
-                   const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapH, TcParams p) {
+                   const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapH,
+                   const __grid_constant__ CUtensorMap mapS, TcParams p) {
   using SM = WalkSmem<DK, DVT>;
   // TMEM columns: C fp32 [DK], bf16 snapshot of C as MMA operand [DK/2], S [64], H [64]
   constexpr uint32_t TM_C = 0, TM_CB = DK, TM_S = DK + DK / 2, TM_H = TM_S + 64;
@@ -646,12 +718,14 @@ __global__ void __launch_bounds__(NTW, 1)
   __shared__ volatile int group_flag[2];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tile = blockIdx.x, g = blockIdx.y, slice = blockIdx.z;
+  // segment slowest in the grid: the CTAs of segment 0, which need no summary, are dispatched first
+  const int tile = blockIdx.x, slice = blockIdx.y, g = blockIdx.z;
   const int blk = slice % p.nb, bh = slice / p.nb;
   const int v0 = tile * DVT;
-  const int seg_len = p.seg_chunks * L;
-  const int T0 = g * seg_len, T1 = min(p.S, T0 + seg_len);
-  const int nck = (T1 - T0 + L - 1) / L;
+  int s0, s1;
+  seg_range(p, g, s0, s1);  // this segment's processing-order chunks
+  const int T0 = s0 * L;
+  const int nck = s1 - s0;
   const bool ret = p.retention != 0;
   const bool last_seg = g == p.G - 1;
   const uint32_t sm_u = smem_u32(sm);
@@ -676,6 +750,7 @@ __global__ void __launch_bounds__(NTW, 1)
     mbar_init(&bars.p_full, 4);
     mbar_init(&bars.mm_done, 1);
     mbar_init(&bars.drain, 2);
+    mbar_init(&bars.comp, 1);
     abort_flag = 0;
     group_flag[0] = group_flag[1] = 0;
     fence_mbar_init();
@@ -683,83 +758,125 @@ __global__ void __launch_bounds__(NTW, 1)
     prefetch_tensormap(&mapK);
     prefetch_tensormap(&mapV);
     prefetch_tensormap(&mapH);
+    if (p.NU > 0) prefetch_tensormap(&mapS);
   }
   if (warp == 0) tmem_alloc(&tmem_base, TM_COLS);
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = tmem_base;
 
-  grid_dep_wait();  // summaries and gate planes come from the kernels before this one
+  // Summaries and gate planes come from the kernels before this one.  Segment 0 needs no summary:
+  // when segment summaries run (the previous kernel, which signals its dependents only after its
+  // own wait for the gate preparation), its CTAs start walking while the summaries are computed.
+  if (g > 0 || p.NU == 0) grid_dep_wait();
   // ---- start state of the segment (see the file header); warps 3-10 fill TMEM and n.
   // It is stabilised at m_start, so lam starts at m_start.
   float m_start = ret ? 0.f : (p.m0 ? p.m0[bh] : 0.f);
   const float m_init = m_start;
   float gsum = 0.f;
-  for (int j = 0; j < g; ++j) {
-    const float A = p.segA[(size_t)bh * (p.G - 1) + j], Bm = p.segB[(size_t)bh * (p.G - 1) + j];
+  const int nun = units_before(p, g);  // summary units before this segment
+  for (int j = 0; j < nun; ++j) {
+    const float A = p.segA[(size_t)bh * p.NU + j], Bm = p.segB[(size_t)bh * p.NU + j];
     if (!ret) m_start = fmaxf(A + m_start, Bm);
     gsum += A;
   }
+  const float wc0 = expf(gsum + m_init - m_start);
+  // Weights of the earlier units' summaries at m_start, once (the gate buffers are free until
+  // the producer's first chunk).
+  float* pw = gmem;  // [nun]
+  if (tid == 0) {
+    float after = gsum;
+    for (int j = 0; j < nun; ++j) {
+      after -= p.segA[(size_t)bh * p.NU + j];
+      pw[j] = expf(p.segB[(size_t)bh * p.NU + j] + after - m_start);
+    }
+  }
+  __syncthreads();
+  // The start state of this CTA's rows, wc0 C0 + sum_j pw_j dC_j, into TMEM: wc0 C0 (or zeros)
+  // first, then each earlier unit's tile rows land in the stage area (free until the producer's
+  // first load) through TMA, 32-column boxes with 128-byte swizzle so that the 32 lanes of a warp
+  // read 32 rows at one column without bank conflicts, and the warps owning the TMEM lanes add
+  // them in.  The loads of a unit are all in flight at once.
   if (warp >= 3 && warp < 11) {
     const int quarter = warp & 3, half = (warp - 3) >> 2;
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     const int row = acc_row<DVT>(quarter, lane);
-    const float wc0 = expf(gsum + m_init - m_start);
     for (int c0 = half * (DK / 2); c0 < (half + 1) * (DK / 2); c0 += 16) {
       float r[16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) r[j] = 0.f;
-      if (row >= 0) {
-        if (p.C0) {
-          const float4* src = reinterpret_cast<const float4*>(p.C0 + ((size_t)slice * p.dv + v0 + row) * p.dk + c0);
+      for (int jj = 0; jj < 16; ++jj) r[jj] = 0.f;
+      if (row >= 0 && p.C0) {
+        const float4* src = reinterpret_cast<const float4*>(p.C0 + ((size_t)slice * p.dv + v0 + row) * p.dk + c0);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float4 x = src[j];
-            r[4 * j] = wc0 * x.x;
-            r[4 * j + 1] = wc0 * x.y;
-            r[4 * j + 2] = wc0 * x.z;
-            r[4 * j + 3] = wc0 * x.w;
-          }
-        }
-        float after = gsum;
-        for (int jg = 0; jg < g; ++jg) {
-          after -= p.segA[(size_t)bh * (p.G - 1) + jg];
-          const float wj = expf(p.segB[(size_t)bh * (p.G - 1) + jg] + after - m_start);
-          const float4* src = reinterpret_cast<const float4*>(
-              p.dC + (((size_t)slice * (p.G - 1) + jg) * p.dv + v0 + row) * p.dk + c0);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float4 x = src[j];
-            r[4 * j] += wj * x.x;
-            r[4 * j + 1] += wj * x.y;
-            r[4 * j + 2] += wj * x.z;
-            r[4 * j + 3] += wj * x.w;
-          }
+        for (int jj = 0; jj < 4; ++jj) {
+          const float4 x = src[jj];
+          r[4 * jj] = wc0 * x.x;
+          r[4 * jj + 1] = wc0 * x.y;
+          r[4 * jj + 2] = wc0 * x.z;
+          r[4 * jj + 3] = wc0 * x.w;
         }
       }
       tmem_st16(tm + lane_off + TM_C + c0, r);
     }
     tmem_wait_st();
-    if (SN) {
-      if (tid == 96) {  // scalar normaliser: one value per (batch, head), in nvec[0]
-        float x = p.n0 ? wc0 * p.n0[bh] : 0.f;
-        float after = gsum;
-        for (int jg = 0; jg < g; ++jg) {
-          after -= p.segA[(size_t)bh * (p.G - 1) + jg];
-          x += expf(p.segB[(size_t)bh * (p.G - 1) + jg] + after - m_start) *
-               p.dn[((size_t)slice * (p.G - 1) + jg) * p.dk];
+  }
+  static_assert(DVT * DK * 4 <= 2 * SM::STAGE, "a summary tile fits the stage area");
+  for (int j = 0; j < nun; ++j) {
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&bars.comp, DVT * DK * 4);
+      const int r0 = ((int)slice * p.NU + j) * p.dv + v0;
+      for (int rb = 0; rb < (DVT + 63) / 64; ++rb)
+        for (int cb = 0; cb < DK / 32; ++cb)
+          tma_load_2d(sm + (rb * (DK / 32) + cb) * 8192, &mapS, 32 * cb, r0 + 64 * rb, &bars.comp);
+    }
+    if (!mbar_wait(&bars.comp, j & 1, p.wait)) {  // give up on the data, but let the copies land
+      abort_flag = 1;
+      mbar_wait(&bars.comp, j & 1, WAIT_DEFAULT);
+    }
+    if (warp >= 3 && warp < 11) {
+      const int quarter = warp & 3, half = (warp - 3) >> 2;
+      const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+      const int row = acc_row<DVT>(quarter, lane);
+      const int rr = row & 63;
+      const float w = pw[j];
+      tc_fence_after();
+      for (int c0 = half * (DK / 2); c0 < (half + 1) * (DK / 2); c0 += 32) {
+        float r[32];
+        tmem_ld32(tm + lane_off + TM_C + c0, r);
+        tmem_wait_ld();
+        if (row >= 0) {
+          const uint8_t* box = sm + ((row >> 6) * (DK / 32) + (c0 >> 5)) * 8192 + rr * 128;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float4 x = *reinterpret_cast<const float4*>(box + ((k ^ (rr & 7)) << 4));
+            r[4 * k] += w * x.x;
+            r[4 * k + 1] += w * x.y;
+            r[4 * k + 2] += w * x.z;
+            r[4 * k + 3] += w * x.w;
+          }
         }
+        tmem_st16(tm + lane_off + TM_C + c0, *reinterpret_cast<float(*)[16]>(r));
+        tmem_st16(tm + lane_off + TM_C + c0 + 16, *reinterpret_cast<float(*)[16]>(r + 16));
+      }
+      tmem_wait_st();
+      tc_fence_before();
+    }
+    fence_proxy_async_smem();  // the reads of the stage area come before the next TMA writes
+    __syncthreads();           // the stage area takes the next unit
+  }
+  // n (vector, or the scalar normaliser's one value per head) the same way, by the other warps
+  if (warp >= 11 || warp < 3) {
+    const int nt2 = warp >= 11 ? tid - 352 : 128 + tid;  // 0..223
+    if (SN) {
+      if (nt2 == 0) {
+        float x = p.n0 ? wc0 * p.n0[bh] : 0.f;
+        for (int jg = 0; jg < nun; ++jg) x += pw[jg] * p.dn[((size_t)slice * p.NU + jg) * p.dk];
         nvec[0] = x;
       }
     } else if (!ret)
-      for (int col = tid - 96; col < DK; col += 256) {
+      for (int col = nt2; col < DK; col += 224) {
         float x = p.n0 ? wc0 * p.n0[(size_t)slice * p.dk + col] : 0.f;
-        float after = gsum;
-        for (int jg = 0; jg < g; ++jg) {
-          after -= p.segA[(size_t)bh * (p.G - 1) + jg];
-          x += expf(p.segB[(size_t)bh * (p.G - 1) + jg] + after - m_start) *
-               p.dn[((size_t)slice * (p.G - 1) + jg) * p.dk + col];
-        }
+        for (int jg = 0; jg < nun; ++jg) x += pw[jg] * p.dn[((size_t)slice * p.NU + jg) * p.dk + col];
         nvec[col] = x;
         store_nfrag<DK>(nfrag, col, x);
       }
@@ -861,18 +978,19 @@ __global__ void __launch_bounds__(NTW, 1)
     float pba = 0.f, pbb = 0.f, pxa = 0.f, pxb = 0.f, pca = 0.f, pcb = 0.f, pg = 0.f, pxm = 0.f;
     auto fetch_gates = [&](int c) {
       const size_t r = (size_t)bh * p.sp + T0 + c * L + 2 * lane;
-      const float2 b2 = *reinterpret_cast<const float2*>(p.gb + r);
-      const float2 x2 = *reinterpret_cast<const float2*>(p.gx + r);
-      const float2 c2 = *reinterpret_cast<const float2*>(p.gxc + r);
-      const size_t cr = (size_t)bh * p.ncp + (size_t)g * p.seg_chunks + c;
+      // (L2 loads: segment 0 may read them before its grid has waited on the previous kernel)
+      const float2 b2 = __ldcg(reinterpret_cast<const float2*>(p.gb + r));
+      const float2 x2 = __ldcg(reinterpret_cast<const float2*>(p.gx + r));
+      const float2 c2 = __ldcg(reinterpret_cast<const float2*>(p.gxc + r));
+      const size_t cr = (size_t)bh * p.ncp + (size_t)s0 + c;
       pba = b2.x;
       pbb = b2.y;
       pxa = x2.x;
       pxb = x2.y;
       pca = c2.x;
       pcb = c2.y;
-      pg = p.cg[cr];
-      pxm = p.cxm[cr];
+      pg = __ldcg(p.cg + cr);
+      pxm = __ldcg(p.cxm + cr);
     };
     if (nck > 0) fetch_gates(0);
     float mc = m_start, lam = m_start;
@@ -882,7 +1000,7 @@ __global__ void __launch_bounds__(NTW, 1)
       if (!warp_wait(&bars.empty[b], ((c >> 1) & 1) ^ 1)) break;
       if (lane == 0) {
         uint8_t* base = sm + b * SM::STAGE;
-        const int t0 = chunk_row0(p, g * p.seg_chunks + c);
+        const int t0 = chunk_row0_c<REV>(p, s0 + c);
         mbar_arrive_expect_tx(&bars.full[b], SM::STAGE);
         for (int j = 0; j < DK / 64; ++j) {
           tma_load_3d(base + j * 8192, &mapQ, blk * p.dk + 64 * j, t0, bh, &bars.full[b]);
@@ -917,7 +1035,7 @@ __global__ void __launch_bounds__(NTW, 1)
       // tokens past the end have X = -inf: weight 0, column factor 0
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
-        const int t = tile_row(p, h2 ? tb : ta);  // the token's row in the chunk tiles
+        const int t = tile_row_c<REV>(h2 ? tb : ta);  // the token's row in the chunk tiles
         const float bt = h2 ? bb : ba, mt = h2 ? mb : ma, xt = h2 ? xb : xa;
         if (guard) {
           const float sint = expf(bt + mc - mt);
@@ -1126,7 +1244,7 @@ __global__ void __launch_bounds__(NTW, 1)
     for (int c = 0; c < nck; ++c) {
       const int b = c & 1, gi = c % NGB;
       const GateBuf G = gbuf(gi);
-      const int t0 = chunk_row0(p, g * p.seg_chunks + c);  // first original row of the chunk tile
+      const int t0 = chunk_row0_c<REV>(p, s0 + c);  // first original row of the chunk tile
       const int Lc = min(L, p.S - t0);                        // rows of the tile inside the sequence
       const size_t tok0 = (size_t)bh * p.S + t0;
       // P = S o e^{al_t + be_s} (bf16, rows t, 128-byte swizzled) and its row sums, once the
@@ -1171,19 +1289,18 @@ __global__ void __launch_bounds__(NTW, 1)
         if (lane == 0) mbar_arrive(&bars.s_empty);  // this warp's rows of S have left TMEM
         float rs_lo = 0.f, rs_hi = 0.f;
         uint32_t plo[8], phi[8];
-        // columns kept: [lo, hi] (causal; forward: s <= t for rows inside the sequence, reversed:
-        // tile rows hold the positions backwards, so s >= t; the rows past the end there are the
-        // identity steps, whose columns carry factor 0 and whose h is not stored)
-        const int lo_lo = p.rev ? r_lo : 0, hi_lo = p.rev ? L - 1 : (r_lo < Lc ? r_lo : -1);
-        const int lo_hi = p.rev ? r_hi : 0, hi_hi = p.rev ? L - 1 : (r_hi < Lc ? r_hi : -1);
+        // columns kept (causal): forward s <= t for rows inside the sequence; reversed, the tile rows
+        // hold the positions backwards, so s >= t (rows past the end are identity steps there, whose
+        // columns carry factor 0 and whose h is not stored)
+        const int lim_lo = REV ? r_lo : (r_lo < Lc ? r_lo : -1), lim_hi = REV ? r_hi : (r_hi < Lc ? r_hi : -1);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int s0 = 8 * j + cp;
           const float2 pa = __fmul2_rn(make_float2(r[2 * j], r[2 * j + 1]), make_float2(f_lo[2 * j], f_lo[2 * j + 1]));
           const float2 pb =
               __fmul2_rn(make_float2(r[16 + 2 * j], r[16 + 2 * j + 1]), make_float2(f_hi[2 * j], f_hi[2 * j + 1]));
-          const bool ka0 = s0 >= lo_lo && s0 <= hi_lo, ka1 = s0 + 1 >= lo_lo && s0 + 1 <= hi_lo;
-          const bool kb0 = s0 >= lo_hi && s0 <= hi_hi, kb1 = s0 + 1 >= lo_hi && s0 + 1 <= hi_hi;
+          const bool ka0 = REV ? s0 >= lim_lo : s0 <= lim_lo, ka1 = REV ? s0 + 1 >= lim_lo : s0 + 1 <= lim_lo;
+          const bool kb0 = REV ? s0 >= lim_hi : s0 <= lim_hi, kb1 = REV ? s0 + 1 >= lim_hi : s0 + 1 <= lim_hi;
           const float a0 = ka0 ? pa.x : 0.f;
           const float a1 = ka1 ? pa.y : 0.f;
           const float b0 = kb0 ? pb.x : 0.f;
@@ -1474,17 +1591,63 @@ TcPlan tc_plan(int B, int NH, int S, int nb, int dk, int dv, int num_sms) {
   while ((chunks + G - 1) / G * L > 8192) ++G;
   pl.seg_chunks = chunks > 0 ? (chunks + G - 1) / G : 1;
   pl.G = chunks > 0 ? (chunks + pl.seg_chunks - 1) / pl.seg_chunks : 1;
+  pl.seg0_chunks = pl.seg_chunks;
+  // phase A: CTAs of the walk's value tile, segment 0 summarised in two halves when that still
+  // fits one wave
+  pl.dva = pl.dvt;
+  pl.n_tiles_a = pl.n_tiles;
+  pl.ups = 1;
+  pl.NU = pl.G - 1;
+  if (pl.G > 1 && pl.seg_chunks >= 8) {
+    // Segment 0 needs no summary and walks while the others are summarised, so it gets more
+    // chunks.  Cost model in units of one walk chunk (measured on the large head: ~2.7 us per walk
+    // chunk, ~1.05 us per summary chunk, ~1.5 us per summary composed into a start state, segment 0
+    // starting ~6 us and phase A ~3 us after the call starts):
+    //   end of segment 0     = 2.2 + s0
+    //   end of the others    = 1.1 + 0.39 * (longest unit) + 0.55 * (units composed) + s
+    // over s0 with s = ceil((chunks - s0) / (G - 1)), the two-unit split of segment 0 taken when
+    // its CTAs fit one wave.
+    const long long slices_l = (long long)B * NH * nb;
+    // split segment 0 in two summary units only when the summary CTAs (G units: 2 + (G - 2)) and
+    // segment 0's walk CTAs run at the same time: together one wave
+    const bool can_split = (long long)(pl.G + 1) * pl.n_tiles * slices_l <= num_sms;
+    double best = 1e30;
+    int best_s0 = pl.seg_chunks, best_s = pl.seg_chunks, best_ups = 1;
+    for (int s0 = pl.seg_chunks; s0 <= 2 * pl.seg_chunks && s0 <= 128 && s0 < chunks; ++s0) {
+      const int s = (chunks - s0 + pl.G - 2) / (pl.G - 1);
+      if (s < 4) break;
+      for (int ups = 1; ups <= (can_split ? 2 : 1); ++ups) {
+        const int longest = (s0 + ups - 1) / ups > s ? (s0 + ups - 1) / ups : s;
+        const int composed = ups + pl.G - 2;
+        const double others = 1.1 + 0.39 * longest + 0.55 * composed + s;
+        const double first = 2.2 + s0;
+        const double cost = others > first ? others : first;
+        if (cost < best - 1e-9) {
+          best = cost;
+          best_s0 = s0;
+          best_s = s;
+          best_ups = ups;
+        }
+      }
+    }
+    pl.seg0_chunks = best_s0;
+    pl.seg_chunks = best_s;
+    pl.ups = best_ups;
+    while (pl.G > 1 && pl.seg0_chunks + (pl.G - 2) * pl.seg_chunks >= chunks) --pl.G;  // last segment non-empty
+    pl.NU = pl.G > 1 ? pl.ups + pl.G - 2 : 0;
+    if (pl.G == 1) pl.ups = 1;
+  }
   return pl;
 }
 
 size_t tc_workspace_bytes(const TcPlan& pl, long long BH, int nb, int dk, int dv) {
   const long long slices = BH * nb;
-  const size_t G1 = pl.G > 1 ? pl.G - 1 : 0;
+  const size_t NU = pl.NU;
   size_t off = 256;  // error word
-  off += ((size_t)slices * G1 * dv * dk * 4 + 255) / 256 * 256;
-  off += ((size_t)slices * G1 * dk * 4 + 255) / 256 * 256;
-  off += 2 * (((size_t)BH * G1 * 4 + 255) / 256 * 256);
-  const size_t ncp = (size_t)pl.G * pl.seg_chunks, sp = ncp * L;
+  off += ((size_t)slices * NU * dv * dk * 4 + 255) / 256 * 256;
+  off += ((size_t)slices * NU * dk * 4 + 255) / 256 * 256;
+  off += 2 * (((size_t)BH * NU * 4 + 255) / 256 * 256);
+  const size_t ncp = (size_t)pl.seg0_chunks + (size_t)(pl.G - 1) * pl.seg_chunks, sp = ncp * L;
   off += 3 * (((size_t)BH * sp * 4 + 255) / 256 * 256);
   off += 2 * (((size_t)BH * ncp * 4 + 255) / 256 * 256);
   return off;
@@ -1508,29 +1671,37 @@ static cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 bl
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-template <int DK, int DVT, bool SN>
+template <int DK, int DVA>
+static cudaError_t launch_segment(const TcPlan& pl, const TcParams& prm, const CUtensorMap& mk, const CUtensorMap& mv,
+                                  long long slices, cudaStream_t stream) {
+  const int smemA = SegCfg<DK, DVA>::BYTES_FIXED + pl.seg0_chunks * 4;  // + one offset per chunk of a unit
+  cudaError_t e = cudaFuncSetAttribute(tc_segment_kernel<DK, DVA>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemA);
+  if (e != cudaSuccess) return e;
+  dim3 gridA(pl.n_tiles_a, pl.NU, (unsigned)slices);
+  return launch_dependent(tc_segment_kernel<DK, DVA>, gridA, dim3(NTA), smemA, stream, mk, mv, prm);
+}
+
+template <int DK, int DVT, bool SN, bool REV>
 static cudaError_t launch_tc_dk(const TcPlan& pl, const TcParams& prm, const CUtensorMap& mq, const CUtensorMap& mk,
-                                const CUtensorMap& mv, const CUtensorMap& mh, long long slices, cudaStream_t stream,
-                                cudaEvent_t ev0, cudaEvent_t ev1) {
+                                const CUtensorMap& mv, const CUtensorMap& mh, const CUtensorMap& ms, long long slices,
+                                cudaStream_t stream, cudaEvent_t ev0, cudaEvent_t ev1) {
   cudaError_t e;
   const long long BH = slices / prm.nb;
   tc_gate_prep_kernel<<<(unsigned)((BH * prm.ncp + 7) / 8), 256, 0, stream>>>(prm, (int)BH);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (pl.G > 1) {
-    const int smemA = NSA * (DK * 128 + DVT * 128) + (128 * 8 + NSA * L + pl.seg_chunks) * 4 + 1024;
-    e = cudaFuncSetAttribute(tc_segment_kernel<DK, DVT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemA);
-    if (e != cudaSuccess) return e;
-    dim3 gridA(pl.n_tiles, pl.G - 1, (unsigned)slices);
-    e = launch_dependent(tc_segment_kernel<DK, DVT>, gridA, dim3(NTA), smemA, stream, mk, mv, prm);
+  if (pl.NU > 0) {
+    e = pl.dva == 256   ? launch_segment<DK, 256>(pl, prm, mk, mv, slices, stream)
+        : pl.dva == 128 ? launch_segment<DK, 128>(pl, prm, mk, mv, slices, stream)
+                        : launch_segment<DK, 64>(pl, prm, mk, mv, slices, stream);
     if (e != cudaSuccess) return e;
   }
   const int smemC = WalkSmem<DK, DVT>::BYTES;
-  e = cudaFuncSetAttribute(tc_walk_kernel<DK, DVT, SN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemC);
+  e = cudaFuncSetAttribute(tc_walk_kernel<DK, DVT, SN, REV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemC);
   if (e != cudaSuccess) return e;
   if (ev0) cudaEventRecord(ev0, stream);
-  dim3 gridC(pl.n_tiles, pl.G, (unsigned)slices);
-  e = launch_dependent(tc_walk_kernel<DK, DVT, SN>, gridC, dim3(NTW), smemC, stream, mq, mk, mv, mh, prm);
+  dim3 gridC(pl.n_tiles, (unsigned)slices, pl.G);
+  e = launch_dependent(tc_walk_kernel<DK, DVT, SN, REV>, gridC, dim3(NTW), smemC, stream, mq, mk, mv, mh, ms, prm);
   if (ev1) cudaEventRecord(ev1, stream);
   return e;
 }
@@ -1568,18 +1739,27 @@ cudaError_t launch_tc(const WalkArgs& a, const TcPlan& pl, void* ws, cudaStream_
   prm.n_out = a.n_out;
   prm.m_out = a.m_out;
   char* w = static_cast<char*>(ws);
-  const size_t G1 = pl.G > 1 ? pl.G - 1 : 0;
+  const size_t NU = pl.NU;
+  prm.seg0_chunks = pl.seg0_chunks;
+  prm.ups = pl.ups;
+  prm.NU = pl.NU;
+  prm.n_tiles_a = pl.n_tiles_a;
   prm.err = reinterpret_cast<unsigned int*>(w);
   size_t off = 256;
   prm.dC = reinterpret_cast<float*>(w + off);
-  off += ((size_t)slices * G1 * a.dv * a.dk * 4 + 255) / 256 * 256;
+  off += ((size_t)slices * NU * a.dv * a.dk * 4 + 255) / 256 * 256;
   prm.dn = reinterpret_cast<float*>(w + off);
-  off += ((size_t)slices * G1 * a.dk * 4 + 255) / 256 * 256;
+  off += ((size_t)slices * NU * a.dk * 4 + 255) / 256 * 256;
   prm.segA = reinterpret_cast<float*>(w + off);
-  off += ((size_t)BH * G1 * 4 + 255) / 256 * 256;
+  off += ((size_t)BH * NU * 4 + 255) / 256 * 256;
   prm.segB = reinterpret_cast<float*>(w + off);
-  off += ((size_t)BH * G1 * 4 + 255) / 256 * 256;
-  prm.ncp = pl.G * pl.seg_chunks;
+  off += ((size_t)BH * NU * 4 + 255) / 256 * 256;
+  prm.ncp = pl.seg0_chunks + (pl.G - 1) * pl.seg_chunks;
+  // the segment summaries [slices * NU * dv rows][dk] fp32, read back by the walk through TMA
+  CUtensorMap ms;
+  memset(&ms, 0, sizeof(ms));
+  if (pl.NU > 0 && !make_map_f32_2d(&ms, prm.dC, (uint64_t)a.dk, (uint64_t)slices * pl.NU * a.dv, 64))
+    return cudaErrorInvalidValue;
   prm.sp = prm.ncp * L;
   prm.wait = a.wait_cycles > 0 ? a.wait_cycles : WAIT_DEFAULT;
   prm.nbias = a.retention ? nullptr : a.nbias;
@@ -1592,21 +1772,26 @@ cudaError_t launch_tc(const WalkArgs& a, const TcPlan& pl, void* ws, cudaStream_
   }
   cudaError_t e = cudaMemsetAsync(w, 0, 4, stream);
   if (e != cudaSuccess) return e;
-  if (prm.nbias) {
-    if (a.dk == 256 && pl.dvt == 128) return launch_tc_dk<256, 128, true>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
-    if (a.dk == 256 && pl.dvt == 64) return launch_tc_dk<256, 64, true>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
-    if (a.dk == 128 && pl.dvt == 128) return launch_tc_dk<128, 128, true>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
-    if (a.dk == 128 && pl.dvt == 64) return launch_tc_dk<128, 64, true>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
-    if (a.dk == 64 && pl.dvt == 128) return launch_tc_dk<64, 128, true>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
-    if (a.dk == 64 && pl.dvt == 64) return launch_tc_dk<64, 64, true>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
-    return cudaErrorInvalidValue;
-  }
-  if (a.dk == 256 && pl.dvt == 128) return launch_tc_dk<256, 128, false>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
-  if (a.dk == 256 && pl.dvt == 64) return launch_tc_dk<256, 64, false>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
-  if (a.dk == 128 && pl.dvt == 128) return launch_tc_dk<128, 128, false>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
-  if (a.dk == 128 && pl.dvt == 64) return launch_tc_dk<128, 64, false>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
-  if (a.dk == 64 && pl.dvt == 128) return launch_tc_dk<64, 128, false>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
-  if (a.dk == 64 && pl.dvt == 64) return launch_tc_dk<64, 64, false>(pl, prm, mq, mk, mv, mh, slices, stream, ev0, ev1);
+#define MLSTM_TC_DISPATCH(SNV, REVV)                                                                       \
+  do {                                                                                                   \
+    if (a.dk == 256 && pl.dvt == 128)                                                                    \
+      return launch_tc_dk<256, 128, SNV, REVV>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1);       \
+    if (a.dk == 256 && pl.dvt == 64)                                                                     \
+      return launch_tc_dk<256, 64, SNV, REVV>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1);        \
+    if (a.dk == 128 && pl.dvt == 128)                                                                    \
+      return launch_tc_dk<128, 128, SNV, REVV>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1);       \
+    if (a.dk == 128 && pl.dvt == 64)                                                                     \
+      return launch_tc_dk<128, 64, SNV, REVV>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1);        \
+    if (a.dk == 64 && pl.dvt == 128)                                                                     \
+      return launch_tc_dk<64, 128, SNV, REVV>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1);        \
+    if (a.dk == 64 && pl.dvt == 64)                                                                      \
+      return launch_tc_dk<64, 64, SNV, REVV>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1);         \
+  } while (0)
+  // walk variants: the vector normaliser forward and reversed, the scalar normaliser forward
+  if (prm.nbias && !prm.rev) MLSTM_TC_DISPATCH(true, false);
+  else if (!prm.nbias && prm.rev) MLSTM_TC_DISPATCH(false, true);
+  else if (!prm.nbias) MLSTM_TC_DISPATCH(false, false);
+#undef MLSTM_TC_DISPATCH
   return cudaErrorInvalidValue;
 }
 

@@ -68,10 +68,15 @@ cudaError_t launch_simt_walk(const WalkArgs& a, cudaStream_t stream);
 // Tensor-core (tcgen05) chunkwise prefill: bf16, chunk 64, block key width 64/128/256,
 // block value width a multiple of 64.
 struct TcPlan {
-  int dvt;         // value rows per CTA (MMA M): 128 or 64
-  int n_tiles;     // value tiles per block
-  int G;           // sequence segments per (batch, head, block)
-  int seg_chunks;  // chunks per segment
+  int dvt;          // value rows per walk CTA (MMA M): 128 or 64
+  int n_tiles;      // value tiles per block
+  int G;            // sequence segments per (batch, head, block)
+  int seg_chunks;   // chunks per segment (segments 1 .. G-1)
+  int seg0_chunks;  // chunks of segment 0
+  int dva;          // value rows per segment-summary CTA (64, 128 or 256)
+  int n_tiles_a;    // summary CTAs per block and unit
+  int ups;          // summary units per segment (1 or 2)
+  int NU;           // summary units: ups * (G - 1)
 };
 bool tc_supported(int dtype, int chunk, int dk, int dv, int DHQK, int DHV);
 int tc_num_sms();

@@ -352,6 +352,9 @@ mlstm_status_t mlstm_fwd_chunkwise_plan(const mlstm_fwd_params_t* p, mlstm_fwd_p
     plan->ctas_main = (int)(s.tcp.n_tiles * s.tcp.G * s.BH * s.nb);
     plan->kernels = (s.BH == 0 || s.S == 0) ? 0 : (s.tcp.G > 1 ? 3 : 2);
     plan->workspace_bytes = fwd_layout(s).total;
+    plan->seg0_chunks = s.tcp.seg0_chunks;
+    plan->seg_chunks = s.tcp.seg_chunks;
+    plan->summary_units = s.tcp.NU;
     return MLSTM_OK;
   }
   plan->tensor_core = 0;

@@ -40,4 +40,19 @@ inline bool make_map_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, ui
   return r == CUDA_SUCCESS;
 }
 
+// 2-D fp32 tensor [d1][d0] (d0 contiguous, d0 * 4 bytes a multiple of 16), box {32, box_rows}
+// (128-byte rows), 128-byte swizzle.
+inline bool make_map_f32_2d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {d0, d1};
+  const cuuint64_t strides[1] = {d0 * 4};
+  const cuuint32_t box[2] = {32, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace mlstm

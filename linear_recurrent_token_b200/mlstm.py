@@ -41,7 +41,8 @@ GDN2_RECURRENT, GDN2_CHUNK = 0, 1
 
 class FwdPlan(ctypes.Structure):
     _fields_ = [("tensor_core", ctypes.c_int), ("segments", ctypes.c_int), ("dv_tile", ctypes.c_int),
-                ("ctas_main", ctypes.c_int), ("kernels", ctypes.c_int), ("workspace_bytes", ctypes.c_size_t)]
+                ("ctas_main", ctypes.c_int), ("kernels", ctypes.c_int), ("workspace_bytes", ctypes.c_size_t),
+                ("seg0_chunks", ctypes.c_int), ("seg_chunks", ctypes.c_int), ("summary_units", ctypes.c_int)]
 
 
 class MlstmError(RuntimeError):
