@@ -74,8 +74,11 @@ typedef enum {
   MLSTM_ERR_WORKSPACE = 5,  /* workspace NULL or smaller than the size query       */
   MLSTM_ERR_CUDA = 6,       /* the CUDA runtime reported an error at launch        */
   MLSTM_ERR_ALIAS = 7,      /* an output overlaps an input it must not overlap     */
-  MLSTM_ERR_TIMEOUT = 8     /* a bounded device-side wait ran out (reported by the
+  MLSTM_ERR_TIMEOUT = 8,    /* a bounded device-side wait ran out (reported by the
                                status calls after the work has finished)           */
+  MLSTM_ERR_BOUNDS = 9      /* bounds-checked build only: an access failed its check
+                               and was skipped (status calls; see
+                               mlstm_fwd_chunkwise_bounds_record)                  */
 } mlstm_status_t;
 
 typedef enum { MLSTM_F32 = 0, MLSTM_BF16 = 1 } mlstm_dtype_t;
@@ -208,6 +211,9 @@ size_t mlstm_noalloc_scratch_bytes(void);
  *                      have no such waits)
  *   MLSTM_ERR_TIMEOUT  a wait ran out (params->wait_limit_cycles); that call's outputs and
  *                      final state are unspecified, the workspace can be used again
+ *   MLSTM_ERR_BOUNDS   (bounds-checked build only) an access failed its check and was
+ *                      skipped; outputs unspecified; mlstm_fwd_chunkwise_bounds_record says
+ *                      which
  *   MLSTM_ERR_CUDA     the synchronisation or the read failed (for example an earlier
  *                      asynchronous error on the stream)
  *   MLSTM_ERR_NULL / _SHAPE / _DTYPE as for mlstm_fwd_chunkwise (workspace NULL: _NULL when
@@ -218,6 +224,29 @@ size_t mlstm_noalloc_scratch_bytes(void);
 mlstm_status_t mlstm_fwd_chunkwise_status(const mlstm_fwd_params_t* p, const void* workspace,
                                           mlstm_stream_t stream);
 mlstm_status_t mlstm_fwd_chunkwise_noalloc_status(const mlstm_fwd_params_t* p, mlstm_stream_t stream);
+
+/*
+ * Bounds-checked debug build.  libmlstm_checked.so is the same library compiled with every
+ * plain global access of the tensor-core prefill kernels (gate preparation, segment
+ * summaries, walk) checked against its buffer's extent, every TMA copy's coordinates checked
+ * against the copy rules (innermost coordinate on a 16-byte boundary, stores from
+ * non-negative coordinates, the box overlapping its tensor) and every offset into the h
+ * staging tile checked against the tile, before the access is made.  A failing check skips
+ * the access and records the first failure in the workspace; nothing traps.  The status calls
+ * above then return MLSTM_ERR_BOUNDS.  The checks cost time: the build is for tests.
+ *
+ * mlstm_bounds_checked: 1 in libmlstm_checked.so, 0 in libmlstm.so.
+ * mlstm_fwd_chunkwise_bounds_record: synchronises `stream` and copies the first failure of
+ * the last prefill with `workspace` (arguments as for mlstm_fwd_chunkwise_status) to *site (0:
+ * none; the site numbers name the kernel step and buffer, see the library's bounds.cuh),
+ * *index (the offending index or coordinate) and *extent (its limit).  Any of the three
+ * pointers may be NULL.  In libmlstm.so it reports no failure.  MLSTM_ERR_CUDA if the read
+ * fails; argument errors as for mlstm_fwd_chunkwise_status.
+ */
+int mlstm_bounds_checked(void);
+mlstm_status_t mlstm_fwd_chunkwise_bounds_record(const mlstm_fwd_params_t* p, const void* workspace,
+                                                 mlstm_stream_t stream, int* site, long long* index,
+                                                 long long* extent);
 
 /*
  * The same prefill over the reversed sequence: token S-1 is read first and token 0 last;
@@ -248,8 +277,10 @@ mlstm_status_t mlstm_fwd_chunkwise_reversed(const mlstm_fwd_params_t* p,
  * (batch, head), shared by the head's blocks.  Arguments as for mlstm_fwd_chunkwise, except:
  *   bias    [NH]   fp32   required (if S > 0)
  *   n0, n_out [B,NH] fp32 stabilised scalar normaliser (NULL = zero / not written)
- * retention is rejected (MLSTM_ERR_SHAPE: retention has no normaliser).  Runs on the SIMT fp32
- * kernels for every dtype; workspace: mlstm_fwd_chunkwise_scalar_normaliser_workspace_size.
+ * retention is rejected (MLSTM_ERR_SHAPE: retention has no normaliser).  Runs on the
+ * tensor-core kernels for the sizes mlstm_fwd_chunkwise runs there (bf16, chunk 64, block
+ * widths 64/128/256; status calls as for mlstm_fwd_chunkwise), else on the SIMT fp32 kernels;
+ * workspace: mlstm_fwd_chunkwise_scalar_normaliser_workspace_size.
  */
 size_t mlstm_fwd_chunkwise_scalar_normaliser_workspace_size(const mlstm_fwd_params_t* p);
 mlstm_status_t mlstm_fwd_chunkwise_scalar_normaliser(const mlstm_fwd_params_t* p,

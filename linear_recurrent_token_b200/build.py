@@ -1,4 +1,5 @@
-"""Builds libmlstm.so in-tree with nvcc for sm_100a (B200)."""
+"""Builds libmlstm.so in-tree with nvcc for sm_100a (B200), and libmlstm_checked.so: the same
+library with the bounds checks of the tensor-core prefill compiled in (MLSTM_BOUNDS_CHECK)."""
 from __future__ import annotations
 
 import glob
@@ -11,6 +12,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmlstm.so")
+LIB_CHECKED = os.path.join(PKG, "libmlstm_checked.so")
+# sources whose objects differ in the bounds-checked build (the others are linked as they are)
+CHECKED_SOURCES = ("chunkwise_tc.cu", "mlstm_api.cu")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -25,9 +29,9 @@ def sources():
 
 
 def _stale() -> bool:
-    if not os.path.exists(LIB):
+    if not os.path.exists(LIB) or not os.path.exists(LIB_CHECKED):
         return True
-    t = os.path.getmtime(LIB)
+    t = min(os.path.getmtime(LIB), os.path.getmtime(LIB_CHECKED))
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) \
         + glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(d) > t for d in deps)
@@ -41,31 +45,39 @@ def nvcc() -> str:
 
 def build(force: bool = False, verbose: bool = False) -> str:
     """Compile every csrc/*.cu (in parallel, objects under _build/) and link them into
-    linear_recurrent_token_b200/libmlstm.so (static cudart)."""
+    linear_recurrent_token_b200/libmlstm.so (static cudart); compile CHECKED_SOURCES again with
+    -DMLSTM_BOUNDS_CHECK and link libmlstm_checked.so from those and the other objects."""
     if not force and not _stale():
         return LIB
     from concurrent.futures import ThreadPoolExecutor
     objdir = os.path.join(ROOT, "_build")
-    os.makedirs(objdir, exist_ok=True)
+    os.makedirs(os.path.join(objdir, "checked"), exist_ok=True)
     compile_flags = [f for f in NVCC_FLAGS if f != "-shared"]
 
-    def compile_one(src):
-        obj = os.path.join(objdir, os.path.basename(src) + ".o")
-        cmd = [nvcc()] + compile_flags + ["-I", INCLUDE, "-I", CSRC, "-c", "-o", obj, src]
+    def compile_one(job):
+        src, checked = job
+        obj = os.path.join(objdir, "checked" if checked else "", os.path.basename(src) + ".o")
+        cmd = [nvcc()] + compile_flags + (["-DMLSTM_BOUNDS_CHECK"] if checked else []) \
+            + ["-I", INCLUDE, "-I", CSRC, "-c", "-o", obj, src]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
         subprocess.check_call(cmd)
         return obj
 
     srcs = sources()
-    with ThreadPoolExecutor(max_workers=min(len(srcs), os.cpu_count() or 4)) as ex:
-        objs = list(ex.map(compile_one, srcs))
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [nvcc()] + NVCC_FLAGS + ["-o", tmp] + objs
-    if verbose:
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
+    jobs = [(s, False) for s in srcs] + [(s, True) for s in srcs if os.path.basename(s) in CHECKED_SOURCES]
+    with ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 4)) as ex:
+        objs = list(ex.map(compile_one, jobs))
+    plain = objs[:len(srcs)]
+    checked = {os.path.basename(o)[:-2]: o for o in objs[len(srcs):]}
+    variants = ((LIB, plain), (LIB_CHECKED, [checked.get(os.path.basename(o)[:-2], o) for o in plain]))
+    for lib, lib_objs in variants:
+        tmp = lib + ".tmp%d" % os.getpid()
+        cmd = [nvcc()] + NVCC_FLAGS + ["-o", tmp] + lib_objs
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        subprocess.check_call(cmd)
+        os.replace(tmp, lib)
     return LIB
 
 

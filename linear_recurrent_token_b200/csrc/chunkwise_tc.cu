@@ -36,6 +36,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "bounds.cuh"
 #include "sm100.cuh"
 #include "tma_host.h"
 
@@ -76,6 +77,7 @@ struct TcParams {
   // (halves when ups = 2), the others in one: NU units in all, by CTAs of dv / n_tiles_a value
   // rows each
   int seg0_chunks, ups, NU, n_tiles_a;
+  int BH, slices;  // batch x heads, slices (BH x num_blocks): extents for the bounds-checked build
 };
 
 // Processing-order chunks [s0, s1) of segment g.
@@ -154,6 +156,11 @@ __device__ __forceinline__ void gate_vals(const TcParams& p, size_t tok, int hea
     lf = retention_log_gamma(head);
     li = 0.f;
   } else {
+    if (!in_bounds(p.err, BS_GATE_INPUT, (long long)tok, (long long)p.BH * p.S)) {
+      lf = 0.f;
+      li = -INFINITY;
+      return;
+    }
     lf = log_sigmoid(p.fg[tok]);
     li = p.ig[tok];
   }
@@ -302,10 +309,12 @@ __global__ void __launch_bounds__(256) tc_gate_prep_kernel(TcParams p, int BH) {
   if (lane == 0) ex = -INFINITY;
   const float xca = fmaxf(ex, xa), xcb = fmaxf(xca, xb);
   const size_t r = (size_t)bh * p.sp + t0 + ta;
-  *reinterpret_cast<float2*>(p.gb + r) = make_float2(ba, bb);
-  *reinterpret_cast<float2*>(p.gx + r) = make_float2(xa, xb);
-  *reinterpret_cast<float2*>(p.gxc + r) = make_float2(xca, xcb);
-  if (lane == 31) {
+  if (in_bounds(p.err, BS_GATE_PLANES, (long long)r + 1, (long long)p.BH * p.sp)) {
+    *reinterpret_cast<float2*>(p.gb + r) = make_float2(ba, bb);
+    *reinterpret_cast<float2*>(p.gx + r) = make_float2(xa, xb);
+    *reinterpret_cast<float2*>(p.gxc + r) = make_float2(xca, xcb);
+  }
+  if (lane == 31 && in_bounds(p.err, BS_GATE_CHUNK, (long long)bh * p.ncp + c, (long long)p.BH * p.ncp)) {
     p.cg[(size_t)bh * p.ncp + c] = bb;
     p.cxm[(size_t)bh * p.ncp + c] = xcb;
   }
@@ -385,9 +394,12 @@ __global__ void __launch_bounds__(NTA, 1)
     const int row0 = chunk_row0(p, u0 + c);
     mbar_arrive_expect_tx(&full[st], KB + VB);
     for (int jj = 0; jj < DK / 64; ++jj)
-      tma_load_3d(kb + jj * 8192, &mapK, blk * p.dk + 64 * jj, row0, bh, &full[st]);
+      if (tma_box_ok(p.err, BS_SEG_TMA, blk * p.dk + 64 * jj, row0, 8, p.DHQK, p.S, L, false) &&
+          in_bounds(p.err, BS_SEG_TMA, bh, p.BH))
+        tma_load_3d(kb + jj * 8192, &mapK, blk * p.dk + 64 * jj, row0, bh, &full[st]);
     for (int jj = 0; jj < DVA / 64; ++jj)
-      tma_load_3d(kb + KB + jj * 8192, &mapV, blk * p.dv + v0 + 64 * jj, row0, bh, &full[st]);
+      if (tma_box_ok(p.err, BS_SEG_TMA, blk * p.dv + v0 + 64 * jj, row0, 8, p.DHV, p.S, L, false))
+        tma_load_3d(kb + KB + jj * 8192, &mapV, blk * p.dv + v0 + 64 * jj, row0, bh, &full[st]);
   };
   // K and V are inputs: the first stages load while the previous kernel finishes
   int n_issued = 0;  // chunks whose loads thread 0 has issued
@@ -408,8 +420,9 @@ __global__ void __launch_bounds__(NTA, 1)
     // chunk totals in passes of NTA (a unit has at most a few hundred chunks)
     for (int base = 0; base < nck; base += NTA) {
       const int c = base + tid;
-      const float gcv = c < nck ? p.cg[crow + c] : 0.f;
-      const float xmv = c < nck ? p.cxm[crow + c] : -INFINITY;
+      const bool cin = c < nck && in_bounds(p.err, BS_SEG_CHUNK, (long long)(crow + c), (long long)p.BH * p.ncp);
+      const float gcv = cin ? p.cg[crow + c] : 0.f;
+      const float xmv = cin ? p.cxm[crow + c] : -INFINITY;
       float inc = gcv;
       for (int o = 1; o < 32; o <<= 1) {
         const float u = __shfl_up_sync(0xffffffffu, inc, o);
@@ -438,7 +451,8 @@ __global__ void __launch_bounds__(NTA, 1)
     if (p.retention) Mg = 0.f;
     __syncthreads();
     for (int c = tid; c < nck; c += NTA) coff[c] = total - coff[c] - Mg;
-    if (tile == 0 && blk == 0 && tid == 0) {
+    if (tile == 0 && blk == 0 && tid == 0 &&
+        in_bounds(p.err, BS_SEG_SCALARS, (long long)bh * p.NU + j, (long long)p.BH * p.NU)) {
       p.segA[(size_t)bh * p.NU + j] = total;
       p.segB[(size_t)bh * p.NU + j] = Mg;
     }
@@ -454,7 +468,9 @@ __global__ void __launch_bounds__(NTA, 1)
     // omega_s = e^{coff_c + X_s}: lane -> tokens 2 lane, 2 lane + 1 (X of the next chunk
     // prefetched into registers)
     const float* gxr = p.gx + (size_t)bh * p.sp + T0 + 2 * lane;
-    float2 gxn = *reinterpret_cast<const float2*>(gxr);
+    const long long gxr0 = (long long)bh * p.sp + T0 + 2 * lane, gx_ext = (long long)p.BH * p.sp;
+    float2 gxn = make_float2(-INFINITY, -INFINITY);
+    if (in_bounds(p.err, BS_SEG_CHUNK, gxr0 + 1, gx_ext)) gxn = *reinterpret_cast<const float2*>(gxr);
     float osum = 0.f;  // scalar normaliser: this lane's share of the unit's sum of weights
     for (int c = 0; c < nck; ++c) {
       const int st = c % NS;
@@ -473,14 +489,17 @@ __global__ void __launch_bounds__(NTA, 1)
       else
         *reinterpret_cast<float2*>(omb + st * L + 2 * lane) = om2;
       osum += om2.x + om2.y;
-      if (c + 1 < nck) gxn = *reinterpret_cast<const float2*>(gxr + (size_t)(c + 1) * L);
+      if (c + 1 < nck && in_bounds(p.err, BS_SEG_CHUNK, gxr0 + (long long)(c + 1) * L + 1, gx_ext))
+        gxn = *reinterpret_cast<const float2*>(gxr + (size_t)(c + 1) * L);
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[st]);
     }
     if (p.nbias && !p.retention) {  // dn of the scalar normaliser: sum over the unit of omega_s
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) osum += __shfl_xor_sync(0xffffffffu, osum, o);
-      if (lane == 0 && tile == 0 && !abort_flag) p.dn[((size_t)slice * p.NU + j) * p.dk] = osum;
+      if (lane == 0 && tile == 0 && !abort_flag &&
+          in_bounds(p.err, BS_SEG_DN, ((long long)slice * p.NU + j) * p.dk, (long long)p.slices * p.NU * p.dk))
+        p.dn[((size_t)slice * p.NU + j) * p.dk] = osum;
     }
   } else if (warp == 1) {
     // =============================================================== MMA warp
@@ -574,7 +593,10 @@ __global__ void __launch_bounds__(NTA, 1)
         float r[32];
         tmem_ld32(tm + ((uint32_t)(32 * quarter) << 16) + a * DK + c0, r);
         tmem_wait_ld();
-        if (dst && !abort_flag)
+        if (dst && !abort_flag &&
+            in_bounds(p.err, BS_SEG_DC,
+                      (((long long)slice * p.NU + j) * p.dv + v0 + a * MA + row) * p.dk + c0 + 31,
+                      (long long)p.slices * p.NU * p.dv * p.dk))
 #pragma unroll
           for (int jj = 0; jj < 32; jj += 4)
             *reinterpret_cast<float4*>(dst + c0 + jj) = make_float4(r[jj], r[jj + 1], r[jj + 2], r[jj + 3]);
@@ -587,7 +609,9 @@ __global__ void __launch_bounds__(NTA, 1)
       for (int col = gt; col < ncg * 8 && dn0 + col < DK; col += 128) {
         float x = 0.f;
         for (int r = 0; r < nrg; ++r) x += dnp[(r * ncg + col / 8) * 8 + (col & 7)];
-        if (!abort_flag) p.dn[((size_t)slice * p.NU + j) * p.dk + dn0 + col] = x;
+        if (!abort_flag && in_bounds(p.err, BS_SEG_DN, ((long long)slice * p.NU + j) * p.dk + dn0 + col,
+                                     (long long)p.slices * p.NU * p.dk))
+          p.dn[((size_t)slice * p.NU + j) * p.dk + dn0 + col] = x;
       }
     }
   }
@@ -771,10 +795,11 @@ __global__ void __launch_bounds__(NTW, 1)
   if (g > 0 || p.NU == 0) grid_dep_wait();
   // ---- start state of the segment (see the file header); warps 3-10 fill TMEM and n.
   // It is stabilised at m_start, so lam starts at m_start.
-  float m_start = ret ? 0.f : (p.m0 ? p.m0[bh] : 0.f);
+  float m_start = ret ? 0.f : (p.m0 && in_bounds(p.err, BS_WALK_START, bh, p.BH) ? p.m0[bh] : 0.f);
   const float m_init = m_start;
   float gsum = 0.f;
-  const int nun = units_before(p, g);  // summary units before this segment
+  int nun = units_before(p, g);  // summary units before this segment
+  if (nun > 0 && !in_bounds(p.err, BS_WALK_START, (long long)bh * p.NU + nun - 1, (long long)p.BH * p.NU)) nun = 0;
   for (int j = 0; j < nun; ++j) {
     const float A = p.segA[(size_t)bh * p.NU + j], Bm = p.segB[(size_t)bh * p.NU + j];
     if (!ret) m_start = fmaxf(A + m_start, Bm);
@@ -805,7 +830,9 @@ __global__ void __launch_bounds__(NTW, 1)
       float r[16];
 #pragma unroll
       for (int jj = 0; jj < 16; ++jj) r[jj] = 0.f;
-      if (row >= 0 && p.C0) {
+      if (row >= 0 && p.C0 &&
+          in_bounds(p.err, BS_WALK_START, ((long long)slice * p.dv + v0 + row) * p.dk + c0 + 15,
+                    (long long)p.slices * p.dv * p.dk)) {
         const float4* src = reinterpret_cast<const float4*>(p.C0 + ((size_t)slice * p.dv + v0 + row) * p.dk + c0);
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
@@ -827,7 +854,9 @@ __global__ void __launch_bounds__(NTW, 1)
       const int r0 = ((int)slice * p.NU + j) * p.dv + v0;
       for (int rb = 0; rb < (DVT + 63) / 64; ++rb)
         for (int cb = 0; cb < DK / 32; ++cb)
-          tma_load_2d(sm + (rb * (DK / 32) + cb) * 8192, &mapS, 32 * cb, r0 + 64 * rb, &bars.comp);
+          if (tma_box_ok(p.err, BS_WALK_SUM_TMA, 32 * cb, r0 + 64 * rb, 4, p.dk, (long long)p.slices * p.NU * p.dv,
+                         64, true))  // held to a store's rule: the tile must start inside the summaries
+            tma_load_2d(sm + (rb * (DK / 32) + cb) * 8192, &mapS, 32 * cb, r0 + 64 * rb, &bars.comp);
     }
     if (!mbar_wait(&bars.comp, j & 1, p.wait)) {  // give up on the data, but let the copies land
       abort_flag = 1;
@@ -869,14 +898,21 @@ __global__ void __launch_bounds__(NTW, 1)
     const int nt2 = warp >= 11 ? tid - 352 : 128 + tid;  // 0..223
     if (SN) {
       if (nt2 == 0) {
-        float x = p.n0 ? wc0 * p.n0[bh] : 0.f;
-        for (int jg = 0; jg < nun; ++jg) x += pw[jg] * p.dn[((size_t)slice * p.NU + jg) * p.dk];
+        float x = p.n0 && in_bounds(p.err, BS_WALK_START, bh, p.BH) ? wc0 * p.n0[bh] : 0.f;
+        for (int jg = 0; jg < nun; ++jg)
+          if (in_bounds(p.err, BS_WALK_START, ((long long)slice * p.NU + jg) * p.dk, (long long)p.slices * p.NU * p.dk))
+            x += pw[jg] * p.dn[((size_t)slice * p.NU + jg) * p.dk];
         nvec[0] = x;
       }
     } else if (!ret)
       for (int col = nt2; col < DK; col += 224) {
-        float x = p.n0 ? wc0 * p.n0[(size_t)slice * p.dk + col] : 0.f;
-        for (int jg = 0; jg < nun; ++jg) x += pw[jg] * p.dn[((size_t)slice * p.NU + jg) * p.dk + col];
+        float x = p.n0 && in_bounds(p.err, BS_WALK_START, (long long)slice * p.dk + col, (long long)p.slices * p.dk)
+                      ? wc0 * p.n0[(size_t)slice * p.dk + col]
+                      : 0.f;
+        for (int jg = 0; jg < nun; ++jg)
+          if (in_bounds(p.err, BS_WALK_START, ((long long)slice * p.NU + jg) * p.dk + col,
+                        (long long)p.slices * p.NU * p.dk))
+            x += pw[jg] * p.dn[((size_t)slice * p.NU + jg) * p.dk + col];
         nvec[col] = x;
         store_nfrag<DK>(nfrag, col, x);
       }
@@ -978,11 +1014,14 @@ __global__ void __launch_bounds__(NTW, 1)
     float pba = 0.f, pbb = 0.f, pxa = 0.f, pxb = 0.f, pca = 0.f, pcb = 0.f, pg = 0.f, pxm = 0.f;
     auto fetch_gates = [&](int c) {
       const size_t r = (size_t)bh * p.sp + T0 + c * L + 2 * lane;
+      const size_t cr = (size_t)bh * p.ncp + (size_t)s0 + c;
+      if (!in_bounds(p.err, BS_WALK_GATES, (long long)r + 1, (long long)p.BH * p.sp) ||
+          !in_bounds(p.err, BS_WALK_GATES, (long long)cr, (long long)p.BH * p.ncp))
+        return;
       // (L2 loads: segment 0 may read them before its grid has waited on the previous kernel)
       const float2 b2 = __ldcg(reinterpret_cast<const float2*>(p.gb + r));
       const float2 x2 = __ldcg(reinterpret_cast<const float2*>(p.gx + r));
       const float2 c2 = __ldcg(reinterpret_cast<const float2*>(p.gxc + r));
-      const size_t cr = (size_t)bh * p.ncp + (size_t)s0 + c;
       pba = b2.x;
       pbb = b2.y;
       pxa = x2.x;
@@ -1002,12 +1041,15 @@ __global__ void __launch_bounds__(NTW, 1)
         uint8_t* base = sm + b * SM::STAGE;
         const int t0 = chunk_row0_c<REV>(p, s0 + c);
         mbar_arrive_expect_tx(&bars.full[b], SM::STAGE);
-        for (int j = 0; j < DK / 64; ++j) {
-          tma_load_3d(base + j * 8192, &mapQ, blk * p.dk + 64 * j, t0, bh, &bars.full[b]);
-          tma_load_3d(base + SM::QB + j * 8192, &mapK, blk * p.dk + 64 * j, t0, bh, &bars.full[b]);
-        }
+        for (int j = 0; j < DK / 64; ++j)
+          if (tma_box_ok(p.err, BS_WALK_TMA, blk * p.dk + 64 * j, t0, 8, p.DHQK, p.S, L, false) &&
+              in_bounds(p.err, BS_WALK_TMA, bh, p.BH)) {
+            tma_load_3d(base + j * 8192, &mapQ, blk * p.dk + 64 * j, t0, bh, &bars.full[b]);
+            tma_load_3d(base + SM::QB + j * 8192, &mapK, blk * p.dk + 64 * j, t0, bh, &bars.full[b]);
+          }
         for (int j = 0; j < DVT / 64; ++j)
-          tma_load_3d(base + SM::QB + SM::KB + j * 8192, &mapV, blk * p.dv + v0 + 64 * j, t0, bh, &bars.full[b]);
+          if (tma_box_ok(p.err, BS_WALK_TMA, blk * p.dv + v0 + 64 * j, t0, 8, p.DHV, p.S, L, false))
+            tma_load_3d(base + SM::QB + SM::KB + j * 8192, &mapV, blk * p.dv + v0 + 64 * j, t0, bh, &bars.full[b]);
         n_issued = c + 1;
       }
       // gate quantities of chunk c into buffer gi (lane: tokens 2 lane, 2 lane + 1)
@@ -1069,7 +1111,9 @@ __global__ void __launch_bounds__(NTW, 1)
       if (lane == 0) mbar_arrive(&bars.gfull[gi]);
       if (c + 1 < nck) fetch_gates(c + 1);
     }
-    if (lane == 0 && !abort_flag && last_seg && !ret && tile == 0 && blk == 0 && p.m_out) p.m_out[bh] = mc;
+    if (lane == 0 && !abort_flag && last_seg && !ret && tile == 0 && blk == 0 && p.m_out &&
+        in_bounds(p.err, BS_WALK_FINAL, bh, p.BH))
+      p.m_out[bh] = mc;
   } else if (warp == 1) {
     // =============================================================== chain MMAs
     const uint64_t vw_mn = smem_desc_sw128(sm_u + SM::OVW, 8192, 1024);  // V o u, MN-major
@@ -1225,7 +1269,8 @@ __global__ void __launch_bounds__(NTW, 1)
         float r[32];
         tmem_ld32(tm + lane_off + TM_C + c0, r);
         tmem_wait_ld();
-        if (row >= 0) {
+        if (row >= 0 && in_bounds(p.err, BS_WALK_FINAL, ((long long)slice * p.dv + v0 + row) * p.dk + c0 + 31,
+                                  (long long)p.slices * p.dv * p.dk)) {
           float* dst = p.C_out + ((size_t)slice * p.dv + v0 + row) * p.dk + c0;
 #pragma unroll
           for (int j = 0; j < 32; j += 4)
@@ -1240,7 +1285,7 @@ __global__ void __launch_bounds__(NTW, 1)
     const bool first = gt == 0;
     const uint32_t ps_u = sm_u + SM::OP, hs_u = sm_u + SM::OH;
     const bool use_og = p.og != nullptr && !ret;
-    const float nbias_h = SN ? p.nbias[bh % p.NH] : 0.f;
+    const float nbias_h = SN && in_bounds(p.err, BS_WALK_BIAS, bh % p.NH, p.NH) ? p.nbias[bh % p.NH] : 0.f;
     for (int c = 0; c < nck; ++c) {
       const int b = c & 1, gi = c % NGB;
       const GateBuf G = gbuf(gi);
@@ -1394,19 +1439,25 @@ __global__ void __launch_bounds__(NTW, 1)
           for (int j = 0; j < 8; j += 2) {
             const int t = 8 * (j + (lane >> 4)) + (lane & 7);
             const uint32_t addr = hs_u + (d0 >> 6) * 8192 + t * 128 + ((((d0 & 63) >> 3) ^ (t & 7)) << 4);
-            stmatrix_x4_trans(addr, plo[j], phi[j], plo[j + 1], phi[j + 1]);
+            if (in_bounds(p.err, BS_WALK_H_STAGE, (long long)(addr - hs_u) + 15, (DVT / 64) * 8192))
+              stmatrix_x4_trans(addr, plo[j], phi[j], plo[j + 1], phi[j + 1]);
           }
         }
       }
       if (use_og) {  // h <- h o o_t on the staged tile
         named_bar(WG_OUT, 128);
-        apply_ogate<DVT>(hs_u, p.og + tok0 * p.DHV + (size_t)blk * p.dv + v0, p.DHV, Lc, gt);
+        // (the largest index it reads: its last row's last column)
+        if (in_bounds(p.err, BS_WALK_OGATE, (long long)(tok0 + Lc - 1) * p.DHV + blk * p.dv + v0 + DVT - 1,
+                      (long long)p.BH * p.S * p.DHV))
+          apply_ogate<DVT>(hs_u, p.og + tok0 * p.DHV + (size_t)blk * p.dv + v0, p.DHV, Lc, gt);
       }
       fence_proxy_async_smem();
       named_bar(WG_OUT, 128);
       if (first) {
         for (int j = 0; j < DVT / 64; ++j)
-          tma_store_3d(&mapH, sm + SM::OH + j * 8192, blk * p.dv + v0 + 64 * j, t0, bh);
+          if (tma_box_ok(p.err, BS_WALK_H_TMA, blk * p.dv + v0 + 64 * j, t0, 8, p.DHV, p.S, L, true) &&
+              in_bounds(p.err, BS_WALK_H_TMA, bh, p.BH))
+            tma_store_3d(&mapH, sm + SM::OH + j * 8192, blk * p.dv + v0 + 64 * j, t0, bh);
         bulk_commit();
         mbar_arrive(&bars.gempty[gi]);
       }
@@ -1534,9 +1585,13 @@ __global__ void __launch_bounds__(NTW, 1)
     }
     // final n after the last update, back in units of e^{m}
     if (SN) {
-      if (nck > 0 && last_seg && tile == 0 && blk == 0 && p.n_out && !abort_flag && nt == 0) p.n_out[bh] = fin * n_sc;
+      if (nck > 0 && last_seg && tile == 0 && blk == 0 && p.n_out && !abort_flag && nt == 0 &&
+          in_bounds(p.err, BS_WALK_FINAL, bh, p.BH))
+        p.n_out[bh] = fin * n_sc;
     } else if (nck > 0 && last_seg && !ret && tile == 0 && p.n_out && !abort_flag)
-      for (int col = nt; col < DK; col += 128) p.n_out[(size_t)slice * p.dk + col] = fin * nvec[col];
+      for (int col = nt; col < DK; col += 128)
+        if (in_bounds(p.err, BS_WALK_FINAL, (long long)slice * p.dk + col, (long long)p.slices * p.dk))
+          p.n_out[(size_t)slice * p.dk + col] = fin * nvec[col];
   }
 
   // Drain before TMEM is freed and the CTA exits: every MMA issued and every Q/K/V load issued
@@ -1770,7 +1825,10 @@ cudaError_t launch_tc(const WalkArgs& a, const TcPlan& pl, void* ws, cudaStream_
     *planes[i] = reinterpret_cast<float*>(w + off);
     off += ((size_t)BH * (i < 3 ? prm.sp : prm.ncp) * 4 + 255) / 256 * 256;
   }
-  cudaError_t e = cudaMemsetAsync(w, 0, 4, stream);
+  prm.BH = BH;
+  prm.slices = (int)slices;
+  // the error word and, for the bounds-checked build, its record (bytes 16..39)
+  cudaError_t e = cudaMemsetAsync(w, 0, 64, stream);
   if (e != cudaSuccess) return e;
 #define MLSTM_TC_DISPATCH(SNV, REVV)                                                                       \
   do {                                                                                                   \

@@ -3,6 +3,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include "bounds.cuh"
 #include "kernels.h"
 #include "mlstm.h"
 
@@ -316,7 +317,7 @@ mlstm_status_t check_bwd(const mlstm_fwd_params_t* p, FwdShape* s) {
 
 extern "C" {
 
-int mlstm_abi_version(void) { return (2 << 16) | 0; }
+int mlstm_abi_version(void) { return (2 << 16) | 1; }
 
 const char* mlstm_status_string(mlstm_status_t s) {
   switch (s) {
@@ -329,6 +330,7 @@ const char* mlstm_status_string(mlstm_status_t s) {
     case MLSTM_ERR_CUDA: return "CUDA runtime error at launch";
     case MLSTM_ERR_ALIAS: return "an output overlaps an input";
     case MLSTM_ERR_TIMEOUT: return "a bounded device-side wait ran out";
+    case MLSTM_ERR_BOUNDS: return "an access failed its bounds check and was skipped";
   }
   return "unknown status";
 }
@@ -391,7 +393,8 @@ static mlstm_status_t read_error_word(const FwdShape& s, const void* ws, cudaStr
   unsigned int word = 0;
   const char* base = static_cast<const char*>(ws) + fwd_layout(s).tc;
   if (cudaMemcpy(&word, base, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return MLSTM_ERR_CUDA;
-  return word == 0 ? MLSTM_OK : MLSTM_ERR_TIMEOUT;
+  // bits 0, 1: a wait ran out (segment summaries, walk); bit 2: a bounds check failed
+  return word == 0 ? MLSTM_OK : (word & 4u) ? MLSTM_ERR_BOUNDS : MLSTM_ERR_TIMEOUT;
 }
 
 mlstm_status_t mlstm_fwd_chunkwise_status(const mlstm_fwd_params_t* p, const void* workspace,
@@ -401,6 +404,27 @@ mlstm_status_t mlstm_fwd_chunkwise_status(const mlstm_fwd_params_t* p, const voi
   if (st != MLSTM_OK) return st;
   if (s.tc && s.BH > 0 && s.S > 0 && !workspace) return MLSTM_ERR_NULL;
   return read_error_word(s, workspace, (cudaStream_t)stream);
+}
+
+int mlstm_bounds_checked(void) { return mlstm::kBoundsChecked ? 1 : 0; }
+
+mlstm_status_t mlstm_fwd_chunkwise_bounds_record(const mlstm_fwd_params_t* p, const void* workspace,
+                                                 mlstm_stream_t stream, int* site, long long* index,
+                                                 long long* extent) {
+  FwdShape s;
+  mlstm_status_t st = check_fwd(p, &s);
+  if (st != MLSTM_OK) return st;
+  if (s.tc && s.BH > 0 && s.S > 0 && !workspace) return MLSTM_ERR_NULL;
+  mlstm::BoundsRecord r = {};
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MLSTM_ERR_CUDA;
+  if (mlstm::kBoundsChecked && s.tc && s.BH > 0 && s.S > 0) {
+    const char* base = static_cast<const char*>(workspace) + fwd_layout(s).tc + 16;
+    if (cudaMemcpy(&r, base, sizeof(r), cudaMemcpyDeviceToHost) != cudaSuccess) return MLSTM_ERR_CUDA;
+  }
+  if (site) *site = r.count ? r.site : 0;
+  if (index) *index = r.count ? r.index : 0;
+  if (extent) *extent = r.count ? r.extent : 0;
+  return MLSTM_OK;
 }
 
 // Workspace of the reversed-sequence pass: the forward's, then reversed copies of the

@@ -10,7 +10,8 @@
 //                       to both q and k.  HBM-bound: one read and one write of q and k.
 // gn_gate_kernel        y = (h - mean) / sqrt(var + eps) * w + b, times silu(g), one group =
 //                       one (batch, head, token) row of DHV values, two passes over values
-//                       held in registers.  HBM-bound: read h and g, write y.
+//                       held in registers; narrow rows take four rows per thread with every
+//                       load issued up front.  HBM-bound: read h and g, write y.
 //
 // Both take tensors laid out [B, NH, S, D] with D contiguous, fp32 or bf16, 16-byte vectors.
 #include <cuda_bf16.h>
@@ -73,21 +74,12 @@ __global__ void __launch_bounds__(ROT_THREADS) theta_rotate_kernel(const T* q, c
   const int b = blockIdx.y;
   const long long t = (long long)blockIdx.x * tpc + tl;
   if (tl >= tpc || t >= S) return;
-  const double pos = (double)((pos0 ? pos0[b] : 0LL) + t);
-  const double l2b = log2((double)base);
   float cs[PP], sn[PP];
-#pragma unroll
-  for (int u = 0; u < PP; ++u) {
-    const int j = c * PP + u;
-    const double theta = exp2(-(2.0 * j / D) * l2b);
-    double s_, c_;
-    sincos(pos * theta, &s_, &c_);
-    cs[u] = (float)c_;
-    sn[u] = (float)s_;
-  }
   const size_t head_stride = (size_t)S * D;
   const size_t base_off = ((size_t)b * NH * S + t) * D + (size_t)c * V::N;
   for (int h0 = 0; h0 < NH; h0 += ROT_HEADS) {
+    // the loads of this round are issued first; the first round's angles are computed while
+    // they are in flight
     uint4 xq[ROT_HEADS], xk[ROT_HEADS];
 #pragma unroll
     for (int u = 0; u < ROT_HEADS; ++u) {
@@ -95,6 +87,22 @@ __global__ void __launch_bounds__(ROT_THREADS) theta_rotate_kernel(const T* q, c
         const size_t off = base_off + (size_t)(h0 + u) * head_stride;
         xq[u] = *reinterpret_cast<const uint4*>(q + off);
         xk[u] = *reinterpret_cast<const uint4*>(k + off);
+      }
+    }
+    if (h0 == 0) {
+      // angle p theta_j in double (positions in the millions keep it exact to far below fp32
+      // resolution), reduced to [-pi, pi] by the nearest multiple of 2 pi in double, then
+      // cos / sin in fp32 on the reduced angle; theta_{j+1} = theta_j base^{-2/D}
+      const double pos = (double)((pos0 ? pos0[b] : 0LL) + t);
+      const double l2b = log2((double)base);
+      double theta = exp2(-(2.0 * (c * PP) / D) * l2b);
+      const double ratio = exp2(-(2.0 / D) * l2b);
+#pragma unroll
+      for (int u = 0; u < PP; ++u) {
+        const double x = pos * theta;
+        const double turns = rint(x * 0.15915494309189535);  // x / (2 pi)
+        sincosf((float)fma(-turns, 6.283185307179586, x), &sn[u], &cs[u]);
+        theta *= ratio;
       }
     }
 #pragma unroll
@@ -145,84 +153,108 @@ __device__ __forceinline__ float row_sum(float v, float* red) {
   }
 }
 
-// one row of DHV = R * Vec::N values per R threads; GN_THREADS / R rows per CTA
-template <typename T, int R>
-__global__ void __launch_bounds__(GN_THREADS) gn_gate_kernel(const T* h, const T* g, const float* w, const float* bb,
-                                                            float eps, T* y, long long rows, int NH, int S) {
+// CTA = a block of token rows of one (batch, head); a row of DHV = R * NV * Vec::N values is
+// spread over R threads with NV 16-byte vectors each, and a thread takes RT rows GN_THREADS / R
+// apart.  The thread's channels are the same for all its rows, so their weight and bias are
+// loaded once; every h and g load of the thread is issued before the first reduction.
+template <typename T, int R, int NV, int RT>
+__global__ void __launch_bounds__(GN_THREADS, 3) gn_gate_kernel(const T* h, const T* g, const float* w, const float* bb,
+                                                            float eps, T* y, int NH, int S, int nblk) {
   using V = Vec<T>;
-  constexpr int RPC = GN_THREADS / R, DHV = R * V::N;
+  constexpr int RPC = GN_THREADS / R, E = NV * V::N, DHV = R * E;
   __shared__ float red[GN_THREADS / 32];
   const int rl = threadIdx.x / R, c = threadIdx.x % R;
-  const long long row = (long long)blockIdx.x * RPC + rl;
-  const bool act = row < rows;
-  const size_t off = (size_t)row * DHV + (size_t)c * V::N;
-  const int ch = (int)((row / S) % NH) * DHV + c * V::N;  // this thread's first channel
-  // every load this thread needs is issued here, before the reductions
-  float x[V::N], gv[V::N], wv[V::N], bv[V::N];
-  uint4 hraw = make_uint4(0, 0, 0, 0), graw = make_uint4(0, 0, 0, 0);
-  if (act) {
-    hraw = *reinterpret_cast<const uint4*>(h + off);
-    if (g) graw = *reinterpret_cast<const uint4*>(g + off);
+  const int bh = blockIdx.x / nblk, tb = blockIdx.x - bh * nblk;
+  const int ch = (bh % NH) * DHV + c * E;  // this thread's first channel
+  float wv[E], bv[E];
 #pragma unroll
-    for (int e = 0; e < V::N; e += 4) {
-      const float4 w4 = w ? *reinterpret_cast<const float4*>(w + ch + e) : make_float4(1.f, 1.f, 1.f, 1.f);
-      const float4 b4 = bb ? *reinterpret_cast<const float4*>(bb + ch + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-      wv[e] = w4.x, wv[e + 1] = w4.y, wv[e + 2] = w4.z, wv[e + 3] = w4.w;
-      bv[e] = b4.x, bv[e + 1] = b4.y, bv[e + 2] = b4.z, bv[e + 3] = b4.w;
+  for (int e = 0; e < E; e += 4) {
+    const float4 w4 = w ? *reinterpret_cast<const float4*>(w + ch + e) : make_float4(1.f, 1.f, 1.f, 1.f);
+    const float4 b4 = bb ? *reinterpret_cast<const float4*>(bb + ch + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+    wv[e] = w4.x, wv[e + 1] = w4.y, wv[e + 2] = w4.z, wv[e + 3] = w4.w;
+    bv[e] = b4.x, bv[e + 1] = b4.y, bv[e + 2] = b4.z, bv[e + 3] = b4.w;
+  }
+  uint4 hraw[RT][NV], graw[RT][NV];
+  size_t off[RT];
+  bool act[RT];
+#pragma unroll
+  for (int i = 0; i < RT; ++i) {
+    const int t = (tb * RT + i) * RPC + rl;  // token of the row
+    act[i] = t < S;
+    off[i] = ((size_t)bh * S + t) * DHV + (size_t)c * E;
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      hraw[i][v] = graw[i][v] = make_uint4(0, 0, 0, 0);
+      if (act[i]) {
+        hraw[i][v] = *reinterpret_cast<const uint4*>(h + off[i] + v * V::N);
+        if (g) graw[i][v] = *reinterpret_cast<const uint4*>(g + off[i] + v * V::N);
+      }
     }
   }
-  V::unpack(hraw, x);
-  V::unpack(graw, gv);
-  float s = 0.f;
 #pragma unroll
-  for (int e = 0; e < V::N; ++e) s += x[e];
-  const float mean = row_sum<R>(s, red) * (1.f / DHV);
-  float d2 = 0.f;
-  if (act) {
+  for (int i = 0; i < RT; ++i) {
+    float x[E];
 #pragma unroll
-    for (int e = 0; e < V::N; ++e) d2 = fmaf(x[e] - mean, x[e] - mean, d2);
+    for (int v = 0; v < NV; ++v) V::unpack(hraw[i][v], x + v * V::N);
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) s += x[e];
+    const float mean = row_sum<R>(s, red) * (1.f / DHV);
+    float d2 = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) d2 = fmaf(x[e] - mean, x[e] - mean, d2);
+    const float var = row_sum<R>(d2, red) * (1.f / DHV);
+    if (act[i]) {
+      const float rstd = rsqrtf(var + eps);
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        float gv[V::N];
+        V::unpack(graw[i][v], gv);
+#pragma unroll
+        for (int e = 0; e < V::N; ++e) {
+          const int k = v * V::N + e;
+          float o = fmaf((x[k] - mean) * rstd, wv[k], bv[k]);
+          // silu(g) = g / (1 + e^{-g}); the fast exponential and divide are accurate to a few
+          // fp32 ulps, far inside the bf16 rounding of the output (fp32 outputs keep expf)
+          if (g) o *= V::N == 8 ? __fdividef(gv[e], 1.f + __expf(-gv[e])) : gv[e] / (1.f + expf(-gv[e]));
+          x[k] = o;
+        }
+        *reinterpret_cast<uint4*>(y + off[i] + v * V::N) = V::pack(x + v * V::N);
+      }
+    }
   }
-  const float var = row_sum<R>(d2, red) * (1.f / DHV);
-  if (!act) return;
-  const float rstd = 1.f / sqrtf(var + eps);
-#pragma unroll
-  for (int e = 0; e < V::N; ++e) {
-    float o = fmaf((x[e] - mean) * rstd, wv[e], bv[e]);
-    if (g) o *= gv[e] / (1.f + expf(-gv[e]));
-    x[e] = o;
-  }
-  *reinterpret_cast<uint4*>(y + off) = V::pack(x);
 }
 
 template <typename T>
 cudaError_t launch_gn_t(long long rows, int NH, int S, int DHV, const void* h, const void* g, const float* w,
                         const float* b, float eps, void* y, cudaStream_t stream) {
-  const int R = DHV / Vec<T>::N;
-  const long long rpc = R >= GN_THREADS ? 1 : GN_THREADS / R;
-  const long long blocks = (rows + rpc - 1) / rpc;
-  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const int n = DHV / Vec<T>::N;           // 16-byte vectors per row
+  const int nv = n >= 2 ? 2 : 1, R = n / nv;  // two vectors per thread where the row has them
+  const int rt = R <= 32 ? 2 : 1;          // rows per thread while a row's reduction stays in a warp
+  const long long rpc = (long long)rt * (GN_THREADS / R);
+  const long long nblk = ((long long)S + rpc - 1) / rpc, BH = rows / S;
+  if (nblk * BH > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const unsigned blocks = (unsigned)(nblk * BH);
   const T* hp = static_cast<const T*>(h);
   const T* gp = static_cast<const T*>(g);
   T* yp = static_cast<T*>(y);
-#define GN_CASE(RR)                                                                              \
-  case RR:                                                                                       \
-    gn_gate_kernel<T, RR><<<(unsigned)blocks, GN_THREADS, 0, stream>>>(hp, gp, w, b, eps, yp, rows, NH, S); \
-    break;
-  switch (R) {
-    GN_CASE(1)
-    GN_CASE(2)
-    GN_CASE(4)
-    GN_CASE(8)
-    GN_CASE(16)
-    GN_CASE(32)
-    GN_CASE(64)
-    GN_CASE(128)
-    GN_CASE(256)
-    default:
-      return cudaErrorInvalidValue;
+#define GN_CASE(RR, NVV)                                                                                  \
+  if (R == RR && nv == NVV) {                                                                             \
+    gn_gate_kernel<T, RR, NVV, (RR <= 32 ? 2 : 1)><<<blocks, GN_THREADS, 0, stream>>>(hp, gp, w, b, eps, yp, NH, S, \
+                                                                                      (int)nblk);         \
+    return cudaGetLastError();                                                                            \
   }
+  GN_CASE(1, 1)
+  GN_CASE(1, 2)
+  GN_CASE(2, 2)
+  GN_CASE(4, 2)
+  GN_CASE(8, 2)
+  GN_CASE(16, 2)
+  GN_CASE(32, 2)
+  GN_CASE(64, 2)
+  GN_CASE(128, 2)
 #undef GN_CASE
-  return cudaGetLastError();
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
@@ -235,8 +267,8 @@ bool theta_rotate_supported(int D, int dtype) {
 bool gn_gate_supported(int DHV, int dtype) {
   const int n = dtype == 0 ? 4 : 8;
   if (DHV <= 0 || DHV % n) return false;
-  const int R = DHV / n;
-  return R <= GN_THREADS && (R & (R - 1)) == 0;
+  const int v = DHV / n;  // 16-byte vectors per row: 1 .. 256, a power of two
+  return v <= GN_THREADS && (v & (v - 1)) == 0;
 }
 
 cudaError_t launch_theta_rotate(int B, int NH, int S, int D, int dtype, const void* q, const void* k, void* qo,

@@ -8,6 +8,7 @@ is present, these functions raise.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -15,6 +16,8 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmlstm.so")
+# the bounds-checked debug build of the same library (include/mlstm.h, mlstm_bounds_checked)
+LIB_CHECKED_PATH = os.path.join(_PKG, "libmlstm_checked.so")
 
 MLSTM_F32, MLSTM_BF16 = 0, 1
 _DTYPES = {torch.float32: MLSTM_F32, torch.bfloat16: MLSTM_BF16}
@@ -51,68 +54,95 @@ class MlstmError(RuntimeError):
         self.status = status
 
 
-_lib = None
+_libs = {}
+_use_checked = False
 
 
 def lib():
-    """The loaded libmlstm.so (raises if it has not been built)."""
-    global _lib
-    if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
-                               "`python -m linear_recurrent_token_b200.build` (nvcc, sm_100a)")
-        L = ctypes.CDLL(LIB_PATH)
-        P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
-        L.mlstm_fwd_chunkwise_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
-        L.mlstm_fwd_chunkwise_workspace_size.restype = Z
-        L.mlstm_fwd_chunkwise_plan.argtypes = [ctypes.POINTER(FwdParams), ctypes.POINTER(FwdPlan)]
-        L.mlstm_fwd_chunkwise_plan.restype = I
-        L.mlstm_fwd_chunkwise.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 14 + [Z, P]
-        L.mlstm_fwd_chunkwise.restype = I
-        L.mlstm_fwd_chunkwise_timed.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 14 + [Z, P, P, P]
-        L.mlstm_fwd_chunkwise_timed.restype = I
-        L.mlstm_fwd_chunkwise_noalloc.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 13 + [P]
-        L.mlstm_fwd_chunkwise_noalloc.restype = I
-        L.mlstm_fwd_chunkwise_status.argtypes = [ctypes.POINTER(FwdParams), P, P]
-        L.mlstm_fwd_chunkwise_status.restype = I
-        L.mlstm_fwd_chunkwise_noalloc_status.argtypes = [ctypes.POINTER(FwdParams), P]
-        L.mlstm_fwd_chunkwise_noalloc_status.restype = I
-        L.mlstm_noalloc_scratch_bytes.argtypes = []
-        L.mlstm_noalloc_scratch_bytes.restype = Z
-        L.mlstm_fwd_chunkwise_reversed_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
-        L.mlstm_fwd_chunkwise_reversed_workspace_size.restype = Z
-        L.mlstm_fwd_chunkwise_reversed.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 14 + [Z, P]
-        L.mlstm_fwd_chunkwise_reversed.restype = I
-        L.mlstm_fwd_chunkwise_scalar_normaliser_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
-        L.mlstm_fwd_chunkwise_scalar_normaliser_workspace_size.restype = Z
-        L.mlstm_fwd_chunkwise_scalar_normaliser.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 15 + [Z, P]
-        L.mlstm_fwd_chunkwise_scalar_normaliser.restype = I
-        F = ctypes.c_float
-        L.mlstm_theta_rotate.argtypes = [ctypes.POINTER(FwdParams), P, P, P, F, P, P, P]
-        L.mlstm_theta_rotate.restype = I
-        L.mlstm_group_norm_gate.argtypes = [ctypes.POINTER(FwdParams), P, P, P, P, F, P, P]
-        L.mlstm_group_norm_gate.restype = I
-        L.mlstm_fwd_chunkwise_msr_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
-        L.mlstm_fwd_chunkwise_msr_workspace_size.restype = Z
-        L.mlstm_fwd_chunkwise_msr.argtypes = [ctypes.POINTER(FwdParams), P, P, P, P, P, P, F, P, P, P, F, P, P, P,
-                                              P, P, P, P, P, Z, P]
-        L.mlstm_fwd_chunkwise_msr.restype = I
-        L.mlstm_gdn2_workspace_size.argtypes = [ctypes.POINTER(Gdn2Params)]
-        L.mlstm_gdn2_workspace_size.restype = Z
-        L.mlstm_gdn2_fwd.argtypes = [ctypes.POINTER(Gdn2Params)] + [P] * 10 + [Z, P]
-        L.mlstm_gdn2_fwd.restype = I
-        L.mlstm_bwd_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
-        L.mlstm_bwd_workspace_size.restype = Z
-        L.mlstm_bwd.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 22 + [Z, P]
-        L.mlstm_bwd.restype = I
-        L.mlstm_step.argtypes = [ctypes.POINTER(StepParams)] + [P] * 10 + [P]
-        L.mlstm_step.restype = I
-        L.mlstm_status_string.argtypes = [I]
-        L.mlstm_status_string.restype = ctypes.c_char_p
-        L.mlstm_abi_version.argtypes = []
-        L.mlstm_abi_version.restype = I
-        _lib = L
-    return _lib
+    """The loaded libmlstm.so, or libmlstm_checked.so inside `with bounds_checked():` (raises if
+    it has not been built)."""
+    path = LIB_CHECKED_PATH if _use_checked else LIB_PATH
+    if path not in _libs:
+        _libs[path] = _load(path)
+    return _libs[path]
+
+
+@contextlib.contextmanager
+def bounds_checked():
+    """Every call made inside the block goes to libmlstm_checked.so, the bounds-checked debug
+    build (its status calls return 9 = MLSTM_ERR_BOUNDS when a check failed; bounds_record
+    says where).  Not thread-safe: it switches the library for the whole module."""
+    global _use_checked
+    prev = _use_checked
+    _use_checked = True
+    try:
+        yield lib()
+    finally:
+        _use_checked = prev
+
+
+def _load(path):
+    """Loads one build of the library and declares the C signatures."""
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m linear_recurrent_token_b200.build` (nvcc, sm_100a)")
+    L = ctypes.CDLL(path)
+    P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.mlstm_fwd_chunkwise_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
+    L.mlstm_fwd_chunkwise_workspace_size.restype = Z
+    L.mlstm_fwd_chunkwise_plan.argtypes = [ctypes.POINTER(FwdParams), ctypes.POINTER(FwdPlan)]
+    L.mlstm_fwd_chunkwise_plan.restype = I
+    L.mlstm_fwd_chunkwise.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 14 + [Z, P]
+    L.mlstm_fwd_chunkwise.restype = I
+    L.mlstm_fwd_chunkwise_timed.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 14 + [Z, P, P, P]
+    L.mlstm_fwd_chunkwise_timed.restype = I
+    L.mlstm_fwd_chunkwise_noalloc.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 13 + [P]
+    L.mlstm_fwd_chunkwise_noalloc.restype = I
+    L.mlstm_fwd_chunkwise_status.argtypes = [ctypes.POINTER(FwdParams), P, P]
+    L.mlstm_fwd_chunkwise_status.restype = I
+    L.mlstm_fwd_chunkwise_noalloc_status.argtypes = [ctypes.POINTER(FwdParams), P]
+    L.mlstm_fwd_chunkwise_noalloc_status.restype = I
+    L.mlstm_bounds_checked.argtypes = []
+    L.mlstm_bounds_checked.restype = I
+    LL = ctypes.c_longlong
+    L.mlstm_fwd_chunkwise_bounds_record.argtypes = [ctypes.POINTER(FwdParams), P, P, ctypes.POINTER(I),
+                                                    ctypes.POINTER(LL), ctypes.POINTER(LL)]
+    L.mlstm_fwd_chunkwise_bounds_record.restype = I
+    L.mlstm_noalloc_scratch_bytes.argtypes = []
+    L.mlstm_noalloc_scratch_bytes.restype = Z
+    L.mlstm_fwd_chunkwise_reversed_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
+    L.mlstm_fwd_chunkwise_reversed_workspace_size.restype = Z
+    L.mlstm_fwd_chunkwise_reversed.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 14 + [Z, P]
+    L.mlstm_fwd_chunkwise_reversed.restype = I
+    L.mlstm_fwd_chunkwise_scalar_normaliser_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
+    L.mlstm_fwd_chunkwise_scalar_normaliser_workspace_size.restype = Z
+    L.mlstm_fwd_chunkwise_scalar_normaliser.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 15 + [Z, P]
+    L.mlstm_fwd_chunkwise_scalar_normaliser.restype = I
+    F = ctypes.c_float
+    L.mlstm_theta_rotate.argtypes = [ctypes.POINTER(FwdParams), P, P, P, F, P, P, P]
+    L.mlstm_theta_rotate.restype = I
+    L.mlstm_group_norm_gate.argtypes = [ctypes.POINTER(FwdParams), P, P, P, P, F, P, P]
+    L.mlstm_group_norm_gate.restype = I
+    L.mlstm_fwd_chunkwise_msr_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
+    L.mlstm_fwd_chunkwise_msr_workspace_size.restype = Z
+    L.mlstm_fwd_chunkwise_msr.argtypes = [ctypes.POINTER(FwdParams), P, P, P, P, P, P, F, P, P, P, F, P, P, P,
+                                          P, P, P, P, P, Z, P]
+    L.mlstm_fwd_chunkwise_msr.restype = I
+    L.mlstm_gdn2_workspace_size.argtypes = [ctypes.POINTER(Gdn2Params)]
+    L.mlstm_gdn2_workspace_size.restype = Z
+    L.mlstm_gdn2_fwd.argtypes = [ctypes.POINTER(Gdn2Params)] + [P] * 10 + [Z, P]
+    L.mlstm_gdn2_fwd.restype = I
+    L.mlstm_bwd_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
+    L.mlstm_bwd_workspace_size.restype = Z
+    L.mlstm_bwd.argtypes = [ctypes.POINTER(FwdParams)] + [P] * 22 + [Z, P]
+    L.mlstm_bwd.restype = I
+    L.mlstm_step.argtypes = [ctypes.POINTER(StepParams)] + [P] * 10 + [P]
+    L.mlstm_step.restype = I
+    L.mlstm_status_string.argtypes = [I]
+    L.mlstm_status_string.restype = ctypes.c_char_p
+    L.mlstm_abi_version.argtypes = []
+    L.mlstm_abi_version.restype = I
+    return L
 
 
 def status_string(status: int) -> str:
@@ -151,10 +181,22 @@ def fwd_status(params: FwdParams, workspace=None, stream=None, noalloc: bool = F
     """Outcome of the bounded device-side waits of the last prefill with these params and this
     workspace (mlstm_fwd_chunkwise_status; noalloc=True: of the last mlstm_fwd_chunkwise_noalloc,
     mlstm_fwd_chunkwise_noalloc_status).  Synchronises the stream.  Returns the status code:
-    0 = ok, 8 = a wait ran out (MLSTM_ERR_TIMEOUT)."""
+    0 = ok, 8 = a wait ran out (MLSTM_ERR_TIMEOUT), 9 = a check of the bounds-checked build
+    failed (MLSTM_ERR_BOUNDS)."""
     if noalloc:
         return int(lib().mlstm_fwd_chunkwise_noalloc_status(ctypes.byref(params), _stream_ptr(stream)))
     return int(lib().mlstm_fwd_chunkwise_status(ctypes.byref(params), _ptr(workspace), _stream_ptr(stream)))
+
+
+def bounds_record(params: FwdParams, workspace, stream=None):
+    """First failed check of the last prefill with this workspace in the bounds-checked build
+    (mlstm_fwd_chunkwise_bounds_record): (site, index, extent), site 0 when none failed."""
+    site, index, extent = ctypes.c_int(0), ctypes.c_longlong(0), ctypes.c_longlong(0)
+    st = lib().mlstm_fwd_chunkwise_bounds_record(ctypes.byref(params), _ptr(workspace), _stream_ptr(stream),
+                                                 ctypes.byref(site), ctypes.byref(index), ctypes.byref(extent))
+    if st != 0:
+        raise MlstmError(st, "mlstm_fwd_chunkwise_bounds_record")
+    return site.value, index.value, extent.value
 
 
 def workspace_size(params: FwdParams) -> int:

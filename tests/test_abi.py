@@ -30,10 +30,28 @@ def test_library_builds_and_exports_every_declared_symbol():
         assert hasattr(lib, name), name
 
 
+def test_bounds_checked_build_loads_and_exports_every_declared_symbol():
+    build.build()
+    assert mlstm.lib().mlstm_bounds_checked() == 0
+    with mlstm.bounds_checked() as lib:
+        assert mlstm.lib() is lib and lib.mlstm_bounds_checked() == 1
+        for name in declared_functions():
+            assert hasattr(lib, name), name
+        assert lib.mlstm_abi_version() == mlstm_default_abi()
+        # argument validation is the same library code
+        assert lib.mlstm_fwd_chunkwise_status(None, ctypes.c_void_p(G_), ctypes.c_void_p(0)) == 1
+    assert mlstm.lib().mlstm_bounds_checked() == 0
+
+
+def mlstm_default_abi():
+    return mlstm.lib().mlstm_abi_version()
+
+
 def test_status_strings_and_version():
-    for code in range(9):
+    for code in range(10):
         assert mlstm.status_string(code) != "unknown status"
     assert mlstm.status_string(8) == "a bounded device-side wait ran out"
+    assert mlstm.status_string(9) == "an access failed its bounds check and was skipped"
     assert mlstm.status_string(99) == "unknown status"
     assert mlstm.lib().mlstm_abi_version() >> 16 == 2
 
@@ -55,6 +73,11 @@ def test_status_calls_validate_before_touching_the_device():
     assert mlstm.plan(tc)["tensor_core"] == 1
     assert L.mlstm_fwd_chunkwise_status(ctypes.byref(tc), None, P(0)) == 1  # its error word lives there
     assert L.mlstm_fwd_chunkwise_noalloc_status(None, P(0)) == 1
+    I, LL = ctypes.c_int(5), ctypes.c_longlong(5)
+    assert L.mlstm_fwd_chunkwise_bounds_record(None, P(G_), P(0), None, None, None) == 1
+    assert L.mlstm_fwd_chunkwise_bounds_record(ctypes.byref(params(B=-1)), P(G_), P(0), ctypes.byref(I),
+                                               ctypes.byref(LL), None) == 2
+    assert L.mlstm_fwd_chunkwise_bounds_record(ctypes.byref(tc), None, P(0), None, None, None) == 1
 
 
 def fwd(p, q=A, k=B_, v=C_, ig=D_, fg=E_, og=None, C0=None, n0=None, m0=None, h=F_, C=None, n=None, m=None,
