@@ -15,6 +15,7 @@ sample of the same workload (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import contextlib
 import json
 import os
 import statistics
@@ -153,6 +154,19 @@ def dist_barrier(world: int):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
+
+
+# ------------------------------------------------------------------ NVTX
+@contextlib.contextmanager
+def nvtx(name):
+    """An NVTX range around a bench region (named in a timeline profiler's view)."""
+    import torch
+
+    torch.cuda.nvtx.range_push(name)
+    try:
+        yield
+    finally:
+        torch.cuda.nvtx.range_pop()
 
 
 # ------------------------------------------------------------------ L2 flush
@@ -308,20 +322,22 @@ def run_chunkwise(w, steps, warmup, flush_bytes, clocks):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     clocks.mark(True)
     t_wall = time.perf_counter()
-    for e in ev:
-        flush(float(len(ev)))
-        e[0].record(stream)
-        one()
-        e[1].record(stream)
-    torch.cuda.synchronize()
+    with nvtx(f"prefill steps: {w.name}"):
+        for e in ev:
+            flush(float(len(ev)))
+            e[0].record(stream)
+            one()
+            e[1].record(stream)
+        torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall
     # the dominant kernel alone: the same calls with events recorded by the library around it
     evk = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(max(3, steps // 2))]
-    for e in evk:
-        flush(2.0)
-        one((e[0], e[1]))
-    torch.cuda.synchronize()
+    with nvtx(f"prefill, walk timed alone: {w.name}"):
+        for e in evk:
+            flush(2.0)
+            one((e[0], e[1]))
+        torch.cuda.synchronize()
     clocks.mark(False)
     step_ms = [a.elapsed_time(b) for a, b in ev]
     main_ms = [c.elapsed_time(d) for c, d in evk]
@@ -397,11 +413,12 @@ def run_chunkwise_e2e(w, steps, tensors):
     pipeline(2)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s_in)
-    pipeline(steps)
-    s_in.wait_stream(s_out)
-    e1.record(s_in)
-    torch.cuda.synchronize()
+    with nvtx(f"prefill end to end, host buffers: {w.name}"):
+        e0.record(s_in)
+        pipeline(steps)
+        s_in.wait_stream(s_out)
+        e1.record(s_in)
+        torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
     h2d = sum(t.numel() * t.element_size() for t in ((hq, hk, hv) + (() if w.retention else (hig, hfg))))
     d2h = sum(t.numel() * t.element_size() for t in ((oh, oC) + (() if w.retention else (on_, om))))
@@ -431,12 +448,13 @@ def run_decode(w, steps, warmup, clocks):
     # state exceeds L2, so no flush is needed between steps)
     e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks.mark(True)
-    e_a.record(stream)
-    for i in range(steps):
-        t = (warmup + i) % T
-        mlstm.step(q[t], k[t], v[t], ig[t], fg[t], C, n, m, h=h[t], stream=stream)
-    e_b.record(stream)
-    torch.cuda.synchronize()
+    with nvtx(f"decode steps: {w.name}"):
+        e_a.record(stream)
+        for i in range(steps):
+            t = (warmup + i) % T
+            mlstm.step(q[t], k[t], v[t], ig[t], fg[t], C, n, m, h=h[t], stream=stream)
+        e_b.record(stream)
+        torch.cuda.synchronize()
     clocks.mark(False)
     step_ms = [e_a.elapsed_time(e_b) / steps] * steps
 
@@ -486,11 +504,12 @@ def run_decode(w, steps, warmup, clocks):
     pipeline(2)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s_in)
-    pipeline(steps)
-    s_in.wait_stream(s_out)
-    e1.record(s_in)
-    torch.cuda.synchronize()
+    with nvtx(f"decode end to end, host buffers: {w.name}"):
+        e0.record(s_in)
+        pipeline(steps)
+        s_in.wait_stream(s_out)
+        e1.record(s_in)
+        torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / steps
     h2d = sum(x[0].numel() * x.element_size() for x in (hq, hk, hv, hig, hfg))
     d2h = oh.numel() * oh.element_size()
@@ -536,10 +555,11 @@ def run_backward(w, steps, warmup, flush_bytes, clocks):
     for _ in range(steps):
         flush(1.0)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        mlstm.bwd(q, k, v, dh, ig, fg, num_blocks=w.num_blocks, retention=w.retention, workspace=ws)
-        b.record()
-        torch.cuda.synchronize()
+        with nvtx(f"backward step: {w.name}"):
+            a.record()
+            mlstm.bwd(q, k, v, dh, ig, fg, num_blocks=w.num_blocks, retention=w.retention, workspace=ws)
+            b.record()
+            torch.cuda.synchronize()
         ms.append(a.elapsed_time(b))
     clocks.mark(False)
     return ms
@@ -569,9 +589,10 @@ def run_reversed(w, steps, warmup, flush_bytes):
     for _ in range(steps):
         flush(1.0)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        call()
-        b.record()
+        with nvtx(f"reversed step: {w.name}"):
+            a.record()
+            call()
+            b.record()
         torch.cuda.synchronize()
         ms.append(a.elapsed_time(b))
     return ms
@@ -602,9 +623,10 @@ def run_scalar_normaliser(w, steps, warmup, flush_bytes):
     for _ in range(steps):
         flush(1.0)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        call()
-        b.record()
+        with nvtx(f"scalar-normaliser step: {w.name}"):
+            a.record()
+            call()
+            b.record()
         torch.cuda.synchronize()
         ms.append(a.elapsed_time(b))
     return ms
@@ -653,9 +675,10 @@ def run_msr(w, steps, warmup, flush_bytes, hbm_peak):
         for _ in range(steps):
             flush(1.0)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            call()
-            b.record()
+            with nvtx(f"retention block, {name}: {w.name}"):
+                a.record()
+                call()
+                b.record()
             torch.cuda.synchronize()
             ms.append(a.elapsed_time(b))
         out[name] = statistics.median(ms)
@@ -699,9 +722,10 @@ def run_gdn2(steps, warmup, flush_bytes, peaks, sm_mhz):
         for _ in range(steps):
             flush(1.0)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            call()
-            b.record()
+            with nvtx("GDN-2 step"):
+                a.record()
+                call()
+                b.record()
             torch.cuda.synchronize()
             ms.append(a.elapsed_time(b))
         return statistics.median(ms)
