@@ -704,6 +704,20 @@ def gdn2_flops(B, H, T, K, V):
     return B * H * T * 9 * K * V
 
 
+def gdn2_chunk_on_tensor_cores(wl):
+    """Whether mlstm_gdn2_fwd runs the chunk mode on the tensor-core kernels for this workload
+    (the library's rule: bf16, chunk 64, K 128, V 64 or 128)."""
+    return wl.dtype == "bf16" and wl.chunk == 64 and wl.K == 128 and wl.V in (64, 128) and wl.T > 0
+
+
+def gdn2_min_bytes(wl):
+    """Bytes a GDN-2 prefill must move: q, k, v (dtype), g, b, w (fp32) read once, o written,
+    the fp32 state read and written."""
+    esz = 2 if wl.dtype == "bf16" else 4
+    tok = wl.B * wl.H * wl.T
+    return tok * (2 * wl.K * esz + wl.V * esz + 2 * wl.K * 4 + wl.V * 4 + wl.V * esz) + 2 * wl.B * wl.H * wl.K * wl.V * 4
+
+
 def run_gdn2(steps, warmup, flush_bytes, peaks, sm_mhz):
     """Gated DeltaNet-2: the prefill workload in both modes (fused recurrent, chunk) and the
     decode workload (one token per sequence, state in place), inputs resident, L2 flushed
@@ -746,11 +760,23 @@ def run_gdn2(steps, warmup, flush_bytes, peaks, sm_mhz):
             for mode in ("recurrent", "chunk"):
                 ms = timed(lambda: mlstm.gdn2_fwd(q, k, v, g, b, w, S0, mode=mode, chunk=wl.chunk, o=o, S_out=S_out))
                 tf = flops / (ms * 1e-3) / 1e12
+                if mode == "chunk" and gdn2_chunk_on_tensor_cores(wl):
+                    # the whole call against HBM: every input read once, o written, the state
+                    # read and written (the per-chunk slots between the two kernels are not
+                    # algorithmic bytes); its flops against the bf16 tensor peak beside it
+                    nbytes = gdn2_min_bytes(wl)
+                    gbs = nbytes / (ms * 1e-3) / 1e9
+                    roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": gbs / peaks["hbm_gbs"], "traffic": None, "bytes_per_launch": nbytes,
+                            "tensor_frac": tf / peaks["bf16_tflops"], "flops_per_launch": flops,
+                            "kernel": "gdn2_tc_prep_kernel (warp-level bf16 MMAs) + gdn2_tc_scan_kernel (tcgen05)"}
+                else:
+                    roof = {"bound": "alu", "achieved": tf, "peak": fp32_peak, "unit": "TFLOP/s",
+                            "frac": tf / fp32_peak, "traffic": None,
+                            "kernel": "gdn2_%s_kernel (fp32 SIMT)" % mode, "flops_per_launch": flops,
+                            "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x median SM clock"}
                 modes[mode] = {"value": wl.B * wl.T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
-                               "roofline": {"bound": "alu", "achieved": tf, "peak": fp32_peak, "unit": "TFLOP/s",
-                                            "frac": tf / fp32_peak, "traffic": None,
-                                            "kernel": "gdn2_%s_kernel (fp32 SIMT)" % mode, "flops_per_launch": flops,
-                                            "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x median SM clock"}}
+                               "roofline": roof}
             out[wl.name] = {"workload": wl.describe(), **modes}
         else:
             S = S0.clone()
@@ -791,6 +817,8 @@ def gdn2_over_ranks(gdn2, world, sm_mhz):
                 r["peak"] = fp32_simt_peak_tflops(sm_mhz)
             r["achieved"] = r["achieved"] * scale
             r["frac"] = r["achieved"] / r["peak"]
+            if "tensor_frac" in r:
+                r["tensor_frac"] = r["tensor_frac"] * scale
             e["roofline"] = r
             if mode is None:
                 val = e

@@ -402,7 +402,10 @@ mlstm_status_t mlstm_fwd_chunkwise_msr(const mlstm_fwd_params_t* p,
  *             K in {32, 64, 128, 256}.
  *             MLSTM_GDN2_CHUNK: chunks of p->chunk tokens (a multiple of 4, at most 64), dense
  *             products and one triangular solve per chunk (Gdn2Mode::Chunk); needs g <= 0.
- *             Unsupported sizes: MLSTM_ERR_SHAPE.
+ *             bf16 with chunk 64, K = 128 and V = 64 or 128 runs on the tensor cores (the
+ *             per-chunk matrices for all chunks at once, then one pass per head with the
+ *             state in tensor memory; bf16 operands, fp32 accumulation and state); other sizes
+ *             on fp32 SIMT kernels.  Unsupported sizes: MLSTM_ERR_SHAPE.
  *   q, k      [B,H,T,K]  dtype       required (if T > 0); k usually unit-norm (caller's choice)
  *   v         [B,H,T,V]  dtype       required
  *   g         [B,H,T,K]  fp32        log decay (log alpha), <= 0 for a decay
@@ -427,6 +430,13 @@ size_t mlstm_gdn2_workspace_size(const mlstm_gdn2_params_t* p);
 mlstm_status_t mlstm_gdn2_fwd(const mlstm_gdn2_params_t* p, const void* q, const void* k, const void* v,
                               const float* g, const float* b, const float* w, const float* S0, void* o,
                               float* S_out, void* workspace, size_t workspace_bytes, mlstm_stream_t stream);
+/* Outcome of the bounded device-side waits of the last mlstm_gdn2_fwd enqueued on `stream` with
+ * `workspace` and these params: synchronises `stream`; MLSTM_OK, or MLSTM_ERR_TIMEOUT when a
+ * wait of the tensor-core chunk kernels ran out (that call's o and S_out are unspecified; the
+ * workspace can be used again); MLSTM_OK always for the other paths, which have no such waits.
+ * MLSTM_ERR_CUDA if the synchronisation or the read fails; argument errors as mlstm_gdn2_fwd
+ * (workspace NULL: MLSTM_ERR_NULL when the tensor-core path would run). */
+mlstm_status_t mlstm_gdn2_status(const mlstm_gdn2_params_t* p, const void* workspace, mlstm_stream_t stream);
 
 /*
  * One recurrent decode step for every sequence of the batch, state updated in

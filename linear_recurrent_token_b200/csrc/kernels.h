@@ -54,6 +54,13 @@ int gdn2_chunk_vtile(int L, int K, int V);
 size_t gdn2_chunk_workspace_bytes(long long BH, int T, int L, int K);
 // mode 0: fused recurrent (token by token); 1: chunk of `chunk` tokens (needs ws)
 cudaError_t launch_gdn2(const Gdn2Args& a, int mode, int chunk, void* ws, cudaStream_t stream);
+// chunk mode on the tensor cores (gdn2_tc.cu): bf16, chunk 64, K 128, V 64 or 128, T > 0.  Its
+// workspace starts with a GDN2_TC_HEADER-byte header whose first word is the error word of the
+// bounded waits (bit 0: a wait ran out), then one slot per (batch x head, chunk).
+constexpr size_t GDN2_TC_HEADER = 256;
+bool gdn2_tc_supported(int chunk, int K, int V, int dtype, int T);
+size_t gdn2_tc_workspace_bytes(long long BH, int T, int V);
+cudaError_t launch_gdn2_tc(const Gdn2Args& a, void* ws, cudaStream_t stream);
 
 cudaError_t launch_gate_prep(int BH, int S, int n_per_head, const float* ig, const float* fg,
                              const float* m0, const float* n0, float* m_tok, float* m_init,

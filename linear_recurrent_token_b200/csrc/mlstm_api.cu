@@ -880,7 +880,24 @@ mlstm_status_t mlstm_fwd_chunkwise_msr(const mlstm_fwd_params_t* p, const void* 
 size_t mlstm_gdn2_workspace_size(const mlstm_gdn2_params_t* p) {
   if (!p || p->mode != MLSTM_GDN2_CHUNK || p->B < 0 || p->H < 0 || p->T < 0 || p->K < 1) return 0;
   if (p->chunk < 4 || p->chunk > 64 || p->chunk % 4) return 0;
+  if (gdn2_tc_supported(p->chunk, p->K, p->V, p->dtype == MLSTM_BF16 ? 1 : 0, p->T))
+    return gdn2_tc_workspace_bytes((long long)p->B * p->H, p->T, p->V);
   return gdn2_chunk_workspace_bytes((long long)p->B * p->H, p->T, p->chunk, p->K);
+}
+
+mlstm_status_t mlstm_gdn2_status(const mlstm_gdn2_params_t* p, const void* workspace, mlstm_stream_t stream) {
+  if (!p) return MLSTM_ERR_NULL;
+  if (p->dtype != MLSTM_F32 && p->dtype != MLSTM_BF16) return MLSTM_ERR_DTYPE;
+  if (p->B < 0 || p->H < 0 || p->T < 0 || p->K < 1 || p->V < 1) return MLSTM_ERR_SHAPE;
+  if (p->mode != MLSTM_GDN2_RECURRENT && p->mode != MLSTM_GDN2_CHUNK) return MLSTM_ERR_SHAPE;
+  const bool tc = p->mode == MLSTM_GDN2_CHUNK && (long long)p->B * p->H > 0 &&
+                  gdn2_tc_supported(p->chunk, p->K, p->V, p->dtype == MLSTM_BF16 ? 1 : 0, p->T);
+  if (tc && !workspace) return MLSTM_ERR_NULL;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MLSTM_ERR_CUDA;
+  if (!tc) return MLSTM_OK;  // no bounded waits ran
+  unsigned int word = 0;
+  if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return MLSTM_ERR_CUDA;
+  return word == 0 ? MLSTM_OK : MLSTM_ERR_TIMEOUT;
 }
 
 mlstm_status_t mlstm_gdn2_fwd(const mlstm_gdn2_params_t* p, const void* q, const void* k, const void* v,
@@ -920,6 +937,8 @@ mlstm_status_t mlstm_gdn2_fwd(const mlstm_gdn2_params_t* p, const void* q, const
              : cudaMemsetAsync(S_out, 0, bS, (cudaStream_t)stream);
     return e == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA;
   }
+  if (p->mode == MLSTM_GDN2_CHUNK && gdn2_tc_supported(p->chunk, p->K, p->V, a.dtype, p->T))
+    return launch_gdn2_tc(a, workspace, (cudaStream_t)stream) == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA;
   return launch_gdn2(a, p->mode, p->chunk, workspace, (cudaStream_t)stream) == cudaSuccess ? MLSTM_OK
                                                                                              : MLSTM_ERR_CUDA;
 }

@@ -131,6 +131,8 @@ def _load(path):
     L.mlstm_gdn2_workspace_size.argtypes = [ctypes.POINTER(Gdn2Params)]
     L.mlstm_gdn2_workspace_size.restype = Z
     L.mlstm_gdn2_fwd.argtypes = [ctypes.POINTER(Gdn2Params)] + [P] * 10 + [Z, P]
+    L.mlstm_gdn2_status.argtypes = [ctypes.POINTER(Gdn2Params), P, P]
+    L.mlstm_gdn2_status.restype = I
     L.mlstm_gdn2_fwd.restype = I
     L.mlstm_bwd_workspace_size.argtypes = [ctypes.POINTER(FwdParams)]
     L.mlstm_bwd_workspace_size.restype = Z
@@ -360,6 +362,19 @@ def gdn2_workspace_size(params: Gdn2Params) -> int:
     return int(lib().mlstm_gdn2_workspace_size(ctypes.byref(params)))
 
 
+def gdn2_params(q, v, mode: str = "recurrent", chunk: int = 64) -> Gdn2Params:
+    B, H, T, K = q.shape
+    return Gdn2Params(int(B), int(H), int(T), int(K), int(v.shape[-1]), _dtype_code(q),
+                      GDN2_CHUNK if mode == "chunk" else GDN2_RECURRENT, int(chunk))
+
+
+def gdn2_status(q, v, workspace, *, mode: str = "chunk", chunk: int = 64, stream=None) -> int:
+    """Outcome of the bounded waits of the last gdn2_fwd with this workspace (mlstm_gdn2_status;
+    synchronises): 0 ok, 8 a wait ran out (MLSTM_ERR_TIMEOUT)."""
+    p = gdn2_params(q, v, mode, chunk)
+    return int(lib().mlstm_gdn2_status(ctypes.byref(p), _ptr(workspace), _stream_ptr(stream)))
+
+
 def gdn2_fwd(q, k, v, g, b, w, S0=None, *, mode: str = "recurrent", chunk: int = 64, o=None, S_out=None,
              return_state: bool = True, workspace=None, stream=None):
     """Gated DeltaNet-2 (mlstm_gdn2_fwd): q, k [B,H,T,K], v [B,H,T,V] (fp32 or bf16); g, b
@@ -367,8 +382,7 @@ def gdn2_fwd(q, k, v, g, b, w, S0=None, *, mode: str = "recurrent", chunk: int =
     S_out may be S0 (in place: the decode step).  Returns (o, S_out)."""
     B, H, T, K = q.shape
     V = v.shape[-1]
-    p = Gdn2Params(int(B), int(H), int(T), int(K), int(V), _dtype_code(q),
-                   GDN2_CHUNK if mode == "chunk" else GDN2_RECURRENT, int(chunk))
+    p = gdn2_params(q, v, mode, chunk)
     if o is None:
         o = torch.empty((B, H, T, V), dtype=q.dtype, device=q.device)
     if return_state and S_out is None:

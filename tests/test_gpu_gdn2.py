@@ -88,3 +88,50 @@ def test_empty_sequence_copies_the_state():
     o, S = run(inp, "f32", "recurrent")
     assert o.shape == (2, 2, 0, 64)
     np.testing.assert_array_equal(S, inp["S0"])
+
+
+# The chunk mode on the tensor cores (bf16, chunk 64, K = 128, V = 64 or 128): the per-chunk
+# matrices built for all chunks at once, then one pass per head with the state in tensor memory.
+@pytest.mark.parametrize("B,H,T,V,state,inplace", [
+    (2, 3, 200, 128, True, False),   # ragged last chunk
+    (1, 4, 64, 64, True, True),      # one chunk, V = 64, state in place
+    (2, 2, 1, 128, False, False),    # a single token
+    (1, 2, 700, 64, True, False),    # eleven chunks, V = 64
+    (3, 2, 1000, 128, True, True),   # sixteen chunks, in place
+])
+def test_chunk_tensor_core(B, H, T, V, state, inplace):
+    inp = inputs.gdn2_inputs(B, H, T, 128, V, "bf16", seed=80 + T, with_state=state)
+    td = torch.bfloat16
+    p = mlstm.gdn2_params(dev(inp["q"], td), dev(inp["v"], td), "chunk", 64)
+    ws_bytes = mlstm.gdn2_workspace_size(p)
+    nch = (T + 63) // 64
+    assert ws_bytes == 256 + B * H * nch * (65536 + 384 * V + 512)  # the tensor-core slots
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    q = dev(inp["q"], td)
+    S0 = dev(inp["S0"])
+    o, S = mlstm.gdn2_fwd(q, dev(inp["k"], td), dev(inp["v"], td), dev(inp["g"]), dev(inp["b"]), dev(inp["w"]), S0,
+                          mode="chunk", chunk=64, workspace=ws, S_out=S0 if inplace and S0 is not None else None)
+    assert mlstm.gdn2_status(q, o, ws) == 0, "a bounded wait ran out"
+    check(inp, "bf16", host(o), host(S))
+
+
+def test_chunk_tensor_core_strong_decay():
+    """log decays down to about -20 per token: the diagonal 16-token blocks whose decay spans
+    more than e^{40} are summed pair by pair; the off-diagonal factors underflow to zero."""
+    inp = inputs.gdn2_inputs(1, 2, 150, 128, 128, "bf16", seed=83)
+    inp["g"] = (inp["g"] * 60).astype(np.float32)
+    o, S = run(inp, "bf16", "chunk", chunk=64)
+    check(inp, "bf16", o, S)
+
+
+def test_chunk_tensor_core_prefill_workload_sampled():
+    """The GDN-2 prefill workload (B8 H16 T2048 128 x 128, bf16) in one call; the oracle on the
+    heads of the first batch entry."""
+    wl = [w for w in inputs.GDN2_WORKLOADS if w.name == "gdn2_prefill"][0]
+    inp = inputs.gdn2_inputs(wl.B, wl.H, wl.T, wl.K, wl.V, wl.dtype, seed=7)
+    o, S = run(inp, "bf16", "chunk", chunk=64)
+    sub = {k_: (None if x is None else x[:1]) for k_, x in inp.items()}
+    o_ref, S_ref = oracle.gdn2_sequential(sub["q"], sub["k"], sub["v"], sub["g"], sub["b"], sub["w"], sub["S0"])
+    errs = {"o": slice_relerr(o[:1], o_ref, 2), "S": slice_relerr(S[:1], S_ref, 2)}
+    assert all(e <= TOL["bf16"] for e in errs.values()), errs
+    assert np.isfinite(o).all() and np.isfinite(S).all()
