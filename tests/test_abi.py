@@ -338,6 +338,18 @@ def test_gdn2_validation():
     assert gdn2_call(mode=1, chunk=8) == 5                          # no workspace
     assert gdn2_call(mode=1, chunk=8, ws=H_, ws_bytes=16) == 5      # too small
     assert gdn2_call(mode=1, chunk=8, ws=A, ws_bytes=1 << 30) == 7  # workspace over q
+    # the tensor-core chunk path (bf16, chunk 64, K 128, V 64 / 128): a 256-byte header (the
+    # error word of its bounded waits), then per (batch, head, chunk) a slot of Wk, Qw, Kt, nBt
+    # (4 x 16 KiB), U, Ur, Ou (3 x 128 V bytes) and e^{G_L} (512 bytes)
+    for V in (64, 128):
+        tc = mlstm.Gdn2Params(2, 3, 130, 128, V, 1, 1, 64)
+        assert mlstm.gdn2_workspace_size(tc) == 256 + 6 * 3 * (65536 + 384 * V + 512)
+    P = ctypes.c_void_p
+    L = mlstm.lib()
+    assert L.mlstm_gdn2_status(None, P(G_), P(0)) == 1
+    assert L.mlstm_gdn2_status(ctypes.byref(mlstm.Gdn2Params(2, 3, 130, 128, 128, 5, 1, 64)), P(G_), P(0)) == 3
+    assert L.mlstm_gdn2_status(ctypes.byref(mlstm.Gdn2Params(2, 3, -1, 128, 128, 1, 1, 64)), P(G_), P(0)) == 2
+    assert L.mlstm_gdn2_status(ctypes.byref(mlstm.Gdn2Params(2, 3, 130, 128, 128, 1, 1, 64)), None, P(0)) == 1
 
 
 def test_header_is_plain_c(tmp_path):
