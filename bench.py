@@ -921,7 +921,8 @@ def compact_legs(line):
         legs["bwd_" + e["workload"].split(":")[0]] = {"tok/s": _r(e["value"]), "ms": _r(e["ms_per_step"]),
                                                        e["roofline"]["bound"]: _r(e["roofline"]["frac"])}
     for e in line.get("scalar_normaliser", []):
-        legs["scalar_norm_" + e["workload"].split(":")[0]] = {"tok/s": _r(e["value"]), "ms": _r(e["ms_per_step"])}
+        legs["scalar_norm_" + e["workload"].split(":")[0]] = {"tok/s": _r(e["value"]), "ms": _r(e["ms_per_step"]),
+                                                              e["roofline"]["bound"]: _r(e["roofline"]["frac"])}
     if "msr_block" in line:
         e = line["msr_block"]
         legs["msr_block"] = {"tok/s": _r(e["value"]), "ms": _r(e["ms_per_step"]), "fwd_ms": _r(e["forward_ms"])}
@@ -931,7 +932,9 @@ def compact_legs(line):
             continue
         for mode in ("recurrent", "chunk"):
             if mode in val:
-                legs[f"gdn2_{mode}"] = {"tok/s": _r(val[mode]["value"]), "ms": _r(val[mode]["ms_per_step"])}
+                r = val[mode]["roofline"]
+                legs[f"gdn2_{mode}"] = {"tok/s": _r(val[mode]["value"]), "ms": _r(val[mode]["ms_per_step"]),
+                                        r["bound"]: _r(r["frac"])}
         if "recurrent" not in val and "roofline" in val:
             legs["gdn2_decode"] = {"GB/s": _r(val["value"]), "hbm": _r(val["roofline"]["frac"])}
     return legs
@@ -1142,14 +1145,26 @@ def main():
             nms = dist_max(statistics.median(ms), world)
             flops = chunkwise_flops(wn.B, wn.NH, wn.S, wn.dk, wn.dv, wn.chunk, wn.num_blocks, False)
             tf = flops / (nms * 1e-3) / 1e12
-            peak = fp32_simt_peak_tflops(sm_mhz)
+            import torch
+
+            from linear_recurrent_token_b200 import mlstm
+            tdn = torch.bfloat16 if wn.dtype == "bf16" else torch.float32
+            tc = mlstm.plan(mlstm.fwd_params(wn.B, wn.NH, wn.S, wn.DHQK, wn.DHV, wn.chunk, wn.num_blocks, tdn,
+                                             False))["tensor_core"] == 1
+            if tc:  # the scalar-normaliser walk on the tensor cores: flops against the bf16 peak
+                peak = peaks["bf16_tflops"]
+                roof = {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                        "traffic": None, "kernel": "whole call (gate prep, segment summaries, tcgen05 walk with "
+                        "the scalar normaliser)", "flops_per_launch": flops, "peak_source": "measured bf16 burst"}
+            else:
+                peak = fp32_simt_peak_tflops(sm_mhz)
+                roof = {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                        "traffic": None, "kernel": "SIMT chunkwise walk, scalar normaliser",
+                        "flops_per_launch": flops,
+                        "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x median SM clock"}
             line["scalar_normaliser"].append({
                 "workload": wn.describe(), "value": wn.B * wn.S * world / (nms * 1e-3), "unit": "tokens/s",
-                "ms_per_step": nms, "steps": len(ms),
-                "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
-                             "traffic": None, "kernel": "SIMT chunkwise walk, scalar normaliser",
-                             "flops_per_launch": flops,
-                             "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x median SM clock"}})
+                "ms_per_step": nms, "steps": len(ms), "roofline": roof})
             line["gpu_launches"] += len(ms) * 2
     if bwd:
         sm_mhz = line["clocks"].get("sm_mhz")
