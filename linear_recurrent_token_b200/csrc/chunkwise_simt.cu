@@ -31,9 +31,41 @@ size_t simt_walk_smem_bytes(int chunk, int dk, int dv_tile) {
 }
 
 int simt_walk_pick_tile(int chunk, int dk, int dv) {
-  int tv = dv < 32 ? dv : 32;
+  // value-row tile: 32 rows, or 16 for narrow blocks so that more CTAs share the work
+  int tv = dv <= 32 ? (dv < 16 ? dv : 16) : 32;
   while (tv > 1 && simt_walk_smem_bytes(chunk, dk, tv) > 227 * 1024) tv /= 2;
   return simt_walk_smem_bytes(chunk, dk, tv) <= 227 * 1024 ? tv : 0;
+}
+
+// Shared-memory dot products with four independent partial sums (the loops are latency-bound
+// with one accumulator).
+__device__ __forceinline__ float dot_smem(const float* x, const float* y, int n) {
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
+  int i = 0;
+  for (; i + 4 <= n; i += 4)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) a[u] = fmaf(x[i + u], y[i + u], a[u]);
+  for (; i < n; ++i) a[0] = fmaf(x[i], y[i], a[0]);
+  return (a[0] + a[1]) + (a[2] + a[3]);
+}
+// sum_i x[i] y[i * ystride]
+__device__ __forceinline__ float dot_smem_strided(const float* x, const float* y, int ystride, int n) {
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
+  int i = 0;
+  for (; i + 4 <= n; i += 4)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) a[u] = fmaf(x[i + u], y[(i + u) * ystride], a[u]);
+  for (; i < n; ++i) a[0] = fmaf(x[i], y[i * ystride], a[0]);
+  return (a[0] + a[1]) + (a[2] + a[3]);
+}
+__device__ __forceinline__ float sum_smem(const float* x, int n) {
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
+  int i = 0;
+  for (; i + 4 <= n; i += 4)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) a[u] += x[i + u];
+  for (; i < n; ++i) a[0] += x[i];
+  return (a[0] + a[1]) + (a[2] + a[3]);
 }
 
 template <typename T>
@@ -107,11 +139,21 @@ __global__ void __launch_bounds__(256) simt_walk_kernel(WalkArgs a) {
       }
     }
     __syncthreads();
-    if (tid == 0 && !ret) {
-      float run = 0.f;
-      for (int t = 0; t < Lc; ++t) {
-        run += bl[t];
-        bl[t] = run;
+    if (tid < 32 && !ret) {  // inclusive cumulative sum of log f over the chunk: a warp scan, each
+                             // lane over a run of ceil(Lc / 32) consecutive entries
+      const int per = (Lc + 31) / 32, t0 = tid * per, t1 = min(t0 + per, Lc);
+      float part = 0.f;
+      for (int t = t0; t < t1; ++t) part += bl[t];
+      float run = part;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, run, o);
+        if (tid >= o) run += u;
+      }
+      float acc = run - part;
+      for (int t = t0; t < t1; ++t) {
+        acc += bl[t];
+        bl[t] = acc;
       }
     }
     __syncthreads();
@@ -126,9 +168,7 @@ __global__ void __launch_bounds__(256) simt_walk_kernel(WalkArgs a) {
       const int t = i / L, s = i % L;
       float p = 0.f;
       if (s <= t && t < Lc) {
-        float dot = 0.f;
-        for (int c = 0; c < dk; ++c) dot += Qs[t * ldk + c] * Ks[s * ldk + c];
-        p = dot * expf(bl[t] - bl[s] + li[s] - mt[t]);
+        p = dot_smem(Qs + t * ldk, Ks + s * ldk, dk) * expf(bl[t] - bl[s] + li[s] - mt[t]);
       }
       Ps[t * (L + 1) + s] = p;
     }
@@ -142,18 +182,15 @@ __global__ void __launch_bounds__(256) simt_walk_kernel(WalkArgs a) {
       }
     } else if (!ret) {
       for (int t = tid; t < Lc; t += nt) {
-        float rs = 0.f, qn = 0.f;
-        for (int s = 0; s <= t; ++s) rs += Ps[t * (L + 1) + s];
-        for (int c = 0; c < dk; ++c) qn += Qs[t * ldk + c] * ns[c];
+        const float rs = sum_smem(Ps + t * (L + 1), t + 1), qn = dot_smem(Qs + t * ldk, ns, dk);
         den[t] = fmaxf(fabsf(rs + sint[t] * qn), expf(-mt[t]));
       }
     }
     __syncthreads();
     for (int i = tid; i < Lc * tv; i += nt) {
       const int t = i / tv, r = i % tv;
-      float acc_i = 0.f, acc_c = 0.f;
-      for (int s = 0; s <= t; ++s) acc_i += Ps[t * (L + 1) + s] * Vs[s * TV + r];
-      for (int c = 0; c < dk; ++c) acc_c += Qs[t * ldk + c] * Cs[r * ldk + c];
+      const float acc_i = dot_smem_strided(Ps + t * (L + 1), Vs + r, TV, t + 1);
+      const float acc_c = dot_smem(Qs + t * ldk, Cs + r * ldk, dk);
       float hv = acc_i + sint[t] * acc_c;
       const size_t hi = (tok0 + t) * DHV + (size_t)blk * dv + v0 + r;
       if (!ret) {
@@ -165,9 +202,13 @@ __global__ void __launch_bounds__(256) simt_walk_kernel(WalkArgs a) {
     __syncthreads();
     for (int i = tid; i < tv * dk; i += nt) {
       const int r = i / dk, c = i % dk;
-      float acc = 0.f;
-      for (int s = 0; s < Lc; ++s) acc += wv[s] * Vs[s * TV + r] * Ks[s * ldk + c];
-      Cs[r * ldk + c] = decay * Cs[r * ldk + c] + acc;
+      float a4[4] = {0.f, 0.f, 0.f, 0.f};
+      int s = 0;
+      for (; s + 4 <= Lc; s += 4)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) a4[u] = fmaf(wv[s + u] * Vs[(s + u) * TV + r], Ks[(s + u) * ldk + c], a4[u]);
+      for (; s < Lc; ++s) a4[0] = fmaf(wv[s] * Vs[s * TV + r], Ks[s * ldk + c], a4[0]);
+      Cs[r * ldk + c] = decay * Cs[r * ldk + c] + ((a4[0] + a4[1]) + (a4[2] + a4[3]));
     }
     if (scalar_n) {
       if (tid == 0) {

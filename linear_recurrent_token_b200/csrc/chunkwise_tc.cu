@@ -120,6 +120,24 @@ __device__ __forceinline__ int tile_row_c(int t) {
   return REV ? L - 1 - t : t;
 }
 
+// A 64-column tile of q, k, v or h at (column x of the head row, token row, head bh).  Blocks
+// narrower than 64 columns (pad) are addressed as block blk of a {width, nb, S, BH} tensor: the
+// load fills the missing columns with zeros, the store writes only the block's columns.
+__device__ __forceinline__ void tile_load(void* dst, const CUtensorMap* map, bool pad, int x, int blk, int row, int bh,
+                                          uint64_t* bar) {
+  if (pad)
+    tma_load_4d(dst, map, 0, blk, row, bh, bar);
+  else
+    tma_load_3d(dst, map, x, row, bh, bar);
+}
+__device__ __forceinline__ void tile_store(const CUtensorMap* map, const void* src, bool pad, int x, int blk, int row,
+                                           int bh) {
+  if (pad)
+    tma_store_4d(map, src, 0, blk, row, bh);
+  else
+    tma_store_3d(map, src, x, row, bh);
+}
+
 // Lane / row mapping of an M-row accumulator: thread (warp w, lane l) owns row
 // 32w+l for M=128; row 16w+l for M=64 (lanes 16..31 hold no row).
 template <int M>
@@ -246,10 +264,12 @@ __device__ __noinline__ void scale_tmem_lane(uint32_t taddr, float f) {
 // multiplied by the output gate og[t][d] (og points at token t0, value column v0; row stride
 // ld), tokens t < Lc; the 128 threads of the output group share the work
 template <int DVT>
-__device__ __noinline__ void apply_ogate(uint32_t hs_u, const __nv_bfloat16* og, size_t ld, int Lc, int gt) {
+__device__ __noinline__ void apply_ogate(uint32_t hs_u, const __nv_bfloat16* og, size_t ld, int Lc, int gt,
+                                         int ncol) {
   constexpr int NCH = DVT / 8;
   for (int i = gt; i < Lc * NCH; i += 128) {
     const int t = i / NCH, d = 8 * (i % NCH);
+    if (d >= ncol) continue;  // columns past a narrow block
     const uint32_t a = hs_u + (d >> 6) * 8192 + t * 128 + ((((d & 63) >> 3) ^ (t & 7)) << 4);
     uint4 h = ld_shared_v4(a);
     const uint4 o = *reinterpret_cast<const uint4*>(og + t * ld + d);
@@ -341,7 +361,7 @@ struct SegCfg {
   static constexpr int BYTES_FIXED = NS * STAGE + (128 * 8 + NS * L) * 4 + 1024;
 };
 
-template <int DK, int DVA>
+template <int DK, int DVA, bool PAD>
 __global__ void __launch_bounds__(NTA, 1)
     tc_segment_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV, TcParams p) {
   using CF = SegCfg<DK, DVA>;
@@ -396,10 +416,10 @@ __global__ void __launch_bounds__(NTA, 1)
     for (int jj = 0; jj < DK / 64; ++jj)
       if (tma_box_ok(p.err, BS_SEG_TMA, blk * p.dk + 64 * jj, row0, 8, p.DHQK, p.S, L, false) &&
           in_bounds(p.err, BS_SEG_TMA, bh, p.BH))
-        tma_load_3d(kb + jj * 8192, &mapK, blk * p.dk + 64 * jj, row0, bh, &full[st]);
+        tile_load(kb + jj * 8192, &mapK, PAD && p.dk < DK, blk * p.dk + 64 * jj, blk, row0, bh, &full[st]);
     for (int jj = 0; jj < DVA / 64; ++jj)
       if (tma_box_ok(p.err, BS_SEG_TMA, blk * p.dv + v0 + 64 * jj, row0, 8, p.DHV, p.S, L, false))
-        tma_load_3d(kb + KB + jj * 8192, &mapV, blk * p.dv + v0 + 64 * jj, row0, bh, &full[st]);
+        tile_load(kb + KB + jj * 8192, &mapV, PAD && p.dv < DVA, blk * p.dv + v0 + 64 * jj, blk, row0, bh, &full[st]);
   };
   // K and V are inputs: the first stages load while the previous kernel finishes
   int n_issued = 0;  // chunks whose loads thread 0 has issued
@@ -593,20 +613,23 @@ __global__ void __launch_bounds__(NTA, 1)
         float r[32];
         tmem_ld32(tm + ((uint32_t)(32 * quarter) << 16) + a * DK + c0, r);
         tmem_wait_ld();
-        if (dst && !abort_flag &&
+        // (rows and columns past a narrow block's dv x dk are padding)
+        const int ncol = PAD ? min(32, p.dk - c0) : 32;
+        if (dst && !abort_flag && (!PAD || v0 + a * MA + row < p.dv) && ncol > 0 &&
             in_bounds(p.err, BS_SEG_DC,
-                      (((long long)slice * p.NU + j) * p.dv + v0 + a * MA + row) * p.dk + c0 + 31,
+                      (((long long)slice * p.NU + j) * p.dv + v0 + a * MA + row) * p.dk + c0 + ncol - 1,
                       (long long)p.slices * p.NU * p.dv * p.dk))
 #pragma unroll
           for (int jj = 0; jj < 32; jj += 4)
-            *reinterpret_cast<float4*>(dst + c0 + jj) = make_float4(r[jj], r[jj + 1], r[jj + 2], r[jj + 3]);
+            if (jj < ncol)
+              *reinterpret_cast<float4*>(dst + c0 + jj) = make_float4(r[jj], r[jj + 1], r[jj + 2], r[jj + 3]);
       }
     }
     if (do_dn) {
       *reinterpret_cast<float4*>(dnp + gt * 8) = make_float4(dacc[0].x, dacc[0].y, dacc[1].x, dacc[1].y);
       *reinterpret_cast<float4*>(dnp + gt * 8 + 4) = make_float4(dacc[2].x, dacc[2].y, dacc[3].x, dacc[3].y);
       named_bar(1, 128);
-      for (int col = gt; col < ncg * 8 && dn0 + col < DK; col += 128) {
+      for (int col = gt; col < ncg * 8 && dn0 + col < (PAD ? p.dk : DK); col += 128) {
         float x = 0.f;
         for (int r = 0; r < nrg; ++r) x += dnp[(r * ncg + col / 8) * 8 + (col & 7)];
         if (!abort_flag && in_bounds(p.err, BS_SEG_DN, ((long long)slice * p.NU + j) * p.dk + dn0 + col,
@@ -712,7 +735,7 @@ struct WalkBars {
   uint64_t comp;   // the summary tiles of the start state (prologue)
 };
 
-template <int DK, int DVT, bool SN, bool REV>
+template <int DK, int DVT, bool SN, bool REV, bool PAD>
 __global__ void __launch_bounds__(NTW, 1)
     tc_walk_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                    const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapH,
@@ -830,7 +853,7 @@ __global__ void __launch_bounds__(NTW, 1)
       float r[16];
 #pragma unroll
       for (int jj = 0; jj < 16; ++jj) r[jj] = 0.f;
-      if (row >= 0 && p.C0 &&
+      if (row >= 0 && p.C0 && (!PAD || (v0 + row < p.dv && c0 < p.dk)) &&  // (narrow blocks: padding stays zero)
           in_bounds(p.err, BS_WALK_START, ((long long)slice * p.dv + v0 + row) * p.dk + c0 + 15,
                     (long long)p.slices * p.dv * p.dk)) {
         const float4* src = reinterpret_cast<const float4*>(p.C0 + ((size_t)slice * p.dv + v0 + row) * p.dk + c0);
@@ -850,10 +873,11 @@ __global__ void __launch_bounds__(NTW, 1)
   static_assert(DVT * DK * 4 <= 2 * SM::STAGE, "a summary tile fits the stage area");
   for (int j = 0; j < nun; ++j) {
     if (tid == 0) {
-      mbar_arrive_expect_tx(&bars.comp, DVT * DK * 4);
+      const int ncb = PAD ? min(DK, p.dk + 31) / 32 : DK / 32;  // 32-column boxes holding the block's columns
+      mbar_arrive_expect_tx(&bars.comp, (uint32_t)((DVT + 63) / 64 * ncb * 8192));
       const int r0 = ((int)slice * p.NU + j) * p.dv + v0;
       for (int rb = 0; rb < (DVT + 63) / 64; ++rb)
-        for (int cb = 0; cb < DK / 32; ++cb)
+        for (int cb = 0; cb < ncb; ++cb)
           if (tma_box_ok(p.err, BS_WALK_SUM_TMA, 32 * cb, r0 + 64 * rb, 4, p.dk, (long long)p.slices * p.NU * p.dv,
                          64, true))  // held to a store's rule: the tile must start inside the summaries
             tma_load_2d(sm + (rb * (DK / 32) + cb) * 8192, &mapS, 32 * cb, r0 + 64 * rb, &bars.comp);
@@ -873,7 +897,7 @@ __global__ void __launch_bounds__(NTW, 1)
         float r[32];
         tmem_ld32(tm + lane_off + TM_C + c0, r);
         tmem_wait_ld();
-        if (row >= 0) {
+        if (row >= 0 && (!PAD || (v0 + row < p.dv && c0 < p.dk))) {  // (narrow blocks: padding stays zero)
           const uint8_t* box = sm + ((row >> 6) * (DK / 32) + (c0 >> 5)) * 8192 + rr * 128;
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
@@ -906,6 +930,11 @@ __global__ void __launch_bounds__(NTW, 1)
       }
     } else if (!ret)
       for (int col = nt2; col < DK; col += 224) {
+        if (PAD && col >= p.dk) {  // padding of a narrow block
+          nvec[col] = 0.f;
+          store_nfrag<DK>(nfrag, col, 0.f);
+          continue;
+        }
         float x = p.n0 && in_bounds(p.err, BS_WALK_START, (long long)slice * p.dk + col, (long long)p.slices * p.dk)
                       ? wc0 * p.n0[(size_t)slice * p.dk + col]
                       : 0.f;
@@ -1044,12 +1073,13 @@ __global__ void __launch_bounds__(NTW, 1)
         for (int j = 0; j < DK / 64; ++j)
           if (tma_box_ok(p.err, BS_WALK_TMA, blk * p.dk + 64 * j, t0, 8, p.DHQK, p.S, L, false) &&
               in_bounds(p.err, BS_WALK_TMA, bh, p.BH)) {
-            tma_load_3d(base + j * 8192, &mapQ, blk * p.dk + 64 * j, t0, bh, &bars.full[b]);
-            tma_load_3d(base + SM::QB + j * 8192, &mapK, blk * p.dk + 64 * j, t0, bh, &bars.full[b]);
+            tile_load(base + j * 8192, &mapQ, PAD && p.dk < DK, blk * p.dk + 64 * j, blk, t0, bh, &bars.full[b]);
+            tile_load(base + SM::QB + j * 8192, &mapK, PAD && p.dk < DK, blk * p.dk + 64 * j, blk, t0, bh, &bars.full[b]);
           }
         for (int j = 0; j < DVT / 64; ++j)
           if (tma_box_ok(p.err, BS_WALK_TMA, blk * p.dv + v0 + 64 * j, t0, 8, p.DHV, p.S, L, false))
-            tma_load_3d(base + SM::QB + SM::KB + j * 8192, &mapV, blk * p.dv + v0 + 64 * j, t0, bh, &bars.full[b]);
+            tile_load(base + SM::QB + SM::KB + j * 8192, &mapV, PAD && p.dv < DVT, blk * p.dv + v0 + 64 * j, blk, t0, bh,
+                      &bars.full[b]);
         n_issued = c + 1;
       }
       // gate quantities of chunk c into buffer gi (lane: tokens 2 lane, 2 lane + 1)
@@ -1269,12 +1299,15 @@ __global__ void __launch_bounds__(NTW, 1)
         float r[32];
         tmem_ld32(tm + lane_off + TM_C + c0, r);
         tmem_wait_ld();
-        if (row >= 0 && in_bounds(p.err, BS_WALK_FINAL, ((long long)slice * p.dv + v0 + row) * p.dk + c0 + 31,
-                                  (long long)p.slices * p.dv * p.dk)) {
+        const int ncol = PAD ? min(32, p.dk - c0) : 32;  // (narrow blocks: padding is not written)
+        if (row >= 0 && (!PAD || v0 + row < p.dv) && ncol > 0 &&
+            in_bounds(p.err, BS_WALK_FINAL, ((long long)slice * p.dv + v0 + row) * p.dk + c0 + ncol - 1,
+                      (long long)p.slices * p.dv * p.dk)) {
           float* dst = p.C_out + ((size_t)slice * p.dv + v0 + row) * p.dk + c0;
 #pragma unroll
           for (int j = 0; j < 32; j += 4)
-            *reinterpret_cast<float4*>(dst + j) = make_float4(fin * r[j], fin * r[j + 1], fin * r[j + 2], fin * r[j + 3]);
+            if (j < ncol)
+              *reinterpret_cast<float4*>(dst + j) = make_float4(fin * r[j], fin * r[j + 1], fin * r[j + 2], fin * r[j + 3]);
         }
       }
     }
@@ -1447,9 +1480,10 @@ __global__ void __launch_bounds__(NTW, 1)
       if (use_og) {  // h <- h o o_t on the staged tile
         named_bar(WG_OUT, 128);
         // (the largest index it reads: its last row's last column)
-        if (in_bounds(p.err, BS_WALK_OGATE, (long long)(tok0 + Lc - 1) * p.DHV + blk * p.dv + v0 + DVT - 1,
+        const int ncol = PAD ? min(DVT, p.dv - v0) : DVT;  // (narrow blocks: only the block's columns)
+        if (in_bounds(p.err, BS_WALK_OGATE, (long long)(tok0 + Lc - 1) * p.DHV + blk * p.dv + v0 + ncol - 1,
                       (long long)p.BH * p.S * p.DHV))
-          apply_ogate<DVT>(hs_u, p.og + tok0 * p.DHV + (size_t)blk * p.dv + v0, p.DHV, Lc, gt);
+          apply_ogate<DVT>(hs_u, p.og + tok0 * p.DHV + (size_t)blk * p.dv + v0, p.DHV, Lc, gt, ncol);
       }
       fence_proxy_async_smem();
       named_bar(WG_OUT, 128);
@@ -1457,7 +1491,7 @@ __global__ void __launch_bounds__(NTW, 1)
         for (int j = 0; j < DVT / 64; ++j)
           if (tma_box_ok(p.err, BS_WALK_H_TMA, blk * p.dv + v0 + 64 * j, t0, 8, p.DHV, p.S, L, true) &&
               in_bounds(p.err, BS_WALK_H_TMA, bh, p.BH))
-            tma_store_3d(&mapH, sm + SM::OH + j * 8192, blk * p.dv + v0 + 64 * j, t0, bh);
+            tile_store(&mapH, sm + SM::OH + j * 8192, PAD && p.dv < DVT, blk * p.dv + v0 + 64 * j, blk, t0, bh);
         bulk_commit();
         mbar_arrive(&bars.gempty[gi]);
       }
@@ -1589,7 +1623,7 @@ __global__ void __launch_bounds__(NTW, 1)
           in_bounds(p.err, BS_WALK_FINAL, bh, p.BH))
         p.n_out[bh] = fin * n_sc;
     } else if (nck > 0 && last_seg && !ret && tile == 0 && p.n_out && !abort_flag)
-      for (int col = nt; col < DK; col += 128)
+      for (int col = nt; col < (PAD ? p.dk : DK); col += 128)
         if (in_bounds(p.err, BS_WALK_FINAL, (long long)slice * p.dk + col, (long long)p.slices * p.dk))
           p.n_out[(size_t)slice * p.dk + col] = fin * nvec[col];
   }
@@ -1620,8 +1654,9 @@ __global__ void __launch_bounds__(NTW, 1)
 // ===================================================================== host side
 bool tc_supported(int dtype, int chunk, int dk, int dv, int DHQK, int DHV) {
   if (dtype != 1 || chunk != L) return false;
-  if (dk != 64 && dk != 128 && dk != 256) return false;
-  if (dv % 64 != 0) return false;
+  // block widths below 64 run padded to 64 (zero-filled columns / rows)
+  if (dk != 64 && dk != 128 && dk != 256 && !(dk < 64 && dk % 8 == 0)) return false;
+  if (dv % 64 != 0 && !(dv < 64 && dv % 8 == 0 && dk <= 64)) return false;
   if (DHQK % 8 != 0 || DHV % 8 != 0) return false;
   return true;
 }
@@ -1635,7 +1670,7 @@ int tc_num_sms() {
 TcPlan tc_plan(int B, int NH, int S, int nb, int dk, int dv, int num_sms) {
   TcPlan pl;
   pl.dvt = (dv % 128 == 0) ? 128 : 64;
-  pl.n_tiles = dv / pl.dvt;
+  pl.n_tiles = (dv + pl.dvt - 1) / pl.dvt;  // (a block narrower than 64 is one padded tile)
   const int chunks = (S + L - 1) / L;
   const long long base = (long long)B * NH * nb * pl.n_tiles;
   int G = base > 0 ? (int)(num_sms / base) : 1;
@@ -1726,17 +1761,17 @@ static cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 bl
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-template <int DK, int DVA>
+template <int DK, int DVA, bool PAD>
 static cudaError_t launch_segment(const TcPlan& pl, const TcParams& prm, const CUtensorMap& mk, const CUtensorMap& mv,
                                   long long slices, cudaStream_t stream) {
   const int smemA = SegCfg<DK, DVA>::BYTES_FIXED + pl.seg0_chunks * 4;  // + one offset per chunk of a unit
-  cudaError_t e = cudaFuncSetAttribute(tc_segment_kernel<DK, DVA>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemA);
+  cudaError_t e = cudaFuncSetAttribute(tc_segment_kernel<DK, DVA, PAD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemA);
   if (e != cudaSuccess) return e;
   dim3 gridA(pl.n_tiles_a, pl.NU, (unsigned)slices);
-  return launch_dependent(tc_segment_kernel<DK, DVA>, gridA, dim3(NTA), smemA, stream, mk, mv, prm);
+  return launch_dependent(tc_segment_kernel<DK, DVA, PAD>, gridA, dim3(NTA), smemA, stream, mk, mv, prm);
 }
 
-template <int DK, int DVT, bool SN, bool REV>
+template <int DK, int DVT, bool SN, bool REV, bool PAD>
 static cudaError_t launch_tc_dk(const TcPlan& pl, const TcParams& prm, const CUtensorMap& mq, const CUtensorMap& mk,
                                 const CUtensorMap& mv, const CUtensorMap& mh, const CUtensorMap& ms, long long slices,
                                 cudaStream_t stream, cudaEvent_t ev0, cudaEvent_t ev1) {
@@ -1746,17 +1781,17 @@ static cudaError_t launch_tc_dk(const TcPlan& pl, const TcParams& prm, const CUt
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (pl.NU > 0) {
-    e = pl.dva == 256   ? launch_segment<DK, 256>(pl, prm, mk, mv, slices, stream)
-        : pl.dva == 128 ? launch_segment<DK, 128>(pl, prm, mk, mv, slices, stream)
-                        : launch_segment<DK, 64>(pl, prm, mk, mv, slices, stream);
+    e = pl.dva == 256   ? launch_segment<DK, 256, false>(pl, prm, mk, mv, slices, stream)
+        : pl.dva == 128 ? launch_segment<DK, 128, PAD>(pl, prm, mk, mv, slices, stream)
+                        : launch_segment<DK, 64, PAD>(pl, prm, mk, mv, slices, stream);
     if (e != cudaSuccess) return e;
   }
   const int smemC = WalkSmem<DK, DVT>::BYTES;
-  e = cudaFuncSetAttribute(tc_walk_kernel<DK, DVT, SN, REV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemC);
+  e = cudaFuncSetAttribute(tc_walk_kernel<DK, DVT, SN, REV, PAD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemC);
   if (e != cudaSuccess) return e;
   if (ev0) cudaEventRecord(ev0, stream);
   dim3 gridC(pl.n_tiles, (unsigned)slices, pl.G);
-  e = launch_dependent(tc_walk_kernel<DK, DVT, SN, REV>, gridC, dim3(NTW), smemC, stream, mq, mk, mv, mh, ms, prm);
+  e = launch_dependent(tc_walk_kernel<DK, DVT, SN, REV, PAD>, gridC, dim3(NTW), smemC, stream, mq, mk, mv, mh, ms, prm);
   if (ev1) cudaEventRecord(ev1, stream);
   return e;
 }
@@ -1766,10 +1801,16 @@ cudaError_t launch_tc(const WalkArgs& a, const TcPlan& pl, void* ws, cudaStream_
   const long long BH = (long long)a.B * a.NH, slices = BH * a.nb;
   if (slices == 0 || a.S == 0) return cudaSuccess;
   CUtensorMap mq, mk, mv, mh;
-  if (!make_map_bf16_3d(&mq, a.q, a.DHQK, a.S, BH, L) || !make_map_bf16_3d(&mk, a.k, a.DHQK, a.S, BH, L) ||
-      !make_map_bf16_3d(&mv, a.v, a.DHV, a.S, BH, L) ||
-      !make_map_bf16_3d(&mh, a.h, a.DHV, a.S, BH, L))
-    return cudaErrorInvalidValue;
+  // blocks narrower than 64 columns: 4-D maps {block width, nb, S, BH} (tiles zero-padded to 64)
+  const bool qk_ok = a.dk < 64 ? make_map_bf16_blocks(&mq, a.q, a.dk, a.nb, a.S, BH, L) &&
+                                     make_map_bf16_blocks(&mk, a.k, a.dk, a.nb, a.S, BH, L)
+                               : make_map_bf16_3d(&mq, a.q, a.DHQK, a.S, BH, L) &&
+                                     make_map_bf16_3d(&mk, a.k, a.DHQK, a.S, BH, L);
+  const bool vh_ok = a.dv < 64 ? make_map_bf16_blocks(&mv, a.v, a.dv, a.nb, a.S, BH, L) &&
+                                     make_map_bf16_blocks(&mh, a.h, a.dv, a.nb, a.S, BH, L)
+                               : make_map_bf16_3d(&mv, a.v, a.DHV, a.S, BH, L) &&
+                                     make_map_bf16_3d(&mh, a.h, a.DHV, a.S, BH, L);
+  if (!qk_ok || !vh_ok) return cudaErrorInvalidValue;
   TcParams prm;
   prm.S = a.S;
   prm.NH = a.NH;
@@ -1830,20 +1871,24 @@ cudaError_t launch_tc(const WalkArgs& a, const TcPlan& pl, void* ws, cudaStream_
   // the error word and, for the bounds-checked build, its record (bytes 16..39)
   cudaError_t e = cudaMemsetAsync(w, 0, 64, stream);
   if (e != cudaSuccess) return e;
+  const int dkp = a.dk < 64 ? 64 : a.dk;  // key width of the kernels (narrow blocks padded)
+  const bool pad = a.dk < 64 || a.dv < 64;  // kernels that mask the padding of narrow blocks
 #define MLSTM_TC_DISPATCH(SNV, REVV)                                                                       \
   do {                                                                                                   \
     if (a.dk == 256 && pl.dvt == 128)                                                                    \
-      return launch_tc_dk<256, 128, SNV, REVV>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1);       \
+      return launch_tc_dk<256, 128, SNV, REVV, false>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1);       \
     if (a.dk == 256 && pl.dvt == 64)                                                                     \
-      return launch_tc_dk<256, 64, SNV, REVV>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1);        \
+      return launch_tc_dk<256, 64, SNV, REVV, false>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1);        \
     if (a.dk == 128 && pl.dvt == 128)                                                                    \
-      return launch_tc_dk<128, 128, SNV, REVV>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1);       \
+      return launch_tc_dk<128, 128, SNV, REVV, false>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1);       \
     if (a.dk == 128 && pl.dvt == 64)                                                                     \
-      return launch_tc_dk<128, 64, SNV, REVV>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1);        \
-    if (a.dk == 64 && pl.dvt == 128)                                                                     \
-      return launch_tc_dk<64, 128, SNV, REVV>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1);        \
-    if (a.dk == 64 && pl.dvt == 64)                                                                      \
-      return launch_tc_dk<64, 64, SNV, REVV>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1);         \
+      return launch_tc_dk<128, 64, SNV, REVV, false>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1);        \
+    if (dkp == 64 && pl.dvt == 128)                                                                      \
+      return pad ? launch_tc_dk<64, 128, SNV, REVV, true>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1) \
+                 : launch_tc_dk<64, 128, SNV, REVV, false>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1); \
+    if (dkp == 64 && pl.dvt == 64)                                                                       \
+      return pad ? launch_tc_dk<64, 64, SNV, REVV, true>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1) \
+                 : launch_tc_dk<64, 64, SNV, REVV, false>(pl, prm, mq, mk, mv, mh, ms, slices, stream, ev0, ev1); \
   } while (0)
   // walk variants: the vector normaliser forward and reversed, the scalar normaliser forward
   if (prm.nbias && !prm.rev) MLSTM_TC_DISPATCH(true, false);

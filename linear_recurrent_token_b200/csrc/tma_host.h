@@ -40,6 +40,24 @@ inline bool make_map_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, ui
   return r == CUDA_SUCCESS;
 }
 
+// A block of d0 < 64 columns of a row-major bf16 tensor [d3][d2][row] whose rows hold d1 such
+// blocks side by side (row = d1 * d0 values), as a 4-D tensor {d0, d1, d2, d3}; box {64, 1,
+// box_rows, 1}, 128-byte swizzle: a load fills columns d0..63 of each tile row with zeros and a
+// store writes only the block's d0 columns.  d0 * 2 must be a multiple of 16.
+inline bool make_map_bf16_blocks(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                                 uint64_t d3, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {d0, d1, d2, d3};
+  const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+  const cuuint32_t box[4] = {64, 1, box_rows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // 2-D fp32 tensor [d1][d0] (d0 contiguous, d0 * 4 bytes a multiple of 16), box {32, box_rows}
 // (128-byte rows), 128-byte swizzle.
 inline bool make_map_f32_2d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint32_t box_rows) {

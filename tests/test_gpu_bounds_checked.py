@@ -26,6 +26,8 @@ CASES = [
     (1, 3, 1000, 64, 64, 1, True, True, False, False),      # retention
     (1, 2, 1500, 128, 256, 1, False, True, True, True),     # reversed, several segments, ragged
     (1, 8, 4100, 256, 512, 1, False, False, False, False),  # the large head, several segments, ragged
+    (2, 2, 700, 64, 64, 2, False, True, True, False),       # 32 x 32 blocks, zero-padded tiles
+    (1, 2, 600, 64, 64, 4, False, True, True, True),        # 16 x 16 blocks, reversed
 ]
 
 

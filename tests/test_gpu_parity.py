@@ -316,6 +316,13 @@ TC_CASES = [
     (1, 2, 1000, 128, 256, 1, False, True, True),
     (2, 2, 700, 64, 256, 1, True, True, False),
     (1, 3, 777, 64, 512, 1, False, True, True),
+    # blocks narrower than 64 (zero-padded tiles): 32 x 32, 16 x 16 over several segments,
+    # 32 x 128 (keys padded), 64 x 32 (values padded)
+    (2, 2, 300, 64, 64, 2, False, True, True),
+    (1, 2, 1000, 64, 64, 4, False, True, True),
+    (2, 2, 256, 64, 256, 2, False, False, False),
+    (1, 2, 700, 128, 64, 2, True, True, False),
+    (1, 3, 200, 32, 32, 2, False, True, False),
 ]
 
 
@@ -542,6 +549,7 @@ SN_TC_CASES = [
     (2, 2, 333, 64, 128, 1, False, False),     # ragged last chunk, zero initial state
     (1, 4, 2048, 256, 512, 1, False, True),    # the large-head shape
     (2, 2, 640, 128, 128, 2, True, True),      # two blocks sharing the head's scalar n
+    (1, 2, 700, 64, 64, 2, True, True),        # 32 x 32 blocks (zero-padded tiles)
 ]
 
 
