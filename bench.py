@@ -829,9 +829,16 @@ def gdn2_over_ranks(gdn2, world, sm_mhz):
 
 
 def backward_uses_cluster(dtype, dk, dv):
-    """Whether mlstm_bwd runs the cluster kernel (warp-level bf16 MMAs) for these block widths:
-    bf16, key width 64 / 128 / 256, value width a multiple of 64 up to 512 (the library's rule)."""
-    return dtype == "bf16" and dk in (64, 128, 256) and dv % 64 == 0 and 64 <= dv <= 512
+    """Whether mlstm_bwd runs the cluster kernel (warp-level bf16 MMAs) for these block widths
+    (the library's rule): bf16; key width 64 / 128 / 256 or narrower (a multiple of 8, padded);
+    value width a multiple of 64 up to 512, or narrower (a multiple of 8) with keys at most 64."""
+    if dtype != "bf16":
+        return False
+    if dk not in (64, 128, 256) and not (dk < 64 and dk % 8 == 0):
+        return False
+    if dv < 64:
+        return dv % 8 == 0 and dk <= 64
+    return dv % 64 == 0 and dv <= 512
 
 
 def backward_line(w, ms, sm_mhz, cpu: bool, peaks=None):

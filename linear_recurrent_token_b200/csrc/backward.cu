@@ -964,9 +964,12 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
   const int nck = (S + BCL - 1) / BCL;
   for (int blk = 0; blk < a.nb; ++blk) {
     const size_t slice = (size_t)bh * a.nb + blk;
-    const size_t qoff = (size_t)bh * S * a.DHQK + (size_t)blk * DK;
+    // (blocks narrower than DK key columns or BCV value rows run zero-padded: every global
+    // access below is masked to the block's dk x dv)
+    const int dkr = a.dk;
+    const size_t qoff = (size_t)bh * S * a.DHQK + (size_t)blk * dkr;
     const size_t voff = (size_t)bh * S * a.DHV + (size_t)blk * dv + r0;
-    const size_t soff = slice * (size_t)dv * DK + (size_t)r0 * DK;  // this CTA's rows of a state
+    const size_t soff = slice * (size_t)dv * dkr + (size_t)r0 * dkr;  // this CTA's rows of a state
 
     // chunk inputs, gate logs, W and P (every CTA: the key-side products are redundant)
     auto load_chunk = [&](int t0, int Lc) {
@@ -978,7 +981,7 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
       for (int i = 0; i < NQL; ++i) {
         const int e = tid + i * BCT, t = e / (DK / 8), c = (e % (DK / 8)) * 8;
         uq[i] = uk[i] = make_uint4(0, 0, 0, 0);
-        if (t < Lc) {
+        if (t < Lc && c < dkr) {
           uq[i] = *reinterpret_cast<const uint4*>(q + qoff + (size_t)(t0 + t) * a.DHQK + c);
           uk[i] = *reinterpret_cast<const uint4*>(k + qoff + (size_t)(t0 + t) * a.DHQK + c);
         }
@@ -986,7 +989,7 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
       {
         const int t = tid / (BCV / 8), c = (tid % (BCV / 8)) * 8;
         uint4 uv = make_uint4(0, 0, 0, 0), uh = uv, uo = uv;
-        if (t < Lc) {
+        if (t < Lc && r0 + c < dv) {
           const size_t off = voff + (size_t)(t0 + t) * a.DHV + c;
           uv = *reinterpret_cast<const uint4*>(v + off);
           uh = *reinterpret_cast<const uint4*>(dh + off);
@@ -1071,9 +1074,9 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
       for (int nt = 0; nt < NS; ++nt) {
         const int c = hc * (DK / 2) + 8 * nt + 2 * tq, r = 16 * rt + g;
         float2 x = make_float2(0.f, 0.f), y = x;
-        if (src) {
-          x = *reinterpret_cast<const float2*>(src + soff + (size_t)r * DK + c);
-          y = *reinterpret_cast<const float2*>(src + soff + (size_t)(r + 8) * DK + c);
+        if (src && c < dkr) {
+          if (r0 + r < dv) x = *reinterpret_cast<const float2*>(src + soff + (size_t)r * dkr + c);
+          if (r0 + r + 8 < dv) y = *reinterpret_cast<const float2*>(src + soff + (size_t)(r + 8) * dkr + c);
         }
         st[nt][0] = x.x;
         st[nt][1] = x.y;
@@ -1087,8 +1090,11 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
 #pragma unroll
       for (int nt = 0; nt < NS; ++nt) {
         const int c = hc * (DK / 2) + 8 * nt + 2 * tq, r = 16 * rt + g;
-        const float2 x = *reinterpret_cast<const float2*>(src + soff + (size_t)r * DK + c);
-        const float2 y = *reinterpret_cast<const float2*>(src + soff + (size_t)(r + 8) * DK + c);
+        if (c >= dkr) continue;
+        const float2 x = r0 + r < dv ? *reinterpret_cast<const float2*>(src + soff + (size_t)r * dkr + c)
+                                     : make_float2(0.f, 0.f);
+        const float2 y = r0 + r + 8 < dv ? *reinterpret_cast<const float2*>(src + soff + (size_t)(r + 8) * dkr + c)
+                                         : make_float2(0.f, 0.f);
         part += st[nt][0] * x.x + st[nt][1] * x.y + st[nt][2] * y.x + st[nt][3] * y.y;
       }
       return part;
@@ -1098,7 +1104,7 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
 
     // ------------------------------------------------------------------ phase 1 (forward)
     load_state(a.C0);
-    for (int c = tid; c < DK; c += BCT) nv[c] = (!ret && a.n0) ? a.n0[slice * DK + c] : 0.f;
+    for (int c = tid; c < DK; c += BCT) nv[c] = (!ret && a.n0 && c < dkr) ? a.n0[slice * dkr + c] : 0.f;
     for (int ch = 0; ch < nck; ++ch) {
       const int t0 = ch * BCL, Lc = min(BCL, S - t0);
       state_to_cb();
@@ -1148,7 +1154,7 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
               const float o = Of[t * LDF + r + j], dhv = dHf[t * LDF + r + j];
               dn2[j] = t < Lc ? o * dhv / den : 0.f;
               pp[h2] += o * dhv * hn;
-              if (a.dog && t < Lc) a.dog[voff + (size_t)(t0 + t) * a.DHV + r + j] = dhv * hn;
+              if (a.dog && t < Lc && r0 + r + j < dv) a.dog[voff + (size_t)(t0 + t) * a.DHV + r + j] = dhv * hn;
             }
             *reinterpret_cast<uint32_t*>(dNb + t * LDV + r) = bf2(dn2[0], dn2[1]);
           }
@@ -1233,7 +1239,7 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
           y.z += dd * (At * nv[c + 2] + wk.z);
           y.w += dd * (At * nv[c + 3] + wk.w);
         }
-        *reinterpret_cast<float4*>(a.dq + qoff + (size_t)(t0 + t) * a.DHQK + c) = y;
+        if (c < dkr) *reinterpret_cast<float4*>(a.dq + qoff + (size_t)(t0 + t) * a.DHQK + c) = y;
       }
       {  // state to the chunk end: C' <- A_L C' + (V o w)^T K
         const float AL = eA[Lc - 1];
@@ -1258,7 +1264,7 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
     if (!ret && (a.dC || a.dn)) {
       float part = a.dC ? state_dot(a.dC) : 0.f;
       if (a.dn && rank == 0)
-        for (int c = tid; c < DK; c += BCT) part += a.dn[slice * DK + c] * nv[c];
+        for (int c = tid; c < dkr; c += BCT) part += a.dn[slice * dkr + c] * nv[c];
       const float s2 = cl_block_sum(part, red);
       if (tid == 0) scal[0] += s2;
     }
@@ -1266,7 +1272,7 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
 
     // ------------------------------------------------------------------ phase 2 (backward)
     load_state(a.dC);
-    for (int c = tid; c < DK; c += BCT) nv[c] = (!ret && a.dn) ? a.dn[slice * DK + c] : 0.f;
+    for (int c = tid; c < DK; c += BCT) nv[c] = (!ret && a.dn && c < dkr) ? a.dn[slice * dkr + c] : 0.f;
     for (int ch = nck - 1; ch >= 0; --ch) {
       const int t0 = ch * BCL, Lc = min(BCL, S - t0);
       state_to_cb();  // D entering from the later chunks
@@ -1311,7 +1317,8 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
             const float x0 = acc[nt][2 * h2] + w * acc2[nt][2 * h2];
             const float x1 = acc[nt][2 * h2 + 1] + w * acc2[nt][2 * h2 + 1];
             if (s2 < Lc) {
-              *reinterpret_cast<float2*>(a.dv_out + voff + (size_t)(t0 + s2) * a.DHV + r) = make_float2(x0, x1);
+              if (r0 + r < dv)
+                *reinterpret_cast<float2*>(a.dv_out + voff + (size_t)(t0 + s2) * a.DHV + r) = make_float2(x0, x1);
               const float2 vv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(Vb + s2 * LDV + r));
               dip[h2] += vv.x * x0 + vv.y * x1;
             }
@@ -1372,7 +1379,7 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
           const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kk.y));
           atomicAdd(&tdn[s2], xn.x * k01.x + xn.y * k01.y + xn.z * k23.x + xn.w * k23.y);
         }
-        *reinterpret_cast<float4*>(a.dk_out + qoff + (size_t)(t0 + s2) * a.DHQK + c) = x;
+        if (c < dkr) *reinterpret_cast<float4*>(a.dk_out + qoff + (size_t)(t0 + s2) * a.DHQK + c) = x;
       }
       {  // D <- A_L D + (dN o A)^T Q
         const float AL = eA[Lc - 1];
@@ -1403,16 +1410,19 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
 #pragma unroll
       for (int nt = 0; nt < NS; ++nt) {
         const int c = hc * (DK / 2) + 8 * nt + 2 * tq, r = 16 * rt + g;
-        *reinterpret_cast<float2*>(a.dC0 + soff + (size_t)r * DK + c) = make_float2(st[nt][0], st[nt][1]);
-        *reinterpret_cast<float2*>(a.dC0 + soff + (size_t)(r + 8) * DK + c) = make_float2(st[nt][2], st[nt][3]);
+        if (c >= dkr) continue;
+        if (r0 + r < dv)
+          *reinterpret_cast<float2*>(a.dC0 + soff + (size_t)r * dkr + c) = make_float2(st[nt][0], st[nt][1]);
+        if (r0 + r + 8 < dv)
+          *reinterpret_cast<float2*>(a.dC0 + soff + (size_t)(r + 8) * dkr + c) = make_float2(st[nt][2], st[nt][3]);
       }
     }
     if (!ret) {
       float part = a.C0 ? state_dot(a.C0) : 0.f;
       if (rank == 0)
-        for (int c = tid; c < DK; c += BCT) {
-          if (a.dn0) a.dn0[slice * DK + c] = nv[c];
-          if (a.n0) part += nv[c] * a.n0[slice * DK + c];
+        for (int c = tid; c < dkr; c += BCT) {
+          if (a.dn0) a.dn0[slice * dkr + c] = nv[c];
+          if (a.n0) part += nv[c] * a.n0[slice * dkr + c];
         }
       const float s2 = cl_block_sum(part, red);
       if (tid == 0) scal[1] += s2;
@@ -1450,8 +1460,11 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
 // supported): bf16, block key width 64 / 128 / 256, value width a multiple of 64 up to 512
 int bwd_cluster_size(int dtype, int dk, int dv) {
   if (dtype != 1) return 0;
-  if (dk != 64 && dk != 128 && dk != 256) return 0;
-  if (dv % BCV != 0 || dv / BCV > 8 || dv < BCV) return 0;
+  // key widths 64 / 128 / 256, or narrower (a multiple of 8) run as 64 with zero padding;
+  // value widths a multiple of 64 up to 512, or narrower (a multiple of 8) as one padded CTA
+  if (dk != 64 && dk != 128 && dk != 256 && !(dk < 64 && dk % 8 == 0)) return 0;
+  if (dv < BCV) return dv % 8 == 0 && dk <= 64 ? 1 : 0;
+  if (dv % BCV != 0 || dv / BCV > 8) return 0;
   return dv / BCV;
 }
 
@@ -1522,7 +1535,7 @@ cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream) {
   if (nc > 0) {
     if (a.dk == 256) return launch_cluster_dk<256>(a, BH, nc, stream);
     if (a.dk == 128) return launch_cluster_dk<128>(a, BH, nc, stream);
-    if (a.dk == 64) return launch_cluster_dk<64>(a, BH, nc, stream);
+    if (a.dk <= 64) return launch_cluster_dk<64>(a, BH, nc, stream);
     return cudaErrorInvalidValue;
   }
   const int L = bwd_chunk_len(a.dk, a.dv);

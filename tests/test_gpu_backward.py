@@ -118,14 +118,19 @@ def test_backward_retention_workload_sampled_heads():
 
 
 # ---------------------------------------------------------------- the cluster kernel
-# Blocks whose state does not fit one CTA (bf16, key width 64/128/256, value width a multiple
-# of 64 up to 512): a thread-block cluster per head, 64 value rows per CTA.
+# bf16 blocks of key width 64/128/256 and value width a multiple of 64 up to 512, and narrower
+# blocks zero-padded to 64: a thread-block cluster per head, 64 value rows per CTA.
 @pytest.mark.parametrize("case", [
     # seed, B, NH, S, DHQK, DHV, nb, retention, with_state, with_o, with_dstate
     (11, 1, 2, 200, 256, 512, 1, False, True, True, True),     # the large-head shape, ragged last chunk
     (12, 1, 1, 96, 256, 512, 1, True, True, False, True),      # retention
     (13, 2, 1, 70, 128, 384, 1, False, False, False, False),   # six CTAs per cluster, no state
     (14, 1, 1, 64, 512, 1024, 2, False, True, True, True),     # two blocks of 256 x 512
+    # blocks narrower than 64 keys or values: zero-padded tiles, every global access masked
+    (16, 2, 2, 300, 64, 64, 2, False, True, True, True),       # 32 x 32 (the small block-diagonal shape)
+    (17, 1, 2, 130, 64, 64, 4, False, True, False, True),      # 16 x 16
+    (18, 1, 1, 200, 64, 256, 2, True, True, False, False),     # 32 x 128, retention
+    (19, 2, 1, 100, 128, 64, 2, False, True, True, True),      # 64 x 32
 ])
 def test_backward_cluster_kernel_parity(case):
     seed, B, NH, S, DHQK, DHV, nb, retention, with_state, with_o, with_dstate = case
