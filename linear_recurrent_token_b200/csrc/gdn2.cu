@@ -213,6 +213,83 @@ __global__ void __launch_bounds__(32 * STEP_WARPS) gdn2_step_kernel(Gdn2Args a) 
   }
 }
 
+// The same step with 16-byte state accesses, for V a multiple of 128: a CTA takes 128 value
+// columns of one head, lane = four adjacent columns (a warp covers a 512-byte stretch of a
+// state row), the 8 warps split the key rows; every state load of a thread is issued before
+// the first use.
+template <typename T, int RPW>
+__global__ void __launch_bounds__(32 * STEP_WARPS, 2) gdn2_step_v4_kernel(Gdn2Args a) {
+  constexpr int K = RPW * STEP_WARPS;
+  __shared__ float qs[K], ks[K], es[K], bks[K];
+  __shared__ float4 red[2][STEP_WARPS][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long long bh = blockIdx.y;
+  const int j = blockIdx.x * 128 + 4 * lane;  // first of this lane's four columns
+  const int i0 = warp * RPW;
+  const float* S0 = a.S0 ? a.S0 + bh * K * a.V : nullptr;
+  float4 S[RPW];
+#pragma unroll
+  for (int m = 0; m < RPW; ++m)
+    S[m] = S0 ? *reinterpret_cast<const float4*>(S0 + (size_t)(i0 + m) * a.V + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = threadIdx.x; i < K; i += 32 * STEP_WARPS) {
+    const size_t x = bh * K + i;
+    const float kk = ld_in(static_cast<const T*>(a.k) + x);
+    qs[i] = ld_in(static_cast<const T*>(a.q) + x);
+    ks[i] = kk;
+    es[i] = expf(a.g[x]);
+    bks[i] = a.b[x] * kk;
+  }
+  float4 u;
+  {
+    const float4 wv = *reinterpret_cast<const float4*>(a.w + bh * a.V + j);
+    const T* vp = static_cast<const T*>(a.v) + bh * a.V + j;
+    u = make_float4(wv.x * ld_in(vp), wv.y * ld_in(vp + 1), wv.z * ld_in(vp + 2), wv.w * ld_in(vp + 3));
+  }
+  __syncthreads();
+  float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int m = 0; m < RPW; ++m) {
+    const float e = es[i0 + m], kk = ks[i0 + m];
+    S[m].x *= e, S[m].y *= e, S[m].z *= e, S[m].w *= e;
+    r.x = fmaf(kk, S[m].x, r.x), r.y = fmaf(kk, S[m].y, r.y), r.z = fmaf(kk, S[m].z, r.z), r.w = fmaf(kk, S[m].w, r.w);
+  }
+  red[0][warp][lane] = r;
+  __syncthreads();
+  r = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int x = 0; x < STEP_WARPS; ++x) {
+    const float4 p = red[0][x][lane];
+    r.x += p.x, r.y += p.y, r.z += p.z, r.w += p.w;
+  }
+  float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+  float* So = a.S_out ? a.S_out + bh * K * a.V : nullptr;
+#pragma unroll
+  for (int m = 0; m < RPW; ++m) {
+    const float kk = ks[i0 + m], bk = bks[i0 + m], qq = qs[i0 + m];
+    S[m].x = fmaf(kk, u.x, fmaf(-bk, r.x, S[m].x));
+    S[m].y = fmaf(kk, u.y, fmaf(-bk, r.y, S[m].y));
+    S[m].z = fmaf(kk, u.z, fmaf(-bk, r.z, S[m].z));
+    S[m].w = fmaf(kk, u.w, fmaf(-bk, r.w, S[m].w));
+    y.x = fmaf(qq, S[m].x, y.x), y.y = fmaf(qq, S[m].y, y.y), y.z = fmaf(qq, S[m].z, y.z), y.w = fmaf(qq, S[m].w, y.w);
+    if (So) *reinterpret_cast<float4*>(So + (size_t)(i0 + m) * a.V + j) = S[m];
+  }
+  red[1][warp][lane] = y;
+  __syncthreads();
+  if (warp == 0) {
+    y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int x = 0; x < STEP_WARPS; ++x) {
+      const float4 p = red[1][x][lane];
+      y.x += p.x, y.y += p.y, y.z += p.z, y.w += p.w;
+    }
+    T* op = static_cast<T*>(a.o) + bh * a.V + j;
+    st_out(op, y.x);
+    st_out(op + 1, y.y);
+    st_out(op + 2, y.z);
+    st_out(op + 3, y.w);
+  }
+}
+
 // ------------------------------------------------------------------ chunk (WY block form)
 constexpr int CH_THREADS = 256;
 
@@ -488,6 +565,22 @@ cudaError_t launch_gdn2(const Gdn2Args& a, int mode, int chunk, void* ws, cudaSt
   const long long BH = (long long)a.B * a.H;
   if (BH == 0 || (a.T == 0 && !a.S_out)) return cudaSuccess;
   if (BH > 65535) return cudaErrorInvalidValue;
+  if (mode == 0 && a.T == 1 && a.V % 128 == 0 && a.K <= 128) {  // (K 256 would not fit the registers)
+    const dim3 grid(a.V / 128, (unsigned)BH);
+#define STEP4(RPW)                                                                        \
+  if (a.dtype == 0)                                                                       \
+    gdn2_step_v4_kernel<float, RPW><<<grid, 32 * STEP_WARPS, 0, stream>>>(a);             \
+  else                                                                                    \
+    gdn2_step_v4_kernel<__nv_bfloat16, RPW><<<grid, 32 * STEP_WARPS, 0, stream>>>(a);
+    switch (a.K) {
+      case 32: STEP4(4) break;
+      case 64: STEP4(8) break;
+      case 128: STEP4(16) break;
+      default: return cudaErrorInvalidValue;
+    }
+#undef STEP4
+    return cudaGetLastError();
+  }
   if (mode == 0 && a.T == 1) {
     const dim3 grid((a.V + 31) / 32, (unsigned)BH);
 #define STEP(RPW)                                                                         \

@@ -75,9 +75,11 @@ def test_decode_steps_match_the_prefill():
     check(inp, "bf16", host(torch.cat(outs, dim=2)), host(S))
 
 
-@pytest.mark.parametrize("dtype,K,V,state", [("f32", 64, 40, True), ("bf16", 256, 96, False), ("f32", 32, 32, True)])
+@pytest.mark.parametrize("dtype,K,V,state", [("f32", 64, 40, True), ("bf16", 256, 96, False), ("f32", 32, 32, True),
+                                             ("bf16", 128, 256, True), ("f32", 64, 128, False)])
 def test_decode_step(dtype, K, V, state):
-    """One token per sequence (the decode kernel), state in place, ragged value tile."""
+    """One token per sequence (the decode kernels: 16-byte state accesses when V is a multiple
+    of 128 and K at most 128, else one column per lane), state in place, ragged value tile."""
     inp = inputs.gdn2_inputs(5, 3, 1, K, V, dtype, seed=76, with_state=state)
     o, S = run(inp, dtype, "recurrent", inplace=state)
     check(inp, dtype, o, S)
