@@ -425,6 +425,10 @@ typedef struct {
   mlstm_dtype_t dtype;
   int mode;  /* mlstm_gdn2_mode_t */
   int chunk; /* chunk mode only */
+  /* Bound of every device-side wait of the tensor-core chunk kernels, in SM cycles; 0 = the
+   * default (about two seconds).  A limit shorter than a copy takes makes the call fail with
+   * MLSTM_ERR_TIMEOUT (see mlstm_gdn2_status).  Ignored by the other paths. */
+  long long wait_limit_cycles;
 } mlstm_gdn2_params_t;
 size_t mlstm_gdn2_workspace_size(const mlstm_gdn2_params_t* p);
 mlstm_status_t mlstm_gdn2_fwd(const mlstm_gdn2_params_t* p, const void* q, const void* k, const void* v,

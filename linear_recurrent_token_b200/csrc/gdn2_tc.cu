@@ -531,8 +531,12 @@ struct ScanSmem {
   static constexpr int BYTES = STAGE + Slot<V>::BYTES + (int)sizeof(ScanBars) + 1024;
 };
 
-__device__ __noinline__ bool scan_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  const bool ok = !*abort_flag && mbar_wait(bar, parity, SCAN_WAIT);
+// (a wait that took longer than the limit counts as run out even when the phase completed during
+// a hardware suspension: the limit is the caller's bound on the time spent waiting)
+__device__ __noinline__ bool scan_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                            long long limit) {
+  const long long t0 = clock64();
+  const bool ok = !*abort_flag && mbar_wait(bar, parity, limit) && clock64() - t0 <= limit;
   if (!ok) *abort_flag = 1;
   return __all_sync(0xffffffffu, ok);
 }
@@ -569,8 +573,9 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1) gdn2_tc_scan_kernel(Gdn2Args 
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = tmem_base;
+  const long long wlim = a.wait > 0 ? a.wait : SCAN_WAIT;  // (the drain below keeps the default)
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
-    return __all_sync(0xffffffffu, mbar_test_wait(bar, parity)) || scan_wait_slow(bar, parity, &abort_flag);
+    return __all_sync(0xffffffffu, mbar_test_wait(bar, parity)) || scan_wait_slow(bar, parity, &abort_flag, wlim);
   };
   const uint8_t* slots = ws + (size_t)bh * nch * SL::BYTES;
   int n_issued = 0;

@@ -41,6 +41,7 @@ cudaError_t launch_gn_gate(long long rows, int NH, int S, int DHV, int dtype, co
 // (S0 NULL = zeros, S_out NULL = not written, S_out == S0 in place); o [B,H,T,V] dtype.
 struct Gdn2Args {
   int B, H, T, K, V, dtype;
+  long long wait;  // bound of the tensor-core chunk kernels' waits (SM cycles), 0 = default
   const void *q, *k, *v;
   const float *g, *b, *w;
   const float* S0;

@@ -36,7 +36,8 @@ class StepParams(ctypes.Structure):
 
 class Gdn2Params(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int), ("K", ctypes.c_int),
-                ("V", ctypes.c_int), ("dtype", ctypes.c_int), ("mode", ctypes.c_int), ("chunk", ctypes.c_int)]
+                ("V", ctypes.c_int), ("dtype", ctypes.c_int), ("mode", ctypes.c_int), ("chunk", ctypes.c_int),
+                ("wait_limit_cycles", ctypes.c_longlong)]
 
 
 GDN2_RECURRENT, GDN2_CHUNK = 0, 1
@@ -362,10 +363,10 @@ def gdn2_workspace_size(params: Gdn2Params) -> int:
     return int(lib().mlstm_gdn2_workspace_size(ctypes.byref(params)))
 
 
-def gdn2_params(q, v, mode: str = "recurrent", chunk: int = 64) -> Gdn2Params:
+def gdn2_params(q, v, mode: str = "recurrent", chunk: int = 64, wait_limit_cycles: int = 0) -> Gdn2Params:
     B, H, T, K = q.shape
     return Gdn2Params(int(B), int(H), int(T), int(K), int(v.shape[-1]), _dtype_code(q),
-                      GDN2_CHUNK if mode == "chunk" else GDN2_RECURRENT, int(chunk))
+                      GDN2_CHUNK if mode == "chunk" else GDN2_RECURRENT, int(chunk), int(wait_limit_cycles))
 
 
 def gdn2_status(q, v, workspace, *, mode: str = "chunk", chunk: int = 64, stream=None) -> int:
@@ -376,13 +377,13 @@ def gdn2_status(q, v, workspace, *, mode: str = "chunk", chunk: int = 64, stream
 
 
 def gdn2_fwd(q, k, v, g, b, w, S0=None, *, mode: str = "recurrent", chunk: int = 64, o=None, S_out=None,
-             return_state: bool = True, workspace=None, stream=None):
+             return_state: bool = True, workspace=None, stream=None, wait_limit_cycles: int = 0):
     """Gated DeltaNet-2 (mlstm_gdn2_fwd): q, k [B,H,T,K], v [B,H,T,V] (fp32 or bf16); g, b
     [B,H,T,K] and w [B,H,T,V] fp32; S0 [B,H,K,V] fp32 or None.  mode "recurrent" or "chunk".
     S_out may be S0 (in place: the decode step).  Returns (o, S_out)."""
     B, H, T, K = q.shape
     V = v.shape[-1]
-    p = gdn2_params(q, v, mode, chunk)
+    p = gdn2_params(q, v, mode, chunk, wait_limit_cycles)
     if o is None:
         o = torch.empty((B, H, T, V), dtype=q.dtype, device=q.device)
     if return_state and S_out is None:

@@ -61,6 +61,10 @@ def test_params_struct_matches_header_layout():
     assert ctypes.sizeof(mlstm.FwdParams) == 48
     assert mlstm.FwdParams.wait_limit_cycles.offset == 40
     assert mlstm.fwd_params(1, 1, 1, 16, 16).wait_limit_cycles == 0
+    # GDN-2: eight ints, then its wait limit at offset 32
+    assert ctypes.sizeof(mlstm.Gdn2Params) == 40
+    assert mlstm.Gdn2Params.wait_limit_cycles.offset == 32
+    assert mlstm.Gdn2Params(1, 1, 1, 128, 128, 1, 1, 64).wait_limit_cycles == 0
 
 
 def test_status_calls_validate_before_touching_the_device():

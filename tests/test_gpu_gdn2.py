@@ -137,3 +137,23 @@ def test_chunk_tensor_core_prefill_workload_sampled():
     errs = {"o": slice_relerr(o[:1], o_ref, 2), "S": slice_relerr(S[:1], S_ref, 2)}
     assert all(e <= TOL["bf16"] for e in errs.values()), errs
     assert np.isfinite(o).all() and np.isfinite(S).all()
+
+
+def test_chunk_tensor_core_wait_limit_reports_timeout_then_workspace_is_reusable():
+    """A wait bound of 256 SM cycles (shorter than any copy): the scan's first wait runs out, the
+    kernel drains its copies and returns, the status call reports MLSTM_ERR_TIMEOUT promptly, and
+    a normal call on the same workspace then matches the oracle."""
+    import time
+    inp = inputs.gdn2_inputs(1, 2, 300, 128, 128, "bf16", seed=88)
+    td = torch.bfloat16
+    q, k, v = dev(inp["q"], td), dev(inp["k"], td), dev(inp["v"], td)
+    g, b, w, S0 = dev(inp["g"]), dev(inp["b"]), dev(inp["w"]), dev(inp["S0"])
+    ws = torch.empty(mlstm.gdn2_workspace_size(mlstm.gdn2_params(q, v, "chunk", 64)), dtype=torch.uint8,
+                     device="cuda")
+    t0 = time.time()
+    mlstm.gdn2_fwd(q, k, v, g, b, w, S0, mode="chunk", chunk=64, workspace=ws, wait_limit_cycles=256)
+    assert mlstm.gdn2_status(q, v, ws) == 8
+    assert time.time() - t0 < 5.0
+    o, S = mlstm.gdn2_fwd(q, k, v, g, b, w, S0, mode="chunk", chunk=64, workspace=ws)
+    assert mlstm.gdn2_status(q, v, ws) == 0
+    check(inp, "bf16", host(o), host(S))
