@@ -439,7 +439,9 @@ mlstm_status_t mlstm_gdn2_fwd(const mlstm_gdn2_params_t* p, const void* q, const
  * wait of the tensor-core chunk kernels ran out (that call's o and S_out are unspecified; the
  * workspace can be used again); MLSTM_OK always for the other paths, which have no such waits.
  * MLSTM_ERR_CUDA if the synchronisation or the read fails; argument errors as mlstm_gdn2_fwd
- * (workspace NULL: MLSTM_ERR_NULL when the tensor-core path would run). */
+ * (workspace NULL: MLSTM_ERR_NULL when the tensor-core path would run).  In the bounds-checked
+ * build (see mlstm_bounds_checked) a failed check gives MLSTM_ERR_BOUNDS, with the first failure
+ * at bytes 16..39 of the workspace as {int site; int count; long long index; long long extent}. */
 mlstm_status_t mlstm_gdn2_status(const mlstm_gdn2_params_t* p, const void* workspace, mlstm_stream_t stream);
 
 /*

@@ -14,7 +14,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmlstm.so")
 LIB_CHECKED = os.path.join(PKG, "libmlstm_checked.so")
 # sources whose objects differ in the bounds-checked build (the others are linked as they are)
-CHECKED_SOURCES = ("chunkwise_tc.cu", "mlstm_api.cu")
+CHECKED_SOURCES = ("chunkwise_tc.cu", "gdn2_tc.cu", "mlstm_api.cu")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -1,14 +1,15 @@
-// Bounds-checked debug build of the tensor-core prefill.
+// Bounds-checked debug build of the tensor-core kernels.
 //
-// Compiled with -DMLSTM_BOUNDS_CHECK (the library libmlstm_checked.so), the gate preparation,
-// segment-summary and walk kernels check, before making it, every plain global access against
-// the extent of its buffer and every TMA copy's coordinates against the copy rules (the
-// innermost coordinate on a 16-byte boundary, a store from non-negative coordinates, a box that
-// overlaps its tensor), and every staging-tile offset of the h store against the tile.  A
-// failing check skips the access, sets bit 2 (value 4) of the workspace error word and records
-// the first failure (site, index, extent) at bytes 16..39 of the workspace; the call's status
-// is then MLSTM_ERR_BOUNDS.  Nothing traps.  In the normal build every check is the constant
-// true and compiles away.
+// Compiled with -DMLSTM_BOUNDS_CHECK (the library libmlstm_checked.so), the mLSTM prefill's gate
+// preparation, segment-summary and walk kernels and the GDN-2 chunk kernels check, before making
+// it, every plain global access against the extent of its buffer, every TMA copy's coordinates
+// against the copy rules (the innermost coordinate on a 16-byte boundary, a store from
+// non-negative coordinates, a box that overlaps its tensor) and every staging-tile offset of the
+// h store against the tile.  A failing check skips the access, sets bit 2 (value 4) of the
+// workspace error word and records the first failure (site, index, extent) at bytes 16..39 of
+// the workspace (the GDN-2 kernels: of their own workspace's header); the call's status is then
+// MLSTM_ERR_BOUNDS.  Nothing traps.  In the normal build every check is the constant true and
+// compiles away.
 #pragma once
 
 namespace mlstm {
@@ -33,6 +34,11 @@ enum BoundsSite : int {
   BS_WALK_H_TMA = 15,    // h tile stores
   BS_WALK_FINAL = 16,    // C_out / n_out / m_out written
   BS_WALK_BIAS = 17,     // scalar-normaliser bias read
+  BS_GDN_INPUT = 18,     // GDN-2 chunk prep: q, k, g, b, v, w rows read
+  BS_GDN_SLOT = 19,      // GDN-2 chunk prep: writes into the chunk's workspace slot
+  BS_GDN_COPY = 20,      // GDN-2 chunk scan: slot copied into a stage
+  BS_GDN_STATE = 21,     // GDN-2 chunk scan: S0 read, S_out written
+  BS_GDN_OUT = 22,       // GDN-2 chunk scan: o written
 };
 
 struct BoundsRecord {

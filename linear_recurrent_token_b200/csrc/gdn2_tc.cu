@@ -25,6 +25,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "bounds.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -123,7 +124,7 @@ struct PrepSmem {
 
 // One CTA per (chunk, batch x head): the chunk's slot (see Slot).
 template <int V>
-__global__ void __launch_bounds__(PREP_THREADS, 1) gdn2_tc_prep_kernel(Gdn2Args a, uint8_t* ws) {
+__global__ void __launch_bounds__(PREP_THREADS, 1) gdn2_tc_prep_kernel(Gdn2Args a, uint8_t* ws, unsigned int* err) {
   using SM = PrepSmem<V>;
   using SL = Slot<V>;
   constexpr int VP = SM::VP;
@@ -171,7 +172,7 @@ __global__ void __launch_bounds__(PREP_THREADS, 1) gdn2_tc_prep_kernel(Gdn2Args 
       const int e = tid + x * PREP_THREADS, t = e / (TK / 4), i = 4 * (e % (TK / 4));
       gv[x] = bv[x] = make_float4(0.f, 0.f, 0.f, 0.f);
       kr[x] = qr[x] = make_uint2(0u, 0u);
-      if (t < Lc) {
+      if (t < Lc && in_bounds(err, BS_GDN_INPUT, (long long)(tok0 + t) * TK + i + 3, (long long)a.B * a.H * a.T * TK)) {
         gv[x] = *reinterpret_cast<const float4*>(g + (size_t)t * TK + i);
         bv[x] = *reinterpret_cast<const float4*>(b + (size_t)t * TK + i);
         kr[x] = *reinterpret_cast<const uint2*>(k + (size_t)t * TK + i);
@@ -183,7 +184,7 @@ __global__ void __launch_bounds__(PREP_THREADS, 1) gdn2_tc_prep_kernel(Gdn2Args 
       const int e = tid + x * PREP_THREADS, t = e / (V / 4), j = 4 * (e % (V / 4));
       wv[x] = make_float4(0.f, 0.f, 0.f, 0.f);
       vr[x] = make_uint2(0u, 0u);
-      if (t < Lc) {
+      if (t < Lc && in_bounds(err, BS_GDN_INPUT, (long long)(tok0 + t) * V + j + 3, (long long)a.B * a.H * a.T * V)) {
         wv[x] = *reinterpret_cast<const float4*>(w + (size_t)t * V + j);
         vr[x] = *reinterpret_cast<const uint2*>(v + (size_t)t * V + j);
       }
@@ -252,7 +253,8 @@ __global__ void __launch_bounds__(PREP_THREADS, 1) gdn2_tc_prep_kernel(Gdn2Args 
       nb[j] = pack2(-bk.x * f0, -bk.y * f1);
     }
     *reinterpret_cast<uint4*>(Kd + t * KP + col) = make_uint4(kd[0], kd[1], kd[2], kd[3]);
-    *reinterpret_cast<uint4*>(slot + SL::KT + tile_chunk(t, col)) = make_uint4(kt[0], kt[1], kt[2], kt[3]);
+    if (in_bounds(err, BS_GDN_SLOT, SL::KT + tile_chunk(t, col) + 15, SL::NBT))
+      *reinterpret_cast<uint4*>(slot + SL::KT + tile_chunk(t, col)) = make_uint4(kt[0], kt[1], kt[2], kt[3]);
     // nBt transposed (rows = key channels, 64 tokens wide: a K-major operand) staged where Wk
     // will be, in the slot's swizzled layout
 #pragma unroll
@@ -265,7 +267,8 @@ __global__ void __launch_bounds__(PREP_THREADS, 1) gdn2_tc_prep_kernel(Gdn2Args 
   }
   for (int e = bt; e < TL * V / 8; e += BT) {
     const int t = e / (V / 8), col = 8 * (e % (V / 8));
-    *reinterpret_cast<uint4*>(slot + SL::U + tile_chunk(t, col)) = *reinterpret_cast<const uint4*>(Ub + t * VP + col);
+    if (in_bounds(err, BS_GDN_SLOT, SL::U + tile_chunk(t, col) + 15, SL::UR))
+      *reinterpret_cast<uint4*>(slot + SL::U + tile_chunk(t, col)) = *reinterpret_cast<const uint4*>(Ub + t * VP + col);
   }
   for (int i = bt; i < TK; i += BT) reinterpret_cast<float*>(slot + SL::EGL)[i] = __expf(GLr[i]);
   }
@@ -493,11 +496,13 @@ __global__ void __launch_bounds__(PREP_THREADS, 1) gdn2_tc_prep_kernel(Gdn2Args 
   // Wk, Qw (swizzled tiles), Ur and Ou into the slot
   for (int e = tid; e < TL * TK / 8; e += PREP_THREADS) {
     const int t = e >> 4, col = 8 * (e & 15);
+    if (!in_bounds(err, BS_GDN_SLOT, SL::QW + tile_chunk(t, col) + 15, SL::KT)) continue;
     *reinterpret_cast<uint4*>(slot + SL::WK + tile_chunk(t, col)) = *reinterpret_cast<const uint4*>(Wkb + t * KP + col);
     *reinterpret_cast<uint4*>(slot + SL::QW + tile_chunk(t, col)) = *reinterpret_cast<const uint4*>(Kd + t * KP + col);
   }
   for (int e = tid; e < TL * V / 8; e += PREP_THREADS) {
     const int t = e / (V / 8), col = 8 * (e % (V / 8));
+    if (!in_bounds(err, BS_GDN_SLOT, SL::OU + (t * V + col) * 2 + 15, SL::EGL)) continue;
     *reinterpret_cast<uint4*>(slot + SL::UR + (t * V + col) * 2) = *reinterpret_cast<const uint4*>(Urb + t * VP + col);
     *reinterpret_cast<uint4*>(slot + SL::OU + (t * V + col) * 2) = *reinterpret_cast<const uint4*>(Y1b + t * VP + col);
   }
@@ -587,7 +592,8 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1) gdn2_tc_scan_kernel(Gdn2Args 
       if (!wait(&bars.empty[b], ((c >> 1) & 1) ^ 1)) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(&bars.full[b], SL::BYTES);
-        bulk_load(sm + b * STAGE, slots + (size_t)c * SL::BYTES, SL::BYTES, &bars.full[b]);
+        if (in_bounds(err, BS_GDN_COPY, c, nch))
+          bulk_load(sm + b * STAGE, slots + (size_t)c * SL::BYTES, SL::BYTES, &bars.full[b]);
       }
       n_issued = c + 1;
       __syncwarp();
@@ -646,7 +652,10 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1) gdn2_tc_scan_kernel(Gdn2Args 
       float r[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j)
-        r[j] = (row >= 0 && a.S0) ? a.S0[((size_t)bh * TK + i0 + j) * V + row] : 0.f;
+        r[j] = (row >= 0 && a.S0 &&
+                in_bounds(err, BS_GDN_STATE, ((long long)bh * TK + i0 + j) * V + row, (long long)a.B * a.H * TK * V))
+                   ? a.S0[((size_t)bh * TK + i0 + j) * V + row]
+                   : 0.f;
       tmem_st16(tm + lo + TM_S + i0, r);
     }
     tmem_wait_st();
@@ -710,7 +719,9 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1) gdn2_tc_scan_kernel(Gdn2Args 
         tmem_wait_ld();
         if (row >= 0 && !abort_flag)
 #pragma unroll
-          for (int j = 0; j < 32; ++j) a.S_out[((size_t)bh * TK + i0 + j) * V + row] = r[j];
+          for (int j = 0; j < 32; ++j)
+            if (in_bounds(err, BS_GDN_STATE, ((long long)bh * TK + i0 + j) * V + row, (long long)a.B * a.H * TK * V))
+              a.S_out[((size_t)bh * TK + i0 + j) * V + row] = r[j];
       }
     }
   } else {
@@ -735,7 +746,8 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1) gdn2_tc_scan_kernel(Gdn2Args 
       if (row >= 0 && !abort_flag)
 #pragma unroll
         for (int t = 0; t < TL; ++t)
-          if (t < Lc) o[(size_t)(t0 + t) * V + row] = __float2bfloat16_rn(r[t] + __bfloat162float(ou[t * V + row]));
+          if (t < Lc && in_bounds(err, BS_GDN_OUT, ((long long)bh * a.T + t0 + t) * V + row, (long long)a.B * a.H * a.T * V))
+            o[(size_t)(t0 + t) * V + row] = __float2bfloat16_rn(r[t] + __bfloat162float(ou[t * V + row]));
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.empty[b]);
     }
@@ -766,14 +778,15 @@ cudaError_t launch_tc_v(const Gdn2Args& a, void* ws, cudaStream_t stream) {
   const int nch = (a.T + TL - 1) / TL;
   unsigned int* err = static_cast<unsigned int*>(ws);
   uint8_t* slots = static_cast<uint8_t*>(ws) + GDN2_TC_HEADER;
-  cudaError_t e = cudaMemsetAsync(err, 0, sizeof(unsigned int), stream);
+  // the error word and, for the bounds-checked build, its record (bytes 16..39)
+  cudaError_t e = cudaMemsetAsync(err, 0, 64, stream);
   if (e != cudaSuccess) return e;
   const int smem_p = PrepSmem<V>::BYTES, smem_s = ScanSmem<V>::BYTES;
   e = cudaFuncSetAttribute(gdn2_tc_prep_kernel<V>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_p);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(gdn2_tc_scan_kernel<V>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_s);
   if (e != cudaSuccess) return e;
-  gdn2_tc_prep_kernel<V><<<dim3((unsigned)nch, (unsigned)BH), PREP_THREADS, smem_p, stream>>>(a, slots);
+  gdn2_tc_prep_kernel<V><<<dim3((unsigned)nch, (unsigned)BH), PREP_THREADS, smem_p, stream>>>(a, slots, err);
   gdn2_tc_scan_kernel<V><<<(unsigned)BH, SCAN_THREADS, smem_s, stream>>>(a, slots, err, nch);
   return cudaGetLastError();
 }

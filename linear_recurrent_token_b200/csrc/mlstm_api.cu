@@ -897,7 +897,7 @@ mlstm_status_t mlstm_gdn2_status(const mlstm_gdn2_params_t* p, const void* works
   if (!tc) return MLSTM_OK;  // no bounded waits ran
   unsigned int word = 0;
   if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return MLSTM_ERR_CUDA;
-  return word == 0 ? MLSTM_OK : MLSTM_ERR_TIMEOUT;
+  return word == 0 ? MLSTM_OK : (word & 4u) ? MLSTM_ERR_BOUNDS : MLSTM_ERR_TIMEOUT;
 }
 
 mlstm_status_t mlstm_gdn2_fwd(const mlstm_gdn2_params_t* p, const void* q, const void* k, const void* v,

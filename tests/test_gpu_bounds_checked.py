@@ -129,3 +129,23 @@ def test_normal_build_reports_no_record():
     ws = torch.zeros(mlstm.workspace_size(p), dtype=torch.uint8, device="cuda")
     assert mlstm.lib().mlstm_bounds_checked() == 0
     assert mlstm.bounds_record(p, ws) == (0, 0, 0)
+
+
+@pytest.mark.parametrize("B,H,T,V", [(2, 3, 200, 128), (1, 2, 130, 64)])
+def test_checked_build_gdn2_chunk_finds_no_bad_access(B, H, T, V):
+    """The GDN-2 chunk kernels on the tensor cores through the checked build: status OK, an
+    empty failure record at bytes 16..39 of the workspace, oracle parity."""
+    inp = inputs.gdn2_inputs(B, H, T, 128, V, "bf16", seed=90 + T)
+    td = torch.bfloat16
+    with mlstm.bounds_checked():
+        q, v = dev(inp["q"], td), dev(inp["v"], td)
+        ws = torch.zeros(mlstm.gdn2_workspace_size(mlstm.gdn2_params(q, v, "chunk", 64)), dtype=torch.uint8,
+                         device="cuda")
+        o, S = mlstm.gdn2_fwd(q, dev(inp["k"], td), v, dev(inp["g"]), dev(inp["b"]), dev(inp["w"]), dev(inp["S0"]),
+                              mode="chunk", chunk=64, workspace=ws)
+        st = mlstm.gdn2_status(q, v, ws)
+    rec = ws[16:40].cpu().numpy().view(np.int32)
+    assert st == 0 and rec[1] == 0, (mlstm.status_string(st), rec)
+    o_ref, S_ref = oracle.gdn2_sequential(inp["q"], inp["k"], inp["v"], inp["g"], inp["b"], inp["w"], inp["S0"])
+    errs = {"o": slice_relerr(host(o), o_ref, 2), "S": slice_relerr(host(S), S_ref, 2)}
+    assert all(e <= TOL["bf16"] for e in errs.values()), errs
