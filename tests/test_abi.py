@@ -374,3 +374,37 @@ def test_header_is_plain_c(tmp_path):
     r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", f"{ROOT}/include",
                         "-fsyntax-only", str(src)], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+@pytest.mark.parametrize("shape", [
+    # B, NH, S, DHQK, DHV, nb, retention
+    (1, 8, 8192, 256, 512, 1, False),   # the large head
+    (8, 8, 2048, 64, 64, 1, True),      # the retention workload
+    (4, 4, 512, 64, 64, 2, False),      # 32 x 32 blocks (zero-padded tiles)
+    (1, 2, 1000, 128, 256, 1, False),
+    (2, 3, 70, 64, 64, 1, False),       # two chunks, ragged
+    (1, 1, 64, 32, 32, 2, False),       # one chunk of 16 x 16 blocks
+    (1, 4, 20000, 128, 128, 1, False),  # many short segments
+])
+def test_tensor_core_plan_covers_the_sequence(shape):
+    """The tensor-core plan (host logic, no GPU): segments cover the chunks once, the last segment
+    is not empty, one summary unit per segment but the last (segment 0 may be split in two), the
+    walk's CTAs (value tiles x slices x heads x segments) fit the 148 SMs of a B200 when there is
+    more than one segment, and the workspace holds the summaries."""
+    B, NH, S, DHQK, DHV, nb, retention = shape
+    p = mlstm.fwd_params(B, NH, S, DHQK, DHV, 64, nb, torch.bfloat16, retention)
+    pl = mlstm.plan(p)
+    assert pl["tensor_core"] == 1, pl
+    chunks = (S + 63) // 64
+    G, s0, s = pl["segments"], pl["seg0_chunks"], pl["seg_chunks"]
+    assert G >= 1
+    if G > 1:
+        assert s0 + (G - 2) * s < chunks <= s0 + (G - 1) * s, pl
+        assert pl["summary_units"] >= G - 1 and pl["summary_units"] <= G, pl
+    else:
+        assert pl["summary_units"] == 0
+    dk, dv = DHQK // nb, DHV // nb
+    tiles = -(-dv // pl["dv_tile"])
+    assert pl["ctas_main"] == B * NH * nb * tiles * G
+    assert pl["ctas_main"] <= 148 or G == 1
+    assert pl["workspace_bytes"] >= B * NH * nb * pl["summary_units"] * dv * dk * 4
