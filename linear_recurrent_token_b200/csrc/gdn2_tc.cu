@@ -209,6 +209,25 @@ __global__ void __launch_bounds__(PREP_THREADS, 1) gdn2_tc_prep_kernel(Gdn2Args 
     }
   }
   __syncthreads();
+  // The CTAs run one per SM, in waves: the inputs of the chunk of the CTA one wave later (block
+  // index + the SM count) are prefetched into L2 while this chunk is computed, so that CTA's
+  // loads above find them there instead of all CTAs of a wave fetching from HBM at once.
+  if (warp == 0 && lane < 6 && a.nsm > 0) {
+    const long long nid = (long long)blockIdx.y * gridDim.x + blockIdx.x + a.nsm;
+    if (nid < (long long)gridDim.x * gridDim.y) {
+      const int t2 = (int)(nid % gridDim.x) * TL;
+      const size_t tok2 = (size_t)(nid / gridDim.x) * a.T + t2;
+      const uint32_t rows = (uint32_t)min(TL, a.T - t2);
+      const void* src = lane == 0 ? (const void*)(static_cast<const __nv_bfloat16*>(a.q) + tok2 * TK)
+                        : lane == 1 ? (const void*)(static_cast<const __nv_bfloat16*>(a.k) + tok2 * TK)
+                        : lane == 2 ? (const void*)(static_cast<const __nv_bfloat16*>(a.v) + tok2 * V)
+                        : lane == 3 ? (const void*)(a.g + tok2 * TK)
+                        : lane == 4 ? (const void*)(a.b + tok2 * TK)
+                                    : (const void*)(a.w + tok2 * V);
+      const uint32_t row_bytes = lane < 2 ? TK * 2 : lane == 2 ? V * 2 : lane < 5 ? TK * 4 : V * 4;
+      prefetch_l2_bulk(src, rows * row_bytes);
+    }
+  }
   {  // G: cumulative sums down each key channel, four threads per channel (16 rows each)
     const int i = tid & (TK - 1), part = tid >> 7;
     float run = 0.f;
@@ -786,7 +805,11 @@ cudaError_t launch_tc_v(const Gdn2Args& a, void* ws, cudaStream_t stream) {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(gdn2_tc_scan_kernel<V>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_s);
   if (e != cudaSuccess) return e;
-  gdn2_tc_prep_kernel<V><<<dim3((unsigned)nch, (unsigned)BH), PREP_THREADS, smem_p, stream>>>(a, slots, err);
+  Gdn2Args pa = a;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&pa.nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    pa.nsm = 0;  // no prefetch
+  gdn2_tc_prep_kernel<V><<<dim3((unsigned)nch, (unsigned)BH), PREP_THREADS, smem_p, stream>>>(pa, slots, err);
   gdn2_tc_scan_kernel<V><<<(unsigned)BH, SCAN_THREADS, smem_s, stream>>>(a, slots, err, nch);
   return cudaGetLastError();
 }

@@ -42,6 +42,7 @@ cudaError_t launch_gn_gate(long long rows, int NH, int S, int DHV, int dtype, co
 struct Gdn2Args {
   int B, H, T, K, V, dtype;
   long long wait;  // bound of the tensor-core chunk kernels' waits (SM cycles), 0 = default
+  int nsm;         // SMs of the device (set by the tensor-core chunk launcher)
   const void *q, *k, *v;
   const float *g, *b, *w;
   const float* S0;

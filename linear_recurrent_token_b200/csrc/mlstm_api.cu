@@ -930,6 +930,7 @@ mlstm_status_t mlstm_gdn2_fwd(const mlstm_gdn2_params_t* p, const void* q, const
   Gdn2Args a;
   a.B = p->B, a.H = p->H, a.T = p->T, a.K = p->K, a.V = p->V, a.dtype = p->dtype == MLSTM_BF16 ? 1 : 0;
   a.wait = p->wait_limit_cycles > 0 ? p->wait_limit_cycles : 0;
+  a.nsm = 0;
   a.q = q, a.k = k, a.v = v, a.g = g, a.b = b, a.w = w, a.S0 = S0, a.o = o, a.S_out = S_out;
   if (p->T == 0) {  // the final state is the initial state
     cudaError_t e = cudaSuccess;
