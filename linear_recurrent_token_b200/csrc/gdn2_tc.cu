@@ -52,6 +52,10 @@ struct Slot {
                        OU = UR + V * 128, EGL = OU + V * 128, BYTES = EGL + TK * 4;
 };
 
+// `bytes` (a multiple of 16) of global memory from `src` (16-byte aligned) into L2, no completion
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&h);
