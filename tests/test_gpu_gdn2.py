@@ -100,6 +100,8 @@ def test_empty_sequence_copies_the_state():
     (2, 2, 1, 128, False, False),    # a single token
     (1, 2, 700, 64, True, False),    # eleven chunks, V = 64
     (3, 2, 1000, 128, True, True),   # sixteen chunks, in place
+    (2, 80, 130, 128, True, False),  # 480 chunk CTAs (several waves: each prefetches a later CTA's
+                                     # inputs into L2), ragged last chunks of two tokens
 ])
 def test_chunk_tensor_core(B, H, T, V, state, inplace):
     inp = inputs.gdn2_inputs(B, H, T, 128, V, "bf16", seed=80 + T, with_state=state)
