@@ -895,7 +895,8 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
   const int NC = (int)cl.num_blocks(), rank = (int)cl.block_rank();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tq = lane & 3;
-  const int bh = blockIdx.y, head = bh % a.NH;
+  // one cluster per (batch x head, block): the blocks of a head run side by side
+  const int bh = blockIdx.y, blk = blockIdx.z, head = bh % a.NH;
   const int dv = a.dv, S = a.S, r0 = rank * BCV;
   const bool ret = a.retention != 0;
   const bf16_t* q = static_cast<const bf16_t*>(a.q);
@@ -903,14 +904,19 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
   const bf16_t* v = static_cast<const bf16_t*>(a.v);
   const bf16_t* dh = static_cast<const bf16_t*>(a.dh);
   const bf16_t* og = ret ? nullptr : static_cast<const bf16_t*>(a.og);
-  float* wlf = a.ws + (size_t)bh * 8 * S;
+  // workspace (bwd_workspace_bytes): per (batch x head, block) the gate logs and the per-token
+  // values of phase 1; per batch x head the forget / input gate gradient sums (zeroed before the
+  // launch, added to by every block); per (batch x head, block) the block's final-state terms
+  const size_t nbh = (size_t)a.B * a.NH;
+  float* wlf = a.ws + ((size_t)bh * a.nb + blk) * 6 * S;
   float* wli = wlf + S;
   float* wm = wli + S;
-  float* wr = wm + S;
-  float* wdi = wr + S;
-  float* wden = wdi + S;
+  float* wden = wm + S;
   float* wd = wden + S;
   float* wdd = wd + S;
+  float* wr = a.ws + nbh * a.nb * 6 * S + (size_t)bh * 2 * S;
+  float* wdi = wr + S;
+  float* wsc = a.ws + nbh * a.nb * 6 * S + nbh * 2 * S + ((size_t)bh * a.nb + blk) * 2;
   // this warp's share of the state: rows 16 rt .. +16, key columns hc DK/2 .. +DK/2
   const int rt = warp & 3, hc = warp >> 2;
   float st[NS][4];
@@ -950,10 +956,6 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
         }
       }
     }
-    for (int t = tid; t < S; t += BCT) {
-      wr[t] = 0.f;
-      wdi[t] = 0.f;
-    }
   }
   if (tid == 0) {
     scal[0] = 0.f;
@@ -962,7 +964,7 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
   cl.sync();
 
   const int nck = (S + BCL - 1) / BCL;
-  for (int blk = 0; blk < a.nb; ++blk) {
+  {
     const size_t slice = (size_t)bh * a.nb + blk;
     // (blocks narrower than DK key columns or BCV value rows run zero-padded: every global
     // access below is masked to the block's dk x dv)
@@ -1429,31 +1431,50 @@ __global__ void __launch_bounds__(BCT, 1) bwd_cluster_kernel(BwdArgs a) {
     }
     cl.sync();
   }
-  // ---- gate gradients (rank 0): dlf_t = sum_{tau >= t} r_tau + the final-state term
-  if (!ret && rank == 0 && warp == 0) {
+  // ---- this block's final-state terms (summed over the cluster) for the gate gradients, which
+  // bwd_gate_grad_kernel forms once every block of the head is done
+  if (rank == 0 && tid == 0) {
     float sc2 = 0.f, sc3 = 0.f;
     for (int i = 0; i < NC; ++i) {
       sc2 += cl.map_shared_rank(scal, i)[0];
       sc3 += cl.map_shared_rank(scal, i)[1];
     }
-    const int seg = (S + 31) / 32, t_lo = lane * seg, t_hi = min(S, t_lo + seg);
-    float sum = 0.f;
-    for (int t = t_lo; t < t_hi; ++t) sum += wr[t];
-    float later = sum;
-    for (int o = 1; o < 32; o <<= 1) {
-      const float y = __shfl_down_sync(0xffffffffu, later, o);
-      if (lane + o < 32) later += y;
-    }
-    float acc = later - sum + sc2;
-    for (int t = t_hi - 1; t >= t_lo; --t) {
-      acc += wr[t];
-      const float ft = a.fg[(size_t)bh * S + t];
-      if (a.dfg) a.dfg[(size_t)bh * S + t] = acc / (1.f + expf(ft));
-      if (a.dig) a.dig[(size_t)bh * S + t] = wdi[t];
-    }
-    if (lane == 0 && a.dm0) a.dm0[bh] = sc3;
+    wsc[0] = sc2;
+    wsc[1] = sc3;
   }
   cl.sync();  // no CTA leaves while rank 0 may still read its shared memory
+}
+
+// Gate gradients of the cluster kernel, one warp per batch x head, after every block of the head:
+// dlf_t = sum_{tau >= t} r_tau + the final-state terms (summed over the blocks), the forget-gate
+// pre-activation gradient dlf_t sigmoid(-f_t), the input-gate gradient and dm0.
+__global__ void __launch_bounds__(32) bwd_gate_grad_kernel(BwdArgs a) {
+  const int bh = blockIdx.x, lane = threadIdx.x, S = a.S;
+  const size_t nbh = (size_t)a.B * a.NH;
+  const float* wr = a.ws + nbh * a.nb * 6 * S + (size_t)bh * 2 * S;
+  const float* wdi = wr + S;
+  const float* wsc = a.ws + nbh * a.nb * 6 * S + nbh * 2 * S + (size_t)bh * a.nb * 2;
+  float sc2 = 0.f, sc3 = 0.f;
+  for (int b = 0; b < a.nb; ++b) {
+    sc2 += wsc[2 * b];
+    sc3 += wsc[2 * b + 1];
+  }
+  const int seg = (S + 31) / 32, t_lo = lane * seg, t_hi = min(S, t_lo + seg);
+  float sum = 0.f;
+  for (int t = t_lo; t < t_hi; ++t) sum += wr[t];
+  float later = sum;
+  for (int o = 1; o < 32; o <<= 1) {
+    const float y = __shfl_down_sync(0xffffffffu, later, o);
+    if (lane + o < 32) later += y;
+  }
+  float acc = later - sum + sc2;
+  for (int t = t_hi - 1; t >= t_lo; --t) {
+    acc += wr[t];
+    const float ft = a.fg[(size_t)bh * S + t];
+    if (a.dfg) a.dfg[(size_t)bh * S + t] = acc / (1.f + expf(ft));
+    if (a.dig) a.dig[(size_t)bh * S + t] = wdi[t];
+  }
+  if (lane == 0 && a.dm0) a.dm0[bh] = sc3;
 }
 
 // value rows per CTA of the cluster kernel, and its cluster size for these widths (0: not
@@ -1474,7 +1495,7 @@ cudaError_t launch_cluster_dk(const BwdArgs& a, long long BH, int nc, cudaStream
   cudaError_t e = cudaFuncSetAttribute(bwd_cluster_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)nc, (unsigned)BH, 1);
+  cfg.gridDim = dim3((unsigned)nc, (unsigned)BH, (unsigned)a.nb);
   cfg.blockDim = dim3(BCT, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -1485,7 +1506,14 @@ cudaError_t launch_cluster_dk(const BwdArgs& a, long long BH, int nc, cudaStream
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, bwd_cluster_kernel<DK>, a);
+  // the gate-gradient sums that every block adds to start at zero
+  const size_t nbh = (size_t)BH;
+  e = cudaMemsetAsync(a.ws + nbh * a.nb * 6 * a.S, 0, nbh * 2 * a.S * sizeof(float), stream);
+  if (e != cudaSuccess) return e;
+  e = cudaLaunchKernelEx(&cfg, bwd_cluster_kernel<DK>, a);
+  if (e != cudaSuccess || a.retention) return e;
+  bwd_gate_grad_kernel<<<(unsigned)BH, 32, 0, stream>>>(a);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -1494,7 +1522,13 @@ size_t bwd_smem_bytes(int dk, int dv) {
   return ((size_t)dv * (dk + 1) + 4 * (size_t)dk + 5 * (size_t)dv + NTB / 32 + NTB) * sizeof(float);
 }
 
-size_t bwd_workspace_bytes(long long BH, int S) { return (size_t)BH * 8 * (size_t)S * sizeof(float); }
+// the SIMT kernels: 8 floats per token of each batch x head; the cluster kernel: 6 per token of each
+// (batch x head, block), 2 per token of each batch x head and 2 per (batch x head, block)
+size_t bwd_workspace_bytes(long long BH, int S, int nb) {
+  const size_t simt = (size_t)BH * 8 * (size_t)S;
+  const size_t cluster = (size_t)BH * ((size_t)nb * 6 * S + 2 * (size_t)S + 2 * (size_t)nb);
+  return (simt > cluster ? simt : cluster) * sizeof(float);
+}
 
 namespace {
 size_t bwd_chunk_smem_bytes(int dk, int dv, int L) {

@@ -123,7 +123,7 @@ struct BwdArgs {
   float* ws;  // bwd_workspace_bytes
 };
 size_t bwd_smem_bytes(int dk, int dv);
-size_t bwd_workspace_bytes(long long BH, int S);
+size_t bwd_workspace_bytes(long long BH, int S, int nb);
 bool bwd_supported(int dk, int dv, int dtype);
 cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream);
 

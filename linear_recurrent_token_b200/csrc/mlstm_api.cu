@@ -628,7 +628,7 @@ mlstm_status_t mlstm_fwd_chunkwise_scalar_normaliser(const mlstm_fwd_params_t* p
 size_t mlstm_bwd_workspace_size(const mlstm_fwd_params_t* p) {
   FwdShape s;
   if (check_bwd(p, &s) != MLSTM_OK) return 0;
-  return bwd_workspace_bytes(s.BH, s.S);
+  return bwd_workspace_bytes(s.BH, s.S, s.nb);
 }
 
 mlstm_status_t mlstm_bwd(const mlstm_fwd_params_t* p, const void* q, const void* k, const void* v,
@@ -668,7 +668,7 @@ mlstm_status_t mlstm_bwd(const mlstm_fwd_params_t* p, const void* q, const void*
                         {digate, BH * S * 4},      {dfgate, BH * S * 4},      {dogate, BH * S * s.DHV * 4},
                         {dC0, cbytes},             {dn0, nbytes},             {dm0, BH * 4}};
   const int nout = (int)(sizeof(outs) / sizeof(outs[0]));
-  const size_t need = bwd_workspace_bytes(s.BH, s.S);
+  const size_t need = bwd_workspace_bytes(s.BH, s.S, s.nb);
   const Range rws{work ? workspace : nullptr, need};
   for (int a = 0; a < nout; ++a) {
     for (const Range& i : ins)

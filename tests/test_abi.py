@@ -211,7 +211,12 @@ def test_bwd_null_align_alias_workspace():
     assert bwd_call(p, ws=0x9000000) == 7          # workspace on top of dq
     assert bwd_call(p, ws_bytes=16) == 5
     assert bwd_call(p, ws=None) == 5
-    assert mlstm.bwd_workspace_size(p) == 2 * 2 * 8 * 64 * 4
+    # per batch x head: max(8 S floats (SIMT kernels), 6 S nb + 2 S + 2 nb floats (cluster kernel))
+    assert mlstm.bwd_workspace_size(p) == 2 * 2 * max(8 * 64, 6 * 64 + 2 * 64 + 2) * 4
+    big = mlstm.fwd_params(1, 8, 8192, 256, 512, 64, 1, torch.bfloat16, False)
+    assert mlstm.bwd_workspace_size(big) == 8 * max(8 * 8192, 6 * 8192 + 2 * 8192 + 2) * 4
+    blocks = mlstm.fwd_params(4, 4, 512, 64, 64, 64, 2, torch.bfloat16, False)
+    assert mlstm.bwd_workspace_size(blocks) == 16 * (6 * 512 * 2 + 2 * 512 + 2 * 2) * 4
     assert mlstm.bwd_workspace_size(params(DHQK=512)) == 0
 
 

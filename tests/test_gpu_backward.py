@@ -131,6 +131,7 @@ def test_backward_retention_workload_sampled_heads():
     (17, 1, 2, 130, 64, 64, 4, False, True, False, True),      # 16 x 16
     (18, 1, 1, 200, 64, 256, 2, True, True, False, False),     # 32 x 128, retention
     (19, 2, 1, 100, 128, 64, 2, False, True, True, True),      # 64 x 32
+    (20, 1, 2, 0, 64, 128, 2, False, True, False, True),       # empty sequence: initial-state gradients
 ])
 def test_backward_cluster_kernel_parity(case):
     seed, B, NH, S, DHQK, DHV, nb, retention, with_state, with_o, with_dstate = case
