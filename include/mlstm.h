@@ -322,7 +322,8 @@ mlstm_status_t mlstm_fwd_chunkwise_scalar_normaliser(const mlstm_fwd_params_t* p
  *                                  initial state; NULL = not written; dn0 and dm0 not in
  *                                  retention mode
  *   workspace, workspace_bytes     at least mlstm_bwd_workspace_size(p) bytes, 16-byte
- *                                  aligned; contents need not be initialised
+ *                                  aligned; contents need not be initialised; required
+ *                                  whenever that size is nonzero (B*NH > 0, also for S = 0)
  * Outputs must not overlap the inputs, each other or the workspace (MLSTM_ERR_ALIAS).
  * Other conventions as for the forward.
  */

@@ -669,7 +669,7 @@ mlstm_status_t mlstm_bwd(const mlstm_fwd_params_t* p, const void* q, const void*
                         {dC0, cbytes},             {dn0, nbytes},             {dm0, BH * 4}};
   const int nout = (int)(sizeof(outs) / sizeof(outs[0]));
   const size_t need = bwd_workspace_bytes(s.BH, s.S, s.nb);
-  const Range rws{work ? workspace : nullptr, need};
+  const Range rws{need > 0 ? workspace : nullptr, need};
   for (int a = 0; a < nout; ++a) {
     for (const Range& i : ins)
       if (overlaps(outs[a], i)) return MLSTM_ERR_ALIAS;
@@ -677,7 +677,9 @@ mlstm_status_t mlstm_bwd(const mlstm_fwd_params_t* p, const void* q, const void*
       if (overlaps(outs[a], outs[b])) return MLSTM_ERR_ALIAS;
     if (overlaps(outs[a], rws)) return MLSTM_ERR_ALIAS;
   }
-  if (work && (!workspace || workspace_bytes < need)) return MLSTM_ERR_WORKSPACE;
+  // (an empty sequence still needs it: the cluster kernel keeps each block's final-state terms
+  // there for the gate-gradient kernel)
+  if (need > 0 && (!workspace || workspace_bytes < need)) return MLSTM_ERR_WORKSPACE;
   cudaStream_t cs = (cudaStream_t)stream;
   if (BH == 0) return MLSTM_OK;  // with S == 0 the kernel still forms the initial-state gradients
   BwdArgs a;

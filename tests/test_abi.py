@@ -217,6 +217,9 @@ def test_bwd_null_align_alias_workspace():
     assert mlstm.bwd_workspace_size(big) == 8 * max(8 * 8192, 6 * 8192 + 2 * 8192 + 2) * 4
     blocks = mlstm.fwd_params(4, 4, 512, 64, 64, 64, 2, torch.bfloat16, False)
     assert mlstm.bwd_workspace_size(blocks) == 16 * (6 * 512 * 2 + 2 * 512 + 2 * 2) * 4
+    # an empty sequence still needs the per-(batch x head, block) final-state terms
+    assert mlstm.bwd_workspace_size(params(S=0)) == 2 * 2 * 2 * 4
+    assert bwd_call(params(S=0), ws=None) == 5
     assert mlstm.bwd_workspace_size(params(DHQK=512)) == 0
 
 
