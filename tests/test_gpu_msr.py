@@ -136,3 +136,34 @@ def test_msr_decode_steps_match_the_block_prefill():
     y_dec = torch.cat(ys, dim=2)
     assert slice_relerr(host(y_dec), host(y_pre), 2) <= TOL["bf16"]
     assert slice_relerr(host(C), host(C_pre), 3) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("S,gate,affine,with_state", [
+    (1000, False, False, False),  # several segments, ragged last chunk, no gate, no affine
+    (64, True, True, True),       # one chunk
+    (2048, True, True, False),    # the retention-block workload's length
+])
+def test_msr_block_retention_heads_of_64(S, gate, affine, with_state):
+    """The block on 64 x 64 retention heads in bf16 (the tensor-core walk, then the GroupNorm +
+    gate pass), with and without the gate and the affine GroupNorm weights, across several
+    segments and a ragged last chunk; compared with the oracle's block on the same inputs."""
+    B, NH, D = 2, 4, 64
+    w = inputs.Workload(2, "msr_fused", B, NH, S, D, D, 64, 1, "bf16", True, 1 / np.sqrt(D))
+    p = mlstm.fwd_params(B, NH, S, D, D, 64, 1, torch.bfloat16, True)
+    assert mlstm.plan(p)["tensor_core"] == 1
+    inp = inputs.forward_inputs(w, seed=S + 5)
+    rng = np.random.default_rng(S)
+    td = torch.bfloat16
+    g = torch.from_numpy(rng.standard_normal((B, NH, S, D)).astype(np.float32)).to(td).float().numpy() if gate else None
+    gw = (1 + 0.3 * rng.standard_normal(NH * D)).astype(np.float32) if affine else None
+    gb = (0.2 * rng.standard_normal(NH * D)).astype(np.float32) if affine else None
+    C0 = (rng.standard_normal((B, NH, 1, D, D)) * 0.2).astype(np.float32) if with_state else None
+    pos0 = np.array([3, 1000], dtype=np.int64)
+    y, C, _, _ = mlstm.fwd_chunkwise_msr(dev(inp["q"], td), dev(inp["k"], td), dev(inp["v"], td), None, None,
+                                         dev(g, td) if gate else None, dev(gw), dev(gb), dev(C0), None, None,
+                                         pos0=torch.from_numpy(pos0).cuda(), eps=1e-5, retention=True)
+    torch.cuda.synchronize()
+    yr, Cr, _, _ = oracle.retention_block(inp["q"], inp["k"], inp["v"], None, None, g, gw, gb, C0, None, None,
+                                          pos0=pos0, eps=1e-5, retention=True, rounding=rounding_of("bf16"))
+    errs = {"y": slice_relerr(host(y), yr, 2), "C": slice_relerr(host(C), Cr, 3)}
+    assert all(e <= TOL["bf16"] for e in errs.values()), errs
