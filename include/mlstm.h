@@ -471,7 +471,8 @@ mlstm_status_t mlstm_step(const mlstm_step_params_t* p,
 /* Static, never-NULL description of a status code. */
 const char* mlstm_status_string(mlstm_status_t s);
 
-/* ABI version: (major << 16) | minor. */
+/* ABI version: (major << 16) | minor.  2.3: mlstm_bwd needs its workspace whenever
+ * mlstm_bwd_workspace_size is nonzero, an empty sequence included. */
 int mlstm_abi_version(void);
 
 #ifdef __cplusplus

@@ -317,7 +317,7 @@ mlstm_status_t check_bwd(const mlstm_fwd_params_t* p, FwdShape* s) {
 
 extern "C" {
 
-int mlstm_abi_version(void) { return (2 << 16) | 2; }
+int mlstm_abi_version(void) { return (2 << 16) | 3; }
 
 const char* mlstm_status_string(mlstm_status_t s) {
   switch (s) {
