@@ -61,12 +61,13 @@ struct Vec<__nv_bfloat16> {
 };
 
 constexpr int ROT_THREADS = 256;
-constexpr int ROT_HEADS = 4;  // heads whose vectors are loaded before any is stored
+constexpr int ROT_HEADS = 2;  // heads whose vectors are loaded before any is stored
 
 // grid (ceil(S / tokens per CTA), B); thread = (token, 16-byte vector of the head dimension)
 template <typename T>
-__global__ void __launch_bounds__(ROT_THREADS) theta_rotate_kernel(const T* q, const T* k, T* qo, T* ko, int NH,
-                                                                  int S, int D, const long long* pos0, float base) {
+// (four CTAs per SM: the 512 CTAs of the retention workload run in one wave)
+__global__ void __launch_bounds__(ROT_THREADS, 4)
+    theta_rotate_kernel(const T* q, const T* k, T* qo, T* ko, int NH, int S, int D, const long long* pos0, float base) {
   using V = Vec<T>;
   constexpr int PP = V::N / 2;  // pairs per vector
   const int cpr = D / V::N, tpc = ROT_THREADS / cpr;
