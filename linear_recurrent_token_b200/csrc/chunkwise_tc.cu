@@ -1694,9 +1694,12 @@ TcPlan tc_plan(int B, int NH, int S, int nb, int dk, int dv, int num_sms) {
     // chunk, ~1.05 us per summary chunk, ~1.5 us per summary composed into a start state, segment 0
     // starting ~6 us and phase A ~3 us after the call starts):
     //   end of segment 0     = 2.2 + s0
-    //   end of the others    = 1.1 + 0.39 * (longest unit) + 0.55 * (units composed) + s
+    //   end of the others    = 1.1 + a * (longest unit) + 0.55 * (units composed) + s
     // over s0 with s = ceil((chunks - s0) / (G - 1)), the two-unit split of segment 0 taken when
-    // its CTAs fit one wave.
+    // its CTAs fit one wave.  a, a summary chunk over a walk chunk, is 0.39 for 256-wide keys and
+    // larger for narrower ones, whose walk chunk is shorter (0.54 fits 64-wide heads: the best
+    // segment-0 length of 32 chunks in two segments measured 21, both modes); in between linear.
+    const double a_sum = 0.39 + 0.15 * (256 - (dk < 64 ? 64 : dk > 256 ? 256 : dk)) / 192.0;
     const long long slices_l = (long long)B * NH * nb;
     // split segment 0 in two summary units only when the summary CTAs (G units: 2 + (G - 2)) and
     // segment 0's walk CTAs run at the same time: together one wave
@@ -1709,7 +1712,7 @@ TcPlan tc_plan(int B, int NH, int S, int nb, int dk, int dv, int num_sms) {
       for (int ups = 1; ups <= (can_split ? 2 : 1); ++ups) {
         const int longest = (s0 + ups - 1) / ups > s ? (s0 + ups - 1) / ups : s;
         const int composed = ups + pl.G - 2;
-        const double others = 1.1 + 0.39 * longest + 0.55 * composed + s;
+        const double others = 1.1 + a_sum * longest + 0.55 * composed + s;
         const double first = 2.2 + s0;
         const double cost = others > first ? others : first;
         if (cost < best - 1e-9) {
