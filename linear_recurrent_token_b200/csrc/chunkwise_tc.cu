@@ -1678,6 +1678,9 @@ TcPlan tc_plan(int B, int NH, int S, int nb, int dk, int dv, int num_sms) {
   // at least 4 chunks per segment, segments no longer than 8192 tokens (phase A keeps one
   // fp32 exponent offset per chunk of its segment in shared memory)
   if (G > chunks / 4) G = chunks / 4 > 0 ? chunks / 4 : 1;
+  // up to 8 chunks one segment: the summaries' own launch and the composition cost more than
+  // they save (8 chunks of 64-wide heads, one segment against two: 0.024 -> 0.021-0.022 ms)
+  if (chunks <= 8) G = 1;
   while ((chunks + G - 1) / G * L > 8192) ++G;
   pl.seg_chunks = chunks > 0 ? (chunks + G - 1) / G : 1;
   pl.G = chunks > 0 ? (chunks + pl.seg_chunks - 1) / pl.seg_chunks : 1;
