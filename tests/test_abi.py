@@ -416,3 +416,19 @@ def test_tensor_core_plan_covers_the_sequence(shape):
     assert pl["ctas_main"] == B * NH * nb * tiles * G
     assert pl["ctas_main"] <= 148 or G == 1
     assert pl["workspace_bytes"] >= B * NH * nb * pl["summary_units"] * dv * dk * 4
+
+
+def test_planner_choices_on_the_measured_workloads():
+    """The plans the cost model gives the workloads it was measured on: the large head in four
+    segments of 32 chunks (three summary units); 64-wide retention heads of 32 chunks in two
+    segments with the longer first (21 + 11); sequences of at most 8 chunks in one segment (no
+    summaries kernel)."""
+    def plan(B, NH, S, DHQK, DHV, nb, ret):
+        return mlstm.plan(mlstm.fwd_params(B, NH, S, DHQK, DHV, 64, nb, torch.bfloat16, ret))
+    pl = plan(1, 8, 8192, 256, 512, 1, False)
+    assert (pl["segments"], pl["seg0_chunks"], pl["seg_chunks"], pl["summary_units"]) == (4, 32, 32, 3)
+    pl = plan(8, 8, 2048, 64, 64, 1, True)
+    assert (pl["segments"], pl["seg0_chunks"], pl["seg_chunks"], pl["summary_units"]) == (2, 21, 11, 1)
+    for shape in ((4, 4, 512, 64, 64, 2, False), (8, 8, 512, 64, 64, 1, True), (1, 2, 450, 128, 128, 1, False)):
+        pl = plan(*shape)
+        assert pl["segments"] == 1 and pl["summary_units"] == 0 and pl["kernels"] == 2, (shape, pl)
