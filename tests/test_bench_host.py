@@ -145,3 +145,17 @@ def test_gdn2_flop_count():
     # decay K V, read-out 2 K V, erase + write 4 K V, output 2 K V per token and head
     assert bench.gdn2_flops(1, 1, 1, 128, 128) == 9 * 128 * 128
     assert bench.gdn2_flops(8, 16, 2048, 128, 128) == 38_654_705_664
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    """Under a launcher with several ranks, `bench.py --impl reference` prints its line from rank
+    0 alone; any other rank exits 0 without work and prints nothing."""
+    import subprocess
+    import sys
+
+    from tests.conftest import ROOT
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip() == ""
